@@ -1,0 +1,269 @@
+/*
+ * kvq.h - C ABI of a quantized paged KV cache with fused-dequant decode attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Sources cited below (titles of the web pages that describe the method):
+ *   [P-vLLM] "KV Cache量化压缩技术与vLLM推理引擎显存优化实战" (yunthe.com)
+ *   [P-prod] "KV Cache Quantization 生产实战：用低精度缓存降低长上下文推理显存" (oh-bug.com)
+ *   [P-mem]  "大模型KV Cache显存优化与量化技术实践" (intelliparadigm.com)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument or descriptor field that names tensor data is a DEVICE
+ *    pointer, unless the comment says "host".  The caller owns all memory; the library
+ *    never allocates or frees device memory and never synchronises a stream, except
+ *    kvq_read_device_fault, which copies a few bytes back and waits for them.
+ *  - All work is enqueued on the given stream, in order; a NULL stream is the legacy
+ *    default stream.
+ *  - Device tensor pointers must be 16-byte aligned.  Tensors are dense, row-major,
+ *    with the shapes given below (outermost dimension first).
+ *  - Arguments are validated on the host before anything is launched: a bad argument
+ *    returns KVQ_ERR_INVALID_ARG, a well-formed request this build does not implement
+ *    returns KVQ_ERR_UNSUPPORTED, and in both cases nothing is enqueued.  A failed
+ *    launch returns KVQ_ERR_CUDA.
+ *  - Values the host cannot see (slot ids, block ids, context lengths, sequence ids
+ *    inside device arrays) are range-checked by the kernels.  An out-of-range entry is
+ *    skipped (its rows are not written / not read) and, when the descriptor carries a
+ *    fault record, counted there.  No kernel traps, asserts or spins without a bound.
+ *
+ * Cache layout ("L0", plain data owned by the caller)
+ * ---------------------------------------------------
+ *  NB = num_blocks, H = num_kv_heads, bs = block_size, D = head_dim.
+ *  A token slot is  slot = block_id * bs + offset,  0 <= offset < bs  ([P-vLLM]
+ *  "PagedAttention与KV Cache量化协同工作原理": fixed-size blocks of usually 16 tokens,
+ *  each managed on its own, holding INT8/FP8 data that attention dequantizes).
+ *
+ *  k_codes, v_codes : [NB][H][bs][D] elements of cache_dtype.  For INT4, two codes per
+ *                     byte: [NB][H][bs][D/2] bytes, element 2i in the low nibble of byte
+ *                     i, element 2i+1 in the high nibble.
+ *  k_scales, v_scales by scale_mode:
+ *    NONE            : unused (BF16 / FP16 caches).
+ *    PER_TOKEN_HEAD  : float32 [NB][H][bs] - one scale per written token and kv head,
+ *                      computed at write time ([P-mem] §3.2 动态量化策略).
+ *    PER_HEAD        : float32 [H]  - static scale per kv head, supplied by the caller
+ *                      ([P-prod] "vLLM：从 FP8 KV Cache 开始试点": per-attention-head).
+ *    PER_TENSOR      : float32 [1]  - static scale for the whole cache.
+ *    KIVI (INT4)     : k_scales = float16 [NB][H][2][D]: plane 0 the scale and plane 1
+ *                      the zero point of each channel over the block's 64 tokens;
+ *                      v_scales = float16 [NB][H][bs][D/64][2]: (scale, zero point) of
+ *                      each token's 64-channel group ([P-prod] "Key 和 Value 的分布不一定
+ *                      相同": keys per channel, values per token).
+ *  residual         : INT4 only.  act_dtype [max_seqs][2][H][residual_cap][D]: the
+ *                     newest tokens of each sequence kept unquantized ([P-prod] same
+ *                     section: a fixed-size higher-precision residual of recent K/V).
+ *                     Index 0 of the second dimension is K, 1 is V.  Position p of a
+ *                     sequence lives in ring row p % residual_cap.
+ *
+ * Quantizers (what kvq_write stores; x is one activation value widened to float32, and
+ * every "/" is an IEEE float32 division rounded to nearest-even)
+ *  INT8  ([P-mem] §3.1 对称量化算法; [P-vLLM] "KV Cache量化策略"):
+ *        dynamic: s = max_d |x_d| / 127  per (token, kv head), stored as float32;
+ *        static : s = the caller's per-head or per-tensor scale;
+ *        code   = clamp(round_half_even(x / s), -128, 127);  s == 0 gives code 0.
+ *        dequantized value = code * s.
+ *  FP8 E4M3 (OCP "E4M3FN": bias 7, no infinities, largest finite 448):
+ *        dynamic: s = max_d |x_d| / 448;  static: caller's scale.
+ *        code = x / s rounded to the nearest E4M3 value (ties to even), magnitudes
+ *        beyond 448 saturate to +-448;  s == 0 gives code 0x00.  value = decode(code)*s.
+ *  INT4 KIVI ([P-prod] "量化不是简单截断精度": X_q = round(X/scale) + zero_point,
+ *        X_deq = (X_q - zero_point) * scale), over a group G of 64 values (one channel
+ *        over the 64 tokens of a block for K, one token over 64 channels for V):
+ *        lo = min(min_G x, 0), hi = max(max_G x, 0);
+ *        s  = float16_rne( (hi - lo) / 15 )      (hi - lo is a float32 subtraction);
+ *        z  = clamp(round_half_even(-lo / s), 0, 15)        (float32 ops, s widened);
+ *        code = clamp(round_half_even(x / s) + z, 0, 15);   s == 0 gives z = code = 0.
+ *        Stored s and z are float16; dequantized value = (code - z) * s.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,   /* malformed argument; nothing was enqueued */
+  KVQ_ERR_UNSUPPORTED = 2,   /* well-formed but not implemented; nothing enqueued */
+  KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  KVQ_ERR_DEVICE_FAULT = 4   /* kvq_read_device_fault found skipped entries */
+} kvq_status;
+
+typedef enum {
+  KVQ_DTYPE_BF16 = 0,
+  KVQ_DTYPE_FP16 = 1,
+  KVQ_DTYPE_FP32 = 2,        /* output only */
+  KVQ_DTYPE_INT8 = 3,
+  KVQ_DTYPE_FP8_E4M3 = 4,
+  KVQ_DTYPE_INT4 = 5
+} kvq_dtype;
+
+typedef enum {
+  KVQ_SCALE_NONE = 0,
+  KVQ_SCALE_PER_TOKEN_HEAD = 1,
+  KVQ_SCALE_PER_HEAD = 2,
+  KVQ_SCALE_PER_TENSOR = 3,
+  KVQ_SCALE_KIVI = 4
+} kvq_scale_mode;
+
+/* Bits of fault[1] (fault[0] counts skipped entries). */
+enum {
+  KVQ_FAULT_SLOT = 1,        /* kvq_write: slot id outside [-1, NB*bs) */
+  KVQ_FAULT_BLOCK = 2,       /* block table entry outside [0, NB) */
+  KVQ_FAULT_CONTEXT = 4,     /* context length outside [0, max_context] or the table */
+  KVQ_FAULT_SEQ = 8,         /* sequence id outside [0, max_seqs) */
+  KVQ_FAULT_INT4_RUN = 16,   /* INT4 page rows not one whole, ordered block */
+  KVQ_FAULT_TIMEOUT = 32     /* a bounded wait inside a kernel ran out */
+};
+
+/*
+ * Cache descriptor.  Plain data: it owns nothing and may be copied freely.
+ *   cache_dtype   BF16 / FP16 (unquantized, element type must equal act_dtype),
+ *                 INT8, FP8_E4M3 or INT4.
+ *   act_dtype     BF16 or FP16: element type of new K/V rows, of q and of the INT4
+ *                 residual ring.
+ *   scale_mode    NONE for BF16/FP16; PER_TOKEN_HEAD, PER_HEAD or PER_TENSOR for INT8
+ *                 and FP8; KIVI for INT4.
+ *   block_size    tokens per block: 1..256 for dense caches; INT4 requires
+ *                 block_size == group_size == 64.
+ *   head_dim      64 or 128.
+ *   group_size, residual_len, residual_cap, max_seqs: INT4 only (64, r, cap, seqs);
+ *                 residual_cap >= residual_len + group_size.  Ignored otherwise.
+ *   fault         optional device int32[2] fault record (NULL: faults are skipped
+ *                 silently).  fault[0] += entries skipped; fault[1] |= KVQ_FAULT_* bits.
+ */
+typedef struct {
+  int32_t cache_dtype;
+  int32_t act_dtype;
+  int32_t scale_mode;
+  int32_t num_blocks;
+  int32_t block_size;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t group_size;
+  int32_t residual_len;
+  int32_t residual_cap;
+  int32_t max_seqs;
+  int32_t reserved0;
+  void* k_codes;
+  void* v_codes;
+  void* k_scales;
+  void* v_scales;
+  void* residual;
+  int32_t* fault;
+} kvq_cache_desc;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* kvq_status_string(kvq_status status);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int kvq_version(void);
+
+/*
+ * Byte sizes the caller must allocate for each pool of a cache described by `cache`
+ * (pointer fields are ignored).  Any out pointer may be NULL.  Host-only; never
+ * touches the device.  Sizes follow the layout above ([P-prod] "KV Cache 的基本内存
+ * 模型": 2 x layers x kv_heads x head_dim x tokens x bytes per value, per layer here,
+ * plus the scale, zero-point and residual bytes that make the real gain smaller).
+ */
+kvq_status kvq_cache_layout(const kvq_cache_desc* cache, size_t* code_bytes_per_pool,
+                            size_t* scale_bytes_per_pool, size_t* residual_bytes);
+
+/*
+ * kvq_write - quantize new K/V rows into the cache ("quantize on write").
+ *   k_new, v_new  act_dtype [num_tokens][H][D], device.
+ *   slot_mapping  int32 [num_tokens], device: destination slot of each row, or -1.
+ *   seq_ids, positions  int32 [num_tokens], device, INT4 only (NULL otherwise): a row
+ *                 with slot -1 and positions[t] >= 0 is copied unquantized into ring row
+ *                 positions[t] % residual_cap of sequence seq_ids[t].
+ *   Dense caches: row t goes to slot slot_mapping[t]; slot -1 skips the row.  K and V
+ *   are quantized separately, each per (token, kv head) for dynamic modes.
+ *   INT4 caches: rows are taken in groups of 64 (rows 64u .. 64u+63).  A group whose
+ *   first slot is >= 0 must map, in order, onto one whole block (slots b*64 .. b*64+63);
+ *   it is quantized as one key group per channel and 64 value groups per channel group.
+ *   A group whose first slot is -1 holds ring rows or skipped rows only.  A trailing
+ *   partial group may hold ring rows only.
+ *   Duplicate destination slots inside one call give an undefined winner.
+ *   Quantizer definitions: see the header comment ([P-mem] §3.1 / §3.2, [P-vLLM]
+ *   "KV Cache量化策略", [P-prod] "量化不是简单截断精度").
+ */
+kvq_status kvq_write(const kvq_cache_desc* cache, const void* k_new, const void* v_new,
+                     int num_tokens, const int32_t* slot_mapping, const int32_t* seq_ids,
+                     const int32_t* positions, cudaStream_t stream);
+
+/*
+ * Workspace bytes kvq_decode_attention needs for this shape (host-only).  The split
+ * plan depends only on (cache geometry, batch, num_q_heads, max_context), so the same
+ * arguments always give the same size.  *bytes may be 0 (no split needed).
+ */
+kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
+                                     int num_q_heads, int max_context, size_t* bytes);
+
+/*
+ * kvq_decode_attention - one query token per sequence attends to its cached context.
+ *   q             act_dtype [batch][num_q_heads][D], device.  num_q_heads must be a
+ *                 multiple of H; query head hq reads kv head hq / (num_q_heads / H).
+ *   block_tables  int32 [batch][max_blocks_per_seq], device: block ids of each sequence
+ *                 in token order; entries past ceil(len/bs) are not read.
+ *   context_lens  int32 [batch], device: tokens to attend to (the current token
+ *                 included); 0 gives an all-zero output row.
+ *   seq_ids       INT4 only, int32 [batch] device or NULL: ring sequence of each batch
+ *                 entry (NULL: entry b uses ring sequence b).
+ *   max_context   host upper bound of context_lens, used to plan the split.
+ *   softmax_scale 0 selects 1/sqrt(D) ([P-mem] §6 Q1 writes softmax(q k^T / sqrt(d))).
+ *   out           out_dtype [batch][num_q_heads][D], device; out_dtype BF16, FP16 or FP32.
+ *   workspace     device scratch of at least kvq_decode_workspace_size() bytes (may be
+ *                 NULL when that size is 0).  Its contents need no initialisation.
+ *   For each (b, hq): o = sum_p softmax_p(scale * q . k_p) v_p over p < context_lens[b],
+ *   where k_p, v_p are the dequantized cache rows; for INT4, positions p < Qb come from
+ *   blocks and the rest from the residual ring, Qb = 64*floor(max(len-residual_len,0)/64).
+ *   Dequantization happens inside the kernel ([P-vLLM] "PagedAttention与KV Cache量化协同
+ *   工作原理"); long contexts are split across CTAs and merged by a log-sum-exp reduce.
+ */
+kvq_status kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int batch,
+                                int num_q_heads, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                const int32_t* seq_ids, int max_context, float softmax_scale,
+                                void* out, int32_t out_dtype, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * kvq_dequant - debug: expand whole blocks back to float32.
+ *   block_ids  int32 [n_blocks], device.
+ *   out        float32 [n_blocks][2][H][bs][D], device; index 0 of dim 1 is K, 1 is V.
+ *   Each value is the dequantized value defined in the header comment.  An out-of-range
+ *   block id leaves its output rows untouched (and is counted in the fault record).
+ */
+kvq_status kvq_dequant(const kvq_cache_desc* cache, const int32_t* block_ids, int n_blocks,
+                       float* out, cudaStream_t stream);
+
+/*
+ * kvq_calibrate_fp8_scales - set-up step: per-kv-head scale from warm-up rows,
+ *   scale_out[h] = (max over tokens and channels of |x[t][h][:]|) / 448, float32 division.
+ *   x          act_dtype [n_tokens][num_kv_heads][head_dim], device.
+ *   scale_out  float32 [num_kv_heads], device.  An all-zero head gives 0.
+ *   ([P-prod] "vLLM：从 FP8 KV Cache 开始试点": scales from a random-token warm-up.)
+ */
+kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_heads,
+                                    int head_dim, int32_t act_dtype, float* scale_out,
+                                    cudaStream_t stream);
+
+/*
+ * kvq_read_device_fault - copy the descriptor's fault record into host `out[2]`
+ *   (count, KVQ_FAULT_* bits), waiting for `stream` first.  If `reset` is non-zero the
+ *   record is cleared afterwards (enqueued on `stream`).  Returns KVQ_ERR_DEVICE_FAULT
+ *   when the count is non-zero, KVQ_OK otherwise, KVQ_ERR_INVALID_ARG if the
+ *   descriptor has no fault record.
+ */
+kvq_status kvq_read_device_fault(const kvq_cache_desc* cache, int32_t* out, int reset,
+                                 cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

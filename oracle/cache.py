@@ -1,0 +1,221 @@
+"""Byte-exact model of the paged, quantized KV cache: scatter on write, gather on read.
+
+TEST INFRASTRUCTURE (oracle): see the package docstring.
+
+The pools are NumPy arrays with exactly the layout written in include/kvq.h, filled
+with a sentinel byte (0x5A) so that a test can check that a write touched only its own
+slots.  A slot is block_id * block_size + offset; each block is managed on its own
+([P-vLLM] "PagedAttention与KV Cache量化协同工作原理": fixed-size blocks, usually of 16
+tokens, stored as INT8/FP8 and dequantized when attention reads them).
+"""
+
+import numpy as np
+
+from . import fp, quant
+
+SENTINEL = 0x5A
+
+DENSE_DTYPES = ("bf16", "fp16", "int8", "fp8")
+
+
+def _bits_of_act(x, act):
+    """Bit patterns (uint16) of activation values given as float64 (exact)."""
+    if act == "bf16":
+        return fp.bf16_bits(np.asarray(x, np.float64).astype(np.float32))
+    if act == "fp16":
+        v = np.asarray(x, np.float64)
+        h = v.astype(np.float16)
+        if not np.array_equal(h.astype(np.float64), v):
+            raise ValueError("value not representable in float16")
+        return h.view(np.uint16)
+    raise ValueError(act)
+
+
+def _value_of_act_bits(bits, act):
+    if act == "bf16":
+        return fp.bf16_value(bits)
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float64)
+
+
+class PagedCache:
+    """One layer's K and V pools.
+
+    cache_dtype: "bf16" | "fp16" | "int8" | "fp8" | "int4"
+    act_dtype:   "bf16" | "fp16"
+    scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "kivi"
+    static_scales: (k_scale, v_scale) float32 arrays [H] or [1] for static modes.
+    """
+
+    def __init__(self, cache_dtype, act_dtype, scale_mode, num_blocks, block_size,
+                 num_kv_heads, head_dim, group_size=64, residual_len=128,
+                 residual_cap=192, max_seqs=0, static_scales=None):
+        self.cd, self.act, self.mode = cache_dtype, act_dtype, scale_mode
+        self.NB, self.bs, self.H, self.D = num_blocks, block_size, num_kv_heads, head_dim
+        self.G, self.R, self.cap, self.max_seqs = group_size, residual_len, residual_cap, max_seqs
+        NB, bs, H, D = self.NB, self.bs, self.H, self.D
+        if cache_dtype in ("bf16", "fp16"):
+            assert scale_mode == "none" and cache_dtype == act_dtype
+            code_dt, code_D = np.uint16, D
+        elif cache_dtype == "int8":
+            code_dt, code_D = np.int8, D
+        elif cache_dtype == "fp8":
+            code_dt, code_D = np.uint8, D
+        elif cache_dtype == "int4":
+            assert scale_mode == "kivi" and block_size == group_size == 64
+            code_dt, code_D = np.uint8, D // 2
+        else:
+            raise ValueError(cache_dtype)
+        self.k_codes = self._sentinel((NB, H, bs, code_D), code_dt)
+        self.v_codes = self._sentinel((NB, H, bs, code_D), code_dt)
+        self.k_scales = self.v_scales = None
+        self.residual = None
+        if scale_mode == "per_token_head":
+            self.k_scales = self._sentinel((NB, H, bs), np.float32)
+            self.v_scales = self._sentinel((NB, H, bs), np.float32)
+        elif scale_mode in ("per_head", "per_tensor"):
+            n = H if scale_mode == "per_head" else 1
+            ks, vs = static_scales
+            self.k_scales = np.asarray(ks, np.float32).reshape(n).copy()
+            self.v_scales = np.asarray(vs, np.float32).reshape(n).copy()
+        elif scale_mode == "kivi":
+            self.k_scales = self._sentinel((NB, H, 2, D), np.float16)
+            self.v_scales = self._sentinel((NB, H, bs, D // group_size, 2), np.float16)
+            self.residual = self._sentinel((max_seqs, 2, H, residual_cap, D), np.uint16)
+
+    @staticmethod
+    def _sentinel(shape, dtype):
+        n = int(np.prod(shape)) * np.dtype(dtype).itemsize
+        return np.full(n, SENTINEL, np.uint8).view(dtype).reshape(shape)
+
+    # ------------------------------------------------------------------ scales
+    def _static_scale(self, which):
+        s = self.k_scales if which == 0 else self.v_scales
+        if self.mode == "per_head":
+            return s                                  # [H]
+        return np.broadcast_to(s, (self.H,))          # per tensor
+
+    # ------------------------------------------------------------------ write
+    def write(self, k_new, v_new, slot_mapping, seq_ids=None, positions=None):
+        """Quantize rows k_new/v_new [T, H, D] (float64 values of act_dtype) into slots.
+
+        Same contract as kvq_write in include/kvq.h.  Out-of-range slots are skipped.
+        """
+        k_new = np.asarray(k_new, np.float64)
+        v_new = np.asarray(v_new, np.float64)
+        slots = np.asarray(slot_mapping, np.int64)
+        if self.cd == "int4":
+            return self._write_int4(k_new, v_new, slots, seq_ids, positions)
+        NB, bs = self.NB, self.bs
+        for t in range(slots.shape[0]):
+            slot = int(slots[t])
+            if slot < 0 or slot >= NB * bs:
+                continue
+            blk, off = divmod(slot, bs)
+            for which, rows in ((0, k_new[t]), (1, v_new[t])):
+                codes = self.k_codes if which == 0 else self.v_codes
+                x = rows.astype(np.float32)            # [H, D], exact
+                if self.cd in ("bf16", "fp16"):
+                    codes[blk, :, off, :] = _bits_of_act(rows, self.act)
+                    continue
+                if self.mode == "per_token_head":
+                    s = (quant.int8_scale_dynamic(x) if self.cd == "int8"
+                         else quant.fp8_scale_dynamic(x))          # [H]
+                    sc = self.k_scales if which == 0 else self.v_scales
+                    sc[blk, :, off] = s
+                else:
+                    s = self._static_scale(which)
+                s2 = np.asarray(s, np.float32)[:, None]
+                if self.cd == "int8":
+                    codes[blk, :, off, :] = quant.int8_quantize(x, s2)
+                else:
+                    codes[blk, :, off, :] = quant.fp8_quantize(x, s2)
+
+    def _write_int4(self, k_new, v_new, slots, seq_ids, positions):
+        T = slots.shape[0]
+        G, bs = self.G, self.bs
+        for u in range(0, T, G):
+            rows = range(u, min(u + G, T))
+            first = int(slots[u])
+            if first >= 0:
+                # one whole block, in order
+                if len(rows) != G or first % bs != 0 or first >= self.NB * bs:
+                    continue
+                if not all(int(slots[u + i]) == first + i for i in range(G)):
+                    continue
+                blk = first // bs
+                for h in range(self.H):
+                    kc, ks, kz = quant.int4_keys_block(k_new[u:u + G, h, :].astype(np.float32))
+                    self.k_codes[blk, h] = quant.pack_nibbles(kc)
+                    self.k_scales[blk, h, 0, :] = ks
+                    self.k_scales[blk, h, 1, :] = kz
+                    for i in range(G):
+                        vc, vs, vz = quant.int4_values_row(v_new[u + i, h, :], self.G)
+                        self.v_codes[blk, h, i] = quant.pack_nibbles(vc)
+                        self.v_scales[blk, h, i, :, 0] = vs
+                        self.v_scales[blk, h, i, :, 1] = vz
+            else:
+                for t in rows:
+                    if int(slots[t]) != -1 or positions is None or int(positions[t]) < 0:
+                        continue
+                    sid = int(seq_ids[t])
+                    if sid < 0 or sid >= self.max_seqs:
+                        continue
+                    row = int(positions[t]) % self.cap
+                    self.residual[sid, 0, :, row, :] = _bits_of_act(k_new[t], self.act)
+                    self.residual[sid, 1, :, row, :] = _bits_of_act(v_new[t], self.act)
+
+    # ------------------------------------------------------------------ read
+    def dequant_block(self, blk):
+        """float64 [2, H, bs, D] of one block (index 0 = K, 1 = V)."""
+        out = np.empty((2, self.H, self.bs, self.D), np.float64)
+        for which in (0, 1):
+            codes = self.k_codes if which == 0 else self.v_codes
+            c = codes[blk]
+            if self.cd in ("bf16", "fp16"):
+                out[which] = _value_of_act_bits(c, self.act)
+            elif self.cd == "int8":
+                s = (self.k_scales if which == 0 else self.v_scales)
+                s = s[blk] if self.mode == "per_token_head" else \
+                    np.broadcast_to(self._static_scale(which)[:, None], (self.H, self.bs))
+                out[which] = quant.int8_dequantize(c, s)
+            elif self.cd == "fp8":
+                s = (self.k_scales if which == 0 else self.v_scales)
+                s = s[blk] if self.mode == "per_token_head" else \
+                    np.broadcast_to(self._static_scale(which)[:, None], (self.H, self.bs))
+                out[which] = quant.fp8_dequantize(c, s)
+            else:
+                q = quant.unpack_nibbles(c)                      # [H, bs, D]
+                if which == 0:
+                    s = self.k_scales[blk, :, 0, :].astype(np.float64)   # [H, D]
+                    z = self.k_scales[blk, :, 1, :].astype(np.float64)
+                    out[0] = (q.astype(np.float64) - z[:, None, :]) * s[:, None, :]
+                else:
+                    vs = self.v_scales[blk].astype(np.float64)   # [H, bs, D/G, 2]
+                    s = np.repeat(vs[..., 0], self.G, axis=-1)   # [H, bs, D]
+                    z = np.repeat(vs[..., 1], self.G, axis=-1)
+                    out[1] = (q.astype(np.float64) - z) * s
+        return out
+
+    def quantized_prefix(self, n):
+        """INT4: number of leading positions read from blocks; the rest is in the ring."""
+        if self.cd != "int4":
+            return n
+        return self.G * (max(n - self.R, 0) // self.G)
+
+    def gather(self, block_table_row, n, seq_id=None):
+        """Dequantized K and V of one sequence: two float64 arrays [H, n, D]."""
+        K = np.empty((self.H, n, self.D), np.float64)
+        V = np.empty((self.H, n, self.D), np.float64)
+        qb = self.quantized_prefix(n)
+        nblk = (qb + self.bs - 1) // self.bs
+        for i in range(nblk):
+            blk = int(block_table_row[i])
+            d = self.dequant_block(blk)
+            lo, hi = i * self.bs, min((i + 1) * self.bs, qb)
+            K[:, lo:hi] = d[0, :, :hi - lo]
+            V[:, lo:hi] = d[1, :, :hi - lo]
+        for p in range(qb, n):
+            row = p % self.cap
+            K[:, p] = _value_of_act_bits(self.residual[seq_id, 0, :, row, :], self.act)
+            V[:, p] = _value_of_act_bits(self.residual[seq_id, 1, :, row, :], self.act)
+        return K, V

@@ -1,0 +1,181 @@
+"""Quantizers and dequantizers, one group at a time, in the pages' steps.
+
+TEST INFRASTRUCTURE (oracle): see the package docstring.
+
+Inputs are activation values (bfloat16 or float16 values, exactly representable in
+binary32) given as NumPy arrays; outputs are codes and scales with the bit patterns the
+cache stores.
+
+Readings of the pages taken here (each listed in the design doc):
+  * "round" is round-half-to-even: the INT8 snippet of [P-mem] §3.1 对称量化算法 uses
+    torch.round, which rounds half to even.
+  * x / scale and the scale itself are IEEE binary32: the snippet returns the scale as
+    ``.float()``; a fp32 scale per token per head is the dynamic variant of [P-mem]
+    §3.2 动态量化策略.
+  * An all-zero group (max |x| = 0) has scale 0 and codes 0, with no division.
+  * INT4 uses the affine form of [P-prod] "量化不是简单截断精度"
+    (X_q = round(X/scale) + zero_point; X_deq = (X_q - zero_point) * scale) with the
+    range widened to include 0, so the zero point is an integer in [0, 15].
+"""
+
+import numpy as np
+
+from . import fp
+
+INT8_QMAX = 127.0
+FP8_QMAX = fp.E4M3_MAX
+INT4_LEVELS = 15.0
+
+
+# ----------------------------------------------------------------------------- INT8
+def int8_scale_dynamic(rows):
+    """Per-row symmetric MinMax scale s = max|x| / 127 (binary32), rows [..., D].
+
+    [P-mem] §3.1 对称量化算法 (scale = max(abs(x)) / 127) applied per token per kv head
+    ([P-mem] §3.2 动态量化策略: a scale for each token's K/V vector).
+    """
+    rows = np.asarray(rows, dtype=np.float32)
+    m = np.max(np.abs(rows), axis=-1)
+    return fp.div32(m, np.float32(INT8_QMAX))
+
+
+def int8_quantize(rows, scale):
+    """q = clamp(round_half_even(x / s), -128, 127) with x / s in binary32.
+
+    [P-mem] §3.1 对称量化算法 (torch.clamp(torch.round(x / scale), -128, 127));
+    [P-vLLM] "KV Cache量化策略" gives the same q = round(x / scale).  ``scale`` broadcasts
+    against rows[..., D] over the last axis; a zero scale gives code 0.
+    """
+    rows = np.asarray(rows, dtype=np.float32)
+    s = np.asarray(scale, dtype=np.float32)[..., None] if np.ndim(scale) == rows.ndim - 1 \
+        else np.asarray(scale, dtype=np.float32)
+    r = fp.div32(rows, s)
+    q = np.clip(fp.round_half_even(r), -128, 127)
+    q = np.where(s == 0, 0, q)
+    return q.astype(np.int8)
+
+
+def int8_dequantize(codes, scale):
+    """x_hat = q * s ([P-mem] §3.1: q_x.float() * scale), evaluated in float64."""
+    s = np.asarray(scale, dtype=np.float64)
+    codes = np.asarray(codes)
+    if s.ndim == codes.ndim - 1:
+        s = s[..., None]
+    return codes.astype(np.float64) * s
+
+
+# ----------------------------------------------------------------------------- FP8
+def fp8_scale_dynamic(rows):
+    """Per-row scale s = max|x| / 448 (binary32)."""
+    rows = np.asarray(rows, dtype=np.float32)
+    return fp.div32(np.max(np.abs(rows), axis=-1), np.float32(FP8_QMAX))
+
+
+def fp8_calibrate(warmup):
+    """Per-kv-head scale from warm-up rows [T, H, D]: max over tokens and channels / 448.
+
+    [P-prod] "vLLM：从 FP8 KV Cache 开始试点": per-attention-head FP8 scales may come from a
+    random-token warm-up.  448 is the largest finite E4M3 magnitude.
+    """
+    w = np.asarray(warmup, dtype=np.float32)
+    m = np.max(np.abs(w), axis=(0, 2))
+    return fp.div32(m, np.float32(FP8_QMAX))
+
+
+def fp8_quantize(rows, scale):
+    """code = E4M3(x / s): binary32 quotient, nearest E4M3 (ties even), saturate at 448.
+
+    [P-vLLM] "KV Cache量化策略" (FP8 E4M3 storage with a scale); a zero scale gives 0x00.
+    """
+    rows = np.asarray(rows, dtype=np.float32)
+    s = np.asarray(scale, dtype=np.float32)
+    if s.ndim == rows.ndim - 1:
+        s = s[..., None]
+    r = fp.div32(rows, s)
+    r = np.where(s == 0, np.float32(0.0), r)
+    codes = fp.e4m3_encode(r)
+    return np.where(np.broadcast_to(s == 0, codes.shape), np.uint8(0), codes).astype(np.uint8)
+
+
+def fp8_dequantize(codes, scale):
+    s = np.asarray(scale, dtype=np.float64)
+    codes = np.asarray(codes)
+    if s.ndim == codes.ndim - 1:
+        s = s[..., None]
+    return fp.e4m3_decode(codes) * s
+
+
+# ----------------------------------------------------------------------------- INT4
+def int4_quantize_group(values):
+    """Asymmetric 4-bit quantization of one group (1-D array of binary32 values).
+
+    Returns (codes uint8 in 0..15, scale float16, zero point float16).
+      lo = min(min x, 0); hi = max(max x, 0)
+      s  = float16(binary32((hi - lo) / 15))       -- stored, and used from here on
+      z  = clamp(round_half_even(-lo / s), 0, 15)
+      q  = clamp(round_half_even(x / s) + z, 0, 15)
+    [P-prod] "量化不是简单截断精度": X_q = round(X/scale) + zero_point.
+    """
+    x = np.asarray(values, dtype=np.float32).reshape(-1)
+    lo = np.minimum(x.min(), np.float32(0.0))
+    hi = np.maximum(x.max(), np.float32(0.0))
+    s32 = fp.div32(fp.sub32(hi, lo), np.float32(INT4_LEVELS))
+    s16 = fp.f16(s32)
+    if s16 == 0:
+        return np.zeros(x.shape, np.uint8), np.float16(0.0), np.float16(0.0)
+    sw = np.float32(s16)
+    z = np.clip(fp.round_half_even(fp.div32(-lo, sw)), 0, 15)
+    q = np.clip(fp.round_half_even(fp.div32(x, sw)) + z, 0, 15)
+    return q.astype(np.uint8), s16, np.float16(z)
+
+
+def int4_dequantize(codes, scale, zero):
+    """X_deq = (X_q - zero_point) * scale ([P-prod] "量化不是简单截断精度"), float64."""
+    return (np.asarray(codes, np.float64) - np.float64(zero)) * np.float64(scale)
+
+
+def int4_keys_block(k_rows):
+    """KIVI keys: one group per channel over the block's tokens.
+
+    k_rows [64, D] (one kv head).  Returns codes [64, D], scale [D], zero [D].
+    [P-prod] "Key 和 Value 的分布不一定相同": key cache per channel (KIVI).
+    """
+    k_rows = np.asarray(k_rows, dtype=np.float32)
+    T, D = k_rows.shape
+    codes = np.empty((T, D), np.uint8)
+    s = np.empty(D, np.float16)
+    z = np.empty(D, np.float16)
+    for d in range(D):
+        codes[:, d], s[d], z[d] = int4_quantize_group(k_rows[:, d])
+    return codes, s, z
+
+
+def int4_values_row(v_row, group=64):
+    """KIVI values: one group per token over each run of `group` channels.
+
+    v_row [D] (one token, one kv head).  Returns codes [D], scale [D/group], zero [D/group].
+    [P-prod] "Key 和 Value 的分布不一定相同": value cache per token.
+    """
+    v_row = np.asarray(v_row, dtype=np.float32)
+    D = v_row.shape[0]
+    codes = np.empty(D, np.uint8)
+    s = np.empty(D // group, np.float16)
+    z = np.empty(D // group, np.float16)
+    for gi in range(D // group):
+        sl = slice(gi * group, (gi + 1) * group)
+        codes[sl], s[gi], z[gi] = int4_quantize_group(v_row[sl])
+    return codes, s, z
+
+
+def pack_nibbles(codes):
+    """Two 4-bit codes per byte along the last axis: element 2i low, 2i+1 high."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+def unpack_nibbles(packed):
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
