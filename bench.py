@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized paged KV-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5] [--impl ours|reference]
+
+A step is one serving step of one layer: kvq_write of the batch's new K/V rows into the
+quantized paged cache, then kvq_decode_attention over every cached position (split-K
+kernel + reduce).  The cache of the previous positions is resident in HBM; the timed
+step is bracketed by CUDA events on the launching stream, with a 512 MiB memset before
+every step so no cache byte is served from L2.  Metric: KV GB/s = algorithmic bytes of
+the step / step time; tokens/s = batch / step time.  One JSON line on stdout.
+
+--impl reference times the float64 CPU oracle (the only other implementation of the
+method) on a bounded sample of the same workload; under torchrun only rank 0 runs it.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized paged decode attention: KV GB/s and % of HBM roofline; tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {
+    "c5": "Llama-3-70B-shaped layer: batch 24, 64 q heads / 8 kv heads, head_dim 128, "
+          "context 16384, block 16, INT8 per-token-head scales",
+    "c5-fp8": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
+              "block 16, FP8 E4M3 per-kv-head scales (256-token warm-up)",
+    "c5-bf16": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
+               "block 16, unquantized bf16 cache",
+    "c2": "Llama-2-7B-shaped layer: batch 4, 32 heads MHA, head_dim 128, context 2048, block 16, "
+          "INT8 per-token-head, 4 outlier channels x10 in K and V",
+    "c3": "Llama-3-8B-shaped layer: batch 64, 32/8 heads, head_dim 128, context U[1024, 8192], "
+          "block 16, FP8 E4M3 per-kv-head scales",
+    "c4": "70B-shaped KIVI INT4 layer: batch 16, 64/8 heads, head_dim 128, context 32768, "
+          "block 64, keys per channel / values per token, 128-token bf16 residual",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c5", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------- peaks
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(workload):
+    """dram bytes per launch of the decode kernel from the committed ncu summary, or None
+    when the summary is missing or was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_%s.md" % workload.replace("-", "_"))
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_launch:\s*(\d+)", text)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_source_hash():
+        return None
+    return int(m.group(1))
+
+
+def kernel_source_hash():
+    d = os.path.join(ROOT, "quantized_paged_kv_02_b200", "csrc")
+    hsh = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.startswith("kvq_decode"):
+            with open(os.path.join(d, name), "rb") as f:
+                hsh.update(f.read())
+    return hsh.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or (self.uuid and self.uuid not in f[0]):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_unit_step(w, unit_rows, b, kvh, static):
+    """Set up an oracle cache for one (sequence, kv head) and return a callable that
+    performs the step's work for it: quantize the new row, then attention of its query
+    heads over every cached position.  float64 CPU oracle, single process."""
+    import numpy as np
+    import torch
+    from oracle import attention, cache
+    from quantized_paged_kv_02_b200 import inputs
+    s = w.spec
+    n = int(w.context_lens[b])
+    r0 = int(w.seq_start[b])
+    k = unit_rows["k"][b].astype(np.float64)[:, None, :]      # [n, 1, D]
+    v = unit_rows["v"][b].astype(np.float64)[:, None, :]
+    st = None
+    if static is not None:
+        st = (static[0][kvh:kvh + 1], static[1][kvh:kvh + 1])
+    bs = s.block_size
+    if s.cache_dtype == "int4":
+        qb = 64 * (max(n - 128, 0) // 64)
+        nblk = qb // 64
+    else:
+        qb, nblk = n, -(-n // bs)
+    mode = "per_head" if s.scale_mode in ("per_head", "per_tensor") else s.scale_mode
+    oc = cache.PagedCache(s.cache_dtype, s.act_dtype, mode, max(nblk, 1), bs, 1, s.head_dim,
+                          residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
+                          max_seqs=1, static_scales=st)
+    table = np.arange(max(nblk, 1))
+    slots = np.array([p if p < qb else -1 for p in range(n)])
+    pos = np.array([-1 if p < qb else p for p in range(n)])
+    oc.write(k[:n - 1], v[:n - 1], slots[:n - 1], np.zeros(n - 1, np.int64), pos[:n - 1])
+    g = s.num_q_heads // s.num_kv_heads
+    q = unit_rows["q"][b][kvh * g:(kvh + 1) * g].astype(np.float64)[None]
+    del r0, torch
+
+    def step():
+        oc.write(k[n - 1:n], v[n - 1:n], slots[n - 1:n], np.zeros(1, np.int64), pos[n - 1:n])
+        return attention.decode_attention(oc, q, table[None, :], np.array([n]), seq_ids=np.array([0]))
+    return step
+
+
+def oracle_inputs(w, units):
+    """Host copies of the rows the sampled units need (read from the seeded workload)."""
+    import numpy as np
+    import torch
+    rows = {"k": {}, "v": {}, "q": {}}
+    for b, kvh in units:
+        r0, r1 = int(w.seq_start[b]), int(w.seq_start[b + 1])
+        rows["k"][b] = w.k[r0:r1, kvh].to(torch.float32).cpu().numpy()
+        rows["v"][b] = w.v[r0:r1, kvh].to(torch.float32).cpu().numpy()
+        rows["q"][b] = w.q[b].to(torch.float32).cpu().numpy()
+    del np
+    return rows
+
+
+def unit_bytes(w, b):
+    from quantized_paged_kv_02_b200 import roofline
+    s = w.spec
+    g = s.num_q_heads // s.num_kv_heads
+    return (roofline.decode_bytes(s.cache_dtype, s.scale_mode, g, 1, s.head_dim, s.block_size,
+                                  [int(w.context_lens[b])])
+            + roofline.write_bytes(s.cache_dtype, s.scale_mode, 1, 1, s.head_dim,
+                                   to_ring=s.cache_dtype == "int4"))
+
+
+def unit_workload(name):
+    """One (sequence, kv head) unit of the named workload, on the CPU: batch 1, one kv
+    head with its whole GQA group, the workload's context length (mean of the range for
+    variable lengths).  Same distributions and layout as the full workload."""
+    import dataclasses
+    from quantized_paged_kv_02_b200 import inputs
+    full = inputs._spec(name, False)
+    g = full.num_q_heads // full.num_kv_heads
+    n = full.lens[0] if full.lens else (full.len_range[0] + full.len_range[1]) // 2
+    spec = dataclasses.replace(full, name=full.name + "-unit", batch=1, num_kv_heads=1,
+                               num_q_heads=g, lens=[n], len_range=None, slack_blocks=0)
+    return inputs.from_spec(spec, "cpu")
+
+
+def run_oracle_sample(w, static, budget_s=15.0, max_units=64):
+    """Time the oracle on (b, kvh) units in order; stop once about budget_s seconds of
+    wall time (set-up of each unit's cache included) have passed.  Only the steps count
+    toward the reported rate."""
+    from threadpoolctl import threadpool_limits
+    units = [(b, h) for b in range(w.spec.batch) for h in range(w.spec.num_kv_heads)]
+    done, nbytes, t_total = 0, 0, 0.0
+    t_start = time.perf_counter()
+    with threadpool_limits(limits=1):
+        for b, kvh in units[:max_units]:
+            if done and time.perf_counter() - t_start >= budget_s:
+                break
+            rows = oracle_inputs(w, [(b, kvh)])
+            step = oracle_unit_step(w, rows, b, kvh, static)
+            t0 = time.perf_counter()
+            step()
+            t_total += time.perf_counter() - t0
+            nbytes += unit_bytes(w, b)
+            done += 1
+    return {"units": done, "bytes": nbytes, "seconds": t_total}
+
+
+# ----------------------------------------------------------------------------- ours
+def build_state(workload, device, seed):
+    import torch
+    from quantized_paged_kv_02_b200 import inputs, kvq
+    w = inputs.make(workload, device=device, seed=seed)
+    s = w.spec
+    static = None
+    sk = sv = None
+    if s.scale_mode in ("per_head", "per_tensor"):
+        sk = torch.empty(s.num_kv_heads, dtype=torch.float32, device=device)
+        sv = torch.empty(s.num_kv_heads, dtype=torch.float32, device=device)
+        kvq.kvq_calibrate_fp8_scales(w.warmup_k, sk)
+        kvq.kvq_calibrate_fp8_scales(w.warmup_v, sv)
+        static = (sk.cpu().numpy(), sv.cpu().numpy())
+    c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
+                         s.num_kv_heads, s.head_dim, device=device,
+                         residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
+                         max_seqs=s.batch, static_k_scale=sk, static_v_scale=sv)
+    if s.cache_dtype == "int4":
+        idx, slots, sid, pos = inputs.int4_group_rows(w)
+        idx = idx.to(device)
+        c.write(w.k[idx].contiguous(), w.v[idx].contiguous(), slots.to(device), sid.to(device),
+                pos.to(device))
+    else:
+        c.write(w.k, w.v, w.slot_mapping)
+    # the step's new token: the last position of every sequence
+    last = (w.seq_start[1:] - 1).to(device)
+    new = {"k": w.k[last].contiguous(), "v": w.v[last].contiguous()}
+    if s.cache_dtype == "int4":
+        new["slots"] = torch.full((s.batch,), -1, dtype=torch.int32, device=device)
+        new["seq_ids"] = torch.arange(s.batch, dtype=torch.int32, device=device)
+        new["positions"] = (w.context_lens - 1).to(torch.int32)
+    else:
+        new["slots"] = w.slot_mapping[last].contiguous()
+        new["seq_ids"] = new["positions"] = None
+    return w, c, new, static
+
+
+def main_ours(args):
+    import torch
+    import torch.distributed as dist
+    from quantized_paged_kv_02_b200 import build
+    build.build()
+    from quantized_paged_kv_02_b200 import kvq, roofline
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    w, cache, new, static = build_state(args.workload, device, seed=rank)
+    s = w.spec
+    B = s.batch
+    out = torch.empty(w.q.shape, dtype=torch.bfloat16, device=device)
+    max_ctx = w.max_context
+    ws_n = cache.workspace_size(B, s.num_q_heads, max_ctx)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=device) if ws_n else None
+    stream = torch.cuda.current_stream()
+
+    def write():
+        cache.write(new["k"], new["v"], new["slots"], new["seq_ids"], new["positions"])
+
+    def decode():
+        kvq.kvq_decode_attention(cache.desc, w.q, w.block_tables, w.context_lens, max_ctx, out, ws)
+
+    lens = w.context_lens.cpu().tolist()
+    dec_bytes = roofline.decode_bytes(s.cache_dtype, s.scale_mode, s.num_q_heads, s.num_kv_heads,
+                                      s.head_dim, s.block_size, lens)
+    wr_bytes = roofline.write_bytes(s.cache_dtype, s.scale_mode, B, s.num_kv_heads, s.head_dim,
+                                    to_ring=s.cache_dtype == "int4")
+    step_bytes = dec_bytes + wr_bytes
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+
+    # warm-up (at least ~1 s under load so the clock sampler sees the steady state)
+    sampler = ClockSampler(str(torch.cuda.get_device_properties(device).uuid))
+    sampler.start()
+    t_w = time.perf_counter()
+    i = 0
+    while i < max(3, args.warmup) or time.perf_counter() - t_w < 1.0:
+        flush.zero_()
+        write()
+        decode()
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
+    warm = i
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream)
+        write()
+        e[1].record(stream)
+        decode()
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    ms = statistics.mean(step_ms)
+    dms = statistics.mean(dec_ms)
+    if world > 1:
+        t = torch.tensor([ms, dms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, dms = t.tolist()
+
+    # end to end through the C ABI: host inputs in pinned memory, copies inside the region
+    E = args.e2e_steps
+    h = {k2: new[k2].cpu().pin_memory() for k2 in ("k", "v", "slots")}
+    hq = w.q.cpu().pin_memory()
+    hl = w.context_lens.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dk, dv, dslots = torch.empty_like(new["k"]), torch.empty_like(new["v"]), torch.empty_like(new["slots"])
+    dq, dl = torch.empty_like(w.q), torch.empty_like(w.context_lens)
+    h2d = sum(t.numel() * t.element_size() for t in (h["k"], h["v"], h["slots"], hq, hl))
+    d2h = hout.numel() * hout.element_size()
+    e2e_ms = []
+    for k in range(E + 3):
+        flush.zero_()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dk.copy_(h["k"], non_blocking=True)
+        dv.copy_(h["v"], non_blocking=True)
+        dslots.copy_(h["slots"], non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        dl.copy_(hl, non_blocking=True)
+        kvq.kvq_write(cache.desc, dk, dv, dslots, new["seq_ids"], new["positions"])
+        kvq.kvq_decode_attention(cache.desc, dq, w.block_tables, dl, max_ctx, out, ws)
+        hout.copy_(out, non_blocking=True)
+        b2.record(stream)
+        b2.synchronize()
+        if k >= 3:
+            e2e_ms.append(a.elapsed_time(b2))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = t.item()
+
+    peak, peak_kind = hbm_peak()
+    achieved = dec_bytes / (dms * 1e-3) / 1e9
+    launches_per_step = 2 + (1 if ws_n else 0)
+    result = {
+        "metric": METRIC,
+        "value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": warm,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp32",
+        "cache_dtype": s.cache_dtype,
+        "data": "synthetic",
+        "config": {"workload": "%s: %s; step = kvq_write of %d new tokens + decode attention"
+                               % (args.workload, WORKLOADS[args.workload], B),
+                   "global_batch": B * world, "seq_len": max_ctx, "parallelism": "dp%d" % world,
+                   "l2": "flushed: 512 MiB memset before every timed step (outside the events)"},
+        "tokens_per_s": round(world * B / (ms * 1e-3), 1),
+        "hbm_frac_of_%s" % peak_kind: round(step_bytes / (ms * 1e-3) / 1e9 / peak, 4),
+        "bytes_per_step": step_bytes,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_kind": peak_kind, "kernel": "kvq_decode_attention (split kernel + reduce)",
+                     "bytes_per_launch": dec_bytes, "ms_per_launch": round(dms, 5),
+                     "traffic": profile_traffic(args.workload)},
+        "e2e": {"value": round(world * step_bytes / (e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e, 5), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = run_oracle_sample(w, static)
+        result["cpu_baseline"] = {
+            "value": round(r["bytes"] / r["seconds"] / 1e9, 6), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": "%d of %d (sequence, kv head) units, each: quantize the new row + float64 "
+                      "attention of its %d query heads over all cached positions; %.1f s"
+                      % (r["units"], B * s.num_kv_heads, s.num_q_heads // s.num_kv_heads,
+                         r["seconds"])}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def main_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    from quantized_paged_kv_02_b200 import inputs
+    from threadpoolctl import threadpool_limits
+    w = unit_workload(args.workload)
+    static = None
+    if w.spec.scale_mode in ("per_head", "per_tensor"):
+        from oracle import quant
+        static = (quant.fp8_calibrate(w.warmup_k.float().numpy()),
+                  quant.fp8_calibrate(w.warmup_v.float().numpy()))
+    rows = oracle_inputs(w, [(0, 0)])
+    step = oracle_unit_step(w, rows, 0, 0, static)
+    nbytes = unit_bytes(w, 0)
+    with threadpool_limits(limits=1):
+        for _ in range(max(1, args.warmup)):
+            step()
+        times = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            step()
+            times.append(time.perf_counter() - t0)
+    sec = statistics.mean(times)
+    value = nbytes / sec / 1e9
+    del torch
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "%s: %s; step = one (sequence, kv head) unit of the serving step"
+                               % (args.workload, WORKLOADS[args.workload])},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "unit (sequence 0, kv head 0): quantize the new row + float64 "
+                                   "attention of its query heads over every cached position"},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)

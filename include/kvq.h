@@ -128,7 +128,7 @@ enum {
  *                 residual ring.
  *   scale_mode    NONE for BF16/FP16; PER_TOKEN_HEAD, PER_HEAD or PER_TENSOR for INT8
  *                 and FP8; KIVI for INT4.
- *   block_size    tokens per block: 1..256 for dense caches; INT4 requires
+ *   block_size    tokens per block: 1..1024 for dense caches; INT4 requires
  *                 block_size == group_size == 64.
  *   head_dim      64 or 128.
  *   group_size, residual_len, residual_cap, max_seqs: INT4 only (64, r, cap, seqs);
@@ -164,14 +164,16 @@ const char* kvq_status_string(kvq_status status);
 int kvq_version(void);
 
 /*
- * Byte sizes the caller must allocate for each pool of a cache described by `cache`
- * (pointer fields are ignored).  Any out pointer may be NULL.  Host-only; never
- * touches the device.  Sizes follow the layout above ([P-prod] "KV Cache 的基本内存
- * 模型": 2 x layers x kv_heads x head_dim x tokens x bytes per value, per layer here,
- * plus the scale, zero-point and residual bytes that make the real gain smaller).
+ * Byte sizes the caller must allocate for the pools of a cache described by `cache`
+ * (pointer fields are ignored): each of k_codes / v_codes, k_scales, v_scales and
+ * residual.  Any out pointer may be NULL.  Host-only; never touches the device.  The
+ * sizes follow the layout above ([P-prod] "KV Cache 的基本内存模型": 2 x layers x
+ * kv_heads x head_dim x tokens x bytes per value, per layer here, plus the scale,
+ * zero-point and residual bytes that make the real gain smaller).
  */
 kvq_status kvq_cache_layout(const kvq_cache_desc* cache, size_t* code_bytes_per_pool,
-                            size_t* scale_bytes_per_pool, size_t* residual_bytes);
+                            size_t* k_scale_bytes, size_t* v_scale_bytes,
+                            size_t* residual_bytes);
 
 /*
  * kvq_write - quantize new K/V rows into the cache ("quantize on write").

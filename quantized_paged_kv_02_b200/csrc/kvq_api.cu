@@ -1,0 +1,230 @@
+// C ABI entry points: host-side validation, layout arithmetic and dispatch.
+// Declarations and the contract of every call are in include/kvq.h.
+#include <cmath>
+#include <cstdint>
+
+#include "kvq_decode_common.cuh"
+
+namespace kvq {
+
+int code_bits(int cd) {
+  switch (cd) {
+    case KVQ_DTYPE_BF16:
+    case KVQ_DTYPE_FP16: return 16;
+    case KVQ_DTYPE_INT8:
+    case KVQ_DTYPE_FP8_E4M3: return 8;
+    case KVQ_DTYPE_INT4: return 4;
+  }
+  return 0;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
+  if (c == nullptr) return KVQ_ERR_INVALID_ARG;
+  g->cache_dtype = c->cache_dtype;
+  g->act_dtype = c->act_dtype;
+  g->scale_mode = c->scale_mode;
+  g->NB = c->num_blocks;
+  g->bs = c->block_size;
+  g->H = c->num_kv_heads;
+  g->D = c->head_dim;
+  g->group = c->group_size;
+  g->residual_len = c->residual_len;
+  g->residual_cap = c->residual_cap;
+  g->max_seqs = c->max_seqs;
+  if (code_bits(c->cache_dtype) == 0) return KVQ_ERR_INVALID_ARG;
+  if (c->act_dtype != KVQ_DTYPE_BF16 && c->act_dtype != KVQ_DTYPE_FP16) return KVQ_ERR_INVALID_ARG;
+  if (c->num_blocks < 1 || c->num_kv_heads < 1 || c->block_size < 1 || c->block_size > 1024)
+    return KVQ_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if (c->k_codes == nullptr || c->v_codes == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(c->k_codes) || !aligned16(c->v_codes)) return KVQ_ERR_INVALID_ARG;
+  switch (c->cache_dtype) {
+    case KVQ_DTYPE_BF16:
+    case KVQ_DTYPE_FP16:
+      if (c->scale_mode != KVQ_SCALE_NONE) return KVQ_ERR_INVALID_ARG;
+      if (c->cache_dtype != c->act_dtype) return KVQ_ERR_UNSUPPORTED;
+      break;
+    case KVQ_DTYPE_INT8:
+    case KVQ_DTYPE_FP8_E4M3:
+      if (c->scale_mode != KVQ_SCALE_PER_TOKEN_HEAD && c->scale_mode != KVQ_SCALE_PER_HEAD &&
+          c->scale_mode != KVQ_SCALE_PER_TENSOR)
+        return KVQ_ERR_INVALID_ARG;
+      if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
+      if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
+      break;
+    case KVQ_DTYPE_INT4:
+      if (c->scale_mode != KVQ_SCALE_KIVI) return KVQ_ERR_INVALID_ARG;
+      if (c->group_size != 64 || c->block_size != 64) return KVQ_ERR_UNSUPPORTED;
+      if (c->residual_len < 0 || c->residual_cap < c->residual_len + c->group_size) return KVQ_ERR_INVALID_ARG;
+      if (c->max_seqs < 1 || c->residual == nullptr || !aligned16(c->residual)) return KVQ_ERR_INVALID_ARG;
+      if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
+      if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
+      break;
+  }
+  return KVQ_OK;
+}
+
+static kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "KVQ_OK";
+    case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+    case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+    case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+    case KVQ_ERR_DEVICE_FAULT: return "KVQ_ERR_DEVICE_FAULT";
+  }
+  return "KVQ_UNKNOWN_STATUS";
+}
+
+int kvq_version(void) { return 100; }
+
+kvq_status kvq_cache_layout(const kvq_cache_desc* c, size_t* code_bytes, size_t* k_scale_bytes,
+                            size_t* v_scale_bytes, size_t* residual_bytes) {
+  if (c == nullptr) return KVQ_ERR_INVALID_ARG;
+  kvq_cache_desc probe = *c;
+  // validate the geometry without requiring real pointers
+  static char dummy[16] __attribute__((aligned(16)));
+  probe.k_codes = probe.v_codes = probe.k_scales = probe.v_scales = probe.residual = dummy;
+  Geometry g;
+  const kvq_status st = validate_desc(&probe, &g);
+  if (st != KVQ_OK) return st;
+  const size_t rows = static_cast<size_t>(g.NB) * g.H * g.bs;
+  const size_t cb = rows * g.D * code_bits(g.cache_dtype) / 8;
+  size_t ks = 0, vs = 0, rb = 0;
+  switch (g.scale_mode) {
+    case KVQ_SCALE_PER_TOKEN_HEAD: ks = vs = rows * 4; break;
+    case KVQ_SCALE_PER_HEAD: ks = vs = static_cast<size_t>(g.H) * 4; break;
+    case KVQ_SCALE_PER_TENSOR: ks = vs = 4; break;
+    case KVQ_SCALE_KIVI:
+      ks = static_cast<size_t>(g.NB) * g.H * 2 * g.D * 2;
+      vs = rows * (g.D / 64) * 2 * 2;
+      rb = static_cast<size_t>(g.max_seqs) * 2 * g.H * g.residual_cap * g.D * 2;
+      break;
+  }
+  if (code_bytes) *code_bytes = cb;
+  if (k_scale_bytes) *k_scale_bytes = ks;
+  if (v_scale_bytes) *v_scale_bytes = vs;
+  if (residual_bytes) *residual_bytes = rb;
+  return KVQ_OK;
+}
+
+kvq_status kvq_write(const kvq_cache_desc* c, const void* k_new, const void* v_new,
+                     int num_tokens, const int32_t* slot_mapping, const int32_t* seq_ids,
+                     const int32_t* positions, cudaStream_t stream) {
+  Geometry g;
+  kvq_status st = validate_desc(c, &g);
+  if (st != KVQ_OK) return st;
+  if (num_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  if (num_tokens == 0) return KVQ_OK;
+  if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+  if (g.cache_dtype == KVQ_DTYPE_INT4)
+    return from_cuda(launch_write_int4(*c, g, k_new, v_new, num_tokens, slot_mapping, seq_ids,
+                                       positions, stream));
+  return from_cuda(launch_write_dense(*c, g, k_new, v_new, num_tokens, slot_mapping, stream));
+}
+
+kvq_status kvq_decode_workspace_size(const kvq_cache_desc* c, int batch, int num_q_heads,
+                                     int max_context, size_t* bytes) {
+  if (c == nullptr || bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  kvq_cache_desc probe = *c;
+  static char dummy[16] __attribute__((aligned(16)));
+  probe.k_codes = probe.v_codes = probe.k_scales = probe.v_scales = probe.residual = dummy;
+  Geometry g;
+  kvq_status st = validate_desc(&probe, &g);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 || max_context < 0)
+    return KVQ_ERR_INVALID_ARG;
+  DecodePlan p;
+  st = plan_decode(g, batch, num_q_heads, max_context, &p);
+  if (st != KVQ_OK) return st;
+  *bytes = p.ws_bytes;
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_cache_desc* c, const void* q, int batch,
+                                int num_q_heads, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                const int32_t* seq_ids, int max_context, float softmax_scale,
+                                void* out, int32_t out_dtype, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream) {
+  Geometry g;
+  kvq_status st = validate_desc(c, &g);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 || max_context < 0 ||
+      max_blocks_per_seq < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (out_dtype != KVQ_DTYPE_BF16 && out_dtype != KVQ_DTYPE_FP16 && out_dtype != KVQ_DTYPE_FP32)
+    return KVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (q == nullptr || block_tables == nullptr || context_lens == nullptr || out == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return KVQ_ERR_INVALID_ARG;
+  DecodeArgs a{};
+  a.c = c;
+  a.geo = g;
+  st = plan_decode(g, batch, num_q_heads, max_context, &a.plan);
+  if (st != KVQ_OK) return st;
+  if (a.plan.ws_bytes > 0) {
+    if (workspace == nullptr || workspace_bytes < a.plan.ws_bytes || !aligned16(workspace))
+      return KVQ_ERR_INVALID_ARG;
+    const size_t rows = static_cast<size_t>(batch) * num_q_heads * a.plan.splits;
+    a.ws_o = static_cast<float*>(workspace);
+    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       (rows * g.D * sizeof(float) + 255) / 256 * 256);
+  }
+  a.q = q;
+  a.batch = batch;
+  a.Hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_blocks = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.seq_ids = seq_ids;
+  a.max_context = max_context;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(g.D));
+  a.scale_log2 = scale * kLog2e;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_decode(a, stream));
+}
+
+kvq_status kvq_dequant(const kvq_cache_desc* c, const int32_t* block_ids, int n_blocks,
+                       float* out, cudaStream_t stream) {
+  Geometry g;
+  kvq_status st = validate_desc(c, &g);
+  if (st != KVQ_OK) return st;
+  if (n_blocks < 0) return KVQ_ERR_INVALID_ARG;
+  if (n_blocks == 0) return KVQ_OK;
+  if (block_ids == nullptr || out == nullptr) return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_dequant(*c, g, block_ids, n_blocks, out, stream));
+}
+
+kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_heads, int head_dim,
+                                    int32_t act_dtype, float* scale_out, cudaStream_t stream) {
+  if (n_tokens < 0 || num_kv_heads < 1 || head_dim < 1) return KVQ_ERR_INVALID_ARG;
+  if (act_dtype != KVQ_DTYPE_BF16 && act_dtype != KVQ_DTYPE_FP16) return KVQ_ERR_INVALID_ARG;
+  if (scale_out == nullptr || (n_tokens > 0 && x == nullptr)) return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, scale_out, stream));
+}
+
+kvq_status kvq_read_device_fault(const kvq_cache_desc* c, int32_t* out, int reset,
+                                 cudaStream_t stream) {
+  if (c == nullptr || out == nullptr || c->fault == nullptr) return KVQ_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemcpyAsync(out, c->fault, 2 * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && reset) e = cudaMemsetAsync(c->fault, 0, 2 * sizeof(int32_t), stream);
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  return out[0] != 0 ? KVQ_ERR_DEVICE_FAULT : KVQ_OK;
+}
+
+}  // extern "C"

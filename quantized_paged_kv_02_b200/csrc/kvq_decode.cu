@@ -1,0 +1,107 @@
+// Decode dispatch: split plan, kernel choice, and the split-K log-sum-exp reduce.
+//
+// The reduce merges the S partials (m_s, l_s, o_s) of each (sequence, query head):
+//   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  out = sum_s o_s 2^(m_s - M) / L,
+// the usual merge of softmax partial sums over disjoint token ranges (the pages leave
+// the split of long contexts open; it follows from decode reading every cached
+// position at each step, [P-prod] "为什么长上下文更需要 KV Cache Quantization").
+#include <algorithm>
+
+#include "kvq_decode_common.cuh"
+
+namespace kvq {
+namespace {
+
+__global__ void __launch_bounds__(128) split_reduce_kernel(DecodeParams p, bool int4) {
+  const int row = blockIdx.x;                 // b * Hq + hq
+  const int b = row / p.Hq;
+  const SeqInfo si = seq_info(p, b, int4);
+  const int S = (si.n + p.chunk - 1) / p.chunk;
+  const float* ml = p.ws_ml + static_cast<long>(row) * p.splits * 2;
+  const float* o = p.ws_o + static_cast<long>(row) * p.splits * p.D;
+  float M = -INFINITY;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[2 * s]);
+  float L = 0.f;
+  for (int s = 0; s < S; ++s) L += (M == -INFINITY) ? 0.f : ml[2 * s + 1] * exp2f(ml[2 * s] - M);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float w = (M == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);
+      acc = fmaf(o[static_cast<long>(s) * p.D + d], w, acc);
+    }
+    store_out(p, static_cast<long>(row) * p.D + d, acc * inv);
+  }
+}
+
+}  // namespace
+
+kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_context,
+                       DecodePlan* p) {
+  p->g = num_q_heads / g.H;
+  p->kernel = 0;
+  p->g_tile = (p->g % 2 == 0) ? 2 : 1;
+  const long units = static_cast<long>(batch) * g.H * (p->g / p->g_tile);
+  const int gran = g.cache_dtype == KVQ_DTYPE_INT4 ? 64 : g.bs;
+  // aim for about 8 resident CTAs per SM, without splits shorter than 256 tokens
+  const long target = 8L * kNumSMs;
+  long S = units > 0 ? (target + units - 1) / units : 1;
+  const long max_split_by_len = std::max(1L, (static_cast<long>(max_context) + 255) / 256);
+  S = std::max(1L, std::min(S, max_split_by_len));
+  long chunk = (static_cast<long>(max_context) + S - 1) / S;
+  chunk = std::max(1L, (chunk + gran - 1) / gran) * gran;
+  S = std::max(1L, (static_cast<long>(max_context) + chunk - 1) / chunk);
+  p->splits = static_cast<int>(S);
+  p->chunk = static_cast<int>(chunk);
+  p->ws_bytes = 0;
+  if (S > 1) {
+    const size_t rows = static_cast<size_t>(batch) * num_q_heads * S;
+    const size_t o_bytes = (rows * g.D * sizeof(float) + 255) / 256 * 256;
+    p->ws_bytes = o_bytes + rows * 2 * sizeof(float);
+  }
+  return KVQ_OK;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+  const Geometry& g = a.geo;
+  DecodeParams p{};
+  p.q = a.q;
+  p.tables = a.block_tables;
+  p.lens = a.context_lens;
+  p.seq_ids = a.seq_ids;
+  p.max_blocks = a.max_blocks;
+  p.max_context = a.max_context;
+  p.k_codes = a.c->k_codes;
+  p.v_codes = a.c->v_codes;
+  p.k_scales = a.c->k_scales;
+  p.v_scales = a.c->v_scales;
+  p.residual = a.c->residual;
+  p.NB = g.NB;
+  p.bs = g.bs;
+  p.H = g.H;
+  p.Hq = a.Hq;
+  p.D = g.D;
+  p.g = a.plan.g;
+  p.cap = g.residual_cap;
+  p.rlen = g.residual_len;
+  p.max_seqs = g.max_seqs;
+  p.mode = g.scale_mode;
+  p.splits = a.plan.splits;
+  p.chunk = a.plan.chunk;
+  p.scale_log2 = a.scale_log2;
+  p.out = a.out;
+  p.out_dtype = a.out_dtype;
+  p.ws_o = a.ws_o;
+  p.ws_ml = a.ws_ml;
+  p.fault = a.c->fault;
+  if (a.batch == 0) return cudaSuccess;
+  cudaError_t e = launch_decode_simt(a, p, s);
+  if (e != cudaSuccess) return e;
+  if (p.splits > 1) {
+    split_reduce_kernel<<<a.batch * a.Hq, 128, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace kvq

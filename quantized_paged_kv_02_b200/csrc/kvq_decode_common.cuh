@@ -1,0 +1,101 @@
+// Pieces shared by the decode kernels: parameters, per-sequence bounds, block lookup,
+// and the epilogue that writes either a split partial or the final output row.
+#pragma once
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+struct DecodeParams {
+  const void* q;             // [B][Hq][D] act
+  const int32_t* tables;     // [B][max_blocks]
+  const int32_t* lens;       // [B]
+  const int32_t* seq_ids;    // [B] or null (INT4 ring)
+  int max_blocks, max_context;
+  const void* k_codes;
+  const void* v_codes;
+  const void* k_scales;
+  const void* v_scales;
+  const void* residual;
+  int NB, bs, H, Hq, D, g, cap, rlen, max_seqs, mode;
+  int splits, chunk;
+  float scale_log2;
+  void* out;
+  int out_dtype;
+  float* ws_o;               // [B][Hq][S][D]
+  float* ws_ml;              // [B][Hq][S][2]  (max, sum) in the log2 domain
+  int32_t* fault;
+};
+
+struct SeqInfo {
+  int n;     // positions to attend to (0 when the entry was rejected)
+  int qb;    // INT4: positions read from blocks; the rest come from the ring
+  int sid;   // INT4: ring sequence
+};
+
+// Bounds of sequence b.  A context length outside [0, max_context] or beyond what the
+// block table can address, or an INT4 ring id outside [0, max_seqs), rejects the whole
+// sequence (its output row is zero).  `report` selects the one thread that counts it.
+__device__ __forceinline__ SeqInfo seq_info(const DecodeParams& p, int b, bool int4,
+                                            bool report = false) {
+  SeqInfo s;
+  int n = p.lens[b];
+  int bits = 0;
+  if (n < 0 || n > p.max_context) bits |= KVQ_FAULT_CONTEXT;
+  s.sid = b;
+  s.qb = n;
+  if (int4) {
+    s.sid = p.seq_ids ? p.seq_ids[b] : b;
+    if (s.sid < 0 || s.sid >= p.max_seqs) bits |= KVQ_FAULT_SEQ;
+    const int over = n - p.rlen;
+    s.qb = over > 0 ? 64 * (over / 64) : 0;
+    if (s.qb / 64 > p.max_blocks) bits |= KVQ_FAULT_CONTEXT;
+  } else if (static_cast<long>(n) > static_cast<long>(p.max_blocks) * p.bs) {
+    bits |= KVQ_FAULT_CONTEXT;
+  }
+  if (bits) {
+    if (report) record_fault(p.fault, bits);
+    n = 0;
+    s.qb = 0;
+  }
+  s.n = n;
+  return s;
+}
+
+// Physical block of page `page` of sequence b, or -1 (counted) when out of range.
+__device__ __forceinline__ int block_of(const DecodeParams& p, int b, int page) {
+  const int blk = p.tables[static_cast<long>(b) * p.max_blocks + page];
+  if (blk < 0 || blk >= p.NB) {
+    record_fault(p.fault, KVQ_FAULT_BLOCK);
+    return -1;
+  }
+  return blk;
+}
+
+__device__ __forceinline__ void store_out(const DecodeParams& p, long idx, float v) {
+  if (p.out_dtype == KVQ_DTYPE_FP32) static_cast<float*>(p.out)[idx] = v;
+  else if (p.out_dtype == KVQ_DTYPE_BF16) static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+  else static_cast<__half*>(p.out)[idx] = __float2half_rn(v);
+}
+
+// M, L: running max and sum (log2 domain) of this CTA's share; O: unnormalised output.
+__device__ __forceinline__ void store_partial_or_output(const DecodeParams& p, int b, int hq,
+                                                        int split, int d, float M, float L,
+                                                        float O) {
+  const long row = static_cast<long>(b) * p.Hq + hq;
+  if (p.splits == 1) {
+    store_out(p, row * p.D + d, L > 0.f ? O / L : 0.f);
+    return;
+  }
+  const long part = row * p.splits + split;
+  p.ws_o[part * p.D + d] = O;
+  if (d == 0) {
+    p.ws_ml[part * 2] = M;
+    p.ws_ml[part * 2 + 1] = L;
+  }
+}
+
+cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
+
+}  // namespace kvq

@@ -1,0 +1,282 @@
+// Split-K paged decode attention on CUDA cores (fp32 FMA), and the split reduce.
+//
+// One CTA covers (split, kv head, up to two query heads of its GQA group, sequence).
+// Each warp walks the split's token range in batches; a lane owns a 16-element chunk
+// of the head dimension for one row at a time (16 bytes of INT8/FP8 codes, 8 bytes of
+// packed INT4, 16 bytes of BF16/FP16), so a warp instruction reads whole 128-byte rows.
+// Scores are reduced over the lanes of a row with shuffles; each lane group runs its
+// own online softmax (running max, running sum, fp32 accumulator) in the log2 domain,
+// and groups, warps and finally splits are merged with log-sum-exp weights.
+//
+// Dequantization is fused into the inner products ([P-vLLM]
+// "PagedAttention与KV Cache量化协同工作原理": INT8/FP8 blocks are dequantized inside the
+// attention kernel): per-token / per-head scales multiply the dot product and the
+// softmax weight rather than every element; INT4 keys use (code - zero) * scale per
+// channel and INT4 values (code - zero) * scale per token group ([P-prod]
+// "量化不是简单截断精度").  Decode reads every cached position of the sequence each step
+// ([P-prod] "为什么长上下文更需要 KV Cache Quantization"), so this kernel is bound by
+// HBM bandwidth when the ALUs keep up (small GQA groups).
+#include "kvq_internal.cuh"
+#include "kvq_decode_common.cuh"
+
+namespace kvq {
+namespace {
+
+template <int CD> struct Chunk;
+// 1-byte codes: 16 elements in a uint4
+template <> struct Chunk<KVQ_DTYPE_INT8> { static constexpr int EPL = 16, BYTES = 16; };
+template <> struct Chunk<KVQ_DTYPE_FP8_E4M3> { static constexpr int EPL = 16, BYTES = 16; };
+template <> struct Chunk<KVQ_DTYPE_BF16> { static constexpr int EPL = 8, BYTES = 16; };
+template <> struct Chunk<KVQ_DTYPE_FP16> { static constexpr int EPL = 8, BYTES = 16; };
+template <> struct Chunk<KVQ_DTYPE_INT4> { static constexpr int EPL = 16, BYTES = 8; };
+
+// Load EPL cache elements of one row chunk as floats (codes only; scales applied outside).
+template <int CD>
+__device__ __forceinline__ void load_codes(const uint8_t* p, float* f) {
+  if constexpr (CD == KVQ_DTYPE_INT8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const int8_t* c = reinterpret_cast<const int8_t*>(&u);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f[i] = static_cast<float>(c[i]);
+  } else if constexpr (CD == KVQ_DTYPE_FP8_E4M3) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_fp8x2_storage_t* c = reinterpret_cast<const __nv_fp8x2_storage_t*>(&u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(c[i], __NV_E4M3);
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+  } else if constexpr (CD == KVQ_DTYPE_BF16) {
+    unpack8<__nv_bfloat16>(*reinterpret_cast<const uint4*>(p), f);
+  } else if constexpr (CD == KVQ_DTYPE_FP16) {
+    unpack8<__half>(*reinterpret_cast<const uint4*>(p), f);
+  } else {  // INT4: 8 bytes, element 2i in the low nibble of byte i
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const uint8_t* c = reinterpret_cast<const uint8_t*>(&u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = static_cast<float>(c[i] & 0xF);
+      f[2 * i + 1] = static_cast<float>(c[i] >> 4);
+    }
+  }
+}
+
+template <typename TA, int CD, int D, int GT>
+__global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
+  constexpr int NW = 4;
+  constexpr int EPL = Chunk<CD>::EPL;
+  constexpr int CB = Chunk<CD>::BYTES;
+  constexpr int LPR = D / EPL;          // lanes per row
+  constexpr int RPI = 32 / LPR;         // rows per warp instruction
+  constexpr int U = 4;                  // rows per lane per batch
+  constexpr bool kInt4 = CD == KVQ_DTYPE_INT4;
+  constexpr int ROWB = D * CB / EPL;    // bytes per cache row
+
+  const int split = blockIdx.x;
+  const int tiles = p.g / GT;
+  const int kvh = blockIdx.y / tiles;
+  const int hq0 = kvh * p.g + (blockIdx.y % tiles) * GT;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = lane % LPR, grp = lane / LPR;
+
+  const SeqInfo si = seq_info(p, b, kInt4, blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+  const int t0 = split * p.chunk;
+  const int t1 = min(si.n, t0 + p.chunk);
+
+  // query chunk (pre-multiplied by softmax_scale * log2 e)
+  float qf[GT][EPL];
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    const TA* qp = static_cast<const TA*>(p.q) + (static_cast<long>(b) * p.Hq + hq0 + h) * D + c * EPL;
+#pragma unroll
+    for (int i = 0; i < EPL; i += 8) {
+      float f[8];
+      unpack8<TA>(*reinterpret_cast<const uint4*>(qp + i), f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) qf[h][i + j] = f[j] * p.scale_log2;
+    }
+  }
+  float m[GT], l[GT], acc[GT][EPL];
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[h][i] = 0.f;
+  }
+  const float* ksc = static_cast<const float*>(p.k_scales);
+  const float* vsc = static_cast<const float*>(p.v_scales);
+  float khead = 1.f, vhead = 1.f;
+  if constexpr (!kInt4) {
+    if (p.mode == KVQ_SCALE_PER_HEAD) { khead = ksc[kvh]; vhead = vsc[kvh]; }
+    if (p.mode == KVQ_SCALE_PER_TENSOR) { khead = ksc[0]; vhead = vsc[0]; }
+  }
+
+  constexpr int BATCH = RPI * U;
+  for (int base = t0 + warp * BATCH; base < t1; base += NW * BATCH) {
+    float kf[U][EPL], vf[U][EPL];
+    float kscale[U], vscale[U];
+    bool valid[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int pos = base + grp + RPI * j;
+      valid[j] = pos < t1;
+      kscale[j] = khead;
+      vscale[j] = vhead;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) { kf[j][i] = 0.f; vf[j][i] = 0.f; }
+      if (!valid[j]) continue;
+      if (kInt4 && pos >= si.qb) {
+        // residual ring row (unquantized activations)
+        const long rrow = ((static_cast<long>(si.sid) * 2) * p.H + kvh) * p.cap + pos % p.cap;
+        const long vrow = ((static_cast<long>(si.sid) * 2 + 1) * p.H + kvh) * p.cap + pos % p.cap;
+        const TA* kr = static_cast<const TA*>(p.residual) + rrow * D + c * EPL;
+        const TA* vr = static_cast<const TA*>(p.residual) + vrow * D + c * EPL;
+#pragma unroll
+        for (int i = 0; i < EPL; i += 8) {
+          unpack8<TA>(*reinterpret_cast<const uint4*>(kr + i), &kf[j][i]);
+          unpack8<TA>(*reinterpret_cast<const uint4*>(vr + i), &vf[j][i]);
+        }
+        continue;
+      }
+      const int blk = block_of(p, b, pos / p.bs);
+      if (blk < 0) { valid[j] = false; continue; }
+      const int off = pos % p.bs;
+      const long row = (static_cast<long>(blk) * p.H + kvh) * p.bs + off;
+      load_codes<CD>(static_cast<const uint8_t*>(p.k_codes) + row * ROWB + c * CB, kf[j]);
+      load_codes<CD>(static_cast<const uint8_t*>(p.v_codes) + row * ROWB + c * CB, vf[j]);
+      if constexpr (kInt4) {
+        const __half* ksz = static_cast<const __half*>(p.k_scales) + (static_cast<long>(blk) * p.H + kvh) * 2 * D;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int d = c * EPL + i;
+          kf[j][i] = (kf[j][i] - __half2float(ksz[D + d])) * __half2float(ksz[d]);
+        }
+        const __half* vsz = static_cast<const __half*>(p.v_scales) + (row * (D / 64) + (c * EPL) / 64) * 2;
+        const float vz = __half2float(vsz[1]);
+        vscale[j] = __half2float(vsz[0]);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) vf[j][i] -= vz;
+      } else if (p.mode == KVQ_SCALE_PER_TOKEN_HEAD) {
+        kscale[j] = ksc[row];
+        vscale[j] = vsc[row];
+      }
+    }
+    // scores of the U rows for each head
+    float s[GT][U];
+#pragma unroll
+    for (int h = 0; h < GT; ++h) {
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        float d = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) d = fmaf(qf[h][i], kf[j][i], d);
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        s[h][j] = valid[j] ? d * kscale[j] : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < GT; ++h) {
+      float mx = m[h];
+#pragma unroll
+      for (int j = 0; j < U; ++j) mx = fmaxf(mx, s[h][j]);
+      if (mx == -INFINITY) continue;
+      const float corr = exp2f(m[h] - mx);
+      m[h] = mx;
+      l[h] *= corr;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) acc[h][i] *= corr;
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const float pj = valid[j] ? exp2f(s[h][j] - mx) : 0.f;
+        l[h] += pj;
+        const float pv = pj * vscale[j];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[h][i] = fmaf(pv, vf[j][i], acc[h][i]);
+      }
+    }
+  }
+
+  // merge the lane groups of this warp (lanes with the same chunk c)
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    float M = m[h];
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float f = (M == -INFINITY) ? 0.f : exp2f(m[h] - M);
+    float L = l[h] * f;
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      float a = acc[h][i] * f;
+#pragma unroll
+      for (int o = LPR; o < 32; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      acc[h][i] = a;
+    }
+    m[h] = M;
+    l[h] = L;
+  }
+  __shared__ float sm_acc[NW][GT][D];
+  __shared__ float sm_ml[NW][GT][2];
+  if (grp == 0) {
+#pragma unroll
+    for (int h = 0; h < GT; ++h) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) sm_acc[warp][h][c * EPL + i] = acc[h][i];
+      if (c == 0) { sm_ml[warp][h][0] = m[h]; sm_ml[warp][h][1] = l[h]; }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < GT * D; e += blockDim.x) {
+    const int h = e / D, d = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_ml[w][h][0]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = (M == -INFINITY) ? 0.f : exp2f(sm_ml[w][h][0] - M);
+      L += sm_ml[w][h][1] * f;
+      O += sm_acc[w][h][d] * f;
+    }
+    store_partial_or_output(p, b, hq0 + h, split, d, M, L, O);
+  }
+}
+
+template <typename TA, int CD, int D>
+cudaError_t launch_cd(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  if (p.g % 2 == 0) decode_simt_kernel<TA, CD, D, 2><<<grid, 128, 0, s>>>(p);
+  else decode_simt_kernel<TA, CD, D, 1><<<grid, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename TA, int D>
+cudaError_t launch_d(int cd, const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  switch (cd) {
+    case KVQ_DTYPE_INT8: return launch_cd<TA, KVQ_DTYPE_INT8, D>(p, grid, s);
+    case KVQ_DTYPE_FP8_E4M3: return launch_cd<TA, KVQ_DTYPE_FP8_E4M3, D>(p, grid, s);
+    case KVQ_DTYPE_BF16: return launch_cd<TA, KVQ_DTYPE_BF16, D>(p, grid, s);
+    case KVQ_DTYPE_FP16: return launch_cd<TA, KVQ_DTYPE_FP16, D>(p, grid, s);
+    case KVQ_DTYPE_INT4: return launch_cd<TA, KVQ_DTYPE_INT4, D>(p, grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  const int gt = (a.plan.g % 2 == 0) ? 2 : 1;
+  const dim3 grid(a.plan.splits, a.geo.H * (a.plan.g / gt), a.batch);
+  if (a.geo.act_dtype == KVQ_DTYPE_BF16)
+    return a.geo.D == 128 ? launch_d<__nv_bfloat16, 128>(a.geo.cache_dtype, p, grid, s)
+                          : launch_d<__nv_bfloat16, 64>(a.geo.cache_dtype, p, grid, s);
+  return a.geo.D == 128 ? launch_d<__half, 128>(a.geo.cache_dtype, p, grid, s)
+                        : launch_d<__half, 64>(a.geo.cache_dtype, p, grid, s);
+}
+
+}  // namespace kvq

@@ -1,0 +1,118 @@
+// kvq_dequant (debug) and kvq_calibrate_fp8_scales (set-up) kernels.
+//
+// Dequantized values follow the definitions in include/kvq.h: INT8 / FP8 code * scale
+// ([P-mem] §3.1 对称量化算法: q.float() * scale), INT4 (code - zero) * scale ([P-prod]
+// "量化不是简单截断精度": X_dequant = (X_q - zero_point) * scale).
+// The calibration scale is max|x| / 448 per kv head over warm-up rows ([P-prod]
+// "vLLM：从 FP8 KV Cache 开始试点": scales from a random-token warm-up).
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+struct DequantParams {
+  const int32_t* ids;
+  int n;
+  const void* k_codes;
+  const void* v_codes;
+  const void* k_scales;
+  const void* v_scales;
+  int NB, bs, H, D, cd, act, mode;
+  float* out;
+  int32_t* fault;
+};
+
+// grid (n_blocks, 2, H): one CTA writes one [bs][D] tile of K or V.
+__global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
+  const int i = blockIdx.x, kv = blockIdx.y, h = blockIdx.z;
+  const int blk = p.ids[i];
+  if (blk < 0 || blk >= p.NB) {
+    if (threadIdx.x == 0 && kv == 0 && h == 0) record_fault(p.fault, KVQ_FAULT_BLOCK);
+    return;
+  }
+  const long tile = (static_cast<long>(blk) * p.H + h) * p.bs;   // first row of the tile
+  float* out = p.out + (((static_cast<long>(i) * 2 + kv) * p.H + h) * p.bs) * p.D;
+  const void* codes = kv ? p.v_codes : p.k_codes;
+  const void* sc = kv ? p.v_scales : p.k_scales;
+  for (int e = threadIdx.x; e < p.bs * p.D; e += blockDim.x) {
+    const int t = e / p.D, d = e % p.D;
+    float x;
+    switch (p.cd) {
+      case KVQ_DTYPE_BF16:
+        x = __bfloat162float(static_cast<const __nv_bfloat16*>(codes)[(tile + t) * p.D + d]);
+        break;
+      case KVQ_DTYPE_FP16:
+        x = __half2float(static_cast<const __half*>(codes)[(tile + t) * p.D + d]);
+        break;
+      case KVQ_DTYPE_INT8:
+      case KVQ_DTYPE_FP8_E4M3: {
+        const uint8_t c = static_cast<const uint8_t*>(codes)[(tile + t) * p.D + d];
+        const float* s = static_cast<const float*>(sc);
+        const float sv = p.mode == KVQ_SCALE_PER_TOKEN_HEAD ? s[tile + t]
+                         : p.mode == KVQ_SCALE_PER_HEAD   ? s[h] : s[0];
+        const float cv = p.cd == KVQ_DTYPE_INT8 ? static_cast<float>(static_cast<int8_t>(c))
+                                                : e4m3_to_float(c);
+        x = cv * sv;
+        break;
+      }
+      default: {  // INT4
+        const uint8_t byte = static_cast<const uint8_t*>(codes)[(tile + t) * (p.D / 2) + d / 2];
+        const int c = (d & 1) ? (byte >> 4) : (byte & 0xF);
+        const __half* sz = static_cast<const __half*>(sc);
+        float s, z;
+        if (kv == 0) {
+          const long base = (static_cast<long>(blk) * p.H + h) * 2 * p.D;
+          s = __half2float(sz[base + d]);
+          z = __half2float(sz[base + p.D + d]);
+        } else {
+          const long base = (((static_cast<long>(blk) * p.H + h) * p.bs + t) * (p.D / 64) + d / 64) * 2;
+          s = __half2float(sz[base]);
+          z = __half2float(sz[base + 1]);
+        }
+        x = (static_cast<float>(c) - z) * s;
+      }
+    }
+    out[e] = x;
+  }
+}
+
+template <typename TA>
+__global__ void __launch_bounds__(256) calibrate_kernel(const TA* x, int n, int H, int D, float* out) {
+  const int h = blockIdx.x;
+  float m = 0.f;
+  for (long e = threadIdx.x; e < static_cast<long>(n) * D; e += blockDim.x) {
+    const long t = e / D, d = e % D;
+    m = fmaxf(m, fabsf(Act<TA>::to_f(x[(t * H + h) * D + d])));
+  }
+  __shared__ float red[32];
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) out[h] = div_rn(m, 448.f);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int32_t* ids, int n,
+                           float* out, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  DequantParams p{ids, n, c.k_codes, c.v_codes, c.k_scales, c.v_scales,
+                  g.NB, g.bs, g.H, g.D, g.cache_dtype, g.act_dtype, g.scale_mode, out, c.fault};
+  dequant_kernel<<<dim3(n, 2, g.H), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float* out,
+                             cudaStream_t s) {
+  if (act == KVQ_DTYPE_BF16)
+    calibrate_kernel<__nv_bfloat16><<<H, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n, H, D, out);
+  else
+    calibrate_kernel<__half><<<H, 256, 0, s>>>(static_cast<const __half*>(x), n, H, D, out);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,306 @@
+// kvq_write kernels: quantize new K/V rows into the paged cache.
+//
+// Dense caches (INT8 / FP8 E4M3 / BF16 / FP16): one group of D*2/16 lanes per
+// (kv tensor, token, kv head) row; each lane loads 16 bytes of activations, the group
+// reduces max|x| with shuffles, and each lane stores its codes.  Rows are ordered
+// (K or V, token, head) so a warp's loads cover contiguous memory.
+//   INT8: [P-mem] §3.1 对称量化算法 (scale = max|x|/127, q = clamp(round(x/scale),-128,127))
+//         with one fp32 scale per token per head ([P-mem] §3.2 动态量化策略).
+//   FP8 : [P-vLLM] "KV Cache量化策略：INT8与FP8精度对比与选择" (E4M3 storage with a scale);
+//         per-head static scales as in [P-prod] "vLLM：从 FP8 KV Cache 开始试点".
+// INT4 KIVI: one CTA per (64-row group, kv head).  Keys are quantized per channel over
+// the block's 64 tokens, values per token over 64-channel groups ([P-prod] "Key 和 Value
+// 的分布不一定相同"), with the affine form of [P-prod] "量化不是简单截断精度".  Rows that
+// belong to no block are copied unquantized into the residual ring.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+struct WriteParams {
+  const void* k;
+  const void* v;
+  const int32_t* slots;
+  int T;
+  void* k_codes;
+  void* v_codes;
+  float* k_scales;
+  float* v_scales;
+  int NB, bs, H;
+  int scale_mode;
+  int32_t* fault;
+};
+
+template <int CD> struct QMax;
+template <> struct QMax<KVQ_DTYPE_INT8> { static constexpr float v = 127.f; };
+template <> struct QMax<KVQ_DTYPE_FP8_E4M3> { static constexpr float v = 448.f; };
+
+__device__ __forceinline__ uint8_t quant_int8(float x, float s) {
+  if (s == 0.f) return 0;
+  int q = __float2int_rn(div_rn(x, s));
+  q = max(-128, min(127, q));
+  return static_cast<uint8_t>(static_cast<int8_t>(q));
+}
+
+__device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
+  if (s == 0.f) return 0;
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(div_rn(x, s), __NV_SATFINITE, __NV_E4M3));
+}
+
+template <typename TA, int CD, int D>
+__global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
+  constexpr int LPR = D * 2 / 16;   // lanes per row
+  constexpr int RPW = 32 / LPR;     // rows per warp
+  const int lane = threadIdx.x & 31;
+  const long warp = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int l = lane % LPR;
+  const long row = warp * RPW + lane / LPR;
+  const long TH = static_cast<long>(p.T) * p.H;
+  const bool valid = row < 2 * TH;
+  const int kv = valid ? static_cast<int>(row / TH) : 0;
+  const long th = valid ? row % TH : 0;
+  const int t = static_cast<int>(th / p.H);
+  const int h = static_cast<int>(th % p.H);
+  const int slot = valid ? p.slots[t] : -1;
+  const long nslots = static_cast<long>(p.NB) * p.bs;
+  const bool write = valid && slot >= 0 && slot < nslots;
+  if (valid && l == 0 && kv == 0 && h == 0 && (slot < -1 || slot >= nslots)) record_fault(p.fault, KVQ_FAULT_SLOT);
+
+  uint4 u = make_uint4(0, 0, 0, 0);
+  const TA* src = static_cast<const TA*>(kv ? p.v : p.k) + th * D + l * 8;
+  if (write) u = *reinterpret_cast<const uint4*>(src);
+  const int blk = write ? slot / p.bs : 0;
+  const int off = write ? slot % p.bs : 0;
+  const long rowoff = (static_cast<long>(blk) * p.H + h) * p.bs + off;   // [NB][H][bs]
+
+  if constexpr (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) {
+    if (write) reinterpret_cast<uint4*>(kv ? p.v_codes : p.k_codes)[(rowoff * D + l * 8) / 8] = u;
+  } else {
+    float x[8];
+    unpack8<TA>(u, x);
+    float s;
+    if (p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD) {
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      s = div_rn(m, QMax<CD>::v);
+      if (write && l == 0) (kv ? p.v_scales : p.k_scales)[rowoff] = s;
+    } else {
+      const float* sp = kv ? p.v_scales : p.k_scales;
+      s = sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0];
+    }
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
+      if (i < 4) w0 |= c << (8 * i); else w1 |= c << (8 * (i - 4));
+    }
+    if (write) {
+      uint8_t* dst = static_cast<uint8_t*>(kv ? p.v_codes : p.k_codes) + rowoff * D + l * 8;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ INT4 (KIVI)
+struct Int4WriteParams {
+  const void* k;
+  const void* v;
+  const int32_t* slots;
+  const int32_t* seq_ids;
+  const int32_t* positions;
+  int T;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  __half* k_sz;     // [NB][H][2][D]
+  __half* v_sz;     // [NB][H][64][D/64][2]
+  void* residual;   // [max_seqs][2][H][cap][D]
+  int NB, H, cap, max_seqs;
+  int32_t* fault;
+};
+
+struct Int4Group {
+  float sw;       // stored fp16 scale, widened
+  __half s16;
+  int z;
+};
+
+// lo/hi are the group's min and max; the range is widened to include 0.
+__device__ __forceinline__ Int4Group int4_group(float lo, float hi) {
+  lo = fminf(lo, 0.f);
+  hi = fmaxf(hi, 0.f);
+  Int4Group g;
+  g.s16 = __float2half_rn(div_rn(__fsub_rn(hi, lo), 15.f));
+  g.sw = __half2float(g.s16);
+  g.z = (g.sw == 0.f) ? 0 : max(0, min(15, __float2int_rn(div_rn(-lo, g.sw))));
+  return g;
+}
+
+__device__ __forceinline__ int int4_code(float x, const Int4Group& g) {
+  if (g.sw == 0.f) return 0;
+  return max(0, min(15, __float2int_rn(div_rn(x, g.sw)) + g.z));
+}
+
+template <typename TA, int D>
+__global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
+  constexpr int G = 64;
+  __shared__ float xs[G][D + 1];
+  __shared__ __align__(16) uint8_t cs[G][D];
+  __shared__ int ok_s;
+  const int u = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int r0 = u * G;
+  const int nr = min(G, p.T - r0);
+  const int first = p.slots[r0];
+
+  if (first >= 0) {
+    // one whole block, in order
+    if (tid == 0) ok_s = (nr == G && first % G == 0 && first / G < p.NB) ? 1 : 0;
+    __syncthreads();
+    int mine = (tid < nr) ? (p.slots[r0 + tid] == first + tid) : 1;
+    int ok = __syncthreads_and(mine && ok_s);
+    if (!ok) {
+      if (tid == 0) record_fault(p.fault, KVQ_FAULT_INT4_RUN);
+      return;
+    }
+    const long blk = first / G;
+    for (int kv = 0; kv < 2; ++kv) {
+      const TA* src = static_cast<const TA*>(kv ? p.v : p.k);
+      // stage the 64 rows of this head as float
+      for (int i = tid; i < G * D / 8; i += blockDim.x) {
+        const int t = i / (D / 8), c = i % (D / 8);
+        const uint4 w = *reinterpret_cast<const uint4*>(src + (static_cast<long>(r0 + t) * p.H + h) * D + c * 8);
+        float f[8];
+        unpack8<TA>(w, f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xs[t][c * 8 + j] = f[j];
+      }
+      __syncthreads();
+      if (kv == 0) {
+        // keys: one group per channel over the 64 tokens
+        for (int d = tid; d < D; d += blockDim.x) {
+          float lo = xs[0][d], hi = xs[0][d];
+          for (int t = 1; t < G; ++t) { lo = fminf(lo, xs[t][d]); hi = fmaxf(hi, xs[t][d]); }
+          const Int4Group g = int4_group(lo, hi);
+          for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g));
+          __half* sz = p.k_sz + (blk * p.H + h) * 2 * D;
+          sz[d] = g.s16;
+          sz[D + d] = __int2half_rn(g.z);
+        }
+      } else {
+        // values: one group per token per 64 channels
+        for (int i = tid; i < G * (D / 64); i += blockDim.x) {
+          const int t = i / (D / 64), gi = i % (D / 64);
+          float lo = xs[t][gi * 64], hi = lo;
+          for (int j = 1; j < 64; ++j) { lo = fminf(lo, xs[t][gi * 64 + j]); hi = fmaxf(hi, xs[t][gi * 64 + j]); }
+          const Int4Group g = int4_group(lo, hi);
+          for (int j = 0; j < 64; ++j) cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g));
+          __half* sz = p.v_sz + (((blk * p.H + h) * G + t) * (D / 64) + gi) * 2;
+          sz[0] = g.s16;
+          sz[1] = __int2half_rn(g.z);
+        }
+      }
+      __syncthreads();
+      // pack two codes per byte (element 2i low nibble) and store 16 bytes at a time
+      uint8_t* dst = (kv ? p.v_codes : p.k_codes) + (blk * p.H + h) * G * (D / 2);
+      for (int i = tid; i < G * D / 32; i += blockDim.x) {
+        const int t = i / (D / 32), c = i % (D / 32);
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t x = 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int e = c * 32 + j * 8 + b * 2;
+            x |= static_cast<uint32_t>(cs[t][e] | (cs[t][e + 1] << 4)) << (8 * b);
+          }
+          w[j] = x;
+        }
+        *reinterpret_cast<uint4*>(dst + t * (D / 2) + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      __syncthreads();
+    }
+  } else {
+    // residual rows: copied unquantized into ring row positions[t] % cap
+    for (int i = tid; i < nr * 2 * (D / 8); i += blockDim.x) {
+      const int r = i / (2 * (D / 8));
+      const int kv = (i / (D / 8)) % 2;
+      const int c = i % (D / 8);
+      const int t = r0 + r;
+      const int slot = p.slots[t];
+      const bool lead = (kv == 0 && c == 0);
+      if (slot != -1) {
+        if (lead) record_fault(p.fault, KVQ_FAULT_INT4_RUN);
+        continue;
+      }
+      const int pos = p.positions ? p.positions[t] : -1;
+      if (pos < 0) continue;
+      const int sid = p.seq_ids ? p.seq_ids[t] : -1;
+      if (sid < 0 || sid >= p.max_seqs) {
+        if (lead) record_fault(p.fault, KVQ_FAULT_SEQ);
+        continue;
+      }
+      const TA* src = static_cast<const TA*>(kv ? p.v : p.k) + (static_cast<long>(t) * p.H + h) * D + c * 8;
+      TA* dst = static_cast<TA*>(p.residual) +
+                ((static_cast<long>(sid * 2 + kv) * p.H + h) * p.cap + pos % p.cap) * D + c * 8;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+}
+
+template <typename TA, int CD, int D>
+cudaError_t dense_launch(const WriteParams& p, cudaStream_t s) {
+  constexpr int LPR = D * 2 / 16;
+  const long rows = 2L * p.T * p.H;
+  const long threads = (rows * LPR + 31) / 32 * 32;
+  const long blocks = (threads + 255) / 256;
+  if (blocks == 0) return cudaSuccess;
+  write_dense_kernel<TA, CD, D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename TA, int D>
+cudaError_t dense_by_cd(int cd, const WriteParams& p, cudaStream_t s) {
+  switch (cd) {
+    case KVQ_DTYPE_INT8: return dense_launch<TA, KVQ_DTYPE_INT8, D>(p, s);
+    case KVQ_DTYPE_FP8_E4M3: return dense_launch<TA, KVQ_DTYPE_FP8_E4M3, D>(p, s);
+    case KVQ_DTYPE_BF16: return dense_launch<TA, KVQ_DTYPE_BF16, D>(p, s);
+    case KVQ_DTYPE_FP16: return dense_launch<TA, KVQ_DTYPE_FP16, D>(p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_write_dense(const kvq_cache_desc& c, const Geometry& g, const void* k,
+                               const void* v, int T, const int32_t* slots, cudaStream_t s) {
+  WriteParams p{k, v, slots, T, c.k_codes, c.v_codes, static_cast<float*>(c.k_scales),
+                static_cast<float*>(c.v_scales), g.NB, g.bs, g.H, g.scale_mode, c.fault};
+  if (g.act_dtype == KVQ_DTYPE_BF16)
+    return g.D == 128 ? dense_by_cd<__nv_bfloat16, 128>(g.cache_dtype, p, s)
+                      : dense_by_cd<__nv_bfloat16, 64>(g.cache_dtype, p, s);
+  return g.D == 128 ? dense_by_cd<__half, 128>(g.cache_dtype, p, s)
+                    : dense_by_cd<__half, 64>(g.cache_dtype, p, s);
+}
+
+cudaError_t launch_write_int4(const kvq_cache_desc& c, const Geometry& g, const void* k,
+                              const void* v, int T, const int32_t* slots, const int32_t* seq_ids,
+                              const int32_t* positions, cudaStream_t s) {
+  Int4WriteParams p{k, v, slots, seq_ids, positions, T,
+                    static_cast<uint8_t*>(c.k_codes), static_cast<uint8_t*>(c.v_codes),
+                    static_cast<__half*>(c.k_scales), static_cast<__half*>(c.v_scales),
+                    c.residual, g.NB, g.H, g.residual_cap, g.max_seqs, c.fault};
+  const dim3 grid((T + 63) / 64, g.H);
+  if (grid.x == 0) return cudaSuccess;
+  if (g.act_dtype == KVQ_DTYPE_BF16) {
+    if (g.D == 128) write_int4_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
+    else write_int4_kernel<__nv_bfloat16, 64><<<grid, 128, 0, s>>>(p);
+  } else {
+    if (g.D == 128) write_int4_kernel<__half, 128><<<grid, 128, 0, s>>>(p);
+    else write_int4_kernel<__half, 64><<<grid, 128, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,76 @@
+"""Shared test helpers: build the CUDA library, fill a GPU cache and an oracle cache from
+the same seeded workload, compare them."""
+
+import os
+
+import numpy as np
+import torch
+
+from quantized_paged_kv_02_b200 import inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "quantized_paged_kv_02_b200", "libkvq.so")
+
+
+def ensure_built():
+    from quantized_paged_kv_02_b200 import build
+    build.build()
+    return LIB
+
+
+def np64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def oracle_static_scales(w):
+    from oracle import quant
+    if w.spec.scale_mode in ("per_head", "per_tensor"):
+        ks = quant.fp8_calibrate(np64(w.warmup_k).astype(np.float32))
+        vs = quant.fp8_calibrate(np64(w.warmup_v).astype(np.float32))
+        if w.spec.scale_mode == "per_tensor":
+            ks, vs = ks.max(keepdims=True), vs.max(keepdims=True)
+        return ks, vs
+    return None
+
+
+def oracle_cache(w, static=None):
+    """Oracle cache holding every row of workload w."""
+    from oracle import cache
+    s = w.spec
+    c = cache.PagedCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
+                         s.num_kv_heads, s.head_dim, residual_len=inputs.RESIDUAL_LEN,
+                         residual_cap=inputs.RESIDUAL_CAP, max_seqs=max(s.batch, 1),
+                         static_scales=static)
+    k, v = np64(w.k), np64(w.v)
+    if s.cache_dtype == "int4":
+        idx, slots, sid, pos = inputs.int4_group_rows(w)
+        c.write(k[idx.numpy()], v[idx.numpy()], slots.numpy(), sid.numpy(), pos.numpy())
+    else:
+        c.write(k, v, w.slot_mapping.cpu().numpy())
+    return c
+
+
+def gpu_cache(w, device="cuda", static=None, fill=0x5A):
+    """GPU cache holding every row of workload w, written by kvq_write."""
+    from quantized_paged_kv_02_b200 import kvq
+    s = w.spec
+    sk = sv = None
+    if static is not None:
+        sk, sv = (torch.as_tensor(np.asarray(x, np.float32), device=device) for x in static)
+    c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
+                         s.num_kv_heads, s.head_dim, device=device,
+                         residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
+                         max_seqs=max(s.batch, 1), static_k_scale=sk, static_v_scale=sv, fill=fill)
+    k, v = w.k.to(device), w.v.to(device)
+    if s.cache_dtype == "int4":
+        idx, slots, sid, pos = inputs.int4_group_rows(w)
+        idx = idx.to(device)
+        c.write(k[idx].contiguous(), v[idx].contiguous(), slots.to(device), sid.to(device),
+                pos.to(device))
+    else:
+        c.write(k, v, w.slot_mapping.to(device))
+    return c
+
+
+def pool_bytes(t, n):
+    return t[:n].cpu().numpy().view(np.uint8)

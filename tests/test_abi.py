@@ -1,0 +1,112 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared symbol, computes
+layouts and workspace sizes on the host, and rejects bad arguments before launching."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.helpers import ROOT, ensure_built
+
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = ensure_built()
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 9
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_binding_names_match_header():
+    from quantized_paged_kv_02_b200 import kvq
+    assert sorted(kvq.EXPORTS) == declared_symbols()
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    from quantized_paged_kv_02_b200 import kvq
+    monkeypatch.setattr(kvq, "LIB_PATH", "/nonexistent/libkvq.so")
+    with pytest.raises(ImportError):
+        kvq._load()
+
+
+def _desc(kvq, **kw):
+    d = kvq.CacheDesc()
+    base = dict(cache_dtype=3, act_dtype=0, scale_mode=1, num_blocks=16, block_size=16,
+                num_kv_heads=4, head_dim=128, group_size=64, residual_len=128, residual_cap=192,
+                max_seqs=2)
+    base.update(kw)
+    for k, v in base.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_layout_sizes(lib):
+    from quantized_paged_kv_02_b200 import kvq
+    assert kvq.kvq_cache_layout(_desc(kvq)) == (16 * 4 * 16 * 128, 16 * 4 * 16 * 4, 16 * 4 * 16 * 4, 0)
+    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=4, scale_mode=2)) == (131072, 16, 16, 0)
+    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=0, scale_mode=0)) == (262144, 0, 0, 0)
+    c, ks, vs, r = kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=4, block_size=64))
+    assert c == 16 * 4 * 64 * 64 and ks == 16 * 4 * 2 * 128 * 2
+    assert vs == 16 * 4 * 64 * 2 * 2 * 2 and r == 2 * 2 * 4 * 192 * 128 * 2
+    with pytest.raises(kvq.KVQError):
+        kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=4, block_size=16))
+
+
+def test_workspace_plan_is_deterministic(lib):
+    from quantized_paged_kv_02_b200 import kvq
+    d = _desc(kvq, num_kv_heads=8)
+    a = kvq.kvq_decode_workspace_size(d, 24, 64, 16384)
+    assert a == kvq.kvq_decode_workspace_size(d, 24, 64, 16384) and a > 0
+    assert kvq.kvq_decode_workspace_size(d, 1, 8, 16) == 0       # one split: no workspace
+    with pytest.raises(kvq.KVQError):
+        kvq.kvq_decode_workspace_size(d, 2, 12, 100)              # 12 not a multiple of 8
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    from quantized_paged_kv_02_b200 import kvq
+    L = kvq.lib
+    d = _desc(kvq)                 # null pools
+    null = ctypes.c_void_p(0)
+    assert L.kvq_write(ctypes.byref(d), null, null, 4, null, null, null, null) == 1
+    assert L.kvq_write(None, null, null, 4, null, null, null, null) == 1
+    fake = ctypes.c_void_p(0x1000)
+    d2 = _desc(kvq)
+    d2.k_codes = d2.v_codes = d2.k_scales = d2.v_scales = 0x1000
+    assert L.kvq_write(ctypes.byref(d2), null, null, 4, null, null, null, null) == 1
+    assert L.kvq_write(ctypes.byref(d2), fake, fake, -1, fake, null, null, null) == 1
+    assert L.kvq_write(ctypes.byref(d2), fake, fake, 0, fake, null, null, null) == 0   # no work
+    d3 = _desc(kvq, head_dim=96)
+    d3.k_codes = d3.v_codes = d3.k_scales = d3.v_scales = 0x1000
+    assert L.kvq_write(ctypes.byref(d3), fake, fake, 1, fake, null, null, null) == 2   # unsupported
+    # decode: bad head count, bad out dtype, missing workspace
+    assert L.kvq_decode_attention(ctypes.byref(d2), fake, 2, 6, fake, 4, fake, null, 64, 0.0,
+                                  fake, 2, null, 0, null) == 1
+    assert L.kvq_decode_attention(ctypes.byref(d2), fake, 2, 8, fake, 4, fake, null, 64, 0.0,
+                                  fake, 7, null, 0, null) == 1
+    assert L.kvq_decode_attention(ctypes.byref(d2), fake, 24, 32, fake, 1024, fake, null, 16384,
+                                  0.0, fake, 2, null, 0, null) == 1
+    assert L.kvq_decode_attention(ctypes.byref(d2), fake, 2, 8, fake, 4, fake, null, 64,
+                                  ctypes.c_float(float("nan")), fake, 2, null, 0, null) == 1
+    # misaligned pool
+    d4 = _desc(kvq)
+    d4.k_codes, d4.v_codes, d4.k_scales, d4.v_scales = 0x1001, 0x1000, 0x1000, 0x1000
+    assert L.kvq_write(ctypes.byref(d4), fake, fake, 1, fake, null, null, null) == 1
+    # mixed passthrough (bf16 cache, fp16 activations) is unsupported
+    d5 = _desc(kvq, cache_dtype=0, act_dtype=1, scale_mode=0)
+    d5.k_codes = d5.v_codes = 0x1000
+    assert L.kvq_write(ctypes.byref(d5), fake, fake, 1, fake, null, null, null) == 2
+    assert kvq.kvq_status_string(2) == "KVQ_ERR_UNSUPPORTED"

@@ -1,0 +1,139 @@
+"""GPU parity of paged decode attention against the float64 oracle.
+
+The GPU cache is written by kvq_write and the oracle cache by the oracle; their codes
+are identical (test_gpu_write), so the attention check compares against attention over
+the same dequantized cache.  Tolerance: max |gpu - oracle| <= 2e-3 with float32 output;
+a bfloat16 output must be within one bfloat16 ulp of the correctly rounded oracle value.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, fp
+from quantized_paged_kv_02_b200 import inputs
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+SMALL = ["c1", "c2", "c3", "c4", "c5", "c5-fp8", "c5-bf16"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    helpers.ensure_built()
+
+
+def _workload(name, **kw):
+    return inputs.make(name, small=(name != "c1"), **kw)
+
+
+def _decode(gc, w, out_dtype=torch.float32, lens=None, max_context=None, tables=None):
+    lens = w.context_lens if lens is None else lens
+    mc = int(lens.max()) if max_context is None else max_context
+    tables = w.block_tables if tables is None else tables
+    return gc.decode(w.q.cuda(), tables.cuda(), lens.cuda(), mc, out_dtype=out_dtype)
+
+
+def _oracle(oc, w, lens=None):
+    lens = w.context_lens if lens is None else lens
+    return attention.decode_attention(oc, helpers.np64(w.q), w.block_tables.cpu().numpy(),
+                                      lens.cpu().numpy())
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_decode_matches_oracle(name):
+    w = _workload(name)
+    static = helpers.oracle_static_scales(w)
+    oc = helpers.oracle_cache(w, static)
+    gc = helpers.gpu_cache(w, static=static)
+    want = _oracle(oc, w)
+    got = _decode(gc, w).cpu().numpy().astype(np.float64)
+    err = np.abs(got - want).max()
+    assert err <= TOL, err
+    # bf16 output: within one bf16 ulp of the correctly rounded oracle value
+    gotb = _decode(gc, w, torch.bfloat16).float().cpu().numpy().astype(np.float64)
+    wantb = fp.bf16_round(want)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(wantb), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(gotb - wantb) <= ulp * 1.0001)
+    assert gc.read_fault() == (0, 0)
+
+
+@pytest.mark.parametrize("name", ["c2", "c4", "c5-fp8"])
+def test_split_count_does_not_change_result(name):
+    w = _workload(name)
+    static = helpers.oracle_static_scales(w)
+    gc = helpers.gpu_cache(w, static=static)
+    a = _decode(gc, w).cpu()
+    # a larger host bound changes the split plan (more, shorter splits or fewer, longer)
+    for mc in (w.max_context * 3, w.max_context * 40):
+        # tables must address the larger bound: pad with block 0 (never read)
+        pad = (mc + w.spec.block_size - 1) // w.spec.block_size
+        tab = torch.zeros((w.spec.batch, max(pad, w.block_tables.shape[1])), dtype=torch.int32)
+        tab[:, :w.block_tables.shape[1]] = w.block_tables.cpu()
+        b = _decode(gc, w, max_context=mc, tables=tab).cpu()
+        assert (a - b).abs().max().item() <= 1e-5
+
+
+def test_edge_lengths_zero_one_and_ragged():
+    w = _workload("c5")
+    gc = helpers.gpu_cache(w)
+    oc = helpers.oracle_cache(w)
+    lens = torch.tensor([0, 1, 17], dtype=torch.int32)
+    got = _decode(gc, w, lens=lens, max_context=int(w.context_lens.max())).cpu().numpy()
+    want = _oracle(oc, w, lens)
+    assert np.all(got[0] == 0)
+    np.testing.assert_allclose(got[1:], want[1:], atol=TOL, rtol=0)
+    # one token: the output is exactly the dequantized v_0 (softmax weight 1)
+    K, V = oc.gather(w.block_tables.numpy()[1], 1)
+    g = w.spec.num_q_heads // w.spec.num_kv_heads
+    for hq in range(w.spec.num_q_heads):
+        np.testing.assert_allclose(got[1, hq], V[hq // g, 0], rtol=2.0 ** -22, atol=0)
+
+
+def test_block_permutation_invariance_on_gpu():
+    w = _workload("c3")
+    static = helpers.oracle_static_scales(w)
+    gc = helpers.gpu_cache(w, static=static)
+    a = _decode(gc, w).cpu()
+    perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(9)).to(torch.int32)
+    w2 = inputs.make("c3", small=True)
+    bs = w.spec.block_size
+    slots = w2.slot_mapping.clone()
+    slots = perm[slots.long() // bs] * bs + slots % bs
+    w2.slot_mapping = slots.to(torch.int32)
+    w2.block_tables = perm[w.block_tables.long()].to(torch.int32)
+    gc2 = helpers.gpu_cache(w2, static=static)
+    b = _decode(gc2, w2).cpu()
+    assert torch.equal(a, b)
+
+
+def test_bad_block_and_context_are_flagged_not_faulted():
+    w = _workload("c2")
+    gc = helpers.gpu_cache(w)
+    tables = w.block_tables.clone()
+    tables[0, 3] = w.num_blocks + 7            # out of range block id
+    lens = w.context_lens.clone()
+    lens[1] = 10 ** 6                          # beyond max_context
+    out = gc.decode(w.q.cuda(), tables.cuda(), lens.cuda(), int(w.context_lens.max()))
+    torch.cuda.synchronize()
+    cnt, bits = gc.read_fault()
+    assert cnt > 0 and (bits & 2) and (bits & 4)
+    assert torch.all(out[1] == 0)
+    assert torch.isfinite(out).all()
+
+
+def test_zero_query_gives_mean_of_values():
+    w = _workload("c5-fp8")
+    static = helpers.oracle_static_scales(w)
+    gc = helpers.gpu_cache(w, static=static)
+    oc = helpers.oracle_cache(w, static)
+    w.q = torch.zeros_like(w.q)
+    got = _decode(gc, w).cpu().numpy()
+    g = w.spec.num_q_heads // w.spec.num_kv_heads
+    for b in range(w.spec.batch):
+        n = int(w.context_lens[b])
+        K, V = oc.gather(w.block_tables.numpy()[b], n)
+        for hq in range(w.spec.num_q_heads):
+            np.testing.assert_allclose(got[b, hq], V[hq // g].mean(axis=0), atol=1e-5, rtol=0)

@@ -1,0 +1,129 @@
+"""GPU parity of quantize-on-write, calibration and dequant against the oracle.
+
+Codes, scales, zero points and residual rows must be byte-identical to the oracle's,
+and every byte the write should not touch must keep the sentinel."""
+
+import numpy as np
+import pytest
+import torch
+
+from quantized_paged_kv_02_b200 import inputs
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["c1", "c2", "c3", "c4", "c5", "c5-fp8", "c5-bf16"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    helpers.ensure_built()
+
+
+def _workload(name):
+    return inputs.make(name, small=(name != "c1"))
+
+
+def _compare_pools(gc, oc):
+    n_code = gc.sizes[0]
+    np.testing.assert_array_equal(helpers.pool_bytes(gc.k_codes, n_code), oc.k_codes.reshape(-1).view(np.uint8))
+    np.testing.assert_array_equal(helpers.pool_bytes(gc.v_codes, n_code), oc.v_codes.reshape(-1).view(np.uint8))
+    if oc.mode in ("per_token_head", "kivi"):
+        np.testing.assert_array_equal(helpers.pool_bytes(gc.k_scales, gc.sizes[1]),
+                                      oc.k_scales.reshape(-1).view(np.uint8))
+        np.testing.assert_array_equal(helpers.pool_bytes(gc.v_scales, gc.sizes[2]),
+                                      oc.v_scales.reshape(-1).view(np.uint8))
+    if oc.residual is not None:
+        np.testing.assert_array_equal(helpers.pool_bytes(gc.residual, gc.sizes[3]),
+                                      oc.residual.reshape(-1).view(np.uint8))
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_write_bit_exact(name):
+    w = _workload(name)
+    static = helpers.oracle_static_scales(w)
+    oc = helpers.oracle_cache(w, static)
+    gc = helpers.gpu_cache(w, static=static)
+    torch.cuda.synchronize()
+    _compare_pools(gc, oc)
+    assert gc.read_fault() == (0, 0)
+
+
+def test_fp8_calibration_bit_exact():
+    from oracle import quant
+    from quantized_paged_kv_02_b200 import kvq
+    w = inputs.make("c3", small=True)
+    for x in (w.warmup_k, w.warmup_v):
+        out = torch.empty(x.shape[1], dtype=torch.float32, device="cuda")
+        kvq.kvq_calibrate_fp8_scales(x.cuda(), out)
+        want = quant.fp8_calibrate(helpers.np64(x).astype(np.float32))
+        np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_dequant_matches_oracle(name):
+    w = _workload(name)
+    static = helpers.oracle_static_scales(w)
+    oc = helpers.oracle_cache(w, static)
+    gc = helpers.gpu_cache(w, static=static)
+    used = sorted(set(w.block_tables.cpu().numpy().reshape(-1).tolist()) & set(
+        (w.slot_mapping[w.slot_mapping >= 0].cpu().numpy() // w.spec.block_size).tolist()))
+    ids = torch.tensor(used, dtype=torch.int32, device="cuda")
+    got = gc.dequant(ids).cpu().numpy().astype(np.float64)
+    for i, blk in enumerate(used):
+        want = oc.dequant_block(blk)
+        # code * scale is rounded once to binary32 on the GPU
+        np.testing.assert_allclose(got[i], want, rtol=2.0 ** -24, atol=0)
+
+
+def test_write_edge_cases():
+    """Zero rows (scale 0), a row that saturates, skipped (-1) and out-of-range slots."""
+    from oracle import cache as ocache
+    from quantized_paged_kv_02_b200 import kvq
+    H, D, bs, NB = 2, 128, 16, 4
+    g = torch.Generator().manual_seed(3)
+    k = torch.randn(7, H, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(7, H, D, generator=g).to(torch.bfloat16)
+    k[1] = 0
+    v[2, 0] = 0
+    k[3, 1, 5] = 3.0e38                      # huge outlier: everything else rounds to 0
+    k[4, 0, 0] = -1e-30                      # tiny negative
+    slots = torch.tensor([5, 17, 63, 33, 0, 64, -1], dtype=torch.int32)   # 64 is out of range
+    for cd in ("int8", "fp8"):
+        mode = "per_token_head"
+        oc = ocache.PagedCache(cd, "bf16", mode, NB, bs, H, D)
+        oc.write(helpers.np64(k), helpers.np64(v), slots.numpy())
+        gc = kvq.PagedKVCache(cd, "bf16", mode, NB, bs, H, D)
+        gc.write(k.cuda(), v.cuda(), slots.cuda())
+        torch.cuda.synchronize()
+        n = gc.sizes[0]
+        np.testing.assert_array_equal(helpers.pool_bytes(gc.k_codes, n), oc.k_codes.reshape(-1).view(np.uint8))
+        np.testing.assert_array_equal(helpers.pool_bytes(gc.v_codes, n), oc.v_codes.reshape(-1).view(np.uint8))
+        np.testing.assert_array_equal(helpers.pool_bytes(gc.k_scales, gc.sizes[1]), oc.k_scales.reshape(-1).view(np.uint8))
+        assert gc.read_fault() == (1, 1)       # one bad slot, KVQ_FAULT_SLOT
+    # static FP8 scale with values far beyond 448 * s: saturation, signed zero
+    sk = torch.tensor([0.01, 1e-3]), torch.tensor([0.5, 2.0])
+    oc = ocache.PagedCache("fp8", "bf16", "per_head", NB, bs, H, D,
+                           static_scales=(sk[0].numpy(), sk[1].numpy()))
+    oc.write(helpers.np64(k), helpers.np64(v), slots.numpy())
+    gc = kvq.PagedKVCache("fp8", "bf16", "per_head", NB, bs, H, D,
+                          static_k_scale=sk[0].cuda(), static_v_scale=sk[1].cuda())
+    gc.write(k.cuda(), v.cuda(), slots.cuda())
+    torch.cuda.synchronize()
+    n = gc.sizes[0]
+    np.testing.assert_array_equal(helpers.pool_bytes(gc.k_codes, n), oc.k_codes.reshape(-1).view(np.uint8))
+    np.testing.assert_array_equal(helpers.pool_bytes(gc.v_codes, n), oc.v_codes.reshape(-1).view(np.uint8))
+
+
+def test_int4_bad_run_is_skipped_and_counted():
+    from quantized_paged_kv_02_b200 import kvq
+    H, D = 1, 128
+    k = torch.randn(64, H, D).to(torch.bfloat16).cuda()
+    slots = torch.arange(64, 128, dtype=torch.int32)
+    slots[10] = 200                                   # not one ordered block
+    gc = kvq.PagedKVCache("int4", "bf16", "kivi", 4, 64, H, D, max_seqs=1)
+    gc.write(k, k, slots.cuda())
+    torch.cuda.synchronize()
+    assert np.all(helpers.pool_bytes(gc.k_codes, gc.sizes[0]) == 0x5A)
+    cnt, bits = gc.read_fault()
+    assert cnt == 1 and bits == 16
