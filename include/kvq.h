@@ -234,6 +234,41 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int 
                                 size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Size of the device scratch array used by kvq_decode_attention_noalloc (16 MiB).  Every
+ * GPU that loads the library reserves this much for the life of the process.
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * kvq_decode_attention_noalloc - kvq_decode_attention without a caller workspace.
+ *   (No counterpart in the pages: this entry point exists for callers, not for the method.)
+ *   Some callers cannot hand the library a workspace: a plugin running inside a host
+ *   inference engine that plans all device memory itself and passes the plugin only its
+ *   input and output buffers; a server that gives nearly all of HBM to the KV-cache pool up
+ *   front, so a per-call allocation could fail mid-request; a decode loop that must not call
+ *   the allocator on its hot path because cudaMalloc/cudaFree can synchronize the device.
+ *   This variant takes the same arguments as kvq_decode_attention minus the workspace and
+ *   uses a fixed, file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES instead.  It calls no
+ *   cudaMalloc, cudaFree or other allocating routine.
+ *   - The scratch of the CURRENT device is used: make the device that owns `stream` current.
+ *     The first call on each device looks up the array's device address (set-up); make that
+ *     first call before any stream capture.
+ *   - Returns KVQ_ERR_INVALID_ARG, with nothing enqueued, when this shape needs more scratch
+ *     than KVQ_NOALLOC_SCRATCH_BYTES (kvq_decode_workspace_size tells the need).  Returns
+ *     KVQ_ERR_CUDA if the address look-up fails.
+ *   - All calls on a device share the one array, and it keeps whatever the last call left
+ *     there (nothing in it needs to start at zero).  Calls that overlap on the GPU (for
+ *     example on two streams without ordering between them) race on the array and give
+ *     wrong results: serialize them.
+ */
+kvq_status kvq_decode_attention_noalloc(const kvq_cache_desc* cache, const void* q, int batch,
+                                        int num_q_heads, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* context_lens,
+                                        const int32_t* seq_ids, int max_context,
+                                        float softmax_scale, void* out, int32_t out_dtype,
+                                        cudaStream_t stream);
+
+/*
  * kvq_dequant - debug: expand whole blocks back to float32.
  *   block_ids  int32 [n_blocks], device.
  *   out        float32 [n_blocks][2][H][bs][D], device; index 0 of dim 1 is K, 1 is V.

@@ -24,7 +24,7 @@ STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "K
 FAULT_BITS = {"slot": 1, "block": 2, "context": 4, "seq": 8, "int4_run": 16, "timeout": 32}
 EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
-           "kvq_calibrate_fp8_scales", "kvq_read_device_fault")
+           "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc")
 
 
 class CacheDesc(ctypes.Structure):
@@ -63,6 +63,7 @@ def _load():
         "kvq_dequant": (I, [D, P, I, P, P]),
         "kvq_calibrate_fp8_scales": (I, [P, I, I, I, ctypes.c_int32, P, P]),
         "kvq_read_device_fault": (I, [D, ctypes.POINTER(ctypes.c_int32), I, P]),
+        "kvq_decode_attention_noalloc": (I, [D, P, I, I, P, I, P, P, I, F, P, ctypes.c_int32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -144,6 +145,19 @@ def kvq_decode_attention(desc, q, block_tables, context_lens, max_context, out, 
         _ptr(_i32(context_lens)), _ptr(_i32(seq_ids)), int(max_context), float(softmax_scale),
         _ptr(out), DTYPE[out_dt], _ptr(workspace), ws_bytes, _stream(stream)),
         "kvq_decode_attention")
+    return out
+
+
+def kvq_decode_attention_noalloc(desc, q, block_tables, context_lens, max_context, out,
+                                 seq_ids=None, softmax_scale=0.0, stream=None):
+    """kvq_decode_attention with the library's own fixed device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory when they decode)."""
+    B, Hq, _ = q.shape
+    out_dt = {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[out.dtype]
+    _check(lib.kvq_decode_attention_noalloc(
+        ctypes.byref(desc), _ptr(q), B, Hq, _ptr(_i32(block_tables)), int(block_tables.shape[1]),
+        _ptr(_i32(context_lens)), _ptr(_i32(seq_ids)), int(max_context), float(softmax_scale),
+        _ptr(out), DTYPE[out_dt], _stream(stream)), "kvq_decode_attention_noalloc")
     return out
 
 
