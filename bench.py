@@ -55,6 +55,10 @@ def parse():
     ap.add_argument("--workload", default="c5", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--min-warmup-s", type=float, default=1.0,
+                    help="keep warming up for at least this many seconds")
     return ap.parse_args()
 
 
@@ -249,10 +253,16 @@ def run_oracle_sample(w, static, budget_s=15.0, max_units=64):
 
 
 # ----------------------------------------------------------------------------- ours
-def build_state(workload, device, seed):
+def build_state(workload, device, seed, batch=0):
+    import dataclasses
     import torch
     from quantized_paged_kv_02_b200 import inputs, kvq
-    w = inputs.make(workload, device=device, seed=seed)
+    spec = inputs._spec(workload, False)
+    spec.seed = seed
+    if batch:
+        lens = spec.lens[:1] * batch if spec.lens else None
+        spec = dataclasses.replace(spec, batch=batch, lens=lens)
+    w = inputs.from_spec(spec, device)
     s = w.spec
     static = None
     sk = sv = None
@@ -300,7 +310,7 @@ def main_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
-    w, cache, new, static = build_state(args.workload, device, seed=rank)
+    w, cache, new, static = build_state(args.workload, device, seed=rank, batch=args.batch)
     s = w.spec
     B = s.batch
     out = torch.empty(w.q.shape, dtype=torch.bfloat16, device=device)
@@ -328,7 +338,7 @@ def main_ours(args):
     sampler.start()
     t_w = time.perf_counter()
     i = 0
-    while i < max(3, args.warmup) or time.perf_counter() - t_w < 1.0:
+    while i < max(3, args.warmup) or time.perf_counter() - t_w < args.min_warmup_s:
         flush.zero_()
         write()
         decode()
@@ -373,7 +383,7 @@ def main_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in (h["k"], h["v"], h["slots"], hq, hl))
     d2h = hout.numel() * hout.element_size()
     e2e_ms = []
-    for k in range(E + 3):
+    for k in range(E + 3 if E > 0 else 0):
         flush.zero_()
         a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -389,7 +399,7 @@ def main_ours(args):
         b2.synchronize()
         if k >= 3:
             e2e_ms.append(a.elapsed_time(b2))
-    e2e = statistics.mean(e2e_ms)
+    e2e = statistics.mean(e2e_ms) if e2e_ms else float("nan")
     if world > 1:
         t = torch.tensor([e2e], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -33,26 +33,32 @@
  *  "PagedAttention与KV Cache量化协同工作原理": fixed-size blocks of usually 16 tokens,
  *  each managed on its own, holding INT8/FP8 data that attention dequantizes).
  *
- *  k_codes, v_codes : [NB][H][bs][D] elements of cache_dtype.  For INT4, two codes per
- *                     byte: [NB][H][bs][D/2] bytes, element 2i in the low nibble of byte
- *                     i, element 2i+1 in the high nibble.
- *  k_scales, v_scales by scale_mode:
- *    NONE            : unused (BF16 / FP16 caches).
- *    PER_TOKEN_HEAD  : float32 [NB][H][bs] - one scale per written token and kv head,
- *                      computed at write time ([P-mem] §3.2 动态量化策略).
- *    PER_HEAD        : float32 [H]  - static scale per kv head, supplied by the caller
- *                      ([P-prod] "vLLM：从 FP8 KV Cache 开始试点": per-attention-head).
- *    PER_TENSOR      : float32 [1]  - static scale for the whole cache.
- *    KIVI (INT4)     : k_scales = float16 [NB][H][2][D]: plane 0 the scale and plane 1
- *                      the zero point of each channel over the block's 64 tokens;
- *                      v_scales = float16 [NB][H][bs][D/64][2]: (scale, zero point) of
- *                      each token's 64-channel group ([P-prod] "Key 和 Value 的分布不一定
- *                      相同": keys per channel, values per token).
- *  residual         : INT4 only.  act_dtype [max_seqs][2][H][residual_cap][D]: the
- *                     newest tokens of each sequence kept unquantized ([P-prod] same
- *                     section: a fixed-size higher-precision residual of recent K/V).
- *                     Index 0 of the second dimension is K, 1 is V.  Position p of a
- *                     sequence lives in ring row p % residual_cap.
+ *  pages : [NB][H][record] bytes.  One record holds everything decode reads for one
+ *          (block, kv head), contiguous, so a single copy moves it:
+ *            row_bytes   = D * bits / 8            (bits: 16 BF16/FP16, 8 INT8/FP8, 4 INT4)
+ *            K codes     at offset 0              : [bs][row_bytes]
+ *            V codes     at offset bs*row_bytes   : [bs][row_bytes]
+ *            scales      at offset 2*bs*row_bytes (off_s):
+ *              PER_TOKEN_HEAD : float32 K scale [bs], then float32 V scale [bs]
+ *                               (one scale per written token and kv head, [P-mem] §3.2
+ *                               动态量化策略)
+ *              KIVI (INT4)    : float16 K scale [D], float16 K zero point [D] (each channel
+ *                               over the block's 64 tokens), then float16 V (scale, zero
+ *                               point) [bs][D/64][2] (each token's 64-channel group)
+ *                               ([P-prod] "Key 和 Value 的分布不一定相同": keys per channel,
+ *                               values per token)
+ *              other modes    : nothing
+ *            record      = off_s + scale bytes, rounded up to a multiple of 128 bytes
+ *                          (e.g. INT8, bs 16, D 128: 2048 + 2048 + 128 = 4224 bytes)
+ *          INT4 codes pack two per byte: element 2i in the low nibble of byte i, element
+ *          2i+1 in the high nibble.  Padding bytes at the end of a record are never written.
+ *  k_scales, v_scales : static scales only - PER_HEAD: float32 [H] ([P-prod] "vLLM：从 FP8 KV
+ *          Cache 开始试点": per-attention-head); PER_TENSOR: float32 [1].  Unused otherwise.
+ *  residual : INT4 only.  act_dtype [max_seqs][2][H][residual_cap][D]: the newest tokens of
+ *          each sequence kept unquantized ([P-prod] "Key 和 Value 的分布不一定相同": a
+ *          fixed-size higher-precision residual of recent K/V).  Index 0 of the second
+ *          dimension is K, 1 is V.  Position p of a sequence lives in ring row
+ *          p % residual_cap.
  *
  * Quantizers (what kvq_write stores; x is one activation value widened to float32, and
  * every "/" is an IEEE float32 division rounded to nearest-even)
@@ -149,11 +155,10 @@ typedef struct {
   int32_t residual_cap;
   int32_t max_seqs;
   int32_t reserved0;
-  void* k_codes;
-  void* v_codes;
-  void* k_scales;
-  void* v_scales;
-  void* residual;
+  void* pages;         /* [NB][H][record] */
+  float* k_scales;     /* static scales (PER_HEAD / PER_TENSOR) */
+  float* v_scales;
+  void* residual;      /* INT4 ring */
   int32_t* fault;
 } kvq_cache_desc;
 
@@ -164,15 +169,15 @@ const char* kvq_status_string(kvq_status status);
 int kvq_version(void);
 
 /*
- * Byte sizes the caller must allocate for the pools of a cache described by `cache`
- * (pointer fields are ignored): each of k_codes / v_codes, k_scales, v_scales and
- * residual.  Any out pointer may be NULL.  Host-only; never touches the device.  The
- * sizes follow the layout above ([P-prod] "KV Cache 的基本内存模型": 2 x layers x
+ * Sizes for a cache described by `cache` (pointer fields are ignored): bytes of one
+ * record, of the whole `pages` pool (NB*H records), of each static scale array, and of
+ * the residual ring.  Any out pointer may be NULL.  Host-only; never touches the device.
+ * The sizes follow the layout above ([P-prod] "KV Cache 的基本内存模型": 2 x layers x
  * kv_heads x head_dim x tokens x bytes per value, per layer here, plus the scale,
  * zero-point and residual bytes that make the real gain smaller).
  */
-kvq_status kvq_cache_layout(const kvq_cache_desc* cache, size_t* code_bytes_per_pool,
-                            size_t* k_scale_bytes, size_t* v_scale_bytes,
+kvq_status kvq_cache_layout(const kvq_cache_desc* cache, size_t* record_bytes,
+                            size_t* pages_bytes, size_t* static_scale_bytes,
                             size_t* residual_bytes);
 
 /*

@@ -38,12 +38,19 @@ def _value_of_act_bits(bits, act):
 
 
 class PagedCache:
-    """One layer's K and V pools.
+    """One layer's paged cache.
 
     cache_dtype: "bf16" | "fp16" | "int8" | "fp8" | "int4"
     act_dtype:   "bf16" | "fp16"
     scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "kivi"
     static_scales: (k_scale, v_scale) float32 arrays [H] or [1] for static modes.
+
+    ``pages`` is the byte pool [NB][H][record] of include/kvq.h: per (block, kv head),
+    K codes [bs][row_bytes], V codes [bs][row_bytes], then the per-token scales (float32
+    K [bs], V [bs]) or the KIVI parameters (float16 K scale [D], K zero [D], V (scale,
+    zero) [bs][D/64][2]), padded to a multiple of 128 bytes.  The attributes k_codes,
+    v_codes, k_scales, v_scales are typed views into it (static scales are arrays of
+    their own).
     """
 
     def __init__(self, cache_dtype, act_dtype, scale_mode, num_blocks, block_size,
@@ -55,37 +62,49 @@ class PagedCache:
         NB, bs, H, D = self.NB, self.bs, self.H, self.D
         if cache_dtype in ("bf16", "fp16"):
             assert scale_mode == "none" and cache_dtype == act_dtype
-            code_dt, code_D = np.uint16, D
+            code_dt, row_bytes = np.uint16, 2 * D
         elif cache_dtype == "int8":
-            code_dt, code_D = np.int8, D
+            code_dt, row_bytes = np.int8, D
         elif cache_dtype == "fp8":
-            code_dt, code_D = np.uint8, D
+            code_dt, row_bytes = np.uint8, D
         elif cache_dtype == "int4":
             assert scale_mode == "kivi" and block_size == group_size == 64
-            code_dt, code_D = np.uint8, D // 2
+            code_dt, row_bytes = np.uint8, D // 2
         else:
             raise ValueError(cache_dtype)
-        self.k_codes = self._sentinel((NB, H, bs, code_D), code_dt)
-        self.v_codes = self._sentinel((NB, H, bs, code_D), code_dt)
+        off_s = 2 * bs * row_bytes
+        if scale_mode == "per_token_head":
+            scale_bytes = 8 * bs
+        elif scale_mode == "kivi":
+            scale_bytes = 2 * D * 2 + bs * (D // group_size) * 2 * 2
+        else:
+            scale_bytes = 0
+        self.row_bytes = row_bytes
+        self.record = -(-(off_s + scale_bytes) // 128) * 128
+        self.pages = np.full((NB, H, self.record), SENTINEL, np.uint8)
+        pg = self.pages
+        n_el = row_bytes // np.dtype(code_dt).itemsize
+        self.k_codes = pg[:, :, 0:bs * row_bytes].view(code_dt).reshape(NB, H, bs, n_el)
+        self.v_codes = pg[:, :, bs * row_bytes:off_s].view(code_dt).reshape(NB, H, bs, n_el)
         self.k_scales = self.v_scales = None
         self.residual = None
         if scale_mode == "per_token_head":
-            self.k_scales = self._sentinel((NB, H, bs), np.float32)
-            self.v_scales = self._sentinel((NB, H, bs), np.float32)
+            self.k_scales = pg[:, :, off_s:off_s + 4 * bs].view(np.float32).reshape(NB, H, bs)
+            self.v_scales = pg[:, :, off_s + 4 * bs:off_s + 8 * bs].view(np.float32).reshape(NB, H, bs)
         elif scale_mode in ("per_head", "per_tensor"):
             n = H if scale_mode == "per_head" else 1
             ks, vs = static_scales
             self.k_scales = np.asarray(ks, np.float32).reshape(n).copy()
             self.v_scales = np.asarray(vs, np.float32).reshape(n).copy()
         elif scale_mode == "kivi":
-            self.k_scales = self._sentinel((NB, H, 2, D), np.float16)
-            self.v_scales = self._sentinel((NB, H, bs, D // group_size, 2), np.float16)
-            self.residual = self._sentinel((max_seqs, 2, H, residual_cap, D), np.uint16)
-
-    @staticmethod
-    def _sentinel(shape, dtype):
-        n = int(np.prod(shape)) * np.dtype(dtype).itemsize
-        return np.full(n, SENTINEL, np.uint8).view(dtype).reshape(shape)
+            # K scale [D] then K zero [D] as [NB][H][2][D]; V (scale, zero) [bs][D/G][2]
+            self.k_scales = pg[:, :, off_s:off_s + 4 * D].view(np.float16).reshape(NB, H, 2, D)
+            self.v_scales = pg[:, :, off_s + 4 * D:off_s + scale_bytes].view(np.float16).reshape(
+                NB, H, bs, D // group_size, 2)
+            self.residual = np.full(max_seqs * 2 * H * residual_cap * D * 2, SENTINEL,
+                                    np.uint8).view(np.uint16).reshape(max_seqs, 2, H, residual_cap, D)
+        # the views must alias the pool
+        assert np.shares_memory(self.k_codes, self.pages)
 
     # ------------------------------------------------------------------ scales
     def _static_scale(self, which):

@@ -20,7 +20,8 @@ int code_bits(int cd) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
+// Geometry and record layout of a descriptor (no pointer checks).
+static kvq_status validate_geometry(const kvq_cache_desc* c, Geometry* g) {
   if (c == nullptr) return KVQ_ERR_INVALID_ARG;
   g->cache_dtype = c->cache_dtype;
   g->act_dtype = c->act_dtype;
@@ -38,8 +39,6 @@ kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
   if (c->num_blocks < 1 || c->num_kv_heads < 1 || c->block_size < 1 || c->block_size > 1024)
     return KVQ_ERR_INVALID_ARG;
   if (c->head_dim != 64 && c->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
-  if (c->k_codes == nullptr || c->v_codes == nullptr) return KVQ_ERR_INVALID_ARG;
-  if (!aligned16(c->k_codes) || !aligned16(c->v_codes)) return KVQ_ERR_INVALID_ARG;
   switch (c->cache_dtype) {
     case KVQ_DTYPE_BF16:
     case KVQ_DTYPE_FP16:
@@ -51,18 +50,34 @@ kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
       if (c->scale_mode != KVQ_SCALE_PER_TOKEN_HEAD && c->scale_mode != KVQ_SCALE_PER_HEAD &&
           c->scale_mode != KVQ_SCALE_PER_TENSOR)
         return KVQ_ERR_INVALID_ARG;
-      if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
-      if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
       break;
     case KVQ_DTYPE_INT4:
       if (c->scale_mode != KVQ_SCALE_KIVI) return KVQ_ERR_INVALID_ARG;
       if (c->group_size != 64 || c->block_size != 64) return KVQ_ERR_UNSUPPORTED;
       if (c->residual_len < 0 || c->residual_cap < c->residual_len + c->group_size) return KVQ_ERR_INVALID_ARG;
-      if (c->max_seqs < 1 || c->residual == nullptr || !aligned16(c->residual)) return KVQ_ERR_INVALID_ARG;
-      if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
-      if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
+      if (c->max_seqs < 1) return KVQ_ERR_INVALID_ARG;
       break;
   }
+  g->row_bytes = c->head_dim * code_bits(c->cache_dtype) / 8;
+  g->off_v = g->bs * g->row_bytes;
+  g->off_s = 2 * g->bs * g->row_bytes;
+  g->scale_bytes = 0;
+  if (g->scale_mode == KVQ_SCALE_PER_TOKEN_HEAD) g->scale_bytes = 8 * g->bs;
+  if (g->scale_mode == KVQ_SCALE_KIVI) g->scale_bytes = 4 * g->D + g->bs * (g->D / 64) * 4;
+  g->record = (g->off_s + g->scale_bytes + 127) / 128 * 128;
+  return KVQ_OK;
+}
+
+kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
+  const kvq_status st = validate_geometry(c, g);
+  if (st != KVQ_OK) return st;
+  if (c->pages == nullptr || !aligned16(c->pages)) return KVQ_ERR_INVALID_ARG;
+  if (c->scale_mode == KVQ_SCALE_PER_HEAD || c->scale_mode == KVQ_SCALE_PER_TENSOR) {
+    if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
+  }
+  if (c->cache_dtype == KVQ_DTYPE_INT4 && (c->residual == nullptr || !aligned16(c->residual)))
+    return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
 
@@ -87,32 +102,19 @@ const char* kvq_status_string(kvq_status s) {
 
 int kvq_version(void) { return 100; }
 
-kvq_status kvq_cache_layout(const kvq_cache_desc* c, size_t* code_bytes, size_t* k_scale_bytes,
-                            size_t* v_scale_bytes, size_t* residual_bytes) {
-  if (c == nullptr) return KVQ_ERR_INVALID_ARG;
-  kvq_cache_desc probe = *c;
-  // validate the geometry without requiring real pointers
-  static char dummy[16] __attribute__((aligned(16)));
-  probe.k_codes = probe.v_codes = probe.k_scales = probe.v_scales = probe.residual = dummy;
+kvq_status kvq_cache_layout(const kvq_cache_desc* c, size_t* record_bytes, size_t* pages_bytes,
+                            size_t* static_scale_bytes, size_t* residual_bytes) {
   Geometry g;
-  const kvq_status st = validate_desc(&probe, &g);
+  const kvq_status st = validate_geometry(c, &g);
   if (st != KVQ_OK) return st;
-  const size_t rows = static_cast<size_t>(g.NB) * g.H * g.bs;
-  const size_t cb = rows * g.D * code_bits(g.cache_dtype) / 8;
-  size_t ks = 0, vs = 0, rb = 0;
-  switch (g.scale_mode) {
-    case KVQ_SCALE_PER_TOKEN_HEAD: ks = vs = rows * 4; break;
-    case KVQ_SCALE_PER_HEAD: ks = vs = static_cast<size_t>(g.H) * 4; break;
-    case KVQ_SCALE_PER_TENSOR: ks = vs = 4; break;
-    case KVQ_SCALE_KIVI:
-      ks = static_cast<size_t>(g.NB) * g.H * 2 * g.D * 2;
-      vs = rows * (g.D / 64) * 2 * 2;
-      rb = static_cast<size_t>(g.max_seqs) * 2 * g.H * g.residual_cap * g.D * 2;
-      break;
-  }
-  if (code_bytes) *code_bytes = cb;
-  if (k_scale_bytes) *k_scale_bytes = ks;
-  if (v_scale_bytes) *v_scale_bytes = vs;
+  size_t ss = 0, rb = 0;
+  if (g.scale_mode == KVQ_SCALE_PER_HEAD) ss = static_cast<size_t>(g.H) * 4;
+  if (g.scale_mode == KVQ_SCALE_PER_TENSOR) ss = 4;
+  if (g.scale_mode == KVQ_SCALE_KIVI)
+    rb = static_cast<size_t>(g.max_seqs) * 2 * g.H * g.residual_cap * g.D * 2;
+  if (record_bytes) *record_bytes = static_cast<size_t>(g.record);
+  if (pages_bytes) *pages_bytes = static_cast<size_t>(g.NB) * g.H * g.record;
+  if (static_scale_bytes) *static_scale_bytes = ss;
   if (residual_bytes) *residual_bytes = rb;
   return KVQ_OK;
 }
@@ -136,11 +138,8 @@ kvq_status kvq_write(const kvq_cache_desc* c, const void* k_new, const void* v_n
 kvq_status kvq_decode_workspace_size(const kvq_cache_desc* c, int batch, int num_q_heads,
                                      int max_context, size_t* bytes) {
   if (c == nullptr || bytes == nullptr) return KVQ_ERR_INVALID_ARG;
-  kvq_cache_desc probe = *c;
-  static char dummy[16] __attribute__((aligned(16)));
-  probe.k_codes = probe.v_codes = probe.k_scales = probe.v_scales = probe.residual = dummy;
   Geometry g;
-  kvq_status st = validate_desc(&probe, &g);
+  kvq_status st = validate_geometry(c, &g);
   if (st != KVQ_OK) return st;
   if (batch < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 || max_context < 0)
     return KVQ_ERR_INVALID_ARG;

@@ -36,10 +36,43 @@ __global__ void __launch_bounds__(128) split_reduce_kernel(DecodeParams p, bool 
 
 }  // namespace
 
+// Splits for the tensor-core kernel: one CTA per (sequence, kv head, split); pick the
+// split count whose CTA count fills whole waves of the resident slots (3 CTAs per SM),
+// preferring fewer splits, with at least 256 tokens per split.
+static void plan_mma(const Geometry& g, int batch, int max_context, DecodePlan* p) {
+  const long units = static_cast<long>(batch) * g.H;
+  const long slots = 3L * kNumSMs;
+  const long max_s = std::max(1L, std::min(64L, (static_cast<long>(max_context) + 255) / 256));
+  long best_s = 1;
+  double best = -1.0;
+  for (long S = 1; S <= max_s; ++S) {
+    const long ctas = units * S;
+    const long waves = (ctas + slots - 1) / slots;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    const double score = eff - 0.004 * static_cast<double>(S);
+    if (score > best + 1e-9) { best = score; best_s = S; }
+  }
+  long chunk = (static_cast<long>(max_context) + best_s - 1) / best_s;
+  chunk = std::max(1L, (chunk + g.bs - 1) / g.bs) * g.bs;
+  p->splits = static_cast<int>(std::max(1L, (static_cast<long>(max_context) + chunk - 1) / chunk));
+  p->chunk = static_cast<int>(chunk);
+}
+
 kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_context,
                        DecodePlan* p) {
   p->g = num_q_heads / g.H;
-  p->kernel = 0;
+  p->kernel = mma_supported(g, p->g) ? 1 : 0;
+  if (p->kernel == 1) {
+    p->g_tile = p->g;
+    plan_mma(g, batch, max_context, p);
+    p->ws_bytes = 0;
+    if (p->splits > 1) {
+      const size_t rows = static_cast<size_t>(batch) * num_q_heads * p->splits;
+      const size_t o_bytes = (rows * g.D * sizeof(float) + 255) / 256 * 256;
+      p->ws_bytes = o_bytes + rows * 2 * sizeof(float);
+    }
+    return KVQ_OK;
+  }
   p->g_tile = (p->g % 2 == 0) ? 2 : 1;
   const long units = static_cast<long>(batch) * g.H * (p->g / p->g_tile);
   const int gran = g.cache_dtype == KVQ_DTYPE_INT4 ? 64 : g.bs;
@@ -71,11 +104,14 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.seq_ids = a.seq_ids;
   p.max_blocks = a.max_blocks;
   p.max_context = a.max_context;
-  p.k_codes = a.c->k_codes;
-  p.v_codes = a.c->v_codes;
-  p.k_scales = a.c->k_scales;
-  p.v_scales = a.c->v_scales;
+  p.pages = static_cast<const uint8_t*>(a.c->pages);
+  p.k_static = a.c->k_scales;
+  p.v_static = a.c->v_scales;
   p.residual = a.c->residual;
+  p.record = g.record;
+  p.off_v = g.off_v;
+  p.off_s = g.off_s;
+  p.row_bytes = g.row_bytes;
   p.NB = g.NB;
   p.bs = g.bs;
   p.H = g.H;
@@ -88,6 +124,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.mode = g.scale_mode;
   p.splits = a.plan.splits;
   p.chunk = a.plan.chunk;
+  p.act_fp16 = g.act_dtype == KVQ_DTYPE_FP16;
   p.scale_log2 = a.scale_log2;
   p.out = a.out;
   p.out_dtype = a.out_dtype;
@@ -95,7 +132,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.ws_ml = a.ws_ml;
   p.fault = a.c->fault;
   if (a.batch == 0) return cudaSuccess;
-  cudaError_t e = launch_decode_simt(a, p, s);
+  cudaError_t e = a.plan.kernel == 1 ? launch_decode_mma(a, p, s) : launch_decode_simt(a, p, s);
   if (e != cudaSuccess) return e;
   if (p.splits > 1) {
     split_reduce_kernel<<<a.batch * a.Hq, 128, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);

@@ -12,13 +12,14 @@ struct DecodeParams {
   const int32_t* lens;       // [B]
   const int32_t* seq_ids;    // [B] or null (INT4 ring)
   int max_blocks, max_context;
-  const void* k_codes;
-  const void* v_codes;
-  const void* k_scales;
-  const void* v_scales;
+  const uint8_t* pages;      // [NB][H][record]
+  const float* k_static;     // PER_HEAD / PER_TENSOR scales
+  const float* v_static;
   const void* residual;
+  int record, off_v, off_s, row_bytes;
   int NB, bs, H, Hq, D, g, cap, rlen, max_seqs, mode;
   int splits, chunk;
+  int act_fp16;              // activations (q, ring) are fp16 rather than bf16
   float scale_log2;
   void* out;
   int out_dtype;
@@ -97,5 +98,7 @@ __device__ __forceinline__ void store_partial_or_output(const DecodeParams& p, i
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
+// true when the tensor-core kernel covers this geometry and GQA group size
+bool mma_supported(const Geometry& g, int group);
 
 }  // namespace kvq

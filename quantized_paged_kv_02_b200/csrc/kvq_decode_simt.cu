@@ -107,12 +107,10 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
 #pragma unroll
     for (int i = 0; i < EPL; ++i) acc[h][i] = 0.f;
   }
-  const float* ksc = static_cast<const float*>(p.k_scales);
-  const float* vsc = static_cast<const float*>(p.v_scales);
   float khead = 1.f, vhead = 1.f;
   if constexpr (!kInt4) {
-    if (p.mode == KVQ_SCALE_PER_HEAD) { khead = ksc[kvh]; vhead = vsc[kvh]; }
-    if (p.mode == KVQ_SCALE_PER_TENSOR) { khead = ksc[0]; vhead = vsc[0]; }
+    if (p.mode == KVQ_SCALE_PER_HEAD) { khead = p.k_static[kvh]; vhead = p.v_static[kvh]; }
+    if (p.mode == KVQ_SCALE_PER_TENSOR) { khead = p.k_static[0]; vhead = p.v_static[0]; }
   }
 
   constexpr int BATCH = RPI * U;
@@ -145,24 +143,25 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
       const int blk = block_of(p, b, pos / p.bs);
       if (blk < 0) { valid[j] = false; continue; }
       const int off = pos % p.bs;
-      const long row = (static_cast<long>(blk) * p.H + kvh) * p.bs + off;
-      load_codes<CD>(static_cast<const uint8_t*>(p.k_codes) + row * ROWB + c * CB, kf[j]);
-      load_codes<CD>(static_cast<const uint8_t*>(p.v_codes) + row * ROWB + c * CB, vf[j]);
+      const uint8_t* rec = p.pages + (static_cast<long>(blk) * p.H + kvh) * p.record;
+      load_codes<CD>(rec + off * ROWB + c * CB, kf[j]);
+      load_codes<CD>(rec + p.off_v + off * ROWB + c * CB, vf[j]);
       if constexpr (kInt4) {
-        const __half* ksz = static_cast<const __half*>(p.k_scales) + (static_cast<long>(blk) * p.H + kvh) * 2 * D;
+        const __half* ksz = reinterpret_cast<const __half*>(rec + p.off_s);   // scale [D], zero [D]
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
           const int d = c * EPL + i;
           kf[j][i] = (kf[j][i] - __half2float(ksz[D + d])) * __half2float(ksz[d]);
         }
-        const __half* vsz = static_cast<const __half*>(p.v_scales) + (row * (D / 64) + (c * EPL) / 64) * 2;
+        const __half* vsz = ksz + 2 * D + (off * (D / 64) + (c * EPL) / 64) * 2;
         const float vz = __half2float(vsz[1]);
         vscale[j] = __half2float(vsz[0]);
 #pragma unroll
         for (int i = 0; i < EPL; ++i) vf[j][i] -= vz;
       } else if (p.mode == KVQ_SCALE_PER_TOKEN_HEAD) {
-        kscale[j] = ksc[row];
-        vscale[j] = vsc[row];
+        const float* sc = reinterpret_cast<const float*>(rec + p.off_s);
+        kscale[j] = sc[off];
+        vscale[j] = sc[p.bs + off];
       }
     }
     // scores of the U rows for each head

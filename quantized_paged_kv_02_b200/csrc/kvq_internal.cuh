@@ -59,6 +59,8 @@ struct Geometry {
   int cache_dtype, act_dtype, scale_mode;
   int NB, bs, H, D;
   int group, residual_len, residual_cap, max_seqs;
+  // page record of one (block, kv head): K codes at 0, V codes at off_v, scales at off_s
+  int row_bytes, off_v, off_s, scale_bytes, record;
 };
 
 kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g);

@@ -13,11 +13,11 @@ namespace {
 struct DequantParams {
   const int32_t* ids;
   int n;
-  const void* k_codes;
-  const void* v_codes;
-  const void* k_scales;
-  const void* v_scales;
+  const uint8_t* pages;        // [NB][H][record]
+  const float* k_static;
+  const float* v_static;
   int NB, bs, H, D, cd, act, mode;
+  int record, off_v, off_s, row_bytes;
   float* out;
   int32_t* fault;
 };
@@ -30,44 +30,43 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
     if (threadIdx.x == 0 && kv == 0 && h == 0) record_fault(p.fault, KVQ_FAULT_BLOCK);
     return;
   }
-  const long tile = (static_cast<long>(blk) * p.H + h) * p.bs;   // first row of the tile
+  const uint8_t* rec = p.pages + (static_cast<long>(blk) * p.H + h) * p.record;
+  const uint8_t* codes = rec + (kv ? p.off_v : 0);
   float* out = p.out + (((static_cast<long>(i) * 2 + kv) * p.H + h) * p.bs) * p.D;
-  const void* codes = kv ? p.v_codes : p.k_codes;
-  const void* sc = kv ? p.v_scales : p.k_scales;
   for (int e = threadIdx.x; e < p.bs * p.D; e += blockDim.x) {
     const int t = e / p.D, d = e % p.D;
     float x;
     switch (p.cd) {
       case KVQ_DTYPE_BF16:
-        x = __bfloat162float(static_cast<const __nv_bfloat16*>(codes)[(tile + t) * p.D + d]);
+        x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(codes + t * p.row_bytes)[d]);
         break;
       case KVQ_DTYPE_FP16:
-        x = __half2float(static_cast<const __half*>(codes)[(tile + t) * p.D + d]);
+        x = __half2float(reinterpret_cast<const __half*>(codes + t * p.row_bytes)[d]);
         break;
       case KVQ_DTYPE_INT8:
       case KVQ_DTYPE_FP8_E4M3: {
-        const uint8_t c = static_cast<const uint8_t*>(codes)[(tile + t) * p.D + d];
-        const float* s = static_cast<const float*>(sc);
-        const float sv = p.mode == KVQ_SCALE_PER_TOKEN_HEAD ? s[tile + t]
-                         : p.mode == KVQ_SCALE_PER_HEAD   ? s[h] : s[0];
+        const uint8_t c = codes[t * p.row_bytes + d];
+        const float* s = reinterpret_cast<const float*>(rec + p.off_s) + (kv ? p.bs : 0);
+        const float* st = kv ? p.v_static : p.k_static;
+        const float sv = p.mode == KVQ_SCALE_PER_TOKEN_HEAD ? s[t]
+                         : p.mode == KVQ_SCALE_PER_HEAD   ? st[h] : st[0];
         const float cv = p.cd == KVQ_DTYPE_INT8 ? static_cast<float>(static_cast<int8_t>(c))
                                                 : e4m3_to_float(c);
         x = cv * sv;
         break;
       }
       default: {  // INT4
-        const uint8_t byte = static_cast<const uint8_t*>(codes)[(tile + t) * (p.D / 2) + d / 2];
+        const uint8_t byte = codes[t * p.row_bytes + d / 2];
         const int c = (d & 1) ? (byte >> 4) : (byte & 0xF);
-        const __half* sz = static_cast<const __half*>(sc);
+        const __half* sz = reinterpret_cast<const __half*>(rec + p.off_s);
         float s, z;
         if (kv == 0) {
-          const long base = (static_cast<long>(blk) * p.H + h) * 2 * p.D;
-          s = __half2float(sz[base + d]);
-          z = __half2float(sz[base + p.D + d]);
+          s = __half2float(sz[d]);
+          z = __half2float(sz[p.D + d]);
         } else {
-          const long base = (((static_cast<long>(blk) * p.H + h) * p.bs + t) * (p.D / 64) + d / 64) * 2;
-          s = __half2float(sz[base]);
-          z = __half2float(sz[base + 1]);
+          const __half* v = sz + 2 * p.D + (t * (p.D / 64) + d / 64) * 2;
+          s = __half2float(v[0]);
+          z = __half2float(v[1]);
         }
         x = (static_cast<float>(c) - z) * s;
       }
@@ -100,8 +99,9 @@ __global__ void __launch_bounds__(256) calibrate_kernel(const TA* x, int n, int 
 cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int32_t* ids, int n,
                            float* out, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  DequantParams p{ids, n, c.k_codes, c.v_codes, c.k_scales, c.v_scales,
-                  g.NB, g.bs, g.H, g.D, g.cache_dtype, g.act_dtype, g.scale_mode, out, c.fault};
+  DequantParams p{ids, n, static_cast<const uint8_t*>(c.pages), c.k_scales, c.v_scales,
+                  g.NB, g.bs, g.H, g.D, g.cache_dtype, g.act_dtype, g.scale_mode,
+                  g.record, g.off_v, g.off_s, g.row_bytes, out, c.fault};
   dequant_kernel<<<dim3(n, 2, g.H), 256, 0, s>>>(p);
   return cudaGetLastError();
 }

@@ -22,11 +22,11 @@ struct WriteParams {
   const void* v;
   const int32_t* slots;
   int T;
-  void* k_codes;
-  void* v_codes;
-  float* k_scales;
-  float* v_scales;
+  uint8_t* pages;            // [NB][H][record]
+  const float* k_static;     // PER_HEAD / PER_TENSOR scales
+  const float* v_static;
   int NB, bs, H;
+  int record, off_v, off_s;
   int scale_mode;
   int32_t* fault;
 };
@@ -54,11 +54,11 @@ __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
   const int lane = threadIdx.x & 31;
   const long warp = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int l = lane % LPR;
-  const long row = warp * RPW + lane / LPR;
+  const long task = warp * RPW + lane / LPR;   // (K or V, token, head), head fastest
   const long TH = static_cast<long>(p.T) * p.H;
-  const bool valid = row < 2 * TH;
-  const int kv = valid ? static_cast<int>(row / TH) : 0;
-  const long th = valid ? row % TH : 0;
+  const bool valid = task < 2 * TH;
+  const int kv = valid ? static_cast<int>(task / TH) : 0;
+  const long th = valid ? task % TH : 0;
   const int t = static_cast<int>(th / p.H);
   const int h = static_cast<int>(th % p.H);
   const int slot = valid ? p.slots[t] : -1;
@@ -71,10 +71,14 @@ __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
   if (write) u = *reinterpret_cast<const uint4*>(src);
   const int blk = write ? slot / p.bs : 0;
   const int off = write ? slot % p.bs : 0;
-  const long rowoff = (static_cast<long>(blk) * p.H + h) * p.bs + off;   // [NB][H][bs]
+  // record of (block, head); this row's codes and (per-token) scale inside it
+  uint8_t* rec = p.pages + (static_cast<long>(blk) * p.H + h) * p.record;
+  constexpr int ROWB = (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) ? 2 * D : D;
+  uint8_t* dst_row = rec + (kv ? p.off_v : 0) + off * ROWB;
+  float* scale_slot = reinterpret_cast<float*>(rec + p.off_s) + (kv ? p.bs : 0) + off;
 
   if constexpr (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) {
-    if (write) reinterpret_cast<uint4*>(kv ? p.v_codes : p.k_codes)[(rowoff * D + l * 8) / 8] = u;
+    if (write) *reinterpret_cast<uint4*>(dst_row + l * 16) = u;
   } else {
     float x[8];
     unpack8<TA>(u, x);
@@ -86,9 +90,9 @@ __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       s = div_rn(m, QMax<CD>::v);
-      if (write && l == 0) (kv ? p.v_scales : p.k_scales)[rowoff] = s;
+      if (write && l == 0) *scale_slot = s;
     } else {
-      const float* sp = kv ? p.v_scales : p.k_scales;
+      const float* sp = kv ? p.v_static : p.k_static;
       s = sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0];
     }
     uint32_t w0 = 0, w1 = 0;
@@ -97,10 +101,7 @@ __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
       uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
       if (i < 4) w0 |= c << (8 * i); else w1 |= c << (8 * (i - 4));
     }
-    if (write) {
-      uint8_t* dst = static_cast<uint8_t*>(kv ? p.v_codes : p.k_codes) + rowoff * D + l * 8;
-      *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
-    }
+    if (write) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w0, w1);
   }
 }
 
@@ -112,12 +113,10 @@ struct Int4WriteParams {
   const int32_t* seq_ids;
   const int32_t* positions;
   int T;
-  uint8_t* k_codes;
-  uint8_t* v_codes;
-  __half* k_sz;     // [NB][H][2][D]
-  __half* v_sz;     // [NB][H][64][D/64][2]
+  uint8_t* pages;   // [NB][H][record]: K codes, V codes, K scale [D], K zero [D], V (s,z) [64][D/64][2]
   void* residual;   // [max_seqs][2][H][cap][D]
   int NB, H, cap, max_seqs;
+  int record, off_v, off_s;
   int32_t* fault;
 };
 
@@ -165,6 +164,9 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
       return;
     }
     const long blk = first / G;
+    uint8_t* rec = p.pages + (blk * p.H + h) * p.record;
+    __half* k_sz = reinterpret_cast<__half*>(rec + p.off_s);          // scale [D], zero [D]
+    __half* v_sz = k_sz + 2 * D;                                     // [64][D/64][2]
     for (int kv = 0; kv < 2; ++kv) {
       const TA* src = static_cast<const TA*>(kv ? p.v : p.k);
       // stage the 64 rows of this head as float
@@ -184,9 +186,8 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
           for (int t = 1; t < G; ++t) { lo = fminf(lo, xs[t][d]); hi = fmaxf(hi, xs[t][d]); }
           const Int4Group g = int4_group(lo, hi);
           for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g));
-          __half* sz = p.k_sz + (blk * p.H + h) * 2 * D;
-          sz[d] = g.s16;
-          sz[D + d] = __int2half_rn(g.z);
+          k_sz[d] = g.s16;
+          k_sz[D + d] = __int2half_rn(g.z);
         }
       } else {
         // values: one group per token per 64 channels
@@ -196,14 +197,14 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
           for (int j = 1; j < 64; ++j) { lo = fminf(lo, xs[t][gi * 64 + j]); hi = fmaxf(hi, xs[t][gi * 64 + j]); }
           const Int4Group g = int4_group(lo, hi);
           for (int j = 0; j < 64; ++j) cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g));
-          __half* sz = p.v_sz + (((blk * p.H + h) * G + t) * (D / 64) + gi) * 2;
+          __half* sz = v_sz + (t * (D / 64) + gi) * 2;
           sz[0] = g.s16;
           sz[1] = __int2half_rn(g.z);
         }
       }
       __syncthreads();
       // pack two codes per byte (element 2i low nibble) and store 16 bytes at a time
-      uint8_t* dst = (kv ? p.v_codes : p.k_codes) + (blk * p.H + h) * G * (D / 2);
+      uint8_t* dst = rec + (kv ? p.off_v : 0);
       for (int i = tid; i < G * D / 32; i += blockDim.x) {
         const int t = i / (D / 32), c = i % (D / 32);
         uint32_t w[4];
@@ -275,8 +276,8 @@ cudaError_t dense_by_cd(int cd, const WriteParams& p, cudaStream_t s) {
 
 cudaError_t launch_write_dense(const kvq_cache_desc& c, const Geometry& g, const void* k,
                                const void* v, int T, const int32_t* slots, cudaStream_t s) {
-  WriteParams p{k, v, slots, T, c.k_codes, c.v_codes, static_cast<float*>(c.k_scales),
-                static_cast<float*>(c.v_scales), g.NB, g.bs, g.H, g.scale_mode, c.fault};
+  WriteParams p{k, v, slots, T, static_cast<uint8_t*>(c.pages), c.k_scales, c.v_scales,
+                g.NB, g.bs, g.H, g.record, g.off_v, g.off_s, g.scale_mode, c.fault};
   if (g.act_dtype == KVQ_DTYPE_BF16)
     return g.D == 128 ? dense_by_cd<__nv_bfloat16, 128>(g.cache_dtype, p, s)
                       : dense_by_cd<__nv_bfloat16, 64>(g.cache_dtype, p, s);
@@ -287,10 +288,9 @@ cudaError_t launch_write_dense(const kvq_cache_desc& c, const Geometry& g, const
 cudaError_t launch_write_int4(const kvq_cache_desc& c, const Geometry& g, const void* k,
                               const void* v, int T, const int32_t* slots, const int32_t* seq_ids,
                               const int32_t* positions, cudaStream_t s) {
-  Int4WriteParams p{k, v, slots, seq_ids, positions, T,
-                    static_cast<uint8_t*>(c.k_codes), static_cast<uint8_t*>(c.v_codes),
-                    static_cast<__half*>(c.k_scales), static_cast<__half*>(c.v_scales),
-                    c.residual, g.NB, g.H, g.residual_cap, g.max_seqs, c.fault};
+  Int4WriteParams p{k, v, slots, seq_ids, positions, T, static_cast<uint8_t*>(c.pages),
+                    c.residual, g.NB, g.H, g.residual_cap, g.max_seqs, g.record, g.off_v, g.off_s,
+                    c.fault};
   const dim3 grid((T + 63) / 64, g.H);
   if (grid.x == 0) return cudaSuccess;
   if (g.act_dtype == KVQ_DTYPE_BF16) {

@@ -34,9 +34,9 @@ class CacheDesc(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("group_size", ctypes.c_int32),
                 ("residual_len", ctypes.c_int32), ("residual_cap", ctypes.c_int32),
                 ("max_seqs", ctypes.c_int32), ("reserved0", ctypes.c_int32),
-                ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
-                ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
-                ("residual", ctypes.c_void_p), ("fault", ctypes.c_void_p)]
+                ("pages", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+                ("v_scales", ctypes.c_void_p), ("residual", ctypes.c_void_p),
+                ("fault", ctypes.c_void_p)]
 
 
 class KVQError(RuntimeError):
@@ -116,6 +116,7 @@ def kvq_version():
 
 
 def kvq_cache_layout(desc):
+    """(record bytes, pages pool bytes, static scale bytes, residual bytes)."""
     sizes = [ctypes.c_size_t(0) for _ in range(4)]
     _check(lib.kvq_cache_layout(ctypes.byref(desc), *[ctypes.byref(s) for s in sizes]),
            "kvq_cache_layout")
@@ -184,7 +185,8 @@ def kvq_read_device_fault(desc, reset=True, stream=None):
 
 # ----------------------------------------------------------------------------- holder
 class PagedKVCache:
-    """One layer's K/V pools, allocated with torch in the layout of include/kvq.h."""
+    """One layer's cache, allocated with torch in the layout of include/kvq.h: the page
+    records pool, the static scale arrays (PER_HEAD / PER_TENSOR) and the INT4 ring."""
 
     def __init__(self, cache_dtype, act_dtype, scale_mode, num_blocks, block_size, num_kv_heads,
                  head_dim, device="cuda", group_size=64, residual_len=128, residual_cap=192,
@@ -199,36 +201,30 @@ class PagedKVCache:
         self.num_blocks, self.block_size = num_blocks, block_size
         self.num_kv_heads, self.head_dim = num_kv_heads, head_dim
         self.device = torch.device(device)
-        code_b, ks_b, vs_b, res_b = kvq_cache_layout(d)
-
-        def buf(n):
-            return torch.full((max(n, 16),), fill, dtype=torch.uint8, device=self.device)
-
-        self.k_codes, self.v_codes = buf(code_b), buf(code_b)
-        self.k_scales = buf(ks_b) if ks_b else None
-        self.v_scales = buf(vs_b) if vs_b else None
-        self.residual = buf(res_b) if res_b else None
-        if scale_mode in ("per_head", "per_tensor"):
-            n = num_kv_heads if scale_mode == "per_head" else 1
-            for dst, src in ((self.k_scales, static_k_scale), (self.v_scales, static_v_scale)):
-                if src is not None:
-                    dst[:4 * n].view(torch.float32).copy_(src.reshape(n).to(torch.float32))
+        self.record, pages_b, ss_b, res_b = kvq_cache_layout(d)
+        self.pages = torch.full((pages_b,), fill, dtype=torch.uint8, device=self.device)
+        self.k_scales = self.v_scales = self.residual = None
+        if ss_b:
+            n = ss_b // 4
+            self.k_scales = torch.zeros(max(n, 4), dtype=torch.float32, device=self.device)
+            self.v_scales = torch.zeros(max(n, 4), dtype=torch.float32, device=self.device)
+            if static_k_scale is not None:
+                self.k_scales[:n].copy_(static_k_scale.reshape(n).to(torch.float32))
+            if static_v_scale is not None:
+                self.v_scales[:n].copy_(static_v_scale.reshape(n).to(torch.float32))
+        if res_b:
+            self.residual = torch.full((res_b,), fill, dtype=torch.uint8, device=self.device)
         self.fault = torch.zeros(4, dtype=torch.int32, device=self.device) if fault else None
-        d.k_codes, d.v_codes = self.k_codes.data_ptr(), self.v_codes.data_ptr()
+        d.pages = self.pages.data_ptr()
         d.k_scales = self.k_scales.data_ptr() if self.k_scales is not None else None
         d.v_scales = self.v_scales.data_ptr() if self.v_scales is not None else None
         d.residual = self.residual.data_ptr() if self.residual is not None else None
         d.fault = self.fault.data_ptr() if self.fault is not None else None
-        self.sizes = (code_b, ks_b, vs_b, res_b)
+        self.sizes = (self.record, pages_b, ss_b, res_b)
 
-    # views in the header's shapes (for tests and debugging)
-    def code_view(self, which):
-        t = self.k_codes if which == 0 else self.v_codes
-        D = self.head_dim // 2 if self.cache_dtype == "int4" else self.head_dim
-        dt = {"bf16": torch.bfloat16, "fp16": torch.float16, "int8": torch.int8,
-              "fp8": torch.uint8, "int4": torch.uint8}[self.cache_dtype]
-        n = self.sizes[0]
-        return t[:n].view(dt).view(self.num_blocks, self.num_kv_heads, self.block_size, D)
+    def records(self):
+        """The pages pool as [NB][H][record] bytes."""
+        return self.pages.view(self.num_blocks, self.num_kv_heads, self.record)
 
     def write(self, k_new, v_new, slot_mapping, seq_ids=None, positions=None, stream=None):
         kvq_write(self.desc, k_new, v_new, slot_mapping, seq_ids, positions, stream)

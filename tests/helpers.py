@@ -74,3 +74,11 @@ def gpu_cache(w, device="cuda", static=None, fill=0x5A):
 
 def pool_bytes(t, n):
     return t[:n].cpu().numpy().view(np.uint8)
+
+
+def assert_same_cache(gc, oc):
+    """Byte-for-byte equality of the GPU cache and the oracle cache (pages pool, ring)."""
+    np.testing.assert_array_equal(pool_bytes(gc.pages, gc.sizes[1]), oc.pages.reshape(-1))
+    if oc.residual is not None:
+        np.testing.assert_array_equal(pool_bytes(gc.residual, gc.sizes[3]),
+                                      oc.residual.reshape(-1).view(np.uint8))

@@ -55,13 +55,21 @@ def _desc(kvq, **kw):
 
 
 def test_layout_sizes(lib):
+    """Record = K codes + V codes + per-token scales (or KIVI parameters), padded to 128."""
     from quantized_paged_kv_02_b200 import kvq
-    assert kvq.kvq_cache_layout(_desc(kvq)) == (16 * 4 * 16 * 128, 16 * 4 * 16 * 4, 16 * 4 * 16 * 4, 0)
-    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=4, scale_mode=2)) == (131072, 16, 16, 0)
-    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=0, scale_mode=0)) == (262144, 0, 0, 0)
-    c, ks, vs, r = kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=4, block_size=64))
-    assert c == 16 * 4 * 64 * 64 and ks == 16 * 4 * 2 * 128 * 2
-    assert vs == 16 * 4 * 64 * 2 * 2 * 2 and r == 2 * 2 * 4 * 192 * 128 * 2
+    # INT8 per token, bs 16, D 128: 2048 + 2048 + 128
+    assert kvq.kvq_cache_layout(_desc(kvq)) == (4224, 16 * 4 * 4224, 0, 0)
+    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=4, scale_mode=2)) == (4096, 16 * 4 * 4096, 16, 0)
+    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=4, scale_mode=3)) == (4096, 16 * 4 * 4096, 4, 0)
+    assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=0, scale_mode=0)) == (8192, 16 * 4 * 8192, 0, 0)
+    # INT4 KIVI, bs 64: 4096 + 4096 + (512 K scale/zero + 512 V scale/zero)
+    rec, pg, ss, r = kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=4, block_size=64))
+    assert rec == 9216 and pg == 16 * 4 * 9216 and ss == 0
+    assert r == 2 * 2 * 4 * 192 * 128 * 2
+    # D 64, bs 16: 1024 + 1024 + 128, already a multiple of 128
+    assert kvq.kvq_cache_layout(_desc(kvq, head_dim=64))[0] == 2176
+    # bs 5: 640 + 640 + 40 -> 1408 after padding
+    assert kvq.kvq_cache_layout(_desc(kvq, block_size=5))[0] == 1408
     with pytest.raises(kvq.KVQError):
         kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=4, block_size=16))
 
@@ -85,12 +93,12 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert L.kvq_write(None, null, null, 4, null, null, null, null) == 1
     fake = ctypes.c_void_p(0x1000)
     d2 = _desc(kvq)
-    d2.k_codes = d2.v_codes = d2.k_scales = d2.v_scales = 0x1000
+    d2.pages = 0x1000
     assert L.kvq_write(ctypes.byref(d2), null, null, 4, null, null, null, null) == 1
     assert L.kvq_write(ctypes.byref(d2), fake, fake, -1, fake, null, null, null) == 1
     assert L.kvq_write(ctypes.byref(d2), fake, fake, 0, fake, null, null, null) == 0   # no work
     d3 = _desc(kvq, head_dim=96)
-    d3.k_codes = d3.v_codes = d3.k_scales = d3.v_scales = 0x1000
+    d3.pages = 0x1000
     assert L.kvq_write(ctypes.byref(d3), fake, fake, 1, fake, null, null, null) == 2   # unsupported
     # decode: bad head count, bad out dtype, missing workspace
     assert L.kvq_decode_attention(ctypes.byref(d2), fake, 2, 6, fake, 4, fake, null, 64, 0.0,
@@ -103,10 +111,14 @@ def test_invalid_arguments_rejected_before_launch(lib):
                                   ctypes.c_float(float("nan")), fake, 2, null, 0, null) == 1
     # misaligned pool
     d4 = _desc(kvq)
-    d4.k_codes, d4.v_codes, d4.k_scales, d4.v_scales = 0x1001, 0x1000, 0x1000, 0x1000
+    d4.pages = 0x1001
     assert L.kvq_write(ctypes.byref(d4), fake, fake, 1, fake, null, null, null) == 1
     # mixed passthrough (bf16 cache, fp16 activations) is unsupported
     d5 = _desc(kvq, cache_dtype=0, act_dtype=1, scale_mode=0)
-    d5.k_codes = d5.v_codes = 0x1000
+    d5.pages = 0x1000
+    # static scales are required for per-head modes
+    d6 = _desc(kvq, cache_dtype=4, scale_mode=2)
+    d6.pages = 0x1000
+    assert L.kvq_write(ctypes.byref(d6), fake, fake, 1, fake, null, null, null) == 1
     assert L.kvq_write(ctypes.byref(d5), fake, fake, 1, fake, null, null, null) == 2
     assert kvq.kvq_status_string(2) == "KVQ_ERR_UNSUPPORTED"

@@ -25,17 +25,7 @@ def _workload(name):
 
 
 def _compare_pools(gc, oc):
-    n_code = gc.sizes[0]
-    np.testing.assert_array_equal(helpers.pool_bytes(gc.k_codes, n_code), oc.k_codes.reshape(-1).view(np.uint8))
-    np.testing.assert_array_equal(helpers.pool_bytes(gc.v_codes, n_code), oc.v_codes.reshape(-1).view(np.uint8))
-    if oc.mode in ("per_token_head", "kivi"):
-        np.testing.assert_array_equal(helpers.pool_bytes(gc.k_scales, gc.sizes[1]),
-                                      oc.k_scales.reshape(-1).view(np.uint8))
-        np.testing.assert_array_equal(helpers.pool_bytes(gc.v_scales, gc.sizes[2]),
-                                      oc.v_scales.reshape(-1).view(np.uint8))
-    if oc.residual is not None:
-        np.testing.assert_array_equal(helpers.pool_bytes(gc.residual, gc.sizes[3]),
-                                      oc.residual.reshape(-1).view(np.uint8))
+    helpers.assert_same_cache(gc, oc)
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -96,10 +86,7 @@ def test_write_edge_cases():
         gc = kvq.PagedKVCache(cd, "bf16", mode, NB, bs, H, D)
         gc.write(k.cuda(), v.cuda(), slots.cuda())
         torch.cuda.synchronize()
-        n = gc.sizes[0]
-        np.testing.assert_array_equal(helpers.pool_bytes(gc.k_codes, n), oc.k_codes.reshape(-1).view(np.uint8))
-        np.testing.assert_array_equal(helpers.pool_bytes(gc.v_codes, n), oc.v_codes.reshape(-1).view(np.uint8))
-        np.testing.assert_array_equal(helpers.pool_bytes(gc.k_scales, gc.sizes[1]), oc.k_scales.reshape(-1).view(np.uint8))
+        helpers.assert_same_cache(gc, oc)
         assert gc.read_fault() == (1, 1)       # one bad slot, KVQ_FAULT_SLOT
     # static FP8 scale with values far beyond 448 * s: saturation, signed zero
     sk = torch.tensor([0.01, 1e-3]), torch.tensor([0.5, 2.0])
@@ -110,9 +97,7 @@ def test_write_edge_cases():
                           static_k_scale=sk[0].cuda(), static_v_scale=sk[1].cuda())
     gc.write(k.cuda(), v.cuda(), slots.cuda())
     torch.cuda.synchronize()
-    n = gc.sizes[0]
-    np.testing.assert_array_equal(helpers.pool_bytes(gc.k_codes, n), oc.k_codes.reshape(-1).view(np.uint8))
-    np.testing.assert_array_equal(helpers.pool_bytes(gc.v_codes, n), oc.v_codes.reshape(-1).view(np.uint8))
+    helpers.assert_same_cache(gc, oc)
 
 
 def test_int4_bad_run_is_skipped_and_counted():
@@ -124,6 +109,6 @@ def test_int4_bad_run_is_skipped_and_counted():
     gc = kvq.PagedKVCache("int4", "bf16", "kivi", 4, 64, H, D, max_seqs=1)
     gc.write(k, k, slots.cuda())
     torch.cuda.synchronize()
-    assert np.all(helpers.pool_bytes(gc.k_codes, gc.sizes[0]) == 0x5A)
+    assert np.all(helpers.pool_bytes(gc.pages, gc.sizes[1]) == 0x5A)
     cnt, bits = gc.read_fault()
     assert cnt == 1 and bits == 16
