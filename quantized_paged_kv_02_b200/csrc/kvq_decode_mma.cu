@@ -38,6 +38,7 @@ namespace {
 constexpr int kConsumers = 4;
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kD = 128;
+constexpr float kRescale = 8.f;   // log2 headroom before the running max is re-reduced
 
 template <int CD> struct Code;
 template <> struct Code<KVQ_DTYPE_INT8> { static constexpr int B = 1; static constexpr bool kBf16 = false; };
@@ -169,7 +170,8 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     const int g = p.g;
     // Q^T fragments for head n = r: thread j covers d in [32j, 32j+32); k-step kc uses
     // d = 32j + 4kc + {0,1} (b0) and {2,3} (b1), the same d <-> k map the K codes use.
-    uint32_t qb[8][2];
+    uint32_t qb[8][2];              // fp16/bf16 Q fragments (FP8, BF16, FP16 caches)
+    uint32_t qt[3][4][2];           // int8 Q terms (INT8 caches), see below
     float qscale = p.scale_log2;
     {
       float qv[32];
@@ -191,7 +193,45 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
 #pragma unroll
         for (int e = 0; e < 32; ++e) qv[e] = 0.f;
       }
-      if constexpr (kBf16) {
+      if constexpr (CD == KVQ_DTYPE_INT8) {
+        // q = sq * (Q0 + Q1/128 + Q2/16384) with int8 terms, sq = max|q| / 127 over the
+        // group: |Q1|, |Q2| <= 64 and the error is about max|q| * 2^-22, so K . Q runs on
+        // the integer tensor cores (K codes used as they are, int32 sums exact).
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(qv[e]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float sq = amax / 127.f;
+        const float inv = amax > 0.f ? 127.f / amax : 0.f;
+        uint32_t w[3][8];
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[t][e] = 0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = qv[e];
+          const int q0 = max(-127, min(127, __float2int_rn(x * inv)));
+          const float r1 = fmaf(-static_cast<float>(q0), sq, x);
+          const int q1 = max(-127, min(127, __float2int_rn(r1 * inv * 128.f)));
+          const float r2 = fmaf(-static_cast<float>(q1), sq * (1.f / 128.f), r1);
+          const int q2 = max(-127, min(127, __float2int_rn(r2 * inv * 16384.f)));
+          const int sh = 8 * (e & 3);
+          w[0][e >> 2] |= static_cast<uint32_t>(q0 & 0xFF) << sh;
+          w[1][e >> 2] |= static_cast<uint32_t>(q1 & 0xFF) << sh;
+          w[2][e >> 2] |= static_cast<uint32_t>(q2 & 0xFF) << sh;
+        }
+        // k-step kc: b0 <- elements 8kc..8kc+3, b1 <- 8kc+4..8kc+7 of [32j, 32j+32)
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            qt[t][kc][0] = w[t][2 * kc];
+            qt[t][kc][1] = w[t][2 * kc + 1];
+          }
+        qscale *= sq;
+      } else if constexpr (kBf16) {
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
           qb[kc][0] = pack_bf16x2(qv[4 * kc], qv[4 * kc + 1]);
@@ -245,6 +285,7 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     const int sk0 = swzb(L::OFF_S + 4 * r), sk1 = swzb(L::OFF_S + 4 * (r + 8));
     const int sv0 = swzb(L::OFF_S + 4 * BS + 4 * r), sv1 = swzb(L::OFF_S + 4 * BS + 4 * (r + 8));
 
+    float vlim = 0.f, vinv = 0.f;   // 2^(ev+1) and 2^-ev of the V normaliser (PT only)
     for (int i = warp; i < npages; i += kConsumers) {
       const int s = i % kStages;
       // all lanes wait; the decision is made warp-uniform before any shuffle below
@@ -252,47 +293,73 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         if (lane == 0) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
         break;
       }
+      const uint8_t* st = tiles + s * STAGE;
       const bool pvalid = valid[s] != 0;
-      const uint8_t* kt = tiles + s * STAGE;
-      const uint8_t* vt = kt;                                    // V offsets include OFF_V
       const int pos0 = t0 + i * BS;
       const bool full_page = pvalid && pos0 + BS <= t1;          // warp-uniform
-      // ------------------------------------------------ S^T = K Q^T (two accumulator chains)
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (Code<CD>::B == 1) {
-        uint32_t w0[8], w1[8];
+      // ------------------------------------------------ stage -> registers, then hand the
+      // stage back to the producer before any math, so the ring refills during compute
+      uint4 kw[2][KCH], vw[4][VCH];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 a = lds128(kt + koff[0][c]);
-          const uint4 b2 = lds128(kt + koff[1][c]);
-          w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
-          w1[4 * c] = b2.x; w1[4 * c + 1] = b2.y; w1[4 * c + 2] = b2.z; w1[4 * c + 3] = b2.w;
+      for (int c = 0; c < KCH; ++c) {
+        kw[0][c] = lds128(st + koff[0][c]);
+        kw[1][c] = lds128(st + koff[1][c]);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int c = 0; c < VCH; ++c) vw[t][c] = lds128(st + voff[t][c]);
+      float ks0 = 1.f, ks1 = 1.f, vs0 = 0.f, vs1 = 0.f;
+      if constexpr (PT) {
+        ks0 = *reinterpret_cast<const float*>(st + sk0);
+        ks1 = *reinterpret_cast<const float*>(st + sk1);
+        vs0 = *reinterpret_cast<const float*>(st + sv0);
+        vs1 = *reinterpret_cast<const float*>(st + sv1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+
+      // ------------------------------------------------ S^T = K Q^T
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (CD == KVQ_DTYPE_INT8) {
+        // integer tensor cores: m16n8k32, k-step kc takes words 2kc (a0/a1) and 2kc+1
+        // (a2/a3) of rows r and r+8, i.e. d = 32j + 8kc + 0..7, matching the Q terms
+        const uint32_t w0[8] = {kw[0][0].x, kw[0][0].y, kw[0][0].z, kw[0][0].w,
+                                kw[0][1].x, kw[0][1].y, kw[0][1].z, kw[0][1].w};
+        const uint32_t w1[8] = {kw[1][0].x, kw[1][0].y, kw[1][0].z, kw[1][0].w,
+                                kw[1][1].x, kw[1][1].y, kw[1][1].z, kw[1][1].w};
+        int i0[4] = {0, 0, 0, 0}, i1[4] = {0, 0, 0, 0}, i2[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int kc = 0; kc < 4; ++kc) {
+          const uint32_t a[4] = {w0[2 * kc], w1[2 * kc], w0[2 * kc + 1], w1[2 * kc + 1]};
+          mma_s8(i0, a, qt[0][kc]);
+          mma_s8(i1, a, qt[1][kc]);
+          mma_s8(i2, a, qt[2][kc]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sa[e] = fmaf(fmaf(static_cast<float>(i2[e]), 1.f / 128.f, static_cast<float>(i1[e])), 1.f / 128.f,
+                       static_cast<float>(i0[e]));
+      } else if constexpr (Code<CD>::B == 1) {
+        const uint32_t w0[8] = {kw[0][0].x, kw[0][0].y, kw[0][0].z, kw[0][0].w,
+                                kw[0][1].x, kw[0][1].y, kw[0][1].z, kw[0][1].w};
+        const uint32_t w1[8] = {kw[1][0].x, kw[1][0].y, kw[1][0].z, kw[1][0].w,
+                                kw[1][1].x, kw[1][1].y, kw[1][1].z, kw[1][1].w};
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
           uint32_t a[4];
-          if constexpr (CD == KVQ_DTYPE_INT8) {
-            const uint32_t x0 = w0[kc] ^ 0x80808080u, x1 = w1[kc] ^ 0x80808080u;
-            a[0] = i8x2_to_f16x2(x0, kLoPair);
-            a[1] = i8x2_to_f16x2(x1, kLoPair);
-            a[2] = i8x2_to_f16x2(x0, kHiPair);
-            a[3] = i8x2_to_f16x2(x1, kHiPair);
-          } else {
-            a[0] = e4m3x2_to_f16x2(w0[kc] & 0xFFFFu);
-            a[1] = e4m3x2_to_f16x2(w1[kc] & 0xFFFFu);
-            a[2] = e4m3x2_to_f16x2(w0[kc] >> 16);
-            a[3] = e4m3x2_to_f16x2(w1[kc] >> 16);
-          }
+          a[0] = e4m3x2_to_f16x2(w0[kc] & 0xFFFFu);
+          a[1] = e4m3x2_to_f16x2(w1[kc] & 0xFFFFu);
+          a[2] = e4m3x2_to_f16x2(w0[kc] >> 16);
+          a[3] = e4m3x2_to_f16x2(w1[kc] >> 16);
           mma_f16((kc & 1) ? sb : sa, a, qb[kc]);
         }
       } else {
         // 16-bit codes: elements 32j + 4kc + {0,1} / {2,3} are whole words
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          const uint4 a0 = lds128(kt + koff[0][h]);
-          const uint4 c0 = lds128(kt + koff[1][h]);
-          const uint32_t w0[4] = {a0.x, a0.y, a0.z, a0.w};
-          const uint32_t w1[4] = {c0.x, c0.y, c0.z, c0.w};
+          const uint32_t w0[4] = {kw[0][h].x, kw[0][h].y, kw[0][h].z, kw[0][h].w};
+          const uint32_t w1[4] = {kw[1][h].x, kw[1][h].y, kw[1][h].z, kw[1][h].w};
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const uint32_t a[4] = {w0[2 * e], w1[2 * e], w0[2 * e + 1], w1[2 * e + 1]};
@@ -302,37 +369,35 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         }
       }
       // ------------------------------------------------ scale, mask, online softmax
-      float f0 = qscale, f1 = qscale;
-      if constexpr (PT) {
-        f0 *= *reinterpret_cast<const float*>(kt + sk0);
-        f1 *= *reinterpret_cast<const float*>(kt + sk1);
-      }
       // (token r, head 2j), (r, 2j+1), (r+8, 2j), (r+8, 2j+1)
+      const float f0 = qscale * ks0, f1 = qscale * ks1;
       float s00 = (sa[0] + sb[0]) * f0, s01 = (sa[1] + sb[1]) * f0;
       float s10 = (sa[2] + sb[2]) * f1, s11 = (sa[3] + sb[3]) * f1;
-      bool v0 = true, v1 = true;
       if (!full_page) {
-        v0 = pvalid && pos0 + r < t1;
-        v1 = pvalid && pos0 + r + 8 < t1;
-        if (!v0) s00 = s01 = -INFINITY;
-        if (!v1) s10 = s11 = -INFINITY;
+        const bool v0 = pvalid && pos0 + r < t1;
+        const bool v1 = pvalid && pos0 + r + 8 < t1;
+        if (!v0) { s00 = s01 = -INFINITY; vs0 = 0.f; }
+        if (!v1) { s10 = s11 = -INFINITY; vs1 = 0.f; }
       }
-      float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
+      // The running max only needs to move when a score exceeds it by more than 2^8 in
+      // weight (one vote); otherwise P <= 2^8 stays well inside fp16 and the softmax is
+      // unchanged (the same reference max is used for numerator and denominator).
+      const bool grow = s00 > m[0] + kRescale || s10 > m[0] + kRescale ||
+                        s01 > m[1] + kRescale || s11 > m[1] + kRescale;
+      if (__any_sync(0xffffffffu, grow)) {
+        float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, off));
-        tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, off));
-      }
-      const float mn0 = fmaxf(m[0], tm0), mn1 = fmaxf(m[1], tm1);
-      const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float c0 = ex2(m[0] - base0), c1 = ex2(m[1] - base1);   // 0 while nothing was seen
-      m[0] = mn0;
-      m[1] = mn1;
-      const float p00 = ex2(s00 - base0), p10 = ex2(s10 - base0);
-      const float p01 = ex2(s01 - base1), p11 = ex2(s11 - base1);
-      l[0] = l[0] * c0 + p00 + p10;
-      l[1] = l[1] * c1 + p01 + p11;
-      if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
+        for (int off = 4; off < 32; off <<= 1) {
+          tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, off));
+          tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, off));
+        }
+        const float mn0 = fmaxf(m[0], tm0), mn1 = fmaxf(m[1], tm1);
+        const float c0 = m[0] == -INFINITY ? 0.f : ex2(m[0] - mn0);
+        const float c1 = m[1] == -INFINITY ? 0.f : ex2(m[1] - mn1);
+        m[0] = mn0;
+        m[1] = mn1;
+        l[0] *= c0;
+        l[1] *= c1;
 #pragma unroll
         for (int md = 0; md < 8; ++md) {
           o[md][0] *= c0;
@@ -341,31 +406,37 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
           o[md][3] *= c1;
         }
       }
-      // fold the per-token V scale into P, normalised by 2^ev (a power of two tracking
-      // the largest V scale seen, so P stays inside fp16's range)
+      const float base0 = m[0] == -INFINITY ? 0.f : m[0], base1 = m[1] == -INFINITY ? 0.f : m[1];
+      const float p00 = ex2(s00 - base0), p10 = ex2(s10 - base0);
+      const float p01 = ex2(s01 - base1), p11 = ex2(s11 - base1);
+      l[0] += p00 + p10;
+      l[1] += p01 + p11;
+      // fold the per-token V scale into P, normalised by 2^ev (a power of two that only
+      // grows, re-reduced when some token's scale reaches 2^(ev+1))
       float w0 = 1.f, w1 = 1.f;
       if constexpr (PT) {
-        const float vs0 = v0 ? *reinterpret_cast<const float*>(kt + sv0) : 0.f;
-        const float vs1 = v1 ? *reinterpret_cast<const float*>(kt + sv1) : 0.f;
-        float vm = fmaxf(vs0, vs1);
+        if (__any_sync(0xffffffffu, vs0 >= vlim || vs1 >= vlim)) {
+          float vm = fmaxf(vs0, vs1);
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-        if (vm > 0.f) {
-          const int e = exponent_of(vm);
-          if (e > ev) {
-            if (ev != INT_MIN) {
-              const float down = pow2i(ev - e);
+          for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+          if (vm > 0.f) {
+            const int e = exponent_of(vm);
+            if (e > ev) {
+              if (ev != INT_MIN) {
+                const float down = pow2i(ev - e);
 #pragma unroll
-              for (int md = 0; md < 8; ++md)
+                for (int md = 0; md < 8; ++md)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) o[md][c] *= down;
+                  for (int c = 0; c < 4; ++c) o[md][c] *= down;
+              }
+              ev = e;
+              vlim = pow2i(ev + 1);
+              vinv = pow2i(-ev);
             }
-            ev = e;
           }
         }
-        const float inv = ev == INT_MIN ? 0.f : pow2i(-ev);
-        w0 = vs0 * inv;
-        w1 = vs1 * inv;
+        w0 = vs0 * vinv;
+        w1 = vs1 * vinv;
       }
       const float q00 = p00 * w0, q01 = p01 * w0, q10 = p10 * w1, q11 = p11 * w1;
       // ------------------------------------------------ P^T fragments: hi + lo halves,
@@ -396,26 +467,22 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       // ------------------------------------------------ O^T += V^T P^T
       // m-tile md, rows r / r+8 <-> d = 16r + 2md / +1; k = tokens 2j, 2j+1, 2j+8, 2j+9.
       // Rows of invalid tokens carry P = 0, but their codes may be anything: zero them.
-      bool va = true, vb = true, vc = true, vd = true;
       if (!full_page) {
-        va = pvalid && pos0 + 2 * j < t1;
-        vb = pvalid && pos0 + 2 * j + 1 < t1;
-        vc = pvalid && pos0 + 2 * j + 8 < t1;
-        vd = pvalid && pos0 + 2 * j + 9 < t1;
+        const bool va = pvalid && pos0 + 2 * j < t1, vb = pvalid && pos0 + 2 * j + 1 < t1;
+        const bool vc = pvalid && pos0 + 2 * j + 8 < t1, vd = pvalid && pos0 + 2 * j + 9 < t1;
+#pragma unroll
+        for (int c = 0; c < VCH; ++c) {
+          if (!va) vw[0][c] = make_uint4(0, 0, 0, 0);
+          if (!vb) vw[1][c] = make_uint4(0, 0, 0, 0);
+          if (!vc) vw[2][c] = make_uint4(0, 0, 0, 0);
+          if (!vd) vw[3][c] = make_uint4(0, 0, 0, 0);
+        }
       }
       if constexpr (Code<CD>::B == 1) {
-        uint4 u0 = lds128(vt + voff[0][0]);
-        uint4 u1 = lds128(vt + voff[1][0]);
-        uint4 u2 = lds128(vt + voff[2][0]);
-        uint4 u3 = lds128(vt + voff[3][0]);
-        if (!full_page) {
-          if (!va) u0 = make_uint4(0, 0, 0, 0);
-          if (!vb) u1 = make_uint4(0, 0, 0, 0);
-          if (!vc) u2 = make_uint4(0, 0, 0, 0);
-          if (!vd) u3 = make_uint4(0, 0, 0, 0);
-        }
-        const uint32_t x0[4] = {u0.x, u0.y, u0.z, u0.w}, x1[4] = {u1.x, u1.y, u1.z, u1.w};
-        const uint32_t x2[4] = {u2.x, u2.y, u2.z, u2.w}, x3[4] = {u3.x, u3.y, u3.z, u3.w};
+        const uint32_t x0[4] = {vw[0][0].x, vw[0][0].y, vw[0][0].z, vw[0][0].w};
+        const uint32_t x1[4] = {vw[1][0].x, vw[1][0].y, vw[1][0].z, vw[1][0].w};
+        const uint32_t x2[4] = {vw[2][0].x, vw[2][0].y, vw[2][0].z, vw[2][0].w};
+        const uint32_t x3[4] = {vw[3][0].x, vw[3][0].y, vw[3][0].z, vw[3][0].w};
 #pragma unroll
         for (int md = 0; md < 8; ++md) {
           const int w = md >> 1;
@@ -442,23 +509,10 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         uint32_t x0[8], x1[8], x2[8], x3[8];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint4 u0 = lds128(vt + voff[0][h]);
-          const uint4 u1 = lds128(vt + voff[1][h]);
-          const uint4 u2 = lds128(vt + voff[2][h]);
-          const uint4 u3 = lds128(vt + voff[3][h]);
-          x0[4 * h] = u0.x; x0[4 * h + 1] = u0.y; x0[4 * h + 2] = u0.z; x0[4 * h + 3] = u0.w;
-          x1[4 * h] = u1.x; x1[4 * h + 1] = u1.y; x1[4 * h + 2] = u1.z; x1[4 * h + 3] = u1.w;
-          x2[4 * h] = u2.x; x2[4 * h + 1] = u2.y; x2[4 * h + 2] = u2.z; x2[4 * h + 3] = u2.w;
-          x3[4 * h] = u3.x; x3[4 * h + 1] = u3.y; x3[4 * h + 2] = u3.z; x3[4 * h + 3] = u3.w;
-        }
-        if (!full_page) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (!va) x0[e] = 0;
-            if (!vb) x1[e] = 0;
-            if (!vc) x2[e] = 0;
-            if (!vd) x3[e] = 0;
-          }
+          x0[4 * h] = vw[0][h].x; x0[4 * h + 1] = vw[0][h].y; x0[4 * h + 2] = vw[0][h].z; x0[4 * h + 3] = vw[0][h].w;
+          x1[4 * h] = vw[1][h].x; x1[4 * h + 1] = vw[1][h].y; x1[4 * h + 2] = vw[1][h].z; x1[4 * h + 3] = vw[1][h].w;
+          x2[4 * h] = vw[2][h].x; x2[4 * h + 1] = vw[2][h].y; x2[4 * h + 2] = vw[2][h].z; x2[4 * h + 3] = vw[2][h].w;
+          x3[4 * h] = vw[3][h].x; x3[4 * h + 1] = vw[3][h].y; x3[4 * h + 2] = vw[3][h].z; x3[4 * h + 3] = vw[3][h].w;
         }
 #pragma unroll
         for (int md = 0; md < 8; ++md) {
@@ -474,8 +528,6 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
     }
     // complete the row sums: lanes with the same j hold the same heads
 #pragma unroll
