@@ -16,19 +16,28 @@ __global__ void __launch_bounds__(128) split_reduce_kernel(DecodeParams p, bool 
   const int row = blockIdx.x;                 // b * Hq + hq
   const int b = row / p.Hq;
   const SeqInfo si = seq_info(p, b, int4);
-  const int S = (si.n + p.chunk - 1) / p.chunk;
+  // splits that hold work: the token splits covering [0, n), or, when the INT4 ring has
+  // a split of its own, the block splits covering [0, qb) plus the ring split
+  const int S = (p.ring_split >= 0 ? si.qb + p.chunk - 1 : si.n + p.chunk - 1) / p.chunk;
+  const bool ring = p.ring_split >= 0 && si.n > si.qb;
   const float* ml = p.ws_ml + static_cast<long>(row) * p.splits * 2;
   const float* o = p.ws_o + static_cast<long>(row) * p.splits * p.D;
+  auto slot = [&](int k) { return k < S ? k : p.ring_split; };
+  const int K = S + (ring ? 1 : 0);
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[2 * s]);
+  for (int k = 0; k < K; ++k) M = fmaxf(M, ml[2 * slot(k)]);
   float L = 0.f;
-  for (int s = 0; s < S; ++s) L += (M == -INFINITY) ? 0.f : ml[2 * s + 1] * exp2f(ml[2 * s] - M);
+  for (int k = 0; k < K; ++k) {
+    const float mk = ml[2 * slot(k)];
+    L += (M == -INFINITY || mk == -INFINITY) ? 0.f : ml[2 * slot(k) + 1] * exp2f(mk - M);
+  }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
     float acc = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float w = (M == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);
-      acc = fmaf(o[static_cast<long>(s) * p.D + d], w, acc);
+    for (int k = 0; k < K; ++k) {
+      const float mk = ml[2 * slot(k)];
+      const float w = (M == -INFINITY || mk == -INFINITY) ? 0.f : exp2f(mk - M);
+      acc = fmaf(o[static_cast<long>(slot(k)) * p.D + d], w, acc);
     }
     store_out(p, static_cast<long>(row) * p.D + d, acc * inv);
   }
@@ -62,6 +71,21 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
                        DecodePlan* p) {
   p->g = num_q_heads / g.H;
   p->kernel = mma_supported(g, p->g) ? 1 : 0;
+  if (int4_mma_supported(g, p->g)) {
+    // INT4 blocks on tensor cores: splits over the quantized prefix (64-token blocks)
+    // plus one split for the residual ring, computed by the CUDA-core kernel
+    p->kernel = 2;
+    p->g_tile = p->g;
+    const int max_qb = 64 * (std::max(max_context - g.residual_len, 0) / 64);
+    Geometry gg = g;
+    gg.bs = 64;
+    plan_mma(gg, batch, std::max(max_qb, 64), p);
+    p->splits += 1;                              // the ring
+    const size_t rows = static_cast<size_t>(batch) * num_q_heads * p->splits;
+    const size_t o_bytes = (rows * g.D * sizeof(float) + 255) / 256 * 256;
+    p->ws_bytes = o_bytes + rows * 2 * sizeof(float);
+    return KVQ_OK;
+  }
   if (p->kernel == 1) {
     p->g_tile = p->g;
     plan_mma(g, batch, max_context, p);
@@ -124,6 +148,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.mode = g.scale_mode;
   p.splits = a.plan.splits;
   p.chunk = a.plan.chunk;
+  p.ring_split = a.plan.kernel == 2 ? a.plan.splits - 1 : -1;
   p.act_fp16 = g.act_dtype == KVQ_DTYPE_FP16;
   p.scale_log2 = a.scale_log2;
   p.out = a.out;
@@ -132,7 +157,13 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.ws_ml = a.ws_ml;
   p.fault = a.c->fault;
   if (a.batch == 0) return cudaSuccess;
-  cudaError_t e = a.plan.kernel == 1 ? launch_decode_mma(a, p, s) : launch_decode_simt(a, p, s);
+  cudaError_t e;
+  if (a.plan.kernel == 2) {
+    e = launch_decode_int4(a, p, s);                 // block splits
+    if (e == cudaSuccess) e = launch_decode_simt(a, p, s);   // ring split
+  } else {
+    e = a.plan.kernel == 1 ? launch_decode_mma(a, p, s) : launch_decode_simt(a, p, s);
+  }
   if (e != cudaSuccess) return e;
   if (p.splits > 1) {
     split_reduce_kernel<<<a.batch * a.Hq, 128, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);

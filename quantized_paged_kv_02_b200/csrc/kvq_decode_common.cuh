@@ -2,6 +2,8 @@
 // and the epilogue that writes either a split partial or the final output row.
 #pragma once
 
+#include <cuda.h>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -19,6 +21,7 @@ struct DecodeParams {
   int record, off_v, off_s, row_bytes;
   int NB, bs, H, Hq, D, g, cap, rlen, max_seqs, mode;
   int splits, chunk;
+  int ring_split;            // INT4 with tensor-core pages: slot of the ring partial, else -1
   int act_fp16;              // activations (q, ring) are fp16 rather than bf16
   float scale_log2;
   void* out;
@@ -100,5 +103,9 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaS
 cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 // true when the tensor-core kernel covers this geometry and GQA group size
 bool mma_supported(const Geometry& g, int group);
+bool int4_mma_supported(const Geometry& g, int group);
+cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
+// Tensor map over the pages pool viewed as rows of 128 bytes; one box = one record.
+bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows);
 
 }  // namespace kvq

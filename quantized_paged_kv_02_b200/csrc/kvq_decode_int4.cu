@@ -1,0 +1,450 @@
+// Paged split-K decode attention over KIVI INT4 pages on tensor cores (head_dim 128,
+// block 64, GQA groups of 3..8 query heads).
+//
+// KIVI keeps keys per channel and values per token ([P-prod] "Key 和 Value 的分布不一定
+// 相同"), each as X_q = round(X/scale) + zero_point ([P-prod] "量化不是简单截断精度"):
+//   k_hat[t][d] = (c[t][d] - zk[d]) * sk[d]   (one (scale, zero) per channel per block)
+//   v_hat[t][d] = (c[t][d] - zv[t][G]) * sv[t][G]   (G = the 64-channel group of d)
+// A per-channel key scale cannot leave the sum over channels, so for each block the
+// consumer forms q'[d] = q[d] * sk[d] (exact in fp32; split into fp16 hi + lo halves, 22
+// bits, so nothing is lost) and the tensor cores see integer A values (c - zk) in fp16:
+// nibbles are placed in the mantissa of 1024.0 and (1024 + zk) is subtracted, exactly.
+// S^T = (C - Zk) Q'^T with two mma.sync m16n8k16 per k-step.  For P V, the value scale
+// of each token's channel group is folded into P (one P operand per group, with the same
+// power-of-two normaliser as the INT8 kernel), and A = (c - zv) of two tokens per register
+// is assembled with a byte permute.  The residual ring (the newest tokens, unquantized)
+// is a separate split handled by the CUDA-core kernel; the reduce merges both.
+//
+// Structure as the dense tensor-core kernel: warp 4 stages one 9 KiB record per block
+// (64 tokens of K and V codes plus all scales and zero points) with one 128-byte-swizzled
+// TMA copy into an mbarrier ring; warps 0-3 consume blocks round-robin (16 tokens per
+// MMA tile, four tiles per block).
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <mutex>
+
+#include "kvq_decode_common.cuh"
+#include "kvq_ptx.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kC = 4;                     // consumer warps
+constexpr int kT = 32 * (kC + 1);
+constexpr int kD = 128;
+constexpr int kBS = 64;
+constexpr int kRowB = kD / 2;             // 64 bytes of codes per token
+constexpr int kOffV = kBS * kRowB;        // 4096
+constexpr int kOffKs = 2 * kBS * kRowB;   // 8192: K scale [128] fp16
+constexpr int kOffKz = kOffKs + 2 * kD;   // 8448: K zero point [128] fp16
+constexpr int kOffVsz = kOffKs + 4 * kD;  // 8704: V (scale, zero) [64][2][2] fp16
+constexpr int kRec = kOffVsz + kBS * 2 * 4;   // 9216
+constexpr int kRecRows = kRec / 128;      // 72
+constexpr int kStage = kRec;              // already a multiple of 1024
+constexpr int kStages = 7;
+constexpr int kTiles = kStages * kStage;
+constexpr int kBytes = 1024 + kTiles + kStages * 16 + kStages * 4;
+constexpr float kRescale4 = 8.f;
+static_assert(kStage % 1024 == 0, "stages start on the swizzle period");
+static_assert(kC * 8 * (kD + 2) * 4 <= kTiles, "merge buffer");
+
+__device__ __forceinline__ int swzb4(int off) {
+  return (off & ~127) + ((((off >> 4) & 7) ^ ((off >> 7) & 7)) << 4) + (off & 15);
+}
+
+// (nibble s, nibble s+4) of w as fp16 (1024 + code) pairs minus the constant pair zc
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int s, uint32_t zc) {
+  const uint32_t h = ((w >> (4 * s)) & 0x000F000Fu) | 0x64006400u;
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(zc));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__global__ void __launch_bounds__(kT, 2)
+decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* tiles = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTiles);
+  uint64_t* empty = full + kStages;
+  int* valid = reinterpret_cast<int*>(empty + kStages);
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SeqInfo si = seq_info(p, b, true, split == 0 && kvh == 0 && threadIdx.x == 0);
+  const int t0 = split * p.chunk;                         // a multiple of 64
+  const int t1 = min(si.qb, t0 + p.chunk);                // blocks only; the ring is elsewhere
+  const int npages = t1 > t0 ? (t1 - t0) / kBS : 0;
+  const int page0 = t0 / kBS;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  float o[8][4];
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  int ev = INT_MIN;
+  const int r = lane >> 2, j = lane & 3;
+#pragma unroll
+  for (int md = 0; md < 8; ++md)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o[md][c] = 0.f;
+
+  if (warp == kC) {
+    // ---------------------------------------------------------------- producer
+    bool ok_run = true;
+    int issued = 0;
+    for (int base = 0; base < npages && ok_run; base += 32) {
+      int blk = -1;
+      if (base + lane < npages) {
+        blk = p.tables[static_cast<long>(b) * p.max_blocks + page0 + base + lane];
+        if (blk < 0 || blk >= p.NB) {
+          record_fault(p.fault, KVQ_FAULT_BLOCK);
+          blk = -1;
+        }
+      }
+      const int cnt = min(32, npages - base);
+      for (int k = 0; k < cnt; ++k) {
+        const int bk = __shfl_sync(0xffffffffu, blk, k);
+        const int i = base + k;
+        const int s = i % kStages;
+        const int round = i / kStages;
+        if (lane == 0) {
+          if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) {
+            record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+            ok_run = false;
+          }
+          if (ok_run) {
+            valid[s] = bk >= 0;
+            if (bk >= 0) {
+              mbar_arrive_expect_tx(&full[s], kRec);
+              tma_load_2d(tiles + s * kStage, &tmap, &full[s], 0, (bk * p.H + kvh) * kRecRows);
+            } else {
+              mbar_arrive(&full[s]);
+            }
+          }
+        }
+        ok_run = __shfl_sync(0xffffffffu, ok_run, 0);
+        if (!ok_run) break;
+        issued = i + 1;
+      }
+    }
+    if (lane == 0) {
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        if (!mbar_wait(&full[i % kStages], (i / kStages) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int g = p.g;
+    // q of head r, channels [32j, 32j+32), as bf16/fp16 pairs scaled by 2^-eq (exact)
+    float qv[32];
+    if (r < g) {
+      const uint16_t* qp = static_cast<const uint16_t*>(p.q) +
+                           (static_cast<long>(b) * p.Hq + kvh * g + r) * kD + 32 * j;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4*>(qp + 8 * c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (p.act_fp16) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+            qv[8 * c + 2 * e] = f.x;
+            qv[8 * c + 2 * e + 1] = f.y;
+          } else {
+            qv[8 * c + 2 * e] = bf16lo(w[e]);
+            qv[8 * c + 2 * e + 1] = bf16hi(w[e]);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) qv[e] = 0.f;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(qv[e]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    // keep |q * scale| well inside fp16 for channel scales up to ~1000
+    const int eq = amax > 0.f ? exponent_of(amax) - 5 : 0;
+    const float qdown = pow2i(-eq);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) qv[e] *= qdown;
+    const float qscale = p.scale_log2 * pow2i(eq);
+
+    float vlim = 0.f, vinv = 0.f;
+    for (int i = warp; i < npages; i += kC) {
+      const int s = i % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kStages) & 1))) {
+        if (lane == 0) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+        break;
+      }
+      const uint8_t* st = tiles + s * kStage;
+      if (valid[s] == 0) {              // bad block id (counted by the producer): skip it
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        continue;
+      }
+      // ------------------------------------------------ per-block key scales -> Q' and Zk
+      // q'[e] = q[32j+e] * sk[32j+e]; k-step kc uses channel pairs (8w+sp, 8w+sp+4) and
+      // (8w+sp+1, 8w+sp+5) with w = kc/2, sp = 2*(kc%2): the pairs the nibble extraction
+      // of word w yields.
+      uint32_t qh[8][2], ql[8][2], zc[4][4];
+      {
+        uint32_t sw[16], zw[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 a = lds128(st + swzb4(kOffKs + 64 * j + 16 * c));
+          const uint4 z = lds128(st + swzb4(kOffKz + 64 * j + 16 * c));
+          sw[4 * c] = a.x; sw[4 * c + 1] = a.y; sw[4 * c + 2] = a.z; sw[4 * c + 3] = a.w;
+          zw[4 * c] = z.x; zw[4 * c + 1] = z.y; zw[4 * c + 2] = z.z; zw[4 * c + 3] = z.w;
+        }
+        float qs[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&sw[e]));
+          qs[2 * e] = qv[2 * e] * f.x;
+          qs[2 * e + 1] = qv[2 * e + 1] * f.y;
+        }
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+          const int e0 = 8 * (kc >> 1) + 2 * (kc & 1);
+          const float a0 = qs[e0], a1 = qs[e0 + 4], c0 = qs[e0 + 1], c1 = qs[e0 + 5];
+          const uint32_t h0 = pack_f16x2(a0, a1), h1 = pack_f16x2(c0, c1);
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+          qh[kc][0] = h0;
+          qh[kc][1] = h1;
+          ql[kc][0] = pack_f16x2(a0 - f0.x, a1 - f0.y);
+          ql[kc][1] = pack_f16x2(c0 - f1.x, c1 - f1.y);
+        }
+        // (1024 + zk[8w+sp'], 1024 + zk[8w+sp'+4]) for sp' = 0..3
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int sp = 0; sp < 4; ++sp) {
+            const int ea = 8 * w + sp, eb = ea + 4;      // halves ea, eb of zw
+            const uint32_t sel = ((ea & 1) ? 0x0032u : 0x0010u) | ((eb & 1) ? 0x7600u : 0x5400u);
+            const uint32_t pair = prmt(zw[ea >> 1], zw[eb >> 1], sel);
+            zc[w][sp] = hadd2(pair, 0x64006400u);
+          }
+      }
+#pragma unroll 1
+      for (int mt = 0; mt < kBS / 16; ++mt) {
+        const int tr0 = 16 * mt + r, tr1 = tr0 + 8;
+        // ------------------------------------------------ S^T = (C - Zk) Q'^T
+        const uint4 k0 = lds128(st + swzb4(kRowB * tr0 + 16 * j));
+        const uint4 k1 = lds128(st + swzb4(kRowB * tr1 + 16 * j));
+        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+          const int w = kc >> 1, sp = 2 * (kc & 1);
+          const uint32_t a[4] = {nib_pair(w0[w], sp, zc[w][sp]), nib_pair(w1[w], sp, zc[w][sp]),
+                                 nib_pair(w0[w], sp + 1, zc[w][sp + 1]), nib_pair(w1[w], sp + 1, zc[w][sp + 1])};
+          mma_f16(sa, a, qh[kc]);
+          mma_f16(sb, a, ql[kc]);
+        }
+        // ------------------------------------------------ softmax (log2 domain)
+        float s00 = (sa[0] + sb[0]) * qscale, s01 = (sa[1] + sb[1]) * qscale;
+        float s10 = (sa[2] + sb[2]) * qscale, s11 = (sa[3] + sb[3]) * qscale;
+        const bool grow = s00 > m[0] + kRescale4 || s10 > m[0] + kRescale4 ||
+                          s01 > m[1] + kRescale4 || s11 > m[1] + kRescale4;
+        if (__any_sync(0xffffffffu, grow)) {
+          float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, off));
+            tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, off));
+          }
+          const float mn0 = fmaxf(m[0], tm0), mn1 = fmaxf(m[1], tm1);
+          const float c0 = m[0] == -INFINITY ? 0.f : ex2(m[0] - mn0);
+          const float c1 = m[1] == -INFINITY ? 0.f : ex2(m[1] - mn1);
+          m[0] = mn0;
+          m[1] = mn1;
+          l[0] *= c0;
+          l[1] *= c1;
+#pragma unroll
+          for (int md = 0; md < 8; ++md) {
+            o[md][0] *= c0;
+            o[md][1] *= c1;
+            o[md][2] *= c0;
+            o[md][3] *= c1;
+          }
+        }
+        const float base0 = m[0] == -INFINITY ? 0.f : m[0], base1 = m[1] == -INFINITY ? 0.f : m[1];
+        const float p00 = ex2(s00 - base0), p10 = ex2(s10 - base0);
+        const float p01 = ex2(s01 - base1), p11 = ex2(s11 - base1);
+        l[0] += p00 + p10;
+        l[1] += p01 + p11;
+        // ------------------------------------------------ value scales folded into P
+        // vsz for token t, group G: (scale, zero) fp16 at kOffVsz + 8t + 4G
+        const uint32_t sz00 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr0));
+        const uint32_t sz01 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr0 + 4));
+        const uint32_t sz10 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr1));
+        const uint32_t sz11 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr1 + 4));
+        float vs[2][2] = {{__half2float(__ushort_as_half(sz00 & 0xFFFF)), __half2float(__ushort_as_half(sz01 & 0xFFFF))},
+                          {__half2float(__ushort_as_half(sz10 & 0xFFFF)), __half2float(__ushort_as_half(sz11 & 0xFFFF))}};
+        if (__any_sync(0xffffffffu, vs[0][0] >= vlim || vs[0][1] >= vlim || vs[1][0] >= vlim || vs[1][1] >= vlim)) {
+          float vm = fmaxf(fmaxf(vs[0][0], vs[0][1]), fmaxf(vs[1][0], vs[1][1]));
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+          if (vm > 0.f) {
+            const int e = exponent_of(vm);
+            if (e > ev) {
+              if (ev != INT_MIN) {
+                const float down = pow2i(ev - e);
+#pragma unroll
+                for (int md = 0; md < 8; ++md)
+#pragma unroll
+                  for (int c = 0; c < 4; ++c) o[md][c] *= down;
+              }
+              ev = e;
+              vlim = pow2i(ev + 1);
+              vinv = pow2i(-ev);
+            }
+          }
+        }
+        uint32_t pbh[2][2], pbl[2][2];
+#pragma unroll
+        for (int G = 0; G < 2; ++G) {
+          const float w0g = vs[0][G] * vinv, w1g = vs[1][G] * vinv;
+          const float q00 = p00 * w0g, q01 = p01 * w0g, q10 = p10 * w1g, q11 = p11 * w1g;
+          const uint32_t h0 = pack_f16x2(q00, q01), h1 = pack_f16x2(q10, q11);
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+          const uint32_t e0 = pack_f16x2(q00 - f0.x, q01 - f0.y), e1 = pack_f16x2(q10 - f1.x, q11 - f1.y);
+          pbh[G][0] = movmatrix_trans(h0);
+          pbh[G][1] = movmatrix_trans(h1);
+          pbl[G][0] = movmatrix_trans(e0);
+          pbl[G][1] = movmatrix_trans(e1);
+        }
+        // ------------------------------------------------ O^T += (C - Zv)^T P'^T
+        // tile md: group G = md/4, byte k = md%4 of the word holding channels
+        // 64G + 8r .. +7 of a token; rows r / r+8 <-> d = 64G + 8r + 2k / +1
+        const int ta = 16 * mt + 2 * j;
+        const int tt[4] = {ta, ta + 1, ta + 8, ta + 9};
+        uint32_t vwd[4][2], zv[2][2];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int G = 0; G < 2; ++G)
+            vwd[t][G] = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffV + kRowB * tt[t] + 32 * G + 4 * r));
+#pragma unroll
+        for (int G = 0; G < 2; ++G) {
+          const uint32_t za = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[0] + 4 * G));
+          const uint32_t zb = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[1] + 4 * G));
+          const uint32_t zc2 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[2] + 4 * G));
+          const uint32_t zd = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[3] + 4 * G));
+          // zero points are the high halves: (1024 + z_a, 1024 + z_b)
+          zv[G][0] = hadd2(prmt(za, zb, 0x7632u), 0x64006400u);
+          zv[G][1] = hadd2(prmt(zc2, zd, 0x7632u), 0x64006400u);
+        }
+#pragma unroll
+        for (int md = 0; md < 8; ++md) {
+          const int G = md >> 2, k = md & 3;
+          const uint32_t sel = static_cast<uint32_t>(k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12));
+          const uint32_t Y = prmt(vwd[0][G], vwd[1][G], sel);   // bytes (ta_k, ta_k, tb_k, tb_k)
+          const uint32_t Z = prmt(vwd[2][G], vwd[3][G], sel);
+          const uint32_t a[4] = {hsub2((Y & 0x000F000Fu) | 0x64006400u, zv[G][0]),
+                                 hsub2(((Y >> 4) & 0x000F000Fu) | 0x64006400u, zv[G][0]),
+                                 hsub2((Z & 0x000F000Fu) | 0x64006400u, zv[G][1]),
+                                 hsub2(((Z >> 4) & 0x000F000Fu) | 0x64006400u, zv[G][1])};
+          mma_f16(o[md], a, pbh[G]);
+          mma_f16(o[md], a, pbl[G]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
+      l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
+    }
+  }
+  __syncthreads();
+
+  float* red_o = reinterpret_cast<float*>(tiles);           // [warp][head][D]
+  float* red_ml = red_o + kC * 8 * kD;                      // [warp][head][2]
+  if (warp < kC) {
+    const float vmul = ev == INT_MIN ? 0.f : pow2i(ev);
+#pragma unroll
+    for (int md = 0; md < 8; ++md) {
+      const int d0 = 64 * (md >> 2) + 8 * r + 2 * (md & 3);
+      red_o[(warp * 8 + 2 * j) * kD + d0] = o[md][0] * vmul;
+      red_o[(warp * 8 + 2 * j + 1) * kD + d0] = o[md][1] * vmul;
+      red_o[(warp * 8 + 2 * j) * kD + d0 + 1] = o[md][2] * vmul;
+      red_o[(warp * 8 + 2 * j + 1) * kD + d0 + 1] = o[md][3] * vmul;
+    }
+    if (r == 0) {
+      red_ml[(warp * 8 + 2 * j) * 2] = m[0];
+      red_ml[(warp * 8 + 2 * j) * 2 + 1] = l[0];
+      red_ml[(warp * 8 + 2 * j + 1) * 2] = m[1];
+      red_ml[(warp * 8 + 2 * j + 1) * 2 + 1] = l[1];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.g * kD; e += kT) {
+    const int h = e / kD, d = e % kD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kC; ++w) M = fmaxf(M, red_ml[(w * 8 + h) * 2]);
+    float Lsum = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kC; ++w) {
+      const float mw = red_ml[(w * 8 + h) * 2];
+      const float f = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      Lsum += red_ml[(w * 8 + h) * 2 + 1] * f;
+      O += red_o[(w * 8 + h) * kD + d] * f;
+    }
+    store_partial_or_output(p, b, kvh * p.g + h, split, d, M, Lsum, O);
+  }
+}
+
+}  // namespace
+
+bool int4_mma_supported(const Geometry& g, int group) {
+  return g.cache_dtype == KVQ_DTYPE_INT4 && g.D == kD && g.bs == kBS && g.record == kRec &&
+         group >= 3 && group <= 8;
+}
+
+cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(decode_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap tm;
+  const long rows = static_cast<long>(a.geo.NB) * a.geo.H * kRecRows;
+  if (!make_pages_map(&tm, a.c->pages, rows, kRecRows)) return cudaErrorInvalidValue;
+  // page splits only; the ring split is launched separately
+  const dim3 grid(p.ring_split, a.geo.H, a.batch);
+  decode_int4_kernel<<<grid, kT, kBytes, s>>>(p, tm);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

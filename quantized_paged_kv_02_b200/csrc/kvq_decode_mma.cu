@@ -579,35 +579,6 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   }
 }
 
-// ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
-}
-
-// Tensor map over the pages pool viewed as rows of 128 bytes; one box is one record
-// (rec_rows rows), copied with 128-byte swizzle.
-bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows) {
-  auto enc = encoder();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(rec_rows)};
-  cuuint32_t es[2] = {1, 1};
-  const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                           box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return res == CUDA_SUCCESS;
-}
-
 template <int CD, int BS, bool PT>
 cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
   using L = Layout<CD, BS, PT>;
@@ -634,6 +605,35 @@ cudaError_t launch_bs(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s
 }
 
 }  // namespace
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// Tensor map over the pages pool viewed as rows of 128 bytes; one box is one record
+// (rec_rows rows), copied with 128-byte swizzle.
+bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows) {
+  auto enc = encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(rec_rows)};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                           box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
+}
 
 bool mma_supported(const Geometry& g, int groups) {
   if (g.D != kD || groups < 3 || groups > 8) return false;

@@ -74,7 +74,9 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
   constexpr bool kInt4 = CD == KVQ_DTYPE_INT4;
   constexpr int ROWB = D * CB / EPL;    // bytes per cache row
 
-  const int split = blockIdx.x;
+  // ring-only launch (INT4 blocks on tensor cores): this grid covers [qb, n) from the ring
+  const bool ring_only = p.ring_split >= 0;
+  const int split = ring_only ? p.ring_split : blockIdx.x;
   const int tiles = p.g / GT;
   const int kvh = blockIdx.y / tiles;
   const int hq0 = kvh * p.g + (blockIdx.y % tiles) * GT;
@@ -83,8 +85,8 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
   const int c = lane % LPR, grp = lane / LPR;
 
   const SeqInfo si = seq_info(p, b, kInt4, blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0);
-  const int t0 = split * p.chunk;
-  const int t1 = min(si.n, t0 + p.chunk);
+  const int t0 = ring_only ? si.qb : split * p.chunk;
+  const int t1 = ring_only ? si.n : min(si.n, t0 + p.chunk);
 
   // query chunk (pre-multiplied by softmax_scale * log2 e)
   float qf[GT][EPL];
@@ -270,7 +272,7 @@ cudaError_t launch_d(int cd, const DecodeParams& p, dim3 grid, cudaStream_t s) {
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
   const int gt = (a.plan.g % 2 == 0) ? 2 : 1;
-  const dim3 grid(a.plan.splits, a.geo.H * (a.plan.g / gt), a.batch);
+  const dim3 grid(p.ring_split >= 0 ? 1 : a.plan.splits, a.geo.H * (a.plan.g / gt), a.batch);
   if (a.geo.act_dtype == KVQ_DTYPE_BF16)
     return a.geo.D == 128 ? launch_d<__nv_bfloat16, 128>(a.geo.cache_dtype, p, grid, s)
                           : launch_d<__nv_bfloat16, 64>(a.geo.cache_dtype, p, grid, s);
