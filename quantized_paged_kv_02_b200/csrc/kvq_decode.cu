@@ -12,34 +12,59 @@
 namespace kvq {
 namespace {
 
-__global__ void __launch_bounds__(128) split_reduce_kernel(DecodeParams p, bool int4) {
-  const int row = blockIdx.x;                 // b * Hq + hq
+// One warp per (sequence, query head): lane k computes the weight of split slot k
+// (k < 32; longer lists loop), lanes own 4 consecutive channels of the output.
+__global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool int4) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);   // b * Hq + hq
+  const int lane = threadIdx.x & 31;
+  if (row >= p.rows) return;
   const int b = row / p.Hq;
   const SeqInfo si = seq_info(p, b, int4);
   // splits that hold work: the token splits covering [0, n), or, when the INT4 ring has
   // a split of its own, the block splits covering [0, qb) plus the ring split
   const int S = (p.ring_split >= 0 ? si.qb + p.chunk - 1 : si.n + p.chunk - 1) / p.chunk;
   const bool ring = p.ring_split >= 0 && si.n > si.qb;
+  const int K = S + (ring ? 1 : 0);
   const float* ml = p.ws_ml + static_cast<long>(row) * p.splits * 2;
   const float* o = p.ws_o + static_cast<long>(row) * p.splits * p.D;
   auto slot = [&](int k) { return k < S ? k : p.ring_split; };
-  const int K = S + (ring ? 1 : 0);
+  // max over the splits
   float M = -INFINITY;
-  for (int k = 0; k < K; ++k) M = fmaxf(M, ml[2 * slot(k)]);
+  for (int k = lane; k < K; k += 32) M = fmaxf(M, ml[2 * slot(k)]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float L = 0.f;
-  for (int k = 0; k < K; ++k) {
-    const float mk = ml[2 * slot(k)];
-    L += (M == -INFINITY || mk == -INFINITY) ? 0.f : ml[2 * slot(k) + 1] * exp2f(mk - M);
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int k = 0; k < K; ++k) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const bool has_d = 4 * lane < p.D;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    const int k = k0 + lane;
+    float w = 0.f;
+    if (k < K) {
       const float mk = ml[2 * slot(k)];
-      const float w = (M == -INFINITY || mk == -INFINITY) ? 0.f : exp2f(mk - M);
-      acc = fmaf(o[static_cast<long>(slot(k)) * p.D + d], w, acc);
+      w = (M == -INFINITY || mk == -INFINITY) ? 0.f : exp2f(mk - M);
+      L = fmaf(ml[2 * slot(k) + 1], w, L);
     }
-    store_out(p, static_cast<long>(row) * p.D + d, acc * inv);
+    const int n = min(32, K - k0);
+    for (int i = 0; i < n; ++i) {
+      const float wi = __shfl_sync(0xffffffffu, w, i);
+      if (has_d) {
+        const float4 v = *reinterpret_cast<const float4*>(o + static_cast<long>(slot(k0 + i)) * p.D + 4 * lane);
+        acc.x = fmaf(v.x, wi, acc.x);
+        acc.y = fmaf(v.y, wi, acc.y);
+        acc.z = fmaf(v.z, wi, acc.z);
+        acc.w = fmaf(v.w, wi, acc.w);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (has_d) {
+    const long base = static_cast<long>(row) * p.D + 4 * lane;
+    store_out(p, base, acc.x * inv);
+    store_out(p, base + 1, acc.y * inv);
+    store_out(p, base + 2, acc.z * inv);
+    store_out(p, base + 3, acc.w * inv);
   }
 }
 
@@ -149,6 +174,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.splits = a.plan.splits;
   p.chunk = a.plan.chunk;
   p.ring_split = a.plan.kernel == 2 ? a.plan.splits - 1 : -1;
+  p.rows = a.batch * a.Hq;
   p.act_fp16 = g.act_dtype == KVQ_DTYPE_FP16;
   p.scale_log2 = a.scale_log2;
   p.out = a.out;
@@ -166,7 +192,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   }
   if (e != cudaSuccess) return e;
   if (p.splits > 1) {
-    split_reduce_kernel<<<a.batch * a.Hq, 128, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);
+    split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);
     e = cudaGetLastError();
   }
   return e;

@@ -22,6 +22,7 @@ struct DecodeParams {
   int NB, bs, H, Hq, D, g, cap, rlen, max_seqs, mode;
   int splits, chunk;
   int ring_split;            // INT4 with tensor-core pages: slot of the ring partial, else -1
+  int rows;                  // batch * Hq
   int act_fp16;              // activations (q, ring) are fp16 rather than bf16
   float scale_log2;
   void* out;
