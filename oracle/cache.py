@@ -125,29 +125,37 @@ class PagedCache:
         if self.cd == "int4":
             return self._write_int4(k_new, v_new, slots, seq_ids, positions)
         NB, bs = self.NB, self.bs
-        for t in range(slots.shape[0]):
-            slot = int(slots[t])
-            if slot < 0 or slot >= NB * bs:
+        keep = (slots >= 0) & (slots < NB * bs)
+        t_idx = np.nonzero(keep)[0]
+        if np.unique(slots[t_idx]).size != t_idx.size:
+            # a slot named twice: rows are applied in order, so the later one stays
+            for t in t_idx:
+                self._write_rows(k_new[t:t + 1], v_new[t:t + 1], slots[t:t + 1])
+            return
+        self._write_rows(k_new[t_idx], v_new[t_idx], slots[t_idx])
+
+    def _write_rows(self, k_rows, v_rows, slots):
+        """Quantize rows [n, H, D] into distinct, in-range slots [n].  Every (token, kv
+        head) row is quantized on its own, so the rows are processed together."""
+        blk, off = np.divmod(slots, self.bs)
+        for which, rows in ((0, k_rows), (1, v_rows)):
+            codes = self.k_codes if which == 0 else self.v_codes
+            x = rows.astype(np.float32)                # [n, H, D], exact
+            if self.cd in ("bf16", "fp16"):
+                codes[blk, :, off, :] = _bits_of_act(rows, self.act)
                 continue
-            blk, off = divmod(slot, bs)
-            for which, rows in ((0, k_new[t]), (1, v_new[t])):
-                codes = self.k_codes if which == 0 else self.v_codes
-                x = rows.astype(np.float32)            # [H, D], exact
-                if self.cd in ("bf16", "fp16"):
-                    codes[blk, :, off, :] = _bits_of_act(rows, self.act)
-                    continue
-                if self.mode == "per_token_head":
-                    s = (quant.int8_scale_dynamic(x) if self.cd == "int8"
-                         else quant.fp8_scale_dynamic(x))          # [H]
-                    sc = self.k_scales if which == 0 else self.v_scales
-                    sc[blk, :, off] = s
-                else:
-                    s = self._static_scale(which)
-                s2 = np.asarray(s, np.float32)[:, None]
-                if self.cd == "int8":
-                    codes[blk, :, off, :] = quant.int8_quantize(x, s2)
-                else:
-                    codes[blk, :, off, :] = quant.fp8_quantize(x, s2)
+            if self.mode == "per_token_head":
+                s = (quant.int8_scale_dynamic(x) if self.cd == "int8"
+                     else quant.fp8_scale_dynamic(x))              # [n, H]
+                sc = self.k_scales if which == 0 else self.v_scales
+                sc[blk, :, off] = s
+            else:
+                s = np.broadcast_to(self._static_scale(which), x.shape[:2])
+            s2 = np.asarray(s, np.float32)[..., None]
+            if self.cd == "int8":
+                codes[blk, :, off, :] = quant.int8_quantize(x, s2)
+            else:
+                codes[blk, :, off, :] = quant.fp8_quantize(x, s2)
 
     def _write_int4(self, k_new, v_new, slots, seq_ids, positions):
         T = slots.shape[0]
@@ -162,16 +170,18 @@ class PagedCache:
                 if not all(int(slots[u + i]) == first + i for i in range(G)):
                     continue
                 blk = first // bs
-                for h in range(self.H):
-                    kc, ks, kz = quant.int4_keys_block(k_new[u:u + G, h, :].astype(np.float32))
-                    self.k_codes[blk, h] = quant.pack_nibbles(kc)
-                    self.k_scales[blk, h, 0, :] = ks
-                    self.k_scales[blk, h, 1, :] = kz
-                    for i in range(G):
-                        vc, vs, vz = quant.int4_values_row(v_new[u + i, h, :], self.G)
-                        self.v_codes[blk, h, i] = quant.pack_nibbles(vc)
-                        self.v_scales[blk, h, i, :, 0] = vs
-                        self.v_scales[blk, h, i, :, 1] = vz
+                # keys per (head, channel) over the block's rows; values per (row, head,
+                # channel group); every group on its own, all heads at once
+                kb = np.swapaxes(k_new[u:u + G].astype(np.float32), 0, 1)     # [H, G, D]
+                kc, ks, kz = quant.int4_keys_block(kb)
+                self.k_codes[blk] = quant.pack_nibbles(kc)
+                self.k_scales[blk, :, 0, :] = ks
+                self.k_scales[blk, :, 1, :] = kz
+                vb = np.swapaxes(v_new[u:u + G].astype(np.float32), 0, 1)     # [H, G, D]
+                vc, vs, vz = quant.int4_values_row(vb, self.G)
+                self.v_codes[blk] = quant.pack_nibbles(vc)
+                self.v_scales[blk, :, :, :, 0] = vs
+                self.v_scales[blk, :, :, :, 1] = vz
             else:
                 for t in rows:
                     if int(slots[t]) != -1 or positions is None or int(positions[t]) < 0:

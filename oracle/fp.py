@@ -72,32 +72,28 @@ def e4m3_decode(codes):
     return _E4M3[np.asarray(codes, dtype=np.uint8)]
 
 
-def e4m3_encode(r, chunk=1 << 16):
+def e4m3_encode(r):
     """Encode finite binary32 values r as E4M3FN codes.
 
     The magnitude goes to the nearest finite E4M3 magnitude; an exact tie goes to the
     code with the even mantissa (even code); magnitudes above 448 saturate to 448
     (0x7E).  The sign bit is the sign of r, also when the magnitude rounds to zero.
-    Brute force: the distance to every one of the 127 candidates is compared.
+    The 127 magnitudes increase with the code, so the nearest one is one of the two
+    neighbours of |r| in that sorted list; the tie rule picks the even one of the two
+    (adjacent codes, so exactly one is even).
     """
     r = np.asarray(r, dtype=np.float32)
     flat = r.reshape(-1).astype(np.float64)
-    out = np.empty(flat.shape, dtype=np.uint8)
-    cand = _E4M3_POS[None, :]
-    for i in range(0, flat.size, chunk):
-        # saturation first: a magnitude beyond 448 encodes as 448
-        a = np.minimum(np.abs(flat[i:i + chunk]), E4M3_MAX)[:, None]
-        dist = np.abs(a - cand)                       # [n, 127]
-        best = dist.min(axis=1, keepdims=True)
-        hits = dist == best                           # one or two candidates
-        # lowest even code among the hits if there is a tie, else the single hit
-        codes_idx = np.arange(127)[None, :]
-        even_hit = hits & (codes_idx % 2 == 0)
-        has_two = hits.sum(axis=1) > 1
-        pick = np.where(has_two, np.argmax(even_hit, axis=1), np.argmax(hits, axis=1))
-        out[i:i + chunk] = pick.astype(np.uint8)
-    neg = np.signbit(flat)
-    out[neg] |= 0x80
+    # saturation first: a magnitude beyond 448 encodes as 448
+    a = np.minimum(np.abs(flat), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 126)   # first >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - _E4M3_POS[lo]
+    d_hi = _E4M3_POS[hi] - a
+    even = np.where(lo % 2 == 0, lo, hi)
+    pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, even))
+    out = pick.astype(np.uint8)
+    out[np.signbit(flat)] |= 0x80
     return out.reshape(r.shape)
 
 

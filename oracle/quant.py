@@ -106,27 +106,37 @@ def fp8_dequantize(codes, scale):
 
 
 # ----------------------------------------------------------------------------- INT4
-def int4_quantize_group(values):
-    """Asymmetric 4-bit quantization of one group (1-D array of binary32 values).
+def int4_quantize_groups(values):
+    """Asymmetric 4-bit quantization of groups along the last axis (binary32 values).
 
-    Returns (codes uint8 in 0..15, scale float16, zero point float16).
+    Every group (1-D slice values[..., :]) is quantized on its own.  Returns (codes
+    uint8 in 0..15 with the shape of values, scale float16 and zero point float16 with
+    the leading shape).
       lo = min(min x, 0); hi = max(max x, 0)
       s  = float16(binary32((hi - lo) / 15))       -- stored, and used from here on
       z  = clamp(round_half_even(-lo / s), 0, 15)
       q  = clamp(round_half_even(x / s) + z, 0, 15)
+    A group whose s is 0 (all values 0) gets codes 0, scale 0, zero point 0.
     [P-prod] "量化不是简单截断精度": X_q = round(X/scale) + zero_point.
     """
-    x = np.asarray(values, dtype=np.float32).reshape(-1)
-    lo = np.minimum(x.min(), np.float32(0.0))
-    hi = np.maximum(x.max(), np.float32(0.0))
+    x = np.asarray(values, dtype=np.float32)
+    lo = np.minimum(x.min(axis=-1), np.float32(0.0))
+    hi = np.maximum(x.max(axis=-1), np.float32(0.0))
     s32 = fp.div32(fp.sub32(hi, lo), np.float32(INT4_LEVELS))
     s16 = fp.f16(s32)
-    if s16 == 0:
-        return np.zeros(x.shape, np.uint8), np.float16(0.0), np.float16(0.0)
-    sw = np.float32(s16)
+    zero_group = s16 == 0
+    sw = np.where(zero_group, np.float32(1.0), np.asarray(s16, np.float32))
     z = np.clip(fp.round_half_even(fp.div32(-lo, sw)), 0, 15)
-    q = np.clip(fp.round_half_even(fp.div32(x, sw)) + z, 0, 15)
-    return q.astype(np.uint8), s16, np.float16(z)
+    q = np.clip(fp.round_half_even(fp.div32(x, sw[..., None])) + z[..., None], 0, 15)
+    q = np.where(zero_group[..., None], 0, q)
+    z = np.where(zero_group, 0, z)
+    return q.astype(np.uint8), np.asarray(s16, np.float16), np.asarray(z, np.float16)
+
+
+def int4_quantize_group(values):
+    """int4_quantize_groups for one group (1-D array): (codes, scale, zero point)."""
+    q, s, z = int4_quantize_groups(np.asarray(values, dtype=np.float32).reshape(1, -1))
+    return q[0], s[0], z[0]
 
 
 def int4_dequantize(codes, scale, zero):
@@ -137,34 +147,26 @@ def int4_dequantize(codes, scale, zero):
 def int4_keys_block(k_rows):
     """KIVI keys: one group per channel over the block's tokens.
 
-    k_rows [64, D] (one kv head).  Returns codes [64, D], scale [D], zero [D].
+    k_rows [64, D] (one kv head), or [..., 64, D] for several heads at once.  Returns
+    codes [..., 64, D], scale [..., D], zero [..., D].
     [P-prod] "Key 和 Value 的分布不一定相同": key cache per channel (KIVI).
     """
     k_rows = np.asarray(k_rows, dtype=np.float32)
-    T, D = k_rows.shape
-    codes = np.empty((T, D), np.uint8)
-    s = np.empty(D, np.float16)
-    z = np.empty(D, np.float16)
-    for d in range(D):
-        codes[:, d], s[d], z[d] = int4_quantize_group(k_rows[:, d])
-    return codes, s, z
+    q, s, z = int4_quantize_groups(np.swapaxes(k_rows, -1, -2))     # groups = channels
+    return np.swapaxes(q, -1, -2), s, z
 
 
 def int4_values_row(v_row, group=64):
     """KIVI values: one group per token over each run of `group` channels.
 
-    v_row [D] (one token, one kv head).  Returns codes [D], scale [D/group], zero [D/group].
+    v_row [D] (one token, one kv head), or [..., D] for several at once.  Returns codes
+    [..., D], scale [..., D/group], zero [..., D/group].
     [P-prod] "Key 和 Value 的分布不一定相同": value cache per token.
     """
     v_row = np.asarray(v_row, dtype=np.float32)
-    D = v_row.shape[0]
-    codes = np.empty(D, np.uint8)
-    s = np.empty(D // group, np.float16)
-    z = np.empty(D // group, np.float16)
-    for gi in range(D // group):
-        sl = slice(gi * group, (gi + 1) * group)
-        codes[sl], s[gi], z[gi] = int4_quantize_group(v_row[sl])
-    return codes, s, z
+    D = v_row.shape[-1]
+    q, s, z = int4_quantize_groups(v_row.reshape(v_row.shape[:-1] + (D // group, group)))
+    return q.reshape(v_row.shape), s, z
 
 
 def pack_nibbles(codes):

@@ -177,10 +177,8 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* c, const void* q, int batc
   if (a.plan.ws_bytes > 0) {
     if (workspace == nullptr || workspace_bytes < a.plan.ws_bytes || !aligned16(workspace))
       return KVQ_ERR_INVALID_ARG;
-    const size_t rows = static_cast<size_t>(batch) * num_q_heads * a.plan.splits;
     a.ws_o = static_cast<float*>(workspace);
-    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                       (rows * g.D * sizeof(float) + 255) / 256 * 256);
+    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + a.plan.ws_ml_off);
   }
   a.q = q;
   a.batch = batch;

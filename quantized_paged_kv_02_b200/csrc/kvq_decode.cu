@@ -68,6 +68,118 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
   }
 }
 
+// Merge of the dense tensor-core kernel's per-warp partials.  One warp per (sequence,
+// query head): it recomputes the page partition (total pages, the pages before its
+// sequence), finds the CTAs whose ranges meet its unit's pages, and takes the partial of
+// every consumer warp that saw at least one of those pages.  Lane k describes candidate
+// k (CTA c_first + k / kSegWarps, warp k % kSegWarps); the partial rows are then read
+// four at a time so their loads overlap.
+__global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
+  constexpr int C = kMmaCtas;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);   // b * Hq + hq
+  const int lane = threadIdx.x & 31;
+  if (row >= p.rows) return;
+  const int b = row / p.Hq, hq = row - b * p.Hq;
+  const int kvh = hq / p.g, h = hq - kvh * p.g;
+  long long tot = 0, before = 0;
+  int npb = 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    const int bb = b0 + lane;
+    const int np = bb < p.batch ? seq_pages(p, bb) : 0;
+    int t = np, q = bb < b ? np : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      t += __shfl_xor_sync(0xffffffffu, t, off);
+      q += __shfl_xor_sync(0xffffffffu, q, off);
+    }
+    tot += t;
+    before += q;
+    if (b >= b0 && b < b0 + 32) npb = __shfl_sync(0xffffffffu, np, b - b0);
+  }
+  const long long P = tot * p.H;
+  const long long U0 = before * p.H + static_cast<long long>(kvh) * npb, U1 = U0 + npb;
+  int c_first = 0, c_last = -1;
+  if (npb > 0) {
+    // CTA c covers [P c / C, P (c+1) / C): the last one starting at or before U0, and
+    // the last one starting before U1
+    c_first = static_cast<int>(((U0 + 1) * C + P - 1) / P) - 1;
+    c_last = static_cast<int>((U1 * C + P - 1) / P) - 1;
+  }
+  const int K = (c_last - c_first + 1) * kSegWarps;
+  const long long u = static_cast<long long>(b) * p.H + kvh;
+  const float* ml = p.ws_ml;
+  const float* o = p.ws_o + 4 * lane;
+  const bool has_d = 4 * lane < p.D;
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    // lane k: does candidate k0 + k hold a partial, and where
+    const int k = k0 + lane;
+    int slot = -1;
+    float mk = -INFINITY, lk = 0.f;
+    if (k < K) {
+      const int c = c_first + k / kSegWarps, w = k % kSegWarps;
+      const long long sc = range_start(P, c, C), ec = range_start(P, c + 1, C);
+      const long long lo = sc > U0 ? sc : U0, hi = ec < U1 ? ec : U1;
+      const long long len = hi - lo;
+      const int first = static_cast<int>((lo - sc) % kSegWarps);   // warp of the first page
+      if (len > 0 && (len >= kSegWarps || ((w - first + kSegWarps) % kSegWarps) < len)) {
+        slot = static_cast<int>(((u + c) * kSegWarps + w) * p.g + h);
+        const float2 v = *reinterpret_cast<const float2*>(ml + 2L * slot);
+        mk = v.x;
+        lk = v.y;
+      }
+    }
+    // rescale what was merged so far to the new maximum
+    float Mc = mk;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
+    const float Mn = fmaxf(M, Mc);
+    if (Mn != -INFINITY && Mn > M) {
+      const float c0 = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      L *= c0;
+      acc.x *= c0; acc.y *= c0; acc.z *= c0; acc.w *= c0;
+      M = Mn;
+    }
+    const float w = (slot >= 0 && mk != -INFINITY) ? exp2f(mk - M) : 0.f;
+    L = fmaf(lk, w, L);
+    const int n = min(32, K - k0);
+    for (int i0 = 0; i0 < n; i0 += 4) {
+      float wi[4];
+      int si[4];
+      float4 v[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = min(i0 + t, 31);
+        wi[t] = __shfl_sync(0xffffffffu, w, i);
+        si[t] = __shfl_sync(0xffffffffu, slot, i);
+        if (i0 + t >= n) wi[t] = 0.f;
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        v[t] = (has_d && wi[t] != 0.f) ? *reinterpret_cast<const float4*>(o + static_cast<long>(si[t]) * p.D)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        acc.x = fmaf(v[t].x, wi[t], acc.x);
+        acc.y = fmaf(v[t].y, wi[t], acc.y);
+        acc.z = fmaf(v[t].z, wi[t], acc.z);
+        acc.w = fmaf(v[t].w, wi[t], acc.w);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (has_d) {
+    const long base = static_cast<long>(row) * p.D + 4 * lane;
+    store_out(p, base, acc.x * inv);
+    store_out(p, base + 1, acc.y * inv);
+    store_out(p, base + 2, acc.z * inv);
+    store_out(p, base + 3, acc.w * inv);
+  }
+}
+
 }  // namespace
 
 // Splits for the tensor-core kernel: one CTA per (sequence, kv head, split); pick the
@@ -106,20 +218,22 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
     gg.bs = 64;
     plan_mma(gg, batch, std::max(max_qb, 64), p);
     p->splits += 1;                              // the ring
+    p->ctas = 0;
     const size_t rows = static_cast<size_t>(batch) * num_q_heads * p->splits;
-    const size_t o_bytes = (rows * g.D * sizeof(float) + 255) / 256 * 256;
-    p->ws_bytes = o_bytes + rows * 2 * sizeof(float);
+    p->ws_ml_off = (rows * g.D * sizeof(float) + 255) / 256 * 256;
+    p->ws_bytes = p->ws_ml_off + rows * 2 * sizeof(float);
     return KVQ_OK;
   }
   if (p->kernel == 1) {
+    // page-balanced CTAs; partial slots (unit + cta) * kSegWarps + warp, g heads each
     p->g_tile = p->g;
-    plan_mma(g, batch, max_context, p);
-    p->ws_bytes = 0;
-    if (p->splits > 1) {
-      const size_t rows = static_cast<size_t>(batch) * num_q_heads * p->splits;
-      const size_t o_bytes = (rows * g.D * sizeof(float) + 255) / 256 * 256;
-      p->ws_bytes = o_bytes + rows * 2 * sizeof(float);
-    }
+    p->splits = 0;
+    p->chunk = 0;
+    p->ctas = kMmaCtas;
+    const size_t slots = (static_cast<size_t>(batch) * g.H + p->ctas - 1) * kSegWarps;
+    const size_t heads = slots * p->g;
+    p->ws_ml_off = (heads * g.D * sizeof(float) + 255) / 256 * 256;
+    p->ws_bytes = p->ws_ml_off + heads * 2 * sizeof(float);
     return KVQ_OK;
   }
   p->g_tile = (p->g % 2 == 0) ? 2 : 1;
@@ -135,11 +249,13 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
   S = std::max(1L, (static_cast<long>(max_context) + chunk - 1) / chunk);
   p->splits = static_cast<int>(S);
   p->chunk = static_cast<int>(chunk);
+  p->ctas = 0;
   p->ws_bytes = 0;
+  p->ws_ml_off = 0;
   if (S > 1) {
     const size_t rows = static_cast<size_t>(batch) * num_q_heads * S;
-    const size_t o_bytes = (rows * g.D * sizeof(float) + 255) / 256 * 256;
-    p->ws_bytes = o_bytes + rows * 2 * sizeof(float);
+    p->ws_ml_off = (rows * g.D * sizeof(float) + 255) / 256 * 256;
+    p->ws_bytes = p->ws_ml_off + rows * 2 * sizeof(float);
   }
   return KVQ_OK;
 }
@@ -175,6 +291,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.chunk = a.plan.chunk;
   p.ring_split = a.plan.kernel == 2 ? a.plan.splits - 1 : -1;
   p.rows = a.batch * a.Hq;
+  p.batch = a.batch;
+  p.ctas = a.plan.ctas;
   p.act_fp16 = g.act_dtype == KVQ_DTYPE_FP16;
   p.scale_log2 = a.scale_log2;
   p.out = a.out;
@@ -191,7 +309,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     e = a.plan.kernel == 1 ? launch_decode_mma(a, p, s) : launch_decode_simt(a, p, s);
   }
   if (e != cudaSuccess) return e;
-  if (p.splits > 1) {
+  if (a.plan.kernel == 1) {
+    segment_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p);
+    e = cudaGetLastError();
+  } else if (p.splits > 1) {
     split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);
     e = cudaGetLastError();
   }

@@ -23,6 +23,8 @@ struct DecodeParams {
   int splits, chunk;
   int ring_split;            // INT4 with tensor-core pages: slot of the ring partial, else -1
   int rows;                  // batch * Hq
+  int batch;
+  int ctas;                  // page-balanced tensor-core kernel: its grid size, else 0
   int act_fp16;              // activations (q, ring) are fp16 rather than bf16
   float scale_log2;
   void* out;
@@ -65,6 +67,34 @@ __device__ __forceinline__ SeqInfo seq_info(const DecodeParams& p, int b, bool i
   }
   s.n = n;
   return s;
+}
+
+// ---------------------------------------------------------------- page-balanced schedule
+// The dense tensor-core kernel runs one CTA per resident slot.  The pages of all
+// (sequence, kv head) units, concatenated in the order (sequence, kv head, page), are cut
+// into ctas contiguous ranges of equal size: CTA c takes [P c / C, P (c + 1) / C).  A CTA
+// range crossing unit boundaries covers several segments (unit, CTA); each consumer warp
+// of the CTA writes one partial per segment it saw, into slot (unit + c) * kSegWarps + warp.
+// (Going from one segment to the next raises the unit index, the CTA index or both, so
+// unit + c never repeats and there are at most units + C - 1 segments.)
+constexpr int kSegWarps = 4;
+constexpr int kMmaCtas = 3 * kNumSMs;   // resident CTAs of the dense tensor-core kernel
+
+__device__ __forceinline__ long long range_start(long long P, int c, int C) {
+  return P * c / C;
+}
+
+// Pages of sequence b (0 when its entry is rejected).
+__device__ __forceinline__ int seq_pages(const DecodeParams& p, int b, bool report = false) {
+  return (seq_info(p, b, false, report).n + p.bs - 1) / p.bs;
+}
+
+// Tokens of a dense-cache sequence whose raw context length is n: n itself, or 0 when
+// seq_info would reject it (outside [0, max_context] or beyond the block table).
+__device__ __forceinline__ int dense_len(const DecodeParams& p, int n) {
+  const bool bad = n < 0 || n > p.max_context ||
+                   static_cast<long>(n) > static_cast<long>(p.max_blocks) * p.bs;
+  return bad ? 0 : n;
 }
 
 // Physical block of page `page` of sequence b, or -1 (counted) when out of range.

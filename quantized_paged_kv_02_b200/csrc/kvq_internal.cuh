@@ -77,14 +77,17 @@ cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int
 cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float* out,
                              cudaStream_t s);
 
-// Split-K plan of the decode kernels: grid (splits, heads-tiles, batch), chunk tokens each.
+// Plan of the decode kernels.  SIMT and INT4: grid (splits, heads-tiles, batch), chunk
+// tokens each.  Dense tensor-core kernel: ctas CTAs over page-balanced ranges.
 struct DecodePlan {
-  int kernel;        // 0 = SIMT, 1 = tensor-core (mma.sync)
+  int kernel;        // 0 = SIMT, 1 = tensor-core (mma.sync), 2 = INT4 tensor-core + ring
   int g;             // query heads per kv head
   int g_tile;        // query heads one CTA covers
-  int splits;        // S
+  int splits;        // S (kernels 0 and 2)
   int chunk;         // tokens per split (multiple of the block size)
-  size_t ws_bytes;   // workspace bytes (0 when splits == 1)
+  int ctas;          // kernel 1: grid size
+  size_t ws_bytes;   // workspace bytes (0 when a single split writes the output)
+  size_t ws_ml_off;  // byte offset of the (max, sum) array inside the workspace
 };
 
 kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_context,
@@ -104,8 +107,8 @@ struct DecodeArgs {
   float scale_log2;          // softmax scale * log2(e)
   void* out;
   int out_dtype;
-  float* ws_o;               // [B][Hq][S][D]
-  float* ws_ml;              // [B][Hq][S][2]
+  float* ws_o;               // partial outputs (layout per kernel)
+  float* ws_ml;              // partial (max, sum) pairs
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

@@ -82,3 +82,37 @@ def assert_same_cache(gc, oc):
     if oc.residual is not None:
         np.testing.assert_array_equal(pool_bytes(gc.residual, gc.sizes[3]),
                                       oc.residual.reshape(-1).view(np.uint8))
+
+
+def single_sequence(w, b):
+    """Workload holding only sequence b of w (batch 1, blocks 0..n-1 of a pool of its own).
+
+    Quantization works row by row (per token and head; INT4 keys per 64-row group of one
+    sequence), so the oracle's codes for this workload equal those of sequence b in the
+    full cache, and its attention output is output row b of the full batch.  Used to
+    check full-size runs on sampled sequences."""
+    import dataclasses
+    s = w.spec
+    r0, r1 = int(w.seq_start[b]), int(w.seq_start[b + 1])
+    n = r1 - r0
+    int4 = s.cache_dtype == "int4"
+    paged = inputs.INT4_GROUP * (max(n - inputs.RESIDUAL_LEN, 0) // inputs.INT4_GROUP) if int4 else n
+    nblk = max(-(-paged // s.block_size), 1)
+    pos = torch.arange(n, dtype=torch.int32)
+    slots = torch.full((n,), -1, dtype=torch.int32)
+    slots[:paged] = pos[:paged]                    # block j holds positions [j*bs, (j+1)*bs)
+    positions = seq_ids = None
+    if int4:
+        positions = torch.full((n,), -1, dtype=torch.int32)
+        positions[paged:] = pos[paged:]
+        seq_ids = torch.full((n,), -1, dtype=torch.int32)
+        seq_ids[paged:] = 0
+    cpu = lambda t: None if t is None else t.cpu()
+    return inputs.Workload(
+        spec=dataclasses.replace(s, batch=1, lens=[n], len_range=None),
+        context_lens=torch.tensor([n], dtype=torch.int32),
+        k=w.k[r0:r1].cpu(), v=w.v[r0:r1].cpu(), q=w.q[b:b + 1].cpu(),
+        seq_start=torch.tensor([0, n], dtype=torch.int64),
+        block_tables=torch.arange(nblk, dtype=torch.int32)[None],
+        num_blocks=nblk, slot_mapping=slots, seq_ids=seq_ids, positions=positions,
+        warmup_k=cpu(w.warmup_k), warmup_v=cpu(w.warmup_v))

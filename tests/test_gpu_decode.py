@@ -137,3 +137,38 @@ def test_zero_query_gives_mean_of_values():
         K, V = oc.gather(w.block_tables.numpy()[b], n)
         for hq in range(w.spec.num_q_heads):
             np.testing.assert_allclose(got[b, hq], V[hq // g].mean(axis=0), atol=1e-5, rtol=0)
+
+
+# Length mixes for the page-balanced tensor-core schedule: (a) fewer pages than CTAs, so
+# most CTAs are empty and every unit is split page by page across CTAs; (b) one long
+# sequence spanning a few hundred CTAs between short and empty ones.
+MIXES = {
+    "sparse": [0, 1, 16, 17, 0, 33, 2, 0, 5, 48, 0, 31],
+    "one-long": [4000, 3, 0, 700, 16],
+}
+KINDS = {
+    "int8": ("int8", "per_token_head"),
+    "fp8": ("fp8", "per_head"),
+    "bf16": ("bf16", "none"),
+}
+
+
+@pytest.mark.parametrize("mix", sorted(MIXES))
+@pytest.mark.parametrize("kind", sorted(KINDS))
+def test_balanced_schedule_length_mixes(kind, mix):
+    cd, mode = KINDS[kind]
+    lens = MIXES[mix]
+    spec = inputs.Spec("mix-%s-%s" % (kind, mix), cd, "bf16", mode, len(lens), 8, 2, 128, 16,
+                       lens=lens, slack_blocks=3, seed=21)
+    w = inputs.from_spec(spec)
+    static = helpers.oracle_static_scales(w)
+    oc = helpers.oracle_cache(w, static)
+    gc = helpers.gpu_cache(w, static=static)
+    got = _decode(gc, w).cpu().numpy().astype(np.float64)
+    want = _oracle(oc, w)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(got[b] == 0)
+    err = np.abs(got - want).max()
+    assert err <= TOL, err
+    assert gc.read_fault() == (0, 0)

@@ -129,6 +129,28 @@ def test_e4m3_encode_matches_exact_rounding_and_torch_in_range():
     np.testing.assert_array_equal(codes, ref)
 
 
+def test_e4m3_encode_equals_brute_force_nearest():
+    """The neighbour search against the plain definition: distance to all 127
+    magnitudes, nearest wins, a tie goes to the even code."""
+    rng = np.random.default_rng(16)
+    t = fp.e4m3_decode_table()[:127]
+    r = np.concatenate([
+        _rand_f32(rng, 20000, -14, 10),
+        ((t[:-1] + t[1:]) / 2).astype(np.float32),
+        np.nextafter(((t[:-1] + t[1:]) / 2).astype(np.float32), np.float32(0)),
+        np.nextafter(((t[:-1] + t[1:]) / 2).astype(np.float32), np.float32(np.inf)),
+        t.astype(np.float32), np.float32([0.0, 448.0, 464.0, 1e30])])
+    r = np.concatenate([r, -r])
+    a = np.minimum(np.abs(r.astype(np.float64)), 448.0)[:, None]
+    dist = np.abs(a - t[None, :])
+    hits = dist == dist.min(axis=1, keepdims=True)
+    two = hits.sum(axis=1) > 1
+    idx = np.arange(127)[None, :]
+    want = np.where(two, np.argmax(hits & (idx % 2 == 0), axis=1), np.argmax(hits, axis=1))
+    want = want.astype(np.uint8) | np.where(np.signbit(r), 0x80, 0).astype(np.uint8)
+    np.testing.assert_array_equal(fp.e4m3_encode(r), want)
+
+
 def test_e4m3_saturation_and_signed_zero():
     r = np.array([448.0, 449.0, 464.0, 500.0, 1e30, -1e30, -464.0, 2.0 ** -10,
                   3 * 2.0 ** -10, -1e-30, -0.0, 0.0], np.float32)
