@@ -41,6 +41,7 @@ namespace kvq {
 namespace {
 
 constexpr int kConsumers = 4;
+constexpr int kIssueLanes = 8;    // producer lanes that issue copies side by side
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kD = 128;
 constexpr float kRescale = 8.f;   // log2 headroom before the running max is re-reduced
@@ -65,15 +66,17 @@ struct Layout {
   // 1 KiB of it reserved per CTA); bytes in flight are what keeps HBM busy
   static constexpr int kSmemPerCta = 228 * 1024 / 3 - 1024;
   static constexpr int kFixed = 1024 + 16 + 4 * 4 + 32 * 4;  // alignment, range, batch ids
-  static constexpr int kStages = (kSmemPerCta - kFixed) / (STAGE + 32) / 2 * 2;
+  static constexpr int kStages = (kSmemPerCta - kFixed) / (STAGE + 32) / kConsumers * kConsumers;
   static constexpr int TILES = kStages * STAGE;
   static constexpr int BARS = kStages * 2 * 8;
   static constexpr int META = kStages * 16 + 16 + 32 * 4;  // page records, range, batch ids
   static constexpr int BYTES = 1024 + TILES + BARS + META;
   static_assert(kStages >= 4 && BYTES <= kSmemPerCta, "ring fits 3 CTAs per SM");
-  // consumers take pages round-robin; a stage's successive rounds then alternate between
-  // at most two warps, which the consumer wait relies on
-  static_assert((2 * kStages) % kConsumers == 0, "even ring depth");
+  // Consumers take pages round-robin, and every round of a stage must go to the same
+  // warp: a warp waiting for round r of a stage whose round r-1 belonged to another warp
+  // (and has not landed yet) would see the parity of round r-2 as complete.
+  static_assert(kStages % kConsumers == 0, "ring depth is a multiple of the consumers");
+  static_assert(kStages >= kIssueLanes, "one issue chunk never waits on its own stages");
   static_assert(REC_ROWS <= 256, "TMA box height");
 };
 
@@ -201,33 +204,36 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         record_fault(p.fault, KVQ_FAULT_BLOCK);
         blk = -1;
       }
-      // lane 0 alone issues the batch: per page one wait for the stage, one record,
-      // one copy, with no warp-wide step in between
+      // lanes 0..7 issue eight pages at once, each: wait for its stage, write the page
+      // record, one copy.  The barrier operations of one page form a dependent chain
+      // of a few hundred cycles; issuing pages side by side overlaps those chains, which
+      // is what lets 4 KiB copies keep pace with HBM.
       ids[lane] = blk;
       __syncwarp();
-      if (lane == 0) {
-        for (int k = 0; k < cur.cnt; ++k) {
-          const int bk = ids[k];
-          const int s = issued % kStages;
-          const int round = issued / kStages;
+      for (int k0 = 0; k0 < cur.cnt && ok_run; k0 += kIssueLanes) {
+        const int n = min(kIssueLanes, cur.cnt - k0);
+        bool ok_lane = true;
+        if (lane < n) {
+          const int i = issued + lane;
+          const int s = i % kStages, round = i / kStages;
+          const int bk = ids[k0 + lane];
           if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) {
             record_fault(p.fault, KVQ_FAULT_TIMEOUT);
-            ok_run = false;
-            break;
-          }
-          meta[s] = make_int4(cur.u, cur.pg0 + k, cur.nb, bk >= 0);
-          if (bk >= 0) {
-            // the whole record of (block, kv head) in one copy
-            mbar_arrive_expect_tx(&full[s], stage_bytes);
-            tma_load_2d(tiles + s * STAGE, &tmap, &full[s], 0, (bk * p.H + cur.kvh) * L::REC_ROWS);
+            ok_lane = false;
           } else {
-            mbar_arrive(&full[s]);
+            meta[s] = make_int4(cur.u, cur.pg0 + k0 + lane, cur.nb, bk >= 0);
+            if (bk >= 0) {
+              // the whole record of (block, kv head) in one copy
+              mbar_arrive_expect_tx(&full[s], stage_bytes);
+              tma_load_2d(tiles + s * STAGE, &tmap, &full[s], 0, (bk * p.H + cur.kvh) * L::REC_ROWS);
+            } else {
+              mbar_arrive(&full[s]);
+            }
           }
-          ++issued;
         }
+        ok_run = __all_sync(0xffffffffu, ok_lane);
+        issued += n;
       }
-      ok_run = __shfl_sync(0xffffffffu, ok_run, 0);
-      issued = __shfl_sync(0xffffffffu, issued, 0);
       cur = nxt;
     }
     // wait until every copy this CTA issued has landed before the CTA can exit
@@ -397,19 +403,8 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
 
   for (int i = warp; i < npages; i += kConsumers) {
     const int s = i % kStages;
-    const int round = i / kStages;
-    // Stage s holds rounds r-1 and r for pages i - kStages and i.  When kStages is not a
-    // multiple of the consumer count, round r-1 belonged to another warp and may not have
-    // landed yet, so the parity of round r alone would be ambiguous (the last completed
-    // phase of that parity is r-2).  Waiting first for round r-1 to be released (its
-    // own round r-2 was released by this warp) makes the full wait unambiguous.
-    bool ok = true;
-    if constexpr (kStages % kConsumers != 0) {
-      if (round > 0) ok = mbar_wait(&empty[s], (round - 1) & 1);
-    }
-    if (ok) ok = mbar_wait(&full[s], round & 1);
     // all lanes wait; the decision is made warp-uniform before any shuffle below
-    if (!__all_sync(0xffffffffu, ok)) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kStages) & 1))) {
       if (lane == 0) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
       break;
     }
