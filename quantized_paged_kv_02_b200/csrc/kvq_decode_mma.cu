@@ -1,4 +1,4 @@
-// Paged split-K decode attention on tensor cores, for GQA groups of 3..8 query heads
+// Paged split-K decode attention on tensor cores, for GQA groups of 1..8 query heads
 // (head_dim 128, dense caches: INT8, FP8 E4M3, BF16, FP16).
 //
 // Schedule: one CTA per resident slot (3 per SM).  The pages of all (sequence, kv head)
@@ -709,7 +709,9 @@ static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 }
 
 // Tensor map over the pages pool viewed as rows of 128 bytes; one box is one record
-// (rec_rows rows), copied with 128-byte swizzle.
+// (rec_rows rows), copied with 128-byte swizzle.  L2 fills are promoted to 256 bytes only
+// when records are whole 256-byte units: a 4224-byte record (33 rows) would otherwise pull
+// 128 bytes of its neighbour into L2 at every other record.
 bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows) {
   auto enc = encoder();
   if (enc == nullptr) return false;
@@ -719,12 +721,16 @@ bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows)
   cuuint32_t es[2] = {1, 1};
   const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           rec_rows % 2 == 0 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                             : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return res == CUDA_SUCCESS;
 }
 
 bool mma_supported(const Geometry& g, int groups) {
-  if (g.D != kD || groups < 3 || groups > 8) return false;
+  // any group of 1..8 query heads fills (part of) the N = 8 side of the tiles; the kernel
+  // is bound by moving pages, so a partly empty tile costs little
+  if (g.D != kD || groups < 1 || groups > 8) return false;
   if (g.bs != 16) return false;   // 8 stages of 16-token tiles fit shared memory 3 CTAs/SM
   switch (g.cache_dtype) {
     case KVQ_DTYPE_INT8:

@@ -79,7 +79,13 @@ def test_workspace_plan_is_deterministic(lib):
     d = _desc(kvq, num_kv_heads=8)
     a = kvq.kvq_decode_workspace_size(d, 24, 64, 16384)
     assert a == kvq.kvq_decode_workspace_size(d, 24, 64, 16384) and a > 0
-    assert kvq.kvq_decode_workspace_size(d, 1, 8, 16) == 0       # one split: no workspace
+    # the CUDA-core kernel (head_dim 64) with a single split writes the output directly
+    assert kvq.kvq_decode_workspace_size(_desc(kvq, num_kv_heads=8, head_dim=64), 1, 8, 16) == 0
+    # the tensor-core kernel always merges per-warp partials through the workspace:
+    # (units + CTAs - 1) * 4 partials of g heads, each D floats plus (max, sum)
+    ctas, D, g, units = 3 * 148, 128, 1, 8
+    heads = (units + ctas - 1) * 4 * g
+    assert kvq.kvq_decode_workspace_size(d, 1, 8, 16) == (heads * D * 4 + 255) // 256 * 256 + heads * 8
     with pytest.raises(kvq.KVQError):
         kvq.kvq_decode_workspace_size(d, 2, 12, 100)              # 12 not a multiple of 8
 
