@@ -8,6 +8,7 @@
 #include <algorithm>
 
 #include "kvq_decode_common.cuh"
+#include "kvq_ptx.cuh"
 
 namespace kvq {
 namespace {
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
 // four at a time so their loads overlap.
 __global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
   constexpr int C = kMmaCtas;
+  griddep_wait();                      // the partials of the decode kernel
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);   // b * Hq + hq
   const int lane = threadIdx.x & 31;
   if (row >= p.rows) return;
@@ -310,8 +312,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   }
   if (e != cudaSuccess) return e;
   if (a.plan.kernel == 1) {
-    segment_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p);
-    e = cudaGetLastError();
+    e = launch_dependent(segment_reduce_kernel, dim3((a.batch * a.Hq + 7) / 8), dim3(256), 0, s, p);
   } else if (p.splits > 1) {
     split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);
     e = cudaGetLastError();

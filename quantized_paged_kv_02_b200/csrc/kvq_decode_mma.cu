@@ -108,6 +108,9 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   constexpr int C = kMmaCtas;                              // the grid (page partition)
   const int cta = blockIdx.x;
 
+  // inputs (pages, q, tables, lengths) may come from the kernel just before this one
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -682,8 +685,8 @@ cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s)
   CUtensorMap tm;
   const long rows = static_cast<long>(a.geo.NB) * a.geo.H * L::REC_ROWS;
   if (!make_pages_map(&tm, a.c->pages, rows, L::REC_ROWS)) return cudaErrorInvalidValue;
-  decode_mma_kernel<CD, BS, PT><<<a.plan.ctas, kThreads, L::BYTES, s>>>(p, tm);
-  return cudaGetLastError();
+  return launch_dependent(decode_mma_kernel<CD, BS, PT>, dim3(a.plan.ctas), dim3(kThreads), L::BYTES,
+                          s, p, tm);
 }
 
 template <int CD, bool PT>

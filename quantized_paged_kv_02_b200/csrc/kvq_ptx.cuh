@@ -56,6 +56,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// ------------------------------------------------------------------ dependent launch
+// A kernel launched with programmatic stream serialization may start before the kernel
+// ahead of it in the stream has finished.  griddep_wait() blocks until that kernel has
+// completed and its writes are visible; call it before touching memory it may have
+// written.  griddep_launch_dependents() lets the next such kernel start early.  Both are
+// no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {

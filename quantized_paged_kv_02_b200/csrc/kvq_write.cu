@@ -13,6 +13,7 @@
 // 的分布不一定相同"), with the affine form of [P-prod] "量化不是简单截断精度".  Rows that
 // belong to no block are copied unquantized into the residual ring.
 #include "kvq_internal.cuh"
+#include "kvq_ptx.cuh"
 
 namespace kvq {
 namespace {
@@ -49,6 +50,7 @@ __device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
 
 template <typename TA, int CD, int D>
 __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
+  griddep_launch_dependents();   // a decode launched after this one may start its set-up
   constexpr int LPR = D * 2 / 16;   // lanes per row
   constexpr int RPW = 32 / LPR;     // rows per warp
   const int lane = threadIdx.x & 31;
@@ -144,6 +146,7 @@ __device__ __forceinline__ int int4_code(float x, const Int4Group& g) {
 
 template <typename TA, int D>
 __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
+  griddep_launch_dependents();   // a decode launched after this one may start its set-up
   constexpr int G = 64;
   __shared__ float xs[G][D + 1];
   __shared__ __align__(16) uint8_t cs[G][D];
