@@ -392,6 +392,34 @@ def main_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms, dms = t.tolist()
 
+    # the same step as one call (kvq_append_decode_attention), dense caches only
+    fused = None
+    if s.cache_dtype != "int4" and K > 0:
+        def fused_step():
+            kvq.kvq_append_decode_attention(cache.desc, new["k"], new["v"], w.q, w.block_tables,
+                                            w.context_lens, max_ctx, out, ws)
+        for _ in range(3):
+            l2.flush()
+            fused_step()
+        fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        torch.cuda.synchronize()
+        for a, b2 in fev:
+            l2.flush()
+            a.record(stream)
+            fused_step()
+            b2.record(stream)
+        torch.cuda.synchronize()
+        fms = statistics.mean(a.elapsed_time(b2) for a, b2 in fev)
+        if world > 1:
+            t = torch.tensor([fms], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            fms = t.item()
+        fused = {"value": round(world * step_bytes / (fms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                 "ms_per_step": round(fms, 5), "tokens_per_s": round(world * B / (fms * 1e-3), 1),
+                 "frac_of_peak": round(step_bytes / (fms * 1e-3) / 1e9 / hbm_peak()[0], 4),
+                 "call": "kvq_append_decode_attention (append step fused into the decode kernel)"}
+
     # end to end through the C ABI: host inputs in pinned memory, copies inside the region
     E = args.e2e_steps
     h = {k2: new[k2].cpu().pin_memory() for k2 in ("k", "v", "slots")}
@@ -459,6 +487,7 @@ def main_ours(args):
         "e2e": {"value": round(world * step_bytes / (e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "append_decode": fused,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }

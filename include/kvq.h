@@ -239,6 +239,32 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int 
                                 size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * kvq_append_decode_attention - one serving step in one call: store this step's K/V row
+ * of every sequence, then attend (kvq_write followed by kvq_decode_attention).
+ *   k_new, v_new  act_dtype [batch][H][D], device: the new token's key and value rows of
+ *                 each sequence.  Row b is stored at position context_lens[b] - 1 of
+ *                 sequence b, i.e. slot block_tables[b][(len-1)/bs]*bs + (len-1)%bs, with
+ *                 exactly the codes and scales kvq_write would store there; a sequence with
+ *                 context_lens[b] == 0 stores nothing.  Then decode attends to positions
+ *                 p < context_lens[b], the new one included.
+ *   Other arguments as kvq_decode_attention (the workspace size is the same; there is no
+ *   seq_ids argument).
+ *   Dense caches (INT8, FP8 E4M3, BF16, FP16) with block_size 16 and head_dim 128 only;
+ *   other caches return KVQ_ERR_UNSUPPORTED (use kvq_write + kvq_decode_attention).
+ *   The pages quantize on write and dequantize inside attention ([P-vLLM]
+ *   "PagedAttention与KV Cache量化协同工作原理"); doing both in one launch saves a kernel and
+ *   its launch per step.  Results equal kvq_write followed by kvq_decode_attention, bit
+ *   for bit.
+ */
+kvq_status kvq_append_decode_attention(const kvq_cache_desc* cache, const void* k_new,
+                                       const void* v_new, const void* q, int batch,
+                                       int num_q_heads, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       int max_context, float softmax_scale, void* out,
+                                       int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream);
+
+/*
  * Size of the device scratch array used by kvq_decode_attention_noalloc (16 MiB).  Every
  * GPU that loads the library reserves this much for the life of the process.
  */

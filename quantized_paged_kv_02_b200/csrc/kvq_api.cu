@@ -87,6 +87,64 @@ static kvq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : 
 
 using namespace kvq;
 
+namespace {
+
+// Shared by kvq_decode_attention and kvq_append_decode_attention (k_new / v_new null for
+// the former).
+kvq_status decode_entry(const kvq_cache_desc* c, const void* k_new, const void* v_new,
+                        const void* q, int batch, int num_q_heads, const int32_t* block_tables,
+                        int max_blocks_per_seq, const int32_t* context_lens,
+                        const int32_t* seq_ids, int max_context, float softmax_scale, void* out,
+                        int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  Geometry g;
+  kvq_status st = validate_desc(c, &g);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 || max_context < 0 ||
+      max_blocks_per_seq < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (out_dtype != KVQ_DTYPE_BF16 && out_dtype != KVQ_DTYPE_FP16 && out_dtype != KVQ_DTYPE_FP32)
+    return KVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  const bool append = k_new != nullptr || v_new != nullptr;
+  if (append && (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new)))
+    return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (q == nullptr || block_tables == nullptr || context_lens == nullptr || out == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return KVQ_ERR_INVALID_ARG;
+  DecodeArgs a{};
+  a.c = c;
+  a.geo = g;
+  st = plan_decode(g, batch, num_q_heads, max_context, &a.plan);
+  if (st != KVQ_OK) return st;
+  // the append step lives in the tensor-core kernel's producer
+  if (append && a.plan.kernel != 1) return KVQ_ERR_UNSUPPORTED;
+  if (a.plan.ws_bytes > 0) {
+    if (workspace == nullptr || workspace_bytes < a.plan.ws_bytes || !aligned16(workspace))
+      return KVQ_ERR_INVALID_ARG;
+    a.ws_o = static_cast<float*>(workspace);
+    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + a.plan.ws_ml_off);
+  }
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.batch = batch;
+  a.Hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_blocks = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.seq_ids = seq_ids;
+  a.max_context = max_context;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(g.D));
+  a.scale_log2 = scale * kLog2e;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_decode(a, stream));
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* kvq_status_string(kvq_status s) {
@@ -150,49 +208,29 @@ kvq_status kvq_decode_workspace_size(const kvq_cache_desc* c, int batch, int num
   return KVQ_OK;
 }
 
+
 kvq_status kvq_decode_attention(const kvq_cache_desc* c, const void* q, int batch,
                                 int num_q_heads, const int32_t* block_tables,
                                 int max_blocks_per_seq, const int32_t* context_lens,
                                 const int32_t* seq_ids, int max_context, float softmax_scale,
                                 void* out, int32_t out_dtype, void* workspace,
                                 size_t workspace_bytes, cudaStream_t stream) {
-  Geometry g;
-  kvq_status st = validate_desc(c, &g);
-  if (st != KVQ_OK) return st;
-  if (batch < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 || max_context < 0 ||
-      max_blocks_per_seq < 1)
-    return KVQ_ERR_INVALID_ARG;
-  if (out_dtype != KVQ_DTYPE_BF16 && out_dtype != KVQ_DTYPE_FP16 && out_dtype != KVQ_DTYPE_FP32)
-    return KVQ_ERR_INVALID_ARG;
-  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
-  if (batch == 0) return KVQ_OK;
-  if (q == nullptr || block_tables == nullptr || context_lens == nullptr || out == nullptr)
-    return KVQ_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(out)) return KVQ_ERR_INVALID_ARG;
-  DecodeArgs a{};
-  a.c = c;
-  a.geo = g;
-  st = plan_decode(g, batch, num_q_heads, max_context, &a.plan);
-  if (st != KVQ_OK) return st;
-  if (a.plan.ws_bytes > 0) {
-    if (workspace == nullptr || workspace_bytes < a.plan.ws_bytes || !aligned16(workspace))
-      return KVQ_ERR_INVALID_ARG;
-    a.ws_o = static_cast<float*>(workspace);
-    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + a.plan.ws_ml_off);
-  }
-  a.q = q;
-  a.batch = batch;
-  a.Hq = num_q_heads;
-  a.block_tables = block_tables;
-  a.max_blocks = max_blocks_per_seq;
-  a.context_lens = context_lens;
-  a.seq_ids = seq_ids;
-  a.max_context = max_context;
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(g.D));
-  a.scale_log2 = scale * kLog2e;
-  a.out = out;
-  a.out_dtype = out_dtype;
-  return from_cuda(launch_decode(a, stream));
+  return decode_entry(c, nullptr, nullptr, q, batch, num_q_heads, block_tables, max_blocks_per_seq,
+                      context_lens, seq_ids, max_context, softmax_scale, out, out_dtype, workspace,
+                      workspace_bytes, stream);
+}
+
+kvq_status kvq_append_decode_attention(const kvq_cache_desc* c, const void* k_new,
+                                       const void* v_new, const void* q, int batch,
+                                       int num_q_heads, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       int max_context, float softmax_scale, void* out,
+                                       int32_t out_dtype, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream) {
+  if (k_new == nullptr || v_new == nullptr) return KVQ_ERR_INVALID_ARG;
+  return decode_entry(c, k_new, v_new, q, batch, num_q_heads, block_tables, max_blocks_per_seq,
+                      context_lens, nullptr, max_context, softmax_scale, out, out_dtype, workspace,
+                      workspace_bytes, stream);
 }
 
 kvq_status kvq_dequant(const kvq_cache_desc* c, const int32_t* block_ids, int n_blocks,

@@ -302,6 +302,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.ws_o = a.ws_o;
   p.ws_ml = a.ws_ml;
   p.fault = a.c->fault;
+  p.k_new = a.k_new;
+  p.v_new = a.v_new;
+  p.pages_w = a.k_new != nullptr ? static_cast<uint8_t*>(a.c->pages) : nullptr;
   if (a.batch == 0) return cudaSuccess;
   cudaError_t e;
   if (a.plan.kernel == 2) {

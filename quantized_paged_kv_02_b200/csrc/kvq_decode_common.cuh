@@ -32,6 +32,11 @@ struct DecodeParams {
   float* ws_o;               // [B][Hq][S][D]
   float* ws_ml;              // [B][Hq][S][2]  (max, sum) in the log2 domain
   int32_t* fault;
+  // append step (kvq_append_decode_attention), else null: this step's K / V row of every
+  // sequence, [B][H][D] act dtype, stored at position context_lens[b] - 1 before decode
+  const void* k_new;
+  const void* v_new;
+  uint8_t* pages_w;          // the pool, writable (append step only)
 };
 
 struct SeqInfo {

@@ -172,6 +172,30 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       npb = (nb + BS - 1) / BS;
       n_ahead = b + 1 < p.batch ? p.lens[b + 1] : 0;
     }
+    // Append step: quantize this step's K and V rows of (sequence b, kv head) into the
+    // unit's last page, exactly as kvq_write stores them (lanes 0-15 the K row, 16-31 the
+    // V row), before that page is copied.  Only this CTA reads that page.
+    auto append_row = [&](int bq, int kvh, int n) {
+      const int pos = n - 1;
+      const int blk = p.tables[static_cast<long>(bq) * p.max_blocks + pos / BS];
+      if (blk < 0 || blk >= p.NB) return;     // the page is skipped (and counted) when read
+      const int kv = lane >> 4, l = lane & 15;
+      const uint4 u = reinterpret_cast<const uint4*>(kv ? p.v_new : p.k_new)
+          [((static_cast<long>(bq) * p.H + kvh) * kD) / 8 + l];
+      uint8_t* rec = p.pages_w + (static_cast<long>(blk) * p.H + kvh) * L::REC;
+      float static_s = 0.f;
+      if constexpr (!PT && Code<CD>::B == 1) {
+        const float* sp = kv ? p.v_static : p.k_static;
+        static_s = sp[p.mode == KVQ_SCALE_PER_HEAD ? kvh : 0];
+      }
+      if (p.act_fp16)
+        quantize_row_part<__half, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT, static_s);
+      else
+        quantize_row_part<__nv_bfloat16, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
+                                                 static_s);
+      fence_proxy_async_global();
+      __syncwarp();
+    };
     struct Batch { int u, kvh, pg0, cnt, nb, raw; };
     auto next_batch = [&]() {
       Batch t{0, 0, 0, 0, 0, -1};
@@ -194,6 +218,7 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       t.cnt = static_cast<int>(min(min(static_cast<long long>(npb - t.pg0), end - gp), 32LL));
       t.u = b * p.H + t.kvh;
       t.nb = nb;
+      if (p.k_new != nullptr && t.pg0 + t.cnt == npb) append_row(b, t.kvh, nb);
       // issued now, checked when the batch is copied (one batch later)
       if (lane < t.cnt) t.raw = p.tables[static_cast<long>(b) * p.max_blocks + t.pg0 + lane];
       gp += t.cnt;

@@ -56,6 +56,64 @@ __device__ __forceinline__ float e4m3_to_float(uint8_t c) {
 // Binary32 quotient with round-to-nearest-even, independent of -prec-div.
 __device__ __forceinline__ float div_rn(float a, float b) { return __fdiv_rn(a, b); }
 
+// ------------------------------------------------------------------ dense quantizers
+// (kvq_write, and the append step of kvq_append_decode_attention: one definition, so the
+// two store identical bytes)
+template <int CD> struct QMax;
+template <> struct QMax<KVQ_DTYPE_INT8> { static constexpr float v = 127.f; };
+template <> struct QMax<KVQ_DTYPE_FP8_E4M3> { static constexpr float v = 448.f; };
+
+__device__ __forceinline__ uint8_t quant_int8(float x, float s) {
+  if (s == 0.f) return 0;
+  int q = __float2int_rn(div_rn(x, s));
+  q = max(-128, min(127, q));
+  return static_cast<uint8_t>(static_cast<int8_t>(q));
+}
+
+__device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
+  if (s == 0.f) return 0;
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(div_rn(x, s), __NV_SATFINITE, __NV_E4M3));
+}
+
+// One lane's share of quantizing one row (one token, one kv head, K or V) into its page
+// record.  A row is handled by D*2/16 consecutive lanes (a power of two dividing 32);
+// lane l holds activation elements [8l, 8l+8) in `u`.  `write` false: the lane joins the
+// shuffles but stores nothing.  Per-token modes reduce max|x| over the row's lanes and
+// store the float32 scale; static modes use `static_s`.  INT8: [P-mem] §3.1 对称量化算法
+// (scale = max|x|/127, q = clamp(round(x/scale), -128, 127)); FP8: [P-vLLM]
+// "KV Cache量化策略" (E4M3 storage with a scale).
+template <typename TA, int CD, int D>
+__device__ __forceinline__ void quantize_row_part(const uint4& u, int l, bool write, int kv, int off,
+                                                  int bs, uint8_t* rec, int off_v, int off_s,
+                                                  bool per_token, float static_s) {
+  constexpr int LPR = D * 2 / 16;
+  constexpr int ROWB = (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) ? 2 * D : D;
+  uint8_t* dst_row = rec + (kv ? off_v : 0) + off * ROWB;
+  if constexpr (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) {
+    if (write) *reinterpret_cast<uint4*>(dst_row + l * 16) = u;
+  } else {
+    float x[8];
+    unpack8<TA>(u, x);
+    float s = static_s;
+    if (per_token) {
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      s = div_rn(m, QMax<CD>::v);
+      if (write && l == 0) reinterpret_cast<float*>(rec + off_s)[(kv ? bs : 0) + off] = s;
+    }
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
+      if (i < 4) w0 |= c << (8 * i); else w1 |= c << (8 * (i - 4));
+    }
+    if (write) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w0, w1);
+  }
+}
+
 // ------------------------------------------------------------------ host helpers
 struct Geometry {
   int cache_dtype, act_dtype, scale_mode;
@@ -100,6 +158,8 @@ struct DecodeArgs {
   Geometry geo;
   DecodePlan plan;
   const void* q;
+  const void* k_new;         // append step: [B][H][D] act dtype, else null
+  const void* v_new;
   int batch, Hq;
   const int32_t* block_tables;
   int max_blocks;

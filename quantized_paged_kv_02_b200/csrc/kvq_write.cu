@@ -32,22 +32,6 @@ struct WriteParams {
   int32_t* fault;
 };
 
-template <int CD> struct QMax;
-template <> struct QMax<KVQ_DTYPE_INT8> { static constexpr float v = 127.f; };
-template <> struct QMax<KVQ_DTYPE_FP8_E4M3> { static constexpr float v = 448.f; };
-
-__device__ __forceinline__ uint8_t quant_int8(float x, float s) {
-  if (s == 0.f) return 0;
-  int q = __float2int_rn(div_rn(x, s));
-  q = max(-128, min(127, q));
-  return static_cast<uint8_t>(static_cast<int8_t>(q));
-}
-
-__device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
-  if (s == 0.f) return 0;
-  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(div_rn(x, s), __NV_SATFINITE, __NV_E4M3));
-}
-
 template <typename TA, int CD, int D>
 __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
   griddep_launch_dependents();   // a decode launched after this one may start its set-up
@@ -75,36 +59,11 @@ __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
   const int off = write ? slot % p.bs : 0;
   // record of (block, head); this row's codes and (per-token) scale inside it
   uint8_t* rec = p.pages + (static_cast<long>(blk) * p.H + h) * p.record;
-  constexpr int ROWB = (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) ? 2 * D : D;
-  uint8_t* dst_row = rec + (kv ? p.off_v : 0) + off * ROWB;
-  float* scale_slot = reinterpret_cast<float*>(rec + p.off_s) + (kv ? p.bs : 0) + off;
-
-  if constexpr (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) {
-    if (write) *reinterpret_cast<uint4*>(dst_row + l * 16) = u;
-  } else {
-    float x[8];
-    unpack8<TA>(u, x);
-    float s;
-    if (p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD) {
-      float m = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
-#pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      s = div_rn(m, QMax<CD>::v);
-      if (write && l == 0) *scale_slot = s;
-    } else {
-      const float* sp = kv ? p.v_static : p.k_static;
-      s = sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0];
-    }
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
-      if (i < 4) w0 |= c << (8 * i); else w1 |= c << (8 * (i - 4));
-    }
-    if (write) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w0, w1);
-  }
+  const float* sp = kv ? p.v_static : p.k_static;
+  const bool is_static = p.scale_mode == KVQ_SCALE_PER_HEAD || p.scale_mode == KVQ_SCALE_PER_TENSOR;
+  const float static_s = is_static ? sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0] : 0.f;
+  quantize_row_part<TA, CD, D>(u, l, write, kv, off, p.bs, rec, p.off_v, p.off_s,
+                               p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD, static_s);
 }
 
 // ------------------------------------------------------------------ INT4 (KIVI)

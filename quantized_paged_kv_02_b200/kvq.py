@@ -24,7 +24,8 @@ STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "K
 FAULT_BITS = {"slot": 1, "block": 2, "context": 4, "seq": 8, "int4_run": 16, "timeout": 32}
 EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
-           "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc")
+           "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc",
+           "kvq_append_decode_attention")
 
 
 class CacheDesc(ctypes.Structure):
@@ -64,6 +65,8 @@ def _load():
         "kvq_calibrate_fp8_scales": (I, [P, I, I, I, ctypes.c_int32, P, P]),
         "kvq_read_device_fault": (I, [D, ctypes.POINTER(ctypes.c_int32), I, P]),
         "kvq_decode_attention_noalloc": (I, [D, P, I, I, P, I, P, P, I, F, P, ctypes.c_int32, P]),
+        "kvq_append_decode_attention": (I, [D, P, P, P, I, I, P, I, P, I, F, P, ctypes.c_int32, P,
+                                            Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +149,21 @@ def kvq_decode_attention(desc, q, block_tables, context_lens, max_context, out, 
         _ptr(_i32(context_lens)), _ptr(_i32(seq_ids)), int(max_context), float(softmax_scale),
         _ptr(out), DTYPE[out_dt], _ptr(workspace), ws_bytes, _stream(stream)),
         "kvq_decode_attention")
+    return out
+
+
+def kvq_append_decode_attention(desc, k_new, v_new, q, block_tables, context_lens, max_context,
+                                out, workspace=None, softmax_scale=0.0, stream=None):
+    """Store each sequence's new K/V row at position context_lens[b] - 1, then decode:
+    kvq_write followed by kvq_decode_attention in one launch (dense caches)."""
+    B, Hq, _ = q.shape
+    out_dt = {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[out.dtype]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.kvq_append_decode_attention(
+        ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _ptr(q), B, Hq, _ptr(_i32(block_tables)),
+        int(block_tables.shape[1]), _ptr(_i32(context_lens)), int(max_context),
+        float(softmax_scale), _ptr(out), DTYPE[out_dt], _ptr(workspace), ws_bytes,
+        _stream(stream)), "kvq_append_decode_attention")
     return out
 
 
@@ -241,6 +259,16 @@ class PagedKVCache:
             workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device) if n else None
         return kvq_decode_attention(self.desc, q, block_tables, context_lens, max_context, out,
                                     workspace, seq_ids, softmax_scale, stream)
+
+    def append_decode(self, k_new, v_new, q, block_tables, context_lens, max_context, out=None,
+                      out_dtype=torch.float32, workspace=None, softmax_scale=0.0, stream=None):
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        if workspace is None:
+            n = self.workspace_size(q.shape[0], q.shape[1], max_context)
+            workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device) if n else None
+        return kvq_append_decode_attention(self.desc, k_new, v_new, q, block_tables, context_lens,
+                                           max_context, out, workspace, softmax_scale, stream)
 
     def dequant(self, block_ids, stream=None):
         out = torch.empty((block_ids.numel(), 2, self.num_kv_heads, self.block_size, self.head_dim),
