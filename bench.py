@@ -37,6 +37,8 @@ WORKLOADS = {
               "block 16, FP8 E4M3 per-kv-head scales (256-token warm-up)",
     "c5-bf16": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
                "block 16, unquantized bf16 cache",
+    "c5-int8-pc": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
+                  "block 16, INT8 static per-(kv head, channel) scales (256-token warm-up)",
     "c2": "Llama-2-7B-shaped layer: batch 4, 32 heads MHA, head_dim 128, context 2048, block 16, "
           "INT8 per-token-head, 4 outlier channels x10 in K and V",
     "c3": "Llama-3-8B-shaped layer: batch 64, 32/8 heads, head_dim 128, context U[1024, 8192], "
@@ -272,6 +274,13 @@ def build_state(workload, device, seed, batch=0):
         sv = torch.empty(s.num_kv_heads, dtype=torch.float32, device=device)
         kvq.kvq_calibrate_fp8_scales(w.warmup_k, sk)
         kvq.kvq_calibrate_fp8_scales(w.warmup_v, sv)
+        static = (sk.cpu().numpy(), sv.cpu().numpy())
+    elif s.scale_mode == "per_channel":
+        qmax = 127.0 if s.cache_dtype == "int8" else 448.0
+        sk = torch.empty((s.num_kv_heads, s.head_dim), dtype=torch.float32, device=device)
+        sv = torch.empty_like(sk)
+        kvq.kvq_calibrate_channel_scales(w.warmup_k, qmax, sk)
+        kvq.kvq_calibrate_channel_scales(w.warmup_v, qmax, sv)
         static = (sk.cpu().numpy(), sv.cpu().numpy())
     c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
                          s.num_kv_heads, s.head_dim, device=device,
@@ -520,6 +529,11 @@ def main_reference(args):
         from oracle import quant
         static = (quant.fp8_calibrate(w.warmup_k.float().numpy()),
                   quant.fp8_calibrate(w.warmup_v.float().numpy()))
+    elif w.spec.scale_mode == "per_channel":
+        from oracle import quant
+        qmax = 127.0 if w.spec.cache_dtype == "int8" else 448.0
+        static = (quant.channel_calibrate(w.warmup_k.float().numpy(), qmax),
+                  quant.channel_calibrate(w.warmup_v.float().numpy(), qmax))
     rows = oracle_inputs(w, [(0, 0)])
     step = oracle_unit_step(w, rows, 0, 0, static)
     nbytes = unit_bytes(w, 0)

@@ -53,7 +53,10 @@
  *          INT4 codes pack two per byte: element 2i in the low nibble of byte i, element
  *          2i+1 in the high nibble.  Padding bytes at the end of a record are never written.
  *  k_scales, v_scales : static scales only - PER_HEAD: float32 [H] ([P-prod] "vLLM：从 FP8 KV
- *          Cache 开始试点": per-attention-head); PER_TENSOR: float32 [1].  Unused otherwise.
+ *          Cache 开始试点": per-attention-head); PER_TENSOR: float32 [1]; PER_CHANNEL: float32
+ *          [H][D], one scale per kv head and channel ([P-vLLM] "KV Cache量化策略：INT8与FP8
+ *          精度对比与选择": INT8 per-tensor or per-channel; [P-prod] "量化不是简单截断精度":
+ *          scales per tensor, head, channel, token or group).  Unused otherwise.
  *  residual : INT4 only.  act_dtype [max_seqs][2][H][residual_cap][D]: the newest tokens of
  *          each sequence kept unquantized ([P-prod] "Key 和 Value 的分布不一定相同": a
  *          fixed-size higher-precision residual of recent K/V).  Index 0 of the second
@@ -64,7 +67,7 @@
  * every "/" is an IEEE float32 division rounded to nearest-even)
  *  INT8  ([P-mem] §3.1 对称量化算法; [P-vLLM] "KV Cache量化策略"):
  *        dynamic: s = max_d |x_d| / 127  per (token, kv head), stored as float32;
- *        static : s = the caller's per-head or per-tensor scale;
+ *        static : s = the caller's per-head, per-tensor or per-(head, channel) scale;
  *        code   = clamp(round_half_even(x / s), -128, 127);  s == 0 gives code 0.
  *        dequantized value = code * s.
  *  FP8 E4M3 (OCP "E4M3FN": bias 7, no infinities, largest finite 448):
@@ -113,7 +116,8 @@ typedef enum {
   KVQ_SCALE_PER_TOKEN_HEAD = 1,
   KVQ_SCALE_PER_HEAD = 2,
   KVQ_SCALE_PER_TENSOR = 3,
-  KVQ_SCALE_KIVI = 4
+  KVQ_SCALE_KIVI = 4,
+  KVQ_SCALE_PER_CHANNEL = 5
 } kvq_scale_mode;
 
 /* Bits of fault[1] (fault[0] counts skipped entries). */
@@ -132,8 +136,9 @@ enum {
  *                 INT8, FP8_E4M3 or INT4.
  *   act_dtype     BF16 or FP16: element type of new K/V rows, of q and of the INT4
  *                 residual ring.
- *   scale_mode    NONE for BF16/FP16; PER_TOKEN_HEAD, PER_HEAD or PER_TENSOR for INT8
- *                 and FP8; KIVI for INT4.
+ *   scale_mode    NONE for BF16/FP16; PER_TOKEN_HEAD, PER_HEAD, PER_TENSOR or
+ *                 PER_CHANNEL for INT8 and FP8; KIVI for INT4.  PER_CHANNEL decodes on
+ *                 the tensor-core path only (block_size 16, head_dim 128).
  *   block_size    tokens per block: 1..1024 for dense caches; INT4 requires
  *                 block_size == group_size == 64.
  *   head_dim      64 or 128.
@@ -156,7 +161,7 @@ typedef struct {
   int32_t max_seqs;
   int32_t reserved0;
   void* pages;         /* [NB][H][record] */
-  float* k_scales;     /* static scales (PER_HEAD / PER_TENSOR) */
+  float* k_scales;     /* static scales (PER_HEAD / PER_TENSOR / PER_CHANNEL) */
   float* v_scales;
   void* residual;      /* INT4 ring */
   int32_t* fault;
@@ -319,6 +324,20 @@ kvq_status kvq_dequant(const kvq_cache_desc* cache, const int32_t* block_ids, in
 kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_heads,
                                     int head_dim, int32_t act_dtype, float* scale_out,
                                     cudaStream_t stream);
+
+/*
+ * kvq_calibrate_channel_scales - set-up step: per-(kv head, channel) scale from warm-up rows,
+ *   scale_out[h][d] = (max over tokens of |x[t][h][d]|) / qmax, float32 division.
+ *   x          act_dtype [n_tokens][num_kv_heads][head_dim], device.
+ *   qmax       largest code magnitude: 127 for INT8, 448 for FP8 E4M3; finite and > 0.
+ *   scale_out  float32 [num_kv_heads][head_dim], device.  An all-zero channel gives 0.
+ *   The static scales of KVQ_SCALE_PER_CHANNEL ([P-vLLM] "vLLM引擎KV Cache量化配置与启动参数
+ *   详解": INT8 scale factors generated offline from calibration data; [P-mem] §3.2
+ *   动态量化策略: static quantization uses fixed scales).
+ */
+kvq_status kvq_calibrate_channel_scales(const void* x, int n_tokens, int num_kv_heads,
+                                        int head_dim, int32_t act_dtype, float qmax,
+                                        float* scale_out, cudaStream_t stream);
 
 /*
  * kvq_read_device_fault - copy the descriptor's fault record into host `out[2]`

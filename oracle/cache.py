@@ -42,8 +42,9 @@ class PagedCache:
 
     cache_dtype: "bf16" | "fp16" | "int8" | "fp8" | "int4"
     act_dtype:   "bf16" | "fp16"
-    scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "kivi"
-    static_scales: (k_scale, v_scale) float32 arrays [H] or [1] for static modes.
+    scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "per_channel" | "kivi"
+    static_scales: (k_scale, v_scale) float32 arrays for static modes: [H] per head, [1]
+                   per tensor, [H, D] per (kv head, channel).
 
     ``pages`` is the byte pool [NB][H][record] of include/kvq.h: per (block, kv head),
     K codes [bs][row_bytes], V codes [bs][row_bytes], then the per-token scales (float32
@@ -91,11 +92,11 @@ class PagedCache:
         if scale_mode == "per_token_head":
             self.k_scales = pg[:, :, off_s:off_s + 4 * bs].view(np.float32).reshape(NB, H, bs)
             self.v_scales = pg[:, :, off_s + 4 * bs:off_s + 8 * bs].view(np.float32).reshape(NB, H, bs)
-        elif scale_mode in ("per_head", "per_tensor"):
-            n = H if scale_mode == "per_head" else 1
+        elif scale_mode in ("per_head", "per_tensor", "per_channel"):
+            shape = {"per_head": (H,), "per_tensor": (1,), "per_channel": (H, D)}[scale_mode]
             ks, vs = static_scales
-            self.k_scales = np.asarray(ks, np.float32).reshape(n).copy()
-            self.v_scales = np.asarray(vs, np.float32).reshape(n).copy()
+            self.k_scales = np.asarray(ks, np.float32).reshape(shape).copy()
+            self.v_scales = np.asarray(vs, np.float32).reshape(shape).copy()
         elif scale_mode == "kivi":
             # K scale [D] then K zero [D] as [NB][H][2][D]; V (scale, zero) [bs][D/G][2]
             self.k_scales = pg[:, :, off_s:off_s + 4 * D].view(np.float16).reshape(NB, H, 2, D)
@@ -108,9 +109,10 @@ class PagedCache:
 
     # ------------------------------------------------------------------ scales
     def _static_scale(self, which):
+        """[H] per head or per tensor, [H, D] per channel."""
         s = self.k_scales if which == 0 else self.v_scales
-        if self.mode == "per_head":
-            return s                                  # [H]
+        if self.mode in ("per_head", "per_channel"):
+            return s
         return np.broadcast_to(s, (self.H,))          # per tensor
 
     # ------------------------------------------------------------------ write
@@ -149,9 +151,13 @@ class PagedCache:
                      else quant.fp8_scale_dynamic(x))              # [n, H]
                 sc = self.k_scales if which == 0 else self.v_scales
                 sc[blk, :, off] = s
+            elif self.mode == "per_channel":
+                s = np.broadcast_to(self._static_scale(which), x.shape)       # [n, H, D]
             else:
                 s = np.broadcast_to(self._static_scale(which), x.shape[:2])
-            s2 = np.asarray(s, np.float32)[..., None]
+            s2 = np.asarray(s, np.float32)
+            if self.mode != "per_channel":
+                s2 = s2[..., None]
             if self.cd == "int8":
                 codes[blk, :, off, :] = quant.int8_quantize(x, s2)
             else:
@@ -202,16 +208,16 @@ class PagedCache:
             c = codes[blk]
             if self.cd in ("bf16", "fp16"):
                 out[which] = _value_of_act_bits(c, self.act)
-            elif self.cd == "int8":
-                s = (self.k_scales if which == 0 else self.v_scales)
-                s = s[blk] if self.mode == "per_token_head" else \
-                    np.broadcast_to(self._static_scale(which)[:, None], (self.H, self.bs))
-                out[which] = quant.int8_dequantize(c, s)
-            elif self.cd == "fp8":
-                s = (self.k_scales if which == 0 else self.v_scales)
-                s = s[blk] if self.mode == "per_token_head" else \
-                    np.broadcast_to(self._static_scale(which)[:, None], (self.H, self.bs))
-                out[which] = quant.fp8_dequantize(c, s)
+            elif self.cd in ("int8", "fp8"):
+                if self.mode == "per_token_head":
+                    s = (self.k_scales if which == 0 else self.v_scales)[blk]          # [H, bs]
+                elif self.mode == "per_channel":
+                    s = np.broadcast_to(self._static_scale(which)[:, None, :],
+                                        (self.H, self.bs, self.D))                   # [H, bs, D]
+                else:
+                    s = np.broadcast_to(self._static_scale(which)[:, None], (self.H, self.bs))
+                deq = quant.int8_dequantize if self.cd == "int8" else quant.fp8_dequantize
+                out[which] = deq(c, s)
             else:
                 q = quant.unpack_nibbles(c)                      # [H, bs, D]
                 if which == 0:

@@ -82,6 +82,19 @@ def fp8_calibrate(warmup):
     return fp.div32(m, np.float32(FP8_QMAX))
 
 
+def channel_calibrate(warmup, qmax):
+    """Per-(kv head, channel) static scale from warm-up rows [T, H, D]: max over the tokens
+    of |x| / qmax (binary32), [H, D].  qmax is 127 for INT8, 448 for FP8.
+
+    [P-vLLM] "KV Cache量化策略：INT8与FP8精度对比与选择" (INT8 with per-tensor or per-channel
+    granularity) and "vLLM引擎KV Cache量化配置与启动参数详解" (INT8 scales generated offline from
+    calibration data); [P-prod] "量化不是简单截断精度" (scale per tensor, head, channel, token or
+    group); [P-mem] §3.2 动态量化策略 (static quantization: fixed scales).
+    """
+    w = np.asarray(warmup, dtype=np.float32)
+    return fp.div32(np.max(np.abs(w), axis=0), np.float32(qmax))
+
+
 def fp8_quantize(rows, scale):
     """code = E4M3(x / s): binary32 quotient, nearest E4M3 (ties even), saturate at 448.
 

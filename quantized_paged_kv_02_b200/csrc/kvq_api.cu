@@ -48,7 +48,7 @@ static kvq_status validate_geometry(const kvq_cache_desc* c, Geometry* g) {
     case KVQ_DTYPE_INT8:
     case KVQ_DTYPE_FP8_E4M3:
       if (c->scale_mode != KVQ_SCALE_PER_TOKEN_HEAD && c->scale_mode != KVQ_SCALE_PER_HEAD &&
-          c->scale_mode != KVQ_SCALE_PER_TENSOR)
+          c->scale_mode != KVQ_SCALE_PER_TENSOR && c->scale_mode != KVQ_SCALE_PER_CHANNEL)
         return KVQ_ERR_INVALID_ARG;
       break;
     case KVQ_DTYPE_INT4:
@@ -72,7 +72,8 @@ kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
   const kvq_status st = validate_geometry(c, g);
   if (st != KVQ_OK) return st;
   if (c->pages == nullptr || !aligned16(c->pages)) return KVQ_ERR_INVALID_ARG;
-  if (c->scale_mode == KVQ_SCALE_PER_HEAD || c->scale_mode == KVQ_SCALE_PER_TENSOR) {
+  if (c->scale_mode == KVQ_SCALE_PER_HEAD || c->scale_mode == KVQ_SCALE_PER_TENSOR ||
+      c->scale_mode == KVQ_SCALE_PER_CHANNEL) {
     if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
     if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
   }
@@ -168,6 +169,7 @@ kvq_status kvq_cache_layout(const kvq_cache_desc* c, size_t* record_bytes, size_
   size_t ss = 0, rb = 0;
   if (g.scale_mode == KVQ_SCALE_PER_HEAD) ss = static_cast<size_t>(g.H) * 4;
   if (g.scale_mode == KVQ_SCALE_PER_TENSOR) ss = 4;
+  if (g.scale_mode == KVQ_SCALE_PER_CHANNEL) ss = static_cast<size_t>(g.H) * g.D * 4;
   if (g.scale_mode == KVQ_SCALE_KIVI)
     rb = static_cast<size_t>(g.max_seqs) * 2 * g.H * g.residual_cap * g.D * 2;
   if (record_bytes) *record_bytes = static_cast<size_t>(g.record);
@@ -250,6 +252,17 @@ kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_head
   if (act_dtype != KVQ_DTYPE_BF16 && act_dtype != KVQ_DTYPE_FP16) return KVQ_ERR_INVALID_ARG;
   if (scale_out == nullptr || (n_tokens > 0 && x == nullptr)) return KVQ_ERR_INVALID_ARG;
   return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, scale_out, stream));
+}
+
+kvq_status kvq_calibrate_channel_scales(const void* x, int n_tokens, int num_kv_heads,
+                                        int head_dim, int32_t act_dtype, float qmax,
+                                        float* scale_out, cudaStream_t stream) {
+  if (n_tokens < 0 || num_kv_heads < 1 || head_dim < 1 || head_dim > 1024) return KVQ_ERR_INVALID_ARG;
+  if (act_dtype != KVQ_DTYPE_BF16 && act_dtype != KVQ_DTYPE_FP16) return KVQ_ERR_INVALID_ARG;
+  if (!(qmax > 0.f) || !std::isfinite(qmax)) return KVQ_ERR_INVALID_ARG;
+  if (scale_out == nullptr || (n_tokens > 0 && x == nullptr)) return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_calibrate_channels(x, n_tokens, num_kv_heads, head_dim, act_dtype, qmax,
+                                             scale_out, stream));
 }
 
 kvq_status kvq_read_device_fault(const kvq_cache_desc* c, int32_t* out, int reset,

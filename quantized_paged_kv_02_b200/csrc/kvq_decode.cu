@@ -210,6 +210,8 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
                        DecodePlan* p) {
   p->g = num_q_heads / g.H;
   p->kernel = mma_supported(g, p->g) ? 1 : 0;
+  // per-channel scales are folded into q and the output by the tensor-core kernel only
+  if (g.scale_mode == KVQ_SCALE_PER_CHANNEL && p->kernel != 1) return KVQ_ERR_UNSUPPORTED;
   if (int4_mma_supported(g, p->g)) {
     // INT4 blocks on tensor cores: splits over the quantized prefix (64-token blocks)
     // plus one split for the residual ring, computed by the CUDA-core kernel

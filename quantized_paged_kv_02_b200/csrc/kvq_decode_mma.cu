@@ -184,15 +184,18 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
           [((static_cast<long>(bq) * p.H + kvh) * kD) / 8 + l];
       uint8_t* rec = p.pages_w + (static_cast<long>(blk) * p.H + kvh) * L::REC;
       float static_s = 0.f;
+      const float* chan_s = nullptr;
       if constexpr (!PT && Code<CD>::B == 1) {
         const float* sp = kv ? p.v_static : p.k_static;
-        static_s = sp[p.mode == KVQ_SCALE_PER_HEAD ? kvh : 0];
+        if (p.mode == KVQ_SCALE_PER_CHANNEL) chan_s = sp + kvh * kD;
+        else static_s = sp[p.mode == KVQ_SCALE_PER_HEAD ? kvh : 0];
       }
       if (p.act_fp16)
-        quantize_row_part<__half, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT, static_s);
+        quantize_row_part<__half, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
+                                          static_s, chan_s);
       else
         quantize_row_part<__nv_bfloat16, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
-                                                 static_s);
+                                                 static_s, chan_s);
       fence_proxy_async_global();
       __syncwarp();
     };
@@ -304,10 +307,17 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
 #pragma unroll
       for (int c = 0; c < 4; ++c) qraw[c] = make_uint4(0, 0, 0, 0);
     }
+    // PER_CHANNEL: K's scale of channel d multiplies every code of that channel, so it
+    // folds into q_d once per unit (q . (c * s) = (q * s) . c)
+    const float* kch = nullptr;
+    if constexpr (!PT && Code<CD>::B == 1) {
+      if (p.mode == KVQ_SCALE_PER_CHANNEL) kch = p.k_static + kvh * kD + 32 * j;
+    }
     auto qv = [&](int e) {
       const uint32_t w2 = (&qraw[e >> 3].x)[(e & 7) >> 1];
       const uint16_t h = static_cast<uint16_t>((e & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
-      return p.act_fp16 ? __half2float(__ushort_as_half(h)) : __bfloat162float(__ushort_as_bfloat16(h));
+      const float f = p.act_fp16 ? __half2float(__ushort_as_half(h)) : __bfloat162float(__ushort_as_bfloat16(h));
+      return kch != nullptr ? f * kch[e] : f;
     };
     if constexpr (CD == KVQ_DTYPE_INT8) {
       // q = sq * (Q0 + Q1/128 + Q2/16384) with int8 terms, sq = max|q| / 127 over the
@@ -391,6 +401,11 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       if (p.mode == KVQ_SCALE_PER_HEAD) vmul = p.v_static[kvh];
       if (p.mode == KVQ_SCALE_PER_TENSOR) vmul = p.v_static[0];
     }
+    // PER_CHANNEL: V's scale of channel d multiplies output channel d
+    const float* vch = nullptr;
+    if constexpr (!PT && Code<CD>::B == 1) {
+      if (p.mode == KVQ_SCALE_PER_CHANNEL) vch = p.v_static + kvh * kD;
+    }
     const long slot = (static_cast<long>(cur_u) + cta) * kSegWarps + warp;
     float* wo = p.ws_o + slot * g * kD;
     float* wml = p.ws_ml + slot * g * 2;
@@ -398,8 +413,14 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
 #pragma unroll
     for (int md = 0; md < 8; ++md) {
       const int d0 = 16 * r + 2 * md;
-      if (h0 < g) *reinterpret_cast<float2*>(wo + h0 * kD + d0) = make_float2(o[md][0] * vmul, o[md][2] * vmul);
-      if (h1 < g) *reinterpret_cast<float2*>(wo + h1 * kD + d0) = make_float2(o[md][1] * vmul, o[md][3] * vmul);
+      float m0 = vmul, m1 = vmul;
+      if (vch != nullptr) {
+        const float2 cv = *reinterpret_cast<const float2*>(vch + d0);
+        m0 = cv.x;
+        m1 = cv.y;
+      }
+      if (h0 < g) *reinterpret_cast<float2*>(wo + h0 * kD + d0) = make_float2(o[md][0] * m0, o[md][2] * m1);
+      if (h1 < g) *reinterpret_cast<float2*>(wo + h1 * kD + d0) = make_float2(o[md][1] * m0, o[md][3] * m1);
     }
     if (r == 0) {
       if (h0 < g) *reinterpret_cast<float2*>(wml + 2 * h0) = make_float2(m[0], l[0]);

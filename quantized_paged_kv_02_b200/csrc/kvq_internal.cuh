@@ -79,13 +79,15 @@ __device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
 // record.  A row is handled by D*2/16 consecutive lanes (a power of two dividing 32);
 // lane l holds activation elements [8l, 8l+8) in `u`.  `write` false: the lane joins the
 // shuffles but stores nothing.  Per-token modes reduce max|x| over the row's lanes and
-// store the float32 scale; static modes use `static_s`.  INT8: [P-mem] §3.1 对称量化算法
-// (scale = max|x|/127, q = clamp(round(x/scale), -128, 127)); FP8: [P-vLLM]
-// "KV Cache量化策略" (E4M3 storage with a scale).
+// store the float32 scale; static modes use `static_s`, or per channel the row's [D]
+// scales `chan_s`.  INT8: [P-mem] §3.1 对称量化算法 (scale = max|x|/127,
+// q = clamp(round(x/scale), -128, 127)); FP8: [P-vLLM] "KV Cache量化策略" (E4M3 storage
+// with a scale).
 template <typename TA, int CD, int D>
 __device__ __forceinline__ void quantize_row_part(const uint4& u, int l, bool write, int kv, int off,
                                                   int bs, uint8_t* rec, int off_v, int off_s,
-                                                  bool per_token, float static_s) {
+                                                  bool per_token, float static_s,
+                                                  const float* chan_s = nullptr) {
   constexpr int LPR = D * 2 / 16;
   constexpr int ROWB = (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) ? 2 * D : D;
   uint8_t* dst_row = rec + (kv ? off_v : 0) + off * ROWB;
@@ -104,10 +106,20 @@ __device__ __forceinline__ void quantize_row_part(const uint4& u, int l, bool wr
       s = div_rn(m, QMax<CD>::v);
       if (write && l == 0) reinterpret_cast<float*>(rec + off_s)[(kv ? bs : 0) + off] = s;
     }
+    // PER_CHANNEL: chan_s is the row's [D] scales; this lane's are [8l, 8l+8)
+    float cs[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cs[i] = s;
+    if (chan_s != nullptr) {
+      const float4 a = reinterpret_cast<const float4*>(chan_s)[2 * l];
+      const float4 b = reinterpret_cast<const float4*>(chan_s)[2 * l + 1];
+      cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+      cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+    }
     uint32_t w0 = 0, w1 = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
+      const uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], cs[i]) : quant_fp8(x[i], cs[i]);
       if (i < 4) w0 |= c << (8 * i); else w1 |= c << (8 * (i - 4));
     }
     if (write) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w0, w1);
@@ -136,6 +148,8 @@ cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int
                            float* out, cudaStream_t s);
 cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float* out,
                              cudaStream_t s);
+cudaError_t launch_calibrate_channels(const void* x, int n, int H, int D, int act, float qmax,
+                                      float* out, cudaStream_t s);
 
 // Plan of the decode kernels.  SIMT and INT4: grid (splits, heads-tiles, batch), chunk
 // tokens each.  Dense tensor-core kernel: ctas CTAs over page-balanced ranges.

@@ -1,4 +1,5 @@
-// kvq_dequant (debug) and kvq_calibrate_fp8_scales (set-up) kernels.
+// kvq_dequant (debug), kvq_calibrate_fp8_scales and kvq_calibrate_channel_scales (set-up)
+// kernels.
 //
 // Dequantized values follow the definitions in include/kvq.h: INT8 / FP8 code * scale
 // ([P-mem] §3.1 对称量化算法: q.float() * scale), INT4 (code - zero) * scale ([P-prod]
@@ -49,7 +50,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
         const float* s = reinterpret_cast<const float*>(rec + p.off_s) + (kv ? p.bs : 0);
         const float* st = kv ? p.v_static : p.k_static;
         const float sv = p.mode == KVQ_SCALE_PER_TOKEN_HEAD ? s[t]
-                         : p.mode == KVQ_SCALE_PER_HEAD   ? st[h] : st[0];
+                         : p.mode == KVQ_SCALE_PER_HEAD   ? st[h]
+                         : p.mode == KVQ_SCALE_PER_CHANNEL ? st[h * p.D + d] : st[0];
         const float cv = p.cd == KVQ_DTYPE_INT8 ? static_cast<float>(static_cast<int8_t>(c))
                                                 : e4m3_to_float(c);
         x = cv * sv;
@@ -94,7 +96,29 @@ __global__ void __launch_bounds__(256) calibrate_kernel(const TA* x, int n, int 
   }
 }
 
+// grid H: thread d of CTA h scans the tokens of channel (h, d).
+template <typename TA>
+__global__ void __launch_bounds__(128) calibrate_channels_kernel(const TA* x, int n, int H, int D,
+                                                                 float qmax, float* out) {
+  const int h = blockIdx.x;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float m = 0.f;
+    for (long t = 0; t < n; ++t) m = fmaxf(m, fabsf(Act<TA>::to_f(x[(t * H + h) * D + d])));
+    out[h * D + d] = div_rn(m, qmax);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_calibrate_channels(const void* x, int n, int H, int D, int act, float qmax,
+                                      float* out, cudaStream_t s) {
+  if (act == KVQ_DTYPE_BF16)
+    calibrate_channels_kernel<__nv_bfloat16><<<H, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n, H, D,
+                                                                qmax, out);
+  else
+    calibrate_channels_kernel<__half><<<H, 128, 0, s>>>(static_cast<const __half*>(x), n, H, D, qmax, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int32_t* ids, int n,
                            float* out, cudaStream_t s) {

@@ -62,8 +62,9 @@ __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
   const float* sp = kv ? p.v_static : p.k_static;
   const bool is_static = p.scale_mode == KVQ_SCALE_PER_HEAD || p.scale_mode == KVQ_SCALE_PER_TENSOR;
   const float static_s = is_static ? sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0] : 0.f;
+  const float* chan_s = p.scale_mode == KVQ_SCALE_PER_CHANNEL ? sp + static_cast<long>(h) * D : nullptr;
   quantize_row_part<TA, CD, D>(u, l, write, kv, off, p.bs, rec, p.off_v, p.off_s,
-                               p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD, static_s);
+                               p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD, static_s, chan_s);
 }
 
 // ------------------------------------------------------------------ INT4 (KIVI)

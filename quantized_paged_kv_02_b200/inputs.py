@@ -13,7 +13,8 @@ Recipe (all on one ``torch.Generator`` seeded with ``seed``, in this order):
      K and V) are multiplied by 10 on those channels;
   5. block table: ``randperm(num_blocks)``; sequence b takes the next ceil(n_b/bs)
      entries, so tables are non-contiguous and the unused blocks are spread out;
-  6. FP8 warm-up rows (when needed): ``randn`` float32 [256, H_kv, D] for K, then V.
+  6. warm-up rows for static scales (per head, per tensor, per channel): ``randn`` float32
+     [256, H_kv, D] for K, then V.
 Values are cast to the activation dtype (round to nearest even) after step 4.
 
 The five named workloads follow the shapes of the method's benchmark configurations
@@ -72,8 +73,11 @@ def _spec(name, small):
         return Spec("c4", "int4", "bf16", "kivi", 16, 64, 8, 128, 64,
                     lens=[32768] * 16, outliers="k", slack_blocks=16)
     if name.startswith("c5"):
-        cd = {"c5": "int8", "c5-int8": "int8", "c5-fp8": "fp8", "c5-bf16": "bf16"}[name]
+        cd = {"c5": "int8", "c5-int8": "int8", "c5-fp8": "fp8", "c5-bf16": "bf16",
+              "c5-int8-pc": "int8"}[name]
         mode = {"int8": "per_token_head", "fp8": "per_head", "bf16": "none"}[cd]
+        if name == "c5-int8-pc":
+            mode = "per_channel"
         if small:
             return Spec(name + "-small", cd, "bf16", mode, 3, 16, 2, 128, 16,
                         lens=[1000, 517, 33], slack_blocks=4)
@@ -109,7 +113,7 @@ def act_torch_dtype(act):
 
 
 def make(name, small=False, device="cpu", seed=None):
-    """Build the named workload ("c1".."c5", "c5-fp8", "c5-bf16") on `device`."""
+    """Build the named workload ("c1".."c5", "c5-fp8", "c5-bf16", "c5-int8-pc") on `device`."""
     spec = _spec(name, small)
     if seed is not None:
         spec.seed = seed
@@ -172,7 +176,7 @@ def from_spec(spec, device="cpu"):
             seq_ids[r0 + paged[b]:r0 + n] = b
         start.append(r0 + n)
     wk = wv = None
-    if spec.cache_dtype == "fp8" and spec.scale_mode in ("per_head", "per_tensor"):
+    if spec.scale_mode in ("per_head", "per_tensor", "per_channel"):
         wk = torch.randn((256, H, D), generator=g, device=device, dtype=torch.float32).to(adt)
         wv = torch.randn((256, H, D), generator=g, device=device, dtype=torch.float32).to(adt)
     dev = torch.device(device)

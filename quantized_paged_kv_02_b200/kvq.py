@@ -18,14 +18,15 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkvq.so")
 
 DTYPE = {"bf16": 0, "fp16": 1, "fp32": 2, "int8": 3, "fp8": 4, "int4": 5}
-SCALE = {"none": 0, "per_token_head": 1, "per_head": 2, "per_tensor": 3, "kivi": 4}
+SCALE = {"none": 0, "per_token_head": 1, "per_head": 2, "per_tensor": 3, "kivi": 4,
+         "per_channel": 5}
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "KVQ_ERR_CUDA",
           4: "KVQ_ERR_DEVICE_FAULT"}
 FAULT_BITS = {"slot": 1, "block": 2, "context": 4, "seq": 8, "int4_run": 16, "timeout": 32}
 EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
            "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc",
-           "kvq_append_decode_attention")
+           "kvq_append_decode_attention", "kvq_calibrate_channel_scales")
 
 
 class CacheDesc(ctypes.Structure):
@@ -67,6 +68,7 @@ def _load():
         "kvq_decode_attention_noalloc": (I, [D, P, I, I, P, I, P, P, I, F, P, ctypes.c_int32, P]),
         "kvq_append_decode_attention": (I, [D, P, P, P, I, I, P, I, P, I, F, P, ctypes.c_int32, P,
                                             Z, P]),
+        "kvq_calibrate_channel_scales": (I, [P, I, I, I, ctypes.c_int32, F, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -190,6 +192,15 @@ def kvq_calibrate_fp8_scales(x, scale_out, stream=None):
     T, H, D = x.shape
     _check(lib.kvq_calibrate_fp8_scales(_ptr(x), T, H, D, DTYPE[_act(x)], _ptr(scale_out),
                                         _stream(stream)), "kvq_calibrate_fp8_scales")
+    return scale_out
+
+
+def kvq_calibrate_channel_scales(x, qmax, scale_out, stream=None):
+    """scale_out[h][d] = max over tokens |x[t][h][d]| / qmax (127 INT8, 448 FP8)."""
+    T, H, D = x.shape
+    _check(lib.kvq_calibrate_channel_scales(_ptr(x), T, H, D, DTYPE[_act(x)], float(qmax),
+                                            _ptr(scale_out), _stream(stream)),
+           "kvq_calibrate_channel_scales")
     return scale_out
 
 

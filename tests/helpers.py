@@ -24,6 +24,10 @@ def np64(t):
 
 def oracle_static_scales(w):
     from oracle import quant
+    if w.spec.scale_mode == "per_channel":
+        qmax = 127.0 if w.spec.cache_dtype == "int8" else 448.0
+        return (quant.channel_calibrate(np64(w.warmup_k).astype(np.float32), qmax),
+                quant.channel_calibrate(np64(w.warmup_v).astype(np.float32), qmax))
     if w.spec.scale_mode in ("per_head", "per_tensor"):
         ks = quant.fp8_calibrate(np64(w.warmup_k).astype(np.float32))
         vs = quant.fp8_calibrate(np64(w.warmup_v).astype(np.float32))

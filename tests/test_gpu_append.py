@@ -65,7 +65,7 @@ def _check(w):
     return got, static
 
 
-@pytest.mark.parametrize("name", ["c5", "c5-fp8", "c5-bf16", "c3", "c2"])
+@pytest.mark.parametrize("name", ["c5", "c5-fp8", "c5-bf16", "c5-int8-pc", "c3", "c2"])
 def test_append_decode_equals_write_then_decode(name):
     w = inputs.make(name, small=True)
     got, static = _check(w)

@@ -12,7 +12,7 @@ from tests import helpers
 
 pytestmark = pytest.mark.gpu
 
-SMALL = ["c1", "c2", "c3", "c4", "c5", "c5-fp8", "c5-bf16"]
+SMALL = ["c1", "c2", "c3", "c4", "c5", "c5-fp8", "c5-bf16", "c5-int8-pc"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -48,6 +48,18 @@ def test_fp8_calibration_bit_exact():
         kvq.kvq_calibrate_fp8_scales(x.cuda(), out)
         want = quant.fp8_calibrate(helpers.np64(x).astype(np.float32))
         np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+def test_channel_calibration_bit_exact():
+    from oracle import quant
+    from quantized_paged_kv_02_b200 import kvq
+    w = inputs.make("c5-int8-pc", small=True)
+    for x in (w.warmup_k, w.warmup_v):
+        for qmax in (127.0, 448.0):
+            out = torch.empty(x.shape[1:], dtype=torch.float32, device="cuda")
+            kvq.kvq_calibrate_channel_scales(x.cuda(), qmax, out)
+            want = quant.channel_calibrate(helpers.np64(x).astype(np.float32), qmax)
+            np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
 
 
 @pytest.mark.parametrize("name", SMALL)

@@ -86,6 +86,69 @@ def test_fp8_grid_exact_attention_equals_sdpa():
         np.testing.assert_allclose(out[0, h], _sdpa(q[0, h], K[:, h], V[:, h], 0.3), rtol=1e-12, atol=1e-12)
 
 
+def test_int8_per_channel_grid_exact_attention_equals_sdpa():
+    """Static per-(head, channel) INT8 scales that are powers of two, values k * s_d with
+    integer |k| <= 127: quantization is exact, so attention equals dense SDPA."""
+    rng = np.random.default_rng(3)
+    T, H, D, g, bs = 50, 2, 64, 4, 16
+    ks = np.exp2(-rng.integers(0, 6, size=(H, D))).astype(np.float32)
+    vs = np.exp2(-rng.integers(0, 6, size=(H, D))).astype(np.float32)
+    K = rng.integers(-127, 128, size=(T, H, D)) * ks[None].astype(np.float64)
+    V = rng.integers(-127, 128, size=(T, H, D)) * vs[None].astype(np.float64)
+    nblk = -(-T // bs)
+    perm = rng.permutation(nblk + 1)[:nblk]
+    slots = np.array([perm[p // bs] * bs + p % bs for p in range(T)])
+    c = cache.PagedCache("int8", "bf16", "per_channel", nblk + 1, bs, H, D, static_scales=(ks, vs))
+    c.write(K, V, slots)
+    K2, V2 = c.gather(perm, T)
+    np.testing.assert_array_equal(K2, np.transpose(K, (1, 0, 2)))
+    np.testing.assert_array_equal(V2, np.transpose(V, (1, 0, 2)))
+    q = fp.bf16_round(rng.standard_normal((1, H * g, D)))
+    out = attention.decode_attention(c, q, perm[None, :], np.array([T]))
+    for hq in range(H * g):
+        ref = _sdpa(q[0, hq], K[:, hq // g], V[:, hq // g], 1.0 / np.sqrt(D))
+        np.testing.assert_allclose(out[0, hq], ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("cd", ["int8", "fp8"])
+def test_per_channel_with_equal_channels_is_per_head(cd):
+    """A per-channel cache whose channels of a head all carry that head's scale stores
+    exactly the bytes of the per-head cache (and dequantizes to the same values)."""
+    rng = np.random.default_rng(4)
+    T, H, D, bs = 37, 3, 64, 16
+    x = fp.bf16_round(rng.standard_normal((T, H, D)) * 3)
+    y = fp.bf16_round(rng.standard_normal((T, H, D)))
+    sh = np.array([0.03, 0.011, 0.2], np.float32)
+    nblk = -(-T // bs)
+    a = cache.PagedCache(cd, "bf16", "per_head", nblk, bs, H, D, static_scales=(sh, sh * 2))
+    b = cache.PagedCache(cd, "bf16", "per_channel", nblk, bs, H, D,
+                         static_scales=(np.repeat(sh[:, None], D, 1), np.repeat((sh * 2)[:, None], D, 1)))
+    a.write(x, y, np.arange(T))
+    b.write(x, y, np.arange(T))
+    np.testing.assert_array_equal(a.pages, b.pages)
+    for blk in range(nblk):
+        np.testing.assert_array_equal(a.dequant_block(blk), b.dequant_block(blk))
+
+
+def test_channel_calibration():
+    """scale[h, d] = binary32(max_t |x[t, h, d]| / qmax); each channel on its own."""
+    rng = np.random.default_rng(5)
+    w = fp.bf16_round(rng.standard_normal((256, 2, 64))).astype(np.float32)
+    s = quant.channel_calibrate(w, 127.0)
+    assert s.shape == (2, 64) and s.dtype == np.float32
+    for h in range(2):
+        for d in (0, 17, 63):
+            assert s[h, d] == fp.div32(np.float32(np.abs(w[:, h, d]).max()), np.float32(127.0))
+    w2 = w.copy()
+    w2[:, 1, 5] *= 4
+    s2 = quant.channel_calibrate(w2, 448.0)
+    s1 = quant.channel_calibrate(w, 448.0)
+    assert s2[1, 5] == fp.div32(np.float32(4 * np.abs(w[:, 1, 5]).max()), np.float32(448.0))
+    mask = np.ones_like(s1, bool)
+    mask[1, 5] = False
+    np.testing.assert_array_equal(s2[mask], s1[mask])
+
+
 def test_int4_grid_exact_attention_equals_sdpa():
     """Keys on a per-channel grid over each 64-token block, values on a per-token grid
     over each 64-channel group, plus unquantized residual rows: exact."""
