@@ -208,6 +208,27 @@ kvq_status kvq_write(const kvq_cache_desc* cache, const void* k_new, const void*
                      const int32_t* positions, cudaStream_t stream);
 
 /*
+ * kvq_flush_ring - INT4: move whole groups of the residual ring into pages.
+ *   For each entry i < n: ring rows of sequence seq_ids[i] at positions
+ *   [positions[i], positions[i] + 64) (ring row p % residual_cap) are quantized into block
+ *   block_ids[i] of every kv head, with exactly the codes, scales and zero points kvq_write
+ *   stores when given those rows with slots block_ids[i]*64 + 0..63.  The ring rows are left
+ *   in place.
+ *   seq_ids, positions, block_ids  int32 [n], device.  positions[i] must be a multiple of 64
+ *   and the 64 positions must still be in the ring (at most residual_cap positions behind
+ *   the newest one written); an entry with a sequence id, block id or position out of range
+ *   is skipped and counted (KVQ_FAULT_SEQ / _BLOCK / _INT4_RUN).
+ *   The residual window of [P-prod] "Key 和 Value 的分布不一定相同" keeps the newest tokens
+ *   unquantized; once more than residual_len + 64 are there, the oldest 64 become one key
+ *   group (one block) and are quantized, which this call does from the ring itself, so the
+ *   caller need not keep its own copy of those rows.
+ *   INT4 caches only (others: KVQ_ERR_UNSUPPORTED).
+ */
+kvq_status kvq_flush_ring(const kvq_cache_desc* cache, const int32_t* seq_ids,
+                          const int32_t* positions, const int32_t* block_ids, int n,
+                          cudaStream_t stream);
+
+/*
  * Workspace bytes kvq_decode_attention needs for this shape (host-only).  The split
  * plan depends only on (cache geometry, batch, num_q_heads, max_context), so the same
  * arguments always give the same size.  *bytes may be 0 (no split needed).

@@ -199,6 +199,21 @@ class PagedCache:
                     self.residual[sid, 0, :, row, :] = _bits_of_act(k_new[t], self.act)
                     self.residual[sid, 1, :, row, :] = _bits_of_act(v_new[t], self.act)
 
+    def flush_ring(self, seq_ids, positions, block_ids):
+        """INT4: quantize ring rows [p0, p0 + 64) of sequence sid into block blk, every kv
+        head, exactly as writing those rows to slots blk*64 .. blk*64+63 would (the contract
+        of kvq_flush_ring in include/kvq.h).  Entries out of range are skipped."""
+        G = self.G
+        for sid, p0, blk in zip(np.asarray(seq_ids).tolist(), np.asarray(positions).tolist(),
+                                np.asarray(block_ids).tolist()):
+            if not (0 <= sid < self.max_seqs) or not (0 <= blk < self.NB) or p0 < 0 or p0 % G:
+                continue
+            rows = [(p0 + t) % self.cap for t in range(G)]
+            k = _value_of_act_bits(self.residual[sid, 0][:, rows, :], self.act)   # [H, G, D]
+            v = _value_of_act_bits(self.residual[sid, 1][:, rows, :], self.act)
+            slots = blk * G + np.arange(G)
+            self._write_int4(np.swapaxes(k, 0, 1), np.swapaxes(v, 0, 1), slots, None, None)
+
     # ------------------------------------------------------------------ read
     def dequant_block(self, blk):
         """float64 [2, H, bs, D] of one block (index 0 = K, 1 = V)."""

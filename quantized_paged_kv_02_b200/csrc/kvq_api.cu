@@ -254,6 +254,18 @@ kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_head
   return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, scale_out, stream));
 }
 
+kvq_status kvq_flush_ring(const kvq_cache_desc* c, const int32_t* seq_ids, const int32_t* positions,
+                          const int32_t* block_ids, int n, cudaStream_t stream) {
+  Geometry g;
+  kvq_status st = validate_desc(c, &g);
+  if (st != KVQ_OK) return st;
+  if (g.cache_dtype != KVQ_DTYPE_INT4) return KVQ_ERR_UNSUPPORTED;
+  if (n < 0) return KVQ_ERR_INVALID_ARG;
+  if (n == 0) return KVQ_OK;
+  if (seq_ids == nullptr || positions == nullptr || block_ids == nullptr) return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_flush_ring(*c, g, seq_ids, positions, block_ids, n, stream));
+}
+
 kvq_status kvq_calibrate_channel_scales(const void* x, int n_tokens, int num_kv_heads,
                                         int head_dim, int32_t act_dtype, float qmax,
                                         float* scale_out, cudaStream_t stream) {

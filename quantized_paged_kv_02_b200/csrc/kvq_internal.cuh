@@ -144,6 +144,8 @@ cudaError_t launch_write_dense(const kvq_cache_desc& c, const Geometry& g, const
 cudaError_t launch_write_int4(const kvq_cache_desc& c, const Geometry& g, const void* k,
                               const void* v, int T, const int32_t* slots, const int32_t* seq_ids,
                               const int32_t* positions, cudaStream_t s);
+cudaError_t launch_flush_ring(const kvq_cache_desc& c, const Geometry& g, const int32_t* seq_ids,
+                              const int32_t* positions, const int32_t* blocks, int n, cudaStream_t s);
 cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int32_t* ids, int n,
                            float* out, cudaStream_t s);
 cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float* out,

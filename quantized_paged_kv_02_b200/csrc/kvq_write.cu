@@ -104,6 +104,73 @@ __device__ __forceinline__ int int4_code(float x, const Int4Group& g) {
   return max(0, min(15, __float2int_rn(div_rn(x, g.sw)) + g.z));
 }
 
+// Quantize the 64 rows of one (block, kv head) into its page record: keys one group per
+// channel over the 64 tokens, values one group per token per 64 channels ([P-prod] "Key 和
+// Value 的分布不一定相同"), codes packed two per byte.  row(kv, t) points at row t (act
+// dtype, D values) of K (kv 0) or V (kv 1).  All 128 threads of the CTA take part.
+template <typename TA, int D, typename RowFn>
+__device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_s,
+                                    float (*xs)[D + 1], uint8_t (*cs)[D]) {
+  constexpr int G = 64;
+  const int tid = threadIdx.x;
+  __half* k_sz = reinterpret_cast<__half*>(rec + off_s);           // scale [D], zero [D]
+  __half* v_sz = k_sz + 2 * D;                                     // [64][D/64][2]
+  for (int kv = 0; kv < 2; ++kv) {
+    // stage the 64 rows of this head as float
+    for (int i = tid; i < G * D / 8; i += blockDim.x) {
+      const int t = i / (D / 8), c = i % (D / 8);
+      const uint4 w = *reinterpret_cast<const uint4*>(row(kv, t) + c * 8);
+      float f[8];
+      unpack8<TA>(w, f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[t][c * 8 + j] = f[j];
+    }
+    __syncthreads();
+    if (kv == 0) {
+      // keys: one group per channel over the 64 tokens
+      for (int d = tid; d < D; d += blockDim.x) {
+        float lo = xs[0][d], hi = xs[0][d];
+        for (int t = 1; t < G; ++t) { lo = fminf(lo, xs[t][d]); hi = fmaxf(hi, xs[t][d]); }
+        const Int4Group g = int4_group(lo, hi);
+        for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g));
+        k_sz[d] = g.s16;
+        k_sz[D + d] = __int2half_rn(g.z);
+      }
+    } else {
+      // values: one group per token per 64 channels
+      for (int i = tid; i < G * (D / 64); i += blockDim.x) {
+        const int t = i / (D / 64), gi = i % (D / 64);
+        float lo = xs[t][gi * 64], hi = lo;
+        for (int j = 1; j < 64; ++j) { lo = fminf(lo, xs[t][gi * 64 + j]); hi = fmaxf(hi, xs[t][gi * 64 + j]); }
+        const Int4Group g = int4_group(lo, hi);
+        for (int j = 0; j < 64; ++j) cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g));
+        __half* sz = v_sz + (t * (D / 64) + gi) * 2;
+        sz[0] = g.s16;
+        sz[1] = __int2half_rn(g.z);
+      }
+    }
+    __syncthreads();
+    // pack two codes per byte (element 2i low nibble) and store 16 bytes at a time
+    uint8_t* dst = rec + (kv ? off_v : 0);
+    for (int i = tid; i < G * D / 32; i += blockDim.x) {
+      const int t = i / (D / 32), c = i % (D / 32);
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t x = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int e = c * 32 + j * 8 + b * 2;
+          x |= static_cast<uint32_t>(cs[t][e] | (cs[t][e + 1] << 4)) << (8 * b);
+        }
+        w[j] = x;
+      }
+      *reinterpret_cast<uint4*>(dst + t * (D / 2) + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncthreads();
+  }
+}
+
 template <typename TA, int D>
 __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
   griddep_launch_dependents();   // a decode launched after this one may start its set-up
@@ -128,63 +195,10 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
     }
     const long blk = first / G;
     uint8_t* rec = p.pages + (blk * p.H + h) * p.record;
-    __half* k_sz = reinterpret_cast<__half*>(rec + p.off_s);          // scale [D], zero [D]
-    __half* v_sz = k_sz + 2 * D;                                     // [64][D/64][2]
-    for (int kv = 0; kv < 2; ++kv) {
-      const TA* src = static_cast<const TA*>(kv ? p.v : p.k);
-      // stage the 64 rows of this head as float
-      for (int i = tid; i < G * D / 8; i += blockDim.x) {
-        const int t = i / (D / 8), c = i % (D / 8);
-        const uint4 w = *reinterpret_cast<const uint4*>(src + (static_cast<long>(r0 + t) * p.H + h) * D + c * 8);
-        float f[8];
-        unpack8<TA>(w, f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xs[t][c * 8 + j] = f[j];
-      }
-      __syncthreads();
-      if (kv == 0) {
-        // keys: one group per channel over the 64 tokens
-        for (int d = tid; d < D; d += blockDim.x) {
-          float lo = xs[0][d], hi = xs[0][d];
-          for (int t = 1; t < G; ++t) { lo = fminf(lo, xs[t][d]); hi = fmaxf(hi, xs[t][d]); }
-          const Int4Group g = int4_group(lo, hi);
-          for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g));
-          k_sz[d] = g.s16;
-          k_sz[D + d] = __int2half_rn(g.z);
-        }
-      } else {
-        // values: one group per token per 64 channels
-        for (int i = tid; i < G * (D / 64); i += blockDim.x) {
-          const int t = i / (D / 64), gi = i % (D / 64);
-          float lo = xs[t][gi * 64], hi = lo;
-          for (int j = 1; j < 64; ++j) { lo = fminf(lo, xs[t][gi * 64 + j]); hi = fmaxf(hi, xs[t][gi * 64 + j]); }
-          const Int4Group g = int4_group(lo, hi);
-          for (int j = 0; j < 64; ++j) cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g));
-          __half* sz = v_sz + (t * (D / 64) + gi) * 2;
-          sz[0] = g.s16;
-          sz[1] = __int2half_rn(g.z);
-        }
-      }
-      __syncthreads();
-      // pack two codes per byte (element 2i low nibble) and store 16 bytes at a time
-      uint8_t* dst = rec + (kv ? p.off_v : 0);
-      for (int i = tid; i < G * D / 32; i += blockDim.x) {
-        const int t = i / (D / 32), c = i % (D / 32);
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t x = 0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int e = c * 32 + j * 8 + b * 2;
-            x |= static_cast<uint32_t>(cs[t][e] | (cs[t][e + 1] << 4)) << (8 * b);
-          }
-          w[j] = x;
-        }
-        *reinterpret_cast<uint4*>(dst + t * (D / 2) + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      __syncthreads();
-    }
+    auto row = [&](int kv, int t) {
+      return static_cast<const TA*>(kv ? p.v : p.k) + (static_cast<long>(r0 + t) * p.H + h) * D;
+    };
+    quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, xs, cs);
   } else {
     // residual rows: copied unquantized into ring row positions[t] % cap
     for (int i = tid; i < nr * 2 * (D / 8); i += blockDim.x) {
@@ -235,7 +249,59 @@ cudaError_t dense_by_cd(int cd, const WriteParams& p, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
+// ------------------------------------------------------------------ INT4 ring flush
+struct Int4FlushParams {
+  const int32_t* seq_ids;
+  const int32_t* positions;
+  const int32_t* blocks;
+  uint8_t* pages;
+  const void* residual;     // [max_seqs][2][H][cap][D]
+  int NB, H, cap, max_seqs;
+  int record, off_v, off_s;
+  int32_t* fault;
+};
+
+// grid (entries, H): quantize ring rows [p0, p0 + 64) of one sequence and kv head into the
+// block's record, exactly as kvq_write stores those rows with slots blk*64 .. blk*64+63.
+template <typename TA, int D>
+__global__ void __launch_bounds__(128) flush_ring_kernel(Int4FlushParams p) {
+  __shared__ float xs[64][D + 1];
+  __shared__ __align__(16) uint8_t cs[64][D];
+  const int e = blockIdx.x, h = blockIdx.y;
+  const int sid = p.seq_ids[e], p0 = p.positions[e], blk = p.blocks[e];
+  int bad = 0;
+  if (sid < 0 || sid >= p.max_seqs) bad = KVQ_FAULT_SEQ;
+  else if (blk < 0 || blk >= p.NB) bad = KVQ_FAULT_BLOCK;
+  else if (p0 < 0 || p0 % 64 != 0) bad = KVQ_FAULT_INT4_RUN;
+  if (bad) {                                // uniform over the CTA
+    if (h == 0 && threadIdx.x == 0) record_fault(p.fault, bad);
+    return;
+  }
+  uint8_t* rec = p.pages + (static_cast<long>(blk) * p.H + h) * p.record;
+  auto row = [&](int kv, int t) {
+    return static_cast<const TA*>(p.residual) +
+           ((static_cast<long>(sid * 2 + kv) * p.H + h) * p.cap + (p0 + t) % p.cap) * D;
+  };
+  quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, xs, cs);
+}
+
 }  // namespace
+
+cudaError_t launch_flush_ring(const kvq_cache_desc& c, const Geometry& g, const int32_t* seq_ids,
+                              const int32_t* positions, const int32_t* blocks, int n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  Int4FlushParams p{seq_ids, positions, blocks, static_cast<uint8_t*>(c.pages), c.residual,
+                    g.NB, g.H, g.residual_cap, g.max_seqs, g.record, g.off_v, g.off_s, c.fault};
+  const dim3 grid(n, g.H);
+  if (g.act_dtype == KVQ_DTYPE_BF16) {
+    if (g.D == 128) flush_ring_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
+    else flush_ring_kernel<__nv_bfloat16, 64><<<grid, 128, 0, s>>>(p);
+  } else {
+    if (g.D == 128) flush_ring_kernel<__half, 128><<<grid, 128, 0, s>>>(p);
+    else flush_ring_kernel<__half, 64><<<grid, 128, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_write_dense(const kvq_cache_desc& c, const Geometry& g, const void* k,
                                const void* v, int T, const int32_t* slots, cudaStream_t s) {

@@ -26,7 +26,7 @@ FAULT_BITS = {"slot": 1, "block": 2, "context": 4, "seq": 8, "int4_run": 16, "ti
 EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
            "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc",
-           "kvq_append_decode_attention", "kvq_calibrate_channel_scales")
+           "kvq_append_decode_attention", "kvq_calibrate_channel_scales", "kvq_flush_ring")
 
 
 class CacheDesc(ctypes.Structure):
@@ -69,6 +69,7 @@ def _load():
         "kvq_append_decode_attention": (I, [D, P, P, P, I, I, P, I, P, I, F, P, ctypes.c_int32, P,
                                             Z, P]),
         "kvq_calibrate_channel_scales": (I, [P, I, I, I, ctypes.c_int32, F, P, P]),
+        "kvq_flush_ring": (I, [D, P, P, P, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -195,6 +196,14 @@ def kvq_calibrate_fp8_scales(x, scale_out, stream=None):
     return scale_out
 
 
+def kvq_flush_ring(desc, seq_ids, positions, block_ids, stream=None):
+    """INT4: quantize ring rows [positions[i], positions[i] + 64) of sequence seq_ids[i]
+    into block block_ids[i] (all kv heads)."""
+    n = int(seq_ids.numel())
+    _check(lib.kvq_flush_ring(ctypes.byref(desc), _ptr(_i32(seq_ids)), _ptr(_i32(positions)),
+                              _ptr(_i32(block_ids)), n, _stream(stream)), "kvq_flush_ring")
+
+
 def kvq_calibrate_channel_scales(x, qmax, scale_out, stream=None):
     """scale_out[h][d] = max over tokens |x[t][h][d]| / qmax (127 INT8, 448 FP8)."""
     T, H, D = x.shape
@@ -280,6 +289,9 @@ class PagedKVCache:
             workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device) if n else None
         return kvq_append_decode_attention(self.desc, k_new, v_new, q, block_tables, context_lens,
                                            max_context, out, workspace, softmax_scale, stream)
+
+    def flush_ring(self, seq_ids, positions, block_ids, stream=None):
+        kvq_flush_ring(self.desc, seq_ids, positions, block_ids, stream)
 
     def dequant(self, block_ids, stream=None):
         out = torch.empty((block_ids.numel(), 2, self.num_kv_heads, self.block_size, self.head_dim),

@@ -288,3 +288,21 @@ def test_int4_prefix_split():
     c = cache.PagedCache("int4", "bf16", "kivi", 4, 64, 1, 128, max_seqs=1)
     assert [c.quantized_prefix(n) for n in (0, 100, 128, 191, 192, 255, 256, 32768)] == \
         [0, 0, 0, 0, 64, 64, 128, 32640]
+
+
+def test_flush_ring_equals_writing_the_rows():
+    """Flushing ring rows [p0, p0+64) into a block stores what writing those rows with the
+    block's slots stores (the definition in include/kvq.h)."""
+    w = inputs.make("c4", small=True)
+    c = _build(w)
+    s = w.spec
+    n0 = int(w.context_lens[0])
+    qb = 64 * (max(n0 - inputs.RESIDUAL_LEN, 0) // 64)
+    used = set(w.block_tables.numpy().reshape(-1).tolist())
+    free = [b for b in range(w.num_blocks) if b not in used][0]
+    c.flush_ring([0], [qb], [free])
+    ref = _build(w)
+    rows = np.arange(int(w.seq_start[0]) + qb, int(w.seq_start[0]) + qb + 64)
+    ref.write(_np(w.k)[rows], _np(w.v)[rows], free * 64 + np.arange(64))
+    np.testing.assert_array_equal(c.pages[free], ref.pages[free])
+    assert not np.array_equal(c.pages[free], _build(w).pages[free])       # it did write
