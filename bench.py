@@ -28,6 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "quantized paged decode attention: KV GB/s and % of HBM roofline; tokens/s"
+FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 
 WORKLOADS = {
@@ -79,6 +80,59 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Measured dense bf16 tensor throughput (burst), TFLOP/s."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def measure_prefill(device, l2, steps=20):
+    """Chunked prefill on a c5-shaped layer (INT8 per-token-head cache, 64/8 heads, D 128,
+    block 16): 4 sequences of 4096 cached tokens whose newest 512 are this chunk's queries,
+    each attending causally.  Algorithmic work: 4 D flops (q.k and p.v) per query head and
+    visible position."""
+    import dataclasses
+    import torch
+    from quantized_paged_kv_02_b200 import inputs, kvq
+    spec = dataclasses.replace(inputs._spec("c5", False), batch=4, lens=[4096] * 4)
+    w = inputs.from_spec(spec, device)
+    s = w.spec
+    c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
+                         s.num_kv_heads, s.head_dim, device=device)
+    c.write(w.k, w.v, w.slot_mapping)
+    L, n = 512, 4096
+    g = torch.Generator(device=device).manual_seed(1)
+    q = torch.randn((s.batch * L, s.num_q_heads, s.head_dim), generator=g, device=device).to(torch.bfloat16)
+    qs = torch.arange(0, s.batch * L + 1, L, dtype=torch.int32, device=device)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=device)
+
+    def call():
+        kvq.kvq_prefill_attention(c.desc, q, qs, L, w.block_tables, w.context_lens, n, out)
+    for _ in range(3):
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        l2.flush()
+        a.record()
+        call()
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    visible = s.batch * sum(n - L + i + 1 for i in range(L))
+    flops = 4.0 * s.head_dim * s.num_q_heads * visible
+    peak, kind = tensor_peak()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+            "frac_of_peak": round(tf / peak, 4), "peak": peak, "peak_kind": kind + " bf16 dense",
+            "config": "c5-shaped layer, INT8 per-token-head cache, 4 sequences x 4096 tokens, "
+                      "512-query causal chunks (kvq_prefill_attention)"}
 
 
 def profile_traffic(workload):
@@ -429,6 +483,9 @@ def main_ours(args):
                  "frac_of_peak": round(step_bytes / (fms * 1e-3) / 1e9 / hbm_peak()[0], 4),
                  "call": "kvq_append_decode_attention (append step fused into the decode kernel)"}
 
+    # chunked prefill on its own c5-shaped case (default workload only)
+    prefill = measure_prefill(device, l2) if args.workload == "c5" and K > 0 else None
+
     # end to end through the C ABI: host inputs in pinned memory, copies inside the region
     E = args.e2e_steps
     h = {k2: new[k2].cpu().pin_memory() for k2 in ("k", "v", "slots")}
@@ -497,6 +554,7 @@ def main_ours(args):
                 "ms_per_step": round(e2e, 5), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "append_decode": fused,
+        "prefill": prefill,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }

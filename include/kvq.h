@@ -291,6 +291,33 @@ kvq_status kvq_append_decode_attention(const kvq_cache_desc* cache, const void* 
                                        cudaStream_t stream);
 
 /*
+ * kvq_prefill_attention - causal attention of a chunk of new queries per sequence over the
+ *   cache (chunked prefill).  The chunk's own K/V rows must already be in the cache
+ *   (kvq_write); the queries are the newest tokens of each sequence.
+ *   q             act_dtype [num_q_tokens][num_q_heads][D], device: the queries of sequence b
+ *                 are rows q_start[b] .. q_start[b+1]-1, in token order.
+ *   q_start       int32 [batch+1], device, non-decreasing, q_start[batch] <= num_q_tokens.
+ *   max_q_len     host upper bound of q_start[b+1] - q_start[b] (sizes the grid); a sequence
+ *                 with more queries, or with more queries than context_lens[b], is skipped
+ *                 and counted (KVQ_FAULT_CONTEXT).
+ *   context_lens  int32 [batch], device: tokens in the cache for sequence b, the chunk's own
+ *                 included.
+ *   out           out_dtype [num_q_tokens][num_q_heads][D], device.
+ *   Other arguments as kvq_decode_attention.  Query i of sequence b sits at position
+ *   p = context_lens[b] - L_b + i (L_b its query count) and attends to positions <= p:
+ *   o = softmax(scale * q . k_t) v_t over t <= p, dequantized inside the kernel.  Chunked
+ *   prefill is one of the techniques [P-prod] "为什么长上下文更需要 KV Cache Quantization"
+ *   names beside KV cache quantization.  Dense caches with block_size 16 and head_dim 128
+ *   (the tensor-core path); others return KVQ_ERR_UNSUPPORTED.  No workspace.
+ */
+kvq_status kvq_prefill_attention(const kvq_cache_desc* cache, const void* q, int num_q_tokens,
+                                 int batch, int num_q_heads, const int32_t* q_start,
+                                 int max_q_len, const int32_t* block_tables,
+                                 int max_blocks_per_seq, const int32_t* context_lens,
+                                 int max_context, float softmax_scale, void* out,
+                                 int32_t out_dtype, cudaStream_t stream);
+
+/*
  * Size of the device scratch array used by kvq_decode_attention_noalloc (16 MiB).  Every
  * GPU that loads the library reserves this much for the life of the process.
  */

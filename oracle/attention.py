@@ -52,3 +52,35 @@ def decode_attention(cache, q, block_tables, context_lens, seq_ids=None,
                 hq = kvh * g + j
                 out[b, hq] = softmax_attention(q[b, hq], K[kvh], V[kvh], scale)
     return out
+
+
+def prefill_attention(cache, q, q_start, block_tables, context_lens, softmax_scale=0.0):
+    """Causal attention of a chunk of new queries over the dequantized cache, float64.
+
+    q [Tq, H_q, D]; the queries of sequence b are rows q_start[b] .. q_start[b+1]-1, the
+    newest tokens of that sequence: query i sits at position p = n_b - L_b + i (n_b =
+    context_lens[b], L_b its query count) and attends to every cached position <= p:
+        z_t = scale * (q . k_t), t <= p;   o = softmax(z) V
+    (chunked prefill, one of the techniques [P-prod] "为什么长上下文更需要 KV Cache
+    Quantization" lists beside KV cache quantization; the chunk's own K/V rows are in the
+    cache before attention runs).  Returns [Tq, H_q, D]; one query row at a time.
+    """
+    q = np.asarray(q, np.float64)
+    Tq, Hq, D = q.shape
+    g = Hq // cache.H
+    scale = softmax_scale if softmax_scale else 1.0 / np.sqrt(D)
+    out = np.zeros((Tq, Hq, D), np.float64)
+    qs = np.asarray(q_start)
+    for b in range(len(context_lens)):
+        n = int(context_lens[b])
+        L = int(qs[b + 1] - qs[b])
+        if L == 0:
+            continue
+        K, V = cache.gather(block_tables[b], n)
+        for i in range(L):
+            p = n - L + i
+            for hq in range(Hq):
+                kvh = hq // g
+                out[qs[b] + i, hq] = softmax_attention(q[qs[b] + i, hq], K[kvh][:p + 1],
+                                                       V[kvh][:p + 1], scale)
+    return out

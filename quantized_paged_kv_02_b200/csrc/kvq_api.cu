@@ -254,6 +254,47 @@ kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_head
   return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, scale_out, stream));
 }
 
+kvq_status kvq_prefill_attention(const kvq_cache_desc* c, const void* q, int num_q_tokens, int batch,
+                                 int num_q_heads, const int32_t* q_start, int max_q_len,
+                                 const int32_t* block_tables, int max_blocks_per_seq,
+                                 const int32_t* context_lens, int max_context, float softmax_scale,
+                                 void* out, int32_t out_dtype, cudaStream_t stream) {
+  Geometry g;
+  kvq_status st = validate_desc(c, &g);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_tokens < 0 || max_q_len < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 ||
+      max_context < 0 || max_blocks_per_seq < 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (out_dtype != KVQ_DTYPE_BF16 && out_dtype != KVQ_DTYPE_FP16 && out_dtype != KVQ_DTYPE_FP32)
+    return KVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  DecodeArgs a{};
+  a.c = c;
+  a.geo = g;
+  st = plan_decode(g, std::max(batch, 1), num_q_heads, max_context, &a.plan);
+  if (st != KVQ_OK) return st;
+  if (a.plan.kernel != 1) return KVQ_ERR_UNSUPPORTED;     // tensor-core geometries only
+  if (batch == 0 || num_q_tokens == 0 || max_q_len == 0) return KVQ_OK;
+  if (q == nullptr || q_start == nullptr || block_tables == nullptr || context_lens == nullptr ||
+      out == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out)) return KVQ_ERR_INVALID_ARG;
+  a.q = q;
+  a.q_start = q_start;
+  a.max_q_len = max_q_len;
+  a.batch = batch;
+  a.Hq = num_q_heads;
+  a.block_tables = block_tables;
+  a.max_blocks = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.max_context = max_context;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(g.D));
+  a.scale_log2 = scale * kLog2e;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  return from_cuda(launch_prefill(a, stream));
+}
+
 kvq_status kvq_flush_ring(const kvq_cache_desc* c, const int32_t* seq_ids, const int32_t* positions,
                           const int32_t* block_ids, int n, cudaStream_t stream) {
   Geometry g;

@@ -264,7 +264,7 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
   return KVQ_OK;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+static DecodeParams make_params(const DecodeArgs& a) {
   const Geometry& g = a.geo;
   DecodeParams p{};
   p.q = a.q;
@@ -307,6 +307,13 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   p.k_new = a.k_new;
   p.v_new = a.v_new;
   p.pages_w = a.k_new != nullptr ? static_cast<uint8_t*>(a.c->pages) : nullptr;
+  p.q_start = a.q_start;
+  return p;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+  const Geometry& g = a.geo;
+  DecodeParams p = make_params(a);
   if (a.batch == 0) return cudaSuccess;
   cudaError_t e;
   if (a.plan.kernel == 2) {
@@ -323,6 +330,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     e = cudaGetLastError();
   }
   return e;
+}
+
+cudaError_t launch_prefill(const DecodeArgs& a, cudaStream_t s) {
+  if (a.batch == 0) return cudaSuccess;
+  return launch_prefill_mma(a, make_params(a), s);
 }
 
 }  // namespace kvq

@@ -37,6 +37,9 @@ struct DecodeParams {
   const void* k_new;
   const void* v_new;
   uint8_t* pages_w;          // the pool, writable (append step only)
+  // prefill (kvq_prefill_attention): q is [Tq][Hq][D]; the queries of sequence b are rows
+  // q_start[b] .. q_start[b+1]-1, the newest tokens of the sequence
+  const int32_t* q_start;
 };
 
 struct SeqInfo {
@@ -137,6 +140,7 @@ __device__ __forceinline__ void store_partial_or_output(const DecodeParams& p, i
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_prefill_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 // true when the tensor-core kernel covers this geometry and GQA group size
 bool mma_supported(const Geometry& g, int group);
 bool int4_mma_supported(const Geometry& g, int group);

@@ -86,7 +86,11 @@ __device__ __forceinline__ int swzb(int off) {
   return (off & ~127) + ((((off >> 4) & 7) ^ ((off >> 7) & 7)) << 4) + (off & 15);
 }
 
-template <int CD, int BS, bool PT>
+// PF false: decode, grid kMmaCtas over page-balanced ranges.  PF true: chunked prefill,
+// grid (query groups of kConsumers tokens, kv heads, sequences); each consumer warp owns one
+// query token (with its g heads), reads every page its causal window covers and writes
+// its output rows itself.
+template <int CD, int BS, bool PT, bool PF>
 __global__ void __launch_bounds__(kThreads, 3)
 decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   using L = Layout<CD, BS, PT>;
@@ -111,17 +115,42 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   // inputs (pages, q, tables, lengths) may come from the kernel just before this one
   griddep_wait();
   griddep_launch_dependents();
+  // prefill: this CTA's sequence, kv head, first query of its group, and the group's
+  // query count L and context n of the sequence
+  int pf_b = 0, pf_kvh = 0, pf_q0 = 0, pf_L = 0, pf_n = 0;
+  if constexpr (PF) {
+    pf_b = blockIdx.z;
+    pf_kvh = blockIdx.y;
+    pf_q0 = blockIdx.x * kConsumers;
+    pf_L = p.q_start[pf_b + 1] - p.q_start[pf_b];
+    pf_n = seq_info(p, pf_b, false, blockIdx.x == 0 && pf_kvh == 0 && threadIdx.x == 0).n;
+    // more queries than positions, or than the grid covers (max_q_len): rejected
+    if (pf_L > pf_n || pf_L > static_cast<int>(gridDim.x) * kConsumers || pf_L < 0) {
+      if (blockIdx.x == 0 && pf_kvh == 0 && threadIdx.x == 0) record_fault(p.fault, KVQ_FAULT_CONTEXT);
+      pf_L = 0;
+    }
+    if (pf_q0 >= pf_L) return;                  // no query of this group (uniform)
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], PF ? kConsumers : 1);   // prefill: every consumer reads every page
     }
     fence_mbar_init();
   }
   // The producer finds this CTA's page range [start, end) and the sequence it starts in.
   long long start = 0, end = 0, seq_first_page = 0;
   int b_first = 0;
-  if (warp == kConsumers) {
+  if constexpr (PF) {
+    // pages [0, npages) of unit (b, kvh): the causal window of the group's last query
+    const int last = pf_n - pf_L + min(pf_q0 + kConsumers, pf_L) - 1;
+    const int npb = (pf_n + BS - 1) / BS;
+    b_first = pf_b;
+    seq_first_page = 0;                         // unit (b, kvh) starts at kvh * npb
+    start = static_cast<long long>(pf_kvh) * npb;
+    end = start + (last + BS) / BS;
+    if (warp == kConsumers && lane == 0) *range_pages = static_cast<int>(end - start);
+  } else if (warp == kConsumers) {
     long long tot = 0;
     for (int b0 = 0; b0 < p.batch; b0 += 32) {
       int np = b0 + lane < p.batch ? seq_pages(p, b0 + lane, cta == 0) : 0;
@@ -292,7 +321,7 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
 
   // Load the query group of unit u = (sequence, kv head) into fragments and clear the
   // running softmax state.
-  auto begin_unit = [&](int u) {
+  auto begin_unit = [&](int u, long qrow) {     // qrow: row of q ([B] decode, [Tq] prefill)
     const int b = u / p.H;
     kvh = u - b * p.H;
     qscale = p.scale_log2;
@@ -300,7 +329,7 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     uint4 qraw[4];
     if (r < g) {
       const uint4* qp = reinterpret_cast<const uint4*>(
-          static_cast<const uint16_t*>(p.q) + (static_cast<long>(b) * p.Hq + kvh * g + r) * kD + 32 * j);
+          static_cast<const uint16_t*>(p.q) + (qrow * p.Hq + kvh * g + r) * kD + 32 * j);
 #pragma unroll
       for (int c = 0; c < 4; ++c) qraw[c] = qp[c];
     } else {
@@ -428,6 +457,46 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     }
   };
 
+  // Prefill: normalise and store this warp's output rows (query row qrow, its g heads).
+  auto write_rows = [&](long qrow) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
+      l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
+    }
+    float vmul = 1.f;
+    if constexpr (PT) vmul = ev == INT_MIN ? 0.f : ldexpf(1.f, ev);
+    if constexpr (!PT) {
+      if (p.mode == KVQ_SCALE_PER_HEAD) vmul = p.v_static[kvh];
+      if (p.mode == KVQ_SCALE_PER_TENSOR) vmul = p.v_static[0];
+    }
+    const float* vch = nullptr;
+    if constexpr (!PT && Code<CD>::B == 1) {
+      if (p.mode == KVQ_SCALE_PER_CHANNEL) vch = p.v_static + kvh * kD;
+    }
+    const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
+    const int h0 = 2 * j, h1 = 2 * j + 1;
+    const long base = (qrow * p.Hq + static_cast<long>(kvh) * g) * kD;
+#pragma unroll
+    for (int md = 0; md < 8; ++md) {
+      const int d0 = 16 * r + 2 * md;
+      float m0 = vmul, m1 = vmul;
+      if (vch != nullptr) {
+        const float2 cv = *reinterpret_cast<const float2*>(vch + d0);
+        m0 = cv.x;
+        m1 = cv.y;
+      }
+      if (h0 < g) {
+        store_out(p, base + h0 * kD + d0, o[md][0] * m0 * inv0);
+        store_out(p, base + h0 * kD + d0 + 1, o[md][2] * m1 * inv0);
+      }
+      if (h1 < g) {
+        store_out(p, base + h1 * kD + d0, o[md][1] * m0 * inv1);
+        store_out(p, base + h1 * kD + d0 + 1, o[md][3] * m1 * inv1);
+      }
+    }
+  };
+
   // Per-thread byte offsets inside a stage tile.  The 128-byte swizzle repeats every 8
   // rows of 128 bytes, so token row t + 8 sits exactly 8 * ROWB bytes after row t.
   // K: token rows r and r+8, this thread's 32 codes [32j, 32j+32) of each row.
@@ -450,7 +519,20 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   static_assert(!PT || (L::OFF_S % 1024 == 0 && 8 * BS == 128), "scale row layout");
   const int soff = L::OFF_S + 4 * r;
 
-  for (int i = warp; i < npages; i += kConsumers) {
+  // prefill: this warp's query token (row of q and out) and its causal window [0, t1)
+  long pf_row = 0;
+  int pf_t1 = 0;
+  bool pf_active = false;
+  if constexpr (PF) {
+    const int idx = pf_q0 + warp;
+    pf_active = idx < pf_L;
+    pf_row = p.q_start[pf_b] + idx;
+    pf_t1 = pf_n - pf_L + idx + 1;
+    cur_u = pf_b * p.H + pf_kvh;
+    if (pf_active) begin_unit(cur_u, pf_row);
+  }
+
+  for (int i = PF ? 0 : warp; i < npages; i += PF ? 1 : kConsumers) {
     const int s = i % kStages;
     // all lanes wait; the decision is made warp-uniform before any shuffle below
     if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kStages) & 1))) {
@@ -458,14 +540,23 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       break;
     }
     const int4 mt = meta[s];
-    if (mt.x != cur_u) {              // warp-uniform: a new (sequence, kv head) unit
-      if (cur_u >= 0) end_unit();
-      cur_u = mt.x;
-      begin_unit(cur_u);
+    if constexpr (!PF) {
+      if (mt.x != cur_u) {              // warp-uniform: a new (sequence, kv head) unit
+        if (cur_u >= 0) end_unit();
+        cur_u = mt.x;
+        begin_unit(cur_u, cur_u / p.H);
+      }
     }
     const uint8_t* st = tiles + s * STAGE;
     const bool pvalid = mt.w != 0;
-    const int pos0 = mt.y * BS, t1 = mt.z;
+    const int pos0 = mt.y * BS, t1 = PF ? pf_t1 : mt.z;
+    if constexpr (PF) {
+      if (!pf_active || pos0 >= t1) {   // nothing of this page is in the warp's window
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        continue;
+      }
+    }
     const bool full_page = pvalid && pos0 + BS <= t1;          // warp-uniform
     // ------------------------------------------------ stage -> registers, then hand the
     // stage back to the producer before any math, so the ring refills during compute
@@ -709,21 +800,25 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       }
     }
   }
-  if (cur_u >= 0) end_unit();
+  if constexpr (PF) {
+    if (pf_active) write_rows(pf_row);
+  } else {
+    if (cur_u >= 0) end_unit();
+  }
 }
 
-template <int CD, int BS, bool PT>
+template <int CD, int BS, bool PT, bool PF>
 cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
   using L = Layout<CD, BS, PT>;
   if (a.geo.record != L::REC) return cudaErrorInvalidValue;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(decode_mma_kernel<CD, BS, PT>,
+    attr_err = cudaFuncSetAttribute(decode_mma_kernel<CD, BS, PT, PF>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     // three rings per SM need the whole unified L1 / shared memory as shared memory
     if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(decode_mma_kernel<CD, BS, PT>,
+      attr_err = cudaFuncSetAttribute(decode_mma_kernel<CD, BS, PT, PF>,
                                       cudaFuncAttributePreferredSharedMemoryCarveout,
                                       cudaSharedmemCarveoutMaxShared);
   });
@@ -731,13 +826,14 @@ cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s)
   CUtensorMap tm;
   const long rows = static_cast<long>(a.geo.NB) * a.geo.H * L::REC_ROWS;
   if (!make_pages_map(&tm, a.c->pages, rows, L::REC_ROWS)) return cudaErrorInvalidValue;
-  return launch_dependent(decode_mma_kernel<CD, BS, PT>, dim3(a.plan.ctas), dim3(kThreads), L::BYTES,
-                          s, p, tm);
+  const dim3 grid = PF ? dim3((a.max_q_len + kConsumers - 1) / kConsumers, a.geo.H, a.batch)
+                       : dim3(a.plan.ctas);
+  return launch_dependent(decode_mma_kernel<CD, BS, PT, PF>, grid, dim3(kThreads), L::BYTES, s, p, tm);
 }
 
-template <int CD, bool PT>
+template <int CD, bool PT, bool PF>
 cudaError_t launch_bs(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
-  if (a.geo.bs == 16) return launch_t<CD, 16, PT>(a, p, s);
+  if (a.geo.bs == 16) return launch_t<CD, 16, PT, PF>(a, p, s);
   return cudaErrorInvalidValue;
 }
 
@@ -790,16 +886,27 @@ bool mma_supported(const Geometry& g, int groups) {
   return false;
 }
 
-cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+template <bool PF>
+static cudaError_t launch_mma_mode(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
   const bool pt = a.geo.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD;
   switch (a.geo.cache_dtype) {
-    case KVQ_DTYPE_INT8: return pt ? launch_bs<KVQ_DTYPE_INT8, true>(a, p, s) : launch_bs<KVQ_DTYPE_INT8, false>(a, p, s);
+    case KVQ_DTYPE_INT8:
+      return pt ? launch_bs<KVQ_DTYPE_INT8, true, PF>(a, p, s) : launch_bs<KVQ_DTYPE_INT8, false, PF>(a, p, s);
     case KVQ_DTYPE_FP8_E4M3:
-      return pt ? launch_bs<KVQ_DTYPE_FP8_E4M3, true>(a, p, s) : launch_bs<KVQ_DTYPE_FP8_E4M3, false>(a, p, s);
-    case KVQ_DTYPE_BF16: return launch_bs<KVQ_DTYPE_BF16, false>(a, p, s);
-    case KVQ_DTYPE_FP16: return launch_bs<KVQ_DTYPE_FP16, false>(a, p, s);
+      return pt ? launch_bs<KVQ_DTYPE_FP8_E4M3, true, PF>(a, p, s)
+                : launch_bs<KVQ_DTYPE_FP8_E4M3, false, PF>(a, p, s);
+    case KVQ_DTYPE_BF16: return launch_bs<KVQ_DTYPE_BF16, false, PF>(a, p, s);
+    case KVQ_DTYPE_FP16: return launch_bs<KVQ_DTYPE_FP16, false, PF>(a, p, s);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  return launch_mma_mode<false>(a, p, s);
+}
+
+cudaError_t launch_prefill_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  return launch_mma_mode<true>(a, p, s);
 }
 
 }  // namespace kvq

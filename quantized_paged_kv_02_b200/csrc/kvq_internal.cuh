@@ -176,6 +176,8 @@ struct DecodeArgs {
   const void* q;
   const void* k_new;         // append step: [B][H][D] act dtype, else null
   const void* v_new;
+  const int32_t* q_start;    // prefill: [B+1] query rows of each sequence, else null
+  int max_q_len;             // prefill: host bound on q_start[b+1] - q_start[b]
   int batch, Hq;
   const int32_t* block_tables;
   int max_blocks;
@@ -190,6 +192,7 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_prefill(const DecodeArgs& a, cudaStream_t s);
 
 // Launch `kernel` so that it may start while the previous kernel in the stream is still
 // running (programmatic dependent launch); the kernel must call griddep_wait() before it

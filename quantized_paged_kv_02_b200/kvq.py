@@ -26,7 +26,8 @@ FAULT_BITS = {"slot": 1, "block": 2, "context": 4, "seq": 8, "int4_run": 16, "ti
 EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
            "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc",
-           "kvq_append_decode_attention", "kvq_calibrate_channel_scales", "kvq_flush_ring")
+           "kvq_append_decode_attention", "kvq_calibrate_channel_scales", "kvq_flush_ring",
+           "kvq_prefill_attention")
 
 
 class CacheDesc(ctypes.Structure):
@@ -70,6 +71,7 @@ def _load():
                                             Z, P]),
         "kvq_calibrate_channel_scales": (I, [P, I, I, I, ctypes.c_int32, F, P, P]),
         "kvq_flush_ring": (I, [D, P, P, P, I, P]),
+        "kvq_prefill_attention": (I, [D, P, I, I, I, P, I, P, I, P, I, F, P, ctypes.c_int32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -196,6 +198,21 @@ def kvq_calibrate_fp8_scales(x, scale_out, stream=None):
     return scale_out
 
 
+def kvq_prefill_attention(desc, q, q_start, max_q_len, block_tables, context_lens, max_context,
+                          out, softmax_scale=0.0, stream=None):
+    """Causal attention of each sequence's chunk of new queries (rows q_start[b] ..
+    q_start[b+1]-1 of q) over the cache."""
+    Tq, Hq, _ = q.shape
+    B = int(q_start.numel()) - 1
+    out_dt = {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float32: "fp32"}[out.dtype]
+    _check(lib.kvq_prefill_attention(
+        ctypes.byref(desc), _ptr(q), Tq, B, Hq, _ptr(_i32(q_start)), int(max_q_len),
+        _ptr(_i32(block_tables)), int(block_tables.shape[1]), _ptr(_i32(context_lens)),
+        int(max_context), float(softmax_scale), _ptr(out), DTYPE[out_dt], _stream(stream)),
+        "kvq_prefill_attention")
+    return out
+
+
 def kvq_flush_ring(desc, seq_ids, positions, block_ids, stream=None):
     """INT4: quantize ring rows [positions[i], positions[i] + 64) of sequence seq_ids[i]
     into block block_ids[i] (all kv heads)."""
@@ -289,6 +306,13 @@ class PagedKVCache:
             workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device) if n else None
         return kvq_append_decode_attention(self.desc, k_new, v_new, q, block_tables, context_lens,
                                            max_context, out, workspace, softmax_scale, stream)
+
+    def prefill(self, q, q_start, max_q_len, block_tables, context_lens, max_context, out=None,
+                out_dtype=torch.float32, softmax_scale=0.0, stream=None):
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        return kvq_prefill_attention(self.desc, q, q_start, max_q_len, block_tables, context_lens,
+                                     max_context, out, softmax_scale, stream)
 
     def flush_ring(self, seq_ids, positions, block_ids, stream=None):
         kvq_flush_ring(self.desc, seq_ids, positions, block_ids, stream)

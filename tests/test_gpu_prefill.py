@@ -1,0 +1,114 @@
+"""kvq_prefill_attention (chunked prefill) against the float64 oracle.
+
+Each sequence's chunk of new queries is its newest tokens (their K/V rows already in the
+cache); query i at position p attends to positions <= p.  Tolerance as decode: max
+|gpu - oracle| <= 2e-3 with float32 output.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention
+from quantized_paged_kv_02_b200 import inputs, kvq
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    helpers.ensure_built()
+
+
+def _queries(w, L, seed):
+    g = torch.Generator().manual_seed(seed)
+    qs = torch.tensor(np.concatenate([[0], np.cumsum(L)]), dtype=torch.int32)
+    q = torch.randn((int(qs[-1]), w.spec.num_q_heads, w.spec.head_dim), generator=g)
+    return q.to(inputs.act_torch_dtype(w.spec.act_dtype)), qs
+
+
+def _prefill(gc, w, q, qs, lens=None):
+    lens = w.context_lens if lens is None else lens
+    L = (qs[1:] - qs[:-1])
+    return gc.prefill(q.cuda(), qs.cuda(), int(L.max()), w.block_tables.cuda(), lens.cuda(),
+                      int(lens.max()))
+
+
+@pytest.mark.parametrize("name,L", [("c5", [37, 1, 33]), ("c5-fp8", [64, 5, 17]),
+                                    ("c5-bf16", [3, 200, 33]), ("c5-int8-pc", [9, 16, 1]),
+                                    ("c3", [7, 30, 1, 12]), ("c2", [40, 19])])
+def test_prefill_matches_oracle(name, L):
+    w = inputs.make(name, small=True)
+    L = [min(x, int(n)) for x, n in zip(L, w.context_lens.tolist())]
+    static = helpers.oracle_static_scales(w)
+    oc = helpers.oracle_cache(w, static)
+    gc = helpers.gpu_cache(w, static=static)
+    q, qs = _queries(w, L, 3)
+    got = _prefill(gc, w, q, qs).cpu().numpy().astype(np.float64)
+    want = attention.prefill_attention(oc, helpers.np64(q), qs.numpy(), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    err = np.abs(got - want).max()
+    assert err <= TOL, err
+    assert gc.read_fault() == (0, 0)
+
+
+def test_one_query_chunk_is_decode():
+    w = inputs.make("c5", small=True)
+    gc = helpers.gpu_cache(w)
+    qs = torch.arange(w.spec.batch + 1, dtype=torch.int32)
+    pre = _prefill(gc, w, w.q, qs)
+    dec = gc.decode(w.q.cuda(), w.block_tables.cuda(), w.context_lens.cuda(), w.max_context)
+    torch.cuda.synchronize()
+    assert (pre - dec).abs().max().item() <= 1e-5
+
+
+def test_rejected_sequences_are_counted_and_left_untouched():
+    w = inputs.make("c5", small=True)
+    gc = helpers.gpu_cache(w)
+    L = [5, 4, 2]
+    q, qs = _queries(w, L, 4)
+    lens = w.context_lens.clone()
+    lens[1] = 3                                   # 4 queries but 3 positions: rejected
+    out = torch.full((int(qs[-1]), w.spec.num_q_heads, w.spec.head_dim), 7.0, device="cuda")
+    kvq.kvq_prefill_attention(gc.desc, q.cuda(), qs.cuda(), 4, w.block_tables.cuda(), lens.cuda(),
+                              int(lens.max()), out)  # max_q_len 4 < 5: sequence 0 rejected too
+    torch.cuda.synchronize()
+    cnt, bits = gc.read_fault()
+    assert cnt >= 2 and (bits & 4)
+    assert torch.all(out[qs[0]:qs[2]] == 7.0)
+    assert torch.all(out[qs[2]:qs[3]] != 7.0)
+
+
+def test_prefill_rejects_unsupported_caches():
+    w = inputs.make("c4", small=True)
+    c = helpers.gpu_cache(w)
+    q, qs = _queries(w, [2, 2], 5)
+    with pytest.raises(kvq.KVQError):
+        _prefill(c, w, q, qs)
+
+
+def test_prefill_full_size_sampled_queries():
+    """A c5-shaped layer (batch 4, context 4096, 512-query chunks) at full size; sampled
+    queries are checked against the oracle's decode at their positions (equal to prefill
+    rows by definition, pinned on the CPU)."""
+    import dataclasses
+    spec = dataclasses.replace(inputs._spec("c5", False), batch=4, lens=[4096] * 4)
+    w = inputs.from_spec(spec, "cuda")
+    gc = helpers.gpu_cache(w)
+    L = [512, 512, 300, 1]
+    q, qs = _queries(w, L, 6)
+    got = _prefill(gc, w, q, qs).cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    for b in (0, 2, 3):
+        sub = helpers.single_sequence(w, b)
+        oc = helpers.oracle_cache(sub)
+        for i in sorted({0, L[b] // 2, L[b] - 1}):
+            p = int(w.context_lens[b]) - L[b] + i
+            want = attention.decode_attention(oc, helpers.np64(q[qs[b] + i])[None],
+                                              sub.block_tables.numpy(), np.array([p + 1]))[0]
+            err = np.abs(got[qs[b] + i] - want).max()
+            assert err <= TOL, (b, i, err)
+    assert gc.read_fault() == (0, 0)

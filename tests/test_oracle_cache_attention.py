@@ -306,3 +306,44 @@ def test_flush_ring_equals_writing_the_rows():
     ref.write(_np(w.k)[rows], _np(w.v)[rows], free * 64 + np.arange(64))
     np.testing.assert_array_equal(c.pages[free], ref.pages[free])
     assert not np.array_equal(c.pages[free], _build(w).pages[free])       # it did write
+
+
+def test_prefill_rows_are_decode_at_their_positions():
+    """Query i of a chunk at position p sees exactly what decode with context p + 1 sees;
+    a one-token chunk is decode."""
+    w = inputs.make("c5", small=True)
+    c = _build(w)
+    lens = w.context_lens.numpy()
+    L = np.array([5, 1, 33])                     # chunk lengths (the last L_b tokens)
+    qs = np.concatenate([[0], np.cumsum(L)])
+    rng = np.random.default_rng(7)
+    q = fp.bf16_round(rng.standard_normal((qs[-1], w.spec.num_q_heads, w.spec.head_dim)))
+    out = attention.prefill_attention(c, q, qs, w.block_tables.numpy(), lens)
+    for b in range(len(lens)):
+        for i in range(L[b]):
+            p = lens[b] - L[b] + i
+            want = attention.decode_attention(c, q[qs[b] + i][None], w.block_tables.numpy()[b:b + 1],
+                                              np.array([p + 1]))
+            np.testing.assert_array_equal(out[qs[b] + i], want[0])
+
+
+def test_prefill_grid_exact_equals_causal_sdpa():
+    """On a grid-exact INT8 cache the chunk's output equals torch's causal SDPA over the
+    dense rows (the prefix positions are all visible, the chunk is causal)."""
+    rng = np.random.default_rng(8)
+    T, H, D, g, bs, L = 45, 2, 64, 2, 16, 13
+    K = _grid_int8_rows(rng, T, H, D)
+    V = _grid_int8_rows(rng, T, H, D)
+    nblk = -(-T // bs)
+    c = cache.PagedCache("int8", "bf16", "per_token_head", nblk, bs, H, D)
+    c.write(K, V, np.arange(T))
+    q = fp.bf16_round(rng.standard_normal((L, H * g, D)))
+    out = attention.prefill_attention(c, q, np.array([0, L]), np.arange(nblk)[None], np.array([T]))
+    for hq in range(H * g):
+        qq = torch.from_numpy(q[:, hq])[None, None]                     # [1, 1, L, D]
+        kk = torch.from_numpy(K[:, hq // g])[None, None]                # [1, 1, T, D]
+        vv = torch.from_numpy(V[:, hq // g])[None, None]
+        mask = torch.ones(L, T, dtype=torch.bool).tril(diagonal=T - L)  # query i sees t <= T-L+i
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask,
+                                                               scale=1.0 / np.sqrt(D))[0, 0]
+        np.testing.assert_allclose(out[:, hq], ref.numpy(), rtol=1e-12, atol=1e-12)
