@@ -6,14 +6,20 @@
 //   k_hat[t][d] = (c[t][d] - zk[d]) * sk[d]   (one (scale, zero) per channel per block)
 //   v_hat[t][d] = (c[t][d] - zv[t][G]) * sv[t][G]   (G = the 64-channel group of d)
 // A per-channel key scale cannot leave the sum over channels, so for each block the
-// consumer forms q'[d] = q[d] * sk[d] (exact in fp32; split into fp16 hi + lo halves, 22
-// bits, so nothing is lost) and the tensor cores see integer A values (c - zk) in fp16:
-// nibbles are placed in the mantissa of 1024.0 and (1024 + zk) is subtracted, exactly.
-// S^T = (C - Zk) Q'^T with two mma.sync m16n8k16 per k-step.  For P V, the value scale
-// of each token's channel group is folded into P (one P operand per group, with the same
-// power-of-two normaliser as the INT8 kernel), and A = (c - zv) of two tokens per register
-// is assembled with a byte permute.  The residual ring (the newest tokens, unquantized)
-// is a separate split handled by the CUDA-core kernel; the reduce merges both.
+// consumer forms q'[d] = q[d] * sk[d] (fp32; split into fp16 hi + lo halves, 22 bits).  The
+// 4-bit codes go to the tensor cores as they are: a code in the mantissa bits of an fp16
+// with a zero exponent is the exact subnormal c * 2^-24, so one mask per register pair
+// replaces a conversion.  The zero points come out as sums computed beside the MMAs:
+//   S^T[t] = 2^24 * (C Q'^T)[t] - sum_d q'[d] zk[d]           (one term per block and head)
+//   O[d]   = 2^24 * (C^T P'^T)[d] - sum_t p'[t] zv[t][G(d)]    (one term per head and group)
+// where p' is P with each token's value scale folded in (per channel group, with the same
+// power-of-two normaliser as the INT8 kernel); the value-side sums follow every rescale
+// of O.  Both subtracted terms and the products they cancel are of similar size (codes
+// and zero points are both in [0, 15]), so the cancellation costs a few bits of fp32.
+// S^T = C Q'^T with two mma.sync m16n8k16 per k-step (hi and lo halves of q').  For P V,
+// A holds the codes of two tokens per register, assembled with a byte permute.  The
+// residual ring (the newest tokens, unquantized) is a separate split handled by the
+// CUDA-core kernel; the reduce merges both.
 //
 // Structure as the dense tensor-core kernel: warp 4 stages one 9 KiB record per block
 // (64 tokens of K and V codes plus all scales and zero points) with one 128-byte-swizzled
@@ -42,7 +48,11 @@ constexpr int kOffVsz = kOffKs + 4 * kD;  // 8704: V (scale, zero) [64][2][2] fp
 constexpr int kRec = kOffVsz + kBS * 2 * 4;   // 9216
 constexpr int kRecRows = kRec / 128;      // 72
 constexpr int kStage = kRec;              // already a multiple of 1024
-constexpr int kStages = 7;
+// Consumers take blocks round-robin, so every round of a stage must go to the same warp
+// (a warp waiting for round r of a stage whose round r-1 belonged to another warp, not yet
+// landed, would see the parity of round r-2 as complete): a multiple of kC stages.
+constexpr int kStages = 8;
+static_assert(kStages % kC == 0, "ring depth is a multiple of the consumers");
 constexpr int kTiles = kStages * kStage;
 constexpr int kBytes = 1024 + kTiles + kStages * 16 + kStages * 4;
 constexpr float kRescale4 = 8.f;
@@ -53,25 +63,10 @@ __device__ __forceinline__ int swzb4(int off) {
   return (off & ~127) + ((((off >> 4) & 7) ^ ((off >> 7) & 7)) << 4) + (off & 15);
 }
 
-// (nibble s, nibble s+4) of w as fp16 (1024 + code) pairs minus the constant pair zc
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int s, uint32_t zc) {
-  const uint32_t h = ((w >> (4 * s)) & 0x000F000Fu) | 0x64006400u;
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(zc));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
+// (nibble s, nibble s+4) of w as the fp16 bit patterns of (code_s, code_s+4) * 2^-24: a
+// 4-bit code placed in the mantissa of a zero exponent is an exact fp16 subnormal, so the
+// tensor cores see c * 2^-24 with no conversion instruction
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int s) { return (w >> (4 * s)) & 0x000F000Fu; }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -103,6 +98,7 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   __syncthreads();
 
   float o[8][4];
+  float cz[2][2] = {{0.f, 0.f}, {0.f, 0.f}};      // [group][head 2j, 2j+1]: sum p' z
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
   int ev = INT_MIN;
   const int r = lane >> 2, j = lane & 3;
@@ -211,7 +207,8 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       // q'[e] = q[32j+e] * sk[32j+e]; k-step kc uses channel pairs (8w+sp, 8w+sp+4) and
       // (8w+sp+1, 8w+sp+5) with w = kc/2, sp = 2*(kc%2): the pairs the nibble extraction
       // of word w yields.
-      uint32_t qh[8][2], ql[8][2], zc[4][4];
+      uint32_t qh[8][2], ql[8][2];
+      float ck0, ck1;
       {
         uint32_t sw[16], zw[16];
 #pragma unroll
@@ -240,16 +237,16 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           ql[kc][0] = pack_f16x2(a0 - f0.x, a1 - f0.y);
           ql[kc][1] = pack_f16x2(c0 - f1.x, c1 - f1.y);
         }
-        // (1024 + zk[8w+sp'], 1024 + zk[8w+sp'+4]) for sp' = 0..3
+        float corr = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-#pragma unroll
-          for (int sp = 0; sp < 4; ++sp) {
-            const int ea = 8 * w + sp, eb = ea + 4;      // halves ea, eb of zw
-            const uint32_t sel = ((ea & 1) ? 0x0032u : 0x0010u) | ((eb & 1) ? 0x7600u : 0x5400u);
-            const uint32_t pair = prmt(zw[ea >> 1], zw[eb >> 1], sel);
-            zc[w][sp] = hadd2(pair, 0x64006400u);
-          }
+        for (int e = 0; e < 16; ++e) {
+          const float2 z = __half22float2(*reinterpret_cast<const __half2*>(&zw[e]));
+          corr = fmaf(qs[2 * e], z.x, fmaf(qs[2 * e + 1], z.y, corr));
+        }
+        corr += __shfl_xor_sync(0xffffffffu, corr, 1);
+        corr += __shfl_xor_sync(0xffffffffu, corr, 2);
+        ck0 = __shfl_sync(0xffffffffu, corr, 8 * j);
+        ck1 = __shfl_sync(0xffffffffu, corr, 8 * j + 4);
       }
 #pragma unroll 1
       for (int mt = 0; mt < kBS / 16; ++mt) {
@@ -262,14 +259,14 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
           const int w = kc >> 1, sp = 2 * (kc & 1);
-          const uint32_t a[4] = {nib_pair(w0[w], sp, zc[w][sp]), nib_pair(w1[w], sp, zc[w][sp]),
-                                 nib_pair(w0[w], sp + 1, zc[w][sp + 1]), nib_pair(w1[w], sp + 1, zc[w][sp + 1])};
+          const uint32_t a[4] = {nib_pair(w0[w], sp), nib_pair(w1[w], sp), nib_pair(w0[w], sp + 1),
+                                 nib_pair(w1[w], sp + 1)};
           mma_f16(sa, a, qh[kc]);
           mma_f16(sb, a, ql[kc]);
         }
         // ------------------------------------------------ softmax (log2 domain)
-        float s00 = (sa[0] + sb[0]) * qscale, s01 = (sa[1] + sb[1]) * qscale;
-        float s10 = (sa[2] + sb[2]) * qscale, s11 = (sa[3] + sb[3]) * qscale;
+        float s00 = fmaf(sa[0] + sb[0], 16777216.f, -ck0) * qscale, s01 = fmaf(sa[1] + sb[1], 16777216.f, -ck1) * qscale;
+        float s10 = fmaf(sa[2] + sb[2], 16777216.f, -ck0) * qscale, s11 = fmaf(sa[3] + sb[3], 16777216.f, -ck1) * qscale;
         const bool grow = s00 > m[0] + kRescale4 || s10 > m[0] + kRescale4 ||
                           s01 > m[1] + kRescale4 || s11 > m[1] + kRescale4;
         if (__any_sync(0xffffffffu, grow)) {
@@ -286,6 +283,7 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           m[1] = mn1;
           l[0] *= c0;
           l[1] *= c1;
+          cz[0][0] *= c0; cz[1][0] *= c0; cz[0][1] *= c1; cz[1][1] *= c1;
 #pragma unroll
           for (int md = 0; md < 8; ++md) {
             o[md][0] *= c0;
@@ -316,6 +314,7 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             if (e > ev) {
               if (ev != INT_MIN) {
                 const float down = pow2i(ev - e);
+                cz[0][0] *= down; cz[0][1] *= down; cz[1][0] *= down; cz[1][1] *= down;
 #pragma unroll
                 for (int md = 0; md < 8; ++md)
 #pragma unroll
@@ -332,6 +331,10 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         for (int G = 0; G < 2; ++G) {
           const float w0g = vs[0][G] * vinv, w1g = vs[1][G] * vinv;
           const float q00 = p00 * w0g, q01 = p01 * w0g, q10 = p10 * w1g, q11 = p11 * w1g;
+          const float z0 = __half2float(__ushort_as_half((G ? sz01 : sz00) >> 16));
+          const float z1 = __half2float(__ushort_as_half((G ? sz11 : sz10) >> 16));
+          cz[G][0] = fmaf(q00, z0, fmaf(q10, z1, cz[G][0]));
+          cz[G][1] = fmaf(q01, z0, fmaf(q11, z1, cz[G][1]));
           const uint32_t h0 = pack_f16x2(q00, q01), h1 = pack_f16x2(q10, q11);
           const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
           const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
@@ -346,32 +349,20 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         // 64G + 8r .. +7 of a token; rows r / r+8 <-> d = 64G + 8r + 2k / +1
         const int ta = 16 * mt + 2 * j;
         const int tt[4] = {ta, ta + 1, ta + 8, ta + 9};
-        uint32_t vwd[4][2], zv[2][2];
+        uint32_t vwd[4][2];
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
           for (int G = 0; G < 2; ++G)
             vwd[t][G] = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffV + kRowB * tt[t] + 32 * G + 4 * r));
 #pragma unroll
-        for (int G = 0; G < 2; ++G) {
-          const uint32_t za = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[0] + 4 * G));
-          const uint32_t zb = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[1] + 4 * G));
-          const uint32_t zc2 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[2] + 4 * G));
-          const uint32_t zd = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tt[3] + 4 * G));
-          // zero points are the high halves: (1024 + z_a, 1024 + z_b)
-          zv[G][0] = hadd2(prmt(za, zb, 0x7632u), 0x64006400u);
-          zv[G][1] = hadd2(prmt(zc2, zd, 0x7632u), 0x64006400u);
-        }
-#pragma unroll
         for (int md = 0; md < 8; ++md) {
           const int G = md >> 2, k = md & 3;
           const uint32_t sel = static_cast<uint32_t>(k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12));
           const uint32_t Y = prmt(vwd[0][G], vwd[1][G], sel);   // bytes (ta_k, ta_k, tb_k, tb_k)
           const uint32_t Z = prmt(vwd[2][G], vwd[3][G], sel);
-          const uint32_t a[4] = {hsub2((Y & 0x000F000Fu) | 0x64006400u, zv[G][0]),
-                                 hsub2(((Y >> 4) & 0x000F000Fu) | 0x64006400u, zv[G][0]),
-                                 hsub2((Z & 0x000F000Fu) | 0x64006400u, zv[G][1]),
-                                 hsub2(((Z >> 4) & 0x000F000Fu) | 0x64006400u, zv[G][1])};
+          const uint32_t a[4] = {Y & 0x000F000Fu, (Y >> 4) & 0x000F000Fu, Z & 0x000F000Fu,
+                                 (Z >> 4) & 0x000F000Fu};
           mma_f16(o[md], a, pbh[G]);
           mma_f16(o[md], a, pbl[G]);
         }
@@ -383,6 +374,19 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     for (int off = 4; off < 32; off <<= 1) {
       l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
       l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
+#pragma unroll
+      for (int G = 0; G < 2; ++G) {
+        cz[G][0] += __shfl_xor_sync(0xffffffffu, cz[G][0], off);
+        cz[G][1] += __shfl_xor_sync(0xffffffffu, cz[G][1], off);
+      }
+    }
+#pragma unroll
+    for (int md = 0; md < 8; ++md) {
+      const int G = md >> 2;
+      o[md][0] = fmaf(o[md][0], 16777216.f, -cz[G][0]);
+      o[md][1] = fmaf(o[md][1], 16777216.f, -cz[G][1]);
+      o[md][2] = fmaf(o[md][2], 16777216.f, -cz[G][0]);
+      o[md][3] = fmaf(o[md][3], 16777216.f, -cz[G][1]);
     }
   }
   __syncthreads();
