@@ -72,6 +72,24 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values, world, device):
+    """Each timing is the slowest rank's: one all-reduce (MAX) of the list over the process
+    group (every rank calls this with the same length, in the same order)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def throughput(nbytes_per_rank, world, ms):
+    """Whole-job GB/s: every rank processes its own nbytes per step (weak scaling), the step
+    time is the slowest rank's."""
+    return world * nbytes_per_rank / (ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- peaks
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -450,10 +468,7 @@ def main_ours(args):
     dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
     ms = statistics.mean(step_ms)
     dms = statistics.mean(dec_ms)
-    if world > 1:
-        t = torch.tensor([ms, dms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, dms = t.tolist()
+    ms, dms = max_over_ranks([ms, dms], world, device)
 
     # the same step as one call (kvq_append_decode_attention), dense caches only
     fused = None
@@ -474,10 +489,7 @@ def main_ours(args):
             b2.record(stream)
         torch.cuda.synchronize()
         fms = statistics.mean(a.elapsed_time(b2) for a, b2 in fev)
-        if world > 1:
-            t = torch.tensor([fms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            fms = t.item()
+        fms, = max_over_ranks([fms], world, device)
         fused = {"value": round(world * step_bytes / (fms * 1e-3) / 1e9, 2), "unit": "GB/s",
                  "ms_per_step": round(fms, 5), "tokens_per_s": round(world * B / (fms * 1e-3), 1),
                  "frac_of_peak": round(step_bytes / (fms * 1e-3) / 1e9 / hbm_peak()[0], 4),
@@ -514,17 +526,14 @@ def main_ours(args):
         if k >= 3:
             e2e_ms.append(a.elapsed_time(b2))
     e2e = statistics.mean(e2e_ms) if e2e_ms else float("nan")
-    if world > 1:
-        t = torch.tensor([e2e], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = t.item()
+    e2e, = max_over_ranks([e2e], world, device)
 
     peak, peak_kind = hbm_peak()
     achieved = dec_bytes / (dms * 1e-3) / 1e9
     launches_per_step = 2 + (1 if ws_n else 0)
     result = {
         "metric": METRIC,
-        "value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2),
+        "value": round(throughput(step_bytes, world, ms), 2),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": K,
