@@ -155,7 +155,8 @@ def measure_prefill(device, l2, steps=20):
 
 def profile_traffic(workload):
     """dram bytes per launch of the decode kernel from the committed ncu summary, or None
-    when the summary is missing or was taken on a different kernel source."""
+    when the summary is missing or was taken on a different kernel source (the summary
+    names the source files its kernel is built from and their hash)."""
     path = os.path.join(ROOT, "profiles", "decode_%s.md" % workload.replace("-", "_"))
     try:
         text = open(path).read()
@@ -163,18 +164,20 @@ def profile_traffic(workload):
         return None
     m = re.search(r"dram_bytes_per_launch:\s*(\d+)", text)
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != kernel_source_hash():
+    f = re.search(r"kernel_sources:\s*(.+)", text)
+    if not m or not h or not f or h.group(1) != kernel_source_hash(f.group(1).split()):
         return None
     return int(m.group(1))
 
 
-def kernel_source_hash():
+def kernel_source_hash(names):
+    """First 16 hex digits of the sha256 of the named files of the library's csrc/, in
+    the order given."""
     d = os.path.join(ROOT, "quantized_paged_kv_02_b200", "csrc")
     hsh = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.startswith("kvq_decode"):
-            with open(os.path.join(d, name), "rb") as f:
-                hsh.update(f.read())
+    for name in names:
+        with open(os.path.join(d, name), "rb") as fh:
+            hsh.update(fh.read())
     return hsh.hexdigest()[:16]
 
 
