@@ -47,6 +47,13 @@
  *                               point) [bs][D/64][2] (each token's 64-channel group)
  *                               ([P-prod] "Key 和 Value 的分布不一定相同": keys per channel,
  *                               values per token)
+ *              KIVI_FLOAT_ZERO: as KIVI, with each zero point field holding the group's
+ *                               float16 minimum m instead of an integer zero point
+ *              INT4_PER_TOKEN : float16 K (scale, zero point) [bs][D/64][2], then float16
+ *                               V (scale, zero point) [bs][D/64][2] (keys grouped like
+ *                               values: [P-prod] "Key 和 Value 的分布不一定相同", the
+ *                               Transformers integration quantizes both per token)
+ *                               The three INT4 modes have records of the same size.
  *              other modes    : nothing
  *            record      = off_s + scale bytes, rounded up to a multiple of 128 bytes
  *                          (e.g. INT8, bs 16, D 128: 2048 + 2048 + 128 = 4224 bytes)
@@ -82,6 +89,13 @@
  *        z  = clamp(round_half_even(-lo / s), 0, 15)        (float32 ops, s widened);
  *        code = clamp(round_half_even(x / s) + z, 0, 15);   s == 0 gives z = code = 0.
  *        Stored s and z are float16; dequantized value = (code - z) * s.
+ *  INT4 KIVI_FLOAT_ZERO (the same groups; the zero point is the group minimum, a float):
+ *        lo = min_G x, hi = max_G x;  s = float16_rne( (hi - lo) / 15 );  m = float16_rne(lo);
+ *        code = clamp(round_half_even( (x - m) / s ), 0, 15)   (float32 ops, s and m widened);
+ *        s == 0 gives code 0.  Stored s and m are float16; dequantized value = code * s + m.
+ *  INT4 PER_TOKEN ([P-prod] "Transformers：适合实验和小规模验证": 4 bits, groups of 64,
+ *        residual of 128): the KIVI quantizer, every group one token over 64 channels, for
+ *        keys as for values.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -117,7 +131,9 @@ typedef enum {
   KVQ_SCALE_PER_HEAD = 2,
   KVQ_SCALE_PER_TENSOR = 3,
   KVQ_SCALE_KIVI = 4,
-  KVQ_SCALE_PER_CHANNEL = 5
+  KVQ_SCALE_PER_CHANNEL = 5,
+  KVQ_SCALE_INT4_PER_TOKEN = 6,
+  KVQ_SCALE_KIVI_FLOAT_ZERO = 7
 } kvq_scale_mode;
 
 /* Bits of fault[1] (fault[0] counts skipped entries). */
@@ -137,7 +153,8 @@ enum {
  *   act_dtype     BF16 or FP16: element type of new K/V rows, of q and of the INT4
  *                 residual ring.
  *   scale_mode    NONE for BF16/FP16; PER_TOKEN_HEAD, PER_HEAD, PER_TENSOR or
- *                 PER_CHANNEL for INT8 and FP8; KIVI for INT4.  PER_CHANNEL decodes on
+ *                 PER_CHANNEL for INT8 and FP8; KIVI, KIVI_FLOAT_ZERO or INT4_PER_TOKEN
+ *                 for INT4.  PER_CHANNEL decodes on
  *                 the tensor-core path only (block_size 16, head_dim 128).
  *   block_size    tokens per block: 1..1024 for dense caches; INT4 requires
  *                 block_size == group_size == 64.

@@ -16,6 +16,7 @@ from . import fp, quant
 SENTINEL = 0x5A
 
 DENSE_DTYPES = ("bf16", "fp16", "int8", "fp8")
+INT4_MODES = ("kivi", "kivi_float_zero", "int4_per_token")
 
 
 def _bits_of_act(x, act):
@@ -42,14 +43,17 @@ class PagedCache:
 
     cache_dtype: "bf16" | "fp16" | "int8" | "fp8" | "int4"
     act_dtype:   "bf16" | "fp16"
-    scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "per_channel" | "kivi"
+    scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "per_channel" for
+                 dense caches; "kivi" | "kivi_float_zero" | "int4_per_token" for INT4
     static_scales: (k_scale, v_scale) float32 arrays for static modes: [H] per head, [1]
                    per tensor, [H, D] per (kv head, channel).
 
     ``pages`` is the byte pool [NB][H][record] of include/kvq.h: per (block, kv head),
     K codes [bs][row_bytes], V codes [bs][row_bytes], then the per-token scales (float32
-    K [bs], V [bs]) or the KIVI parameters (float16 K scale [D], K zero [D], V (scale,
-    zero) [bs][D/64][2]), padded to a multiple of 128 bytes.  The attributes k_codes,
+    K [bs], V [bs]) or the INT4 parameters, padded to a multiple of 128 bytes.  INT4:
+    "kivi" float16 K scale [D], K zero point [D], V (scale, zero point) [bs][D/64][2];
+    "kivi_float_zero" the same with each zero point field holding the group minimum;
+    "int4_per_token" K (scale, zero point) [bs][D/64][2] then V the same.  The attributes k_codes,
     v_codes, k_scales, v_scales are typed views into it (static scales are arrays of
     their own).
     """
@@ -69,15 +73,17 @@ class PagedCache:
         elif cache_dtype == "fp8":
             code_dt, row_bytes = np.uint8, D
         elif cache_dtype == "int4":
-            assert scale_mode == "kivi" and block_size == group_size == 64
+            assert scale_mode in INT4_MODES and block_size == group_size == 64
             code_dt, row_bytes = np.uint8, D // 2
         else:
             raise ValueError(cache_dtype)
         off_s = 2 * bs * row_bytes
         if scale_mode == "per_token_head":
             scale_bytes = 8 * bs
-        elif scale_mode == "kivi":
+        elif scale_mode in ("kivi", "kivi_float_zero"):
             scale_bytes = 2 * D * 2 + bs * (D // group_size) * 2 * 2
+        elif scale_mode == "int4_per_token":
+            scale_bytes = 2 * bs * (D // group_size) * 2 * 2
         else:
             scale_bytes = 0
         self.row_bytes = row_bytes
@@ -97,10 +103,18 @@ class PagedCache:
             ks, vs = static_scales
             self.k_scales = np.asarray(ks, np.float32).reshape(shape).copy()
             self.v_scales = np.asarray(vs, np.float32).reshape(shape).copy()
-        elif scale_mode == "kivi":
-            # K scale [D] then K zero [D] as [NB][H][2][D]; V (scale, zero) [bs][D/G][2]
-            self.k_scales = pg[:, :, off_s:off_s + 4 * D].view(np.float16).reshape(NB, H, 2, D)
-            self.v_scales = pg[:, :, off_s + 4 * D:off_s + scale_bytes].view(np.float16).reshape(
+        elif cache_dtype == "int4":
+            if scale_mode == "int4_per_token":
+                # K (scale, zero) [bs][D/G][2], then V the same
+                half = scale_bytes // 2
+                self.k_scales = pg[:, :, off_s:off_s + half].view(np.float16).reshape(
+                    NB, H, bs, D // group_size, 2)
+            else:
+                # K scale [D] then K zero (or minimum) [D] as [NB][H][2][D]
+                half = 4 * D
+                self.k_scales = pg[:, :, off_s:off_s + half].view(np.float16).reshape(NB, H, 2, D)
+            # V (scale, zero or minimum) [bs][D/G][2]
+            self.v_scales = pg[:, :, off_s + half:off_s + scale_bytes].view(np.float16).reshape(
                 NB, H, bs, D // group_size, 2)
             self.residual = np.full(max_seqs * 2 * H * residual_cap * D * 2, SENTINEL,
                                     np.uint8).view(np.uint16).reshape(max_seqs, 2, H, residual_cap, D)
@@ -178,13 +192,19 @@ class PagedCache:
                 blk = first // bs
                 # keys per (head, channel) over the block's rows; values per (row, head,
                 # channel group); every group on its own, all heads at once
+                fz = self.mode == "kivi_float_zero"
                 kb = np.swapaxes(k_new[u:u + G].astype(np.float32), 0, 1)     # [H, G, D]
-                kc, ks, kz = quant.int4_keys_block(kb)
+                if self.mode == "int4_per_token":
+                    kc, ks, kz = quant.int4_values_row(kb, self.G)            # like values
+                    self.k_scales[blk, :, :, :, 0] = ks
+                    self.k_scales[blk, :, :, :, 1] = kz
+                else:
+                    kc, ks, kz = quant.int4_keys_block(kb, float_zero=fz)
+                    self.k_scales[blk, :, 0, :] = ks
+                    self.k_scales[blk, :, 1, :] = kz
                 self.k_codes[blk] = quant.pack_nibbles(kc)
-                self.k_scales[blk, :, 0, :] = ks
-                self.k_scales[blk, :, 1, :] = kz
                 vb = np.swapaxes(v_new[u:u + G].astype(np.float32), 0, 1)     # [H, G, D]
-                vc, vs, vz = quant.int4_values_row(vb, self.G)
+                vc, vs, vz = quant.int4_values_row(vb, self.G, float_zero=fz)
                 self.v_codes[blk] = quant.pack_nibbles(vc)
                 self.v_scales[blk, :, :, :, 0] = vs
                 self.v_scales[blk, :, :, :, 1] = vz
@@ -234,16 +254,18 @@ class PagedCache:
                 deq = quant.int8_dequantize if self.cd == "int8" else quant.fp8_dequantize
                 out[which] = deq(c, s)
             else:
-                q = quant.unpack_nibbles(c)                      # [H, bs, D]
-                if which == 0:
-                    s = self.k_scales[blk, :, 0, :].astype(np.float64)   # [H, D]
-                    z = self.k_scales[blk, :, 1, :].astype(np.float64)
-                    out[0] = (q.astype(np.float64) - z[:, None, :]) * s[:, None, :]
+                q = quant.unpack_nibbles(c).astype(np.float64)  # [H, bs, D]
+                if which == 0 and self.mode != "int4_per_token":
+                    s = self.k_scales[blk, :, 0, :].astype(np.float64)[:, None, :]   # [H, 1, D]
+                    z = self.k_scales[blk, :, 1, :].astype(np.float64)[:, None, :]
                 else:
-                    vs = self.v_scales[blk].astype(np.float64)   # [H, bs, D/G, 2]
-                    s = np.repeat(vs[..., 0], self.G, axis=-1)   # [H, bs, D]
-                    z = np.repeat(vs[..., 1], self.G, axis=-1)
-                    out[1] = (q.astype(np.float64) - z) * s
+                    sz = (self.k_scales if which == 0 else self.v_scales)[blk].astype(np.float64)
+                    s = np.repeat(sz[..., 0], self.G, axis=-1)   # [H, bs, D]
+                    z = np.repeat(sz[..., 1], self.G, axis=-1)
+                if self.mode == "kivi_float_zero":
+                    out[which] = quant.int4_dequantize_float_zero(q, s, z)
+                else:
+                    out[which] = quant.int4_dequantize(q, s, z)
         return out
 
     def quantized_prefix(self, n):

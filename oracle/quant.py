@@ -16,6 +16,9 @@ Readings of the pages taken here (each listed in the design doc):
   * INT4 uses the affine form of [P-prod] "量化不是简单截断精度"
     (X_q = round(X/scale) + zero_point; X_deq = (X_q - zero_point) * scale) with the
     range widened to include 0, so the zero point is an integer in [0, 15].
+  * The float-zero-point INT4 variant takes the group minimum itself as the offset
+    (X_deq = X_q * scale + min, the range not widened); the pages name only the integer
+    form, so this variant is a reading of "zero point" as a real offset.
 """
 
 import numpy as np
@@ -146,6 +149,39 @@ def int4_quantize_groups(values):
     return q.astype(np.uint8), np.asarray(s16, np.float16), np.asarray(z, np.float16)
 
 
+def int4_quantize_groups_float_zero(values):
+    """Asymmetric 4-bit quantization with a float zero point (the group minimum).
+
+    Every group (1-D slice values[..., :]) on its own.  Returns (codes uint8 in 0..15,
+    scale float16, minimum float16), the last two with the leading shape.
+      lo = min x; hi = max x
+      s  = float16(binary32((hi - lo) / 15));  m = float16(lo)   -- stored, used from here on
+      q  = clamp(round_half_even(binary32(binary32(x - m) / s)), 0, 15)
+    A group whose s is 0 (constant, or a range below float16's reach) gets codes 0.
+    Dequantized value: q * s + m.
+    """
+    x = np.asarray(values, dtype=np.float32)
+    lo = x.min(axis=-1)
+    hi = x.max(axis=-1)
+    s16 = fp.f16(fp.div32(fp.sub32(hi, lo), np.float32(INT4_LEVELS)))
+    m16 = fp.f16(lo)
+    zero_group = s16 == 0
+    sw = np.where(zero_group, np.float32(1.0), np.asarray(s16, np.float32))
+    mw = np.asarray(m16, np.float32)
+    q = np.clip(fp.round_half_even(fp.div32(fp.sub32(x, mw[..., None]), sw[..., None])), 0, 15)
+    q = np.where(zero_group[..., None], 0, q)
+    return q.astype(np.uint8), np.asarray(s16, np.float16), np.asarray(m16, np.float16)
+
+
+def int4_dequantize_float_zero(codes, scale, minimum):
+    """X_deq = X_q * scale + min, float64."""
+    return np.asarray(codes, np.float64) * np.float64(scale) + np.float64(minimum)
+
+
+def _groups(float_zero):
+    return int4_quantize_groups_float_zero if float_zero else int4_quantize_groups
+
+
 def int4_quantize_group(values):
     """int4_quantize_groups for one group (1-D array): (codes, scale, zero point)."""
     q, s, z = int4_quantize_groups(np.asarray(values, dtype=np.float32).reshape(1, -1))
@@ -157,28 +193,30 @@ def int4_dequantize(codes, scale, zero):
     return (np.asarray(codes, np.float64) - np.float64(zero)) * np.float64(scale)
 
 
-def int4_keys_block(k_rows):
+def int4_keys_block(k_rows, float_zero=False):
     """KIVI keys: one group per channel over the block's tokens.
 
     k_rows [64, D] (one kv head), or [..., 64, D] for several heads at once.  Returns
-    codes [..., 64, D], scale [..., D], zero [..., D].
+    codes [..., 64, D], scale [..., D], zero point (or minimum, float_zero) [..., D].
     [P-prod] "Key 和 Value 的分布不一定相同": key cache per channel (KIVI).
     """
     k_rows = np.asarray(k_rows, dtype=np.float32)
-    q, s, z = int4_quantize_groups(np.swapaxes(k_rows, -1, -2))     # groups = channels
+    q, s, z = _groups(float_zero)(np.swapaxes(k_rows, -1, -2))     # groups = channels
     return np.swapaxes(q, -1, -2), s, z
 
 
-def int4_values_row(v_row, group=64):
-    """KIVI values: one group per token over each run of `group` channels.
+def int4_values_row(v_row, group=64, float_zero=False):
+    """One group per token over each run of `group` channels: KIVI values, and keys as well
+    as values in the per-token variant.
 
     v_row [D] (one token, one kv head), or [..., D] for several at once.  Returns codes
-    [..., D], scale [..., D/group], zero [..., D/group].
-    [P-prod] "Key 和 Value 的分布不一定相同": value cache per token.
+    [..., D], scale [..., D/group], zero point (or minimum, float_zero) [..., D/group].
+    [P-prod] "Key 和 Value 的分布不一定相同": value cache per token (KIVI); the Transformers
+    integration quantizes keys and values per token.
     """
     v_row = np.asarray(v_row, dtype=np.float32)
     D = v_row.shape[-1]
-    q, s, z = int4_quantize_groups(v_row.reshape(v_row.shape[:-1] + (D // group, group)))
+    q, s, z = _groups(float_zero)(v_row.reshape(v_row.shape[:-1] + (D // group, group)))
     return q.reshape(v_row.shape), s, z
 
 

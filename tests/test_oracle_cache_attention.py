@@ -189,8 +189,55 @@ def test_int4_grid_exact_attention_equals_sdpa():
         assert np.all(c.k_codes[blk] == cache.SENTINEL) and np.all(c.v_codes[blk] == cache.SENTINEL)
 
 
+@pytest.mark.parametrize("mode", ["int4_per_token", "kivi_float_zero"])
+def test_int4_variants_grid_exact_attention_equals_sdpa(mode):
+    """The per-token variant (keys grouped per token over 64 channels, like values) and the
+    float-zero-point variant (offset = group minimum, the range need not include 0): on
+    their grids quantization is exact, so attention equals SDPA on the dense rows."""
+    rng = np.random.default_rng(3)
+    H, D, n = 1, 128, 64 * 3 + 128 + 21
+    qb = 192
+
+    def grid():
+        k = rng.integers(0, 16, 64)
+        k[0], k[1] = 0, 15
+        e = rng.integers(1, 5)
+        if mode == "kivi_float_zero":
+            return rng.integers(-40, 41) * 2.0 ** -3 + k * 2.0 ** -e
+        return (k - rng.integers(0, 16)) * 2.0 ** -e
+
+    K = np.empty((n, H, D))
+    V = np.empty((n, H, D))
+    for p in range(qb):
+        for gi in range(2):
+            V[p, 0, gi * 64:(gi + 1) * 64] = grid()
+            if mode == "int4_per_token":
+                K[p, 0, gi * 64:(gi + 1) * 64] = grid()
+    if mode == "kivi_float_zero":
+        for blk in range(qb // 64):
+            for d in range(D):
+                K[blk * 64:(blk + 1) * 64, 0, d] = grid()
+    K[qb:] = fp.bf16_round(rng.standard_normal((n - qb, H, D)))
+    V[qb:] = fp.bf16_round(rng.standard_normal((n - qb, H, D)))
+    assert np.array_equal(fp.bf16_round(K), K) and np.array_equal(fp.bf16_round(V), V)
+    c = cache.PagedCache("int4", "bf16", mode, 5, 64, H, D, max_seqs=2)
+    table = np.array([3, 0, 4])
+    slots = np.array([table[p // 64] * 64 + p % 64 for p in range(qb)] + [-1] * (n - qb))
+    pos = np.array([-1] * qb + list(range(qb, n)))
+    c.write(K, V, slots, np.ones(n, np.int64), pos)
+    q = fp.bf16_round(rng.standard_normal((1, 4, D)))
+    out = attention.decode_attention(c, q, table[None, :], np.array([n]), seq_ids=np.array([1]))
+    for hq in range(4):
+        np.testing.assert_allclose(out[0, hq], _sdpa(q[0, hq], K[:, 0], V[:, 0], 1 / np.sqrt(D)),
+                                   rtol=1e-12, atol=1e-12)
+    if mode == "kivi_float_zero":
+        assert np.any(c.k_scales[table, 0, 1, :] > 0)      # minima above 0 occur
+    else:
+        assert c.k_scales.shape[2:] == (64, 2, 2)          # [bs][D/64][(scale, zero)]
+
+
 # ---------------------------------------------------------------- invariants
-@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c5"])
 def test_invariants_on_small_workloads(name):
     w = inputs.make(name, small=True)
     s = w.spec
@@ -290,10 +337,11 @@ def test_int4_prefix_split():
         [0, 0, 0, 0, 64, 64, 128, 32640]
 
 
-def test_flush_ring_equals_writing_the_rows():
+@pytest.mark.parametrize("name", ["c4", "c4-tok", "c4-fzp"])
+def test_flush_ring_equals_writing_the_rows(name):
     """Flushing ring rows [p0, p0+64) into a block stores what writing those rows with the
     block's slots stores (the definition in include/kvq.h)."""
-    w = inputs.make("c4", small=True)
+    w = inputs.make(name, small=True)
     c = _build(w)
     s = w.spec
     n0 = int(w.context_lens[0])

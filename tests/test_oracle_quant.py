@@ -196,3 +196,74 @@ def test_kivi_axes():
     v[70] = 1000.0                                # outlier only in the second group
     vc, vs, vz = quant.int4_values_row(v)
     assert vs.shape == (2,) and vs[1] > 100 * vs[0]
+
+
+# ------------------------------------------------- INT4 with a float zero point (group min)
+def test_int4_float_zero_nearest_code_bruteforce():
+    """Each code minimises |x - (c s + m)| over the 16 codes, given the stored (s, m)."""
+    g = torch.Generator().manual_seed(17)
+    for trial in range(40):
+        x = (torch.randn(64, generator=g) * (0.1 + trial) + (trial % 7 - 3)).to(torch.bfloat16)
+        x = x.float().numpy()
+        c, s, m = quant.int4_quantize_groups_float_zero(x[None])
+        c, s, m = c[0], s[0], m[0]
+        grid = np.arange(16) * np.float64(s) + np.float64(m)
+        d = np.abs(x.astype(np.float64)[:, None] - grid[None, :])
+        chosen = d[np.arange(64), c]
+        assert np.all(chosen <= d.min(axis=1) + 2.0 ** -20 * float(s))
+
+
+def test_int4_float_zero_steps_exact():
+    """s = fp16(fp32((hi - lo) / 15)) and m = fp16(lo), in exact arithmetic; the range is
+    not widened to include 0 (an all-positive group keeps its own minimum)."""
+    x = np.array([3.0, 1.5, 2.25, 7.75] + [2.0] * 60, np.float32)
+    c, s, m = quant.int4_quantize_groups_float_zero(x[None])
+    s_want = exact_round(exact_round(Fraction(775, 100) - Fraction(3, 2), 24, -126) / 15, 24, -126)
+    assert Fraction(float(s[0])) == exact_round(s_want, 11, -14)
+    assert float(m[0]) == 1.5
+    assert c[0][1] == 0 and c[0][3] == 15
+    want2 = _rhe(exact_round(Fraction(1, 2) / Fraction(float(s[0])), 24, -126))   # x = 2.0
+    assert c[0][4] == want2
+
+
+def test_int4_float_zero_grid_exact_round_trip():
+    """Values on the grid m0 + k 2^-e (all 16 codes used, m0 on both sides of 0) come back
+    exactly."""
+    rng = np.random.default_rng(19)
+    for e in (-3, 0, 2, 5):
+        for m0 in (-5.0, -0.75, 0.0, 1.25, 9.0):
+            k = rng.integers(0, 16, 64)
+            k[0], k[1] = 0, 15
+            x = (m0 + k * 2.0 ** -e).astype(np.float32)
+            c, s, m = quant.int4_quantize_groups_float_zero(x[None])
+            assert float(s[0]) == 2.0 ** -e and float(m[0]) == m0
+            np.testing.assert_array_equal(c[0], k)
+            np.testing.assert_array_equal(quant.int4_dequantize_float_zero(c[0], s[0], m[0]),
+                                          x.astype(np.float64))
+
+
+def test_int4_float_zero_constant_group_and_bound():
+    c, s, m = quant.int4_quantize_groups_float_zero(np.full((1, 64), -2.5, np.float32))
+    assert float(s[0]) == 0 and float(m[0]) == -2.5 and not c.any()
+    np.testing.assert_array_equal(quant.int4_dequantize_float_zero(c[0], s[0], m[0]), -2.5)
+    g = torch.Generator().manual_seed(23)
+    x = (torch.randn(128, 64, generator=g) + 3.0).to(torch.bfloat16).float().numpy()
+    c, s, m = quant.int4_quantize_groups_float_zero(x)
+    deq = quant.int4_dequantize_float_zero(c, s[:, None], m[:, None])
+    s64 = s.astype(np.float64)[:, None]
+    # m is a bf16 value, exact in fp16; s is rounded to fp16 (rel. 2^-11)
+    assert np.all(np.abs(x - deq) <= s64 * (0.5 + 15 * 2.0 ** -11) + 1e-12)
+
+
+def test_int4_per_token_keys_group_like_values():
+    """The per-token variant groups each key row over 64-channel runs: an outlier channel
+    raises only its own group's scale, for every token alike."""
+    rng = np.random.default_rng(29)
+    k = rng.standard_normal((64, 128)).astype(np.float32)
+    k[:, 5] = 500.0
+    c, s, z = quant.int4_values_row(k)
+    assert s.shape == (64, 2)
+    assert np.all(s[:, 0] > 20 * s[:, 1])
+    c1, s1, z1 = quant.int4_values_row(k[7])
+    np.testing.assert_array_equal(c[7], c1)
+    np.testing.assert_array_equal(s[7], s1)
