@@ -46,6 +46,10 @@ WORKLOADS = {
           "block 16, FP8 E4M3 per-kv-head scales",
     "c4": "70B-shaped KIVI INT4 layer: batch 16, 64/8 heads, head_dim 128, context 32768, "
           "block 64, keys per channel / values per token, 128-token bf16 residual",
+    "c4-tok": "70B-shaped INT4 layer as c4, keys and values both per token (64-channel groups), "
+              "128-token bf16 residual",
+    "c4-fzp": "70B-shaped KIVI INT4 layer as c4, float zero points (group minimum), "
+              "128-token bf16 residual",
 }
 
 

@@ -52,7 +52,9 @@ static kvq_status validate_geometry(const kvq_cache_desc* c, Geometry* g) {
         return KVQ_ERR_INVALID_ARG;
       break;
     case KVQ_DTYPE_INT4:
-      if (c->scale_mode != KVQ_SCALE_KIVI) return KVQ_ERR_INVALID_ARG;
+      if (c->scale_mode != KVQ_SCALE_KIVI && c->scale_mode != KVQ_SCALE_KIVI_FLOAT_ZERO &&
+          c->scale_mode != KVQ_SCALE_INT4_PER_TOKEN)
+        return KVQ_ERR_INVALID_ARG;
       if (c->group_size != 64 || c->block_size != 64) return KVQ_ERR_UNSUPPORTED;
       if (c->residual_len < 0 || c->residual_cap < c->residual_len + c->group_size) return KVQ_ERR_INVALID_ARG;
       if (c->max_seqs < 1) return KVQ_ERR_INVALID_ARG;
@@ -63,7 +65,9 @@ static kvq_status validate_geometry(const kvq_cache_desc* c, Geometry* g) {
   g->off_s = 2 * g->bs * g->row_bytes;
   g->scale_bytes = 0;
   if (g->scale_mode == KVQ_SCALE_PER_TOKEN_HEAD) g->scale_bytes = 8 * g->bs;
-  if (g->scale_mode == KVQ_SCALE_KIVI) g->scale_bytes = 4 * g->D + g->bs * (g->D / 64) * 4;
+  // INT4: K (scale, zero) per channel [2][D] or per token [bs][D/64][2], then V per token
+  // [bs][D/64][2], all float16; with bs = 64 both K forms take 4 * D bytes
+  if (g->cache_dtype == KVQ_DTYPE_INT4) g->scale_bytes = 4 * g->D + g->bs * (g->D / 64) * 4;
   g->record = (g->off_s + g->scale_bytes + 127) / 128 * 128;
   return KVQ_OK;
 }
@@ -170,7 +174,7 @@ kvq_status kvq_cache_layout(const kvq_cache_desc* c, size_t* record_bytes, size_
   if (g.scale_mode == KVQ_SCALE_PER_HEAD) ss = static_cast<size_t>(g.H) * 4;
   if (g.scale_mode == KVQ_SCALE_PER_TENSOR) ss = 4;
   if (g.scale_mode == KVQ_SCALE_PER_CHANNEL) ss = static_cast<size_t>(g.H) * g.D * 4;
-  if (g.scale_mode == KVQ_SCALE_KIVI)
+  if (g.cache_dtype == KVQ_DTYPE_INT4)
     rb = static_cast<size_t>(g.max_seqs) * 2 * g.H * g.residual_cap * g.D * 2;
   if (record_bytes) *record_bytes = static_cast<size_t>(g.record);
   if (pages_bytes) *pages_bytes = static_cast<size_t>(g.NB) * g.H * g.record;

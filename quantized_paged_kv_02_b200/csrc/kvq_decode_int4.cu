@@ -1,5 +1,5 @@
-// Paged split-K decode attention over KIVI INT4 pages on tensor cores (head_dim 128,
-// block 64, GQA groups of 3..8 query heads).
+// Paged split-K decode attention over INT4 pages on tensor cores (head_dim 128, block 64,
+// GQA groups of 3..8 query heads), for the three INT4 forms of include/kvq.h.
 //
 // KIVI keeps keys per channel and values per token ([P-prod] "Key 和 Value 的分布不一定
 // 相同"), each as X_q = round(X/scale) + zero_point ([P-prod] "量化不是简单截断精度"):
@@ -20,6 +20,17 @@
 // A holds the codes of two tokens per register, assembled with a byte permute.  The
 // residual ring (the newest tokens, unquantized) is a separate split handled by the
 // CUDA-core kernel; the reduce merges both.
+//
+// Float zero point (k_hat = c * sk + mk, v_hat = c * sv + mv, m the group minimum): the
+// same products, with the offsets added instead of subtracted:
+//   S^T[t] = 2^24 * (C Q'^T)[t] + sum_d q[d] mk[d],   O[d] = 2^24 * (C^T P'^T)[d] + sum_t p[t] mv[t][G(d)].
+// Keys per token (k_hat[t][d] = (c[t][d] - zk[t][G]) * sk[t][G], grouped like values): the
+// scale cannot be folded into q, but it is constant over each 64-channel group, so each
+// lane reads its codes as two 8-byte halves (one per group) and every k-step stays inside
+// one group; two accumulators hold the per-group sums and
+//   S^T[t] = sum_G sk[t][G] * (2^24 * (C_G q^T)[t] - zk[t][G] * sum_{d in G} q[d]).
+// q is then the same for every block: its fp16 fragments (one MMA per k-step, q being an
+// activation value scaled by a power of two) and per-group sums are formed once.
 //
 // Structure as the dense tensor-core kernel: warp 4 stages one 9 KiB record per block
 // (64 tokens of K and V codes plus all scales and zero points) with one 128-byte-swizzled
@@ -71,8 +82,16 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w, int s) { return (w >> (
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// INT4 forms of the kernel
+constexpr int kKivi = 0;        // keys per channel, integer zero points
+constexpr int kKiviMin = 1;     // keys per channel, the group minimum as a float zero point
+constexpr int kPerToken = 2;    // keys per token like values, integer zero points
+
+template <int MODE>
 __global__ void __launch_bounds__(kT, 2)
 decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
+  constexpr bool kFz = MODE == kKiviMin;
+  constexpr bool kTok = MODE == kPerToken;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* tiles = smem;
@@ -153,14 +172,16 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   } else {
     // ---------------------------------------------------------------- consumers
     const int g = p.g;
-    // q of head r, channels [32j, 32j+32), as bf16/fp16 pairs scaled by 2^-eq (exact)
+    // q of head r as bf16/fp16 pairs scaled by 2^-eq (exact): channels [32j, 32j+32), or,
+    // keys per token, [16j, 16j+16) and [64+16j, 64+16j+16) (the codes this lane reads)
     float qv[32];
     if (r < g) {
       const uint16_t* qp = static_cast<const uint16_t*>(p.q) +
-                           (static_cast<long>(b) * p.Hq + kvh * g + r) * kD + 32 * j;
+                           (static_cast<long>(b) * p.Hq + kvh * g + r) * kD;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 u = *reinterpret_cast<const uint4*>(qp + 8 * c);
+        const int ch = kTok ? 64 * (c >> 1) + 16 * j + 8 * (c & 1) : 32 * j + 8 * c;
+        const uint4 u = *reinterpret_cast<const uint4*>(qp + ch);
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -189,6 +210,29 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll
     for (int e = 0; e < 32; ++e) qv[e] *= qdown;
     const float qscale = p.scale_log2 * pow2i(eq);
+    // keys per token: q's fp16 fragments and per-group sums, the same for every block;
+    // k-step kc < 4 covers group 0, kc >= 4 group 1
+    uint32_t qt[kTok ? 8 : 1][2];
+    float qg[2][2] = {{0.f, 0.f}, {0.f, 0.f}};        // [group][head 2j, 2j+1]
+    if constexpr (kTok) {
+      float part[2] = {0.f, 0.f};
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        const int e0 = 8 * (kc >> 1) + 2 * (kc & 1);
+        qt[kc][0] = pack_f16x2(qv[e0], qv[e0 + 4]);
+        qt[kc][1] = pack_f16x2(qv[e0 + 1], qv[e0 + 5]);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qt[kc][0]));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qt[kc][1]));
+        part[kc >> 2] += (f0.x + f0.y) + (f1.x + f1.y);     // what the MMAs multiply
+      }
+#pragma unroll
+      for (int G = 0; G < 2; ++G) {
+        part[G] += __shfl_xor_sync(0xffffffffu, part[G], 1);
+        part[G] += __shfl_xor_sync(0xffffffffu, part[G], 2);
+        qg[G][0] = __shfl_sync(0xffffffffu, part[G], 8 * j);
+        qg[G][1] = __shfl_sync(0xffffffffu, part[G], 8 * j + 4);
+      }
+    }
 
     float vlim = 0.f, vinv = 0.f;
     for (int i = warp; i < npages; i += kC) {
@@ -206,10 +250,10 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       // ------------------------------------------------ per-block key scales -> Q' and Zk
       // q'[e] = q[32j+e] * sk[32j+e]; k-step kc uses channel pairs (8w+sp, 8w+sp+4) and
       // (8w+sp+1, 8w+sp+5) with w = kc/2, sp = 2*(kc%2): the pairs the nibble extraction
-      // of word w yields.
-      uint32_t qh[8][2], ql[8][2];
-      float ck0, ck1;
-      {
+      // of word w yields.  (Keys per token: nothing per block.)
+      uint32_t qh[kTok ? 1 : 8][2], ql[kTok ? 1 : 8][2];
+      float ck0 = 0.f, ck1 = 0.f;
+      if constexpr (!kTok) {
         uint32_t sw[16], zw[16];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -237,11 +281,15 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           ql[kc][0] = pack_f16x2(a0 - f0.x, a1 - f0.y);
           ql[kc][1] = pack_f16x2(c0 - f1.x, c1 - f1.y);
         }
+        // integer zero points: ck = sum q' zk (subtracted); float: ck = -sum q mk
         float corr = 0.f;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 z = __half22float2(*reinterpret_cast<const __half2*>(&zw[e]));
-          corr = fmaf(qs[2 * e], z.x, fmaf(qs[2 * e + 1], z.y, corr));
+          if constexpr (kFz)
+            corr = fmaf(-qv[2 * e], z.x, fmaf(-qv[2 * e + 1], z.y, corr));
+          else
+            corr = fmaf(qs[2 * e], z.x, fmaf(qs[2 * e + 1], z.y, corr));
         }
         corr += __shfl_xor_sync(0xffffffffu, corr, 1);
         corr += __shfl_xor_sync(0xffffffffu, corr, 2);
@@ -252,21 +300,56 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       for (int mt = 0; mt < kBS / 16; ++mt) {
         const int tr0 = 16 * mt + r, tr1 = tr0 + 8;
         // ------------------------------------------------ S^T = (C - Zk) Q'^T
-        const uint4 k0 = lds128(st + swzb4(kRowB * tr0 + 16 * j));
-        const uint4 k1 = lds128(st + swzb4(kRowB * tr1 + 16 * j));
-        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        float s00, s01, s10, s11;
+        if constexpr (kTok) {
+          // codes of channels [16j, 16j+16) and [64+16j, 64+16j+16): group 0 in words 0-1
+          const uint2 k0a = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr0 + 8 * j));
+          const uint2 k0b = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr0 + 32 + 8 * j));
+          const uint2 k1a = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr1 + 8 * j));
+          const uint2 k1b = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr1 + 32 + 8 * j));
+          const uint32_t w0[4] = {k0a.x, k0a.y, k0b.x, k0b.y}, w1[4] = {k1a.x, k1a.y, k1b.x, k1b.y};
+          float sg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc) {
-          const int w = kc >> 1, sp = 2 * (kc & 1);
-          const uint32_t a[4] = {nib_pair(w0[w], sp), nib_pair(w1[w], sp), nib_pair(w0[w], sp + 1),
-                                 nib_pair(w1[w], sp + 1)};
-          mma_f16(sa, a, qh[kc]);
-          mma_f16(sb, a, ql[kc]);
+          for (int kc = 0; kc < 8; ++kc) {
+            const int w = kc >> 1, sp = 2 * (kc & 1);
+            const uint32_t a[4] = {nib_pair(w0[w], sp), nib_pair(w1[w], sp), nib_pair(w0[w], sp + 1),
+                                   nib_pair(w1[w], sp + 1)};
+            mma_f16(sg[kc >> 2], a, qt[kc]);
+          }
+          // (scale, zero) of tokens tr0 / tr1, groups 0 and 1: fp16 at kOffKs + 8t + 4G
+          const uint2 z0 = *reinterpret_cast<const uint2*>(st + swzb4(kOffKs + 8 * tr0));
+          const uint2 z1 = *reinterpret_cast<const uint2*>(st + swzb4(kOffKs + 8 * tr1));
+          const float2 a00 = __half22float2(*reinterpret_cast<const __half2*>(&z0.x));   // t0 G0
+          const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&z0.y));   // t0 G1
+          const float2 a10 = __half22float2(*reinterpret_cast<const __half2*>(&z1.x));
+          const float2 a11 = __half22float2(*reinterpret_cast<const __half2*>(&z1.y));
+          s00 = (a00.x * fmaf(sg[0][0], 16777216.f, -a00.y * qg[0][0]) +
+                 a01.x * fmaf(sg[1][0], 16777216.f, -a01.y * qg[1][0])) * qscale;
+          s01 = (a00.x * fmaf(sg[0][1], 16777216.f, -a00.y * qg[0][1]) +
+                 a01.x * fmaf(sg[1][1], 16777216.f, -a01.y * qg[1][1])) * qscale;
+          s10 = (a10.x * fmaf(sg[0][2], 16777216.f, -a10.y * qg[0][0]) +
+                 a11.x * fmaf(sg[1][2], 16777216.f, -a11.y * qg[1][0])) * qscale;
+          s11 = (a10.x * fmaf(sg[0][3], 16777216.f, -a10.y * qg[0][1]) +
+                 a11.x * fmaf(sg[1][3], 16777216.f, -a11.y * qg[1][1])) * qscale;
+        } else {
+          const uint4 k0 = lds128(st + swzb4(kRowB * tr0 + 16 * j));
+          const uint4 k1 = lds128(st + swzb4(kRowB * tr1 + 16 * j));
+          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+          float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int kc = 0; kc < 8; ++kc) {
+            const int w = kc >> 1, sp = 2 * (kc & 1);
+            const uint32_t a[4] = {nib_pair(w0[w], sp), nib_pair(w1[w], sp), nib_pair(w0[w], sp + 1),
+                                   nib_pair(w1[w], sp + 1)};
+            mma_f16(sa, a, qh[kc]);
+            mma_f16(sb, a, ql[kc]);
+          }
+          s00 = fmaf(sa[0] + sb[0], 16777216.f, -ck0) * qscale;
+          s01 = fmaf(sa[1] + sb[1], 16777216.f, -ck1) * qscale;
+          s10 = fmaf(sa[2] + sb[2], 16777216.f, -ck0) * qscale;
+          s11 = fmaf(sa[3] + sb[3], 16777216.f, -ck1) * qscale;
         }
         // ------------------------------------------------ softmax (log2 domain)
-        float s00 = fmaf(sa[0] + sb[0], 16777216.f, -ck0) * qscale, s01 = fmaf(sa[1] + sb[1], 16777216.f, -ck1) * qscale;
-        float s10 = fmaf(sa[2] + sb[2], 16777216.f, -ck0) * qscale, s11 = fmaf(sa[3] + sb[3], 16777216.f, -ck1) * qscale;
         const bool grow = s00 > m[0] + kRescale4 || s10 > m[0] + kRescale4 ||
                           s01 > m[1] + kRescale4 || s11 > m[1] + kRescale4;
         if (__any_sync(0xffffffffu, grow)) {
@@ -333,8 +416,14 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           const float q00 = p00 * w0g, q01 = p01 * w0g, q10 = p10 * w1g, q11 = p11 * w1g;
           const float z0 = __half2float(__ushort_as_half((G ? sz01 : sz00) >> 16));
           const float z1 = __half2float(__ushort_as_half((G ? sz11 : sz10) >> 16));
-          cz[G][0] = fmaf(q00, z0, fmaf(q10, z1, cz[G][0]));
-          cz[G][1] = fmaf(q01, z0, fmaf(q11, z1, cz[G][1]));
+          if constexpr (kFz) {
+            // the minima enter unscaled: cz = -vinv * sum_t p mv
+            cz[G][0] = fmaf(-p00 * vinv, z0, fmaf(-p10 * vinv, z1, cz[G][0]));
+            cz[G][1] = fmaf(-p01 * vinv, z0, fmaf(-p11 * vinv, z1, cz[G][1]));
+          } else {
+            cz[G][0] = fmaf(q00, z0, fmaf(q10, z1, cz[G][0]));
+            cz[G][1] = fmaf(q01, z0, fmaf(q11, z1, cz[G][1]));
+          }
           const uint32_t h0 = pack_f16x2(q00, q01), h1 = pack_f16x2(q10, q11);
           const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
           const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
@@ -439,7 +528,11 @@ cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaS
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(decode_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    attr_err = cudaFuncSetAttribute(decode_int4_kernel<kKivi>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(decode_int4_kernel<kKiviMin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(decode_int4_kernel<kPerToken>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap tm;
@@ -447,7 +540,12 @@ cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaS
   if (!make_pages_map(&tm, a.c->pages, rows, kRecRows)) return cudaErrorInvalidValue;
   // page splits only; the ring split is launched separately
   const dim3 grid(p.ring_split, a.geo.H, a.batch);
-  decode_int4_kernel<<<grid, kT, kBytes, s>>>(p, tm);
+  switch (a.geo.scale_mode) {
+    case KVQ_SCALE_KIVI: decode_int4_kernel<kKivi><<<grid, kT, kBytes, s>>>(p, tm); break;
+    case KVQ_SCALE_KIVI_FLOAT_ZERO: decode_int4_kernel<kKiviMin><<<grid, kT, kBytes, s>>>(p, tm); break;
+    case KVQ_SCALE_INT4_PER_TOKEN: decode_int4_kernel<kPerToken><<<grid, kT, kBytes, s>>>(p, tm); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -12,8 +12,9 @@
 // "PagedAttention与KV Cache量化协同工作原理": INT8/FP8 blocks are dequantized inside the
 // attention kernel): per-token / per-head scales multiply the dot product and the
 // softmax weight rather than every element; INT4 keys use (code - zero) * scale per
-// channel and INT4 values (code - zero) * scale per token group ([P-prod]
-// "量化不是简单截断精度").  Decode reads every cached position of the sequence each step
+// channel (or per token group in the per-token variant) and INT4 values (code - zero) *
+// scale per token group ([P-prod] "量化不是简单截断精度"); the float-zero-point variant
+// dequantizes to code * scale + minimum.  Decode reads every cached position of the sequence each step
 // ([P-prod] "为什么长上下文更需要 KV Cache Quantization"), so this kernel is bound by
 // HBM bandwidth when the ALUs keep up (small GQA groups).
 #include "kvq_internal.cuh"
@@ -149,17 +150,33 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
       load_codes<CD>(rec + off * ROWB + c * CB, kf[j]);
       load_codes<CD>(rec + p.off_v + off * ROWB + c * CB, vf[j]);
       if constexpr (kInt4) {
-        const __half* ksz = reinterpret_cast<const __half*>(rec + p.off_s);   // scale [D], zero [D]
+        // this lane's EPL channels lie in one 64-channel group
+        const __half* sz = reinterpret_cast<const __half*>(rec + p.off_s);
+        const int grp64 = (c * EPL) / 64;
+        const bool fzp = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO;
+        if (p.mode == KVQ_SCALE_INT4_PER_TOKEN) {          // K (scale, zero) [bs][D/64][2]
+          const __half* ksz = sz + (off * (D / 64) + grp64) * 2;
+          const float ks = __half2float(ksz[0]), kz = __half2float(ksz[1]);
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int d = c * EPL + i;
-          kf[j][i] = (kf[j][i] - __half2float(ksz[D + d])) * __half2float(ksz[d]);
+          for (int i = 0; i < EPL; ++i) kf[j][i] = (kf[j][i] - kz) * ks;
+        } else {                                           // K scale [D], zero or minimum [D]
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            const int d = c * EPL + i;
+            const float ks = __half2float(sz[d]), kz = __half2float(sz[D + d]);
+            kf[j][i] = fzp ? fmaf(kf[j][i], ks, kz) : (kf[j][i] - kz) * ks;
+          }
         }
-        const __half* vsz = ksz + 2 * D + (off * (D / 64) + (c * EPL) / 64) * 2;
-        const float vz = __half2float(vsz[1]);
-        vscale[j] = __half2float(vsz[0]);
+        const __half* vsz = sz + 2 * D + (off * (D / 64) + grp64) * 2;
+        const float vs = __half2float(vsz[0]), vz = __half2float(vsz[1]);
+        if (fzp) {                                         // code * s + minimum
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) vf[j][i] -= vz;
+          for (int i = 0; i < EPL; ++i) vf[j][i] = fmaf(vf[j][i], vs, vz);
+        } else {                                           // (code - z), s folded into p
+          vscale[j] = vs;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) vf[j][i] -= vz;
+        }
       } else if (p.mode == KVQ_SCALE_PER_TOKEN_HEAD) {
         const float* sc = reinterpret_cast<const float*>(rec + p.off_s);
         kscale[j] = sc[off];

@@ -3,7 +3,8 @@
 //
 // Dequantized values follow the definitions in include/kvq.h: INT8 / FP8 code * scale
 // ([P-mem] §3.1 对称量化算法: q.float() * scale), INT4 (code - zero) * scale ([P-prod]
-// "量化不是简单截断精度": X_dequant = (X_q - zero_point) * scale).
+// "量化不是简单截断精度": X_dequant = (X_q - zero_point) * scale), or code * scale + minimum
+// for the float-zero-point variant.
 // The calibration scale is max|x| / 448 per kv head over warm-up rows ([P-prod]
 // "vLLM：从 FP8 KV Cache 开始试点": scales from a random-token warm-up).
 #include "kvq_internal.cuh"
@@ -60,17 +61,20 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
       default: {  // INT4
         const uint8_t byte = codes[t * p.row_bytes + d / 2];
         const int c = (d & 1) ? (byte >> 4) : (byte & 0xF);
+        // K per channel [2][D] (KIVI forms) or per token [bs][D/64][2]; V per token
         const __half* sz = reinterpret_cast<const __half*>(rec + p.off_s);
         float s, z;
-        if (kv == 0) {
+        if (kv == 0 && p.mode != KVQ_SCALE_INT4_PER_TOKEN) {
           s = __half2float(sz[d]);
           z = __half2float(sz[p.D + d]);
         } else {
-          const __half* v = sz + 2 * p.D + (t * (p.D / 64) + d / 64) * 2;
+          const __half* v = sz + (kv ? 2 * p.D : 0) + (t * (p.D / 64) + d / 64) * 2;
           s = __half2float(v[0]);
           z = __half2float(v[1]);
         }
-        x = (static_cast<float>(c) - z) * s;
+        // float zero point: code * s + minimum; integer zero point: (code - z) * s
+        x = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO ? fmaf(static_cast<float>(c), s, z)
+                                                : (static_cast<float>(c) - z) * s;
       }
     }
     out[e] = x;

@@ -8,10 +8,11 @@
 //         with one fp32 scale per token per head ([P-mem] §3.2 动态量化策略).
 //   FP8 : [P-vLLM] "KV Cache量化策略：INT8与FP8精度对比与选择" (E4M3 storage with a scale);
 //         per-head static scales as in [P-prod] "vLLM：从 FP8 KV Cache 开始试点".
-// INT4 KIVI: one CTA per (64-row group, kv head).  Keys are quantized per channel over
-// the block's 64 tokens, values per token over 64-channel groups ([P-prod] "Key 和 Value
-// 的分布不一定相同"), with the affine form of [P-prod] "量化不是简单截断精度".  Rows that
-// belong to no block are copied unquantized into the residual ring.
+// INT4: one CTA per (64-row group, kv head).  KIVI quantizes keys per channel over the
+// block's 64 tokens and values per token over 64-channel groups ([P-prod] "Key 和 Value
+// 的分布不一定相同"), with the affine form of [P-prod] "量化不是简单截断精度"; the per-token
+// variant groups keys like values, and the float-zero-point variant offsets each group by
+// its minimum.  Rows that belong to no block are copied unquantized into the residual ring.
 #include "kvq_internal.cuh"
 #include "kvq_ptx.cuh"
 
@@ -78,43 +79,62 @@ struct Int4WriteParams {
   uint8_t* pages;   // [NB][H][record]: K codes, V codes, K scale [D], K zero [D], V (s,z) [64][D/64][2]
   void* residual;   // [max_seqs][2][H][cap][D]
   int NB, H, cap, max_seqs;
-  int record, off_v, off_s;
+  int record, off_v, off_s, mode;
   int32_t* fault;
 };
 
 struct Int4Group {
   float sw;       // stored fp16 scale, widened
   __half s16;
-  int z;
+  float off;      // integer zero point z, or the stored fp16 minimum m widened
+  __half off16;   // what the record stores beside the scale: z or m
 };
 
-// lo/hi are the group's min and max; the range is widened to include 0.
-__device__ __forceinline__ Int4Group int4_group(float lo, float hi) {
-  lo = fminf(lo, 0.f);
-  hi = fmaxf(hi, 0.f);
+// lo/hi are the group's min and max.  Integer zero point: the range is widened to include
+// 0 and z = clamp(round(-lo / s), 0, 15).  Float zero point: the offset is the group
+// minimum m = fp16(lo) itself.
+__device__ __forceinline__ Int4Group int4_group(float lo, float hi, bool float_zero) {
+  if (!float_zero) {
+    lo = fminf(lo, 0.f);
+    hi = fmaxf(hi, 0.f);
+  }
   Int4Group g;
   g.s16 = __float2half_rn(div_rn(__fsub_rn(hi, lo), 15.f));
   g.sw = __half2float(g.s16);
-  g.z = (g.sw == 0.f) ? 0 : max(0, min(15, __float2int_rn(div_rn(-lo, g.sw))));
+  if (float_zero) {
+    g.off16 = __float2half_rn(lo);
+    g.off = __half2float(g.off16);
+  } else {
+    const int z = (g.sw == 0.f) ? 0 : max(0, min(15, __float2int_rn(div_rn(-lo, g.sw))));
+    g.off = static_cast<float>(z);
+    g.off16 = __int2half_rn(z);
+  }
   return g;
 }
 
-__device__ __forceinline__ int int4_code(float x, const Int4Group& g) {
+// integer zero point: clamp(round(x / s) + z, 0, 15); float: clamp(round((x - m) / s), 0, 15)
+__device__ __forceinline__ int int4_code(float x, const Int4Group& g, bool float_zero) {
   if (g.sw == 0.f) return 0;
-  return max(0, min(15, __float2int_rn(div_rn(x, g.sw)) + g.z));
+  const int r = float_zero ? __float2int_rn(div_rn(__fsub_rn(x, g.off), g.sw))
+                           : __float2int_rn(div_rn(x, g.sw)) + static_cast<int>(g.off);
+  return max(0, min(15, r));
 }
 
-// Quantize the 64 rows of one (block, kv head) into its page record: keys one group per
-// channel over the 64 tokens, values one group per token per 64 channels ([P-prod] "Key 和
-// Value 的分布不一定相同"), codes packed two per byte.  row(kv, t) points at row t (act
-// dtype, D values) of K (kv 0) or V (kv 1).  All 128 threads of the CTA take part.
+// Quantize the 64 rows of one (block, kv head) into its page record, codes packed two per
+// byte.  Values: one group per token per 64 channels.  Keys: one group per channel over the
+// 64 tokens (KIVI, [P-prod] "Key 和 Value 的分布不一定相同"), or per token like the values
+// (INT4_PER_TOKEN, the Transformers integration's choice in the same section).
+// row(kv, t) points at row t (act dtype, D values) of K (kv 0) or V (kv 1).  All 128
+// threads of the CTA take part.
 template <typename TA, int D, typename RowFn>
-__device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_s,
+__device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_s, int mode,
                                     float (*xs)[D + 1], uint8_t (*cs)[D]) {
   constexpr int G = 64;
   const int tid = threadIdx.x;
-  __half* k_sz = reinterpret_cast<__half*>(rec + off_s);           // scale [D], zero [D]
-  __half* v_sz = k_sz + 2 * D;                                     // [64][D/64][2]
+  const bool fz = mode == KVQ_SCALE_KIVI_FLOAT_ZERO;
+  const bool k_per_token = mode == KVQ_SCALE_INT4_PER_TOKEN;
+  __half* k_sz = reinterpret_cast<__half*>(rec + off_s);   // [2][D] or [64][D/64][2]
+  __half* v_sz = k_sz + 2 * D;                             // [64][D/64][2]
   for (int kv = 0; kv < 2; ++kv) {
     // stage the 64 rows of this head as float
     for (int i = tid; i < G * D / 8; i += blockDim.x) {
@@ -126,27 +146,29 @@ __device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_
       for (int j = 0; j < 8; ++j) xs[t][c * 8 + j] = f[j];
     }
     __syncthreads();
-    if (kv == 0) {
+    if (kv == 0 && !k_per_token) {
       // keys: one group per channel over the 64 tokens
       for (int d = tid; d < D; d += blockDim.x) {
         float lo = xs[0][d], hi = xs[0][d];
         for (int t = 1; t < G; ++t) { lo = fminf(lo, xs[t][d]); hi = fmaxf(hi, xs[t][d]); }
-        const Int4Group g = int4_group(lo, hi);
-        for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g));
+        const Int4Group g = int4_group(lo, hi, fz);
+        for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g, fz));
         k_sz[d] = g.s16;
-        k_sz[D + d] = __int2half_rn(g.z);
+        k_sz[D + d] = g.off16;
       }
     } else {
-      // values: one group per token per 64 channels
+      // one group per token per 64 channels
+      __half* sz_base = kv ? v_sz : k_sz;
       for (int i = tid; i < G * (D / 64); i += blockDim.x) {
         const int t = i / (D / 64), gi = i % (D / 64);
         float lo = xs[t][gi * 64], hi = lo;
         for (int j = 1; j < 64; ++j) { lo = fminf(lo, xs[t][gi * 64 + j]); hi = fmaxf(hi, xs[t][gi * 64 + j]); }
-        const Int4Group g = int4_group(lo, hi);
-        for (int j = 0; j < 64; ++j) cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g));
-        __half* sz = v_sz + (t * (D / 64) + gi) * 2;
+        const Int4Group g = int4_group(lo, hi, fz);
+        for (int j = 0; j < 64; ++j)
+          cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g, fz));
+        __half* sz = sz_base + (t * (D / 64) + gi) * 2;
         sz[0] = g.s16;
-        sz[1] = __int2half_rn(g.z);
+        sz[1] = g.off16;
       }
     }
     __syncthreads();
@@ -198,7 +220,7 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
     auto row = [&](int kv, int t) {
       return static_cast<const TA*>(kv ? p.v : p.k) + (static_cast<long>(r0 + t) * p.H + h) * D;
     };
-    quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, xs, cs);
+    quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, p.mode, xs, cs);
   } else {
     // residual rows: copied unquantized into ring row positions[t] % cap
     for (int i = tid; i < nr * 2 * (D / 8); i += blockDim.x) {
@@ -257,7 +279,7 @@ struct Int4FlushParams {
   uint8_t* pages;
   const void* residual;     // [max_seqs][2][H][cap][D]
   int NB, H, cap, max_seqs;
-  int record, off_v, off_s;
+  int record, off_v, off_s, mode;
   int32_t* fault;
 };
 
@@ -282,7 +304,7 @@ __global__ void __launch_bounds__(128) flush_ring_kernel(Int4FlushParams p) {
     return static_cast<const TA*>(p.residual) +
            ((static_cast<long>(sid * 2 + kv) * p.H + h) * p.cap + (p0 + t) % p.cap) * D;
   };
-  quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, xs, cs);
+  quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, p.mode, xs, cs);
 }
 
 }  // namespace
@@ -291,7 +313,8 @@ cudaError_t launch_flush_ring(const kvq_cache_desc& c, const Geometry& g, const 
                               const int32_t* positions, const int32_t* blocks, int n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   Int4FlushParams p{seq_ids, positions, blocks, static_cast<uint8_t*>(c.pages), c.residual,
-                    g.NB, g.H, g.residual_cap, g.max_seqs, g.record, g.off_v, g.off_s, c.fault};
+                    g.NB, g.H, g.residual_cap, g.max_seqs, g.record, g.off_v, g.off_s,
+                    g.scale_mode, c.fault};
   const dim3 grid(n, g.H);
   if (g.act_dtype == KVQ_DTYPE_BF16) {
     if (g.D == 128) flush_ring_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
@@ -319,7 +342,7 @@ cudaError_t launch_write_int4(const kvq_cache_desc& c, const Geometry& g, const 
                               const int32_t* positions, cudaStream_t s) {
   Int4WriteParams p{k, v, slots, seq_ids, positions, T, static_cast<uint8_t*>(c.pages),
                     c.residual, g.NB, g.H, g.residual_cap, g.max_seqs, g.record, g.off_v, g.off_s,
-                    c.fault};
+                    g.scale_mode, c.fault};
   const dim3 grid((T + 63) / 64, g.H);
   if (grid.x == 0) return cudaSuccess;
   if (g.act_dtype == KVQ_DTYPE_BF16) {

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 
 DTYPE = {"bf16": 0, "fp16": 1, "fp32": 2, "int8": 3, "fp8": 4, "int4": 5}
 SCALE = {"none": 0, "per_token_head": 1, "per_head": 2, "per_tensor": 3, "kivi": 4,
-         "per_channel": 5}
+         "per_channel": 5, "int4_per_token": 6, "kivi_float_zero": 7}
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "KVQ_ERR_CUDA",
           4: "KVQ_ERR_DEVICE_FAULT"}
 FAULT_BITS = {"slot": 1, "block": 2, "context": 4, "seq": 8, "int4_run": 16, "timeout": 32}

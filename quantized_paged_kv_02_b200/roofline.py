@@ -23,7 +23,10 @@ def decode_bytes(cache_dtype, scale_mode, num_q_heads, num_kv_heads, head_dim, b
             qb = group * (max(n - residual_len, 0) // group)
             nblk = qb // block_size
             total += int(2 * H * qb * D * 0.5)
-            total += H * nblk * 2 * D * 2                  # key scale + zero, fp16
+            if scale_mode == "int4_per_token":             # key scale + zero, fp16
+                total += H * qb * (D // group) * 2 * 2     # per token and channel group
+            else:
+                total += H * nblk * 2 * D * 2              # per channel and block
             total += H * qb * (D // group) * 2 * 2         # value scale + zero, fp16
             total += 2 * H * (n - qb) * D * act_bytes      # ring rows
             total += 4 * nblk

@@ -17,7 +17,7 @@ from tests import helpers
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
-SMALL = ["c1", "c2", "c3", "c4", "c5", "c5-fp8", "c5-bf16", "c5-int8-pc"]
+SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c5", "c5-fp8", "c5-bf16", "c5-int8-pc"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -61,7 +61,7 @@ def test_decode_matches_oracle(name):
     assert gc.read_fault() == (0, 0)
 
 
-@pytest.mark.parametrize("name", ["c2", "c4", "c5-fp8"])
+@pytest.mark.parametrize("name", ["c2", "c4", "c4-tok", "c4-fzp", "c5-fp8"])
 def test_split_count_does_not_change_result(name):
     w = _workload(name)
     static = helpers.oracle_static_scales(w)
@@ -189,3 +189,19 @@ def test_per_channel_needs_the_tensor_core_path():
     helpers.assert_same_cache(gc, oc)             # the write path covers every head_dim
     with pytest.raises(kvq.KVQError):
         _decode(gc, w)
+
+
+@pytest.mark.parametrize("mode", ["kivi", "int4_per_token", "kivi_float_zero"])
+@pytest.mark.parametrize("hq,d", [(4, 128), (16, 64)])
+def test_int4_cuda_core_path(mode, hq, d):
+    """INT4 caches the tensor-core kernel does not take (GQA group 2, or head_dim 64) run on
+    the CUDA-core kernel, for every INT4 form."""
+    spec = inputs.Spec("int4-simt", "int4", "bf16", mode, 2, hq, 2, d, 64, lens=[485, 200],
+                       outliers="k", slack_blocks=3, seed=5)
+    w = inputs.from_spec(spec)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    helpers.assert_same_cache(gc, oc)
+    got = _decode(gc, w).cpu().numpy().astype(np.float64)
+    assert np.abs(got - _oracle(oc, w)).max() <= TOL
+    assert gc.read_fault() == (0, 0)

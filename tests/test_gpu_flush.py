@@ -18,8 +18,9 @@ def _built():
     helpers.ensure_built()
 
 
-def test_flush_then_append_then_decode():
-    spec = inputs.Spec("flush", "int4", "bf16", "kivi", 2, 16, 2, 128, 64, lens=[485, 300],
+@pytest.mark.parametrize("mode", ["kivi", "int4_per_token", "kivi_float_zero"])
+def test_flush_then_append_then_decode(mode):
+    spec = inputs.Spec("flush", "int4", "bf16", mode, 2, 16, 2, 128, 64, lens=[485, 300],
                        outliers="k", slack_blocks=3, seed=11)
     w = inputs.from_spec(spec)
     oc = helpers.oracle_cache(w)
