@@ -184,12 +184,13 @@ __global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
 
 }  // namespace
 
-// Splits for the tensor-core kernel: one CTA per (sequence, kv head, split); pick the
-// split count whose CTA count fills whole waves of the resident slots (3 CTAs per SM),
-// preferring fewer splits, with at least 256 tokens per split.
-static void plan_mma(const Geometry& g, int batch, int max_context, DecodePlan* p) {
+// Splits for the INT4 tensor-core kernel: one CTA per (sequence, kv head, split); pick the
+// split count whose CTA count fills whole waves of the resident slots (per_sm CTAs per SM:
+// 2 for that kernel, bound by its registers), preferring fewer splits, with at least 256
+// tokens per split.
+static void plan_mma(const Geometry& g, int batch, int max_context, DecodePlan* p, long per_sm) {
   const long units = static_cast<long>(batch) * g.H;
-  const long slots = 3L * kNumSMs;
+  const long slots = per_sm * kNumSMs;
   const long max_s = std::max(1L, std::min(64L, (static_cast<long>(max_context) + 255) / 256));
   long best_s = 1;
   double best = -1.0;
@@ -220,7 +221,7 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
     const int max_qb = 64 * (std::max(max_context - g.residual_len, 0) / 64);
     Geometry gg = g;
     gg.bs = 64;
-    plan_mma(gg, batch, std::max(max_qb, 64), p);
+    plan_mma(gg, batch, std::max(max_qb, 64), p, 2);
     p->splits += 1;                              // the ring
     p->ctas = 0;
     const size_t rows = static_cast<size_t>(batch) * num_q_heads * p->splits;

@@ -74,6 +74,17 @@ __device__ __forceinline__ int swzb4(int off) {
   return (off & ~127) + ((((off >> 4) & 7) ^ ((off >> 7) & 7)) << 4) + (off & 15);
 }
 
+// Offsets of the 8-byte (scale, zero) pairs of channel groups 0 and 1 of tokens 16mt + r
+// and 16mt + r + 8 in a per-token parameter array that starts at `base` (a multiple of 128)
+// of a stage: 16 tokens fill one 128-byte swizzle row, so the two are swzb4 of base + 128mt
+// + 8r and of that + 64, in closed form.
+__device__ __forceinline__ int2 sz_offsets(int base, int mt, int r) {
+  const int x = ((base >> 7) + mt) & 7;
+  const int v = ((r >> 1) ^ x) << 4;
+  const int b0 = base + 128 * mt + 8 * (r & 1);
+  return make_int2(b0 + v, b0 + (v ^ 64));
+}
+
 // (nibble s, nibble s+4) of w as the fp16 bit patterns of (code_s, code_s+4) * 2^-24: a
 // 4-bit code placed in the mantissa of a zero exponent is an exact fp16 subnormal, so the
 // tensor cores see c * 2^-24 with no conversion instruction
@@ -235,6 +246,28 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
 
     float vlim = 0.f, vinv = 0.f;
+    // Swizzled offsets of this lane's key and value code words in tile 0 of a stage.  A
+    // tile (16 tokens of 64 bytes) is one 1024-byte swizzle period, so tile mt reads at
+    // the same offsets plus 1024 * mt: the address arithmetic is done once, not per tile.
+    int ko[4];
+    if constexpr (kTok) {
+      ko[0] = swzb4(kRowB * r + 8 * j);
+      ko[1] = swzb4(kRowB * r + 32 + 8 * j);
+      ko[2] = swzb4(kRowB * (r + 8) + 8 * j);
+      ko[3] = swzb4(kRowB * (r + 8) + 32 + 8 * j);
+    } else {
+      ko[0] = swzb4(kRowB * r + 16 * j);
+      ko[1] = swzb4(kRowB * (r + 8) + 16 * j);
+      ko[2] = ko[3] = 0;
+    }
+    int vo[4][2];                  // tokens 2j, 2j+1, 2j+8, 2j+9; channel group G; byte 4r
+    {
+      const int dts[4] = {0, 1, 8, 9};
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int G = 0; G < 2; ++G) vo[t][G] = kOffV + swzb4(kRowB * (2 * j + dts[t]) + 32 * G + 4 * r);
+    }
     for (int i = warp; i < npages; i += kC) {
       const int s = i % kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / kStages) & 1))) {
@@ -298,15 +331,16 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       }
 #pragma unroll 1
       for (int mt = 0; mt < kBS / 16; ++mt) {
-        const int tr0 = 16 * mt + r, tr1 = tr0 + 8;
+        // rows r / r + 8 of the tile: tokens tr0 = 16mt + r and tr1 = tr0 + 8
+        const uint8_t* sm = st + 1024 * mt;                  // this tile's swizzle period
         // ------------------------------------------------ S^T = (C - Zk) Q'^T
         float s00, s01, s10, s11;
         if constexpr (kTok) {
           // codes of channels [16j, 16j+16) and [64+16j, 64+16j+16): group 0 in words 0-1
-          const uint2 k0a = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr0 + 8 * j));
-          const uint2 k0b = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr0 + 32 + 8 * j));
-          const uint2 k1a = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr1 + 8 * j));
-          const uint2 k1b = *reinterpret_cast<const uint2*>(st + swzb4(kRowB * tr1 + 32 + 8 * j));
+          const uint2 k0a = *reinterpret_cast<const uint2*>(sm + ko[0]);
+          const uint2 k0b = *reinterpret_cast<const uint2*>(sm + ko[1]);
+          const uint2 k1a = *reinterpret_cast<const uint2*>(sm + ko[2]);
+          const uint2 k1b = *reinterpret_cast<const uint2*>(sm + ko[3]);
           const uint32_t w0[4] = {k0a.x, k0a.y, k0b.x, k0b.y}, w1[4] = {k1a.x, k1a.y, k1b.x, k1b.y};
           float sg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -317,8 +351,9 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             mma_f16(sg[kc >> 2], a, qt[kc]);
           }
           // (scale, zero) of tokens tr0 / tr1, groups 0 and 1: fp16 at kOffKs + 8t + 4G
-          const uint2 z0 = *reinterpret_cast<const uint2*>(st + swzb4(kOffKs + 8 * tr0));
-          const uint2 z1 = *reinterpret_cast<const uint2*>(st + swzb4(kOffKs + 8 * tr1));
+          const int2 ko2 = sz_offsets(kOffKs, mt, r);
+          const uint2 z0 = *reinterpret_cast<const uint2*>(st + ko2.x);
+          const uint2 z1 = *reinterpret_cast<const uint2*>(st + ko2.y);
           const float2 a00 = __half22float2(*reinterpret_cast<const __half2*>(&z0.x));   // t0 G0
           const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&z0.y));   // t0 G1
           const float2 a10 = __half22float2(*reinterpret_cast<const __half2*>(&z1.x));
@@ -332,8 +367,8 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           s11 = (a10.x * fmaf(sg[0][3], 16777216.f, -a10.y * qg[0][1]) +
                  a11.x * fmaf(sg[1][3], 16777216.f, -a11.y * qg[1][1])) * qscale;
         } else {
-          const uint4 k0 = lds128(st + swzb4(kRowB * tr0 + 16 * j));
-          const uint4 k1 = lds128(st + swzb4(kRowB * tr1 + 16 * j));
+          const uint4 k0 = lds128(sm + ko[0]);
+          const uint4 k1 = lds128(sm + ko[1]);
           const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
           float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -382,10 +417,10 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         l[1] += p01 + p11;
         // ------------------------------------------------ value scales folded into P
         // vsz for token t, group G: (scale, zero) fp16 at kOffVsz + 8t + 4G
-        const uint32_t sz00 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr0));
-        const uint32_t sz01 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr0 + 4));
-        const uint32_t sz10 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr1));
-        const uint32_t sz11 = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffVsz + 8 * tr1 + 4));
+        const int2 vo2 = sz_offsets(kOffVsz, mt, r);
+        const uint2 vz0 = *reinterpret_cast<const uint2*>(st + vo2.x);
+        const uint2 vz1 = *reinterpret_cast<const uint2*>(st + vo2.y);
+        const uint32_t sz00 = vz0.x, sz01 = vz0.y, sz10 = vz1.x, sz11 = vz1.y;
         float vs[2][2] = {{__half2float(__ushort_as_half(sz00 & 0xFFFF)), __half2float(__ushort_as_half(sz01 & 0xFFFF))},
                           {__half2float(__ushort_as_half(sz10 & 0xFFFF)), __half2float(__ushort_as_half(sz11 & 0xFFFF))}};
         if (__any_sync(0xffffffffu, vs[0][0] >= vlim || vs[0][1] >= vlim || vs[1][0] >= vlim || vs[1][1] >= vlim)) {
@@ -436,14 +471,12 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         // ------------------------------------------------ O^T += (C - Zv)^T P'^T
         // tile md: group G = md/4, byte k = md%4 of the word holding channels
         // 64G + 8r .. +7 of a token; rows r / r+8 <-> d = 64G + 8r + 2k / +1
-        const int ta = 16 * mt + 2 * j;
-        const int tt[4] = {ta, ta + 1, ta + 8, ta + 9};
         uint32_t vwd[4][2];
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
           for (int G = 0; G < 2; ++G)
-            vwd[t][G] = *reinterpret_cast<const uint32_t*>(st + swzb4(kOffV + kRowB * tt[t] + 32 * G + 4 * r));
+            vwd[t][G] = *reinterpret_cast<const uint32_t*>(sm + vo[t][G]);
 #pragma unroll
         for (int md = 0; md < 8; ++md) {
           const int G = md >> 2, k = md & 3;
@@ -528,11 +561,17 @@ cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaS
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(decode_int4_kernel<kKivi>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(decode_int4_kernel<kKiviMin>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(decode_int4_kernel<kPerToken>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    // two CTAs per SM (registers): both rings need the maximum shared-memory carveout
+    const void* fns[3] = {reinterpret_cast<const void*>(decode_int4_kernel<kKivi>),
+                          reinterpret_cast<const void*>(decode_int4_kernel<kKiviMin>),
+                          reinterpret_cast<const void*>(decode_int4_kernel<kPerToken>)};
+    for (const void* f : fns) {
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        cudaSharedmemCarveoutMaxShared);
+    }
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap tm;
