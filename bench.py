@@ -250,7 +250,7 @@ def oracle_unit_step(w, unit_rows, b, kvh, static):
     if static is not None:
         st = (static[0][kvh:kvh + 1], static[1][kvh:kvh + 1])
     bs = s.block_size
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         qb = 64 * (max(n - 128, 0) // 64)
         nblk = qb // 64
     else:
@@ -294,7 +294,7 @@ def unit_bytes(w, b):
     return (roofline.decode_bytes(s.cache_dtype, s.scale_mode, g, 1, s.head_dim, s.block_size,
                                   [int(w.context_lens[b])])
             + roofline.write_bytes(s.cache_dtype, s.scale_mode, 1, 1, s.head_dim,
-                                   to_ring=s.cache_dtype == "int4"))
+                                   to_ring=inputs.low_bit(s.cache_dtype)))
 
 
 def unit_workload(name):
@@ -365,7 +365,7 @@ def build_state(workload, device, seed, batch=0):
                          s.num_kv_heads, s.head_dim, device=device,
                          residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
                          max_seqs=s.batch, static_k_scale=sk, static_v_scale=sv)
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         idx, slots, sid, pos = inputs.int4_group_rows(w)
         idx = idx.to(device)
         c.write(w.k[idx].contiguous(), w.v[idx].contiguous(), slots.to(device), sid.to(device),
@@ -375,7 +375,7 @@ def build_state(workload, device, seed, batch=0):
     # the step's new token: the last position of every sequence
     last = (w.seq_start[1:] - 1).to(device)
     new = {"k": w.k[last].contiguous(), "v": w.v[last].contiguous()}
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         new["slots"] = torch.full((s.batch,), -1, dtype=torch.int32, device=device)
         new["seq_ids"] = torch.arange(s.batch, dtype=torch.int32, device=device)
         new["positions"] = (w.context_lens - 1).to(torch.int32)
@@ -437,7 +437,7 @@ def main_ours(args):
     dec_bytes = roofline.decode_bytes(s.cache_dtype, s.scale_mode, s.num_q_heads, s.num_kv_heads,
                                       s.head_dim, s.block_size, lens)
     wr_bytes = roofline.write_bytes(s.cache_dtype, s.scale_mode, B, s.num_kv_heads, s.head_dim,
-                                    to_ring=s.cache_dtype == "int4")
+                                    to_ring=inputs.low_bit(s.cache_dtype))
     step_bytes = dec_bytes + wr_bytes
     l2 = L2Flush(device)
 
@@ -479,7 +479,7 @@ def main_ours(args):
 
     # the same step as one call (kvq_append_decode_attention), dense caches only
     fused = None
-    if s.cache_dtype != "int4" and K > 0:
+    if not inputs.low_bit(s.cache_dtype) and K > 0:
         def fused_step():
             kvq.kvq_append_decode_attention(cache.desc, new["k"], new["v"], w.q, w.block_tables,
                                             w.context_lens, max_ctx, out, ws)

@@ -17,6 +17,7 @@ SENTINEL = 0x5A
 
 DENSE_DTYPES = ("bf16", "fp16", "int8", "fp8")
 INT4_MODES = ("kivi", "kivi_float_zero", "int4_per_token")
+LOW_BIT = {"int4": 4, "int2": 2}              # group-quantized caches: bits per code
 
 
 def _bits_of_act(x, act):
@@ -41,10 +42,11 @@ def _value_of_act_bits(bits, act):
 class PagedCache:
     """One layer's paged cache.
 
-    cache_dtype: "bf16" | "fp16" | "int8" | "fp8" | "int4"
+    cache_dtype: "bf16" | "fp16" | "int8" | "fp8" | "int4" | "int2"
     act_dtype:   "bf16" | "fp16"
     scale_mode:  "none" | "per_token_head" | "per_head" | "per_tensor" | "per_channel" for
-                 dense caches; "kivi" | "kivi_float_zero" | "int4_per_token" for INT4
+                 dense caches; "kivi" | "kivi_float_zero" | "int4_per_token" for INT4 and
+                 2-bit caches (the same groups and records, codes of 4 or 2 bits)
     static_scales: (k_scale, v_scale) float32 arrays for static modes: [H] per head, [1]
                    per tensor, [H, D] per (kv head, channel).
 
@@ -72,9 +74,9 @@ class PagedCache:
             code_dt, row_bytes = np.int8, D
         elif cache_dtype == "fp8":
             code_dt, row_bytes = np.uint8, D
-        elif cache_dtype == "int4":
+        elif cache_dtype in LOW_BIT:
             assert scale_mode in INT4_MODES and block_size == group_size == 64
-            code_dt, row_bytes = np.uint8, D // 2
+            code_dt, row_bytes = np.uint8, D * LOW_BIT[cache_dtype] // 8
         else:
             raise ValueError(cache_dtype)
         off_s = 2 * bs * row_bytes
@@ -103,7 +105,7 @@ class PagedCache:
             ks, vs = static_scales
             self.k_scales = np.asarray(ks, np.float32).reshape(shape).copy()
             self.v_scales = np.asarray(vs, np.float32).reshape(shape).copy()
-        elif cache_dtype == "int4":
+        elif cache_dtype in LOW_BIT:
             if scale_mode == "int4_per_token":
                 # K (scale, zero) [bs][D/G][2], then V the same
                 half = scale_bytes // 2
@@ -138,7 +140,7 @@ class PagedCache:
         k_new = np.asarray(k_new, np.float64)
         v_new = np.asarray(v_new, np.float64)
         slots = np.asarray(slot_mapping, np.int64)
-        if self.cd == "int4":
+        if self.cd in LOW_BIT:
             return self._write_int4(k_new, v_new, slots, seq_ids, positions)
         NB, bs = self.NB, self.bs
         keep = (slots >= 0) & (slots < NB * bs)
@@ -193,19 +195,20 @@ class PagedCache:
                 # keys per (head, channel) over the block's rows; values per (row, head,
                 # channel group); every group on its own, all heads at once
                 fz = self.mode == "kivi_float_zero"
+                bits = LOW_BIT[self.cd]
                 kb = np.swapaxes(k_new[u:u + G].astype(np.float32), 0, 1)     # [H, G, D]
                 if self.mode == "int4_per_token":
-                    kc, ks, kz = quant.int4_values_row(kb, self.G)            # like values
+                    kc, ks, kz = quant.int4_values_row(kb, self.G, bits=bits)  # like values
                     self.k_scales[blk, :, :, :, 0] = ks
                     self.k_scales[blk, :, :, :, 1] = kz
                 else:
-                    kc, ks, kz = quant.int4_keys_block(kb, float_zero=fz)
+                    kc, ks, kz = quant.int4_keys_block(kb, float_zero=fz, bits=bits)
                     self.k_scales[blk, :, 0, :] = ks
                     self.k_scales[blk, :, 1, :] = kz
-                self.k_codes[blk] = quant.pack_nibbles(kc)
+                self.k_codes[blk] = quant.pack_codes(kc, bits)
                 vb = np.swapaxes(v_new[u:u + G].astype(np.float32), 0, 1)     # [H, G, D]
-                vc, vs, vz = quant.int4_values_row(vb, self.G, float_zero=fz)
-                self.v_codes[blk] = quant.pack_nibbles(vc)
+                vc, vs, vz = quant.int4_values_row(vb, self.G, float_zero=fz, bits=bits)
+                self.v_codes[blk] = quant.pack_codes(vc, bits)
                 self.v_scales[blk, :, :, :, 0] = vs
                 self.v_scales[blk, :, :, :, 1] = vz
             else:
@@ -254,7 +257,7 @@ class PagedCache:
                 deq = quant.int8_dequantize if self.cd == "int8" else quant.fp8_dequantize
                 out[which] = deq(c, s)
             else:
-                q = quant.unpack_nibbles(c).astype(np.float64)  # [H, bs, D]
+                q = quant.unpack_codes(c, LOW_BIT[self.cd]).astype(np.float64)  # [H, bs, D]
                 if which == 0 and self.mode != "int4_per_token":
                     s = self.k_scales[blk, :, 0, :].astype(np.float64)[:, None, :]   # [H, 1, D]
                     z = self.k_scales[blk, :, 1, :].astype(np.float64)[:, None, :]
@@ -270,7 +273,7 @@ class PagedCache:
 
     def quantized_prefix(self, n):
         """INT4: number of leading positions read from blocks; the rest is in the ring."""
-        if self.cd != "int4":
+        if self.cd not in LOW_BIT:
             return n
         return self.G * (max(n - self.R, 0) // self.G)
 

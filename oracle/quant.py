@@ -16,6 +16,8 @@ Readings of the pages taken here (each listed in the design doc):
   * INT4 uses the affine form of [P-prod] "量化不是简单截断精度"
     (X_q = round(X/scale) + zero_point; X_deq = (X_q - zero_point) * scale) with the
     range widened to include 0, so the zero point is an integer in [0, 15].
+  * 2-bit caches use the same quantizers with 3 as the largest code ([P-prod] "KV Cache 的基本
+    内存模型" lists 2-bit at 0.25 byte per value; "误区二：INT4 或 2-bit 一定比 FP8 更划算").
   * The float-zero-point INT4 variant takes the group minimum itself as the offset
     (X_deq = X_q * scale + min, the range not widened); the pages name only the integer
     form, so this variant is a reading of "zero point" as a real offset.
@@ -28,6 +30,11 @@ from . import fp
 INT8_QMAX = 127.0
 FP8_QMAX = fp.E4M3_MAX
 INT4_LEVELS = 15.0
+
+
+def levels(bits):
+    """Largest code of a `bits`-bit unsigned code: 15 for INT4, 3 for 2-bit."""
+    return float((1 << bits) - 1)
 
 
 # ----------------------------------------------------------------------------- INT8
@@ -122,53 +129,57 @@ def fp8_dequantize(codes, scale):
 
 
 # ----------------------------------------------------------------------------- INT4
-def int4_quantize_groups(values):
-    """Asymmetric 4-bit quantization of groups along the last axis (binary32 values).
+def int4_quantize_groups(values, bits=4):
+    """Asymmetric 4-bit (or 2-bit) quantization of groups along the last axis (binary32
+    values), with Q = 2^bits - 1 the largest code (15, or 3).
 
     Every group (1-D slice values[..., :]) is quantized on its own.  Returns (codes
-    uint8 in 0..15 with the shape of values, scale float16 and zero point float16 with
+    uint8 in 0..Q with the shape of values, scale float16 and zero point float16 with
     the leading shape).
       lo = min(min x, 0); hi = max(max x, 0)
-      s  = float16(binary32((hi - lo) / 15))       -- stored, and used from here on
-      z  = clamp(round_half_even(-lo / s), 0, 15)
-      q  = clamp(round_half_even(x / s) + z, 0, 15)
+      s  = float16(binary32((hi - lo) / Q))        -- stored, and used from here on
+      z  = clamp(round_half_even(-lo / s), 0, Q)
+      q  = clamp(round_half_even(x / s) + z, 0, Q)
     A group whose s is 0 (all values 0) gets codes 0, scale 0, zero point 0.
     [P-prod] "量化不是简单截断精度": X_q = round(X/scale) + zero_point.
     """
+    Q = levels(bits)
     x = np.asarray(values, dtype=np.float32)
     lo = np.minimum(x.min(axis=-1), np.float32(0.0))
     hi = np.maximum(x.max(axis=-1), np.float32(0.0))
-    s32 = fp.div32(fp.sub32(hi, lo), np.float32(INT4_LEVELS))
+    s32 = fp.div32(fp.sub32(hi, lo), np.float32(Q))
     s16 = fp.f16(s32)
     zero_group = s16 == 0
     sw = np.where(zero_group, np.float32(1.0), np.asarray(s16, np.float32))
-    z = np.clip(fp.round_half_even(fp.div32(-lo, sw)), 0, 15)
-    q = np.clip(fp.round_half_even(fp.div32(x, sw[..., None])) + z[..., None], 0, 15)
+    z = np.clip(fp.round_half_even(fp.div32(-lo, sw)), 0, Q)
+    q = np.clip(fp.round_half_even(fp.div32(x, sw[..., None])) + z[..., None], 0, Q)
     q = np.where(zero_group[..., None], 0, q)
     z = np.where(zero_group, 0, z)
     return q.astype(np.uint8), np.asarray(s16, np.float16), np.asarray(z, np.float16)
 
 
-def int4_quantize_groups_float_zero(values):
-    """Asymmetric 4-bit quantization with a float zero point (the group minimum).
+def int4_quantize_groups_float_zero(values, bits=4):
+    """Asymmetric 4-bit (or 2-bit) quantization with a float zero point (the group
+    minimum), Q = 2^bits - 1 the largest code.
 
-    Every group (1-D slice values[..., :]) on its own.  Returns (codes uint8 in 0..15,
+    Every group (1-D slice values[..., :]) on its own.  Returns (codes uint8 in 0..Q,
     scale float16, minimum float16), the last two with the leading shape.
       lo = min x; hi = max x
-      s  = float16(binary32((hi - lo) / 15));  m = float16(lo)   -- stored, used from here on
-      q  = clamp(round_half_even(binary32(binary32(x - m) / s)), 0, 15)
+      s  = float16(binary32((hi - lo) / Q));  m = float16(lo)    -- stored, used from here on
+      q  = clamp(round_half_even(binary32(binary32(x - m) / s)), 0, Q)
     A group whose s is 0 (constant, or a range below float16's reach) gets codes 0.
     Dequantized value: q * s + m.
     """
+    Q = levels(bits)
     x = np.asarray(values, dtype=np.float32)
     lo = x.min(axis=-1)
     hi = x.max(axis=-1)
-    s16 = fp.f16(fp.div32(fp.sub32(hi, lo), np.float32(INT4_LEVELS)))
+    s16 = fp.f16(fp.div32(fp.sub32(hi, lo), np.float32(Q)))
     m16 = fp.f16(lo)
     zero_group = s16 == 0
     sw = np.where(zero_group, np.float32(1.0), np.asarray(s16, np.float32))
     mw = np.asarray(m16, np.float32)
-    q = np.clip(fp.round_half_even(fp.div32(fp.sub32(x, mw[..., None]), sw[..., None])), 0, 15)
+    q = np.clip(fp.round_half_even(fp.div32(fp.sub32(x, mw[..., None]), sw[..., None])), 0, Q)
     q = np.where(zero_group[..., None], 0, q)
     return q.astype(np.uint8), np.asarray(s16, np.float16), np.asarray(m16, np.float16)
 
@@ -178,8 +189,9 @@ def int4_dequantize_float_zero(codes, scale, minimum):
     return np.asarray(codes, np.float64) * np.float64(scale) + np.float64(minimum)
 
 
-def _groups(float_zero):
-    return int4_quantize_groups_float_zero if float_zero else int4_quantize_groups
+def _groups(float_zero, bits):
+    f = int4_quantize_groups_float_zero if float_zero else int4_quantize_groups
+    return lambda v: f(v, bits)
 
 
 def int4_quantize_group(values):
@@ -193,7 +205,7 @@ def int4_dequantize(codes, scale, zero):
     return (np.asarray(codes, np.float64) - np.float64(zero)) * np.float64(scale)
 
 
-def int4_keys_block(k_rows, float_zero=False):
+def int4_keys_block(k_rows, float_zero=False, bits=4):
     """KIVI keys: one group per channel over the block's tokens.
 
     k_rows [64, D] (one kv head), or [..., 64, D] for several heads at once.  Returns
@@ -201,11 +213,11 @@ def int4_keys_block(k_rows, float_zero=False):
     [P-prod] "Key 和 Value 的分布不一定相同": key cache per channel (KIVI).
     """
     k_rows = np.asarray(k_rows, dtype=np.float32)
-    q, s, z = _groups(float_zero)(np.swapaxes(k_rows, -1, -2))     # groups = channels
+    q, s, z = _groups(float_zero, bits)(np.swapaxes(k_rows, -1, -2))     # groups = channels
     return np.swapaxes(q, -1, -2), s, z
 
 
-def int4_values_row(v_row, group=64, float_zero=False):
+def int4_values_row(v_row, group=64, float_zero=False, bits=4):
     """One group per token over each run of `group` channels: KIVI values, and keys as well
     as values in the per-token variant.
 
@@ -216,8 +228,27 @@ def int4_values_row(v_row, group=64, float_zero=False):
     """
     v_row = np.asarray(v_row, dtype=np.float32)
     D = v_row.shape[-1]
-    q, s, z = _groups(float_zero)(v_row.reshape(v_row.shape[:-1] + (D // group, group)))
+    q, s, z = _groups(float_zero, bits)(v_row.reshape(v_row.shape[:-1] + (D // group, group)))
     return q.reshape(v_row.shape), s, z
+
+
+def pack_codes(codes, bits):
+    """Pack `bits`-bit codes (4 or 2) along the last axis, 8 / bits per byte: element
+    k*i + e of a run of k = 8 / bits goes to bits [bits*e, bits*e + bits) of byte i."""
+    if bits == 4:
+        return pack_nibbles(codes)
+    c = np.asarray(codes, dtype=np.uint8) & 3
+    return c[..., 0::4] | (c[..., 1::4] << 2) | (c[..., 2::4] << 4) | (c[..., 3::4] << 6)
+
+
+def unpack_codes(packed, bits):
+    if bits == 4:
+        return unpack_nibbles(packed)
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (p.shape[-1] * 4,), np.uint8)
+    for e in range(4):
+        out[..., e::4] = (p >> (2 * e)) & 3
+    return out
 
 
 def pack_nibbles(codes):

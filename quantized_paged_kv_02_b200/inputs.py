@@ -32,10 +32,15 @@ RESIDUAL_CAP = 192
 INT4_GROUP = 64
 
 
+def low_bit(cache_dtype):
+    """INT4 and 2-bit caches: 64-token groups, a residual ring of recent tokens."""
+    return cache_dtype in ("int4", "int2")
+
+
 @dataclass
 class Spec:
     name: str
-    cache_dtype: str            # bf16 | fp16 | int8 | fp8 | int4
+    cache_dtype: str            # bf16 | fp16 | int8 | fp8 | int4 | int2
     act_dtype: str              # bf16 | fp16
     scale_mode: str             # none | per_token_head | per_head | per_tensor | per_channel |
                                 # kivi | kivi_float_zero | int4_per_token
@@ -67,14 +72,16 @@ def _spec(name, small):
                         len_range=(100, 700), slack_blocks=9)
         return Spec("c3", "fp8", "bf16", "per_head", 64, 32, 8, 128, 16,
                     len_range=(1024, 8192), slack_blocks=64)
-    if name in ("c4", "c4-tok", "c4-fzp"):
-        # c4-tok: keys and values per token (64-channel groups); c4-fzp: KIVI groups with
-        # the group minimum as a float zero point; same shapes and inputs as c4
-        mode = {"c4": "kivi", "c4-tok": "int4_per_token", "c4-fzp": "kivi_float_zero"}[name]
+    if name in ("c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok", "c4-int2-fzp"):
+        # -tok: keys and values per token (64-channel groups); -fzp: KIVI groups with the
+        # group minimum as a float zero point; -int2: 2-bit codes; shapes and inputs as c4
+        mode = "int4_per_token" if name.endswith("-tok") else \
+            "kivi_float_zero" if name.endswith("-fzp") else "kivi"
+        cd = "int2" if "int2" in name else "int4"
         if small:
-            return Spec(name + "-small", "int4", "bf16", mode, 2, 16, 2, 128, 64,
+            return Spec(name + "-small", cd, "bf16", mode, 2, 16, 2, 128, 64,
                         lens=[485, 200], outliers="k", slack_blocks=3)
-        return Spec(name, "int4", "bf16", mode, 16, 64, 8, 128, 64,
+        return Spec(name, cd, "bf16", mode, 16, 64, 8, 128, 64,
                     lens=[32768] * 16, outliers="k", slack_blocks=16)
     if name.startswith("c5"):
         cd = {"c5": "int8", "c5-int8": "int8", "c5-fp8": "fp8", "c5-bf16": "bf16",
@@ -117,8 +124,8 @@ def act_torch_dtype(act):
 
 
 def make(name, small=False, device="cpu", seed=None):
-    """Build the named workload ("c1".."c5", "c4-tok", "c4-fzp", "c5-fp8", "c5-bf16",
-    "c5-int8-pc") on `device`."""
+    """Build the named workload ("c1".."c5", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok",
+    "c4-int2-fzp", "c5-fp8", "c5-bf16", "c5-int8-pc") on `device`."""
     spec = _spec(name, small)
     if seed is not None:
         spec.seed = seed
@@ -150,7 +157,7 @@ def from_spec(spec, device="cpu"):
     k, v, q = k.to(adt), v.to(adt), q.to(adt)
 
     # paged placement: rows of sequence b at positions 0..n_b-1
-    int4 = spec.cache_dtype == "int4"
+    int4 = low_bit(spec.cache_dtype)
     paged = []
     for n in lens.tolist():
         if int4:

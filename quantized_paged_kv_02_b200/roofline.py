@@ -10,7 +10,7 @@ metadata bytes the same section says make the real gain smaller.  Split partials
 the reduce's round trip are not algorithmic and are not counted.
 """
 
-CODE_BYTES = {"bf16": 2.0, "fp16": 2.0, "int8": 1.0, "fp8": 1.0, "int4": 0.5}
+CODE_BYTES = {"bf16": 2.0, "fp16": 2.0, "int8": 1.0, "fp8": 1.0, "int4": 0.5, "int2": 0.25}
 
 
 def decode_bytes(cache_dtype, scale_mode, num_q_heads, num_kv_heads, head_dim, block_size,
@@ -19,10 +19,10 @@ def decode_bytes(cache_dtype, scale_mode, num_q_heads, num_kv_heads, head_dim, b
     total = 0
     for n in context_lens:
         n = int(n)
-        if cache_dtype == "int4":
+        if cache_dtype in ("int4", "int2"):
             qb = group * (max(n - residual_len, 0) // group)
             nblk = qb // block_size
-            total += int(2 * H * qb * D * 0.5)
+            total += int(2 * H * qb * D * CODE_BYTES[cache_dtype])
             if scale_mode == "int4_per_token":             # key scale + zero, fp16
                 total += H * qb * (D // group) * 2 * 2     # per token and channel group
             else:

@@ -46,7 +46,7 @@ def oracle_cache(w, static=None):
                          residual_cap=inputs.RESIDUAL_CAP, max_seqs=max(s.batch, 1),
                          static_scales=static)
     k, v = np64(w.k), np64(w.v)
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         idx, slots, sid, pos = inputs.int4_group_rows(w)
         c.write(k[idx.numpy()], v[idx.numpy()], slots.numpy(), sid.numpy(), pos.numpy())
     else:
@@ -66,7 +66,7 @@ def gpu_cache(w, device="cuda", static=None, fill=0x5A):
                          residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
                          max_seqs=max(s.batch, 1), static_k_scale=sk, static_v_scale=sv, fill=fill)
     k, v = w.k.to(device), w.v.to(device)
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         idx, slots, sid, pos = inputs.int4_group_rows(w)
         idx = idx.to(device)
         c.write(k[idx].contiguous(), v[idx].contiguous(), slots.to(device), sid.to(device),
@@ -99,7 +99,7 @@ def single_sequence(w, b):
     s = w.spec
     r0, r1 = int(w.seq_start[b]), int(w.seq_start[b + 1])
     n = r1 - r0
-    int4 = s.cache_dtype == "int4"
+    int4 = inputs.low_bit(s.cache_dtype)
     paged = inputs.INT4_GROUP * (max(n - inputs.RESIDUAL_LEN, 0) // inputs.INT4_GROUP) if int4 else n
     nblk = max(-(-paged // s.block_size), 1)
     pos = torch.arange(n, dtype=torch.int32)

@@ -24,7 +24,7 @@ def _build(w, static_scales=None, max_seqs=None):
                          s.num_kv_heads, s.head_dim, residual_len=inputs.RESIDUAL_LEN,
                          residual_cap=inputs.RESIDUAL_CAP,
                          max_seqs=max_seqs or s.batch, static_scales=static_scales)
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         idx, slots, sid, pos = inputs.int4_group_rows(w)
         c.write(_np(w.k)[idx.numpy()], _np(w.v)[idx.numpy()], slots.numpy(), sid.numpy(), pos.numpy())
     else:
@@ -189,22 +189,26 @@ def test_int4_grid_exact_attention_equals_sdpa():
         assert np.all(c.k_codes[blk] == cache.SENTINEL) and np.all(c.v_codes[blk] == cache.SENTINEL)
 
 
-@pytest.mark.parametrize("mode", ["int4_per_token", "kivi_float_zero"])
-def test_int4_variants_grid_exact_attention_equals_sdpa(mode):
-    """The per-token variant (keys grouped per token over 64 channels, like values) and the
-    float-zero-point variant (offset = group minimum, the range need not include 0): on
-    their grids quantization is exact, so attention equals SDPA on the dense rows."""
+@pytest.mark.parametrize("cd,mode", [("int4", "int4_per_token"), ("int4", "kivi_float_zero"),
+                                     ("int2", "kivi"), ("int2", "int4_per_token"),
+                                     ("int2", "kivi_float_zero")])
+def test_int4_variants_grid_exact_attention_equals_sdpa(cd, mode):
+    """The per-token variant (keys grouped per token over 64 channels, like values), the
+    float-zero-point variant (offset = group minimum, the range need not include 0) and the
+    2-bit caches: on their grids quantization is exact, so attention equals SDPA on the
+    dense rows."""
     rng = np.random.default_rng(3)
     H, D, n = 1, 128, 64 * 3 + 128 + 21
     qb = 192
+    Q = int(quant.levels(cache.LOW_BIT[cd]))
 
     def grid():
-        k = rng.integers(0, 16, 64)
-        k[0], k[1] = 0, 15
+        k = rng.integers(0, Q + 1, 64)
+        k[0], k[1] = 0, Q
         e = rng.integers(1, 5)
         if mode == "kivi_float_zero":
             return rng.integers(-40, 41) * 2.0 ** -3 + k * 2.0 ** -e
-        return (k - rng.integers(0, 16)) * 2.0 ** -e
+        return (k - rng.integers(0, Q + 1)) * 2.0 ** -e
 
     K = np.empty((n, H, D))
     V = np.empty((n, H, D))
@@ -213,18 +217,19 @@ def test_int4_variants_grid_exact_attention_equals_sdpa(mode):
             V[p, 0, gi * 64:(gi + 1) * 64] = grid()
             if mode == "int4_per_token":
                 K[p, 0, gi * 64:(gi + 1) * 64] = grid()
-    if mode == "kivi_float_zero":
+    if mode != "int4_per_token":
         for blk in range(qb // 64):
             for d in range(D):
                 K[blk * 64:(blk + 1) * 64, 0, d] = grid()
     K[qb:] = fp.bf16_round(rng.standard_normal((n - qb, H, D)))
     V[qb:] = fp.bf16_round(rng.standard_normal((n - qb, H, D)))
     assert np.array_equal(fp.bf16_round(K), K) and np.array_equal(fp.bf16_round(V), V)
-    c = cache.PagedCache("int4", "bf16", mode, 5, 64, H, D, max_seqs=2)
+    c = cache.PagedCache(cd, "bf16", mode, 5, 64, H, D, max_seqs=2)
     table = np.array([3, 0, 4])
     slots = np.array([table[p // 64] * 64 + p % 64 for p in range(qb)] + [-1] * (n - qb))
     pos = np.array([-1] * qb + list(range(qb, n)))
     c.write(K, V, slots, np.ones(n, np.int64), pos)
+    assert c.record == {"int4": 9216, "int2": 5120}[cd]
     q = fp.bf16_round(rng.standard_normal((1, 4, D)))
     out = attention.decode_attention(c, q, table[None, :], np.array([n]), seq_ids=np.array([1]))
     for hq in range(4):
@@ -232,12 +237,13 @@ def test_int4_variants_grid_exact_attention_equals_sdpa(mode):
                                    rtol=1e-12, atol=1e-12)
     if mode == "kivi_float_zero":
         assert np.any(c.k_scales[table, 0, 1, :] > 0)      # minima above 0 occur
-    else:
+    elif mode == "int4_per_token":
         assert c.k_scales.shape[2:] == (64, 2, 2)          # [bs][D/64][(scale, zero)]
 
 
 # ---------------------------------------------------------------- invariants
-@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c5"])
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2",
+                                  "c4-int2-tok", "c4-int2-fzp", "c5"])
 def test_invariants_on_small_workloads(name):
     w = inputs.make(name, small=True)
     s = w.spec
@@ -263,10 +269,11 @@ def test_invariants_on_small_workloads(name):
         elif s.cache_dtype == "fp8":         # 3 mantissa bits, plus saturation at 448 s
             sk = static[0].astype(np.float64)[:, None, None]
             bound = np.abs(kk) / 16 + np.maximum(np.abs(kk) - 448 * sk, 0) + sk * 2.0 ** -10
-        elif s.cache_dtype == "int4":        # half a step of the widest group
+        elif inputs.low_bit(s.cache_dtype):  # half a step of the widest group
             qb = c.quantized_prefix(n)
             rng_ = np.abs(kk).max() * 2
-            bound = np.full(kk.shape, rng_ / 15 * (0.5 + 15 * 2.0 ** -11))
+            Q = quant.levels(cache.LOW_BIT[s.cache_dtype])
+            bound = np.full(kk.shape, rng_ / Q * (0.5 + Q * 2.0 ** -11))
             bound[:, qb:] = 0                # residual ring rows are exact
         else:
             bound = np.zeros(kk.shape)
@@ -285,7 +292,7 @@ def _build_permuted(w, static, perm):
     new = np.where(slots >= 0, perm[slots // s.block_size] * s.block_size + slots % s.block_size, -1)
     c = cache.PagedCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
                          s.num_kv_heads, s.head_dim, max_seqs=s.batch, static_scales=static)
-    if s.cache_dtype == "int4":
+    if inputs.low_bit(s.cache_dtype):
         idx, _, sid, pos = inputs.int4_group_rows(w)
         c.write(_np(w.k)[idx.numpy()], _np(w.v)[idx.numpy()], new[idx.numpy()], sid.numpy(), pos.numpy())
     else:
@@ -337,7 +344,7 @@ def test_int4_prefix_split():
         [0, 0, 0, 0, 64, 64, 128, 32640]
 
 
-@pytest.mark.parametrize("name", ["c4", "c4-tok", "c4-fzp"])
+@pytest.mark.parametrize("name", ["c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-fzp"])
 def test_flush_ring_equals_writing_the_rows(name):
     """Flushing ring rows [p0, p0+64) into a block stores what writing those rows with the
     block's slots stores (the definition in include/kvq.h)."""

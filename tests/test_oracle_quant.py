@@ -267,3 +267,61 @@ def test_int4_per_token_keys_group_like_values():
     c1, s1, z1 = quant.int4_values_row(k[7])
     np.testing.assert_array_equal(c[7], c1)
     np.testing.assert_array_equal(s[7], s1)
+
+
+# ------------------------------------------------------------------------- 2-bit
+@pytest.mark.parametrize("float_zero", [False, True])
+def test_int2_nearest_code_bruteforce(float_zero):
+    """2-bit groups (codes 0..3): each code is a nearest grid point given the stored
+    parameters, for both zero-point forms."""
+    g = torch.Generator().manual_seed(31)
+    for trial in range(40):
+        x = (torch.randn(64, generator=g) * (0.1 + trial) + (trial % 5 - 2)).to(torch.bfloat16)
+        x = x.float().numpy()
+        if float_zero:
+            c, s, m = quant.int4_quantize_groups_float_zero(x[None], bits=2)
+            grid = np.arange(4) * np.float64(s[0]) + np.float64(m[0])
+        else:
+            c, s, z = quant.int4_quantize_groups(x[None], bits=2)
+            assert 0 <= float(z[0]) <= 3
+            grid = (np.arange(4) - np.float64(z[0])) * np.float64(s[0])
+        d = np.abs(x.astype(np.float64)[:, None] - grid[None, :])
+        chosen = d[np.arange(64), c[0]]
+        assert c.max() <= 3
+        assert np.all(chosen <= d.min(axis=1) + 2.0 ** -20 * float(s[0]))
+
+
+def test_int2_steps_exact():
+    """s = fp16(fp32((hi - lo) / 3)), z = RNE(-lo / s) in exact arithmetic."""
+    x = np.array([3.0, -1.5, 0.25, 2.0] + [0.0] * 60, np.float32)
+    c, s, z = quant.int4_quantize_groups(x[None], bits=2)
+    s_want = exact_round(exact_round(Fraction(3) + Fraction(3, 2), 24, -126) / 3, 24, -126)
+    assert Fraction(float(s[0])) == exact_round(s_want, 11, -14)
+    z_want = max(0, min(3, _rhe(exact_round(Fraction(3, 2) / Fraction(float(s[0])), 24, -126))))
+    assert float(z[0]) == z_want == 1
+    assert list(c[0][:4]) == [3, 0, 1, 2]
+
+
+def test_int2_grid_exact_round_trip():
+    rng = np.random.default_rng(37)
+    for e in (-2, 0, 3):
+        for z0 in (0, 1, 3):
+            k = rng.integers(0, 4, 64)
+            k[0], k[1] = 0, 3
+            x = ((k - z0) * 2.0 ** -e).astype(np.float32)
+            c, s, z = quant.int4_quantize_groups(x[None], bits=2)
+            assert float(s[0]) == 2.0 ** -e and float(z[0]) == z0
+            np.testing.assert_array_equal(c[0], k)
+        m0 = -1.25
+        x = (m0 + k * 2.0 ** -e).astype(np.float32)
+        c, s, m = quant.int4_quantize_groups_float_zero(x[None], bits=2)
+        assert float(s[0]) == 2.0 ** -e and float(m[0]) == m0
+        np.testing.assert_array_equal(c[0], k)
+
+
+def test_crumb_packing():
+    c = np.array([1, 2, 3, 0, 3, 3, 0, 1], np.uint8)
+    p = quant.pack_codes(c, 2)
+    np.testing.assert_array_equal(p, [0b00111001, 0b01001111])
+    np.testing.assert_array_equal(quant.unpack_codes(p, 2), c)
+    np.testing.assert_array_equal(quant.pack_codes(c, 4), quant.pack_nibbles(c))
