@@ -50,6 +50,10 @@ WORKLOADS = {
               "128-token bf16 residual",
     "c4-fzp": "70B-shaped KIVI INT4 layer as c4, float zero points (group minimum), "
               "128-token bf16 residual",
+    "c4-int2": "70B-shaped 2-bit KIVI layer as c4 (codes 0..3, four per byte), "
+               "128-token bf16 residual",
+    "c4-int2-tok": "70B-shaped 2-bit layer as c4, keys and values both per token, "
+                   "128-token bf16 residual",
 }
 
 
@@ -288,7 +292,7 @@ def oracle_inputs(w, units):
 
 
 def unit_bytes(w, b):
-    from quantized_paged_kv_02_b200 import roofline
+    from quantized_paged_kv_02_b200 import inputs, roofline
     s = w.spec
     g = s.num_q_heads // s.num_kv_heads
     return (roofline.decode_bytes(s.cache_dtype, s.scale_mode, g, 1, s.head_dim, s.block_size,
@@ -409,7 +413,7 @@ def main_ours(args):
     import torch.distributed as dist
     from quantized_paged_kv_02_b200 import build
     build.build()
-    from quantized_paged_kv_02_b200 import kvq, roofline
+    from quantized_paged_kv_02_b200 import inputs, kvq, roofline
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)

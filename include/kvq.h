@@ -35,7 +35,8 @@
  *
  *  pages : [NB][H][record] bytes.  One record holds everything decode reads for one
  *          (block, kv head), contiguous, so a single copy moves it:
- *            row_bytes   = D * bits / 8            (bits: 16 BF16/FP16, 8 INT8/FP8, 4 INT4)
+ *            row_bytes   = D * bits / 8            (bits: 16 BF16/FP16, 8 INT8/FP8, 4 INT4,
+ *                                                    2 INT2)
  *            K codes     at offset 0              : [bs][row_bytes]
  *            V codes     at offset bs*row_bytes   : [bs][row_bytes]
  *            scales      at offset 2*bs*row_bytes (off_s):
@@ -53,18 +54,21 @@
  *                               V (scale, zero point) [bs][D/64][2] (keys grouped like
  *                               values: [P-prod] "Key 和 Value 的分布不一定相同", the
  *                               Transformers integration quantizes both per token)
- *                               The three INT4 modes have records of the same size.
+ *                               The three INT4 modes have records of the same size; INT2
+ *                               caches take the same three modes and parameter layouts.
  *              other modes    : nothing
  *            record      = off_s + scale bytes, rounded up to a multiple of 128 bytes
  *                          (e.g. INT8, bs 16, D 128: 2048 + 2048 + 128 = 4224 bytes)
  *          INT4 codes pack two per byte: element 2i in the low nibble of byte i, element
- *          2i+1 in the high nibble.  Padding bytes at the end of a record are never written.
+ *          2i+1 in the high nibble.  INT2 codes pack four per byte: element 4i+e in bits
+ *          [2e, 2e+2) of byte i.  Padding bytes at the end of a record are never written.
+ *          (INT4, D 128: 4096 + 4096 + 1024 = 9216 bytes; INT2: 2048 + 2048 + 1024 = 5120.)
  *  k_scales, v_scales : static scales only - PER_HEAD: float32 [H] ([P-prod] "vLLM：从 FP8 KV
  *          Cache 开始试点": per-attention-head); PER_TENSOR: float32 [1]; PER_CHANNEL: float32
  *          [H][D], one scale per kv head and channel ([P-vLLM] "KV Cache量化策略：INT8与FP8
  *          精度对比与选择": INT8 per-tensor or per-channel; [P-prod] "量化不是简单截断精度":
  *          scales per tensor, head, channel, token or group).  Unused otherwise.
- *  residual : INT4 only.  act_dtype [max_seqs][2][H][residual_cap][D]: the newest tokens of
+ *  residual : INT4 and INT2 only.  act_dtype [max_seqs][2][H][residual_cap][D]: the newest tokens of
  *          each sequence kept unquantized ([P-prod] "Key 和 Value 的分布不一定相同": a
  *          fixed-size higher-precision residual of recent K/V).  Index 0 of the second
  *          dimension is K, 1 is V.  Position p of a sequence lives in ring row
@@ -96,6 +100,8 @@
  *  INT4 PER_TOKEN ([P-prod] "Transformers：适合实验和小规模验证": 4 bits, groups of 64,
  *        residual of 128): the KIVI quantizer, every group one token over 64 channels, for
  *        keys as for values.
+ *  INT2 ([P-prod] "KV Cache 的基本内存模型": 2-bit, 0.25 byte per value; "误区二：INT4 或
+ *        2-bit 一定比 FP8 更划算"): the three INT4 modes with 3 in place of 15 (codes 0..3).
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -122,7 +128,8 @@ typedef enum {
   KVQ_DTYPE_FP32 = 2,        /* output only */
   KVQ_DTYPE_INT8 = 3,
   KVQ_DTYPE_FP8_E4M3 = 4,
-  KVQ_DTYPE_INT4 = 5
+  KVQ_DTYPE_INT4 = 5,
+  KVQ_DTYPE_INT2 = 6
 } kvq_dtype;
 
 typedef enum {
@@ -149,17 +156,17 @@ enum {
 /*
  * Cache descriptor.  Plain data: it owns nothing and may be copied freely.
  *   cache_dtype   BF16 / FP16 (unquantized, element type must equal act_dtype),
- *                 INT8, FP8_E4M3 or INT4.
+ *                 INT8, FP8_E4M3, INT4 or INT2.
  *   act_dtype     BF16 or FP16: element type of new K/V rows, of q and of the INT4
  *                 residual ring.
  *   scale_mode    NONE for BF16/FP16; PER_TOKEN_HEAD, PER_HEAD, PER_TENSOR or
  *                 PER_CHANNEL for INT8 and FP8; KIVI, KIVI_FLOAT_ZERO or INT4_PER_TOKEN
- *                 for INT4.  PER_CHANNEL decodes on
+ *                 for INT4 and INT2.  PER_CHANNEL decodes on
  *                 the tensor-core path only (block_size 16, head_dim 128).
- *   block_size    tokens per block: 1..1024 for dense caches; INT4 requires
+ *   block_size    tokens per block: 1..1024 for dense caches; INT4 / INT2 require
  *                 block_size == group_size == 64.
  *   head_dim      64 or 128.
- *   group_size, residual_len, residual_cap, max_seqs: INT4 only (64, r, cap, seqs);
+ *   group_size, residual_len, residual_cap, max_seqs: INT4 / INT2 only (64, r, cap, seqs);
  *                 residual_cap >= residual_len + group_size.  Ignored otherwise.
  *   fault         optional device int32[2] fault record (NULL: faults are skipped
  *                 silently).  fault[0] += entries skipped; fault[1] |= KVQ_FAULT_* bits.
@@ -206,12 +213,12 @@ kvq_status kvq_cache_layout(const kvq_cache_desc* cache, size_t* record_bytes,
  * kvq_write - quantize new K/V rows into the cache ("quantize on write").
  *   k_new, v_new  act_dtype [num_tokens][H][D], device.
  *   slot_mapping  int32 [num_tokens], device: destination slot of each row, or -1.
- *   seq_ids, positions  int32 [num_tokens], device, INT4 only (NULL otherwise): a row
+ *   seq_ids, positions  int32 [num_tokens], device, INT4 / INT2 only (NULL otherwise): a row
  *                 with slot -1 and positions[t] >= 0 is copied unquantized into ring row
  *                 positions[t] % residual_cap of sequence seq_ids[t].
  *   Dense caches: row t goes to slot slot_mapping[t]; slot -1 skips the row.  K and V
  *   are quantized separately, each per (token, kv head) for dynamic modes.
- *   INT4 caches: rows are taken in groups of 64 (rows 64u .. 64u+63).  A group whose
+ *   INT4 / INT2 caches: rows are taken in groups of 64 (rows 64u .. 64u+63).  A group whose
  *   first slot is >= 0 must map, in order, onto one whole block (slots b*64 .. b*64+63);
  *   it is quantized as one key group per channel and 64 value groups per channel group.
  *   A group whose first slot is -1 holds ring rows or skipped rows only.  A trailing
@@ -225,7 +232,7 @@ kvq_status kvq_write(const kvq_cache_desc* cache, const void* k_new, const void*
                      const int32_t* positions, cudaStream_t stream);
 
 /*
- * kvq_flush_ring - INT4: move whole groups of the residual ring into pages.
+ * kvq_flush_ring - INT4 / INT2: move whole groups of the residual ring into pages.
  *   For each entry i < n: ring rows of sequence seq_ids[i] at positions
  *   [positions[i], positions[i] + 64) (ring row p % residual_cap) are quantized into block
  *   block_ids[i] of every kv head, with exactly the codes, scales and zero points kvq_write
@@ -239,7 +246,7 @@ kvq_status kvq_write(const kvq_cache_desc* cache, const void* k_new, const void*
  *   unquantized; once more than residual_len + 64 are there, the oldest 64 become one key
  *   group (one block) and are quantized, which this call does from the ring itself, so the
  *   caller need not keep its own copy of those rows.
- *   INT4 caches only (others: KVQ_ERR_UNSUPPORTED).
+ *   INT4 and INT2 caches only (others: KVQ_ERR_UNSUPPORTED).
  */
 kvq_status kvq_flush_ring(const kvq_cache_desc* cache, const int32_t* seq_ids,
                           const int32_t* positions, const int32_t* block_ids, int n,
@@ -261,7 +268,7 @@ kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
  *                 in token order; entries past ceil(len/bs) are not read.
  *   context_lens  int32 [batch], device: tokens to attend to (the current token
  *                 included); 0 gives an all-zero output row.
- *   seq_ids       INT4 only, int32 [batch] device or NULL: ring sequence of each batch
+ *   seq_ids       INT4 / INT2 only, int32 [batch] device or NULL: ring sequence of each batch
  *                 entry (NULL: entry b uses ring sequence b).
  *   max_context   host upper bound of context_lens, used to plan the split.
  *   softmax_scale 0 selects 1/sqrt(D) ([P-mem] §6 Q1 writes softmax(q k^T / sqrt(d))).

@@ -14,6 +14,7 @@ int code_bits(int cd) {
     case KVQ_DTYPE_INT8:
     case KVQ_DTYPE_FP8_E4M3: return 8;
     case KVQ_DTYPE_INT4: return 4;
+    case KVQ_DTYPE_INT2: return 2;
   }
   return 0;
 }
@@ -52,6 +53,7 @@ static kvq_status validate_geometry(const kvq_cache_desc* c, Geometry* g) {
         return KVQ_ERR_INVALID_ARG;
       break;
     case KVQ_DTYPE_INT4:
+    case KVQ_DTYPE_INT2:
       if (c->scale_mode != KVQ_SCALE_KIVI && c->scale_mode != KVQ_SCALE_KIVI_FLOAT_ZERO &&
           c->scale_mode != KVQ_SCALE_INT4_PER_TOKEN)
         return KVQ_ERR_INVALID_ARG;
@@ -65,9 +67,9 @@ static kvq_status validate_geometry(const kvq_cache_desc* c, Geometry* g) {
   g->off_s = 2 * g->bs * g->row_bytes;
   g->scale_bytes = 0;
   if (g->scale_mode == KVQ_SCALE_PER_TOKEN_HEAD) g->scale_bytes = 8 * g->bs;
-  // INT4: K (scale, zero) per channel [2][D] or per token [bs][D/64][2], then V per token
-  // [bs][D/64][2], all float16; with bs = 64 both K forms take 4 * D bytes
-  if (g->cache_dtype == KVQ_DTYPE_INT4) g->scale_bytes = 4 * g->D + g->bs * (g->D / 64) * 4;
+  // INT4 / INT2: K (scale, zero) per channel [2][D] or per token [bs][D/64][2], then V per
+  // token [bs][D/64][2], all float16; with bs = 64 both K forms take 4 * D bytes
+  if (low_bit(g->cache_dtype)) g->scale_bytes = 4 * g->D + g->bs * (g->D / 64) * 4;
   g->record = (g->off_s + g->scale_bytes + 127) / 128 * 128;
   return KVQ_OK;
 }
@@ -81,7 +83,7 @@ kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g) {
     if (c->k_scales == nullptr || c->v_scales == nullptr) return KVQ_ERR_INVALID_ARG;
     if (!aligned16(c->k_scales) || !aligned16(c->v_scales)) return KVQ_ERR_INVALID_ARG;
   }
-  if (c->cache_dtype == KVQ_DTYPE_INT4 && (c->residual == nullptr || !aligned16(c->residual)))
+  if (low_bit(c->cache_dtype) && (c->residual == nullptr || !aligned16(c->residual)))
     return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
@@ -174,7 +176,7 @@ kvq_status kvq_cache_layout(const kvq_cache_desc* c, size_t* record_bytes, size_
   if (g.scale_mode == KVQ_SCALE_PER_HEAD) ss = static_cast<size_t>(g.H) * 4;
   if (g.scale_mode == KVQ_SCALE_PER_TENSOR) ss = 4;
   if (g.scale_mode == KVQ_SCALE_PER_CHANNEL) ss = static_cast<size_t>(g.H) * g.D * 4;
-  if (g.cache_dtype == KVQ_DTYPE_INT4)
+  if (low_bit(g.cache_dtype))
     rb = static_cast<size_t>(g.max_seqs) * 2 * g.H * g.residual_cap * g.D * 2;
   if (record_bytes) *record_bytes = static_cast<size_t>(g.record);
   if (pages_bytes) *pages_bytes = static_cast<size_t>(g.NB) * g.H * g.record;
@@ -193,7 +195,7 @@ kvq_status kvq_write(const kvq_cache_desc* c, const void* k_new, const void* v_n
   if (num_tokens == 0) return KVQ_OK;
   if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
-  if (g.cache_dtype == KVQ_DTYPE_INT4)
+  if (low_bit(g.cache_dtype))
     return from_cuda(launch_write_int4(*c, g, k_new, v_new, num_tokens, slot_mapping, seq_ids,
                                        positions, stream));
   return from_cuda(launch_write_dense(*c, g, k_new, v_new, num_tokens, slot_mapping, stream));
@@ -304,7 +306,7 @@ kvq_status kvq_flush_ring(const kvq_cache_desc* c, const int32_t* seq_ids, const
   Geometry g;
   kvq_status st = validate_desc(c, &g);
   if (st != KVQ_OK) return st;
-  if (g.cache_dtype != KVQ_DTYPE_INT4) return KVQ_ERR_UNSUPPORTED;
+  if (!low_bit(g.cache_dtype)) return KVQ_ERR_UNSUPPORTED;
   if (n < 0) return KVQ_ERR_INVALID_ARG;
   if (n == 0) return KVQ_OK;
   if (seq_ids == nullptr || positions == nullptr || block_ids == nullptr) return KVQ_ERR_INVALID_ARG;

@@ -243,7 +243,7 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
   }
   p->g_tile = (p->g % 2 == 0) ? 2 : 1;
   const long units = static_cast<long>(batch) * g.H * (p->g / p->g_tile);
-  const int gran = g.cache_dtype == KVQ_DTYPE_INT4 ? 64 : g.bs;
+  const int gran = low_bit(g.cache_dtype) ? 64 : g.bs;
   // aim for about 8 resident CTAs per SM, without splits shorter than 256 tokens
   const long target = 8L * kNumSMs;
   long S = units > 0 ? (target + units - 1) / units : 1;
@@ -327,7 +327,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.plan.kernel == 1) {
     e = launch_dependent(segment_reduce_kernel, dim3((a.batch * a.Hq + 7) / 8), dim3(256), 0, s, p);
   } else if (p.splits > 1) {
-    split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, g.cache_dtype == KVQ_DTYPE_INT4);
+    split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, low_bit(g.cache_dtype));
     e = cudaGetLastError();
   }
   return e;

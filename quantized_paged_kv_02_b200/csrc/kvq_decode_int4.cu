@@ -51,24 +51,34 @@ constexpr int kC = 4;                     // consumer warps
 constexpr int kT = 32 * (kC + 1);
 constexpr int kD = 128;
 constexpr int kBS = 64;
-constexpr int kRowB = kD / 2;             // 64 bytes of codes per token
-constexpr int kOffV = kBS * kRowB;        // 4096
-constexpr int kOffKs = 2 * kBS * kRowB;   // 8192: K scale [128] fp16
-constexpr int kOffKz = kOffKs + 2 * kD;   // 8448: K zero point [128] fp16
-constexpr int kOffVsz = kOffKs + 4 * kD;  // 8704: V (scale, zero) [64][2][2] fp16
-constexpr int kRec = kOffVsz + kBS * 2 * 4;   // 9216
-constexpr int kRecRows = kRec / 128;      // 72
-constexpr int kStage = kRec;              // already a multiple of 1024
 // Consumers take blocks round-robin, so every round of a stage must go to the same warp
 // (a warp waiting for round r of a stage whose round r-1 belonged to another warp, not yet
 // landed, would see the parity of round r-2 as complete): a multiple of kC stages.
 constexpr int kStages = 8;
 static_assert(kStages % kC == 0, "ring depth is a multiple of the consumers");
-constexpr int kTiles = kStages * kStage;
-constexpr int kBytes = 1024 + kTiles + kStages * 16 + kStages * 4;
 constexpr float kRescale4 = 8.f;
-static_assert(kStage % 1024 == 0, "stages start on the swizzle period");
-static_assert(kC * 8 * (kD + 2) * 4 <= kTiles, "merge buffer");
+
+// Record of one (block, kv head) for BITS-bit codes (4, or 2), head_dim 128, 64 tokens:
+// K codes, V codes, then the float16 parameters (K scale [128] and zero [128], or K (scale,
+// zero) [64][2][2] per token; V (scale, zero) [64][2][2]).
+template <int BITS>
+struct Rec {
+  static constexpr int kRowB = kD * BITS / 8;          // bytes of codes per token: 64 or 32
+  static constexpr int kOffV = kBS * kRowB;            // V codes: 4096 or 2048
+  static constexpr int kOffKs = 2 * kBS * kRowB;       // K parameters: 8192 or 4096
+  static constexpr int kOffKz = kOffKs + 2 * kD;       // K zero points (per channel)
+  static constexpr int kOffVsz = kOffKs + 4 * kD;      // V (scale, zero) per token
+  static constexpr int kRec = kOffVsz + kBS * 2 * 4;   // 9216 or 5120
+  static constexpr int kRecRows = kRec / 128;          // TMA box height: 72 or 40
+  static constexpr int kStage = kRec;                  // a multiple of 1024
+  static constexpr int kTile = 16 * kRowB;             // 16 tokens of codes: 1024 or 512 bytes
+  static constexpr int kTiles = kStages * kStage;
+  static constexpr int kBytes = 1024 + kTiles + kStages * 16 + kStages * 4;
+  static constexpr int PW = 16 / BITS;                 // codes in each 16-bit half of a word
+  static constexpr uint32_t kMask = BITS == 4 ? 0x000F000Fu : 0x00030003u;
+  static_assert(kStage % 1024 == 0, "stages start on the swizzle period");
+  static_assert(kC * 8 * (kD + 2) * 4 <= kTiles, "merge buffer");
+};
 
 __device__ __forceinline__ int swzb4(int off) {
   return (off & ~127) + ((((off >> 4) & 7) ^ ((off >> 7) & 7)) << 4) + (off & 15);
@@ -85,24 +95,32 @@ __device__ __forceinline__ int2 sz_offsets(int base, int mt, int r) {
   return make_int2(b0 + v, b0 + (v ^ 64));
 }
 
-// (nibble s, nibble s+4) of w as the fp16 bit patterns of (code_s, code_s+4) * 2^-24: a
-// 4-bit code placed in the mantissa of a zero exponent is an exact fp16 subnormal, so the
-// tensor cores see c * 2^-24 with no conversion instruction
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int s) { return (w >> (4 * s)) & 0x000F000Fu; }
+// (code s, code s + 16/BITS) of w -- the codes at the same place in its two 16-bit halves
+// -- as the fp16 bit patterns of code * 2^-24: a 4- or 2-bit code placed in the mantissa of
+// a zero exponent is an exact fp16 subnormal, so the tensor cores see c * 2^-24 with no
+// conversion instruction
+template <int BITS>
+__device__ __forceinline__ uint32_t code_pair(uint32_t w, int s) {
+  return (w >> (BITS * s)) & Rec<BITS>::kMask;
+}
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// INT4 forms of the kernel
+// Forms of the kernel (each for 4- and 2-bit codes)
 constexpr int kKivi = 0;        // keys per channel, integer zero points
 constexpr int kKiviMin = 1;     // keys per channel, the group minimum as a float zero point
 constexpr int kPerToken = 2;    // keys per token like values, integer zero points
 
-template <int MODE>
+template <int MODE, int BITS>
 __global__ void __launch_bounds__(kT, 2)
 decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   constexpr bool kFz = MODE == kKiviMin;
   constexpr bool kTok = MODE == kPerToken;
+  using R = Rec<BITS>;
+  constexpr int kRowB = R::kRowB, kOffV = R::kOffV, kOffKs = R::kOffKs, kOffKz = R::kOffKz;
+  constexpr int kOffVsz = R::kOffVsz, kRec = R::kRec, kRecRows = R::kRecRows;
+  constexpr int kStage = R::kStage, kTiles = R::kTiles, PW = R::PW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* tiles = smem;
@@ -229,9 +247,9 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       float part[2] = {0.f, 0.f};
 #pragma unroll
       for (int kc = 0; kc < 8; ++kc) {
-        const int e0 = 8 * (kc >> 1) + 2 * (kc & 1);
-        qt[kc][0] = pack_f16x2(qv[e0], qv[e0 + 4]);
-        qt[kc][1] = pack_f16x2(qv[e0 + 1], qv[e0 + 5]);
+        const int e0 = 2 * PW * (kc / (PW / 2)) + 2 * (kc % (PW / 2));
+        qt[kc][0] = pack_f16x2(qv[e0], qv[e0 + PW]);
+        qt[kc][1] = pack_f16x2(qv[e0 + 1], qv[e0 + PW + 1]);
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qt[kc][0]));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qt[kc][1]));
         part[kc >> 2] += (f0.x + f0.y) + (f1.x + f1.y);     // what the MMAs multiply
@@ -247,26 +265,30 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 
     float vlim = 0.f, vinv = 0.f;
     // Swizzled offsets of this lane's key and value code words in tile 0 of a stage.  A
-    // tile (16 tokens of 64 bytes) is one 1024-byte swizzle period, so tile mt reads at
-    // the same offsets plus 1024 * mt: the address arithmetic is done once, not per tile.
+    // 4-bit tile (16 tokens of 64 bytes) is one 1024-byte swizzle period, so tile mt reads
+    // at the same offsets plus 1024 * mt; a 2-bit tile is half a period, so odd tiles also
+    // flip the chunk index's top bit (offset bit 6).  The address arithmetic is done once.
+    // Keys: 32 channels per lane, [32j, 32j+32); per token, [16j, 16j+16) of each group.
     int ko[4];
     if constexpr (kTok) {
-      ko[0] = swzb4(kRowB * r + 8 * j);
-      ko[1] = swzb4(kRowB * r + 32 + 8 * j);
-      ko[2] = swzb4(kRowB * (r + 8) + 8 * j);
-      ko[3] = swzb4(kRowB * (r + 8) + 32 + 8 * j);
+      ko[0] = swzb4(kRowB * r + 2 * BITS * j);
+      ko[1] = swzb4(kRowB * r + kRowB / 2 + 2 * BITS * j);
+      ko[2] = swzb4(kRowB * (r + 8) + 2 * BITS * j);
+      ko[3] = swzb4(kRowB * (r + 8) + kRowB / 2 + 2 * BITS * j);
     } else {
-      ko[0] = swzb4(kRowB * r + 16 * j);
-      ko[1] = swzb4(kRowB * (r + 8) + 16 * j);
+      ko[0] = swzb4(kRowB * r + 4 * BITS * j);
+      ko[1] = swzb4(kRowB * (r + 8) + 4 * BITS * j);
       ko[2] = ko[3] = 0;
     }
-    int vo[4][2];                  // tokens 2j, 2j+1, 2j+8, 2j+9; channel group G; byte 4r
+    // values: tokens 2j, 2j+1, 2j+8, 2j+9; channels 64G + 8r .. 64G + 8r + 7
+    int vo[4][2];
     {
       const int dts[4] = {0, 1, 8, 9};
 #pragma unroll
       for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int G = 0; G < 2; ++G) vo[t][G] = kOffV + swzb4(kRowB * (2 * j + dts[t]) + 32 * G + 4 * r);
+        for (int G = 0; G < 2; ++G)
+          vo[t][G] = kOffV + swzb4(kRowB * (2 * j + dts[t]) + (kRowB / 2) * G + BITS * r);
     }
     for (int i = warp; i < npages; i += kC) {
       const int s = i % kStages;
@@ -304,8 +326,8 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         }
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
-          const int e0 = 8 * (kc >> 1) + 2 * (kc & 1);
-          const float a0 = qs[e0], a1 = qs[e0 + 4], c0 = qs[e0 + 1], c1 = qs[e0 + 5];
+          const int e0 = 2 * PW * (kc / (PW / 2)) + 2 * (kc % (PW / 2));
+          const float a0 = qs[e0], a1 = qs[e0 + PW], c0 = qs[e0 + 1], c1 = qs[e0 + PW + 1];
           const uint32_t h0 = pack_f16x2(a0, a1), h1 = pack_f16x2(c0, c1);
           const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
           const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
@@ -332,22 +354,33 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll 1
       for (int mt = 0; mt < kBS / 16; ++mt) {
         // rows r / r + 8 of the tile: tokens tr0 = 16mt + r and tr1 = tr0 + 8
-        const uint8_t* sm = st + 1024 * mt;                  // this tile's swizzle period
+        const uint8_t* sm = st + R::kTile * mt;
+        const int flip = BITS == 2 ? 64 * (mt & 1) : 0;      // 2-bit: odd half-periods
         // ------------------------------------------------ S^T = (C - Zk) Q'^T
         float s00, s01, s10, s11;
         if constexpr (kTok) {
-          // codes of channels [16j, 16j+16) and [64+16j, 64+16j+16): group 0 in words 0-1
-          const uint2 k0a = *reinterpret_cast<const uint2*>(sm + ko[0]);
-          const uint2 k0b = *reinterpret_cast<const uint2*>(sm + ko[1]);
-          const uint2 k1a = *reinterpret_cast<const uint2*>(sm + ko[2]);
-          const uint2 k1b = *reinterpret_cast<const uint2*>(sm + ko[3]);
-          const uint32_t w0[4] = {k0a.x, k0a.y, k0b.x, k0b.y}, w1[4] = {k1a.x, k1a.y, k1b.x, k1b.y};
+          // codes of channels [16j, 16j+16) and [64+16j, 64+16j+16): the first BITS/2 words
+          // hold group 0, so k-steps 0-3 stay in group 0 and 4-7 in group 1
+          uint32_t w0[BITS], w1[BITS];
+          if constexpr (BITS == 4) {
+            const uint2 k0a = *reinterpret_cast<const uint2*>(sm + ko[0]);
+            const uint2 k0b = *reinterpret_cast<const uint2*>(sm + ko[1]);
+            const uint2 k1a = *reinterpret_cast<const uint2*>(sm + ko[2]);
+            const uint2 k1b = *reinterpret_cast<const uint2*>(sm + ko[3]);
+            w0[0] = k0a.x; w0[1] = k0a.y; w0[2] = k0b.x; w0[3] = k0b.y;
+            w1[0] = k1a.x; w1[1] = k1a.y; w1[2] = k1b.x; w1[3] = k1b.y;
+          } else {
+            w0[0] = *reinterpret_cast<const uint32_t*>(sm + (ko[0] ^ flip));
+            w0[1] = *reinterpret_cast<const uint32_t*>(sm + (ko[1] ^ flip));
+            w1[0] = *reinterpret_cast<const uint32_t*>(sm + (ko[2] ^ flip));
+            w1[1] = *reinterpret_cast<const uint32_t*>(sm + (ko[3] ^ flip));
+          }
           float sg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
           for (int kc = 0; kc < 8; ++kc) {
-            const int w = kc >> 1, sp = 2 * (kc & 1);
-            const uint32_t a[4] = {nib_pair(w0[w], sp), nib_pair(w1[w], sp), nib_pair(w0[w], sp + 1),
-                                   nib_pair(w1[w], sp + 1)};
+            const int w = kc / (PW / 2), sp = 2 * (kc % (PW / 2));
+            const uint32_t a[4] = {code_pair<BITS>(w0[w], sp), code_pair<BITS>(w1[w], sp),
+                                   code_pair<BITS>(w0[w], sp + 1), code_pair<BITS>(w1[w], sp + 1)};
             mma_f16(sg[kc >> 2], a, qt[kc]);
           }
           // (scale, zero) of tokens tr0 / tr1, groups 0 and 1: fp16 at kOffKs + 8t + 4G
@@ -367,15 +400,25 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           s11 = (a10.x * fmaf(sg[0][3], 16777216.f, -a10.y * qg[0][1]) +
                  a11.x * fmaf(sg[1][3], 16777216.f, -a11.y * qg[1][1])) * qscale;
         } else {
-          const uint4 k0 = lds128(sm + ko[0]);
-          const uint4 k1 = lds128(sm + ko[1]);
-          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+          // codes of channels [32j, 32j+32): BITS words per row
+          uint32_t w0[BITS], w1[BITS];
+          if constexpr (BITS == 4) {
+            const uint4 k0 = lds128(sm + ko[0]);
+            const uint4 k1 = lds128(sm + ko[1]);
+            w0[0] = k0.x; w0[1] = k0.y; w0[2] = k0.z; w0[3] = k0.w;
+            w1[0] = k1.x; w1[1] = k1.y; w1[2] = k1.z; w1[3] = k1.w;
+          } else {
+            const uint2 k0 = *reinterpret_cast<const uint2*>(sm + (ko[0] ^ flip));
+            const uint2 k1 = *reinterpret_cast<const uint2*>(sm + (ko[1] ^ flip));
+            w0[0] = k0.x; w0[1] = k0.y;
+            w1[0] = k1.x; w1[1] = k1.y;
+          }
           float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int kc = 0; kc < 8; ++kc) {
-            const int w = kc >> 1, sp = 2 * (kc & 1);
-            const uint32_t a[4] = {nib_pair(w0[w], sp), nib_pair(w1[w], sp), nib_pair(w0[w], sp + 1),
-                                   nib_pair(w1[w], sp + 1)};
+            const int w = kc / (PW / 2), sp = 2 * (kc % (PW / 2));
+            const uint32_t a[4] = {code_pair<BITS>(w0[w], sp), code_pair<BITS>(w1[w], sp),
+                                   code_pair<BITS>(w0[w], sp + 1), code_pair<BITS>(w1[w], sp + 1)};
             mma_f16(sa, a, qh[kc]);
             mma_f16(sb, a, ql[kc]);
           }
@@ -469,22 +512,42 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           pbl[G][1] = movmatrix_trans(e1);
         }
         // ------------------------------------------------ O^T += (C - Zv)^T P'^T
-        // tile md: group G = md/4, byte k = md%4 of the word holding channels
-        // 64G + 8r .. +7 of a token; rows r / r+8 <-> d = 64G + 8r + 2k / +1
+        // tile md: channel group G = md/4; rows r / r+8 <-> d = 64G + 8r + 2(md%4) / +1.
+        // 4-bit: byte md%4 of the word holding channels 64G + 8r .. +7 of a token, its low /
+        // high nibble.  2-bit: those channels are 2 bytes; byte (md%4)/2, crumbs 2(md%2), +1.
+        // A byte permute puts the byte of tokens (2j, 2j+1) -- and of (2j+8, 2j+9) -- into the
+        // two 16-bit halves of a register, where a shift and a mask leave the codes.
         uint32_t vwd[4][2];
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int G = 0; G < 2; ++G)
-            vwd[t][G] = *reinterpret_cast<const uint32_t*>(sm + vo[t][G]);
+          for (int G = 0; G < 2; ++G) {
+            if constexpr (BITS == 4)
+              vwd[t][G] = *reinterpret_cast<const uint32_t*>(sm + vo[t][G]);
+            else
+              vwd[t][G] = *reinterpret_cast<const uint16_t*>(sm + (vo[t][G] ^ flip));
+          }
 #pragma unroll
         for (int md = 0; md < 8; ++md) {
-          const int G = md >> 2, k = md & 3;
-          const uint32_t sel = static_cast<uint32_t>(k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12));
-          const uint32_t Y = prmt(vwd[0][G], vwd[1][G], sel);   // bytes (ta_k, ta_k, tb_k, tb_k)
-          const uint32_t Z = prmt(vwd[2][G], vwd[3][G], sel);
-          const uint32_t a[4] = {Y & 0x000F000Fu, (Y >> 4) & 0x000F000Fu, Z & 0x000F000Fu,
-                                 (Z >> 4) & 0x000F000Fu};
+          const int G = md >> 2;
+          uint32_t Y, Z;
+          int sh;
+          if constexpr (BITS == 4) {
+            const int k = md & 3;
+            const uint32_t sel = static_cast<uint32_t>(k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12));
+            Y = prmt(vwd[0][G], vwd[1][G], sel);   // bytes (ta_k, ta_k, tb_k, tb_k)
+            Z = prmt(vwd[2][G], vwd[3][G], sel);
+            sh = 0;
+          } else {
+            const int k = (md >> 1) & 1;
+            const uint32_t sel = static_cast<uint32_t>(k | (k << 4) | ((2 + k) << 8) | ((2 + k) << 12));
+            Y = prmt(vwd[0][G] | (vwd[1][G] << 16), 0u, sel);
+            Z = prmt(vwd[2][G] | (vwd[3][G] << 16), 0u, sel);
+            sh = 4 * (md & 1);
+          }
+          constexpr uint32_t m4 = R::kMask;
+          const uint32_t a[4] = {(Y >> sh) & m4, (Y >> (sh + BITS)) & m4, (Z >> sh) & m4,
+                                 (Z >> (sh + BITS)) & m4};
           mma_f16(o[md], a, pbh[G]);
           mma_f16(o[md], a, pbl[G]);
         }
@@ -553,21 +616,26 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 }  // namespace
 
 bool int4_mma_supported(const Geometry& g, int group) {
-  return g.cache_dtype == KVQ_DTYPE_INT4 && g.D == kD && g.bs == kBS && g.record == kRec &&
-         group >= 3 && group <= 8;
+  const bool rec = (g.cache_dtype == KVQ_DTYPE_INT4 && g.record == Rec<4>::kRec) ||
+                   (g.cache_dtype == KVQ_DTYPE_INT2 && g.record == Rec<2>::kRec);
+  return rec && g.D == kD && g.bs == kBS && group >= 3 && group <= 8;
 }
 
-cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+namespace {
+
+template <int BITS>
+cudaError_t launch_bits(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  using R = Rec<BITS>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     // two CTAs per SM (registers): both rings need the maximum shared-memory carveout
-    const void* fns[3] = {reinterpret_cast<const void*>(decode_int4_kernel<kKivi>),
-                          reinterpret_cast<const void*>(decode_int4_kernel<kKiviMin>),
-                          reinterpret_cast<const void*>(decode_int4_kernel<kPerToken>)};
+    const void* fns[3] = {reinterpret_cast<const void*>(decode_int4_kernel<kKivi, BITS>),
+                          reinterpret_cast<const void*>(decode_int4_kernel<kKiviMin, BITS>),
+                          reinterpret_cast<const void*>(decode_int4_kernel<kPerToken, BITS>)};
     for (const void* f : fns) {
       if (attr_err == cudaSuccess)
-        attr_err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+        attr_err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, R::kBytes);
       if (attr_err == cudaSuccess)
         attr_err = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                         cudaSharedmemCarveoutMaxShared);
@@ -575,17 +643,23 @@ cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaS
   });
   if (attr_err != cudaSuccess) return attr_err;
   CUtensorMap tm;
-  const long rows = static_cast<long>(a.geo.NB) * a.geo.H * kRecRows;
-  if (!make_pages_map(&tm, a.c->pages, rows, kRecRows)) return cudaErrorInvalidValue;
+  const long rows = static_cast<long>(a.geo.NB) * a.geo.H * R::kRecRows;
+  if (!make_pages_map(&tm, a.c->pages, rows, R::kRecRows)) return cudaErrorInvalidValue;
   // page splits only; the ring split is launched separately
   const dim3 grid(p.ring_split, a.geo.H, a.batch);
   switch (a.geo.scale_mode) {
-    case KVQ_SCALE_KIVI: decode_int4_kernel<kKivi><<<grid, kT, kBytes, s>>>(p, tm); break;
-    case KVQ_SCALE_KIVI_FLOAT_ZERO: decode_int4_kernel<kKiviMin><<<grid, kT, kBytes, s>>>(p, tm); break;
-    case KVQ_SCALE_INT4_PER_TOKEN: decode_int4_kernel<kPerToken><<<grid, kT, kBytes, s>>>(p, tm); break;
+    case KVQ_SCALE_KIVI: decode_int4_kernel<kKivi, BITS><<<grid, kT, R::kBytes, s>>>(p, tm); break;
+    case KVQ_SCALE_KIVI_FLOAT_ZERO: decode_int4_kernel<kKiviMin, BITS><<<grid, kT, R::kBytes, s>>>(p, tm); break;
+    case KVQ_SCALE_INT4_PER_TOKEN: decode_int4_kernel<kPerToken, BITS><<<grid, kT, R::kBytes, s>>>(p, tm); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  return a.geo.cache_dtype == KVQ_DTYPE_INT2 ? launch_bits<2>(a, p, s) : launch_bits<4>(a, p, s);
 }
 
 }  // namespace kvq

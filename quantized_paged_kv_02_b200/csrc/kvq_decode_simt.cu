@@ -3,7 +3,7 @@
 // One CTA covers (split, kv head, up to two query heads of its GQA group, sequence).
 // Each warp walks the split's token range in batches; a lane owns a 16-element chunk
 // of the head dimension for one row at a time (16 bytes of INT8/FP8 codes, 8 bytes of
-// packed INT4, 16 bytes of BF16/FP16), so a warp instruction reads whole 128-byte rows.
+// packed INT4, 4 of INT2, 16 bytes of BF16/FP16), so a warp instruction reads whole rows.
 // Scores are reduced over the lanes of a row with shuffles; each lane group runs its
 // own online softmax (running max, running sum, fp32 accumulator) in the log2 domain,
 // and groups, warps and finally splits are merged with log-sum-exp weights.
@@ -30,6 +30,7 @@ template <> struct Chunk<KVQ_DTYPE_FP8_E4M3> { static constexpr int EPL = 16, BY
 template <> struct Chunk<KVQ_DTYPE_BF16> { static constexpr int EPL = 8, BYTES = 16; };
 template <> struct Chunk<KVQ_DTYPE_FP16> { static constexpr int EPL = 8, BYTES = 16; };
 template <> struct Chunk<KVQ_DTYPE_INT4> { static constexpr int EPL = 16, BYTES = 8; };
+template <> struct Chunk<KVQ_DTYPE_INT2> { static constexpr int EPL = 16, BYTES = 4; };
 
 // Load EPL cache elements of one row chunk as floats (codes only; scales applied outside).
 template <int CD>
@@ -53,6 +54,10 @@ __device__ __forceinline__ void load_codes(const uint8_t* p, float* f) {
     unpack8<__nv_bfloat16>(*reinterpret_cast<const uint4*>(p), f);
   } else if constexpr (CD == KVQ_DTYPE_FP16) {
     unpack8<__half>(*reinterpret_cast<const uint4*>(p), f);
+  } else if constexpr (CD == KVQ_DTYPE_INT2) {  // 4 bytes, element 4i+e in bits [2e, 2e+2)
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f[i] = static_cast<float>((u >> (2 * i)) & 3u);
   } else {  // INT4: 8 bytes, element 2i in the low nibble of byte i
     const uint2 u = *reinterpret_cast<const uint2*>(p);
     const uint8_t* c = reinterpret_cast<const uint8_t*>(&u);
@@ -72,7 +77,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
   constexpr int LPR = D / EPL;          // lanes per row
   constexpr int RPI = 32 / LPR;         // rows per warp instruction
   constexpr int U = 4;                  // rows per lane per batch
-  constexpr bool kInt4 = CD == KVQ_DTYPE_INT4;
+  constexpr bool kInt4 = CD == KVQ_DTYPE_INT4 || CD == KVQ_DTYPE_INT2;   // group codes + ring
   constexpr int ROWB = D * CB / EPL;    // bytes per cache row
 
   // ring-only launch (INT4 blocks on tensor cores): this grid covers [qb, n) from the ring
@@ -281,6 +286,7 @@ cudaError_t launch_d(int cd, const DecodeParams& p, dim3 grid, cudaStream_t s) {
     case KVQ_DTYPE_BF16: return launch_cd<TA, KVQ_DTYPE_BF16, D>(p, grid, s);
     case KVQ_DTYPE_FP16: return launch_cd<TA, KVQ_DTYPE_FP16, D>(p, grid, s);
     case KVQ_DTYPE_INT4: return launch_cd<TA, KVQ_DTYPE_INT4, D>(p, grid, s);
+    case KVQ_DTYPE_INT2: return launch_cd<TA, KVQ_DTYPE_INT2, D>(p, grid, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -138,6 +138,11 @@ struct Geometry {
 kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g);
 int code_bits(int cache_dtype);
 
+// INT4 and INT2 caches: 64-token groups, zero points, a residual ring of recent tokens
+__host__ __device__ inline bool low_bit(int cache_dtype) {
+  return cache_dtype == KVQ_DTYPE_INT4 || cache_dtype == KVQ_DTYPE_INT2;
+}
+
 // Launchers implemented in the .cu files; return a cudaError_t from the launch.
 cudaError_t launch_write_dense(const kvq_cache_desc& c, const Geometry& g, const void* k,
                                const void* v, int T, const int32_t* slots, cudaStream_t s);

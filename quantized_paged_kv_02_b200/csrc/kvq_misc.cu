@@ -58,9 +58,14 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
         x = cv * sv;
         break;
       }
-      default: {  // INT4
-        const uint8_t byte = codes[t * p.row_bytes + d / 2];
-        const int c = (d & 1) ? (byte >> 4) : (byte & 0xF);
+      default: {  // INT4 (two codes per byte) or INT2 (four)
+        int c;
+        if (p.cd == KVQ_DTYPE_INT4) {
+          const uint8_t byte = codes[t * p.row_bytes + d / 2];
+          c = (d & 1) ? (byte >> 4) : (byte & 0xF);
+        } else {
+          c = (codes[t * p.row_bytes + d / 4] >> (2 * (d & 3))) & 3;
+        }
         // K per channel [2][D] (KIVI forms) or per token [bs][D/64][2]; V per token
         const __half* sz = reinterpret_cast<const __half*>(rec + p.off_s);
         float s, z;

@@ -90,46 +90,49 @@ struct Int4Group {
   __half off16;   // what the record stores beside the scale: z or m
 };
 
-// lo/hi are the group's min and max.  Integer zero point: the range is widened to include
-// 0 and z = clamp(round(-lo / s), 0, 15).  Float zero point: the offset is the group
-// minimum m = fp16(lo) itself.
+// lo/hi are the group's min and max; Q = 15 (INT4) or 3 (INT2) is the largest code.
+// Integer zero point: the range is widened to include 0 and z = clamp(round(-lo / s), 0, Q).
+// Float zero point: the offset is the group minimum m = fp16(lo) itself.
+template <int Q>
 __device__ __forceinline__ Int4Group int4_group(float lo, float hi, bool float_zero) {
   if (!float_zero) {
     lo = fminf(lo, 0.f);
     hi = fmaxf(hi, 0.f);
   }
   Int4Group g;
-  g.s16 = __float2half_rn(div_rn(__fsub_rn(hi, lo), 15.f));
+  g.s16 = __float2half_rn(div_rn(__fsub_rn(hi, lo), static_cast<float>(Q)));
   g.sw = __half2float(g.s16);
   if (float_zero) {
     g.off16 = __float2half_rn(lo);
     g.off = __half2float(g.off16);
   } else {
-    const int z = (g.sw == 0.f) ? 0 : max(0, min(15, __float2int_rn(div_rn(-lo, g.sw))));
+    const int z = (g.sw == 0.f) ? 0 : max(0, min(Q, __float2int_rn(div_rn(-lo, g.sw))));
     g.off = static_cast<float>(z);
     g.off16 = __int2half_rn(z);
   }
   return g;
 }
 
-// integer zero point: clamp(round(x / s) + z, 0, 15); float: clamp(round((x - m) / s), 0, 15)
+// integer zero point: clamp(round(x / s) + z, 0, Q); float: clamp(round((x - m) / s), 0, Q)
+template <int Q>
 __device__ __forceinline__ int int4_code(float x, const Int4Group& g, bool float_zero) {
   if (g.sw == 0.f) return 0;
   const int r = float_zero ? __float2int_rn(div_rn(__fsub_rn(x, g.off), g.sw))
                            : __float2int_rn(div_rn(x, g.sw)) + static_cast<int>(g.off);
-  return max(0, min(15, r));
+  return max(0, min(Q, r));
 }
 
-// Quantize the 64 rows of one (block, kv head) into its page record, codes packed two per
-// byte.  Values: one group per token per 64 channels.  Keys: one group per channel over the
+// Quantize the 64 rows of one (block, kv head) into its page record, BITS-bit codes (4 or
+// 2) packed 8 / BITS per byte.  Values: one group per token per 64 channels.  Keys: one group per channel over the
 // 64 tokens (KIVI, [P-prod] "Key 和 Value 的分布不一定相同"), or per token like the values
 // (INT4_PER_TOKEN, the Transformers integration's choice in the same section).
 // row(kv, t) points at row t (act dtype, D values) of K (kv 0) or V (kv 1).  All 128
 // threads of the CTA take part.
-template <typename TA, int D, typename RowFn>
+template <typename TA, int D, int BITS, typename RowFn>
 __device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_s, int mode,
                                     float (*xs)[D + 1], uint8_t (*cs)[D]) {
   constexpr int G = 64;
+  constexpr int Q = (1 << BITS) - 1;           // largest code
   const int tid = threadIdx.x;
   const bool fz = mode == KVQ_SCALE_KIVI_FLOAT_ZERO;
   const bool k_per_token = mode == KVQ_SCALE_INT4_PER_TOKEN;
@@ -151,8 +154,8 @@ __device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_
       for (int d = tid; d < D; d += blockDim.x) {
         float lo = xs[0][d], hi = xs[0][d];
         for (int t = 1; t < G; ++t) { lo = fminf(lo, xs[t][d]); hi = fmaxf(hi, xs[t][d]); }
-        const Int4Group g = int4_group(lo, hi, fz);
-        for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code(xs[t][d], g, fz));
+        const Int4Group g = int4_group<Q>(lo, hi, fz);
+        for (int t = 0; t < G; ++t) cs[t][d] = static_cast<uint8_t>(int4_code<Q>(xs[t][d], g, fz));
         k_sz[d] = g.s16;
         k_sz[D + d] = g.off16;
       }
@@ -163,37 +166,39 @@ __device__ void quantize_int4_block(RowFn row, uint8_t* rec, int off_v, int off_
         const int t = i / (D / 64), gi = i % (D / 64);
         float lo = xs[t][gi * 64], hi = lo;
         for (int j = 1; j < 64; ++j) { lo = fminf(lo, xs[t][gi * 64 + j]); hi = fmaxf(hi, xs[t][gi * 64 + j]); }
-        const Int4Group g = int4_group(lo, hi, fz);
+        const Int4Group g = int4_group<Q>(lo, hi, fz);
         for (int j = 0; j < 64; ++j)
-          cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code(xs[t][gi * 64 + j], g, fz));
+          cs[t][gi * 64 + j] = static_cast<uint8_t>(int4_code<Q>(xs[t][gi * 64 + j], g, fz));
         __half* sz = sz_base + (t * (D / 64) + gi) * 2;
         sz[0] = g.s16;
         sz[1] = g.off16;
       }
     }
     __syncthreads();
-    // pack two codes per byte (element 2i low nibble) and store 16 bytes at a time
+    // pack (element k of a run of 32 / BITS in bits [BITS k, BITS k + BITS) of a 32-bit
+    // word, i.e. element 2i in the low nibble of byte i, or 4i+e in bits [2e, 2e+2)) and
+    // store 16 bytes at a time
+    constexpr int PER_WORD = 32 / BITS;          // codes per 32-bit word
+    constexpr int PER_16B = 4 * PER_WORD;        // codes per 16-byte store
     uint8_t* dst = rec + (kv ? off_v : 0);
-    for (int i = tid; i < G * D / 32; i += blockDim.x) {
-      const int t = i / (D / 32), c = i % (D / 32);
+    for (int i = tid; i < G * D / PER_16B; i += blockDim.x) {
+      const int t = i / (D / PER_16B), c = i % (D / PER_16B);
       uint32_t w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t x = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int e = c * 32 + j * 8 + b * 2;
-          x |= static_cast<uint32_t>(cs[t][e] | (cs[t][e + 1] << 4)) << (8 * b);
-        }
+        for (int k = 0; k < PER_WORD; ++k)
+          x |= static_cast<uint32_t>(cs[t][c * PER_16B + j * PER_WORD + k]) << (BITS * k);
         w[j] = x;
       }
-      *reinterpret_cast<uint4*>(dst + t * (D / 2) + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(dst + t * (D * BITS / 8) + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     __syncthreads();
   }
 }
 
-template <typename TA, int D>
+template <typename TA, int D, int BITS>
 __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
   griddep_launch_dependents();   // a decode launched after this one may start its set-up
   constexpr int G = 64;
@@ -220,7 +225,7 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
     auto row = [&](int kv, int t) {
       return static_cast<const TA*>(kv ? p.v : p.k) + (static_cast<long>(r0 + t) * p.H + h) * D;
     };
-    quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, p.mode, xs, cs);
+    quantize_int4_block<TA, D, BITS>(row, rec, p.off_v, p.off_s, p.mode, xs, cs);
   } else {
     // residual rows: copied unquantized into ring row positions[t] % cap
     for (int i = tid; i < nr * 2 * (D / 8); i += blockDim.x) {
@@ -285,7 +290,7 @@ struct Int4FlushParams {
 
 // grid (entries, H): quantize ring rows [p0, p0 + 64) of one sequence and kv head into the
 // block's record, exactly as kvq_write stores those rows with slots blk*64 .. blk*64+63.
-template <typename TA, int D>
+template <typename TA, int D, int BITS>
 __global__ void __launch_bounds__(128) flush_ring_kernel(Int4FlushParams p) {
   __shared__ float xs[64][D + 1];
   __shared__ __align__(16) uint8_t cs[64][D];
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(128) flush_ring_kernel(Int4FlushParams p) {
     return static_cast<const TA*>(p.residual) +
            ((static_cast<long>(sid * 2 + kv) * p.H + h) * p.cap + (p0 + t) % p.cap) * D;
   };
-  quantize_int4_block<TA, D>(row, rec, p.off_v, p.off_s, p.mode, xs, cs);
+  quantize_int4_block<TA, D, BITS>(row, rec, p.off_v, p.off_s, p.mode, xs, cs);
 }
 
 }  // namespace
@@ -316,12 +321,17 @@ cudaError_t launch_flush_ring(const kvq_cache_desc& c, const Geometry& g, const 
                     g.NB, g.H, g.residual_cap, g.max_seqs, g.record, g.off_v, g.off_s,
                     g.scale_mode, c.fault};
   const dim3 grid(n, g.H);
-  if (g.act_dtype == KVQ_DTYPE_BF16) {
-    if (g.D == 128) flush_ring_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
-    else flush_ring_kernel<__nv_bfloat16, 64><<<grid, 128, 0, s>>>(p);
-  } else {
-    if (g.D == 128) flush_ring_kernel<__half, 128><<<grid, 128, 0, s>>>(p);
-    else flush_ring_kernel<__half, 64><<<grid, 128, 0, s>>>(p);
+  const int sel = (g.cache_dtype == KVQ_DTYPE_INT4 ? 4 : 0) + (g.act_dtype == KVQ_DTYPE_BF16 ? 2 : 0) +
+                  (g.D == 128 ? 1 : 0);
+  switch (sel) {
+    case 7: flush_ring_kernel<__nv_bfloat16, 128, 4><<<grid, 128, 0, s>>>(p); break;
+    case 6: flush_ring_kernel<__nv_bfloat16, 64, 4><<<grid, 128, 0, s>>>(p); break;
+    case 5: flush_ring_kernel<__half, 128, 4><<<grid, 128, 0, s>>>(p); break;
+    case 4: flush_ring_kernel<__half, 64, 4><<<grid, 128, 0, s>>>(p); break;
+    case 3: flush_ring_kernel<__nv_bfloat16, 128, 2><<<grid, 128, 0, s>>>(p); break;
+    case 2: flush_ring_kernel<__nv_bfloat16, 64, 2><<<grid, 128, 0, s>>>(p); break;
+    case 1: flush_ring_kernel<__half, 128, 2><<<grid, 128, 0, s>>>(p); break;
+    default: flush_ring_kernel<__half, 64, 2><<<grid, 128, 0, s>>>(p); break;
   }
   return cudaGetLastError();
 }
@@ -345,12 +355,17 @@ cudaError_t launch_write_int4(const kvq_cache_desc& c, const Geometry& g, const 
                     g.scale_mode, c.fault};
   const dim3 grid((T + 63) / 64, g.H);
   if (grid.x == 0) return cudaSuccess;
-  if (g.act_dtype == KVQ_DTYPE_BF16) {
-    if (g.D == 128) write_int4_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
-    else write_int4_kernel<__nv_bfloat16, 64><<<grid, 128, 0, s>>>(p);
-  } else {
-    if (g.D == 128) write_int4_kernel<__half, 128><<<grid, 128, 0, s>>>(p);
-    else write_int4_kernel<__half, 64><<<grid, 128, 0, s>>>(p);
+  const int sel = (g.cache_dtype == KVQ_DTYPE_INT4 ? 4 : 0) + (g.act_dtype == KVQ_DTYPE_BF16 ? 2 : 0) +
+                  (g.D == 128 ? 1 : 0);
+  switch (sel) {
+    case 7: write_int4_kernel<__nv_bfloat16, 128, 4><<<grid, 128, 0, s>>>(p); break;
+    case 6: write_int4_kernel<__nv_bfloat16, 64, 4><<<grid, 128, 0, s>>>(p); break;
+    case 5: write_int4_kernel<__half, 128, 4><<<grid, 128, 0, s>>>(p); break;
+    case 4: write_int4_kernel<__half, 64, 4><<<grid, 128, 0, s>>>(p); break;
+    case 3: write_int4_kernel<__nv_bfloat16, 128, 2><<<grid, 128, 0, s>>>(p); break;
+    case 2: write_int4_kernel<__nv_bfloat16, 64, 2><<<grid, 128, 0, s>>>(p); break;
+    case 1: write_int4_kernel<__half, 128, 2><<<grid, 128, 0, s>>>(p); break;
+    default: write_int4_kernel<__half, 64, 2><<<grid, 128, 0, s>>>(p); break;
   }
   return cudaGetLastError();
 }

@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkvq.so")
 
-DTYPE = {"bf16": 0, "fp16": 1, "fp32": 2, "int8": 3, "fp8": 4, "int4": 5}
+DTYPE = {"bf16": 0, "fp16": 1, "fp32": 2, "int8": 3, "fp8": 4, "int4": 5, "int2": 6}
 SCALE = {"none": 0, "per_token_head": 1, "per_head": 2, "per_tensor": 3, "kivi": 4,
          "per_channel": 5, "int4_per_token": 6, "kivi_float_zero": 7}
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "KVQ_ERR_CUDA",

@@ -57,3 +57,12 @@ def test_throughput_is_whole_job():
     assert bench.throughput(1e9, 1, 1.0) == pytest.approx(1000.0)
     assert bench.throughput(1e9, 4, 2.0) == pytest.approx(2000.0)   # 4 ranks, each 1 GB in 2 ms
     assert bench.max_over_ranks([1.0, 2.0], 1, None) == [1.0, 2.0]
+
+
+def test_per_unit_bytes_for_every_workload():
+    """The oracle sample's byte count (bench.unit_bytes) works for every bench workload."""
+    import bench
+    from quantized_paged_kv_02_b200 import inputs
+    for name in bench.WORKLOADS:
+        w = inputs.make(name, small=True)
+        assert bench.unit_bytes(w, 0) > 0

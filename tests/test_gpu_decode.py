@@ -17,7 +17,8 @@ from tests import helpers
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
-SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c5", "c5-fp8", "c5-bf16", "c5-int8-pc"]
+SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok", "c4-int2-fzp", "c5",
+         "c5-fp8", "c5-bf16", "c5-int8-pc"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -61,7 +62,7 @@ def test_decode_matches_oracle(name):
     assert gc.read_fault() == (0, 0)
 
 
-@pytest.mark.parametrize("name", ["c2", "c4", "c4-tok", "c4-fzp", "c5-fp8"])
+@pytest.mark.parametrize("name", ["c2", "c4", "c4-tok", "c4-fzp", "c4-int2", "c5-fp8"])
 def test_split_count_does_not_change_result(name):
     w = _workload(name)
     static = helpers.oracle_static_scales(w)
@@ -74,7 +75,9 @@ def test_split_count_does_not_change_result(name):
         tab = torch.zeros((w.spec.batch, max(pad, w.block_tables.shape[1])), dtype=torch.int32)
         tab[:, :w.block_tables.shape[1]] = w.block_tables.cpu()
         b = _decode(gc, w, max_context=mc, tables=tab).cpu()
-        assert (a - b).abs().max().item() <= 1e-5
+        # only the fp32 summation order changes; the zero-point sums of the group codes
+        # cancel against the products (a few bits, more with 2-bit steps)
+        assert (a - b).abs().max().item() <= 3e-5
 
 
 def test_edge_lengths_zero_one_and_ragged():
@@ -191,12 +194,13 @@ def test_per_channel_needs_the_tensor_core_path():
         _decode(gc, w)
 
 
+@pytest.mark.parametrize("cd", ["int4", "int2"])
 @pytest.mark.parametrize("mode", ["kivi", "int4_per_token", "kivi_float_zero"])
 @pytest.mark.parametrize("hq,d", [(4, 128), (16, 64)])
-def test_int4_cuda_core_path(mode, hq, d):
-    """INT4 caches the tensor-core kernel does not take (GQA group 2, or head_dim 64) run on
-    the CUDA-core kernel, for every INT4 form."""
-    spec = inputs.Spec("int4-simt", "int4", "bf16", mode, 2, hq, 2, d, 64, lens=[485, 200],
+def test_int4_cuda_core_path(cd, mode, hq, d):
+    """INT4 / INT2 caches the tensor-core kernel does not take (GQA group 2, or head_dim 64)
+    run on the CUDA-core kernel, for every form."""
+    spec = inputs.Spec("int4-simt", cd, "bf16", mode, 2, hq, 2, d, 64, lens=[485, 200],
                        outliers="k", slack_blocks=3, seed=5)
     w = inputs.from_spec(spec)
     oc = helpers.oracle_cache(w)

@@ -18,9 +18,11 @@ def _built():
     helpers.ensure_built()
 
 
-@pytest.mark.parametrize("mode", ["kivi", "int4_per_token", "kivi_float_zero"])
-def test_flush_then_append_then_decode(mode):
-    spec = inputs.Spec("flush", "int4", "bf16", mode, 2, 16, 2, 128, 64, lens=[485, 300],
+@pytest.mark.parametrize("cd,mode", [("int4", "kivi"), ("int4", "int4_per_token"),
+                                     ("int4", "kivi_float_zero"), ("int2", "kivi"),
+                                     ("int2", "int4_per_token")])
+def test_flush_then_append_then_decode(cd, mode):
+    spec = inputs.Spec("flush", cd, "bf16", mode, 2, 16, 2, 128, 64, lens=[485, 300],
                        outliers="k", slack_blocks=3, seed=11)
     w = inputs.from_spec(spec)
     oc = helpers.oracle_cache(w)

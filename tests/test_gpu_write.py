@@ -12,7 +12,8 @@ from tests import helpers
 
 pytestmark = pytest.mark.gpu
 
-SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c5", "c5-fp8", "c5-bf16", "c5-int8-pc"]
+SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok", "c4-int2-fzp", "c5",
+         "c5-fp8", "c5-bf16", "c5-int8-pc"]
 
 
 @pytest.fixture(scope="module", autouse=True)
