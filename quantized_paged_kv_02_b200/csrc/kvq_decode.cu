@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
 // sequence), finds the CTAs whose ranges meet its unit's pages, and takes the partial of
 // every consumer warp that saw at least one of those pages.  Lane k describes candidate
 // k (CTA c_first + k / kSegWarps, warp k % kSegWarps); the partial rows are then read
-// four at a time so their loads overlap.
+// sixteen at a time so their loads overlap.
 __global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
   constexpr int C = kMmaCtas;
   griddep_wait();                      // the partials of the decode kernel
@@ -146,23 +146,24 @@ __global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
     const float w = (slot >= 0 && mk != -INFINITY) ? exp2f(mk - M) : 0.f;
     L = fmaf(lk, w, L);
     const int n = min(32, K - k0);
-    for (int i0 = 0; i0 < n; i0 += 4) {
-      float wi[4];
-      int si[4];
-      float4 v[4];
+    constexpr int kRows = 16;          // partial rows in flight per lane
+    for (int i0 = 0; i0 < n; i0 += kRows) {
+      float wi[kRows];
+      int si[kRows];
+      float4 v[kRows];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
+      for (int t = 0; t < kRows; ++t) {
         const int i = min(i0 + t, 31);
         wi[t] = __shfl_sync(0xffffffffu, w, i);
         si[t] = __shfl_sync(0xffffffffu, slot, i);
         if (i0 + t >= n) wi[t] = 0.f;
       }
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
+      for (int t = 0; t < kRows; ++t)
         v[t] = (has_d && wi[t] != 0.f) ? *reinterpret_cast<const float4*>(o + static_cast<long>(si[t]) * p.D)
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
+      for (int t = 0; t < kRows; ++t) {
         acc.x = fmaf(v[t].x, wi[t], acc.x);
         acc.y = fmaf(v[t].y, wi[t], acc.y);
         acc.z = fmaf(v[t].z, wi[t], acc.z);
