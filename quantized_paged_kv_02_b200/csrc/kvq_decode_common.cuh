@@ -40,6 +40,7 @@ struct DecodeParams {
   // prefill (kvq_prefill_attention): q is [Tq][Hq][D]; the queries of sequence b are rows
   // q_start[b] .. q_start[b+1]-1, the newest tokens of the sequence
   const int32_t* q_start;
+  int max_q_len;             // prefill: host bound on a sequence's query count
 };
 
 struct SeqInfo {

@@ -124,8 +124,10 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     pf_q0 = blockIdx.x * kConsumers;
     pf_L = p.q_start[pf_b + 1] - p.q_start[pf_b];
     pf_n = seq_info(p, pf_b, false, blockIdx.x == 0 && pf_kvh == 0 && threadIdx.x == 0).n;
-    // more queries than positions, or than the grid covers (max_q_len): rejected
-    if (pf_L > pf_n || pf_L > static_cast<int>(gridDim.x) * kConsumers || pf_L < 0) {
+    // more queries than positions, or than the host bound max_q_len (which sizes the
+    // grid): rejected
+    if (pf_L > pf_n || pf_L > p.max_q_len || pf_L > static_cast<int>(gridDim.x) * kConsumers ||
+        pf_L < 0) {
       if (blockIdx.x == 0 && pf_kvh == 0 && threadIdx.x == 0) record_fault(p.fault, KVQ_FAULT_CONTEXT);
       pf_L = 0;
     }

@@ -112,3 +112,20 @@ def test_prefill_full_size_sampled_queries():
             err = np.abs(got[qs[b] + i] - want).max()
             assert err <= TOL, (b, i, err)
     assert gc.read_fault() == (0, 0)
+
+
+def test_more_queries_than_max_q_len_are_rejected():
+    """max_q_len is the contract's bound even where the grid covers more queries (a CTA
+    takes four): a sequence of 4 queries with max_q_len 3 is skipped and counted."""
+    w = inputs.make("c5", small=True)
+    gc = helpers.gpu_cache(w)
+    L = [4, 2, 3]
+    q, qs = _queries(w, L, 7)
+    out = torch.full((int(qs[-1]), w.spec.num_q_heads, w.spec.head_dim), 7.0, device="cuda")
+    kvq.kvq_prefill_attention(gc.desc, q.cuda(), qs.cuda(), 3, w.block_tables.cuda(),
+                              w.context_lens.cuda(), w.max_context, out)
+    torch.cuda.synchronize()
+    cnt, bits = gc.read_fault()
+    assert cnt >= 1 and (bits & 4)
+    assert torch.all(out[qs[0]:qs[1]] == 7.0)
+    assert torch.all(out[qs[1]:qs[3]] != 7.0)
