@@ -72,6 +72,17 @@ def test_layout_sizes(lib):
     assert kvq.kvq_cache_layout(_desc(kvq, block_size=5))[0] == 1408
     with pytest.raises(kvq.KVQError):
         kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=4, block_size=16))
+    # the per-token and float-zero-point INT4 forms keep the record size
+    for mode in (6, 7):
+        assert kvq.kvq_cache_layout(_desc(kvq, cache_dtype=5, scale_mode=mode, block_size=64))[0] == 9216
+    # INT2, bs 64: 2048 + 2048 + 1024, every INT4 form; the ring as INT4
+    for mode in (4, 6, 7):
+        rec, pg, ss, r = kvq.kvq_cache_layout(_desc(kvq, cache_dtype=6, scale_mode=mode, block_size=64))
+        assert (rec, pg, ss, r) == (5120, 16 * 4 * 5120, 0, 2 * 2 * 4 * 192 * 128 * 2)
+    # low-bit caches take only the group forms; dense caches not those
+    for cd, mode in ((6, 1), (5, 2), (3, 4), (4, 6), (3, 7)):
+        with pytest.raises(kvq.KVQError):
+            kvq.kvq_cache_layout(_desc(kvq, cache_dtype=cd, scale_mode=mode, block_size=64))
 
 
 def test_workspace_plan_is_deterministic(lib):
