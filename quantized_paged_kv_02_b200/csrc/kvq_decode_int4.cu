@@ -1,5 +1,5 @@
-// Paged split-K decode attention over INT4 pages on tensor cores (head_dim 128, block 64,
-// GQA groups of 3..8 query heads), for the three INT4 forms of include/kvq.h.
+// Paged split-K decode attention over INT4 and INT2 pages on tensor cores (head_dim 128,
+// block 64, GQA groups of 3..8 query heads), for the three group forms of include/kvq.h.
 //
 // KIVI keeps keys per channel and values per token ([P-prod] "Key 和 Value 的分布不一定
 // 相同"), each as X_q = round(X/scale) + zero_point ([P-prod] "量化不是简单截断精度"):
@@ -32,10 +32,15 @@
 // q is then the same for every block: its fp16 fragments (one MMA per k-step, q being an
 // activation value scaled by a power of two) and per-group sums are formed once.
 //
-// Structure as the dense tensor-core kernel: warp 4 stages one 9 KiB record per block
-// (64 tokens of K and V codes plus all scales and zero points) with one 128-byte-swizzled
-// TMA copy into an mbarrier ring; warps 0-3 consume blocks round-robin (16 tokens per
-// MMA tile, four tiles per block).
+// 2-bit codes ([P-prod] "KV Cache 的基本内存模型": 0.25 byte per value) take the same path:
+// a 2-bit code under a zero exponent is the subnormal c * 2^-24 too; a k-step pairs codes
+// s and s + 8 of one 32-bit word instead of s and s + 4, and for P V each token's 16-bit
+// slice of a channel group is spread over a register's halves by the same byte permute.
+//
+// Structure as the dense tensor-core kernel: warp 4 stages one record per block (64
+// tokens of K and V codes plus all scales and zero points: 9 KiB for INT4, 5 KiB for INT2)
+// with one 128-byte-swizzled TMA copy into an mbarrier ring; warps 0-3 consume blocks
+// round-robin (16 tokens per MMA tile, four tiles per block).
 #include <cudaTypedefs.h>
 
 #include <climits>
