@@ -66,3 +66,14 @@ def test_per_unit_bytes_for_every_workload():
     for name in bench.WORKLOADS:
         w = inputs.make(name, small=True)
         assert bench.unit_bytes(w, 0) > 0
+
+
+def test_decode_launch_count_follows_the_dispatch():
+    import bench
+    from quantized_paged_kv_02_b200 import inputs
+    assert bench.decode_launches(inputs._spec("c5", False), 1) == 2      # decode + merge
+    assert bench.decode_launches(inputs._spec("c2", False), 1) == 2      # MHA: same kernel
+    assert bench.decode_launches(inputs._spec("c4", False), 1) == 3      # blocks, ring, reduce
+    assert bench.decode_launches(inputs._spec("c4-int2", False), 1) == 3
+    assert bench.decode_launches(inputs._spec("c1", False), 0) == 1      # head_dim 64, one split
+    assert bench.decode_launches(inputs._spec("c1", False), 1) == 2
