@@ -209,3 +209,19 @@ def test_int4_cuda_core_path(cd, mode, hq, d):
     got = _decode(gc, w).cpu().numpy().astype(np.float64)
     assert np.abs(got - _oracle(oc, w)).max() <= TOL
     assert gc.read_fault() == (0, 0)
+
+
+@pytest.mark.parametrize("cd", ["int4", "int2"])
+@pytest.mark.parametrize("mode", ["kivi", "int4_per_token", "kivi_float_zero"])
+@pytest.mark.parametrize("hq", [6, 10])
+def test_int4_tensor_core_path_partial_groups(cd, mode, hq):
+    """GQA groups of 3 and 5 query heads on the INT4 / INT2 tensor-core kernel (N = 8 heads
+    per tile, the rest masked), against the oracle."""
+    spec = inputs.Spec("int4-g", cd, "bf16", mode, 2, hq, 2, 128, 64, lens=[485, 330],
+                       outliers="k", slack_blocks=3, seed=9)
+    w = inputs.from_spec(spec)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    got = _decode(gc, w).cpu().numpy().astype(np.float64)
+    assert np.abs(got - _oracle(oc, w)).max() <= TOL
+    assert gc.read_fault() == (0, 0)
