@@ -276,10 +276,14 @@ kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
  *   workspace     device scratch of at least kvq_decode_workspace_size() bytes (may be
  *                 NULL when that size is 0).  Its contents need no initialisation.
  *   For each (b, hq): o = sum_p softmax_p(scale * q . k_p) v_p over p < context_lens[b],
- *   where k_p, v_p are the dequantized cache rows; for INT4, positions p < Qb come from
- *   blocks and the rest from the residual ring, Qb = 64*floor(max(len-residual_len,0)/64).
+ *   where k_p, v_p are the dequantized cache rows; for INT4 / INT2, positions p < Qb come
+ *   from blocks and the rest from the residual ring, Qb = 64*floor(max(len-residual_len,0)/64).
  *   Dequantization happens inside the kernel ([P-vLLM] "PagedAttention与KV Cache量化协同
  *   工作原理"); long contexts are split across CTAs and merged by a log-sum-exp reduce.
+ *   Kernels: head_dim 128 with block_size 16 and 1..8 query heads per kv head runs on the
+ *   tensor-core kernel (dense caches); INT4 / INT2 with head_dim 128 and 3..8 query heads per
+ *   kv head on the low-bit tensor-core kernel; everything else on the CUDA-core kernel.
+ *   PER_CHANNEL caches need the tensor-core kernel (KVQ_ERR_UNSUPPORTED otherwise).
  */
 kvq_status kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int batch,
                                 int num_q_heads, const int32_t* block_tables,
