@@ -291,22 +291,6 @@ def oracle_inputs(w, units):
     return rows
 
 
-def decode_launches(spec, ws_bytes):
-    """Kernels one kvq_decode_attention call launches for this geometry (the dispatch in
-    csrc/kvq_decode.cu): the page-balanced tensor-core kernel and its merge for dense caches
-    with head_dim 128 and block 16; for INT4 / INT2 with head_dim 128 and GQA groups of 3..8,
-    the block kernel, the ring kernel and the split reduce; otherwise the CUDA-core kernel
-    and, with a workspace (more than one split), the split reduce."""
-    from quantized_paged_kv_02_b200 import inputs
-    g = spec.num_q_heads // spec.num_kv_heads
-    if inputs.low_bit(spec.cache_dtype):
-        if spec.head_dim == 128 and 3 <= g <= 8:
-            return 3
-    elif spec.head_dim == 128 and spec.block_size == 16 and 1 <= g <= 8:
-        return 2
-    return 1 + (1 if ws_bytes else 0)
-
-
 def unit_bytes(w, b):
     from quantized_paged_kv_02_b200 import inputs, roofline
     s = w.spec
@@ -568,7 +552,7 @@ def main_ours(args):
 
     peak, peak_kind = hbm_peak()
     achieved = dec_bytes / (dms * 1e-3) / 1e9
-    launches_per_step = 1 + decode_launches(s, ws_n)
+    launches_per_step = 1 + cache.decode_plan(B, s.num_q_heads, max_ctx)[1]
     result = {
         "metric": METRIC,
         "value": round(throughput(step_bytes, world, ms), 2),

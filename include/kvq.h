@@ -261,6 +261,23 @@ kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
                                      int num_q_heads, int max_context, size_t* bytes);
 
 /*
+ * kvq_decode_plan - which kernels kvq_decode_attention launches for these arguments (host
+ * only: no device access, no launch; the pages give no counterpart, it reports this
+ * library's dispatch).  Any output pointer may be NULL.
+ *   kernel_out    0: the CUDA-core split kernel; 1: the page-balanced tensor-core kernel
+ *                 (dense caches); 2: the low-bit (INT4 / INT2) tensor-core block kernel
+ *                 plus the CUDA-core kernel for the residual ring.
+ *   launches_out  kernels one call launches, the merge included (1: 2; 2: 3; 0: 1, or 2
+ *                 with more than one split; 0 when batch is 0).
+ *   splits_out    token splits of kernels 0 and 2 (the ring counted as one); for kernel 1,
+ *                 its CTA count (the page ranges).
+ *   Errors as kvq_decode_workspace_size.
+ */
+kvq_status kvq_decode_plan(const kvq_cache_desc* cache, int batch, int num_q_heads,
+                           int max_context, int* kernel_out, int* launches_out,
+                           int* splits_out);
+
+/*
  * kvq_decode_attention - one query token per sequence attends to its cached context.
  *   q             act_dtype [batch][num_q_heads][D], device.  num_q_heads must be a
  *                 multiple of H; query head hq reads kv head hq / (num_q_heads / H).

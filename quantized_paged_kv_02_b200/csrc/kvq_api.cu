@@ -201,6 +201,27 @@ kvq_status kvq_write(const kvq_cache_desc* c, const void* k_new, const void* v_n
   return from_cuda(launch_write_dense(*c, g, k_new, v_new, num_tokens, slot_mapping, stream));
 }
 
+kvq_status kvq_decode_plan(const kvq_cache_desc* c, int batch, int num_q_heads, int max_context,
+                           int* kernel_out, int* launches_out, int* splits_out) {
+  if (c == nullptr) return KVQ_ERR_INVALID_ARG;
+  Geometry g;
+  kvq_status st = validate_geometry(c, &g);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || num_q_heads % g.H != 0 || max_context < 0)
+    return KVQ_ERR_INVALID_ARG;
+  DecodePlan p;
+  st = plan_decode(g, batch, num_q_heads, max_context, &p);
+  if (st != KVQ_OK) return st;
+  // the launches of launch_decode: kernel 1 + segment merge; INT4/INT2 blocks + ring kernel +
+  // split reduce; CUDA-core kernel (+ split reduce when it splits)
+  int launches = p.kernel == 1 ? 2 : p.kernel == 2 ? 3 : (p.splits > 1 ? 2 : 1);
+  if (batch == 0) launches = 0;                       // nothing to do: nothing launched
+  if (kernel_out) *kernel_out = p.kernel;
+  if (launches_out) *launches_out = launches;
+  if (splits_out) *splits_out = p.kernel == 1 ? p.ctas : p.splits;
+  return KVQ_OK;
+}
+
 kvq_status kvq_decode_workspace_size(const kvq_cache_desc* c, int batch, int num_q_heads,
                                      int max_context, size_t* bytes) {
   if (c == nullptr || bytes == nullptr) return KVQ_ERR_INVALID_ARG;

@@ -27,7 +27,7 @@ EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
            "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc",
            "kvq_append_decode_attention", "kvq_calibrate_channel_scales", "kvq_flush_ring",
-           "kvq_prefill_attention")
+           "kvq_prefill_attention", "kvq_decode_plan")
 
 
 class CacheDesc(ctypes.Structure):
@@ -62,6 +62,7 @@ def _load():
                                  ctypes.POINTER(Z)]),
         "kvq_write": (I, [D, P, P, I, P, P, P, P]),
         "kvq_decode_workspace_size": (I, [D, I, I, I, ctypes.POINTER(Z)]),
+        "kvq_decode_plan": (I, [D, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
         "kvq_decode_attention": (I, [D, P, I, I, P, I, P, P, I, F, P, ctypes.c_int32, P, Z, P]),
         "kvq_dequant": (I, [D, P, I, P, P]),
         "kvq_calibrate_fp8_scales": (I, [P, I, I, I, ctypes.c_int32, P, P]),
@@ -142,6 +143,14 @@ def kvq_decode_workspace_size(desc, batch, num_q_heads, max_context):
     _check(lib.kvq_decode_workspace_size(ctypes.byref(desc), batch, num_q_heads, max_context,
                                          ctypes.byref(n)), "kvq_decode_workspace_size")
     return n.value
+
+
+def kvq_decode_plan(desc, batch, num_q_heads, max_context):
+    """(kernel, launches per call, splits or CTAs) of kvq_decode_attention for this shape."""
+    k, n, s = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.kvq_decode_plan(ctypes.byref(desc), batch, num_q_heads, max_context,
+                               ctypes.byref(k), ctypes.byref(n), ctypes.byref(s)), "kvq_decode_plan")
+    return k.value, n.value, s.value
 
 
 def kvq_decode_attention(desc, q, block_tables, context_lens, max_context, out, workspace=None,
@@ -286,6 +295,9 @@ class PagedKVCache:
 
     def workspace_size(self, batch, num_q_heads, max_context):
         return kvq_decode_workspace_size(self.desc, batch, num_q_heads, max_context)
+
+    def decode_plan(self, batch, num_q_heads, max_context):
+        return kvq_decode_plan(self.desc, batch, num_q_heads, max_context)
 
     def decode(self, q, block_tables, context_lens, max_context, out=None, out_dtype=torch.float32,
                workspace=None, seq_ids=None, softmax_scale=0.0, stream=None):

@@ -101,6 +101,26 @@ def test_workspace_plan_is_deterministic(lib):
         kvq.kvq_decode_workspace_size(d, 2, 12, 100)              # 12 not a multiple of 8
 
 
+def test_decode_plan_names_the_dispatch(lib):
+    """kvq_decode_plan (host only) reports the kernel and launch count of a decode call."""
+    from quantized_paged_kv_02_b200 import kvq
+    d = _desc(kvq, num_kv_heads=8)
+    assert kvq.kvq_decode_plan(d, 24, 64, 16384) == (1, 2, 3 * 148)       # tensor cores + merge
+    assert kvq.kvq_decode_plan(d, 4, 8, 2048)[:2] == (1, 2)               # MHA too (g = 1)
+    assert kvq.kvq_decode_plan(d, 0, 64, 16384)[1] == 0                  # empty batch
+    lo = dict(cache_dtype=5, scale_mode=4, block_size=64, num_kv_heads=8)
+    k, n, s = kvq.kvq_decode_plan(_desc(kvq, **lo), 16, 64, 32768)
+    assert (k, n) == (2, 3) and s >= 2                                  # blocks, ring, reduce
+    assert kvq.kvq_decode_plan(_desc(kvq, **dict(lo, cache_dtype=6)), 16, 64, 32768)[:2] == (2, 3)
+    assert kvq.kvq_decode_plan(_desc(kvq, **lo), 16, 16, 32768)[0] == 0   # g = 2: CUDA cores
+    # CUDA-core kernel: one split writes the output (one launch), more add the reduce
+    d64 = _desc(kvq, num_kv_heads=8, head_dim=64)
+    assert kvq.kvq_decode_plan(d64, 1, 8, 16)[:2] == (0, 1)
+    assert kvq.kvq_decode_plan(d64, 1, 8, 16384)[:2] == (0, 2)
+    with pytest.raises(kvq.KVQError):
+        kvq.kvq_decode_plan(d, 2, 12, 100)
+
+
 def test_invalid_arguments_rejected_before_launch(lib):
     from quantized_paged_kv_02_b200 import kvq
     L = kvq.lib
