@@ -4,14 +4,21 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5] [--impl ours|reference]
 
 A step is one serving step of one layer: kvq_write of the batch's new K/V rows into the
-quantized paged cache, then kvq_decode_attention over every cached position (split-K
-kernel + reduce).  The cache of the previous positions is resident in HBM; the timed
+quantized paged cache, then kvq_decode_attention over every cached position (split
+decode kernel with its log-sum-exp merge).  The cache of the previous positions is resident in HBM; the timed
 step is bracketed by CUDA events on the launching stream, with a 512 MiB memset before
 every step so no cache byte is served from L2.  Metric: KV GB/s = algorithmic bytes of
 the step / step time; tokens/s = batch / step time.  One JSON line on stdout.
 
+The default run (workload c5, one GPU) also times, at full size and with the same protocol,
+the decode call of the other target configurations ("configs": c2, c3, c4, c4-int2, c5-fp8,
+c5-bf16), the kvq_write of a 4 x 8192-token prefill chunk ("write_prefill") and chunked
+prefill attention ("prefill"), and the float64 CPU oracle on every host core
+("cpu_baseline").
+
 --impl reference times the float64 CPU oracle (the only other implementation of the
-method) on a bounded sample of the same workload; under torchrun only rank 0 runs it.
+method) on every host core, one (sequence, kv head) unit per core per step; under torchrun
+only rank 0 runs it.
 """
 
 import argparse
@@ -40,6 +47,12 @@ WORKLOADS = {
                "block 16, unquantized bf16 cache",
     "c5-int8-pc": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
                   "block 16, INT8 static per-(kv head, channel) scales (256-token warm-up)",
+    "c5-int8-ph": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
+                  "block 16, INT8 static per-kv-head scales (256-token warm-up)",
+    "c5-int8-pt": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
+                  "block 16, INT8 static per-tensor scale (256-token warm-up)",
+    "c5-fp8-pt": "Llama-3-70B-shaped layer: batch 24, 64/8 heads, head_dim 128, context 16384, "
+                 "block 16, FP8 E4M3 static per-tensor scale (256-token warm-up)",
     "c2": "Llama-2-7B-shaped layer: batch 4, 32 heads MHA, head_dim 128, context 2048, block 16, "
           "INT8 per-token-head, 4 outlier channels x10 in K and V",
     "c3": "Llama-3-8B-shaped layer: batch 64, 32/8 heads, head_dim 128, context U[1024, 8192], "
@@ -237,60 +250,6 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_unit_step(w, unit_rows, b, kvh, static):
-    """Set up an oracle cache for one (sequence, kv head) and return a callable that
-    performs the step's work for it: quantize the new row, then attention of its query
-    heads over every cached position.  float64 CPU oracle, single process."""
-    import numpy as np
-    import torch
-    from oracle import attention, cache
-    from quantized_paged_kv_02_b200 import inputs
-    s = w.spec
-    n = int(w.context_lens[b])
-    r0 = int(w.seq_start[b])
-    k = unit_rows["k"][b].astype(np.float64)[:, None, :]      # [n, 1, D]
-    v = unit_rows["v"][b].astype(np.float64)[:, None, :]
-    st = None
-    if static is not None:
-        st = (static[0][kvh:kvh + 1], static[1][kvh:kvh + 1])
-    bs = s.block_size
-    if inputs.low_bit(s.cache_dtype):
-        qb = 64 * (max(n - 128, 0) // 64)
-        nblk = qb // 64
-    else:
-        qb, nblk = n, -(-n // bs)
-    mode = "per_head" if s.scale_mode in ("per_head", "per_tensor") else s.scale_mode
-    oc = cache.PagedCache(s.cache_dtype, s.act_dtype, mode, max(nblk, 1), bs, 1, s.head_dim,
-                          residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
-                          max_seqs=1, static_scales=st)
-    table = np.arange(max(nblk, 1))
-    slots = np.array([p if p < qb else -1 for p in range(n)])
-    pos = np.array([-1 if p < qb else p for p in range(n)])
-    oc.write(k[:n - 1], v[:n - 1], slots[:n - 1], np.zeros(n - 1, np.int64), pos[:n - 1])
-    g = s.num_q_heads // s.num_kv_heads
-    q = unit_rows["q"][b][kvh * g:(kvh + 1) * g].astype(np.float64)[None]
-    del r0, torch
-
-    def step():
-        oc.write(k[n - 1:n], v[n - 1:n], slots[n - 1:n], np.zeros(1, np.int64), pos[n - 1:n])
-        return attention.decode_attention(oc, q, table[None, :], np.array([n]), seq_ids=np.array([0]))
-    return step
-
-
-def oracle_inputs(w, units):
-    """Host copies of the rows the sampled units need (read from the seeded workload)."""
-    import numpy as np
-    import torch
-    rows = {"k": {}, "v": {}, "q": {}}
-    for b, kvh in units:
-        r0, r1 = int(w.seq_start[b]), int(w.seq_start[b + 1])
-        rows["k"][b] = w.k[r0:r1, kvh].to(torch.float32).cpu().numpy()
-        rows["v"][b] = w.v[r0:r1, kvh].to(torch.float32).cpu().numpy()
-        rows["q"][b] = w.q[b].to(torch.float32).cpu().numpy()
-    del np
-    return rows
-
-
 def unit_bytes(w, b):
     from quantized_paged_kv_02_b200 import inputs, roofline
     s = w.spec
@@ -315,27 +274,141 @@ def unit_workload(name):
     return inputs.from_spec(spec, "cpu")
 
 
-def run_oracle_sample(w, static, budget_s=12.0, wall_cap_s=45.0):
-    """Time the oracle on (b, kvh) units, cycling through the batch in order, until about
-    budget_s seconds of timed oracle work (or wall_cap_s of wall time, set-up of each
-    unit's cache included) have passed.  Only the steps count toward the reported rate."""
+def unit_case(name, tmpdir):
+    """The oracle's inputs for one unit of the named workload (seed 0): its rows, query group
+    and static scales saved as NumPy arrays under tmpdir, plus the plain numbers the oracle
+    needs, so a worker process loads them without torch or a GPU.  Static scales come from
+    the oracle's own calibration of the workload's warm-up rows."""
+    import numpy as np
+    from oracle import quant
+    from quantized_paged_kv_02_b200 import inputs
+    w = unit_workload(name)
+    s = w.spec
+    arrays = {"k": w.k[:, 0].float().numpy(), "v": w.v[:, 0].float().numpy(),
+              "q": w.q[0].float().numpy()}
+    if s.scale_mode in ("per_head", "per_tensor", "per_channel"):
+        qmax = 127.0 if s.cache_dtype == "int8" else 448.0
+        cal = quant.channel_calibrate if s.scale_mode == "per_channel" else quant.head_calibrate
+        arrays["sk"] = cal(w.warmup_k.float().numpy(), qmax)
+        arrays["sv"] = cal(w.warmup_v.float().numpy(), qmax)
+    path = os.path.join(tmpdir, "unit_%s.npz" % name)
+    np.savez(path, **arrays)
+    return {"path": path, "cache_dtype": s.cache_dtype, "act_dtype": s.act_dtype,
+            "scale_mode": s.scale_mode, "block_size": s.block_size, "head_dim": s.head_dim,
+            "n": int(w.context_lens[0]), "low_bit": inputs.low_bit(s.cache_dtype),
+            "residual_len": inputs.RESIDUAL_LEN, "residual_cap": inputs.RESIDUAL_CAP,
+            "bytes": unit_bytes(w, 0), "g": s.num_q_heads // s.num_kv_heads}
+
+
+def oracle_unit_step(case):
+    """Set up an oracle cache for one (sequence, kv head) holding all but its newest row and
+    return a callable that performs the step's work for it: quantize the new row, then
+    float64 attention of its query heads over every cached position."""
+    import numpy as np
+    from oracle import attention, cache
+    arr = np.load(case["path"])
+    n, bs = case["n"], case["block_size"]
+    k = arr["k"].astype(np.float64)[:, None, :]      # [n, 1, D]
+    v = arr["v"].astype(np.float64)[:, None, :]
+    st = (arr["sk"], arr["sv"]) if "sk" in arr else None
+    if case["low_bit"]:
+        qb = 64 * (max(n - case["residual_len"], 0) // 64)
+        nblk = qb // 64
+    else:
+        qb, nblk = n, -(-n // bs)
+    mode = case["scale_mode"]
+    if mode == "per_tensor":           # one kv head: its one scale
+        mode, st = "per_head", (st[0][:1], st[1][:1])
+    oc = cache.PagedCache(case["cache_dtype"], case["act_dtype"], mode, max(nblk, 1), bs, 1,
+                          case["head_dim"], residual_len=case["residual_len"],
+                          residual_cap=case["residual_cap"], max_seqs=1, static_scales=st)
+    table = np.arange(max(nblk, 1))
+    slots = np.array([p if p < qb else -1 for p in range(n)])
+    pos = np.array([-1 if p < qb else p for p in range(n)])
+    oc.write(k[:n - 1], v[:n - 1], slots[:n - 1], np.zeros(n - 1, np.int64), pos[:n - 1])
+    q = arr["q"].astype(np.float64)[None]
+
+    def step():
+        oc.write(k[n - 1:n], v[n - 1:n], slots[n - 1:n], np.zeros(1, np.int64), pos[n - 1:n])
+        return attention.decode_attention(oc, q, table[None, :], np.array([n]), seq_ids=np.array([0]))
+    return step
+
+
+def _oracle_worker(case, cmd_q, res_q):
+    """Worker process of the oracle pool: one BLAS/OpenMP thread, one unit cache; runs one
+    unit step per command and reports its start and end (CLOCK_MONOTONIC, shared by all
+    processes of the host)."""
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
     from threadpoolctl import threadpool_limits
-    units = [(b, h) for b in range(w.spec.batch) for h in range(w.spec.num_kv_heads)]
-    done, nbytes, t_total = 0, 0, 0.0
-    t_start = time.perf_counter()
     with threadpool_limits(limits=1):
-        while True:
-            b, kvh = units[done % len(units)]
-            if done and (t_total >= budget_s or time.perf_counter() - t_start >= wall_cap_s):
-                break
-            rows = oracle_inputs(w, [(b, kvh)])
-            step = oracle_unit_step(w, rows, b, kvh, static)
+        step = oracle_unit_step(case)
+        res_q.put(None)
+        while cmd_q.get() is not None:
             t0 = time.perf_counter()
             step()
-            t_total += time.perf_counter() - t0
-            nbytes += unit_bytes(w, b)
-            done += 1
-    return {"units": done, "bytes": nbytes, "seconds": t_total}
+            res_q.put((t0, time.perf_counter()))
+
+
+class OraclePool:
+    """The float64 oracle on every host core: one spawned process per core of
+    os.sched_getaffinity(0) (spawn, so no process is forked from a CUDA context), each holding
+    its own copy of one (sequence, kv head) unit of the workload.  A round is one unit step on
+    every worker at once; its time is from the first start to the last end."""
+    MAX_WORKERS = 256
+
+    def __init__(self, workload, workers=0):
+        import multiprocessing as mp
+        import tempfile
+        self.tmp = tempfile.TemporaryDirectory(prefix="kvq_oracle_")
+        self.case = unit_case(workload, self.tmp.name)
+        self.cores = len(os.sched_getaffinity(0))
+        self.workers = workers or max(1, min(self.cores, self.MAX_WORKERS))
+        ctx = mp.get_context("spawn")
+        self.res = ctx.Queue()
+        self.cmds = [ctx.Queue() for _ in range(self.workers)]
+        self.procs = [ctx.Process(target=_oracle_worker, args=(self.case, c, self.res), daemon=True)
+                      for c in self.cmds]
+        for pr in self.procs:
+            pr.start()
+        for _ in self.procs:
+            self.res.get(timeout=600)
+
+    def round(self):
+        for c in self.cmds:
+            c.put(1)
+        spans = [self.res.get(timeout=600) for _ in self.cmds]
+        return max(t1 for _, t1 in spans) - min(t0 for t0, _ in spans)
+
+    def bytes_per_round(self):
+        return self.workers * self.case["bytes"]
+
+    def close(self):
+        for c in self.cmds:
+            c.put(None)
+        for pr in self.procs:
+            pr.join(timeout=30)
+        self.tmp.cleanup()
+
+
+def run_oracle_sample(workload, budget_s=10.0):
+    """cpu_baseline: rounds of the oracle pool until about budget_s seconds of rounds."""
+    pool = OraclePool(workload)
+    try:
+        pool.round()                               # untimed: first touch of every cache
+        t, rounds = 0.0, 0
+        while t < budget_s:
+            t += pool.round()
+            rounds += 1
+        value = rounds * pool.bytes_per_round() / t / 1e9
+        return {"value": round(value, 6), "unit": "GB/s", "cores": pool.workers, "kind": "oracle",
+                "host_cores": pool.cores,
+                "sample": "%d rounds of one step of a (sequence, kv head) unit (%d cached tokens, "
+                          "%d query heads; quantize the new row + float64 attention) on each of "
+                          "%d worker processes, one per host core, one thread each; %.1f s"
+                          % (rounds, pool.case["n"], pool.case["g"], pool.workers, t)}
+    finally:
+        pool.close()
 
 
 # ----------------------------------------------------------------------------- ours
@@ -353,10 +426,13 @@ def build_state(workload, device, seed, batch=0):
     static = None
     sk = sv = None
     if s.scale_mode in ("per_head", "per_tensor"):
+        qmax = 127.0 if s.cache_dtype == "int8" else 448.0
         sk = torch.empty(s.num_kv_heads, dtype=torch.float32, device=device)
         sv = torch.empty(s.num_kv_heads, dtype=torch.float32, device=device)
-        kvq.kvq_calibrate_fp8_scales(w.warmup_k, sk)
-        kvq.kvq_calibrate_fp8_scales(w.warmup_v, sv)
+        kvq.kvq_calibrate_head_scales(w.warmup_k, qmax, sk)
+        kvq.kvq_calibrate_head_scales(w.warmup_v, qmax, sv)
+        if s.scale_mode == "per_tensor":          # one scale: the largest per-head one
+            sk, sv = sk.max().reshape(1), sv.max().reshape(1)
         static = (sk.cpu().numpy(), sv.cpu().numpy())
     elif s.scale_mode == "per_channel":
         qmax = 127.0 if s.cache_dtype == "int8" else 448.0
@@ -387,6 +463,114 @@ def build_state(workload, device, seed, batch=0):
         new["slots"] = w.slot_mapping[last].contiguous()
         new["seq_ids"] = new["positions"] = None
     return w, c, new, static
+
+
+# full-size configurations measured beside the main workload in the default run: the
+# decode call alone, with the main workload's timing protocol
+SUB_WORKLOADS = (("c2", "c2"), ("c3", "c3"), ("c4", "c4"), ("c4_int2", "c4-int2"),
+                 ("c5_fp8", "c5-fp8"), ("c5_bf16", "c5-bf16"))
+
+
+def measure_decode_call(workload, device, l2, steps, warmup):
+    """kvq_decode_attention alone (every kernel it launches) on the full-size workload: CUDA
+    events on the launching stream around each call, L2 emptied before each (outside the
+    events), at least `warmup` untimed calls and 0.3 s under load first, clocks sampled."""
+    import torch
+    from quantized_paged_kv_02_b200 import kvq, roofline
+    w, cache, _, _ = build_state(workload, device, seed=0)
+    s = w.spec
+    out = torch.empty(w.q.shape, dtype=torch.bfloat16, device=device)
+    mc = w.max_context
+    ws_n = cache.workspace_size(s.batch, s.num_q_heads, mc)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=device) if ws_n else None
+
+    def decode():
+        kvq.kvq_decode_attention(cache.desc, w.q, w.block_tables, w.context_lens, mc, out, ws)
+    nbytes = roofline.decode_bytes(s.cache_dtype, s.scale_mode, s.num_q_heads, s.num_kv_heads,
+                                   s.head_dim, s.block_size, w.context_lens.cpu().tolist())
+    sampler = ClockSampler(str(torch.cuda.get_device_properties(device).uuid))
+    sampler.start()
+    t0, i = time.perf_counter(), 0
+    while i < max(3, warmup) or time.perf_counter() - t0 < 0.3:
+        l2.flush()
+        decode()
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        l2.flush()
+        a.record()
+        decode()
+        b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    peak, kind = hbm_peak()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res = {"workload": "%s: %s" % (workload, WORKLOADS[workload]), "value": round(gbs, 2),
+           "unit": "GB/s", "ms_per_call": round(ms, 5), "frac": round(gbs / peak, 4),
+           "peak": peak, "peak_kind": kind, "tokens_per_s": round(s.batch / (ms * 1e-3), 1),
+           "bytes_per_call": nbytes,
+           "launches_per_call": cache.decode_plan(s.batch, s.num_q_heads, mc)[1],
+           "calls": steps, "warmup_calls": i, "clocks": clocks}
+    del w, cache, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_write_prefill(device, l2, steps, warmup):
+    """kvq_write of a prefill chunk: 4 sequences x 8192 new tokens of a 70B-shaped layer (8 kv
+    heads, head_dim 128), K and V, into an INT8 per-token-head and an FP8 per-kv-head cache.
+    Algorithmic bytes: the bf16 rows and slot ids read, the codes (and INT8 scales) written."""
+    import dataclasses
+    import torch
+    from quantized_paged_kv_02_b200 import inputs, kvq, roofline
+    peak, kind = hbm_peak()
+    res = {}
+    for cd, mode in (("int8", "per_token_head"), ("fp8", "per_head")):
+        spec = dataclasses.replace(inputs._spec("c5", False), cache_dtype=cd, scale_mode=mode,
+                                   batch=4, lens=[8192] * 4)
+        w = inputs.from_spec(spec, device)
+        s = w.spec
+        sk = sv = None
+        if mode == "per_head":
+            sk = torch.empty(s.num_kv_heads, dtype=torch.float32, device=device)
+            sv = torch.empty_like(sk)
+            kvq.kvq_calibrate_head_scales(w.warmup_k, 448.0, sk)
+            kvq.kvq_calibrate_head_scales(w.warmup_v, 448.0, sv)
+        c = kvq.PagedKVCache(cd, s.act_dtype, mode, w.num_blocks, s.block_size, s.num_kv_heads,
+                             s.head_dim, device=device, static_k_scale=sk, static_v_scale=sv)
+        T = w.k.shape[0]
+
+        def write():
+            kvq.kvq_write(c.desc, w.k, w.v, w.slot_mapping)
+        for _ in range(max(3, warmup)):
+            l2.flush()
+            write()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            l2.flush()
+            a.record()
+            write()
+            b.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+        nbytes = roofline.write_bytes(cd, mode, T, s.num_kv_heads, s.head_dim)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[cd] = {"value": round(gbs, 2), "unit": "GB/s", "ms_per_call": round(ms, 5),
+                   "frac": round(gbs / peak, 4), "peak_kind": kind, "rows": T,
+                   "bytes_per_call": nbytes,
+                   "cache": "%s %s" % (cd, mode)}
+        del w, c
+        torch.cuda.empty_cache()
+    res["config"] = ("kvq_write of 4 x 8192 new tokens (K and V rows [32768, 8, 128] bf16) "
+                     "into a paged cache, block 16; L2 emptied before each call")
+    return res
 
 
 class L2Flush:
@@ -550,6 +734,15 @@ def main_ours(args):
     e2e = statistics.mean(e2e_ms) if e2e_ms else float("nan")
     e2e, = max_over_ranks([e2e], world, device)
 
+    # the other target configurations at full size, one GPU only (at N > 1 every rank would
+    # have to take the same collective steps for them; the scaling run times the main step)
+    configs = None
+    write_prefill = None
+    if world == 1 and K > 0 and args.workload == "c5" and not args.batch:
+        configs = {key: measure_decode_call(name, device, l2, max(K, 20), args.warmup)
+                   for key, name in SUB_WORKLOADS}
+        write_prefill = measure_write_prefill(device, l2, max(K, 20), args.warmup)
+
     peak, peak_kind = hbm_peak()
     achieved = dec_bytes / (dms * 1e-3) / 1e9
     launches_per_step = 1 + cache.decode_plan(B, s.num_q_heads, max_ctx)[1]
@@ -559,7 +752,8 @@ def main_ours(args):
         "unit": "GB/s",
         "n_gpus": world,
         "steps": K,
-        "warmup": warm,
+        "warmup": args.warmup,
+        "warmup_steps_run": warm,
         "ms_per_step": round(ms, 5),
         "higher_is_better": True,
         "scaling": "weak",
@@ -572,7 +766,10 @@ def main_ours(args):
                                   "" if not args.batch else
                                   " (batch reduced to %d for profiling: not a benchmark line)" % B),
                    "global_batch": B * world, "seq_len": max_ctx, "parallelism": "dp%d" % world,
-                   "l2": L2Flush.DESCRIPTION},
+                   "l2": L2Flush.DESCRIPTION,
+                   "warmup": "at least the requested warm-up steps, and at least %.1f s under load "
+                             "so the clocks reach their steady state (warmup_steps_run)"
+                             % args.min_warmup_s},
         "tokens_per_s": round(world * B / (ms * 1e-3), 1),
         "hbm_frac_of_%s" % peak_kind: round(step_bytes / (ms * 1e-3) / 1e9 / peak, 4),
         "bytes_per_step": step_bytes,
@@ -589,19 +786,13 @@ def main_ours(args):
                         ", one packed host-to-device copy of the step's inputs, output copied back"},
         "append_decode": fused,
         "prefill": prefill,
+        "configs": configs,
+        "write_prefill": write_prefill,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = run_oracle_sample(w, static)
-        result["cpu_baseline"] = {
-            "value": round(r["bytes"] / r["seconds"] / 1e9, 6), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": "%d (sequence, kv head) units of the %d in the step, taken in order and "
-                      "cycling; each: quantize the new row + float64 attention of its %d query "
-                      "heads over all cached positions; %.1f s of timed oracle work"
-                      % (r["units"], B * s.num_kv_heads, s.num_q_heads // s.num_kv_heads,
-                         r["seconds"])}
+        result["cpu_baseline"] = run_oracle_sample(args.workload)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -609,47 +800,34 @@ def main_ours(args):
 
 
 def main_reference(args):
+    """The oracle as the reference arm: every host core runs one (sequence, kv head) unit
+    step per round (see OraclePool); a step of this arm is one round."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    import torch
-    from quantized_paged_kv_02_b200 import inputs
-    from threadpoolctl import threadpool_limits
-    w = unit_workload(args.workload)
-    static = None
-    if w.spec.scale_mode in ("per_head", "per_tensor"):
-        from oracle import quant
-        static = (quant.fp8_calibrate(w.warmup_k.float().numpy()),
-                  quant.fp8_calibrate(w.warmup_v.float().numpy()))
-    elif w.spec.scale_mode == "per_channel":
-        from oracle import quant
-        qmax = 127.0 if w.spec.cache_dtype == "int8" else 448.0
-        static = (quant.channel_calibrate(w.warmup_k.float().numpy(), qmax),
-                  quant.channel_calibrate(w.warmup_v.float().numpy(), qmax))
-    rows = oracle_inputs(w, [(0, 0)])
-    step = oracle_unit_step(w, rows, 0, 0, static)
-    nbytes = unit_bytes(w, 0)
-    with threadpool_limits(limits=1):
+    pool = OraclePool(args.workload)
+    try:
         for _ in range(max(1, args.warmup)):
-            step()
-        times = []
-        for _ in range(args.steps):
-            t0 = time.perf_counter()
-            step()
-            times.append(time.perf_counter() - t0)
+            pool.round()
+        times = [pool.round() for _ in range(args.steps)]
+    finally:
+        pool.close()
     sec = statistics.mean(times)
-    value = nbytes / sec / 1e9
-    del torch
+    value = pool.bytes_per_round() / sec / 1e9
+    sample = ("one step of a (sequence, kv head) unit (%d cached tokens, %d query heads; quantize "
+              "the new row + float64 attention over every cached position) on each of %d worker "
+              "processes, one per host core, one thread each" % (pool.case["n"], pool.case["g"],
+                                                                  pool.workers))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "%s: %s; step = one (sequence, kv head) unit of the serving step"
-                               % (args.workload, WORKLOADS[args.workload])},
-        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": "unit (sequence 0, kv head 0): quantize the new row + float64 "
-                                   "attention of its query heads over every cached position"},
+        "config": {"workload": "%s: %s; step = %d (sequence, kv head) units of the serving step, "
+                               "one per host core" % (args.workload, WORKLOADS[args.workload],
+                                                      pool.workers)},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": pool.workers,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)

@@ -253,9 +253,11 @@ kvq_status kvq_flush_ring(const kvq_cache_desc* cache, const int32_t* seq_ids,
                           cudaStream_t stream);
 
 /*
- * Workspace bytes kvq_decode_attention needs for this shape (host-only).  The split
- * plan depends only on (cache geometry, batch, num_q_heads, max_context), so the same
- * arguments always give the same size.  *bytes may be 0 (no split needed).
+ * Workspace bytes kvq_decode_attention needs for this shape (host-only: it reads the
+ * current device's SM count, and launches nothing).  The split plan depends only on (cache
+ * geometry, batch, num_q_heads, max_context) and that SM count (148 on B200, and 148 when
+ * no device can be queried), so the same arguments on the same device always give the same
+ * size.  *bytes may be 0 (no split needed).
  */
 kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
                                      int num_q_heads, int max_context, size_t* bytes);
@@ -265,9 +267,9 @@ kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
  * only: no device access, no launch; the pages give no counterpart, it reports this
  * library's dispatch).  Any output pointer may be NULL.
  *   kernel_out    0: the CUDA-core split kernel; 1: the page-balanced tensor-core kernel
- *                 (dense caches); 2: the low-bit (INT4 / INT2) tensor-core block kernel
- *                 plus the CUDA-core kernel for the residual ring.
- *   launches_out  kernels one call launches, the merge included (1: 2; 2: 3; 0: 1, or 2
+ *                 (dense caches; it merges its own partials); 2: the low-bit (INT4 / INT2)
+ *                 tensor-core block kernel plus the CUDA-core kernel for the residual ring.
+ *   launches_out  kernels one call launches, the merge included (1: 1; 2: 3; 0: 1, or 2
  *                 with more than one split; 0 when batch is 0).
  *   splits_out    token splits of kernels 0 and 2 (the ring counted as one); for kernel 1,
  *                 its CTA count (the page ranges).
@@ -291,12 +293,18 @@ kvq_status kvq_decode_plan(const kvq_cache_desc* cache, int batch, int num_q_hea
  *   softmax_scale 0 selects 1/sqrt(D) ([P-mem] §6 Q1 writes softmax(q k^T / sqrt(d))).
  *   out           out_dtype [batch][num_q_heads][D], device; out_dtype BF16, FP16 or FP32.
  *   workspace     device scratch of at least kvq_decode_workspace_size() bytes (may be
- *                 NULL when that size is 0).  Its contents need no initialisation.
+ *                 NULL when that size is 0).  Its contents need no initialisation: the
+ *                 tensor-core kernel's per-(sequence, kv head) arrival counters in it carry
+ *                 a tag of the call that wrote them, and a counter with another call's tag
+ *                 counts as empty (each call leaves its counters empty when it completes).
+ *                 Two calls that overlap on the GPU must not share a workspace.
  *   For each (b, hq): o = sum_p softmax_p(scale * q . k_p) v_p over p < context_lens[b],
  *   where k_p, v_p are the dequantized cache rows; for INT4 / INT2, positions p < Qb come
  *   from blocks and the rest from the residual ring, Qb = 64*floor(max(len-residual_len,0)/64).
  *   Dequantization happens inside the kernel ([P-vLLM] "PagedAttention与KV Cache量化协同
- *   工作原理"); long contexts are split across CTAs and merged by a log-sum-exp reduce.
+ *   工作原理"); long contexts are split across CTAs and merged by a log-sum-exp reduce (on
+ *   the tensor-core kernel, by the last warp to finish a part of each (sequence, kv head),
+ *   inside the same launch).
  *   Kernels: head_dim 128 with block_size 16 and 1..8 query heads per kv head runs on the
  *   tensor-core kernel (dense caches); INT4 / INT2 with head_dim 128 and 3..8 query heads per
  *   kv head on the low-bit tensor-core kernel; everything else on the CUDA-core kernel.
@@ -364,7 +372,9 @@ kvq_status kvq_prefill_attention(const kvq_cache_desc* cache, const void* q, int
 
 /*
  * Size of the device scratch array used by kvq_decode_attention_noalloc (16 MiB).  Every
- * GPU that loads the library reserves this much for the life of the process.
+ * GPU that loads the library's device code reserves this much for the life of the process
+ * (under CUDA's lazy module loading, at the first kvq_decode_attention_noalloc call on
+ * that device rather than when the library is opened).
  */
 #define KVQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 
@@ -379,12 +389,16 @@ kvq_status kvq_prefill_attention(const kvq_cache_desc* cache, const void* q, int
  *   This variant takes the same arguments as kvq_decode_attention minus the workspace and
  *   uses a fixed, file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES instead.  It calls no
  *   cudaMalloc, cudaFree or other allocating routine.
- *   - The scratch of the CURRENT device is used: make the device that owns `stream` current.
- *     The first call on each device looks up the array's device address (set-up); make that
- *     first call before any stream capture.
+ *   - The scratch of the CURRENT device and context is used: make the device that owns
+ *     `stream` current.  Every call with batch > 0 looks up the array's device address in
+ *     the current context (nothing is cached, so a cudaDeviceReset or a switch of context
+ *     between calls is safe).  Under lazy module loading the first look-up on a device loads
+ *     the library's device code and reserves the array there; make that first call before
+ *     any stream capture and while memory is still free.
  *   - Returns KVQ_ERR_INVALID_ARG, with nothing enqueued, when this shape needs more scratch
  *     than KVQ_NOALLOC_SCRATCH_BYTES (kvq_decode_workspace_size tells the need).  Returns
- *     KVQ_ERR_CUDA if the address look-up fails.
+ *     KVQ_ERR_CUDA if the address look-up fails (for example when the first look-up cannot
+ *     reserve the array because device memory is short).
  *   - All calls on a device share the one array, and it keeps whatever the last call left
  *     there (nothing in it needs to start at zero).  Calls that overlap on the GPU (for
  *     example on two streams without ordering between them) race on the array and give
@@ -417,6 +431,21 @@ kvq_status kvq_dequant(const kvq_cache_desc* cache, const int32_t* block_ids, in
 kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_heads,
                                     int head_dim, int32_t act_dtype, float* scale_out,
                                     cudaStream_t stream);
+
+/*
+ * kvq_calibrate_head_scales - set-up step: per-kv-head scale from warm-up rows,
+ *   scale_out[h] = (max over tokens and channels of |x[t][h][:]|) / qmax, float32 division
+ *   (kvq_calibrate_fp8_scales is this call with qmax = 448).
+ *   x          act_dtype [n_tokens][num_kv_heads][head_dim], device.
+ *   qmax       largest code magnitude: 127 for INT8, 448 for FP8 E4M3; finite and > 0.
+ *   scale_out  float32 [num_kv_heads], device.  An all-zero head gives 0.
+ *   The static scales of KVQ_SCALE_PER_HEAD ([P-mem] §3.2 动态量化策略: static quantization
+ *   keeps fixed scales; [P-prod] "量化不是简单截断精度": a scale per tensor or per head).  A
+ *   per-tensor scale is the largest of the per-head ones.
+ */
+kvq_status kvq_calibrate_head_scales(const void* x, int n_tokens, int num_kv_heads,
+                                     int head_dim, int32_t act_dtype, float qmax,
+                                     float* scale_out, cudaStream_t stream);
 
 /*
  * kvq_calibrate_channel_scales - set-up step: per-(kv head, channel) scale from warm-up rows,

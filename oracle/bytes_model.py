@@ -29,19 +29,27 @@ def decode_step_bytes(cache_dtype, scale_mode, batch, num_q_heads, num_kv_heads,
     """Bytes one decode step must move: cache rows read, metadata read, q read, out written.
 
     Per token and kv head: K and V codes (head_dim x bytes per value) plus their
-    per-token scale bytes; per block and kv head: the KIVI key scales/zeros; per
-    sequence: block-table entries and its context length; q and out once.  INT4 reads
-    the newest tokens from the residual ring at act_bytes per value.
+    per-token scale bytes; per block and kv head: the KIVI key scales/zeros (per token
+    and channel group when keys are grouped per token); per sequence: block-table entries
+    and its context length; q and out once.  INT4 and 2-bit caches read the newest tokens
+    from the residual ring at act_bytes per value.
     """
     D, H = head_dim, num_kv_heads
     total = Fraction(0)
     for n in context_lens:
         n = int(n)
-        if cache_dtype == "int4":
+        if cache_dtype in ("int4", "int2"):
+            # 4-bit or 2-bit codes ([P-prod] "KV Cache 的基本内存模型": 0.5 / 0.25 byte per
+            # value) in whole groups; the newest tokens stay in the residual ring
             qb = group_size * (max(n - residual_len, 0) // group_size)
             nblk = qb // block_size
-            total += 2 * H * qb * D * Fraction(1, 2)                    # codes
-            total += H * nblk * 2 * D * 2                               # K scale+zero fp16
+            total += 2 * H * qb * D * BYTES_PER_VALUE[cache_dtype]     # K and V codes
+            if scale_mode == "int4_per_token":
+                # keys grouped like values: (scale, zero) fp16 per token and channel group
+                total += H * qb * (D // group_size) * 2 * 2
+            else:
+                # KIVI keys: (scale, zero or minimum) fp16 per channel and block
+                total += H * nblk * 2 * D * 2
             total += H * qb * (D // group_size) * 2 * 2                 # V scale+zero fp16
             total += 2 * H * (n - qb) * D * act_bytes                   # residual rows
             total += 4 * nblk

@@ -6,7 +6,7 @@ Inputs are activation values (bfloat16 or float16 values, exactly representable 
 binary32) given as NumPy arrays; outputs are codes and scales with the bit patterns the
 cache stores.
 
-Readings of the pages taken here (each listed in the design doc):
+Readings of the pages taken here:
   * "round" is round-half-to-even: the INT8 snippet of [P-mem] §3.1 对称量化算法 uses
     torch.round, which rounds half to even.
   * x / scale and the scale itself are IEEE binary32: the snippet returns the scale as
@@ -90,6 +90,19 @@ def fp8_calibrate(warmup):
     w = np.asarray(warmup, dtype=np.float32)
     m = np.max(np.abs(w), axis=(0, 2))
     return fp.div32(m, np.float32(FP8_QMAX))
+
+
+def head_calibrate(warmup, qmax):
+    """Per-kv-head static scale from warm-up rows [T, H, D]: max over tokens and channels of
+    |x|, divided by qmax in binary32, [H].  qmax is 127 for INT8, 448 for FP8
+    (fp8_calibrate is this with 448).
+
+    [P-mem] §3.2 动态量化策略: static quantization keeps one fixed scale; [P-vLLM]
+    "KV Cache量化策略：INT8与FP8精度对比与选择": INT8 per tensor; [P-prod] "量化不是简单截断精度":
+    scales per tensor or per head.
+    """
+    w = np.asarray(warmup, dtype=np.float32)
+    return fp.div32(np.max(np.abs(w), axis=(0, 2)), np.float32(qmax))
 
 
 def channel_calibrate(warmup, qmax):

@@ -1,5 +1,6 @@
 // C ABI entry points: host-side validation, layout arithmetic and dispatch.
 // Declarations and the contract of every call are in include/kvq.h.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -96,6 +97,16 @@ using namespace kvq;
 
 namespace {
 
+// Tag of one decode call's arrivals on the per-unit counters of the workspace.  A counter
+// holding another call's tag (left by a call that stopped early) counts as empty, so the
+// workspace needs no clearing between calls.  0 is never used.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> counter{0};
+  uint32_t e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (e == 0) e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+  return e;
+}
+
 // Shared by kvq_decode_attention and kvq_append_decode_attention (k_new / v_new null for
 // the former).
 kvq_status decode_entry(const kvq_cache_desc* c, const void* k_new, const void* v_new,
@@ -132,7 +143,10 @@ kvq_status decode_entry(const kvq_cache_desc* c, const void* k_new, const void* 
       return KVQ_ERR_INVALID_ARG;
     a.ws_o = static_cast<float*>(workspace);
     a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + a.plan.ws_ml_off);
+    if (a.plan.kernel == 1)
+      a.ws_cnt = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + a.plan.ws_cnt_off);
   }
+  a.epoch = next_epoch();
   a.q = q;
   a.k_new = k_new;
   a.v_new = v_new;
@@ -212,9 +226,9 @@ kvq_status kvq_decode_plan(const kvq_cache_desc* c, int batch, int num_q_heads, 
   DecodePlan p;
   st = plan_decode(g, batch, num_q_heads, max_context, &p);
   if (st != KVQ_OK) return st;
-  // the launches of launch_decode: kernel 1 + segment merge; INT4/INT2 blocks + ring kernel +
-  // split reduce; CUDA-core kernel (+ split reduce when it splits)
-  int launches = p.kernel == 1 ? 2 : p.kernel == 2 ? 3 : (p.splits > 1 ? 2 : 1);
+  // the launches of launch_decode: kernel 1 (it merges its own partials); INT4/INT2 blocks +
+  // ring kernel + split reduce; CUDA-core kernel (+ split reduce when it splits)
+  int launches = p.kernel == 1 ? 1 : p.kernel == 2 ? 3 : (p.splits > 1 ? 2 : 1);
   if (batch == 0) launches = 0;                       // nothing to do: nothing launched
   if (kernel_out) *kernel_out = p.kernel;
   if (launches_out) *launches_out = launches;
@@ -278,7 +292,19 @@ kvq_status kvq_calibrate_fp8_scales(const void* x, int n_tokens, int num_kv_head
   if (n_tokens < 0 || num_kv_heads < 1 || head_dim < 1) return KVQ_ERR_INVALID_ARG;
   if (act_dtype != KVQ_DTYPE_BF16 && act_dtype != KVQ_DTYPE_FP16) return KVQ_ERR_INVALID_ARG;
   if (scale_out == nullptr || (n_tokens > 0 && x == nullptr)) return KVQ_ERR_INVALID_ARG;
-  return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, scale_out, stream));
+  return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, 448.f, scale_out,
+                                    stream));
+}
+
+kvq_status kvq_calibrate_head_scales(const void* x, int n_tokens, int num_kv_heads, int head_dim,
+                                     int32_t act_dtype, float qmax, float* scale_out,
+                                     cudaStream_t stream) {
+  if (n_tokens < 0 || num_kv_heads < 1 || head_dim < 1) return KVQ_ERR_INVALID_ARG;
+  if (act_dtype != KVQ_DTYPE_BF16 && act_dtype != KVQ_DTYPE_FP16) return KVQ_ERR_INVALID_ARG;
+  if (!(qmax > 0.f) || !std::isfinite(qmax)) return KVQ_ERR_INVALID_ARG;
+  if (scale_out == nullptr || (n_tokens > 0 && x == nullptr)) return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_calibrate(x, n_tokens, num_kv_heads, head_dim, act_dtype, qmax, scale_out,
+                                    stream));
 }
 
 kvq_status kvq_prefill_attention(const kvq_cache_desc* c, const void* q, int num_q_tokens, int batch,

@@ -31,6 +31,8 @@ struct DecodeParams {
   int out_dtype;
   float* ws_o;               // [B][Hq][S][D]
   float* ws_ml;              // [B][Hq][S][2]  (max, sum) in the log2 domain
+  unsigned long long* ws_cnt;  // dense tensor-core kernel: [B*H] arrival counters
+  uint32_t epoch;            // dense tensor-core kernel: this call's tag (never 0)
   int32_t* fault;
   // append step (kvq_append_decode_attention), else null: this step's K / V row of every
   // sequence, [B][H][D] act dtype, stored at position context_lens[b] - 1 before decode
@@ -79,15 +81,16 @@ __device__ __forceinline__ SeqInfo seq_info(const DecodeParams& p, int b, bool i
 }
 
 // ---------------------------------------------------------------- page-balanced schedule
-// The dense tensor-core kernel runs one CTA per resident slot.  The pages of all
-// (sequence, kv head) units, concatenated in the order (sequence, kv head, page), are cut
-// into ctas contiguous ranges of equal size: CTA c takes [P c / C, P (c + 1) / C).  A CTA
-// range crossing unit boundaries covers several segments (unit, CTA); each consumer warp
-// of the CTA writes one partial per segment it saw, into slot (unit + c) * kSegWarps + warp.
-// (Going from one segment to the next raises the unit index, the CTA index or both, so
-// unit + c never repeats and there are at most units + C - 1 segments.)
+// The dense tensor-core kernel runs one CTA per resident slot (kMmaCtasPerSM per SM).  The
+// pages of all (sequence, kv head) units, concatenated in the order (sequence, kv head,
+// page), are cut into ctas contiguous ranges of equal size: CTA c takes
+// [P c / C, P (c + 1) / C).  A CTA range crossing unit boundaries covers several segments
+// (unit, CTA); each consumer warp of the CTA writes one partial per segment it saw, into
+// slot (unit + c) * kSegWarps + warp.  (Going from one segment to the next raises the unit
+// index, the CTA index or both, so unit + c never repeats and there are at most
+// units + C - 1 segments.)  The last warp to write a partial of a unit merges them all.
 constexpr int kSegWarps = 4;
-constexpr int kMmaCtas = 3 * kNumSMs;   // resident CTAs of the dense tensor-core kernel
+constexpr int kMmaCtasPerSM = 3;
 
 __device__ __forceinline__ long long range_start(long long P, int c, int C) {
   return P * c / C;

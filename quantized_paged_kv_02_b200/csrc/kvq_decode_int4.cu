@@ -201,7 +201,7 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
     if (lane == 0) {
       for (int i = max(0, issued - kStages); i < issued; ++i)
-        if (!mbar_wait(&full[i % kStages], (i / kStages) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+        if (!mbar_drain(&full[i % kStages], (i / kStages) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
     }
   } else {
     // ---------------------------------------------------------------- consumers

@@ -18,7 +18,6 @@
 
 namespace kvq {
 
-constexpr int kNumSMs = 148;            // B200
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ fault record
@@ -137,6 +136,10 @@ struct Geometry {
 
 kvq_status validate_desc(const kvq_cache_desc* c, Geometry* g);
 int code_bits(int cache_dtype);
+// Streaming multiprocessors of the current device (148 on B200; 148 too when no device can
+// be queried, so host-only size queries work without a GPU).  Grids and split plans are
+// sized from it.
+int device_sm_count();
 
 // INT4 and INT2 caches: 64-token groups, zero points, a residual ring of recent tokens
 __host__ __device__ inline bool low_bit(int cache_dtype) {
@@ -153,7 +156,7 @@ cudaError_t launch_flush_ring(const kvq_cache_desc& c, const Geometry& g, const 
                               const int32_t* positions, const int32_t* blocks, int n, cudaStream_t s);
 cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int32_t* ids, int n,
                            float* out, cudaStream_t s);
-cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float* out,
+cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float qmax, float* out,
                              cudaStream_t s);
 cudaError_t launch_calibrate_channels(const void* x, int n, int H, int D, int act, float qmax,
                                       float* out, cudaStream_t s);
@@ -169,6 +172,8 @@ struct DecodePlan {
   int ctas;          // kernel 1: grid size
   size_t ws_bytes;   // workspace bytes (0 when a single split writes the output)
   size_t ws_ml_off;  // byte offset of the (max, sum) array inside the workspace
+  size_t ws_cnt_off; // kernel 1: byte offset of the per-unit arrival counters
+  int sms;           // streaming multiprocessors the plan was made for
 };
 
 kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_context,
@@ -194,6 +199,8 @@ struct DecodeArgs {
   int out_dtype;
   float* ws_o;               // partial outputs (layout per kernel)
   float* ws_ml;              // partial (max, sum) pairs
+  unsigned long long* ws_cnt;  // kernel 1: per-unit arrival counters
+  uint32_t epoch;            // kernel 1: tag of this call's arrivals (never 0)
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

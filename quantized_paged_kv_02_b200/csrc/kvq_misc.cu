@@ -1,4 +1,5 @@
-// kvq_dequant (debug), kvq_calibrate_fp8_scales and kvq_calibrate_channel_scales (set-up)
+// kvq_dequant (debug), kvq_calibrate_fp8_scales, kvq_calibrate_head_scales and
+// kvq_calibrate_channel_scales (set-up)
 // kernels.
 //
 // Dequantized values follow the definitions in include/kvq.h: INT8 / FP8 code * scale
@@ -87,7 +88,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantParams p) {
 }
 
 template <typename TA>
-__global__ void __launch_bounds__(256) calibrate_kernel(const TA* x, int n, int H, int D, float* out) {
+__global__ void __launch_bounds__(256) calibrate_kernel(const TA* x, int n, int H, int D, float qmax,
+                                                        float* out) {
   const int h = blockIdx.x;
   float m = 0.f;
   for (long e = threadIdx.x; e < static_cast<long>(n) * D; e += blockDim.x) {
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(256) calibrate_kernel(const TA* x, int n, int 
   if (threadIdx.x < 32) {
     m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (threadIdx.x == 0) out[h] = div_rn(m, 448.f);
+    if (threadIdx.x == 0) out[h] = div_rn(m, qmax);
   }
 }
 
@@ -139,12 +141,13 @@ cudaError_t launch_dequant(const kvq_cache_desc& c, const Geometry& g, const int
   return cudaGetLastError();
 }
 
-cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float* out,
+cudaError_t launch_calibrate(const void* x, int n, int H, int D, int act, float qmax, float* out,
                              cudaStream_t s) {
   if (act == KVQ_DTYPE_BF16)
-    calibrate_kernel<__nv_bfloat16><<<H, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n, H, D, out);
+    calibrate_kernel<__nv_bfloat16><<<H, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), n, H, D, qmax,
+                                                       out);
   else
-    calibrate_kernel<__half><<<H, 256, 0, s>>>(static_cast<const __half*>(x), n, H, D, out);
+    calibrate_kernel<__half><<<H, 256, 0, s>>>(static_cast<const __half*>(x), n, H, D, qmax, out);
   return cudaGetLastError();
 }
 

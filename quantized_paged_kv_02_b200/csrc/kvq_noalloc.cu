@@ -7,8 +7,6 @@
 // decode with the split partials in a fixed device array that lives in this file, so the
 // caller supplies only inputs and outputs.  The pages have no counterpart: this is an
 // interface convenience, not part of the method.
-#include <mutex>
-
 #include "kvq_internal.cuh"
 
 namespace {
@@ -18,25 +16,16 @@ namespace {
 // stand-in); it passes the device address looked up below.
 static __device__ __align__(256) unsigned char g_decode_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_lock;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device, looked up once per device with
-// that device current (the first call per device does this set-up).
+// Device address of the scratch in the current context of the current device.  Looked up
+// on every call rather than cached: a cached address would outlive a cudaDeviceReset or
+// belong to another context made current on the same device.  Once the module is loaded
+// the look-up allocates nothing; under lazy module loading the first look-up on a device
+// is what loads it (and reserves the array), and it fails if memory is short.
 cudaError_t scratch_of_current_device(void** addr) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> guard(g_lock);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *addr = g_scratch_addr[dev];
+  *addr = p;
   return cudaSuccess;
 }
 
@@ -52,7 +41,9 @@ extern "C" kvq_status kvq_decode_attention_noalloc(
   if (st != KVQ_OK) return st;
   if (need > KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_INVALID_ARG;   // shape too large
   void* scratch = nullptr;
-  if (need > 0 && batch > 0) {
+  // the look-up runs for every non-empty call, whatever this shape needs, so the first
+  // call on a device always does the set-up
+  if (batch > 0) {
     if (scratch_of_current_device(&scratch) != cudaSuccess) return KVQ_ERR_CUDA;
   }
   return kvq_decode_attention(cache, q, batch, num_q_heads, block_tables, max_blocks_per_seq,

@@ -56,6 +56,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// Final wait of a producer for a copy it issued, before its CTA may exit (the copy writes
+// this CTA's shared memory).  Every copy the kernels issue reads a record inside its tensor
+// map (block ids are range-checked first) and completes without waiting on any other agent,
+// so this returns true unless the hardware itself has failed; a first bounded wait that
+// runs out (after a fault has been recorded by the caller's other waits, the GPU may be
+// slow to drain) is followed by a second one before giving up.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  return mbar_wait(bar, parity) || mbar_wait(bar, parity);
+}
+
 // ------------------------------------------------------------------ dependent launch
 // A kernel launched with programmatic stream serialization may start before the kernel
 // ahead of it in the stream has finished.  griddep_wait() blocks until that kernel has

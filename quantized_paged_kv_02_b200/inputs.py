@@ -84,11 +84,12 @@ def _spec(name, small):
         return Spec(name, cd, "bf16", mode, 16, 64, 8, 128, 64,
                     lens=[32768] * 16, outliers="k", slack_blocks=16)
     if name.startswith("c5"):
+        # -pc / -ph / -pt: static scales per (kv head, channel), per kv head, per tensor
         cd = {"c5": "int8", "c5-int8": "int8", "c5-fp8": "fp8", "c5-bf16": "bf16",
-              "c5-int8-pc": "int8"}[name]
+              "c5-int8-pc": "int8", "c5-int8-ph": "int8", "c5-int8-pt": "int8",
+              "c5-fp8-pt": "fp8"}[name]
         mode = {"int8": "per_token_head", "fp8": "per_head", "bf16": "none"}[cd]
-        if name == "c5-int8-pc":
-            mode = "per_channel"
+        mode = {"pc": "per_channel", "ph": "per_head", "pt": "per_tensor"}.get(name[-2:], mode)
         if small:
             return Spec(name + "-small", cd, "bf16", mode, 3, 16, 2, 128, 16,
                         lens=[1000, 517, 33], slack_blocks=4)
@@ -125,7 +126,8 @@ def act_torch_dtype(act):
 
 def make(name, small=False, device="cpu", seed=None):
     """Build the named workload ("c1".."c5", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok",
-    "c4-int2-fzp", "c5-fp8", "c5-bf16", "c5-int8-pc") on `device`."""
+    "c4-int2-fzp", "c5-fp8", "c5-bf16", "c5-int8-pc", "c5-int8-ph", "c5-int8-pt",
+    "c5-fp8-pt") on `device`."""
     spec = _spec(name, small)
     if seed is not None:
         spec.seed = seed

@@ -27,7 +27,7 @@ EXPORTS = ("kvq_status_string", "kvq_version", "kvq_cache_layout", "kvq_write",
            "kvq_decode_workspace_size", "kvq_decode_attention", "kvq_dequant",
            "kvq_calibrate_fp8_scales", "kvq_read_device_fault", "kvq_decode_attention_noalloc",
            "kvq_append_decode_attention", "kvq_calibrate_channel_scales", "kvq_flush_ring",
-           "kvq_prefill_attention", "kvq_decode_plan")
+           "kvq_prefill_attention", "kvq_decode_plan", "kvq_calibrate_head_scales")
 
 
 class CacheDesc(ctypes.Structure):
@@ -71,6 +71,7 @@ def _load():
         "kvq_append_decode_attention": (I, [D, P, P, P, I, I, P, I, P, I, F, P, ctypes.c_int32, P,
                                             Z, P]),
         "kvq_calibrate_channel_scales": (I, [P, I, I, I, ctypes.c_int32, F, P, P]),
+        "kvq_calibrate_head_scales": (I, [P, I, I, I, ctypes.c_int32, F, P, P]),
         "kvq_flush_ring": (I, [D, P, P, P, I, P]),
         "kvq_prefill_attention": (I, [D, P, I, I, I, P, I, P, I, P, I, F, P, ctypes.c_int32, P]),
     }
@@ -228,6 +229,15 @@ def kvq_flush_ring(desc, seq_ids, positions, block_ids, stream=None):
     n = int(seq_ids.numel())
     _check(lib.kvq_flush_ring(ctypes.byref(desc), _ptr(_i32(seq_ids)), _ptr(_i32(positions)),
                               _ptr(_i32(block_ids)), n, _stream(stream)), "kvq_flush_ring")
+
+
+def kvq_calibrate_head_scales(x, qmax, scale_out, stream=None):
+    """scale_out[h] = max over tokens and channels |x[t][h][:]| / qmax (127 INT8, 448 FP8)."""
+    T, H, D = x.shape
+    _check(lib.kvq_calibrate_head_scales(_ptr(x), T, H, D, DTYPE[_act(x)], float(qmax),
+                                         _ptr(scale_out), _stream(stream)),
+           "kvq_calibrate_head_scales")
+    return scale_out
 
 
 def kvq_calibrate_channel_scales(x, qmax, scale_out, stream=None):

@@ -29,8 +29,9 @@ def oracle_static_scales(w):
         return (quant.channel_calibrate(np64(w.warmup_k).astype(np.float32), qmax),
                 quant.channel_calibrate(np64(w.warmup_v).astype(np.float32), qmax))
     if w.spec.scale_mode in ("per_head", "per_tensor"):
-        ks = quant.fp8_calibrate(np64(w.warmup_k).astype(np.float32))
-        vs = quant.fp8_calibrate(np64(w.warmup_v).astype(np.float32))
+        qmax = 127.0 if w.spec.cache_dtype == "int8" else 448.0
+        ks = quant.head_calibrate(np64(w.warmup_k).astype(np.float32), qmax)
+        vs = quant.head_calibrate(np64(w.warmup_v).astype(np.float32), qmax)
         if w.spec.scale_mode == "per_tensor":
             ks, vs = ks.max(keepdims=True), vs.max(keepdims=True)
         return ks, vs

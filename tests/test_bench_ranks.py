@@ -73,10 +73,24 @@ def test_step_launch_count_comes_from_the_library():
     reports for the decode call (host only: the cache can live in CPU memory here)."""
     import bench
     from quantized_paged_kv_02_b200 import inputs, kvq
-    for name, want in (("c5", 2), ("c4", 3), ("c4-int2", 3)):
+    for name, want in (("c5", 1), ("c4", 3), ("c4-int2", 3)):
         s = inputs._spec(name, False)
         c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, 64, s.block_size,
                              s.num_kv_heads, s.head_dim, device="cpu", max_seqs=s.batch,
                              static_k_scale=None, static_v_scale=None)
         assert c.decode_plan(s.batch, s.num_q_heads, 16384)[1] == want
     assert "decode_plan" in open(bench.__file__).read()
+
+
+def test_oracle_pool_runs_rounds_on_worker_processes():
+    """The CPU baseline's pool: spawned workers (no fork from a CUDA context), each with its
+    own unit cache; a round is one step on every worker, timed first start to last end."""
+    import bench
+    pool = bench.OraclePool("c1", workers=2)
+    try:
+        assert pool.workers == 2 and pool.cores >= 1
+        t = pool.round()
+        assert 0.0 < t < 60.0
+        assert pool.bytes_per_round() == 2 * pool.case["bytes"] > 0
+    finally:
+        pool.close()

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
 SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok", "c4-int2-fzp", "c5",
-         "c5-fp8", "c5-bf16", "c5-int8-pc"]
+         "c5-fp8", "c5-bf16", "c5-int8-pc", "c5-int8-ph", "c5-int8-pt", "c5-fp8-pt"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -156,6 +156,9 @@ KINDS = {
     "bf16": ("bf16", "none"),
     "int8-pc": ("int8", "per_channel"),
     "fp8-pc": ("fp8", "per_channel"),
+    "int8-ph": ("int8", "per_head"),
+    "int8-pt": ("int8", "per_tensor"),
+    "fp8-pt": ("fp8", "per_tensor"),
 }
 
 

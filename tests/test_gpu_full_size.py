@@ -21,7 +21,8 @@ from tests import helpers
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
-FULL = ["c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2", "c5", "c5-fp8", "c5-bf16", "c5-int8-pc"]
+FULL = ["c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok", "c4-int2-fzp", "c5",
+        "c5-fp8", "c5-bf16", "c5-int8-pc", "c5-int8-ph", "c5-int8-pt", "c5-fp8-pt"]
 
 
 @pytest.fixture(scope="module", autouse=True)

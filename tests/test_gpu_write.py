@@ -13,7 +13,7 @@ from tests import helpers
 pytestmark = pytest.mark.gpu
 
 SMALL = ["c1", "c2", "c3", "c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok", "c4-int2-fzp", "c5",
-         "c5-fp8", "c5-bf16", "c5-int8-pc"]
+         "c5-fp8", "c5-bf16", "c5-int8-pc", "c5-int8-ph", "c5-int8-pt", "c5-fp8-pt"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -49,6 +49,18 @@ def test_fp8_calibration_bit_exact():
         kvq.kvq_calibrate_fp8_scales(x.cuda(), out)
         want = quant.fp8_calibrate(helpers.np64(x).astype(np.float32))
         np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+def test_head_calibration_bit_exact():
+    from oracle import quant
+    from quantized_paged_kv_02_b200 import kvq
+    w = inputs.make("c5-int8-ph", small=True)
+    for x in (w.warmup_k, w.warmup_v):
+        for qmax in (127.0, 448.0):
+            out = torch.empty(x.shape[1], dtype=torch.float32, device="cuda")
+            kvq.kvq_calibrate_head_scales(x.cuda(), qmax, out)
+            want = quant.head_calibrate(helpers.np64(x).astype(np.float32), qmax)
+            np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
 
 
 def test_channel_calibration_bit_exact():

@@ -69,3 +69,62 @@ def test_decode_step_bytes_components():
     assert b8 - (24 * (4 * 1024 + 4) + 2 * 24 * 64 * 128 * 2) == 830472192
     bf = bytes_model.decode_step_bytes("bf16", "none", 24, 64, 8, 128, [16384] * 24, 16)
     assert bf - (24 * (4 * 1024 + 4) + 2 * 24 * 64 * 128 * 2) == 1610612736
+
+
+def test_decode_step_bytes_low_bit_forms():
+    """2-bit codes and keys grouped per token, decomposed by hand per (sequence, kv head)
+    from the record layout: 16 x 32768 tokens, 8 kv heads, 32640 tokens in 510 blocks of
+    64 and 128 in the bf16 residual ring ([P-prod] "KV Cache 的基本内存模型": 0.25 byte
+    per value for 2-bit; the scale and zero-point bytes are the metadata that section says
+    makes the gain smaller)."""
+    meta = 16 * (4 * 510 + 4)                          # block-table entries + lengths
+    qo = 2 * 16 * 64 * 128 * 2                         # q read + out written, bf16
+    ring = 2 * 128 * 128 * 2                           # K and V ring rows
+    v_sz = 32640 * 2 * 2 * 2                           # V (scale, zero) per token, 2 groups
+    k_sz_chan = 510 * 2 * 128 * 2                      # KIVI K (scale, zero) per channel
+    k_sz_tok = 32640 * 2 * 2 * 2                       # K (scale, zero) per token, 2 groups
+    codes4, codes2 = 32640 * 128 // 2, 32640 * 128 // 4
+    assert (codes4, codes2, v_sz, k_sz_chan, k_sz_tok) == (2088960, 1044480, 261120, 261120, 261120)
+    cases = {
+        ("int4", "kivi"): 2 * codes4 + k_sz_chan + v_sz + ring,
+        ("int4", "kivi_float_zero"): 2 * codes4 + k_sz_chan + v_sz + ring,
+        ("int4", "int4_per_token"): 2 * codes4 + k_sz_tok + v_sz + ring,
+        ("int2", "kivi"): 2 * codes2 + k_sz_chan + v_sz + ring,
+        ("int2", "kivi_float_zero"): 2 * codes2 + k_sz_chan + v_sz + ring,
+        ("int2", "int4_per_token"): 2 * codes2 + k_sz_tok + v_sz + ring,
+    }
+    for (cd, mode), per_unit in cases.items():
+        got = bytes_model.decode_step_bytes(cd, mode, 16, 64, 8, 128, [32768] * 16, 64)
+        assert got == per_unit * 128 + meta + qo, (cd, mode)
+    assert cases[("int2", "kivi")] == 2676736
+    # short sequences: everything in the ring (n <= 128 + 63 keeps no whole group)
+    got = bytes_model.decode_step_bytes("int2", "int4_per_token", 2, 16, 2, 128, [100, 191], 64)
+    assert got == 2 * 2 * (100 + 191) * 128 * 2 + 2 * 4 + 2 * 16 * 128 * 4
+    # one group: 192 tokens -> 64 in a block, 128 in the ring
+    got = bytes_model.decode_step_bytes("int2", "kivi", 1, 8, 1, 128, [192], 64)
+    assert got == (2 * 64 * 32 + 2 * 128 * 2 + 64 * 2 * 4 + 2 * 128 * 128 * 2) + 4 + 4 + 8 * 128 * 4
+
+
+def test_bench_byte_counts_equal_the_oracle_model():
+    """The byte counts the benchmark divides by (the package's roofline module) equal the
+    oracle's model for every workload the benchmark runs, at full size and on a ragged
+    length mix."""
+    import random
+    import bench
+    from quantized_paged_kv_02_b200 import inputs, roofline
+    rng = random.Random(7)
+    for name in sorted(bench.WORKLOADS):
+        s = inputs._spec(name, False)
+        mixes = []
+        if s.lens:
+            mixes.append(s.lens)
+        else:
+            mixes.append([rng.randint(*s.len_range) for _ in range(s.batch)])
+        mixes.append([0, 1, 63, 64, 127, 128, 191, 192, 193, 1000, 4097])
+        for lens in mixes:
+            want = bytes_model.decode_step_bytes(s.cache_dtype, s.scale_mode, len(lens),
+                                                 s.num_q_heads, s.num_kv_heads, s.head_dim,
+                                                 lens, s.block_size)
+            got = roofline.decode_bytes(s.cache_dtype, s.scale_mode, s.num_q_heads,
+                                        s.num_kv_heads, s.head_dim, s.block_size, lens)
+            assert want.denominator == 1 and got == int(want), (name, lens)

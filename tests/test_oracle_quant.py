@@ -102,6 +102,28 @@ def test_fp8_calibration_and_saturation():
     np.testing.assert_array_equal(c, [[0x7E, 0xFE]])
 
 
+def test_head_calibration_exact_and_int8_static_round_trip():
+    """Per-head static scale: max over tokens and channels of |x| / qmax, one binary32
+    rounding of the exact quotient; with qmax 127 the warm-up's largest value gets code
+    +-127 exactly and every warm-up value stays inside the clamp."""
+    g = torch.Generator().manual_seed(4)
+    w = torch.randn(256, 3, 128, generator=g).to(torch.bfloat16).float().numpy()
+    for qmax in (127.0, 448.0):
+        s = quant.head_calibrate(w, qmax)
+        assert s.shape == (3,) and s.dtype == np.float32
+        for h in range(3):
+            m = np.max(np.abs(w[:, h, :]))
+            assert Fraction(float(s[h])) == exact_round(Fraction(float(m)) / Fraction(qmax), 24, -126)
+    np.testing.assert_array_equal(quant.head_calibrate(w, 448.0), quant.fp8_calibrate(w))
+    s = quant.head_calibrate(w, 127.0)
+    for h in range(3):
+        c = quant.int8_quantize(w[:, h, :].reshape(1, -1), s[h:h + 1])
+        assert np.max(np.abs(c.astype(np.int64))) == 127
+    # an all-zero head gives scale 0
+    z = np.zeros((8, 2, 64), np.float32)
+    np.testing.assert_array_equal(quant.head_calibrate(z, 127.0), [0.0, 0.0])
+
+
 def test_fp8_quantize_is_nearest_code():
     g = torch.Generator().manual_seed(5)
     x = torch.randn(64, 128, generator=g).to(torch.bfloat16).float().numpy()
