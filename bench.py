@@ -83,6 +83,9 @@ def parse():
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--min-warmup-s", type=float, default=1.0,
                     help="keep warming up for at least this many seconds")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only chunked prefill on the workload's cache type (--batch "
+                         "sequences of 4096 tokens, 512-query chunks; for profiling)")
     return ap.parse_args()
 
 
@@ -131,21 +134,17 @@ def tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def measure_prefill(device, l2, steps=20):
-    """Chunked prefill on a c5-shaped layer (INT8 per-token-head cache, 64/8 heads, D 128,
-    block 16): 4 sequences of 4096 cached tokens whose newest 512 are this chunk's queries,
-    each attending causally.  Algorithmic work: 4 D flops (q.k and p.v) per query head and
-    visible position."""
-    import dataclasses
+def measure_prefill(device, l2, workload="c5", steps=20, batch=4, n=4096, chunk=512):
+    """Chunked prefill on a layer of the named workload's cache type and heads (c5: INT8
+    per-token-head, 64/8 heads, D 128, block 16): `batch` sequences of n cached tokens whose
+    newest `chunk` are this chunk's queries, each attending causally
+    (kvq_prefill_attention).  Algorithmic work: 4 D flops (q.k and p.v) per query head and
+    visible position; throughput against the measured dense bf16 tensor peak."""
     import torch
-    from quantized_paged_kv_02_b200 import inputs, kvq
-    spec = dataclasses.replace(inputs._spec("c5", False), batch=4, lens=[4096] * 4)
-    w = inputs.from_spec(spec, device)
+    from quantized_paged_kv_02_b200 import kvq
+    w, c, _, _ = build_state(workload, device, 0, batch=batch, lens=[n] * batch)
     s = w.spec
-    c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
-                         s.num_kv_heads, s.head_dim, device=device)
-    c.write(w.k, w.v, w.slot_mapping)
-    L, n = 512, 4096
+    L = chunk
     g = torch.Generator(device=device).manual_seed(1)
     q = torch.randn((s.batch * L, s.num_q_heads, s.head_dim), generator=g, device=device).to(torch.bfloat16)
     qs = torch.arange(0, s.batch * L + 1, L, dtype=torch.int32, device=device)
@@ -168,10 +167,16 @@ def measure_prefill(device, l2, steps=20):
     flops = 4.0 * s.head_dim * s.num_q_heads * visible
     peak, kind = tensor_peak()
     tf = flops / (ms * 1e-3) / 1e12
-    return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
-            "frac_of_peak": round(tf / peak, 4), "peak": peak, "peak_kind": kind + " bf16 dense",
-            "config": "c5-shaped layer, INT8 per-token-head cache, 4 sequences x 4096 tokens, "
-                      "512-query causal chunks (kvq_prefill_attention)"}
+    res = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+           "frac_of_peak": round(tf / peak, 4), "peak": peak, "peak_kind": kind + " bf16 dense",
+           "flops_per_call": flops,
+           "config": "%s layer (%s %s cache, %d/%d heads, head_dim %d, block %d), %d sequences x "
+                     "%d tokens, %d-query causal chunks (kvq_prefill_attention)"
+                     % (workload, s.cache_dtype, s.scale_mode, s.num_q_heads, s.num_kv_heads,
+                        s.head_dim, s.block_size, s.batch, n, L)}
+    del w, c, q, out
+    torch.cuda.empty_cache()
+    return res
 
 
 def profile_traffic(workload):
@@ -412,15 +417,16 @@ def run_oracle_sample(workload, budget_s=10.0):
 
 
 # ----------------------------------------------------------------------------- ours
-def build_state(workload, device, seed, batch=0):
+def build_state(workload, device, seed, batch=0, lens=None):
     import dataclasses
     import torch
     from quantized_paged_kv_02_b200 import inputs, kvq
     spec = inputs._spec(workload, False)
     spec.seed = seed
     if batch:
-        lens = spec.lens[:1] * batch if spec.lens else None
-        spec = dataclasses.replace(spec, batch=batch, lens=lens)
+        if lens is None:
+            lens = spec.lens[:1] * batch if spec.lens else None
+        spec = dataclasses.replace(spec, batch=batch, lens=lens, len_range=None if lens else spec.len_range)
     w = inputs.from_spec(spec, device)
     s = w.spec
     static = None
@@ -602,6 +608,12 @@ def main_ours(args):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.prefill_only:
+        r = measure_prefill(device, L2Flush(device), workload=args.workload,
+                            steps=max(1, args.steps), batch=args.batch or 4)
+        if rank == 0:
+            print(json.dumps({"prefill": r, "note": "profiling run, not a benchmark line"}), flush=True)
+        return
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -690,8 +702,14 @@ def main_ours(args):
                  "frac_of_peak": round(step_bytes / (fms * 1e-3) / 1e9 / hbm_peak()[0], 4),
                  "call": "kvq_append_decode_attention (append step fused into the decode kernel)"}
 
-    # chunked prefill on its own c5-shaped case (default workload only)
-    prefill = measure_prefill(device, l2) if args.workload == "c5" and K > 0 else None
+    # chunked prefill on its own cases (default workload only): the c5-shaped INT8 layer is
+    # the headline; FP8, bf16 and INT4 caches of the same shapes beside it
+    prefill = prefill_more = None
+    if args.workload == "c5" and K > 0 and not args.batch:
+        prefill = measure_prefill(device, l2)
+        if world == 1:
+            prefill_more = {key: measure_prefill(device, l2, workload=name)
+                            for key, name in (("c5_fp8", "c5-fp8"), ("c5_bf16", "c5-bf16"), ("c4", "c4"))}
 
     # end to end through the C ABI: the step's inputs (new K/V rows, slots, q, lengths) packed
     # in one pinned host buffer and copied to the device in one transfer inside the timed
@@ -786,6 +804,7 @@ def main_ours(args):
                         ", one packed host-to-device copy of the step's inputs, output copied back"},
         "append_decode": fused,
         "prefill": prefill,
+        "prefill_configs": prefill_more,
         "configs": configs,
         "write_prefill": write_prefill,
         "gpu_launches": launches_per_step * K,

@@ -267,9 +267,9 @@ kvq_status kvq_decode_workspace_size(const kvq_cache_desc* cache, int batch,
  * only: no device access, no launch; the pages give no counterpart, it reports this
  * library's dispatch).  Any output pointer may be NULL.
  *   kernel_out    0: the CUDA-core split kernel; 1: the page-balanced tensor-core kernel
- *                 (dense caches; it merges its own partials); 2: the low-bit (INT4 / INT2)
- *                 tensor-core block kernel plus the CUDA-core kernel for the residual ring.
- *   launches_out  kernels one call launches, the merge included (1: 1; 2: 3; 0: 1, or 2
+ *                 (dense caches); 2: the low-bit (INT4 / INT2) tensor-core block kernel
+ *                 plus the CUDA-core kernel for the residual ring.
+ *   launches_out  kernels one call launches, the merge included (1: 2; 2: 3; 0: 1, or 2
  *                 with more than one split; 0 when batch is 0).
  *   splits_out    token splits of kernels 0 and 2 (the ring counted as one); for kernel 1,
  *                 its CTA count (the page ranges).
@@ -293,18 +293,13 @@ kvq_status kvq_decode_plan(const kvq_cache_desc* cache, int batch, int num_q_hea
  *   softmax_scale 0 selects 1/sqrt(D) ([P-mem] §6 Q1 writes softmax(q k^T / sqrt(d))).
  *   out           out_dtype [batch][num_q_heads][D], device; out_dtype BF16, FP16 or FP32.
  *   workspace     device scratch of at least kvq_decode_workspace_size() bytes (may be
- *                 NULL when that size is 0).  Its contents need no initialisation: the
- *                 tensor-core kernel's per-(sequence, kv head) arrival counters in it carry
- *                 a tag of the call that wrote them, and a counter with another call's tag
- *                 counts as empty (each call leaves its counters empty when it completes).
- *                 Two calls that overlap on the GPU must not share a workspace.
+ *                 NULL when that size is 0).  Its contents need no initialisation; two
+ *                 calls that overlap on the GPU must not share a workspace.
  *   For each (b, hq): o = sum_p softmax_p(scale * q . k_p) v_p over p < context_lens[b],
  *   where k_p, v_p are the dequantized cache rows; for INT4 / INT2, positions p < Qb come
  *   from blocks and the rest from the residual ring, Qb = 64*floor(max(len-residual_len,0)/64).
  *   Dequantization happens inside the kernel ([P-vLLM] "PagedAttention与KV Cache量化协同
- *   工作原理"); long contexts are split across CTAs and merged by a log-sum-exp reduce (on
- *   the tensor-core kernel, by the last warp to finish a part of each (sequence, kv head),
- *   inside the same launch).
+ *   工作原理"); long contexts are split across CTAs and merged by a log-sum-exp reduce.
  *   Kernels: head_dim 128 with block_size 16 and 1..8 query heads per kv head runs on the
  *   tensor-core kernel (dense caches); INT4 / INT2 with head_dim 128 and 3..8 query heads per
  *   kv head on the low-bit tensor-core kernel; everything else on the CUDA-core kernel.
@@ -360,8 +355,15 @@ kvq_status kvq_append_decode_attention(const kvq_cache_desc* cache, const void* 
  *   p = context_lens[b] - L_b + i (L_b its query count) and attends to positions <= p:
  *   o = softmax(scale * q . k_t) v_t over t <= p, dequantized inside the kernel.  Chunked
  *   prefill is one of the techniques [P-prod] "为什么长上下文更需要 KV Cache Quantization"
- *   names beside KV cache quantization.  Dense caches with block_size 16 and head_dim 128
- *   (the tensor-core path); others return KVQ_ERR_UNSUPPORTED.  No workspace.
+ *   names beside KV cache quantization.  No workspace.
+ *   Supported: head_dim 128 with dense caches of block_size 16, and INT4 / INT2 caches
+ *   (block_size 64).  For INT4 / INT2 the cache is read as it stands after the chunk was
+ *   written: positions below Qb = 64*floor(max(context_lens[b] - residual_len, 0)/64) from
+ *   blocks, the rest from ring sequence b.  GQA groups of 1, 2, 4, 8 (any divisor of 128)
+ *   query heads per kv head run on the 5th-generation tensor cores (tiles of 128 query rows,
+ *   each page dequantized once per tile); other groups of up to 8 on the dense tensor-core
+ *   decode kernel's per-query mode (dense caches only).  Anything else returns
+ *   KVQ_ERR_UNSUPPORTED.
  */
 kvq_status kvq_prefill_attention(const kvq_cache_desc* cache, const void* q, int num_q_tokens,
                                  int batch, int num_q_heads, const int32_t* q_start,

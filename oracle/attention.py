@@ -54,7 +54,8 @@ def decode_attention(cache, q, block_tables, context_lens, seq_ids=None,
     return out
 
 
-def prefill_attention(cache, q, q_start, block_tables, context_lens, softmax_scale=0.0):
+def prefill_attention(cache, q, q_start, block_tables, context_lens, softmax_scale=0.0,
+                      seq_ids=None):
     """Causal attention of a chunk of new queries over the dequantized cache, float64.
 
     q [Tq, H_q, D]; the queries of sequence b are rows q_start[b] .. q_start[b+1]-1, the
@@ -63,7 +64,9 @@ def prefill_attention(cache, q, q_start, block_tables, context_lens, softmax_sca
         z_t = scale * (q . k_t), t <= p;   o = softmax(z) V
     (chunked prefill, one of the techniques [P-prod] "为什么长上下文更需要 KV Cache
     Quantization" lists beside KV cache quantization; the chunk's own K/V rows are in the
-    cache before attention runs).  Returns [Tq, H_q, D]; one query row at a time.
+    cache before attention runs).  For INT4 / 2-bit caches the newest positions come from
+    ring sequence seq_ids[b] (b when seq_ids is None), as in decode.  Returns [Tq, H_q, D];
+    one query row at a time.
     """
     q = np.asarray(q, np.float64)
     Tq, Hq, D = q.shape
@@ -76,7 +79,7 @@ def prefill_attention(cache, q, q_start, block_tables, context_lens, softmax_sca
         L = int(qs[b + 1] - qs[b])
         if L == 0:
             continue
-        K, V = cache.gather(block_tables[b], n)
+        K, V = cache.gather(block_tables[b], n, b if seq_ids is None else int(seq_ids[b]))
         for i in range(L):
             p = n - L + i
             for hq in range(Hq):

@@ -1,6 +1,5 @@
 // C ABI entry points: host-side validation, layout arithmetic and dispatch.
 // Declarations and the contract of every call are in include/kvq.h.
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -97,16 +96,6 @@ using namespace kvq;
 
 namespace {
 
-// Tag of one decode call's arrivals on the per-unit counters of the workspace.  A counter
-// holding another call's tag (left by a call that stopped early) counts as empty, so the
-// workspace needs no clearing between calls.  0 is never used.
-uint32_t next_epoch() {
-  static std::atomic<uint32_t> counter{0};
-  uint32_t e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
-  if (e == 0) e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
-  return e;
-}
-
 // Shared by kvq_decode_attention and kvq_append_decode_attention (k_new / v_new null for
 // the former).
 kvq_status decode_entry(const kvq_cache_desc* c, const void* k_new, const void* v_new,
@@ -143,10 +132,7 @@ kvq_status decode_entry(const kvq_cache_desc* c, const void* k_new, const void* 
       return KVQ_ERR_INVALID_ARG;
     a.ws_o = static_cast<float*>(workspace);
     a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + a.plan.ws_ml_off);
-    if (a.plan.kernel == 1)
-      a.ws_cnt = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + a.plan.ws_cnt_off);
   }
-  a.epoch = next_epoch();
   a.q = q;
   a.k_new = k_new;
   a.v_new = v_new;
@@ -226,9 +212,9 @@ kvq_status kvq_decode_plan(const kvq_cache_desc* c, int batch, int num_q_heads, 
   DecodePlan p;
   st = plan_decode(g, batch, num_q_heads, max_context, &p);
   if (st != KVQ_OK) return st;
-  // the launches of launch_decode: kernel 1 (it merges its own partials); INT4/INT2 blocks +
-  // ring kernel + split reduce; CUDA-core kernel (+ split reduce when it splits)
-  int launches = p.kernel == 1 ? 1 : p.kernel == 2 ? 3 : (p.splits > 1 ? 2 : 1);
+  // the launches of launch_decode: kernel 1 + segment merge; INT4/INT2 blocks + ring kernel +
+  // split reduce; CUDA-core kernel (+ split reduce when it splits)
+  int launches = p.kernel == 1 ? 2 : p.kernel == 2 ? 3 : (p.splits > 1 ? 2 : 1);
   if (batch == 0) launches = 0;                       // nothing to do: nothing launched
   if (kernel_out) *kernel_out = p.kernel;
   if (launches_out) *launches_out = launches;
@@ -325,8 +311,11 @@ kvq_status kvq_prefill_attention(const kvq_cache_desc* c, const void* q, int num
   a.c = c;
   a.geo = g;
   st = plan_decode(g, std::max(batch, 1), num_q_heads, max_context, &a.plan);
-  if (st != KVQ_OK) return st;
-  if (a.plan.kernel != 1) return KVQ_ERR_UNSUPPORTED;     // tensor-core geometries only
+  if (st != KVQ_ERR_UNSUPPORTED && st != KVQ_OK) return st;
+  // the tcgen05 kernel (head_dim 128, block 16 dense / 64 low-bit, GQA groups dividing 128),
+  // else the warp-per-query mode of the dense tensor-core decode kernel
+  a.plan.g = num_q_heads / g.H;
+  if (!prefill_tc_supported(g, a.plan.g) && (st != KVQ_OK || a.plan.kernel != 1)) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0 || num_q_tokens == 0 || max_q_len == 0) return KVQ_OK;
   if (q == nullptr || q_start == nullptr || block_tables == nullptr || context_lens == nullptr ||
       out == nullptr)

@@ -1,5 +1,4 @@
-// Decode dispatch: split plan, kernel choice, and the split-K log-sum-exp reduce of the
-// CUDA-core and low-bit kernels (the dense tensor-core kernel merges its own partials).
+// Decode dispatch: split plan, kernel choice, and the split-K log-sum-exp reduce.
 //
 // The reduce merges the S partials (m_s, l_s, o_s) of each (sequence, query head):
 //   M = max_s m_s,  L = sum_s l_s 2^(m_s - M),  out = sum_s o_s 2^(m_s - M) / L,
@@ -70,6 +69,120 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
   }
 }
 
+// Merge of the dense tensor-core kernel's per-warp partials.  One warp per (sequence,
+// query head): it recomputes the page partition (total pages, the pages before its
+// sequence), finds the CTAs whose ranges meet its unit's pages, and takes the partial of
+// every consumer warp that saw at least one of those pages.  Lane k describes candidate
+// k (CTA c_first + k / kSegWarps, warp k % kSegWarps); the partial rows are then read
+// sixteen at a time so their loads overlap.
+__global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
+  const int C = p.ctas;
+  griddep_wait();                      // the partials of the decode kernel
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);   // b * Hq + hq
+  const int lane = threadIdx.x & 31;
+  if (row >= p.rows) return;
+  const int b = row / p.Hq, hq = row - b * p.Hq;
+  const int kvh = hq / p.g, h = hq - kvh * p.g;
+  long long tot = 0, before = 0;
+  int npb = 0;
+  for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    const int bb = b0 + lane;
+    const int np = bb < p.batch ? seq_pages(p, bb) : 0;
+    int t = np, q = bb < b ? np : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      t += __shfl_xor_sync(0xffffffffu, t, off);
+      q += __shfl_xor_sync(0xffffffffu, q, off);
+    }
+    tot += t;
+    before += q;
+    if (b >= b0 && b < b0 + 32) npb = __shfl_sync(0xffffffffu, np, b - b0);
+  }
+  const long long P = tot * p.H;
+  const long long U0 = before * p.H + static_cast<long long>(kvh) * npb, U1 = U0 + npb;
+  int c_first = 0, c_last = -1;
+  if (npb > 0) {
+    // CTA c covers [P c / C, P (c+1) / C): the last one starting at or before U0, and
+    // the last one starting before U1
+    c_first = static_cast<int>(((U0 + 1) * C + P - 1) / P) - 1;
+    c_last = static_cast<int>((U1 * C + P - 1) / P) - 1;
+  }
+  const int K = (c_last - c_first + 1) * kSegWarps;
+  const long long u = static_cast<long long>(b) * p.H + kvh;
+  const float* ml = p.ws_ml;
+  const float* o = p.ws_o + 4 * lane;
+  const bool has_d = 4 * lane < p.D;
+  float M = -INFINITY, L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    // lane k: does candidate k0 + k hold a partial, and where
+    const int k = k0 + lane;
+    int slot = -1;
+    float mk = -INFINITY, lk = 0.f;
+    if (k < K) {
+      const int c = c_first + k / kSegWarps, w = k % kSegWarps;
+      const long long sc = range_start(P, c, C), ec = range_start(P, c + 1, C);
+      const long long lo = sc > U0 ? sc : U0, hi = ec < U1 ? ec : U1;
+      const long long len = hi - lo;
+      const int first = static_cast<int>((lo - sc) % kSegWarps);   // warp of the first page
+      if (len > 0 && (len >= kSegWarps || ((w - first + kSegWarps) % kSegWarps) < len)) {
+        slot = static_cast<int>(((u + c) * kSegWarps + w) * p.g + h);
+        const float2 v = *reinterpret_cast<const float2*>(ml + 2L * slot);
+        mk = v.x;
+        lk = v.y;
+      }
+    }
+    // rescale what was merged so far to the new maximum
+    float Mc = mk;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
+    const float Mn = fmaxf(M, Mc);
+    if (Mn != -INFINITY && Mn > M) {
+      const float c0 = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      L *= c0;
+      acc.x *= c0; acc.y *= c0; acc.z *= c0; acc.w *= c0;
+      M = Mn;
+    }
+    const float w = (slot >= 0 && mk != -INFINITY) ? exp2f(mk - M) : 0.f;
+    L = fmaf(lk, w, L);
+    const int n = min(32, K - k0);
+    constexpr int kRows = 16;          // partial rows in flight per lane
+    for (int i0 = 0; i0 < n; i0 += kRows) {
+      float wi[kRows];
+      int si[kRows];
+      float4 v[kRows];
+#pragma unroll
+      for (int t = 0; t < kRows; ++t) {
+        const int i = min(i0 + t, 31);
+        wi[t] = __shfl_sync(0xffffffffu, w, i);
+        si[t] = __shfl_sync(0xffffffffu, slot, i);
+        if (i0 + t >= n) wi[t] = 0.f;
+      }
+#pragma unroll
+      for (int t = 0; t < kRows; ++t)
+        v[t] = (has_d && wi[t] != 0.f) ? *reinterpret_cast<const float4*>(o + static_cast<long>(si[t]) * p.D)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int t = 0; t < kRows; ++t) {
+        acc.x = fmaf(v[t].x, wi[t], acc.x);
+        acc.y = fmaf(v[t].y, wi[t], acc.y);
+        acc.z = fmaf(v[t].z, wi[t], acc.z);
+        acc.w = fmaf(v[t].w, wi[t], acc.w);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (has_d) {
+    const long base = static_cast<long>(row) * p.D + 4 * lane;
+    store_out(p, base, acc.x * inv);
+    store_out(p, base + 1, acc.y * inv);
+    store_out(p, base + 2, acc.z * inv);
+    store_out(p, base + 3, acc.w * inv);
+  }
+}
+
 }  // namespace
 
 // Splits for the INT4 tensor-core kernel: one CTA per (sequence, kv head, split); pick the
@@ -108,7 +221,6 @@ int device_sm_count() {
 kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_context,
                        DecodePlan* p) {
   p->sms = device_sm_count();
-  p->ws_cnt_off = 0;
   p->g = num_q_heads / g.H;
   p->kernel = mma_supported(g, p->g) ? 1 : 0;
   // per-channel scales are folded into q and the output by the tensor-core kernel only
@@ -130,18 +242,15 @@ kvq_status plan_decode(const Geometry& g, int batch, int num_q_heads, int max_co
     return KVQ_OK;
   }
   if (p->kernel == 1) {
-    // page-balanced CTAs; partial slots (unit + cta) * kSegWarps + warp, g heads each,
-    // then one 64-bit arrival counter per unit
+    // page-balanced CTAs; partial slots (unit + cta) * kSegWarps + warp, g heads each
     p->g_tile = p->g;
     p->splits = 0;
     p->chunk = 0;
     p->ctas = kMmaCtasPerSM * p->sms;
-    const size_t units = static_cast<size_t>(batch) * g.H;
-    const size_t slots = (units + p->ctas - 1) * kSegWarps;
+    const size_t slots = (static_cast<size_t>(batch) * g.H + p->ctas - 1) * kSegWarps;
     const size_t heads = slots * p->g;
     p->ws_ml_off = (heads * g.D * sizeof(float) + 255) / 256 * 256;
-    p->ws_cnt_off = (p->ws_ml_off + heads * 2 * sizeof(float) + 255) / 256 * 256;
-    p->ws_bytes = p->ws_cnt_off + units * sizeof(unsigned long long);
+    p->ws_bytes = p->ws_ml_off + heads * 2 * sizeof(float);
     return KVQ_OK;
   }
   p->g_tile = (p->g % 2 == 0) ? 2 : 1;
@@ -207,8 +316,6 @@ static DecodeParams make_params(const DecodeArgs& a) {
   p.out_dtype = a.out_dtype;
   p.ws_o = a.ws_o;
   p.ws_ml = a.ws_ml;
-  p.ws_cnt = a.ws_cnt;
-  p.epoch = a.epoch;
   p.fault = a.c->fault;
   p.k_new = a.k_new;
   p.v_new = a.v_new;
@@ -230,7 +337,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     e = a.plan.kernel == 1 ? launch_decode_mma(a, p, s) : launch_decode_simt(a, p, s);
   }
   if (e != cudaSuccess) return e;
-  if (a.plan.kernel != 1 && p.splits > 1) {
+  if (a.plan.kernel == 1) {
+    e = launch_dependent(segment_reduce_kernel, dim3((a.batch * a.Hq + 7) / 8), dim3(256), 0, s, p);
+  } else if (p.splits > 1) {
     split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, low_bit(g.cache_dtype));
     e = cudaGetLastError();
   }
@@ -239,6 +348,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
 
 cudaError_t launch_prefill(const DecodeArgs& a, cudaStream_t s) {
   if (a.batch == 0) return cudaSuccess;
+  if (prefill_tc_supported(a.geo, a.plan.g)) return launch_prefill_tc(a, make_params(a), s);
   return launch_prefill_mma(a, make_params(a), s);
 }
 

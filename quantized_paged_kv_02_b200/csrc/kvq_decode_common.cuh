@@ -31,8 +31,6 @@ struct DecodeParams {
   int out_dtype;
   float* ws_o;               // [B][Hq][S][D]
   float* ws_ml;              // [B][Hq][S][2]  (max, sum) in the log2 domain
-  unsigned long long* ws_cnt;  // dense tensor-core kernel: [B*H] arrival counters
-  uint32_t epoch;            // dense tensor-core kernel: this call's tag (never 0)
   int32_t* fault;
   // append step (kvq_append_decode_attention), else null: this step's K / V row of every
   // sequence, [B][H][D] act dtype, stored at position context_lens[b] - 1 before decode
@@ -88,7 +86,7 @@ __device__ __forceinline__ SeqInfo seq_info(const DecodeParams& p, int b, bool i
 // (unit, CTA); each consumer warp of the CTA writes one partial per segment it saw, into
 // slot (unit + c) * kSegWarps + warp.  (Going from one segment to the next raises the unit
 // index, the CTA index or both, so unit + c never repeats and there are at most
-// units + C - 1 segments.)  The last warp to write a partial of a unit merges them all.
+// units + C - 1 segments.)  The segment reduce merges them.
 constexpr int kSegWarps = 4;
 constexpr int kMmaCtasPerSM = 3;
 
@@ -145,6 +143,10 @@ __device__ __forceinline__ void store_partial_or_output(const DecodeParams& p, i
 cudaError_t launch_decode_simt(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_prefill_mma(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
+// chunked prefill on tcgen05 (128-row query tiles): head_dim 128, block 16, dense caches,
+// GQA groups dividing 128
+bool prefill_tc_supported(const Geometry& g, int group);
+cudaError_t launch_prefill_tc(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 // true when the tensor-core kernel covers this geometry and GQA group size
 bool mma_supported(const Geometry& g, int group);
 bool int4_mma_supported(const Geometry& g, int group);

@@ -4,10 +4,8 @@
 // Schedule: one CTA per resident slot (3 per SM).  The pages of all (sequence, kv head)
 // units, concatenated, are cut into equal contiguous ranges, one per CTA, so every CTA
 // streams the same number of bytes whatever the mix of context lengths, and a CTA's copy
-// pipeline never drains between units.  Every consumer warp that saw pages of a unit
-// writes a partial (O, max, sum) and counts itself on the unit's arrival counter; the last
-// one to arrive merges the unit's partials (log-sum-exp) and writes the output rows, so a
-// decode call is one launch.
+// pipeline never drains between units.  A unit that straddles CTA ranges is finished by
+// the segment reduce (log-sum-exp merge of the per-warp partials).
 //
 // Within a CTA, warp 4 is the producer: it walks the block tables of its range and moves
 // each block's page record (K codes, V codes and per-token scales, contiguous in the
@@ -24,8 +22,7 @@
 // O^T += V^T P^T is a second mma.sync with P split into hi + lo halves (P changes
 // fragment layout in registers with movmatrix).  Per-token V scales are folded into P
 // with a per-warp power-of-two normaliser.  When the unit changes, the warp writes its
-// partial (O, max, sum) to the workspace, arrives on the unit's counter (merging the unit
-// if it is the last) and loads the next query group.
+// partial (O, max, sum) to the workspace and loads the next query group.
 //
 // Dequantization is fused into both contractions ([P-vLLM]
 // "PagedAttention与KV Cache量化协同工作原理"); the split covers long contexts, whose decode
@@ -68,12 +65,11 @@ struct Layout {
   // ring depth: as many stages as fit the shared memory of 3 CTAs per SM (228 KiB per SM,
   // 1 KiB of it reserved per CTA); bytes in flight are what keeps HBM busy
   static constexpr int kSmemPerCta = 228 * 1024 / 3 - 1024;
-  static constexpr int kFixed = 1024 + 16 + 4 * 4 + 32 * 4 + 16 + 16 * kConsumers;
+  static constexpr int kFixed = 1024 + 16 + 4 * 4 + 32 * 4;  // alignment, range, batch ids
   static constexpr int kStages = (kSmemPerCta - kFixed) / (STAGE + 32) / kConsumers * kConsumers;
   static constexpr int TILES = kStages * STAGE;
   static constexpr int BARS = kStages * 2 * 8;
-  // page records, range, batch ids, range start and total, each consumer's unit pages
-  static constexpr int META = kStages * 16 + 16 + 32 * 4 + 16 + 16 * kConsumers;
+  static constexpr int META = kStages * 16 + 16 + 32 * 4;  // page records, range, batch ids
   static constexpr int BYTES = 1024 + TILES + BARS + META;
   static_assert(kStages >= 4 && BYTES <= kSmemPerCta, "ring fits 3 CTAs per SM");
   // Consumers take pages round-robin, and every round of a stage must go to the same
@@ -88,126 +84,6 @@ struct Layout {
 // chunk index is XORed with the 128-byte row index (mod 8).
 __device__ __forceinline__ int swzb(int off) {
   return (off & ~127) + ((((off >> 4) & 7) ^ ((off >> 7) & 7)) << 4) + (off & 15);
-}
-
-// Counts one arrival on a unit's counter: (tag << 32) | arrivals, where a tag other than this
-// call's epoch counts as no arrivals yet (a call that stopped early leaves its count behind).
-// Returns the arrivals including this one, or -1 if the update kept failing (it cannot,
-// since each failure means another arrival succeeded; the bound only keeps the loop finite).
-__device__ __forceinline__ int arrive(unsigned long long* cell, uint32_t epoch) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(cell);
-  for (int it = 0; it < (1 << 16); ++it) {
-    const unsigned long long nxt = static_cast<uint32_t>(cur >> 32) == epoch
-                                       ? cur + 1
-                                       : (static_cast<unsigned long long>(epoch) << 32) | 1ull;
-    const unsigned long long prev = atomicCAS(cell, cur, nxt);
-    if (prev == cur) return static_cast<int>(nxt & 0xffffffffull);
-    cur = prev;
-  }
-  return -1;
-}
-
-// The CTAs whose ranges meet unit pages [U0, U1): c_first is the last CTA starting at or
-// before U0, c_last the last one starting before U1 (CTA c covers [P c / C, P (c+1) / C)).
-// Lane-parallel count of the consumer warps that saw at least one page of the unit: a CTA
-// whose range meets the unit in len pages hands them to min(len, kSegWarps) warps.
-__device__ __forceinline__ int unit_contributors(long long U0, long long U1, long long P, int C,
-                                                 int lane, int* c_first, int* c_last) {
-  const int c0 = static_cast<int>(((U0 + 1) * C + P - 1) / P) - 1;
-  const int c1 = static_cast<int>((U1 * C + P - 1) / P) - 1;
-  int n = 0;
-  for (int cb = c0; cb <= c1; cb += 32) {
-    const int c = cb + lane;
-    if (c <= c1) {
-      const long long sc = range_start(P, c, C), ec = range_start(P, c + 1, C);
-      const long long len = min(ec, U1) - max(sc, U0);
-      n += static_cast<int>(min(len, static_cast<long long>(kSegWarps)));
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
-  *c_first = c0;
-  *c_last = c1;
-  return n;
-}
-
-// Log-sum-exp merge of every partial of unit u (pages [U0, U1)) into its g output rows,
-// by one warp: for each head, lane k weighs candidate k (CTA c_first + k / kSegWarps,
-// warp k % kSegWarps, kept when that warp saw a page of the unit), then the lanes, 4
-// channels each, sum the weighted partial rows, sixteen rows in flight.  Partials are read
-// from L2 (other SMs wrote them).
-__device__ __forceinline__ void merge_unit(const DecodeParams& p, long long u, long long U0, long long U1,
-                                        long long P, int C, int c_first, int c_last, int lane) {
-  const int g = p.g;
-  const int b = static_cast<int>(u / p.H), kvh = static_cast<int>(u - static_cast<long long>(b) * p.H);
-  const int K = (c_last - c_first + 1) * kSegWarps;
-  for (int h = 0; h < g; ++h) {
-    float M = -INFINITY, L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k0 = 0; k0 < K; k0 += 32) {
-      const int k = k0 + lane;
-      long slot = -1;
-      float mk = -INFINITY, lk = 0.f;
-      if (k < K) {
-        const int c = c_first + k / kSegWarps, w = k % kSegWarps;
-        const long long sc = range_start(P, c, C), ec = range_start(P, c + 1, C);
-        const long long lo = sc > U0 ? sc : U0, hi = ec < U1 ? ec : U1;
-        const long long len = hi - lo;
-        const int first = static_cast<int>((lo - sc) % kSegWarps);   // warp of the first page
-        if (len > 0 && (len >= kSegWarps || ((w - first + kSegWarps) % kSegWarps) < len)) {
-          slot = ((u + c) * kSegWarps + w) * g + h;
-          const float2 v = __ldcg(reinterpret_cast<const float2*>(p.ws_ml + 2 * slot));
-          mk = v.x;
-          lk = v.y;
-        }
-      }
-      float Mc = mk;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
-      const float Mn = fmaxf(M, Mc);
-      if (Mn != -INFINITY && Mn > M) {
-        const float c0 = M == -INFINITY ? 0.f : exp2f(M - Mn);
-        L *= c0;
-        acc.x *= c0; acc.y *= c0; acc.z *= c0; acc.w *= c0;
-        M = Mn;
-      }
-      const float w = (slot >= 0 && mk != -INFINITY) ? exp2f(mk - M) : 0.f;
-      L = fmaf(lk, w, L);
-      const int n = min(32, K - k0);
-      constexpr int kRows = 16;
-      for (int i0 = 0; i0 < n; i0 += kRows) {
-        float wi[kRows];
-        long si[kRows];
-        float4 v[kRows];
-#pragma unroll
-        for (int t = 0; t < kRows; ++t) {
-          const int i = min(i0 + t, 31);
-          wi[t] = __shfl_sync(0xffffffffu, w, i);
-          si[t] = __shfl_sync(0xffffffffu, slot, i);
-          if (i0 + t >= n) wi[t] = 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < kRows; ++t)
-          v[t] = wi[t] != 0.f ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + si[t] * kD) + lane)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int t = 0; t < kRows; ++t) {
-          acc.x = fmaf(v[t].x, wi[t], acc.x);
-          acc.y = fmaf(v[t].y, wi[t], acc.y);
-          acc.z = fmaf(v[t].z, wi[t], acc.z);
-          acc.w = fmaf(v[t].w, wi[t], acc.w);
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    const long base = (static_cast<long>(b) * p.Hq + static_cast<long>(kvh) * g + h) * kD + 4 * lane;
-    store_out(p, base, acc.x * inv);
-    store_out(p, base + 1, acc.y * inv);
-    store_out(p, base + 2, acc.z * inv);
-    store_out(p, base + 3, acc.w * inv);
-  }
 }
 
 // PF false: decode, grid p.ctas over page-balanced ranges.  PF true: chunked prefill,
@@ -232,8 +108,6 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   int4* meta = reinterpret_cast<int4*>(empty + kStages);   // per stage: unit, page, tokens, valid
   int* range_pages = reinterpret_cast<int*>(meta + kStages);
   int* ids = range_pages + 4;                               // producer: block ids of a batch
-  long long* range_at = reinterpret_cast<long long*>(ids + 32);   // range start, page total
-  long long* unit_at = range_at + 2;      // consumer w: pages [U0, U1) of its unit at [2w, 2w+1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.ctas;                                    // the grid (page partition)
   const int cta = blockIdx.x;
@@ -277,11 +151,7 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     seq_first_page = 0;                         // unit (b, kvh) starts at kvh * npb
     start = static_cast<long long>(pf_kvh) * npb;
     end = start + (last + BS) / BS;
-    if (warp == kConsumers && lane == 0) {
-      *range_pages = static_cast<int>(end - start);
-      range_at[0] = start;
-      range_at[1] = 0;                          // no merge in prefill
-    }
+    if (warp == kConsumers && lane == 0) *range_pages = static_cast<int>(end - start);
   } else if (warp == kConsumers) {
     long long tot = 0;
     for (int b0 = 0; b0 < p.batch; b0 += 32) {
@@ -312,11 +182,7 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       }
       pre += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      *range_pages = static_cast<int>(end - start);
-      range_at[0] = start;
-      range_at[1] = P;
-    }
+    if (lane == 0) *range_pages = static_cast<int>(end - start);
   }
   __syncthreads();
 
@@ -443,14 +309,6 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   // ---------------------------------------------------------------- consumers
   const int npages = *range_pages;
   const int g = p.g;
-  if constexpr (!PF) {
-    // sequences with no page (empty or rejected) get zero output rows here
-    for (int b = cta * kConsumers + warp; b < p.batch; b += C * kConsumers) {
-      if (seq_pages(p, b) == 0) {
-        for (int i = lane; i < p.Hq * kD; i += 32) store_out(p, static_cast<long>(b) * p.Hq * kD + i, 0.f);
-      }
-    }
-  }
   const int r = lane >> 2, j = lane & 3;
   float o[8][4];
   float m[2], l[2];
@@ -599,23 +457,6 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       if (h0 < g) *reinterpret_cast<float2*>(wml + 2 * h0) = make_float2(m[0], l[0]);
       if (h1 < g) *reinterpret_cast<float2*>(wml + 2 * h1) = make_float2(m[1], l[1]);
     }
-    // publish the partial, then count this warp on the unit's counter; the last of the
-    // unit's contributors merges them all
-    int c_first, c_last;
-    const long long U0 = unit_at[2 * warp], U1 = unit_at[2 * warp + 1], P = range_at[1];
-    const int expect = unit_contributors(U0, U1, P, C, lane, &c_first, &c_last);
-    __threadfence();
-    __syncwarp();
-    int got = 0;
-    if (lane == 0) got = arrive(p.ws_cnt + cur_u, p.epoch);
-    got = __shfl_sync(0xffffffffu, got, 0);
-    if (got < 0) {
-      if (lane == 0) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
-    } else if (got == expect) {
-      __threadfence();
-      merge_unit(p, cur_u, U0, U1, P, C, c_first, c_last, lane);
-      if (lane == 0) atomicExch(p.ws_cnt + cur_u, 0ull);   // leave the counter empty
-    }
   };
 
   // Prefill: normalise and store this warp's output rows (query row qrow, its g heads).
@@ -705,13 +546,6 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       if (mt.x != cur_u) {              // warp-uniform: a new (sequence, kv head) unit
         if (cur_u >= 0) end_unit();
         cur_u = mt.x;
-        if (lane == 0) {
-          // stage i holds global page (range start + i), page mt.y of the unit
-          const long long U0 = range_at[0] + i - mt.y;
-          unit_at[2 * warp] = U0;
-          unit_at[2 * warp + 1] = U0 + (mt.z + BS - 1) / BS;
-        }
-        __syncwarp();
         begin_unit(cur_u, cur_u / p.H);
       }
     }
@@ -996,7 +830,7 @@ cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s)
   if (!make_pages_map(&tm, a.c->pages, rows, L::REC_ROWS)) return cudaErrorInvalidValue;
   const dim3 grid = PF ? dim3((a.max_q_len + kConsumers - 1) / kConsumers, a.geo.H, a.batch)
                        : dim3(a.plan.ctas);
-  if (!PF && (a.plan.ctas < 1 || (a.batch > 0 && p.ws_cnt == nullptr))) return cudaErrorInvalidValue;
+  if (!PF && a.plan.ctas < 1) return cudaErrorInvalidValue;
   return launch_dependent(decode_mma_kernel<CD, BS, PT, PF>, grid, dim3(kThreads), L::BYTES, s, p, tm);
 }
 

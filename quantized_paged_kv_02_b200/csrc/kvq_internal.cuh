@@ -172,7 +172,6 @@ struct DecodePlan {
   int ctas;          // kernel 1: grid size
   size_t ws_bytes;   // workspace bytes (0 when a single split writes the output)
   size_t ws_ml_off;  // byte offset of the (max, sum) array inside the workspace
-  size_t ws_cnt_off; // kernel 1: byte offset of the per-unit arrival counters
   int sms;           // streaming multiprocessors the plan was made for
 };
 
@@ -199,8 +198,6 @@ struct DecodeArgs {
   int out_dtype;
   float* ws_o;               // partial outputs (layout per kernel)
   float* ws_ml;              // partial (max, sum) pairs
-  unsigned long long* ws_cnt;  // kernel 1: per-unit arrival counters
-  uint32_t epoch;            // kernel 1: tag of this call's arrivals (never 0)
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

@@ -1,0 +1,843 @@
+// Chunked-prefill attention over the quantized paged cache on the 5th-generation tensor
+// cores (tcgen05.mma, accumulators in tensor memory), for head_dim 128: INT8, FP8 E4M3,
+// BF16 and FP16 caches with block size 16, and the INT4 / 2-bit group caches (block 64, the
+// newest tokens in the residual ring).
+//
+// A CTA owns one tile of 128 query rows of one (sequence, kv head): 128 / g query tokens x
+// the g query heads that share the kv head (row r = token r / g, head r % g), and walks the
+// causal window of its last query in blocks of 128 cached tokens (8 pages).  Each page is
+// dequantized ONCE into shared memory for all 128 rows, instead of once per query token:
+//
+//   warp 4      producer: one bulk copy per page record (K codes, V codes, per-token scales)
+//               into a ring of raw stages;
+//   warps 6-9   converters: codes -> 16-bit tiles in the tensor cores' 128-byte-swizzled
+//               layout (INT8 through the exact 1024-magic, E4M3 by the hardware conversion,
+//               16-bit caches copied), K as the K-major B operand of S = Q K^T and V as the
+//               MN-major B operand of O = P V, plus the per-token scales of the block;
+//   warp 5      MMA issuer: S_j = Q K_j^T (M 128, N 128 tokens, K 128) into one of two TMEM
+//               score buffers, then O += P_{j-1} V_{j-1} (N 128 channels, K 128 tokens);
+//   warps 0-3   softmax: thread r owns query row r, reads its 128 scores from TMEM, scales
+//               them (per-token K scale, softmax scale, log2 e), masks the causal boundary,
+//               keeps the running max (re-based only when a score exceeds it by 2^8) and sum,
+//               folds the per-token V scale into P, and writes P back over its scores as
+//               fp16 (bf16 for bf16 caches) hi + lo halves, the A operand of the P V MMA.
+//
+// Q lives in TMEM too (written once by the softmax warps), so shared memory holds only the
+// K / V tiles and the raw ring.  The contraction is exact in the codes: for INT8 / FP8 the
+// K and V tiles hold the codes themselves (exact in fp16), q is an exact fp16 copy of the
+// bf16 activations scaled by a power of two (per-channel K scales fold into q as a hi + lo
+// pair), and P's hi + lo halves keep 22 bits.  For INT4 / 2-bit caches the dequantized
+// value (code - zero) * scale (at most 15 significant bits) is split exactly into bf16 hi +
+// lo tiles; S takes both (and both halves of q when activations are fp16), P V takes
+// P hi V hi + P hi V lo + P lo V hi.  Scores, softmax and O accumulate in fp32.  Chunked prefill is one of the techniques [P-prod] "为什么长上下文更需要 KV Cache
+// Quantization" lists beside cache quantization; dequantization inside attention is the
+// design of [P-vLLM] "PagedAttention与KV Cache量化协同工作原理".
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <mutex>
+
+#include "kvq_decode_common.cuh"
+#include "kvq_ptx.cuh"
+#include "kvq_tc.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kRows = 128;          // query rows per tile (MMA M)
+constexpr int kBlk = 128;           // cached tokens per block (MMA N of S, K of P V)
+constexpr int kD = 128;
+constexpr int kPfThreads = 320;     // warps 0-3 softmax, 4 producer, 5 MMA, 6-9 converters
+constexpr int kSoftWarps = 4, kProdWarp = 4, kMmaWarp = 5, kConvWarp0 = 6;
+constexpr int kNB = 2;              // K / V tile buffers
+constexpr int kTile = 32768;        // 128 x 128 16-bit elements
+constexpr float kRescalePf = 8.f;   // log2 headroom before the running max is re-based
+// TMEM columns: scores / P of block j in [128 (j % 2), +128), O in [256, 384), Q from 384
+constexpr uint32_t kTmemCols = 512, kTmO = 256, kTmQ = 384;
+
+// Code width and tile type per cache dtype: 8-bit codes and fp16 caches use fp16 tiles,
+// bf16 caches and the low-bit caches (whose exact values need a bf16 hi + lo pair) bf16.
+template <int CD> struct PfCode;
+template <> struct PfCode<KVQ_DTYPE_INT8> { static constexpr int BITS = 8; static constexpr bool kBf16 = false; };
+template <> struct PfCode<KVQ_DTYPE_FP8_E4M3> { static constexpr int BITS = 8; static constexpr bool kBf16 = false; };
+template <> struct PfCode<KVQ_DTYPE_FP16> { static constexpr int BITS = 16; static constexpr bool kBf16 = false; };
+template <> struct PfCode<KVQ_DTYPE_BF16> { static constexpr int BITS = 16; static constexpr bool kBf16 = true; };
+template <> struct PfCode<KVQ_DTYPE_INT4> { static constexpr int BITS = 4; static constexpr bool kBf16 = true; };
+template <> struct PfCode<KVQ_DTYPE_INT2> { static constexpr int BITS = 2; static constexpr bool kBf16 = true; };
+
+template <int CD, bool PT>
+struct PfLayout {
+  static constexpr int BITS = PfCode<CD>::BITS;
+  static constexpr bool LB = BITS < 8;                     // group codes + residual ring
+  static constexpr int BS = LB ? 64 : 16;
+  static constexpr int PPB = kBlk / BS;                    // pages per block
+  static constexpr int ROWB = kD * BITS / 8;
+  static constexpr int OFF_V = BS * ROWB;
+  static constexpr int OFF_S = 2 * BS * ROWB;
+  // scales: per-token float32 K and V (PT), or the group parameters (K 4 D bytes, V
+  // (scale, zero) per token and 64-channel group)
+  static constexpr int SCALES = LB ? 4 * kD + BS * (kD / 64) * 4 : (PT ? 8 * BS : 0);
+  static constexpr int REC = (OFF_S + SCALES + 127) / 128 * 128;
+  static constexpr int KP = LB ? 2 : 1;                    // K tiles whose sum is K (hi, lo)
+  static constexpr int VP = LB ? 2 : 1;
+  static constexpr int NB = LB ? 1 : kNB;                  // K / V tile buffers
+  static constexpr int RS = LB ? 4 : (BITS == 8 ? 16 : 8); // raw ring stages (pages)
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = NB * KP * kTile;
+  static constexpr int RAW_OFF = V_OFF + NB * VP * kTile;
+  static constexpr int KQ_OFF = RAW_OFF + RS * REC;        // float [NB][128]: K multiplier
+  static constexpr int VS_OFF = KQ_OFF + NB * kBlk * 4;    // float [NB][128]: V scale
+  static constexpr int MISC_OFF = VS_OFF + NB * kBlk * 4;  // per (buffer, converter warp) vmax
+                                                           // and bad-token counts; flags
+  static constexpr int BAR_OFF = MISC_OFF + 128;
+  // raw_full, raw_empty [RS]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
+  // q_ready; fin
+  static constexpr int NBARS = 2 * RS + 3 * NB + 6 + 2;
+  static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + RS * 4 + 64;
+  static_assert(BYTES <= 227 * 1024, "fits the shared memory of one CTA");
+  static_assert(BYTES > 114 * 1024, "one CTA per SM, so TMEM allocation never waits on a peer");
+  static_assert(RS >= PPB, "a block's pages fit the raw ring");
+  static_assert(REC % 16 == 0, "bulk copies move multiples of 16 bytes");
+  static_assert(NB <= kNB, "scale arrays");
+};
+
+struct PfShared {
+  uint64_t* raw_full;
+  uint64_t* raw_empty;
+  uint64_t* k_full;
+  uint64_t* v_full;
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* vfree;
+  uint64_t* pv_done;                // [2]: P V of block j commits to pv_done[j % 2]
+  uint64_t* q_ready;
+  uint64_t* fin;                    // the MMA issuer's final commit
+  int* page_ok;
+  float* kq;                        // [NB][128] K multiplier of each token (NaN: bad page)
+  float* vs;                        // [NB][128] V scale of each token
+  float* vmax;                      // [NB][4] largest V scale seen by each converter warp
+  int* nbad;                        // [NB][4] bad-page tokens seen by each converter warp
+  float* qscale;
+  uint32_t* tmem;
+  volatile int* abort;
+};
+
+// Bounded wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void pf_fail(const DecodeParams& p, volatile int* abort) {
+  record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+  *abort = 1;
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Eight INT8 codes -> eight fp16 values (exact), packed low element first.
+__device__ __forceinline__ uint4 i8x8_to_f16(uint2 w) {
+  const uint32_t a = w.x ^ 0x80808080u, b = w.y ^ 0x80808080u;
+  return make_uint4(i8x2_to_f16x2(a, kLoPair), i8x2_to_f16x2(a, kHiPair), i8x2_to_f16x2(b, kLoPair),
+                    i8x2_to_f16x2(b, kHiPair));
+}
+
+__device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 w) {
+  return make_uint4(e4m3x2_to_f16x2(w.x & 0xFFFFu), e4m3x2_to_f16x2(w.x >> 16),
+                    e4m3x2_to_f16x2(w.y & 0xFFFFu), e4m3x2_to_f16x2(w.y >> 16));
+}
+
+// Swizzled byte offset of 16-byte chunk c (8 elements, c < 16) of row t in a 128 x 128 tile.
+__device__ __forceinline__ uint32_t tile_off(int t, int c) {
+  return static_cast<uint32_t>((c >> 3) * 16384 + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
+// hi + lo split of two fp32 values into 16-bit pairs (fp16, or bf16 for bf16 caches).
+template <bool BF>
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  if constexpr (BF) {
+    hi = pack_bf16x2(a, b);
+    const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+    lo = pack_bf16x2(a - h.x, b - h.y);
+  } else {
+    hi = pack_f16x2(a, b);
+    const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+    lo = pack_f16x2(a - h.x, b - h.y);
+  }
+}
+
+__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+      : "memory");
+}
+
+// Dequantized value of one low-bit code: (code - zero) * scale, or code * scale + minimum
+// (float zero point); exact in float32 for the integer zero point (<= 15 significant bits).
+__device__ __forceinline__ float lb_value(int code, float s, float z, bool fz) {
+  return fz ? fmaf(static_cast<float>(code), s, z) : static_cast<float>(code - static_cast<int>(z)) * s;
+}
+
+// Eight values -> bf16 hi and lo chunks (value = hi + lo, exactly for <= 16 significant bits).
+__device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
+  split2<true>(v[0], v[1], hi.x, lo.x);
+  split2<true>(v[2], v[3], hi.y, lo.y);
+  split2<true>(v[4], v[5], hi.z, lo.z);
+  split2<true>(v[6], v[7], hi.w, lo.w);
+}
+
+template <int CD, bool PT, int QP>
+__global__ void __launch_bounds__(kPfThreads, 1)
+prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
+  using L = PfLayout<CD, PT>;
+  constexpr bool kBf = PfCode<CD>::kBf16;
+  constexpr int BS = L::BS, NB = L::NB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, kvh = blockIdx.y;
+  const int g = p.g, TQ = kRows / g;
+  const int q0 = blockIdx.x * TQ;
+  // the sequence's query count L and context n; a sequence with more queries than
+  // positions, or than the host bound max_q_len, is rejected (counted once)
+  int Lq = p.q_start[b + 1] - p.q_start[b];
+  const SeqInfo si = seq_info(p, b, L::LB, blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0);
+  const int n = si.n;
+  if (Lq > n || Lq > p.max_q_len || Lq < 0) {
+    if (blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0) record_fault(p.fault, KVQ_FAULT_CONTEXT);
+    Lq = 0;
+  }
+  if (q0 >= Lq) return;                                   // uniform: no query of this tile
+  const int pmin = n - Lq + q0;                           // position of the tile's first query
+  const int pmax = n - Lq + min(q0 + TQ, Lq) - 1;         // ... and of its last
+  const int J = pmax / kBlk + 1;                          // blocks of the causal window
+  // pages to copy: those of the causal window (low-bit caches: of the quantized prefix only;
+  // positions from si.qb on come from the residual ring)
+  const int npg = L::LB ? min(pmax / BS + 1, si.qb / BS) : pmax / BS + 1;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  PfShared sh;
+  sh.raw_full = bars;
+  sh.raw_empty = bars + L::RS;
+  sh.k_full = bars + 2 * L::RS;
+  sh.v_full = sh.k_full + NB;
+  sh.vfree = sh.v_full + NB;
+  sh.s_full = sh.vfree + NB;
+  sh.p_full = sh.s_full + 2;
+  sh.pv_done = sh.p_full + 2;
+  sh.q_ready = sh.pv_done + 2;
+  sh.fin = sh.q_ready + 1;
+  sh.page_ok = reinterpret_cast<int*>(bars + L::NBARS);
+  sh.kq = reinterpret_cast<float*>(smem + L::KQ_OFF);
+  sh.vs = reinterpret_cast<float*>(smem + L::VS_OFF);
+  sh.vmax = reinterpret_cast<float*>(smem + L::MISC_OFF);            // [NB][4]
+  sh.nbad = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);         // [NB][4]
+  sh.qscale = reinterpret_cast<float*>(smem + L::MISC_OFF + 64);
+  sh.tmem = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF + 68);
+  sh.abort = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 72);
+  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 80);   // [4] softmax amax
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::RS; ++s) {
+      mbar_init(&sh.raw_full[s], 1);
+      mbar_init(&sh.raw_empty[s], 4);                    // the four converter warps
+    }
+    for (int k = 0; k < NB; ++k) {
+      mbar_init(&sh.k_full[k], 4);
+      mbar_init(&sh.v_full[k], 4);
+      mbar_init(&sh.vfree[k], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&sh.s_full[k], 1);
+      mbar_init(&sh.p_full[k], kSoftWarps);
+      mbar_init(&sh.pv_done[k], 1);
+    }
+    mbar_init(sh.q_ready, kSoftWarps);
+    mbar_init(sh.fin, 1);
+    *sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tc::tmem_alloc(sh.tmem, kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *sh.tmem;
+
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------------ producer
+    const uint8_t* pages = p.pages;
+    int issued = 0;
+    bool ok_run = true;
+    for (int k0 = 0; k0 < npg && ok_run; k0 += 8) {
+      const int cnt = min(8, npg - k0);
+      bool ok_lane = true;
+      if (lane < cnt) {
+        const int k = k0 + lane, s = k % L::RS, round = k / L::RS;
+        const int blk = p.tables[static_cast<long>(b) * p.max_blocks + k];
+        const bool valid = blk >= 0 && blk < p.NB;
+        if (round > 0 && !pf_wait(&sh.raw_empty[s], (round - 1) & 1, sh.abort)) {
+          ok_lane = false;
+        } else {
+          sh.page_ok[s] = valid;
+          if (valid) {
+            mbar_arrive_expect_tx(&sh.raw_full[s], L::REC);
+            bulk_load(smem + L::RAW_OFF + s * L::REC,
+                      pages + (static_cast<long>(blk) * p.H + kvh) * L::REC, L::REC, &sh.raw_full[s]);
+          } else {
+            record_fault(p.fault, KVQ_FAULT_BLOCK);
+            mbar_arrive(&sh.raw_full[s]);
+          }
+        }
+      }
+      ok_run = __all_sync(0xffffffffu, ok_lane);
+      if (!ok_run && lane == 0) pf_fail(p, sh.abort);
+      issued = k0 + cnt;
+    }
+    // every copy issued must land before the CTA may exit
+    if (lane == 0) {
+      for (int k = max(0, issued - L::RS); k < issued; ++k)
+        if (!mbar_drain(&sh.raw_full[k % L::RS], (k / L::RS) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+    }
+  } else if (warp >= kConvWarp0) {
+    // ------------------------------------------------------------ converters
+    // thread (c, rr): 16-byte output chunk c (elements 8c..8c+7 of a row) of rows rr + 8i
+    const int ct = threadIdx.x - kConvWarp0 * 32;        // 0..127
+    const int c = ct & 15, rr = ct >> 4;
+    const int cw = warp - kConvWarp0;
+    if (!pf_wait(sh.q_ready, 0, sh.abort)) pf_fail(p, sh.abort);
+    const float qsc = *sh.qscale;
+    const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
+    const int G = c >> 3;                                 // 64-channel group of the chunk
+    for (int j = 0; j < J && !*sh.abort; ++j) {
+      const int kb = j % NB;
+      // the softmax of block j - NB is done with this buffer's scales (and S j - NB with K)
+      if (j >= NB && !pf_wait(&sh.p_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) {
+        if (lane == 0) pf_fail(p, sh.abort);
+        break;
+      }
+      int bad = 0;
+      bool ok = true;
+      // K: rows rr + 8i of every page of the block, chunk c
+      for (int pp = 0; pp < L::PPB && ok; ++pp) {
+        const int k = j * L::PPB + pp;
+        const bool have = k < npg;
+        const int s = k % L::RS;
+        if (have && !pf_wait(&sh.raw_full[s], (k / L::RS) & 1, sh.abort)) {
+          ok = false;
+          break;
+        }
+        const bool pok = have && sh.page_ok[s];
+        const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
+        if constexpr (!L::LB) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = rr + 8 * h, t = pp * BS + row, pos = j * kBlk + t;
+            const bool valid = pok && pos <= pmax;
+            uint4 out = make_uint4(0, 0, 0, 0);
+            if (valid) {
+              if constexpr (L::BITS == 8) {
+                const uint2 w = *reinterpret_cast<const uint2*>(raw + row * L::ROWB + 8 * c);
+                out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w) : e4m3x8_to_f16(w);
+              } else {
+                out = *reinterpret_cast<const uint4*>(raw + row * L::ROWB + 16 * c);
+              }
+            }
+            *reinterpret_cast<uint4*>(smem + L::K_OFF + kb * kTile + tile_off(t, c)) = out;
+            if (c == 0) {
+              float ks = 1.f;
+              if constexpr (PT) ks = reinterpret_cast<const float*>(raw + L::OFF_S)[row];
+              // tokens of a bad page are marked NaN (masked by the softmax); positions past
+              // the tile's last query are never visible, so their multiplier does not matter
+              const bool badtok = have && !pok && pos <= pmax;
+              sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+              bad += badtok;
+            }
+          }
+        } else {
+          // per-channel K parameters of this chunk (KIVI forms): s[8c..8c+7], z or minimum
+          float ksc[8], kzp[8];
+          if (!ktok && pok) {
+            const uint4 su = *reinterpret_cast<const uint4*>(raw + L::OFF_S + 16 * c);
+            const uint4 zu = *reinterpret_cast<const uint4*>(raw + L::OFF_S + 2 * kD + 16 * c);
+            const __half* sh8 = reinterpret_cast<const __half*>(&su);
+            const __half* zh8 = reinterpret_cast<const __half*>(&zu);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              ksc[e] = __half2float(sh8[e]);
+              kzp[e] = __half2float(zh8[e]);
+            }
+          }
+          for (int i = 0; i < BS / 8; ++i) {
+            const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
+            const bool ring = pos >= si.qb;
+            const bool valid = pos <= pmax && (ring || pok);
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+            if (valid && ring) {
+              const long rrow = ((static_cast<long>(si.sid) * 2) * p.H + kvh) * p.cap + pos % p.cap;
+              const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + rrow * kD + 8 * c);
+              if (p.act_fp16) unpack8<__half>(u, v);
+              else unpack8<__nv_bfloat16>(u, v);
+            } else if (valid) {
+              uint32_t w;
+              if constexpr (L::BITS == 4) w = *reinterpret_cast<const uint32_t*>(raw + row * L::ROWB + 4 * c);
+              else w = *reinterpret_cast<const uint16_t*>(raw + row * L::ROWB + 2 * c);
+              float s1 = 0.f, z1 = 0.f;
+              if (ktok) {
+                const __half2 sz = *reinterpret_cast<const __half2*>(raw + L::OFF_S + (row * 2 + G) * 4);
+                s1 = __low2float(sz);
+                z1 = __high2float(sz);
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int code = (w >> (L::BITS * e)) & ((1 << L::BITS) - 1);
+                v[e] = ktok ? lb_value(code, s1, z1, false) : lb_value(code, ksc[e], kzp[e], fz);
+              }
+            }
+            uint4 hi, lo;
+            split8(v, hi, lo);
+            *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2) * kTile + tile_off(t, c)) = hi;
+            *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
+            if (c == 0) {
+              const bool badtok = !ring && have && !pok && pos <= pmax;
+              sh.kq[kb * kBlk + t] = valid ? qsc : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+              bad += badtok;
+            }
+          }
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) pf_fail(p, sh.abort);
+        break;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, off);
+      if (lane == 0) sh.nbad[kb * 4 + cw] = bad;
+      tc::fence_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.k_full[kb]);
+      // V: wait until P V of block j - NB has read this buffer
+      if (j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
+        if (lane == 0) pf_fail(p, sh.abort);
+        break;
+      }
+      float vm = 0.f;
+      for (int pp = 0; pp < L::PPB; ++pp) {
+        const int k = j * L::PPB + pp;
+        const bool have = k < npg;
+        const int s = k % L::RS;
+        const bool pok = have && sh.page_ok[s];
+        const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
+        if constexpr (!L::LB) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = rr + 8 * h, t = pp * BS + row, pos = j * kBlk + t;
+            const bool valid = pok && pos <= pmax;
+            uint4 out = make_uint4(0, 0, 0, 0);
+            if (valid) {
+              if constexpr (L::BITS == 8) {
+                const uint2 w = *reinterpret_cast<const uint2*>(raw + L::OFF_V + row * L::ROWB + 8 * c);
+                out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w) : e4m3x8_to_f16(w);
+              } else {
+                out = *reinterpret_cast<const uint4*>(raw + L::OFF_V + row * L::ROWB + 16 * c);
+              }
+            }
+            *reinterpret_cast<uint4*>(smem + L::V_OFF + kb * kTile + tile_off(t, c)) = out;
+            if (c == 0) {
+              float vv = 1.f;
+              if constexpr (PT) vv = reinterpret_cast<const float*>(raw + L::OFF_S)[BS + row];
+              vv = valid ? vv : 0.f;
+              sh.vs[kb * kBlk + t] = vv;
+              vm = fmaxf(vm, vv);
+            }
+          }
+        } else {
+          for (int i = 0; i < BS / 8; ++i) {
+            const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
+            const bool ring = pos >= si.qb;
+            const bool valid = pos <= pmax && (ring || pok);
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+            if (valid && ring) {
+              const long vrow = ((static_cast<long>(si.sid) * 2 + 1) * p.H + kvh) * p.cap + pos % p.cap;
+              const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + vrow * kD + 8 * c);
+              if (p.act_fp16) unpack8<__half>(u, v);
+              else unpack8<__nv_bfloat16>(u, v);
+            } else if (valid) {
+              uint32_t w;
+              if constexpr (L::BITS == 4) w = *reinterpret_cast<const uint32_t*>(raw + L::OFF_V + row * L::ROWB + 4 * c);
+              else w = *reinterpret_cast<const uint16_t*>(raw + L::OFF_V + row * L::ROWB + 2 * c);
+              const __half2 sz = *reinterpret_cast<const __half2*>(raw + L::OFF_S + 4 * kD + (row * 2 + G) * 4);
+              const float s1 = __low2float(sz), z1 = __high2float(sz);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = lb_value((w >> (L::BITS * e)) & ((1 << L::BITS) - 1), s1, z1, fz);
+            }
+            uint4 hi, lo;
+            split8(v, hi, lo);
+            *reinterpret_cast<uint4*>(smem + L::V_OFF + (kb * 2) * kTile + tile_off(t, c)) = hi;
+            *reinterpret_cast<uint4*>(smem + L::V_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
+            if (c == 0) {
+              const float vv = valid ? 1.f : 0.f;
+              sh.vs[kb * kBlk + t] = vv;
+              vm = fmaxf(vm, vv);
+            }
+          }
+        }
+        __syncwarp();
+        if (have && lane == 0) mbar_arrive(&sh.raw_empty[s]);   // K and V of the page are read
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+      if (lane == 0) sh.vmax[kb * 4 + cw] = vm;
+      tc::fence_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.v_full[kb]);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t tiles = smem_u32(smem);
+    constexpr uint32_t idS = tc::idesc_f16(kBf, false, kRows, kBlk);
+    constexpr uint32_t idPV = tc::idesc_f16(kBf, true, kRows, kD);
+    if (lane == 0) {
+      bool ok = pf_wait(sh.q_ready, 0, sh.abort);
+      tc::fence_after_sync();
+      auto pv = [&](int jj) -> bool {
+        const int sb = jj & 1, kb = jj % NB;
+        if (!pf_wait(&sh.v_full[kb], (jj / NB) & 1, sh.abort)) return false;
+        if (!pf_wait(&sh.p_full[sb], (jj >> 1) & 1, sh.abort)) return false;
+        tc::fence_after_sync();
+        // P hi V hi (+ P hi V lo + P lo V hi for split V) + P lo V hi ... : pairs (pa, vp),
+        // pa + vp <= 1
+        bool first = jj == 0;
+#pragma unroll
+        for (int pa = 0; pa < 2; ++pa)
+#pragma unroll
+          for (int vp = 0; vp < L::VP; ++vp) {
+            if (pa + vp > 1) continue;
+            const uint32_t vt = tiles + L::V_OFF + (kb * L::VP + vp) * kTile;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              // tokens 16 kk .. 16 kk + 15: chunk kk / 2 of P, its hi (pa 0) or lo (pa 1) half
+              tc::mma_ts(tbase + kTmO, tbase + 128 * sb + 32 * (kk >> 1) + 16 * pa + 8 * (kk & 1),
+                         tc::desc_mnmajor(vt, kk), idPV, first ? 0u : 1u);
+              first = false;
+            }
+          }
+        tc::commit(&sh.vfree[kb]);
+        tc::commit(&sh.pv_done[jj & 1]);
+        return true;
+      };
+      for (int j = 0; j < J && ok; ++j) {
+        const int sb = j & 1, kb = j % NB;
+        if (!pf_wait(&sh.k_full[kb], (j / NB) & 1, sh.abort)) { ok = false; break; }
+        tc::fence_after_sync();
+        bool first = true;
+#pragma unroll
+        for (int qa = 0; qa < QP; ++qa)
+#pragma unroll
+          for (int kp = 0; kp < L::KP; ++kp) {
+            if (qa + kp > 1) continue;
+            const uint32_t kt = tiles + L::K_OFF + (kb * L::KP + kp) * kTile;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              tc::mma_ts(tbase + 128 * sb, tbase + kTmQ + 64 * qa + 8 * kk, tc::desc_kmajor(kt, kk), idS,
+                         first ? 0u : 1u);
+              first = false;
+            }
+          }
+        tc::commit(&sh.s_full[sb]);
+        if (j > 0 && !pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && !pv(J - 1)) ok = false;
+      if (!ok) pf_fail(p, sh.abort);
+      // one more commit covers every MMA issued above: TMEM is freed only after it arrives
+      tc::commit(sh.fin);
+      if (!mbar_drain(sh.fin, 0)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax (row r)
+    const int r = threadIdx.x;                            // 0..127: TMEM lane = query row
+    const int t_loc = r / g, h = r - t_loc * g;
+    const int qi = q0 + t_loc;
+    const bool row_ok = qi < Lq;
+    const int pos_r = n - Lq + qi;
+    const uint32_t lanebase = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    // --- q row -> TMEM (exact fp16 scaled by 2^-eq for quantized caches; 16-bit caches as is)
+    {
+      const long qrow = static_cast<long>(p.q_start[b]) + qi;
+      const uint4* qp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.q) +
+                                                       (qrow * p.Hq + static_cast<long>(kvh) * g + h) * kD);
+      // per-channel K scales fold into q (then q goes to TMEM as a hi + lo pair); with
+      // bf16 tiles and fp16 activations q is split exactly into bf16 hi + lo
+      const float* kch = p.mode == KVQ_SCALE_PER_CHANNEL ? p.k_static + kvh * kD : nullptr;
+      auto elem = [&](const uint4& u, int e) {     // element e (0..7) of 8 packed activations
+        const uint32_t w2 = (&u.x)[e >> 1];
+        const uint16_t hv = static_cast<uint16_t>((e & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
+        return p.act_fp16 ? __half2float(__ushort_as_half(hv)) : __bfloat162float(__ushort_as_bfloat16(hv));
+      };
+      float qscale = p.scale_log2;
+      if (p.mode == KVQ_SCALE_PER_HEAD) qscale *= p.k_static[kvh];
+      if (p.mode == KVQ_SCALE_PER_TENSOR) qscale *= p.k_static[0];
+      float down = 1.f;
+      if constexpr (!kBf) {
+        // the tile's largest |q| (times the channel scale) sets a power-of-two scale that
+        // keeps q inside fp16
+        float amax = 0.f;
+        if (row_ok) {
+#pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const uint4 u = qp[i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(kch != nullptr ? elem(u, e) * kch[8 * i + e] : elem(u, e)));
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) red[warp] = amax;
+        named_sync(2, 128);
+        amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        int eq = 0;
+        if (amax > 0.f && !(p.act_fp16 && kch == nullptr)) eq = ilogbf(amax) - 13;
+        down = ldexpf(1.f, -eq);
+        qscale = ldexpf(qscale, eq);
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 u = row_ok ? qp[8 * half + i] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int d = 64 * half + 8 * i + e;
+            float a = elem(u, e), c2 = elem(u, e + 1);
+            if (kch != nullptr) {
+              a *= kch[d];
+              c2 *= kch[d + 1];
+            }
+            a *= down;
+            c2 *= down;
+            if constexpr (QP == 2) split2<kBf>(a, c2, hi[4 * i + e / 2], lo[4 * i + e / 2]);
+            else hi[4 * i + e / 2] = kBf ? pack_bf16x2(a, c2) : pack_f16x2(a, c2);
+          }
+        }
+        tc::st32(lanebase + kTmQ + 32 * half, hi);
+        if constexpr (QP == 2) tc::st32(lanebase + kTmQ + 64 + 32 * half, lo);
+      }
+      if (threadIdx.x == 0) *sh.qscale = qscale;
+      tc::st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sh.q_ready);
+    }
+    // --- blocks
+    float m = -INFINITY, l = 0.f;
+    int ev = INT_MIN;
+    float vinv = 0.f;
+    bool ok = true;
+    for (int j = 0; j < J; ++j) {
+      const int sb = j & 1, kb = j % NB;
+      if (!pf_wait(&sh.k_full[kb], (j / NB) & 1, sh.abort) ||
+          !pf_wait(&sh.s_full[sb], (j >> 1) & 1, sh.abort)) {
+        ok = false;
+      }
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc::fence_after_sync();
+      // pass 1: the block's largest scaled score of this row (scores are read from TMEM
+      // again in pass 2, so only 32 of them are live at a time)
+      const float* kq = sh.kq + kb * kBlk;
+      const bool fast = sh.nbad[kb * 4] + sh.nbad[kb * 4 + 1] + sh.nbad[kb * 4 + 2] + sh.nbad[kb * 4 + 3] == 0 &&
+                        j * kBlk + kBlk - 1 <= pmin;   // uniform
+      // causal boundary (position <= this row's) and tokens of bad pages (multiplier NaN)
+      const int lim = row_ok ? pos_r - j * kBlk : -1;
+      auto scaled = [&](uint32_t sv, float f, int t) {
+        const float x = __uint_as_float(sv) * f;
+        return (fast || (t <= lim && f == f)) ? x : -INFINITY;
+      };
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32];
+        tc::ld32(lanebase + 128 * sb + 32 * cc, sr);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(kq + 32 * cc + i);
+          const int t = 32 * cc + i;
+          mx = fmaxf(mx, fmaxf(fmaxf(scaled(sr[i], f.x, t), scaled(sr[i + 1], f.y, t + 1)),
+                               fmaxf(scaled(sr[i + 2], f.z, t + 2), scaled(sr[i + 3], f.w, t + 3))));
+        }
+      }
+      if (!pf_wait(&sh.v_full[kb], (j / NB) & 1, sh.abort)) ok = false;
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      // running max (re-based lazily) and V normaliser 2^ev (grows with the largest V scale)
+      float fo = 1.f;
+      const float vmx = fmaxf(fmaxf(sh.vmax[kb * 4], sh.vmax[kb * 4 + 1]),
+                              fmaxf(sh.vmax[kb * 4 + 2], sh.vmax[kb * 4 + 3]));
+      if (vmx > 0.f) {
+        const int e = exponent_of(vmx);
+        if (e > ev) {
+          if (ev != INT_MIN) fo = pow2i(ev - e);
+          ev = e;
+          vinv = pow2i(-ev);
+        }
+      }
+      if (mx > m + kRescalePf) {
+        const float mn = fmaxf(m, mx);
+        const float c0 = m == -INFINITY ? 0.f : ex2(m - mn);
+        l *= c0;
+        fo *= c0;
+        m = mn;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, fo != 1.f)) {
+        // rescale this warp's O rows: P V of block j - 1 must be complete
+        if (!pf_wait(&sh.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, sh.abort)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tc::ld32(lanebase + kTmO + 32 * cc, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
+          tc::st32(lanebase + kTmO + 32 * cc, o);
+        }
+      }
+      const float base = m == -INFINITY ? 0.f : m;
+      const float* vsp = sh.vs + kb * kBlk;
+      // pass 2: P = 2^(x - base), the row sum, and P times the token's V scale / 2^ev as
+      // hi + lo 16-bit halves over the scores
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32];
+        tc::ld32(lanebase + 128 * sb + 32 * cc, sr);
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int t = 32 * cc + 2 * i;
+          const float2 f = *reinterpret_cast<const float2*>(kq + t);
+          const float e0 = ex2(scaled(sr[2 * i], f.x, t) - base);
+          const float e1 = ex2(scaled(sr[2 * i + 1], f.y, t + 1) - base);
+          l += e0 + e1;
+          const float2 v2 = *reinterpret_cast<const float2*>(vsp + t);
+          split2<kBf>(e0 * v2.x * vinv, e1 * v2.y * vinv, ph[i], pl[i]);
+        }
+        // the 32 score columns just read take P of the same 32 tokens: hi halves in the
+        // first 16 columns, lo halves in the next 16
+        st16(lanebase + 128 * sb + 32 * cc, ph);
+        st16(lanebase + 128 * sb + 32 * cc + 16, pl);
+      }
+      tc::st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.p_full[sb]);
+    }
+    if (!ok) {
+      if (lane == 0) pf_fail(p, sh.abort);
+    } else {
+      // --- epilogue: O / l (times 2^ev and the static V scales) -> out
+      if (!pf_wait(&sh.pv_done[(J - 1) & 1], ((J - 1) >> 1) & 1, sh.abort)) ok = false;
+      if (__all_sync(0xffffffffu, ok)) {
+        tc::fence_after_sync();
+        float vmul = 1.f;
+        if (p.mode == KVQ_SCALE_PER_HEAD) vmul = p.v_static[kvh];
+        if (p.mode == KVQ_SCALE_PER_TENSOR) vmul = p.v_static[0];
+        const float inv = l > 0.f ? vmul * pow2i(ev == INT_MIN ? 0 : ev) / l : 0.f;
+        const float* vch = (p.mode == KVQ_SCALE_PER_CHANNEL) ? p.v_static + kvh * kD : nullptr;
+        const long orow = (static_cast<long>(p.q_start[b]) + qi) * p.Hq + static_cast<long>(kvh) * g + h;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tc::ld32(lanebase + kTmO + 32 * cc, o);
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int d = 32 * cc + i;
+              const float v = __uint_as_float(o[i]) * inv * (vch != nullptr ? vch[d] : 1.f);
+              store_out(p, orow * kD + d, v);
+            }
+          }
+        }
+      } else if (lane == 0) {
+        pf_fail(p, sh.abort);
+      }
+    }
+  }
+  // ---------------------------------------------------------------- teardown
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    // the issuer waited for its final commit (every MMA complete) before the barrier
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+template <int CD, bool PT, int QP>
+cudaError_t launch_pf(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  using L = PfLayout<CD, PT>;
+  if (a.geo.record != L::REC) return cudaErrorInvalidValue;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(prefill_tc_kernel<CD, PT, QP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int TQ = kRows / a.plan.g;
+  const dim3 grid((a.max_q_len + TQ - 1) / TQ, a.geo.H, a.batch);
+  prefill_tc_kernel<CD, PT, QP><<<grid, kPfThreads, L::BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const Geometry& g, int group) {
+  if (g.D != kD || group < 1 || kRows % group != 0) return false;
+  switch (g.cache_dtype) {
+    case KVQ_DTYPE_INT8:
+    case KVQ_DTYPE_FP8_E4M3:
+    case KVQ_DTYPE_BF16:
+    case KVQ_DTYPE_FP16: return g.bs == 16;
+    case KVQ_DTYPE_INT4:
+    case KVQ_DTYPE_INT2: return g.bs == 64;
+  }
+  return false;
+}
+
+cudaError_t launch_prefill_tc(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s) {
+  const bool pt = a.geo.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD;
+  const bool pc = a.geo.scale_mode == KVQ_SCALE_PER_CHANNEL;
+  switch (a.geo.cache_dtype) {
+    case KVQ_DTYPE_INT8:
+      if (pt) return launch_pf<KVQ_DTYPE_INT8, true, 1>(a, p, s);
+      return pc ? launch_pf<KVQ_DTYPE_INT8, false, 2>(a, p, s) : launch_pf<KVQ_DTYPE_INT8, false, 1>(a, p, s);
+    case KVQ_DTYPE_FP8_E4M3:
+      if (pt) return launch_pf<KVQ_DTYPE_FP8_E4M3, true, 1>(a, p, s);
+      return pc ? launch_pf<KVQ_DTYPE_FP8_E4M3, false, 2>(a, p, s)
+                : launch_pf<KVQ_DTYPE_FP8_E4M3, false, 1>(a, p, s);
+    case KVQ_DTYPE_BF16: return launch_pf<KVQ_DTYPE_BF16, false, 1>(a, p, s);
+    case KVQ_DTYPE_FP16: return launch_pf<KVQ_DTYPE_FP16, false, 1>(a, p, s);
+    // low-bit: bf16 tiles; fp16 activations go to TMEM as an exact bf16 hi + lo pair
+    case KVQ_DTYPE_INT4:
+      return p.act_fp16 ? launch_pf<KVQ_DTYPE_INT4, false, 2>(a, p, s) : launch_pf<KVQ_DTYPE_INT4, false, 1>(a, p, s);
+    case KVQ_DTYPE_INT2:
+      return p.act_fp16 ? launch_pf<KVQ_DTYPE_INT2, false, 2>(a, p, s) : launch_pf<KVQ_DTYPE_INT2, false, 1>(a, p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kvq

@@ -93,13 +93,11 @@ def test_workspace_plan_is_deterministic(lib):
     # the CUDA-core kernel (head_dim 64) with a single split writes the output directly
     assert kvq.kvq_decode_workspace_size(_desc(kvq, num_kv_heads=8, head_dim=64), 1, 8, 16) == 0
     # the tensor-core kernel always merges per-warp partials through the workspace:
-    # (units + CTAs - 1) * 4 partials of g heads, each D floats plus (max, sum), then one
-    # 8-byte arrival counter per unit (148 SMs when no device can be queried)
+    # (units + CTAs - 1) * 4 partials of g heads, each D floats plus (max, sum); 3 CTAs per
+    # SM (148 SMs when no device can be queried)
     ctas, D, g, units = 3 * 148, 128, 1, 8
     heads = (units + ctas - 1) * 4 * g
-    ml_off = (heads * D * 4 + 255) // 256 * 256
-    cnt_off = (ml_off + heads * 8 + 255) // 256 * 256
-    assert kvq.kvq_decode_workspace_size(d, 1, 8, 16) == cnt_off + units * 8
+    assert kvq.kvq_decode_workspace_size(d, 1, 8, 16) == (heads * D * 4 + 255) // 256 * 256 + heads * 8
     with pytest.raises(kvq.KVQError):
         kvq.kvq_decode_workspace_size(d, 2, 12, 100)              # 12 not a multiple of 8
 
@@ -108,8 +106,8 @@ def test_decode_plan_names_the_dispatch(lib):
     """kvq_decode_plan (host only) reports the kernel and launch count of a decode call."""
     from quantized_paged_kv_02_b200 import kvq
     d = _desc(kvq, num_kv_heads=8)
-    assert kvq.kvq_decode_plan(d, 24, 64, 16384) == (1, 1, 3 * 148)       # merges in-kernel
-    assert kvq.kvq_decode_plan(d, 4, 8, 2048)[:2] == (1, 1)               # MHA too (g = 1)
+    assert kvq.kvq_decode_plan(d, 24, 64, 16384) == (1, 2, 3 * 148)       # tensor cores + merge
+    assert kvq.kvq_decode_plan(d, 4, 8, 2048)[:2] == (1, 2)               # MHA too (g = 1)
     assert kvq.kvq_decode_plan(d, 0, 64, 16384)[1] == 0                  # empty batch
     lo = dict(cache_dtype=5, scale_mode=4, block_size=64, num_kv_heads=8)
     k, n, s = kvq.kvq_decode_plan(_desc(kvq, **lo), 16, 64, 32768)

@@ -73,7 +73,7 @@ def test_step_launch_count_comes_from_the_library():
     reports for the decode call (host only: the cache can live in CPU memory here)."""
     import bench
     from quantized_paged_kv_02_b200 import inputs, kvq
-    for name, want in (("c5", 1), ("c4", 3), ("c4-int2", 3)):
+    for name, want in (("c5", 2), ("c4", 3), ("c4-int2", 3)):
         s = inputs._spec(name, False)
         c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, 64, s.block_size,
                              s.num_kv_heads, s.head_dim, device="cpu", max_seqs=s.batch,

@@ -39,7 +39,9 @@ def _prefill(gc, w, q, qs, lens=None):
 
 @pytest.mark.parametrize("name,L", [("c5", [37, 1, 33]), ("c5-fp8", [64, 5, 17]),
                                     ("c5-bf16", [3, 200, 33]), ("c5-int8-pc", [9, 16, 1]),
-                                    ("c3", [7, 30, 1, 12]), ("c2", [40, 19])])
+                                    ("c3", [7, 30, 1, 12]), ("c2", [40, 19]),
+                                    ("c5", [300, 517, 16]), ("c5-int8-ph", [40, 100, 17]),
+                                    ("c5-int8-pt", [128, 3, 33]), ("c5-fp8-pt", [1, 64, 20])])
 def test_prefill_matches_oracle(name, L):
     w = inputs.make(name, small=True)
     L = [min(x, int(n)) for x, n in zip(L, w.context_lens.tolist())]
@@ -83,11 +85,48 @@ def test_rejected_sequences_are_counted_and_left_untouched():
 
 
 def test_prefill_rejects_unsupported_caches():
-    w = inputs.make("c4", small=True)
+    """head_dim 64 has no tensor-core prefill: refused before any launch."""
+    spec = inputs.Spec("pf-d64", "int8", "fp16", "per_token_head", 2, 8, 4, 64, 16, lens=[40, 7],
+                       slack_blocks=1, seed=5)
+    w = inputs.from_spec(spec)
     c = helpers.gpu_cache(w)
     q, qs = _queries(w, [2, 2], 5)
     with pytest.raises(kvq.KVQError):
         _prefill(c, w, q, qs)
+
+
+@pytest.mark.parametrize("name,L", [("c4", [100, 60]), ("c4-tok", [200, 1]), ("c4-fzp", [64, 130]),
+                                    ("c4-int2", [100, 60]), ("c4-int2-tok", [37, 200]),
+                                    ("c4-int2-fzp", [129, 5])])
+def test_prefill_low_bit_matches_oracle(name, L):
+    """INT4 / 2-bit caches: positions below the quantized prefix come from the 64-token
+    blocks (dequantized exactly into bf16 hi + lo tiles), the newest from the residual ring."""
+    w = inputs.make(name, small=True)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    q, qs = _queries(w, L, 10)
+    got = _prefill(gc, w, q, qs).cpu().numpy().astype(np.float64)
+    want = attention.prefill_attention(oc, helpers.np64(q), qs.numpy(), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    err = np.abs(got - want).max()
+    assert err <= TOL, err
+    assert gc.read_fault() == (0, 0)
+
+
+def test_prefill_low_bit_fp16_activations():
+    """fp16 activations with an INT4 cache: q goes to the tensor cores as an exact bf16
+    hi + lo pair."""
+    spec = inputs.Spec("pf-int4-fp16", "int4", "fp16", "kivi", 2, 8, 1, 128, 64, lens=[300, 150],
+                       outliers="k", slack_blocks=2, seed=34)
+    w = inputs.from_spec(spec)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    q, qs = _queries(w, [150, 150], 11)
+    got = _prefill(gc, w, q, qs).cpu().numpy().astype(np.float64)
+    want = attention.prefill_attention(oc, helpers.np64(q), qs.numpy(), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    assert np.abs(got - want).max() <= TOL
+    assert gc.read_fault() == (0, 0)
 
 
 def test_prefill_full_size_sampled_queries():
@@ -129,3 +168,66 @@ def test_more_queries_than_max_q_len_are_rejected():
     assert cnt >= 1 and (bits & 4)
     assert torch.all(out[qs[0]:qs[1]] == 7.0)
     assert torch.all(out[qs[1]:qs[3]] != 7.0)
+
+
+# Other GQA groups, activation types and cache types: g = 2 (64 query tokens per tile) with
+# fp16 activations, an fp16 cache, and MHA with fp16 activations; lengths that put query
+# tiles across 128-token block boundaries and leave ragged last tiles.
+SPECS = {
+    "g2-fp16act": (inputs.Spec("pf-g2", "int8", "fp16", "per_token_head", 3, 4, 2, 128, 16,
+                               lens=[700, 300, 129], slack_blocks=5, seed=31), [257, 64, 129]),
+    "fp16-cache": (inputs.Spec("pf-fp16", "fp16", "fp16", "none", 2, 8, 1, 128, 16,
+                               lens=[400, 130], slack_blocks=2, seed=32), [200, 130]),
+    "fp8-mha-fp16act": (inputs.Spec("pf-mha", "fp8", "fp16", "per_token_head", 2, 2, 2, 128, 16,
+                                    lens=[333, 47], slack_blocks=2, seed=33), [160, 47]),
+}
+
+
+@pytest.mark.parametrize("key", sorted(SPECS))
+def test_prefill_groups_and_types(key):
+    spec, L = SPECS[key]
+    w = inputs.from_spec(spec)
+    static = helpers.oracle_static_scales(w)
+    oc = helpers.oracle_cache(w, static)
+    gc = helpers.gpu_cache(w, static=static)
+    q, qs = _queries(w, L, 8)
+    got = _prefill(gc, w, q, qs).cpu().numpy().astype(np.float64)
+    want = attention.prefill_attention(oc, helpers.np64(q), qs.numpy(), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    err = np.abs(got - want).max()
+    assert err <= TOL, err
+    assert gc.read_fault() == (0, 0)
+
+
+def test_prefill_bad_block_is_masked_and_counted():
+    """A block-table entry outside the pool: its tokens are left out of every query's window
+    (as if masked), the fault record counts it, and nothing else changes."""
+    w = inputs.make("c5", small=True)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    L = [50, 20, 5]
+    q, qs = _queries(w, L, 9)
+    tables = w.block_tables.clone()
+    tables[0, 2] = w.num_blocks + 3                   # positions 32..47 of sequence 0
+    out = gc.prefill(q.cuda(), qs.cuda(), max(L), tables.cuda(), w.context_lens.cuda(),
+                     int(w.context_lens.max())).cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    cnt, bits = gc.read_fault()
+    assert cnt > 0 and (bits & 2)
+    assert np.isfinite(out).all()
+    # sequence 0 without positions 32..47: the oracle over the remaining positions
+    K, V = oc.gather(w.block_tables.numpy()[0], int(w.context_lens[0]))
+    n = int(w.context_lens[0])
+    keep = np.array([p for p in range(n) if not 32 <= p < 48])
+    g = w.spec.num_q_heads // w.spec.num_kv_heads
+    qq = helpers.np64(q)
+    for i in (0, 25, 49):
+        p = n - L[0] + i
+        vis = keep[keep <= p]
+        for hq in range(w.spec.num_q_heads):
+            want = attention.softmax_attention(qq[i, hq], K[hq // g][vis], V[hq // g][vis],
+                                               1.0 / np.sqrt(w.spec.head_dim))
+            assert np.abs(out[i, hq] - want).max() <= TOL, (i, hq)
+    want = attention.prefill_attention(oc, qq, qs.numpy(), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    assert np.abs(out[qs[1]:] - want[qs[1]:]).max() <= TOL

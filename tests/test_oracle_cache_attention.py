@@ -382,6 +382,29 @@ def test_prefill_rows_are_decode_at_their_positions():
             np.testing.assert_array_equal(out[qs[b] + i], want[0])
 
 
+@pytest.mark.parametrize("name", ["c4", "c4-int2-tok"])
+def test_prefill_rows_are_decode_on_low_bit_caches(name):
+    """INT4 / 2-bit caches: query i at position p sees blocks for positions below the
+    quantized prefix of p + 1 and the residual ring above it, exactly what decode with
+    context p + 1 of the same ring sequence sees (the ring holds every position the
+    chunk needs, since the chunk's rows were written before it)."""
+    w = inputs.make(name, small=True)
+    c = _build(w)
+    lens = w.context_lens.numpy()
+    L = np.array([100, 60])
+    qs = np.concatenate([[0], np.cumsum(L)])
+    rng = np.random.default_rng(9)
+    q = fp.bf16_round(rng.standard_normal((qs[-1], w.spec.num_q_heads, w.spec.head_dim)))
+    out = attention.prefill_attention(c, q, qs, w.block_tables.numpy(), lens)
+    for b in range(len(lens)):
+        for i in (0, L[b] // 2, L[b] - 1):
+            p = lens[b] - L[b] + i
+            want = attention.decode_attention(c, q[qs[b] + i][None], w.block_tables.numpy()[b:b + 1],
+                                              np.array([p + 1]), seq_ids=np.array([b]))
+            if c.quantized_prefix(p + 1) == c.quantized_prefix(lens[b]):
+                np.testing.assert_array_equal(out[qs[b] + i], want[0])
+
+
 def test_prefill_grid_exact_equals_causal_sdpa():
     """On a grid-exact INT8 cache the chunk's output equals torch's causal SDPA over the
     dense rows (the prefix positions are all visible, the chunk is causal)."""
