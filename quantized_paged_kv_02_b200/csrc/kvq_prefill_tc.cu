@@ -47,8 +47,8 @@ namespace {
 constexpr int kRows = 128;          // query rows per tile (MMA M)
 constexpr int kBlk = 128;           // cached tokens per block (MMA N of S, K of P V)
 constexpr int kD = 128;
-constexpr int kPfThreads = 320;     // warps 0-3 softmax, 4 producer, 5 MMA, 6-9 converters
-constexpr int kSoftWarps = 4, kProdWarp = 4, kMmaWarp = 5, kConvWarp0 = 6;
+constexpr int kPfThreads = 448;     // warps 0-7 softmax, 8 producer, 9 MMA, 10-13 converters
+constexpr int kSoftWarps = 8, kProdWarp = 8, kMmaWarp = 9, kConvWarp0 = 10;
 constexpr int kNB = 2;              // K / V tile buffers
 constexpr int kTile = 32768;        // 128 x 128 16-bit elements
 constexpr float kRescalePf = 8.f;   // log2 headroom before the running max is re-based
@@ -82,21 +82,29 @@ struct PfLayout {
   static constexpr int VP = LB ? 2 : 1;
   static constexpr int NB = LB ? 1 : kNB;                  // K / V tile buffers
   static constexpr int RS = LB ? 4 : (BITS == 8 ? 16 : 8); // raw ring stages (pages)
+  // pages the producer issues side by side: at most one per stage, so that no lane of a
+  // group waits on a stage another lane of the same group is filling (a wait two phases
+  // ahead of an mbarrier would see the parity of an older phase as complete)
+  static constexpr int IL = RS < 8 ? RS : 8;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = NB * KP * kTile;
   static constexpr int RAW_OFF = V_OFF + NB * VP * kTile;
   static constexpr int KQ_OFF = RAW_OFF + RS * REC;        // float [NB][128]: K multiplier
   static constexpr int VS_OFF = KQ_OFF + NB * kBlk * 4;    // float [NB][128]: V scale
-  static constexpr int MISC_OFF = VS_OFF + NB * kBlk * 4;  // per (buffer, converter warp) vmax
-                                                           // and bad-token counts; flags
+  static constexpr int XM_OFF = VS_OFF + NB * kBlk * 4;    // float [3][2][128]: row maxima of
+                                                           // the two halves (by block parity),
+                                                           // then the row sums
+  static constexpr int MISC_OFF = XM_OFF + 3 * 2 * kRows * 4;  // per (buffer, converter warp)
+                                                               // vmax and bad-token counts; flags
   static constexpr int BAR_OFF = MISC_OFF + 128;
   // raw_full, raw_empty [RS]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
-  // q_ready; fin
-  static constexpr int NBARS = 2 * RS + 3 * NB + 6 + 2;
+  // q_ready; fin; xch [4]
+  static constexpr int NBARS = 2 * RS + 3 * NB + 6 + 2 + 4;
   static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + RS * 4 + 64;
   static_assert(BYTES <= 227 * 1024, "fits the shared memory of one CTA");
   static_assert(BYTES > 114 * 1024, "one CTA per SM, so TMEM allocation never waits on a peer");
   static_assert(RS >= PPB, "a block's pages fit the raw ring");
+  static_assert(IL <= RS, "one issue group never waits on its own stages");
   static_assert(REC % 16 == 0, "bulk copies move multiples of 16 bytes");
   static_assert(NB <= kNB, "scale arrays");
 };
@@ -112,6 +120,8 @@ struct PfShared {
   uint64_t* pv_done;                // [2]: P V of block j commits to pv_done[j % 2]
   uint64_t* q_ready;
   uint64_t* fin;                    // the MMA issuer's final commit
+  uint64_t* xch;                    // [4]: the two softmax warps of a TMEM lane quarter
+  float* xmax;
   int* page_ok;
   float* kq;                        // [NB][128] K multiplier of each token (NaN: bad page)
   float* vs;                        // [NB][128] V scale of each token
@@ -122,11 +132,14 @@ struct PfShared {
   volatile int* abort;
 };
 
-// Bounded wait that also gives up when another role has aborted.
+// Bounded wait that also gives up when another role has aborted.  After a first test the
+// thread sleeps in the barrier (up to 20 us per try, woken by the phase completing), so the
+// roles that wait (producer, MMA issuer, converters) leave the issue slots to the softmax
+// warps that share their SM sub-partitions.
 __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
     if (*abort) return false;
     if (clock64() - t0 > kWaitCycles) return false;
   }
@@ -238,6 +251,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   sh.pv_done = sh.p_full + 2;
   sh.q_ready = sh.pv_done + 2;
   sh.fin = sh.q_ready + 1;
+  sh.xch = sh.fin + 1;
+  sh.xmax = reinterpret_cast<float*>(smem + L::XM_OFF);
   sh.page_ok = reinterpret_cast<int*>(bars + L::NBARS);
   sh.kq = reinterpret_cast<float*>(smem + L::KQ_OFF);
   sh.vs = reinterpret_cast<float*>(smem + L::VS_OFF);
@@ -246,7 +261,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   sh.qscale = reinterpret_cast<float*>(smem + L::MISC_OFF + 64);
   sh.tmem = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF + 68);
   sh.abort = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 72);
-  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 80);   // [4] softmax amax
+  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 80);   // [8] softmax amax
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::RS; ++s) {
@@ -265,6 +280,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     }
     mbar_init(sh.q_ready, kSoftWarps);
     mbar_init(sh.fin, 1);
+    for (int k = 0; k < 4; ++k) mbar_init(&sh.xch[k], 2);
     *sh.abort = 0;
     fence_mbar_init();
   }
@@ -279,8 +295,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     const uint8_t* pages = p.pages;
     int issued = 0;
     bool ok_run = true;
-    for (int k0 = 0; k0 < npg && ok_run; k0 += 8) {
-      const int cnt = min(8, npg - k0);
+    for (int k0 = 0; k0 < npg && ok_run; k0 += L::IL) {
+      const int cnt = min(L::IL, npg - k0);
       bool ok_lane = true;
       if (lane < cnt) {
         const int k = k0 + lane, s = k % L::RS, round = k / L::RS;
@@ -569,21 +585,27 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax (row r)
-    const int r = threadIdx.x;                            // 0..127: TMEM lane = query row
+    // ------------------------------------------------------------ softmax
+    // warp w: query rows 32 (w % 4) .. + 31 (its TMEM lane quarter), score columns
+    // [64 hf, 64 hf + 64) with hf = w / 4; the two warps of a quarter share each row's
+    // running max through a per-quarter mbarrier
+    const int quarter = warp & 3, hf = warp >> 2;
+    const int r = 32 * quarter + lane;                     // query row (TMEM lane)
     const int t_loc = r / g, h = r - t_loc * g;
     const int qi = q0 + t_loc;
     const bool row_ok = qi < Lq;
     const int pos_r = n - Lq + qi;
-    const uint32_t lanebase = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    // --- q row -> TMEM (exact fp16 scaled by 2^-eq for quantized caches; 16-bit caches as is)
+    const uint32_t lanebase = tbase + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int col0 = 64 * hf;                              // this warp's first score column
+    // --- q row, columns [64 hf, 64 hf + 64) -> TMEM (exact fp16 scaled by 2^-eq for
+    // quantized caches; 16-bit caches as is)
     {
       const long qrow = static_cast<long>(p.q_start[b]) + qi;
       const uint4* qp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.q) +
-                                                       (qrow * p.Hq + static_cast<long>(kvh) * g + h) * kD);
+                                                       (qrow * p.Hq + static_cast<long>(kvh) * g + h) * kD + col0);
       // per-channel K scales fold into q (then q goes to TMEM as a hi + lo pair); with
       // bf16 tiles and fp16 activations q is split exactly into bf16 hi + lo
-      const float* kch = p.mode == KVQ_SCALE_PER_CHANNEL ? p.k_static + kvh * kD : nullptr;
+      const float* kch = p.mode == KVQ_SCALE_PER_CHANNEL ? p.k_static + kvh * kD + col0 : nullptr;
       auto elem = [&](const uint4& u, int e) {     // element e (0..7) of 8 packed activations
         const uint32_t w2 = (&u.x)[e >> 1];
         const uint16_t hv = static_cast<uint16_t>((e & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
@@ -599,7 +621,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         float amax = 0.f;
         if (row_ok) {
 #pragma unroll 4
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             const uint4 u = qp[i];
 #pragma unroll
             for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(kch != nullptr ? elem(u, e) * kch[8 * i + e] : elem(u, e)));
@@ -608,47 +630,49 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
         if (lane == 0) red[warp] = amax;
-        named_sync(2, 128);
-        amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        named_sync(2, 32 * kSoftWarps);
+        amax = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kSoftWarps; ++w2) amax = fmaxf(amax, red[w2]);
         int eq = 0;
         if (amax > 0.f && !(p.act_fp16 && kch == nullptr)) eq = ilogbf(amax) - 13;
         down = ldexpf(1.f, -eq);
         qscale = ldexpf(qscale, eq);
       }
+      uint32_t hi[32], lo[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t hi[32], lo[32];
+      for (int i = 0; i < 8; ++i) {
+        const uint4 u = row_ok ? qp[i] : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 u = row_ok ? qp[8 * half + i] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const int d = 64 * half + 8 * i + e;
-            float a = elem(u, e), c2 = elem(u, e + 1);
-            if (kch != nullptr) {
-              a *= kch[d];
-              c2 *= kch[d + 1];
-            }
-            a *= down;
-            c2 *= down;
-            if constexpr (QP == 2) split2<kBf>(a, c2, hi[4 * i + e / 2], lo[4 * i + e / 2]);
-            else hi[4 * i + e / 2] = kBf ? pack_bf16x2(a, c2) : pack_f16x2(a, c2);
+        for (int e = 0; e < 8; e += 2) {
+          const int d = 8 * i + e;
+          float a = elem(u, e), c2 = elem(u, e + 1);
+          if (kch != nullptr) {
+            a *= kch[d];
+            c2 *= kch[d + 1];
           }
+          a *= down;
+          c2 *= down;
+          if constexpr (QP == 2) split2<kBf>(a, c2, hi[4 * i + e / 2], lo[4 * i + e / 2]);
+          else hi[4 * i + e / 2] = kBf ? pack_bf16x2(a, c2) : pack_f16x2(a, c2);
         }
-        tc::st32(lanebase + kTmQ + 32 * half, hi);
-        if constexpr (QP == 2) tc::st32(lanebase + kTmQ + 64 + 32 * half, lo);
       }
+      tc::st32(lanebase + kTmQ + 32 * hf, hi);
+      if constexpr (QP == 2) tc::st32(lanebase + kTmQ + 64 + 32 * hf, lo);
       if (threadIdx.x == 0) *sh.qscale = qscale;
       tc::st_wait();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(sh.q_ready);
     }
-    // --- blocks
+    // --- blocks.  Running max m (re-based lazily) and V normaliser 2^ev (the exponent of the
+    // largest V scale so far) together set the exponent offset of P: e = 2^(x - m - ev), so
+    // that e times a token's V scale stays below 2^10 in fp16; l and O accumulate in that
+    // scaled domain, and the offset cancels in O / l.
     float m = -INFINITY, l = 0.f;
     int ev = INT_MIN;
-    float vinv = 0.f;
     bool ok = true;
+    float* xm = sh.xmax;                                   // [2][2][128]: block parity, half, row
     for (int j = 0; j < J; ++j) {
       const int sb = j & 1, kb = j % NB;
       if (!pf_wait(&sh.k_full[kb], (j / NB) & 1, sh.abort) ||
@@ -657,89 +681,108 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::fence_after_sync();
-      // pass 1: the block's largest scaled score of this row (scores are read from TMEM
-      // again in pass 2, so only 32 of them are live at a time)
-      const float* kq = sh.kq + kb * kBlk;
+      const float* kq = sh.kq + kb * kBlk + col0;
       const bool fast = sh.nbad[kb * 4] + sh.nbad[kb * 4 + 1] + sh.nbad[kb * 4 + 2] + sh.nbad[kb * 4 + 3] == 0 &&
                         j * kBlk + kBlk - 1 <= pmin;   // uniform
       // causal boundary (position <= this row's) and tokens of bad pages (multiplier NaN)
-      const int lim = row_ok ? pos_r - j * kBlk : -1;
-      auto scaled = [&](uint32_t sv, float f, int t) {
-        const float x = __uint_as_float(sv) * f;
-        return (fast || (t <= lim && f == f)) ? x : -INFINITY;
-      };
+      const int lim = row_ok ? pos_r - j * kBlk - col0 : -1;
+      // pass 1: the largest scaled score of this row's 64 columns (read from TMEM again in
+      // pass 2, so only 32 scores are live at a time)
       float mx = -INFINITY;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t sr[32];
-        tc::ld32(lanebase + 128 * sb + 32 * cc, sr);
+        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 f = *reinterpret_cast<const float4*>(kq + 32 * cc + i);
-          const int t = 32 * cc + i;
-          mx = fmaxf(mx, fmaxf(fmaxf(scaled(sr[i], f.x, t), scaled(sr[i + 1], f.y, t + 1)),
-                               fmaxf(scaled(sr[i + 2], f.z, t + 2), scaled(sr[i + 3], f.w, t + 3))));
+          const float2 x01 = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
+                                        make_float2(f.x, f.y));
+          const float2 x23 = __fmul2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
+                                        make_float2(f.z, f.w));
+          float v0 = x01.x, v1 = x01.y, v2 = x23.x, v3 = x23.y;
+          if (!fast) {
+            const int t = 32 * cc + i;
+            if (!(t <= lim && f.x == f.x)) v0 = -INFINITY;
+            if (!(t + 1 <= lim && f.y == f.y)) v1 = -INFINITY;
+            if (!(t + 2 <= lim && f.z == f.z)) v2 = -INFINITY;
+            if (!(t + 3 <= lim && f.w == f.w)) v3 = -INFINITY;
+          }
+          mx = fmaxf(mx, fmaxf(fmaxf(v0, v1), fmaxf(v2, v3)));
         }
       }
+      // the row's max over both halves: exchange with the partner warp of this quarter
+      xm[(sb * 2 + hf) * kRows + r] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.xch[quarter]);
+      if (!pf_wait(&sh.xch[quarter], j & 1, sh.abort)) ok = false;
       if (!pf_wait(&sh.v_full[kb], (j / NB) & 1, sh.abort)) ok = false;
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      // running max (re-based lazily) and V normaliser 2^ev (grows with the largest V scale)
+      mx = fmaxf(mx, xm[(sb * 2 + (hf ^ 1)) * kRows + r]);
+      // rescale factor of l and O: the max re-based (beyond 2^8) and / or the V normaliser
+      // grown (both the same in the two warps of a row)
       float fo = 1.f;
       const float vmx = fmaxf(fmaxf(sh.vmax[kb * 4], sh.vmax[kb * 4 + 1]),
                               fmaxf(sh.vmax[kb * 4 + 2], sh.vmax[kb * 4 + 3]));
       if (vmx > 0.f) {
-        const int e = exponent_of(vmx);
+        // (floored at 2^-100, so that 2^(x - m - ev) stays finite for any V scale)
+        const int e = max(exponent_of(vmx), -100);
         if (e > ev) {
           if (ev != INT_MIN) fo = pow2i(ev - e);
           ev = e;
-          vinv = pow2i(-ev);
         }
       }
       if (mx > m + kRescalePf) {
         const float mn = fmaxf(m, mx);
-        const float c0 = m == -INFINITY ? 0.f : ex2(m - mn);
-        l *= c0;
-        fo *= c0;
+        fo *= m == -INFINITY ? 0.f : ex2(m - mn);
         m = mn;
       }
+      l *= fo;
       if (j > 0 && __any_sync(0xffffffffu, fo != 1.f)) {
-        // rescale this warp's O rows: P V of block j - 1 must be complete
+        // rescale this warp's half of its O rows: P V of block j - 1 must be complete
         if (!pf_wait(&sh.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, sh.abort)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc::fence_after_sync();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tc::ld32(lanebase + kTmO + 32 * cc, o);
+          tc::ld32(lanebase + kTmO + col0 + 32 * cc, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
-          tc::st32(lanebase + kTmO + 32 * cc, o);
+          tc::st32(lanebase + kTmO + col0 + 32 * cc, o);
         }
       }
-      const float base = m == -INFINITY ? 0.f : m;
-      const float* vsp = sh.vs + kb * kBlk;
-      // pass 2: P = 2^(x - base), the row sum, and P times the token's V scale / 2^ev as
-      // hi + lo 16-bit halves over the scores
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      const float off = (m == -INFINITY ? 0.f : m) + (ev == INT_MIN ? 0.f : static_cast<float>(ev));
+      const float* vsp = sh.vs + kb * kBlk + col0;
+      // pass 2: e = 2^(x - off), the row sum, and e times the token's V scale as hi + lo
+      // 16-bit halves over the 32 score columns just read
+      float2 lsum = make_float2(0.f, 0.f);
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t sr[32];
-        tc::ld32(lanebase + 128 * sb + 32 * cc, sr);
+        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int t = 32 * cc + 2 * i;
           const float2 f = *reinterpret_cast<const float2*>(kq + t);
-          const float e0 = ex2(scaled(sr[2 * i], f.x, t) - base);
-          const float e1 = ex2(scaled(sr[2 * i + 1], f.y, t + 1) - base);
-          l += e0 + e1;
-          const float2 v2 = *reinterpret_cast<const float2*>(vsp + t);
-          split2<kBf>(e0 * v2.x * vinv, e1 * v2.y * vinv, ph[i], pl[i]);
+          float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), f,
+                                make_float2(-off, -off));
+          if (!fast) {
+            if (!(t <= lim && f.x == f.x)) x.x = -INFINITY;
+            if (!(t + 1 <= lim && f.y == f.y)) x.y = -INFINITY;
+          }
+          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          lsum = __fadd2_rn(lsum, e);
+          const float2 w = __fmul2_rn(e, *reinterpret_cast<const float2*>(vsp + t));
+          split2<kBf>(w.x, w.y, ph[i], pl[i]);
         }
         // the 32 score columns just read take P of the same 32 tokens: hi halves in the
         // first 16 columns, lo halves in the next 16
-        st16(lanebase + 128 * sb + 32 * cc, ph);
-        st16(lanebase + 128 * sb + 32 * cc + 16, pl);
+        st16(lanebase + 128 * sb + col0 + 32 * cc, ph);
+        st16(lanebase + 128 * sb + col0 + 32 * cc + 16, pl);
       }
+      l += lsum.x + lsum.y;
       tc::st_wait();
       tc::fence_before_sync();
       __syncwarp();
@@ -748,26 +791,32 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     if (!ok) {
       if (lane == 0) pf_fail(p, sh.abort);
     } else {
-      // --- epilogue: O / l (times 2^ev and the static V scales) -> out
+      // --- epilogue: the row sum over both halves, then O / l (times the static V scales)
+      // for this warp's 64 output columns
+      xm[(2 * 2 + hf) * kRows + r] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.xch[quarter]);
+      if (!pf_wait(&sh.xch[quarter], J & 1, sh.abort)) ok = false;
       if (!pf_wait(&sh.pv_done[(J - 1) & 1], ((J - 1) >> 1) & 1, sh.abort)) ok = false;
       if (__all_sync(0xffffffffu, ok)) {
         tc::fence_after_sync();
+        const float lt = l + xm[(2 * 2 + (hf ^ 1)) * kRows + r];
         float vmul = 1.f;
         if (p.mode == KVQ_SCALE_PER_HEAD) vmul = p.v_static[kvh];
         if (p.mode == KVQ_SCALE_PER_TENSOR) vmul = p.v_static[0];
-        const float inv = l > 0.f ? vmul * pow2i(ev == INT_MIN ? 0 : ev) / l : 0.f;
-        const float* vch = (p.mode == KVQ_SCALE_PER_CHANNEL) ? p.v_static + kvh * kD : nullptr;
+        const float inv = lt > 0.f ? vmul / lt : 0.f;
+        const float* vch = (p.mode == KVQ_SCALE_PER_CHANNEL) ? p.v_static + kvh * kD + col0 : nullptr;
         const long orow = (static_cast<long>(p.q_start[b]) + qi) * p.Hq + static_cast<long>(kvh) * g + h;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tc::ld32(lanebase + kTmO + 32 * cc, o);
+          tc::ld32(lanebase + kTmO + col0 + 32 * cc, o);
           if (row_ok) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int d = 32 * cc + i;
               const float v = __uint_as_float(o[i]) * inv * (vch != nullptr ? vch[d] : 1.f);
-              store_out(p, orow * kD + d, v);
+              store_out(p, orow * kD + col0 + d, v);
             }
           }
         }

@@ -113,6 +113,23 @@ def test_prefill_low_bit_matches_oracle(name, L):
     assert gc.read_fault() == (0, 0)
 
 
+@pytest.mark.parametrize("cd,mode", [("int4", "kivi"), ("int2", "int4_per_token")])
+def test_prefill_low_bit_long_context(cd, mode):
+    """1200 cached tokens (16 blocks of 64 in the quantized prefix, so the four-stage page
+    ring of the low-bit prefill turns over four times) and 300 queries."""
+    spec = inputs.Spec("pf-%s-long" % cd, cd, "bf16", mode, 1, 16, 2, 128, 64, lens=[1200],
+                       outliers="k", slack_blocks=3, seed=35)
+    w = inputs.from_spec(spec)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    q, qs = _queries(w, [300], 12)
+    got = _prefill(gc, w, q, qs).cpu().numpy().astype(np.float64)
+    want = attention.prefill_attention(oc, helpers.np64(q), qs.numpy(), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    assert np.abs(got - want).max() <= TOL
+    assert gc.read_fault() == (0, 0)
+
+
 def test_prefill_low_bit_fp16_activations():
     """fp16 activations with an INT4 cache: q goes to the tensor cores as an exact bf16
     hi + lo pair."""
