@@ -36,6 +36,7 @@
 
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "kvq_decode_common.cuh"
 #include "kvq_ptx.cuh"
@@ -335,6 +336,78 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     const float qsc = *sh.qscale;
     const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
     const int G = c >> 3;                                 // 64-channel group of the chunk
+    // Dense caches: the K (or V) rows of every page of block j -> tile buffer kb, chunk c of
+    // rows rr and rr + 8 of each page: all loads first, then conversions and stores.  The
+    // threads with c == 0 also write the block's per-token multipliers (K: softmax scale x
+    // K scale, NaN for a bad page; V: the V scale) for their 16 tokens and count bad tokens;
+    // after V the warp releases the pages' raw stages.  Returns the largest V scale seen.
+    auto dense_part = [&](int j, int kb, bool isv, int& bad) -> float {
+      constexpr int PPB = L::PPB;
+      using RawT = typename std::conditional<L::BITS == 8, uint2, uint4>::type;
+      RawT w[PPB][2];
+      uint32_t pok = 0;
+#pragma unroll
+      for (int pp = 0; pp < PPB; ++pp) {
+        const int k = j * PPB + pp, s = k % L::RS;
+        if (k < npg && sh.page_ok[s]) pok |= 1u << pp;
+        const uint8_t* src = smem + L::RAW_OFF + s * L::REC + (isv ? L::OFF_V : 0);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          w[pp][h] = *reinterpret_cast<const RawT*>(src + (rr + 8 * h) * L::ROWB + static_cast<int>(sizeof(RawT)) * c);
+      }
+      uint8_t* tile = smem + (isv ? L::V_OFF : L::K_OFF) + kb * kTile;
+#pragma unroll
+      for (int pp = 0; pp < PPB; ++pp)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int t = pp * BS + rr + 8 * h;
+          const bool valid = ((pok >> pp) & 1u) && j * kBlk + t <= pmax;
+          uint4 out = make_uint4(0, 0, 0, 0);
+          if constexpr (L::BITS == 8) {
+            const uint4 cv = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w[pp][h]) : e4m3x8_to_f16(w[pp][h]);
+            if (valid) out = cv;
+          } else {
+            if (valid) out = w[pp][h];
+          }
+          *reinterpret_cast<uint4*>(tile + tile_off(t, c)) = out;
+        }
+      float vm = 0.f;
+      if (c == 0) {
+#pragma unroll
+        for (int pp = 0; pp < PPB; ++pp)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int k = j * PPB + pp, row = rr + 8 * h, t = pp * BS + row, pos = j * kBlk + t;
+            const bool have = k < npg, pk = (pok >> pp) & 1u;
+            const bool valid = pk && pos <= pmax;
+            const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
+            if (!isv) {
+              float ks = 1.f;
+              if constexpr (PT) ks = sc[row];
+              // tokens of a bad page are marked NaN (masked by the softmax); positions past
+              // the tile's last query are never visible, so their multiplier does not matter
+              const bool badtok = have && !pk && pos <= pmax;
+              sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+              bad += badtok;
+            } else {
+              float vv = 1.f;
+              if constexpr (PT) vv = sc[BS + row];
+              vv = valid ? vv : 0.f;
+              sh.vs[kb * kBlk + t] = vv;
+              vm = fmaxf(vm, vv);
+            }
+          }
+      }
+      if (isv) {
+        __syncwarp();
+#pragma unroll
+        for (int pp = 0; pp < PPB; ++pp) {
+          const int k = j * PPB + pp;
+          if (k < npg && lane == 0) mbar_arrive(&sh.raw_empty[k % L::RS]);   // K and V read
+        }
+      }
+      return vm;
+    };
     for (int j = 0; j < J && !*sh.abort; ++j) {
       const int kb = j % NB;
       // the softmax of block j - NB is done with this buffer's scales (and S j - NB with K)
@@ -344,8 +417,19 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       }
       int bad = 0;
       bool ok = true;
-      // K: rows rr + 8i of every page of the block, chunk c
-      for (int pp = 0; pp < L::PPB && ok; ++pp) {
+      if constexpr (!L::LB) {
+        // K of the whole block, rows rr and rr + 8 of every page, chunk c: wait for the pages
+        // (requested a block ago, usually landed), then issue every load before converting,
+        // so a converter thread has 16 independent loads in flight instead of one chain
+#pragma unroll
+        for (int pp = 0; pp < L::PPB; ++pp) {
+          const int k = j * L::PPB + pp;
+          if (k < npg && !pf_wait(&sh.raw_full[k % L::RS], (k / L::RS) & 1, sh.abort)) ok = false;
+        }
+        if (__all_sync(0xffffffffu, ok)) dense_part(j, kb, false, bad);
+      }
+      // K: rows rr + 8i of every page of the block, chunk c (low-bit caches)
+      for (int pp = 0; pp < L::PPB && ok && L::LB; ++pp) {
         const int k = j * L::PPB + pp;
         const bool have = k < npg;
         const int s = k % L::RS;
@@ -355,32 +439,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         }
         const bool pok = have && sh.page_ok[s];
         const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
-        if constexpr (!L::LB) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int row = rr + 8 * h, t = pp * BS + row, pos = j * kBlk + t;
-            const bool valid = pok && pos <= pmax;
-            uint4 out = make_uint4(0, 0, 0, 0);
-            if (valid) {
-              if constexpr (L::BITS == 8) {
-                const uint2 w = *reinterpret_cast<const uint2*>(raw + row * L::ROWB + 8 * c);
-                out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w) : e4m3x8_to_f16(w);
-              } else {
-                out = *reinterpret_cast<const uint4*>(raw + row * L::ROWB + 16 * c);
-              }
-            }
-            *reinterpret_cast<uint4*>(smem + L::K_OFF + kb * kTile + tile_off(t, c)) = out;
-            if (c == 0) {
-              float ks = 1.f;
-              if constexpr (PT) ks = reinterpret_cast<const float*>(raw + L::OFF_S)[row];
-              // tokens of a bad page are marked NaN (masked by the softmax); positions past
-              // the tile's last query are never visible, so their multiplier does not matter
-              const bool badtok = have && !pok && pos <= pmax;
-              sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
-              bad += badtok;
-            }
-          }
-        } else {
+        {
           // per-channel K parameters of this chunk (KIVI forms): s[8c..8c+7], z or minimum
           float ksc[8], kzp[8];
           if (!ktok && pok) {
@@ -450,36 +509,14 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         break;
       }
       float vm = 0.f;
-      for (int pp = 0; pp < L::PPB; ++pp) {
+      if constexpr (!L::LB) vm = dense_part(j, kb, true, bad);
+      for (int pp = 0; pp < L::PPB && L::LB; ++pp) {
         const int k = j * L::PPB + pp;
         const bool have = k < npg;
         const int s = k % L::RS;
         const bool pok = have && sh.page_ok[s];
         const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
-        if constexpr (!L::LB) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int row = rr + 8 * h, t = pp * BS + row, pos = j * kBlk + t;
-            const bool valid = pok && pos <= pmax;
-            uint4 out = make_uint4(0, 0, 0, 0);
-            if (valid) {
-              if constexpr (L::BITS == 8) {
-                const uint2 w = *reinterpret_cast<const uint2*>(raw + L::OFF_V + row * L::ROWB + 8 * c);
-                out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w) : e4m3x8_to_f16(w);
-              } else {
-                out = *reinterpret_cast<const uint4*>(raw + L::OFF_V + row * L::ROWB + 16 * c);
-              }
-            }
-            *reinterpret_cast<uint4*>(smem + L::V_OFF + kb * kTile + tile_off(t, c)) = out;
-            if (c == 0) {
-              float vv = 1.f;
-              if constexpr (PT) vv = reinterpret_cast<const float*>(raw + L::OFF_S)[BS + row];
-              vv = valid ? vv : 0.f;
-              sh.vs[kb * kBlk + t] = vv;
-              vm = fmaxf(vm, vv);
-            }
-          }
-        } else {
+        {
           for (int i = 0; i < BS / 8; ++i) {
             const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
             const bool ring = pos >= si.qb;
