@@ -355,55 +355,47 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         for (int h = 0; h < 2; ++h)
           w[pp][h] = *reinterpret_cast<const RawT*>(src + (rr + 8 * h) * L::ROWB + static_cast<int>(sizeof(RawT)) * c);
       }
-      uint8_t* tile = smem + (isv ? L::V_OFF : L::K_OFF) + kb * kTile;
+      // every page present and every position visible to some query: no per-row tests
+      const bool whole = pok == (1u << PPB) - 1u && j * kBlk + kBlk - 1 <= pmax;
+      // row t of the tile: t & 7 == rr & 7 for all of this thread's rows, so the swizzled
+      // chunk is the same for all; only the row offset changes
+      uint8_t* tile = smem + (isv ? L::V_OFF : L::K_OFF) + kb * kTile + tile_off(rr, c) - rr * 128;
 #pragma unroll
       for (int pp = 0; pp < PPB; ++pp)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int t = pp * BS + rr + 8 * h;
-          const bool valid = ((pok >> pp) & 1u) && j * kBlk + t <= pmax;
-          uint4 out = make_uint4(0, 0, 0, 0);
-          if constexpr (L::BITS == 8) {
-            const uint4 cv = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w[pp][h]) : e4m3x8_to_f16(w[pp][h]);
-            if (valid) out = cv;
-          } else {
-            if (valid) out = w[pp][h];
-          }
-          *reinterpret_cast<uint4*>(tile + tile_off(t, c)) = out;
+          uint4 out;
+          if constexpr (L::BITS == 8) out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w[pp][h]) : e4m3x8_to_f16(w[pp][h]);
+          else out = w[pp][h];
+          if (!whole && !(((pok >> pp) & 1u) && j * kBlk + t <= pmax)) out = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(tile + t * 128) = out;
         }
+      // this thread's token t = ct: its K multiplier (softmax scale x K scale; NaN on a bad
+      // page, masked by the softmax) or its V scale
+      const int t = ct, pp = t >> 4, row = t & 15, k = j * PPB + pp, pos = j * kBlk + t;
+      const bool have = k < npg, pk = (pok >> pp) & 1u;
+      const bool valid = pk && pos <= pmax;
+      const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
       float vm = 0.f;
-      if (c == 0) {
-#pragma unroll
-        for (int pp = 0; pp < PPB; ++pp)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int k = j * PPB + pp, row = rr + 8 * h, t = pp * BS + row, pos = j * kBlk + t;
-            const bool have = k < npg, pk = (pok >> pp) & 1u;
-            const bool valid = pk && pos <= pmax;
-            const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
-            if (!isv) {
-              float ks = 1.f;
-              if constexpr (PT) ks = sc[row];
-              // tokens of a bad page are marked NaN (masked by the softmax); positions past
-              // the tile's last query are never visible, so their multiplier does not matter
-              const bool badtok = have && !pk && pos <= pmax;
-              sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
-              bad += badtok;
-            } else {
-              float vv = 1.f;
-              if constexpr (PT) vv = sc[BS + row];
-              vv = valid ? vv : 0.f;
-              sh.vs[kb * kBlk + t] = vv;
-              vm = fmaxf(vm, vv);
-            }
-          }
-      }
-      if (isv) {
+      if (!isv) {
+        float ks = 1.f;
+        if constexpr (PT) ks = sc[row];
+        // positions past the tile's last query are never visible: their multiplier is unused
+        const bool badtok = have && !pk && pos <= pmax;
+        sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+        bad += badtok;
+      } else {
+        float vv = 1.f;
+        if constexpr (PT) vv = sc[BS + row];
+        vv = valid ? vv : 0.f;
+        sh.vs[kb * kBlk + t] = vv;
+        vm = vv;
         __syncwarp();
 #pragma unroll
-        for (int pp = 0; pp < PPB; ++pp) {
-          const int k = j * PPB + pp;
-          if (k < npg && lane == 0) mbar_arrive(&sh.raw_empty[k % L::RS]);   // K and V read
+        for (int q = 0; q < PPB; ++q) {
+          const int kk = j * PPB + q;
+          if (kk < npg && lane == 0) mbar_arrive(&sh.raw_empty[kk % L::RS]);   // K and V read
         }
       }
       return vm;
@@ -723,29 +715,28 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
                         j * kBlk + kBlk - 1 <= pmin;   // uniform
       // causal boundary (position <= this row's) and tokens of bad pages (multiplier NaN)
       const int lim = row_ok ? pos_r - j * kBlk - col0 : -1;
-      // pass 1: the largest scaled score of this row's 64 columns (read from TMEM again in
-      // pass 2, so only 32 scores are live at a time)
+      // pass 1: this row's 64 scores (one TMEM load), scaled and masked, kept in registers
+      // for pass 2, and their largest
+      float x[64];
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sr[32];
-        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
+      {
+        uint32_t sr[64];
+        tc::ld64(lanebase + 128 * sb + col0, sr);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float4 f = *reinterpret_cast<const float4*>(kq + 32 * cc + i);
+        for (int i = 0; i < 64; i += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(kq + i);
           const float2 x01 = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
                                         make_float2(f.x, f.y));
           const float2 x23 = __fmul2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
                                         make_float2(f.z, f.w));
-          float v0 = x01.x, v1 = x01.y, v2 = x23.x, v3 = x23.y;
+          x[i] = x01.x; x[i + 1] = x01.y; x[i + 2] = x23.x; x[i + 3] = x23.y;
           if (!fast) {
-            const int t = 32 * cc + i;
-            if (!(t <= lim && f.x == f.x)) v0 = -INFINITY;
-            if (!(t + 1 <= lim && f.y == f.y)) v1 = -INFINITY;
-            if (!(t + 2 <= lim && f.z == f.z)) v2 = -INFINITY;
-            if (!(t + 3 <= lim && f.w == f.w)) v3 = -INFINITY;
+            if (!(i <= lim && f.x == f.x)) x[i] = -INFINITY;
+            if (!(i + 1 <= lim && f.y == f.y)) x[i + 1] = -INFINITY;
+            if (!(i + 2 <= lim && f.z == f.z)) x[i + 2] = -INFINITY;
+            if (!(i + 3 <= lim && f.w == f.w)) x[i + 3] = -INFINITY;
           }
-          mx = fmaxf(mx, fmaxf(fmaxf(v0, v1), fmaxf(v2, v3)));
+          mx = fmaxf(mx, fmaxf(fmaxf(x[i], x[i + 1]), fmaxf(x[i + 2], x[i + 3])));
         }
       }
       // the row's max over both halves: exchange with the partner warp of this quarter
@@ -781,41 +772,32 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t o[32];
-          tc::ld32(lanebase + kTmO + col0 + 32 * cc, o);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[16];
+          tc::ld16(lanebase + kTmO + col0 + 16 * cc, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
-          tc::st32(lanebase + kTmO + col0 + 32 * cc, o);
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
+          st16(lanebase + kTmO + col0 + 16 * cc, o);
         }
       }
       const float off = (m == -INFINITY ? 0.f : m) + (ev == INT_MIN ? 0.f : static_cast<float>(ev));
       const float* vsp = sh.vs + kb * kBlk + col0;
       // pass 2: e = 2^(x - off), the row sum, and e times the token's V scale as hi + lo
-      // 16-bit halves over the 32 score columns just read
+      // 16-bit halves over the score columns (each 32-column chunk: hi halves in its first 16
+      // columns, lo halves in the next 16)
       float2 lsum = make_float2(0.f, 0.f);
-#pragma unroll 1
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sr[32];
-        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int t = 32 * cc + 2 * i;
-          const float2 f = *reinterpret_cast<const float2*>(kq + t);
-          float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), f,
-                                make_float2(-off, -off));
-          if (!fast) {
-            if (!(t <= lim && f.x == f.x)) x.x = -INFINITY;
-            if (!(t + 1 <= lim && f.y == f.y)) x.y = -INFINITY;
-          }
-          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          const float2 xo = __fadd2_rn(make_float2(x[t], x[t + 1]), make_float2(-off, -off));
+          const float2 e = make_float2(ex2(xo.x), ex2(xo.y));
           lsum = __fadd2_rn(lsum, e);
           const float2 w = __fmul2_rn(e, *reinterpret_cast<const float2*>(vsp + t));
           split2<kBf>(w.x, w.y, ph[i], pl[i]);
         }
-        // the 32 score columns just read take P of the same 32 tokens: hi halves in the
-        // first 16 columns, lo halves in the next 16
         st16(lanebase + 128 * sb + col0 + 32 * cc, ph);
         st16(lanebase + 128 * sb + col0 + 32 * cc + 16, pl);
       }
