@@ -211,6 +211,75 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
   split2<true>(v[6], v[7], hi.w, lo.w);
 }
 
+// Dense caches, converter thread (c, rr) = (ct % 16, ct / 16): the K (or V) rows of every
+// page of block j -> tile buffer kb, chunk c of rows rr and rr + 8 of each page; all loads
+// first, then conversions and stores.  Thread ct also writes token ct's multiplier (K:
+// softmax scale x K scale, NaN for a bad page; V: the V scale) and counts its bad token;
+// after V the warp releases the pages' raw stages.  Returns token ct's V scale (0 for K).
+// Not inlined: one copy of the code serves both halves, which keeps the kernel's hot code
+// inside the instruction cache.
+template <int CD, bool PT>
+__device__ __noinline__ float dense_part(uint8_t* smem, const PfShared& sh, int j, int kb, bool isv,
+                                         int ct, int npg, int pmax, float qsc, int* bad) {
+  using L = PfLayout<CD, PT>;
+  constexpr int PPB = L::PPB, BS = L::BS;
+  using RawT = typename std::conditional<L::BITS == 8, uint2, uint4>::type;
+  const int c = ct & 15, rr = ct >> 4, lane = ct & 31;
+  RawT w[PPB][2];
+  uint32_t pok = 0;
+#pragma unroll
+  for (int pp = 0; pp < PPB; ++pp) {
+    const int k = j * PPB + pp, s = k % L::RS;
+    if (k < npg && sh.page_ok[s]) pok |= 1u << pp;
+    const uint8_t* src = smem + L::RAW_OFF + s * L::REC + (isv ? L::OFF_V : 0);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      w[pp][h] = *reinterpret_cast<const RawT*>(src + (rr + 8 * h) * L::ROWB + static_cast<int>(sizeof(RawT)) * c);
+  }
+  // every page present and every position visible to some query: no per-row tests
+  const bool whole = pok == (1u << PPB) - 1u && j * kBlk + kBlk - 1 <= pmax;
+  // row t of the tile: t & 7 == rr & 7 for all of this thread's rows, so the swizzled chunk is
+  // the same for all; only the row offset changes
+  uint8_t* tile = smem + (isv ? L::V_OFF : L::K_OFF) + kb * kTile + tile_off(rr, c) - rr * 128;
+#pragma unroll
+  for (int pp = 0; pp < PPB; ++pp)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int t = pp * BS + rr + 8 * h;
+      uint4 out;
+      if constexpr (L::BITS == 8) out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w[pp][h]) : e4m3x8_to_f16(w[pp][h]);
+      else out = w[pp][h];
+      if (!whole && !(((pok >> pp) & 1u) && j * kBlk + t <= pmax)) out = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(tile + t * 128) = out;
+    }
+  const int t = ct, pp = t >> 4, row = t & 15, k = j * PPB + pp, pos = j * kBlk + t;
+  const bool have = k < npg, pk = (pok >> pp) & 1u;
+  const bool valid = pk && pos <= pmax;
+  const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
+  float vm = 0.f;
+  if (!isv) {
+    float ks = 1.f;
+    if constexpr (PT) ks = sc[row];
+    // positions past the tile's last query are never visible: their multiplier is unused
+    const bool badtok = have && !pk && pos <= pmax;
+    sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+    *bad += badtok;
+  } else {
+    float vv = 1.f;
+    if constexpr (PT) vv = sc[BS + row];
+    vv = valid ? vv : 0.f;
+    sh.vs[kb * kBlk + t] = vv;
+    vm = vv;
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < PPB; ++q) {
+      const int kk = j * PPB + q;
+      if (kk < npg && lane == 0) mbar_arrive(&sh.raw_empty[kk % L::RS]);   // K and V read
+    }
+  }
+  return vm;
+}
+
 template <int CD, bool PT, int QP>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
@@ -336,70 +405,6 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     const float qsc = *sh.qscale;
     const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
     const int G = c >> 3;                                 // 64-channel group of the chunk
-    // Dense caches: the K (or V) rows of every page of block j -> tile buffer kb, chunk c of
-    // rows rr and rr + 8 of each page: all loads first, then conversions and stores.  The
-    // threads with c == 0 also write the block's per-token multipliers (K: softmax scale x
-    // K scale, NaN for a bad page; V: the V scale) for their 16 tokens and count bad tokens;
-    // after V the warp releases the pages' raw stages.  Returns the largest V scale seen.
-    auto dense_part = [&](int j, int kb, bool isv, int& bad) -> float {
-      constexpr int PPB = L::PPB;
-      using RawT = typename std::conditional<L::BITS == 8, uint2, uint4>::type;
-      RawT w[PPB][2];
-      uint32_t pok = 0;
-#pragma unroll
-      for (int pp = 0; pp < PPB; ++pp) {
-        const int k = j * PPB + pp, s = k % L::RS;
-        if (k < npg && sh.page_ok[s]) pok |= 1u << pp;
-        const uint8_t* src = smem + L::RAW_OFF + s * L::REC + (isv ? L::OFF_V : 0);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          w[pp][h] = *reinterpret_cast<const RawT*>(src + (rr + 8 * h) * L::ROWB + static_cast<int>(sizeof(RawT)) * c);
-      }
-      // every page present and every position visible to some query: no per-row tests
-      const bool whole = pok == (1u << PPB) - 1u && j * kBlk + kBlk - 1 <= pmax;
-      // row t of the tile: t & 7 == rr & 7 for all of this thread's rows, so the swizzled
-      // chunk is the same for all; only the row offset changes
-      uint8_t* tile = smem + (isv ? L::V_OFF : L::K_OFF) + kb * kTile + tile_off(rr, c) - rr * 128;
-#pragma unroll
-      for (int pp = 0; pp < PPB; ++pp)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int t = pp * BS + rr + 8 * h;
-          uint4 out;
-          if constexpr (L::BITS == 8) out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w[pp][h]) : e4m3x8_to_f16(w[pp][h]);
-          else out = w[pp][h];
-          if (!whole && !(((pok >> pp) & 1u) && j * kBlk + t <= pmax)) out = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(tile + t * 128) = out;
-        }
-      // this thread's token t = ct: its K multiplier (softmax scale x K scale; NaN on a bad
-      // page, masked by the softmax) or its V scale
-      const int t = ct, pp = t >> 4, row = t & 15, k = j * PPB + pp, pos = j * kBlk + t;
-      const bool have = k < npg, pk = (pok >> pp) & 1u;
-      const bool valid = pk && pos <= pmax;
-      const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
-      float vm = 0.f;
-      if (!isv) {
-        float ks = 1.f;
-        if constexpr (PT) ks = sc[row];
-        // positions past the tile's last query are never visible: their multiplier is unused
-        const bool badtok = have && !pk && pos <= pmax;
-        sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
-        bad += badtok;
-      } else {
-        float vv = 1.f;
-        if constexpr (PT) vv = sc[BS + row];
-        vv = valid ? vv : 0.f;
-        sh.vs[kb * kBlk + t] = vv;
-        vm = vv;
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < PPB; ++q) {
-          const int kk = j * PPB + q;
-          if (kk < npg && lane == 0) mbar_arrive(&sh.raw_empty[kk % L::RS]);   // K and V read
-        }
-      }
-      return vm;
-    };
     for (int j = 0; j < J && !*sh.abort; ++j) {
       const int kb = j % NB;
       // the softmax of block j - NB is done with this buffer's scales (and S j - NB with K)
@@ -418,7 +423,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
           const int k = j * L::PPB + pp;
           if (k < npg && !pf_wait(&sh.raw_full[k % L::RS], (k / L::RS) & 1, sh.abort)) ok = false;
         }
-        if (__all_sync(0xffffffffu, ok)) dense_part(j, kb, false, bad);
+        if (__all_sync(0xffffffffu, ok)) dense_part<CD, PT>(smem, sh, j, kb, false, ct, npg, pmax, qsc, &bad);
       }
       // K: rows rr + 8i of every page of the block, chunk c (low-bit caches)
       for (int pp = 0; pp < L::PPB && ok && L::LB; ++pp) {
@@ -501,7 +506,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         break;
       }
       float vm = 0.f;
-      if constexpr (!L::LB) vm = dense_part(j, kb, true, bad);
+      if constexpr (!L::LB) vm = dense_part<CD, PT>(smem, sh, j, kb, true, ct, npg, pmax, qsc, &bad);
       for (int pp = 0; pp < L::PPB && L::LB; ++pp) {
         const int k = j * L::PPB + pp;
         const bool have = k < npg;
@@ -715,28 +720,23 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
                         j * kBlk + kBlk - 1 <= pmin;   // uniform
       // causal boundary (position <= this row's) and tokens of bad pages (multiplier NaN)
       const int lim = row_ok ? pos_r - j * kBlk - col0 : -1;
-      // pass 1: this row's 64 scores (one TMEM load), scaled and masked, kept in registers
-      // for pass 2, and their largest
-      float x[64];
+      // pass 1: the largest scaled score of this row's 64 columns, 32 at a time (read from
+      // TMEM again in pass 2; the loops are not unrolled, to keep the hot code small)
+      auto scaled = [&](uint32_t sv, float f, int t) {
+        const float v = __uint_as_float(sv) * f;
+        return (fast || (t <= lim && f == f)) ? v : -INFINITY;
+      };
       float mx = -INFINITY;
-      {
-        uint32_t sr[64];
-        tc::ld64(lanebase + 128 * sb + col0, sr);
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sr[32];
+        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
 #pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-          const float4 f = *reinterpret_cast<const float4*>(kq + i);
-          const float2 x01 = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
-                                        make_float2(f.x, f.y));
-          const float2 x23 = __fmul2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
-                                        make_float2(f.z, f.w));
-          x[i] = x01.x; x[i + 1] = x01.y; x[i + 2] = x23.x; x[i + 3] = x23.y;
-          if (!fast) {
-            if (!(i <= lim && f.x == f.x)) x[i] = -INFINITY;
-            if (!(i + 1 <= lim && f.y == f.y)) x[i + 1] = -INFINITY;
-            if (!(i + 2 <= lim && f.z == f.z)) x[i + 2] = -INFINITY;
-            if (!(i + 3 <= lim && f.w == f.w)) x[i + 3] = -INFINITY;
-          }
-          mx = fmaxf(mx, fmaxf(fmaxf(x[i], x[i + 1]), fmaxf(x[i + 2], x[i + 3])));
+        for (int i = 0; i < 32; i += 4) {
+          const int t = 32 * cc + i;
+          const float4 f = *reinterpret_cast<const float4*>(kq + t);
+          mx = fmaxf(mx, fmaxf(fmaxf(scaled(sr[i], f.x, t), scaled(sr[i + 1], f.y, t + 1)),
+                               fmaxf(scaled(sr[i + 2], f.z, t + 2), scaled(sr[i + 3], f.w, t + 3))));
         }
       }
       // the row's max over both halves: exchange with the partner warp of this quarter
@@ -783,16 +783,24 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       const float off = (m == -INFINITY ? 0.f : m) + (ev == INT_MIN ? 0.f : static_cast<float>(ev));
       const float* vsp = sh.vs + kb * kBlk + col0;
       // pass 2: e = 2^(x - off), the row sum, and e times the token's V scale as hi + lo
-      // 16-bit halves over the score columns (each 32-column chunk: hi halves in its first 16
-      // columns, lo halves in the next 16)
+      // 16-bit halves over the 32 score columns just read (each chunk: hi halves in its
+      // first 16 columns, lo halves in the next 16)
       float2 lsum = make_float2(0.f, 0.f);
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sr[32];
+        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
         uint32_t ph[16], pl[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int t = 32 * cc + 2 * i;
-          const float2 xo = __fadd2_rn(make_float2(x[t], x[t + 1]), make_float2(-off, -off));
+          const float2 f = *reinterpret_cast<const float2*>(kq + t);
+          float2 xo = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), f,
+                                 make_float2(-off, -off));
+          if (!fast) {
+            if (!(t <= lim && f.x == f.x)) xo.x = -INFINITY;
+            if (!(t + 1 <= lim && f.y == f.y)) xo.y = -INFINITY;
+          }
           const float2 e = make_float2(ex2(xo.x), ex2(xo.y));
           lsum = __fadd2_rn(lsum, e);
           const float2 w = __fmul2_rn(e, *reinterpret_cast<const float2*>(vsp + t));
@@ -831,11 +839,28 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
           uint32_t o[32];
           tc::ld32(lanebase + kTmO + col0 + 32 * cc, o);
           if (row_ok) {
+            float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int d = 32 * cc + i;
-              const float v = __uint_as_float(o[i]) * inv * (vch != nullptr ? vch[d] : 1.f);
-              store_out(p, orow * kD + col0 + d, v);
+            for (int i = 0; i < 32; ++i)
+              v[i] = __uint_as_float(o[i]) * inv * (vch != nullptr ? vch[32 * cc + i] : 1.f);
+            const long e0 = orow * kD + col0 + 32 * cc;          // a multiple of 32 elements
+            if (p.out_dtype == KVQ_DTYPE_FP32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + e0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              const bool bf = p.out_dtype == KVQ_DTYPE_BF16;
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + e0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t q4[4];
+#pragma unroll
+                for (int k2 = 0; k2 < 4; ++k2) {
+                  const float a0 = v[8 * i + 2 * k2], a1 = v[8 * i + 2 * k2 + 1];
+                  q4[k2] = bf ? pack_bf16x2(a0, a1) : pack_f16x2(a0, a1);
+                }
+                dst[i] = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+              }
             }
           }
         }
