@@ -175,16 +175,28 @@ __device__ __forceinline__ uint32_t tile_off(int t, int c) {
 
 // hi + lo split of two fp32 values into 16-bit pairs (fp16, or bf16 for bf16 caches).
 template <bool BF>
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+__device__ __forceinline__ void split2(float2 w, uint32_t& hi, uint32_t& lo) {
+  float2 h;
   if constexpr (BF) {
-    hi = pack_bf16x2(a, b);
-    const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
-    lo = pack_bf16x2(a - h.x, b - h.y);
+    hi = pack_bf16x2(w.x, w.y);
+    h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
   } else {
-    hi = pack_f16x2(a, b);
-    const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-    lo = pack_f16x2(a - h.x, b - h.y);
+    hi = pack_f16x2(w.x, w.y);
+    h = __half22float2(*reinterpret_cast<const __half2*>(&hi));
   }
+  const float2 r = __fadd2_rn(w, make_float2(-h.x, -h.y));
+  lo = BF ? pack_bf16x2(r.x, r.y) : pack_f16x2(r.x, r.y);
+}
+template <bool BF>
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  split2<BF>(make_float2(a, b), hi, lo);
+}
+
+// Largest of three values (one three-input max on sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
@@ -721,24 +733,41 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       // causal boundary (position <= this row's) and tokens of bad pages (multiplier NaN)
       const int lim = row_ok ? pos_r - j * kBlk - col0 : -1;
       // pass 1: the largest scaled score of this row's 64 columns, 32 at a time (read from
-      // TMEM again in pass 2; the loops are not unrolled, to keep the hot code small)
-      auto scaled = [&](uint32_t sv, float f, int t) {
-        const float v = __uint_as_float(sv) * f;
-        return (fast || (t <= lim && f == f)) ? v : -INFINITY;
-      };
-      float mx = -INFINITY;
+      // TMEM again in pass 2; the loops are not unrolled, to keep the hot code small).  Blocks
+      // wholly visible to every row of the tile take a path with no per-score tests.
+      float m0 = -INFINITY, m1 = -INFINITY;
+      if (fast) {
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sr[32];
-        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sr[32];
+          tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const int t = 32 * cc + i;
-          const float4 f = *reinterpret_cast<const float4*>(kq + t);
-          mx = fmaxf(mx, fmaxf(fmaxf(scaled(sr[i], f.x, t), scaled(sr[i + 1], f.y, t + 1)),
-                               fmaxf(scaled(sr[i + 2], f.z, t + 2), scaled(sr[i + 3], f.w, t + 3))));
+          for (int i = 0; i < 32; i += 4) {
+            const float4 f = *reinterpret_cast<const float4*>(kq + 32 * cc + i);
+            const float2 a = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
+                                        make_float2(f.x, f.y));
+            const float2 c = __fmul2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
+                                        make_float2(f.z, f.w));
+            m0 = max3(m0, a.x, a.y);
+            m1 = max3(m1, c.x, c.y);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sr[32];
+          tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const int t = 32 * cc + i;
+            const float2 f = *reinterpret_cast<const float2*>(kq + t);
+            const float2 a = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), f);
+            m0 = fmaxf(m0, (t <= lim && f.x == f.x) ? a.x : -INFINITY);
+            m1 = fmaxf(m1, (t + 1 <= lim && f.y == f.y) ? a.y : -INFINITY);
+          }
         }
       }
+      float mx = fmaxf(m0, m1);
       // the row's max over both halves: exchange with the partner warp of this quarter
       xm[(sb * 2 + hf) * kRows + r] = mx;
       __syncwarp();
@@ -786,29 +815,39 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       // 16-bit halves over the 32 score columns just read (each chunk: hi halves in its
       // first 16 columns, lo halves in the next 16)
       float2 lsum = make_float2(0.f, 0.f);
+      const float2 noff = make_float2(-off, -off);
+      auto pass2 = [&](auto masked) {
 #pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sr[32];
-        tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
-        uint32_t ph[16], pl[16];
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sr[32];
+          tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
+          uint32_t ph[16], pl[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = 32 * cc + 2 * i;
-          const float2 f = *reinterpret_cast<const float2*>(kq + t);
-          float2 xo = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), f,
-                                 make_float2(-off, -off));
-          if (!fast) {
-            if (!(t <= lim && f.x == f.x)) xo.x = -INFINITY;
-            if (!(t + 1 <= lim && f.y == f.y)) xo.y = -INFINITY;
+          for (int i = 0; i < 16; i += 2) {
+            const int t = 32 * cc + 2 * i;
+            const float4 f = *reinterpret_cast<const float4*>(kq + t);
+            const float4 vv = *reinterpret_cast<const float4*>(vsp + t);
+            float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                                   make_float2(f.x, f.y), noff);
+            float2 xb = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i + 2]), __uint_as_float(sr[2 * i + 3])),
+                                   make_float2(f.z, f.w), noff);
+            if constexpr (decltype(masked)::value) {
+              if (!(t <= lim && f.x == f.x)) xa.x = -INFINITY;
+              if (!(t + 1 <= lim && f.y == f.y)) xa.y = -INFINITY;
+              if (!(t + 2 <= lim && f.z == f.z)) xb.x = -INFINITY;
+              if (!(t + 3 <= lim && f.w == f.w)) xb.y = -INFINITY;
+            }
+            const float2 ea = make_float2(ex2(xa.x), ex2(xa.y)), eb = make_float2(ex2(xb.x), ex2(xb.y));
+            lsum = __fadd2_rn(lsum, __fadd2_rn(ea, eb));
+            split2<kBf>(__fmul2_rn(ea, make_float2(vv.x, vv.y)), ph[i], pl[i]);
+            split2<kBf>(__fmul2_rn(eb, make_float2(vv.z, vv.w)), ph[i + 1], pl[i + 1]);
           }
-          const float2 e = make_float2(ex2(xo.x), ex2(xo.y));
-          lsum = __fadd2_rn(lsum, e);
-          const float2 w = __fmul2_rn(e, *reinterpret_cast<const float2*>(vsp + t));
-          split2<kBf>(w.x, w.y, ph[i], pl[i]);
+          st16(lanebase + 128 * sb + col0 + 32 * cc, ph);
+          st16(lanebase + 128 * sb + col0 + 32 * cc + 16, pl);
         }
-        st16(lanebase + 128 * sb + col0 + 32 * cc, ph);
-        st16(lanebase + 128 * sb + col0 + 32 * cc + 16, pl);
-      }
+      };
+      if (fast) pass2(std::false_type{});
+      else pass2(std::true_type{});
       l += lsum.x + lsum.y;
       tc::st_wait();
       tc::fence_before_sync();
