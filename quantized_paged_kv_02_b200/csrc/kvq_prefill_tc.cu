@@ -83,10 +83,10 @@ struct PfLayout {
   static constexpr int VP = LB ? 2 : 1;
   static constexpr int NB = LB ? 1 : kNB;                  // K / V tile buffers
   static constexpr int RS = LB ? 4 : (BITS == 8 ? 16 : 8); // raw ring stages (pages)
-  // pages the producer issues side by side: at most one per stage, so that no lane of a
-  // group waits on a stage another lane of the same group is filling (a wait two phases
-  // ahead of an mbarrier would see the parity of an older phase as complete)
-  static constexpr int IL = RS < 8 ? RS : 8;
+  // the ring turns over in groups of one block's pages, each group with one full and one
+  // empty barrier: the producer issues a block's pages together and the converters wait
+  // once per block
+  static constexpr int RG = RS / PPB;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = NB * KP * kTile;
   static constexpr int RAW_OFF = V_OFF + NB * VP * kTile;
@@ -98,14 +98,14 @@ struct PfLayout {
   static constexpr int MISC_OFF = XM_OFF + 3 * 2 * kRows * 4;  // per (buffer, converter warp)
                                                                // vmax and bad-token counts; flags
   static constexpr int BAR_OFF = MISC_OFF + 128;
-  // raw_full, raw_empty [RS]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
+  // raw_full, raw_empty [RG]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
   // q_ready; fin; xch [4]
-  static constexpr int NBARS = 2 * RS + 3 * NB + 6 + 2 + 4;
+  static constexpr int NBARS = 2 * RG + 3 * NB + 6 + 2 + 4;
   static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + RS * 4 + 64;
   static_assert(BYTES <= 227 * 1024, "fits the shared memory of one CTA");
   static_assert(BYTES > 114 * 1024, "one CTA per SM, so TMEM allocation never waits on a peer");
-  static_assert(RS >= PPB, "a block's pages fit the raw ring");
-  static_assert(IL <= RS, "one issue group never waits on its own stages");
+  static_assert(RS % PPB == 0 && RG >= 1, "the raw ring holds whole blocks");
+  static_assert(PPB <= 32, "one producer lane per page of a block");
   static_assert(REC % 16 == 0, "bulk copies move multiples of 16 bytes");
   static_assert(NB <= kNB, "scale arrays");
 };
@@ -226,17 +226,15 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
 // Dense caches, converter thread (c, rr) = (ct % 16, ct / 16): the K (or V) rows of every
 // page of block j -> tile buffer kb, chunk c of rows rr and rr + 8 of each page; all loads
 // first, then conversions and stores.  Thread ct also writes token ct's multiplier (K:
-// softmax scale x K scale, NaN for a bad page; V: the V scale) and counts its bad token;
-// after V the warp releases the pages' raw stages.  Returns token ct's V scale (0 for K).
-// Not inlined: one copy of the code serves both halves, which keeps the kernel's hot code
-// inside the instruction cache.
+// softmax scale x K scale, NaN for a bad page; V: the V scale).  Returns 1 for a bad token
+// of K (a visible position on a page that failed its table check), token ct's V scale for V.
 template <int CD, bool PT>
-__device__ __noinline__ float dense_part(uint8_t* smem, const PfShared& sh, int j, int kb, bool isv,
-                                         int ct, int npg, int pmax, float qsc, int* bad) {
+__device__ __forceinline__ float dense_part(uint8_t* smem, const PfShared& sh, int j, int kb, bool isv,
+                                            int ct, int npg, int pmax, float qsc) {
   using L = PfLayout<CD, PT>;
   constexpr int PPB = L::PPB, BS = L::BS;
   using RawT = typename std::conditional<L::BITS == 8, uint2, uint4>::type;
-  const int c = ct & 15, rr = ct >> 4, lane = ct & 31;
+  const int c = ct & 15, rr = ct >> 4;
   RawT w[PPB][2];
   uint32_t pok = 0;
 #pragma unroll
@@ -268,28 +266,19 @@ __device__ __noinline__ float dense_part(uint8_t* smem, const PfShared& sh, int 
   const bool have = k < npg, pk = (pok >> pp) & 1u;
   const bool valid = pk && pos <= pmax;
   const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
-  float vm = 0.f;
   if (!isv) {
     float ks = 1.f;
     if constexpr (PT) ks = sc[row];
     // positions past the tile's last query are never visible: their multiplier is unused
     const bool badtok = have && !pk && pos <= pmax;
     sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
-    *bad += badtok;
-  } else {
-    float vv = 1.f;
-    if constexpr (PT) vv = sc[BS + row];
-    vv = valid ? vv : 0.f;
-    sh.vs[kb * kBlk + t] = vv;
-    vm = vv;
-    __syncwarp();
-#pragma unroll
-    for (int q = 0; q < PPB; ++q) {
-      const int kk = j * PPB + q;
-      if (kk < npg && lane == 0) mbar_arrive(&sh.raw_empty[kk % L::RS]);   // K and V read
-    }
+    return badtok ? 1.f : 0.f;
   }
-  return vm;
+  float vv = 1.f;
+  if constexpr (PT) vv = sc[BS + row];
+  vv = valid ? vv : 0.f;
+  sh.vs[kb * kBlk + t] = vv;
+  return vv;
 }
 
 template <int CD, bool PT, int QP>
@@ -324,8 +313,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   PfShared sh;
   sh.raw_full = bars;
-  sh.raw_empty = bars + L::RS;
-  sh.k_full = bars + 2 * L::RS;
+  sh.raw_empty = bars + L::RG;
+  sh.k_full = bars + 2 * L::RG;
   sh.v_full = sh.k_full + NB;
   sh.vfree = sh.v_full + NB;
   sh.s_full = sh.vfree + NB;
@@ -346,7 +335,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 80);   // [8] softmax amax
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L::RS; ++s) {
+    for (int s = 0; s < L::RG; ++s) {
       mbar_init(&sh.raw_full[s], 1);
       mbar_init(&sh.raw_empty[s], 4);                    // the four converter warps
     }
@@ -374,42 +363,50 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
 
   if (warp == kProdWarp) {
     // ------------------------------------------------------------ producer
+    // block j's pages (lane pp: page j PPB + pp) land in ring group j % RG; lane 0 announces
+    // the group's bytes on its full barrier before any copy is issued
     const uint8_t* pages = p.pages;
-    int issued = 0;
+    const int nblk = (npg + L::PPB - 1) / L::PPB;          // blocks with pages to copy
     bool ok_run = true;
-    for (int k0 = 0; k0 < npg && ok_run; k0 += L::IL) {
-      const int cnt = min(L::IL, npg - k0);
+    int jb = 0;
+    for (; jb < nblk && ok_run; ++jb) {
+      const int grp = jb % L::RG, round = jb / L::RG;
       bool ok_lane = true;
-      if (lane < cnt) {
-        const int k = k0 + lane, s = k % L::RS, round = k / L::RS;
-        const int blk = p.tables[static_cast<long>(b) * p.max_blocks + k];
-        const bool valid = blk >= 0 && blk < p.NB;
-        if (round > 0 && !pf_wait(&sh.raw_empty[s], (round - 1) & 1, sh.abort)) {
-          ok_lane = false;
-        } else {
-          sh.page_ok[s] = valid;
-          if (valid) {
-            mbar_arrive_expect_tx(&sh.raw_full[s], L::REC);
-            bulk_load(smem + L::RAW_OFF + s * L::REC,
-                      pages + (static_cast<long>(blk) * p.H + kvh) * L::REC, L::REC, &sh.raw_full[s]);
-          } else {
-            record_fault(p.fault, KVQ_FAULT_BLOCK);
-            mbar_arrive(&sh.raw_full[s]);
-          }
-        }
-      }
+      if (lane == 0 && round > 0 && !pf_wait(&sh.raw_empty[grp], (round - 1) & 1, sh.abort)) ok_lane = false;
       ok_run = __all_sync(0xffffffffu, ok_lane);
-      if (!ok_run && lane == 0) pf_fail(p, sh.abort);
-      issued = k0 + cnt;
+      if (!ok_run) {
+        if (lane == 0) pf_fail(p, sh.abort);
+        break;
+      }
+      const int k = jb * L::PPB + lane, s = k % L::RS;
+      bool valid = false;
+      int blk = -1;
+      if (lane < L::PPB && k < npg) {
+        blk = p.tables[static_cast<long>(b) * p.max_blocks + k];
+        valid = blk >= 0 && blk < p.NB;
+        sh.page_ok[s] = valid;
+        if (!valid) record_fault(p.fault, KVQ_FAULT_BLOCK);
+      }
+      const unsigned nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+      if (lane == 0) mbar_arrive_expect_tx(&sh.raw_full[grp], nvalid * L::REC);
+      __syncwarp();
+      if (valid) {
+        bulk_load(smem + L::RAW_OFF + s * L::REC, pages + (static_cast<long>(blk) * p.H + kvh) * L::REC, L::REC,
+                  &sh.raw_full[grp]);
+      }
     }
     // every copy issued must land before the CTA may exit
     if (lane == 0) {
-      for (int k = max(0, issued - L::RS); k < issued; ++k)
-        if (!mbar_drain(&sh.raw_full[k % L::RS], (k / L::RS) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+      for (int j2 = max(0, jb - L::RG); j2 < jb; ++j2)
+        if (!mbar_drain(&sh.raw_full[j2 % L::RG], (j2 / L::RG) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
     }
   } else if (warp >= kConvWarp0) {
     // ------------------------------------------------------------ converters
-    // thread (c, rr): 16-byte output chunk c (elements 8c..8c+7 of a row) of rows rr + 8i
+    // thread (c, rr): 16-byte output chunk c (elements 8c..8c+7 of a row) of rows rr + 8i.
+    // Per block two parts, K then V, through one copy of the code: part 0 waits for the
+    // block's pages and for the softmax of block j - NB (done with this buffer's K
+    // multipliers, and S of j - NB with its K), part 1 for P V of block j - NB (done with
+    // its V); after part 1 the block's ring group is released.
     const int ct = threadIdx.x - kConvWarp0 * 32;        // 0..127
     const int c = ct & 15, rr = ct >> 4;
     const int cw = warp - kConvWarp0;
@@ -417,156 +414,151 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     const float qsc = *sh.qscale;
     const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
     const int G = c >> 3;                                 // 64-channel group of the chunk
-    for (int j = 0; j < J && !*sh.abort; ++j) {
+    bool fail = false;
+    for (int j = 0; j < J && !fail && !*sh.abort; ++j) {
       const int kb = j % NB;
-      // the softmax of block j - NB is done with this buffer's scales (and S j - NB with K)
-      if (j >= NB && !pf_wait(&sh.p_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) {
-        if (lane == 0) pf_fail(p, sh.abort);
-        break;
-      }
-      int bad = 0;
-      bool ok = true;
-      if constexpr (!L::LB) {
-        // K of the whole block, rows rr and rr + 8 of every page, chunk c: wait for the pages
-        // (requested a block ago, usually landed), then issue every load before converting,
-        // so a converter thread has 16 independent loads in flight instead of one chain
-#pragma unroll
-        for (int pp = 0; pp < L::PPB; ++pp) {
-          const int k = j * L::PPB + pp;
-          if (k < npg && !pf_wait(&sh.raw_full[k % L::RS], (k / L::RS) & 1, sh.abort)) ok = false;
-        }
-        if (__all_sync(0xffffffffu, ok)) dense_part<CD, PT>(smem, sh, j, kb, false, ct, npg, pmax, qsc, &bad);
-      }
-      // K: rows rr + 8i of every page of the block, chunk c (low-bit caches)
-      for (int pp = 0; pp < L::PPB && ok && L::LB; ++pp) {
-        const int k = j * L::PPB + pp;
-        const bool have = k < npg;
-        const int s = k % L::RS;
-        if (have && !pf_wait(&sh.raw_full[s], (k / L::RS) & 1, sh.abort)) {
+      const bool paged = j * L::PPB < npg;               // the block has pages in the ring
+#pragma unroll 1
+      for (int part = 0; part < 2; ++part) {
+        bool ok = true;
+        if (part == 0) {
+          if (j >= NB && !pf_wait(&sh.p_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) ok = false;
+          if (ok && paged && !pf_wait(&sh.raw_full[j % L::RG], (j / L::RG) & 1, sh.abort)) ok = false;
+        } else if (j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
           ok = false;
+        }
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) pf_fail(p, sh.abort);
+          fail = true;
           break;
         }
-        const bool pok = have && sh.page_ok[s];
-        const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
-        {
-          // per-channel K parameters of this chunk (KIVI forms): s[8c..8c+7], z or minimum
-          float ksc[8], kzp[8];
-          if (!ktok && pok) {
-            const uint4 su = *reinterpret_cast<const uint4*>(raw + L::OFF_S + 16 * c);
-            const uint4 zu = *reinterpret_cast<const uint4*>(raw + L::OFF_S + 2 * kD + 16 * c);
-            const __half* sh8 = reinterpret_cast<const __half*>(&su);
-            const __half* zh8 = reinterpret_cast<const __half*>(&zu);
+        // K: bad-token count; V: largest V scale
+        float val = 0.f;
+        if constexpr (!L::LB) {
+          val = dense_part<CD, PT>(smem, sh, j, kb, part == 1, ct, npg, pmax, qsc);
+        } else if (part == 0) {
+          int bad = 0;
+          // K: rows rr + 8i of every page of the block, chunk c (low-bit caches)
+          for (int pp = 0; pp < L::PPB; ++pp) {
+            const int k = j * L::PPB + pp;
+            const bool have = k < npg;
+            const int s = k % L::RS;
+            const bool pok = have && sh.page_ok[s];
+            const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
+            {
+              // per-channel K parameters of this chunk (KIVI forms): s[8c..8c+7], z or minimum
+              float ksc[8], kzp[8];
+              if (!ktok && pok) {
+                const uint4 su = *reinterpret_cast<const uint4*>(raw + L::OFF_S + 16 * c);
+                const uint4 zu = *reinterpret_cast<const uint4*>(raw + L::OFF_S + 2 * kD + 16 * c);
+                const __half* sh8 = reinterpret_cast<const __half*>(&su);
+                const __half* zh8 = reinterpret_cast<const __half*>(&zu);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              ksc[e] = __half2float(sh8[e]);
-              kzp[e] = __half2float(zh8[e]);
-            }
-          }
-          for (int i = 0; i < BS / 8; ++i) {
-            const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
-            const bool ring = pos >= si.qb;
-            const bool valid = pos <= pmax && (ring || pok);
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-            if (valid && ring) {
-              const long rrow = ((static_cast<long>(si.sid) * 2) * p.H + kvh) * p.cap + pos % p.cap;
-              const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + rrow * kD + 8 * c);
-              if (p.act_fp16) unpack8<__half>(u, v);
-              else unpack8<__nv_bfloat16>(u, v);
-            } else if (valid) {
-              uint32_t w;
-              if constexpr (L::BITS == 4) w = *reinterpret_cast<const uint32_t*>(raw + row * L::ROWB + 4 * c);
-              else w = *reinterpret_cast<const uint16_t*>(raw + row * L::ROWB + 2 * c);
-              float s1 = 0.f, z1 = 0.f;
-              if (ktok) {
-                const __half2 sz = *reinterpret_cast<const __half2*>(raw + L::OFF_S + (row * 2 + G) * 4);
-                s1 = __low2float(sz);
-                z1 = __high2float(sz);
+                for (int e = 0; e < 8; ++e) {
+                  ksc[e] = __half2float(sh8[e]);
+                  kzp[e] = __half2float(zh8[e]);
+                }
               }
+              for (int i = 0; i < BS / 8; ++i) {
+                const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
+                const bool ring = pos >= si.qb;
+                const bool valid = pos <= pmax && (ring || pok);
+                float v[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int code = (w >> (L::BITS * e)) & ((1 << L::BITS) - 1);
-                v[e] = ktok ? lb_value(code, s1, z1, false) : lb_value(code, ksc[e], kzp[e], fz);
+                for (int e = 0; e < 8; ++e) v[e] = 0.f;
+                if (valid && ring) {
+                  const long rrow = ((static_cast<long>(si.sid) * 2) * p.H + kvh) * p.cap + pos % p.cap;
+                  const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + rrow * kD + 8 * c);
+                  if (p.act_fp16) unpack8<__half>(u, v);
+                  else unpack8<__nv_bfloat16>(u, v);
+                } else if (valid) {
+                  uint32_t w;
+                  if constexpr (L::BITS == 4) w = *reinterpret_cast<const uint32_t*>(raw + row * L::ROWB + 4 * c);
+                  else w = *reinterpret_cast<const uint16_t*>(raw + row * L::ROWB + 2 * c);
+                  float s1 = 0.f, z1 = 0.f;
+                  if (ktok) {
+                    const __half2 sz = *reinterpret_cast<const __half2*>(raw + L::OFF_S + (row * 2 + G) * 4);
+                    s1 = __low2float(sz);
+                    z1 = __high2float(sz);
+                  }
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const int code = (w >> (L::BITS * e)) & ((1 << L::BITS) - 1);
+                    v[e] = ktok ? lb_value(code, s1, z1, false) : lb_value(code, ksc[e], kzp[e], fz);
+                  }
+                }
+                uint4 hi, lo;
+                split8(v, hi, lo);
+                *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2) * kTile + tile_off(t, c)) = hi;
+                *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
+                if (c == 0) {
+                  const bool badtok = !ring && have && !pok && pos <= pmax;
+                  sh.kq[kb * kBlk + t] = valid ? qsc : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+                  bad += badtok;
+                }
               }
             }
-            uint4 hi, lo;
-            split8(v, hi, lo);
-            *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2) * kTile + tile_off(t, c)) = hi;
-            *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
-            if (c == 0) {
-              const bool badtok = !ring && have && !pok && pos <= pmax;
-              sh.kq[kb * kBlk + t] = valid ? qsc : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
-              bad += badtok;
+          }
+          val = static_cast<float>(bad);
+        } else {
+          float vm = 0.f;
+          for (int pp = 0; pp < L::PPB; ++pp) {
+            const int k = j * L::PPB + pp;
+            const bool have = k < npg;
+            const int s = k % L::RS;
+            const bool pok = have && sh.page_ok[s];
+            const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
+            {
+              for (int i = 0; i < BS / 8; ++i) {
+                const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
+                const bool ring = pos >= si.qb;
+                const bool valid = pos <= pmax && (ring || pok);
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = 0.f;
+                if (valid && ring) {
+                  const long vrow = ((static_cast<long>(si.sid) * 2 + 1) * p.H + kvh) * p.cap + pos % p.cap;
+                  const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + vrow * kD + 8 * c);
+                  if (p.act_fp16) unpack8<__half>(u, v);
+                  else unpack8<__nv_bfloat16>(u, v);
+                } else if (valid) {
+                  uint32_t w;
+                  if constexpr (L::BITS == 4) w = *reinterpret_cast<const uint32_t*>(raw + L::OFF_V + row * L::ROWB + 4 * c);
+                  else w = *reinterpret_cast<const uint16_t*>(raw + L::OFF_V + row * L::ROWB + 2 * c);
+                  const __half2 sz = *reinterpret_cast<const __half2*>(raw + L::OFF_S + 4 * kD + (row * 2 + G) * 4);
+                  const float s1 = __low2float(sz), z1 = __high2float(sz);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) v[e] = lb_value((w >> (L::BITS * e)) & ((1 << L::BITS) - 1), s1, z1, fz);
+                }
+                uint4 hi, lo;
+                split8(v, hi, lo);
+                *reinterpret_cast<uint4*>(smem + L::V_OFF + (kb * 2) * kTile + tile_off(t, c)) = hi;
+                *reinterpret_cast<uint4*>(smem + L::V_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
+                if (c == 0) {
+                  const float vv = valid ? 1.f : 0.f;
+                  sh.vs[kb * kBlk + t] = vv;
+                  vm = fmaxf(vm, vv);
+                }
+              }
             }
           }
+          val = vm;
         }
-      }
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) pf_fail(p, sh.abort);
-        break;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, off);
-      if (lane == 0) sh.nbad[kb * 4 + cw] = bad;
-      tc::fence_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.k_full[kb]);
-      // V: wait until P V of block j - NB has read this buffer
-      if (j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
-        if (lane == 0) pf_fail(p, sh.abort);
-        break;
-      }
-      float vm = 0.f;
-      if constexpr (!L::LB) vm = dense_part<CD, PT>(smem, sh, j, kb, true, ct, npg, pmax, qsc, &bad);
-      for (int pp = 0; pp < L::PPB && L::LB; ++pp) {
-        const int k = j * L::PPB + pp;
-        const bool have = k < npg;
-        const int s = k % L::RS;
-        const bool pok = have && sh.page_ok[s];
-        const uint8_t* raw = smem + L::RAW_OFF + s * L::REC;
-        {
-          for (int i = 0; i < BS / 8; ++i) {
-            const int row = rr + 8 * i, t = pp * BS + row, pos = j * kBlk + t;
-            const bool ring = pos >= si.qb;
-            const bool valid = pos <= pmax && (ring || pok);
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-            if (valid && ring) {
-              const long vrow = ((static_cast<long>(si.sid) * 2 + 1) * p.H + kvh) * p.cap + pos % p.cap;
-              const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.residual) + vrow * kD + 8 * c);
-              if (p.act_fp16) unpack8<__half>(u, v);
-              else unpack8<__nv_bfloat16>(u, v);
-            } else if (valid) {
-              uint32_t w;
-              if constexpr (L::BITS == 4) w = *reinterpret_cast<const uint32_t*>(raw + L::OFF_V + row * L::ROWB + 4 * c);
-              else w = *reinterpret_cast<const uint16_t*>(raw + L::OFF_V + row * L::ROWB + 2 * c);
-              const __half2 sz = *reinterpret_cast<const __half2*>(raw + L::OFF_S + 4 * kD + (row * 2 + G) * 4);
-              const float s1 = __low2float(sz), z1 = __high2float(sz);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = lb_value((w >> (L::BITS * e)) & ((1 << L::BITS) - 1), s1, z1, fz);
-            }
-            uint4 hi, lo;
-            split8(v, hi, lo);
-            *reinterpret_cast<uint4*>(smem + L::V_OFF + (kb * 2) * kTile + tile_off(t, c)) = hi;
-            *reinterpret_cast<uint4*>(smem + L::V_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
-            if (c == 0) {
-              const float vv = valid ? 1.f : 0.f;
-              sh.vs[kb * kBlk + t] = vv;
-              vm = fmaxf(vm, vv);
-            }
-          }
+        if (part == 0) {
+          const unsigned nbad = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(val));
+          if (lane == 0) sh.nbad[kb * 4 + cw] = static_cast<int>(nbad);
+        } else {
+          // V scales are >= 0: their bit patterns order as the values do
+          const unsigned vmb = __reduce_max_sync(0xffffffffu, __float_as_uint(val));
+          if (lane == 0) sh.vmax[kb * 4 + cw] = __uint_as_float(vmb);
         }
+        tc::fence_async_shared();
         __syncwarp();
-        if (have && lane == 0) mbar_arrive(&sh.raw_empty[s]);   // K and V of the page are read
+        if (lane == 0) {
+          mbar_arrive(part == 0 ? &sh.k_full[kb] : &sh.v_full[kb]);
+          if (part == 1 && paged) mbar_arrive(&sh.raw_empty[j % L::RG]);   // K and V read
+        }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-      if (lane == 0) sh.vmax[kb * 4 + cw] = vm;
-      tc::fence_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.v_full[kb]);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
