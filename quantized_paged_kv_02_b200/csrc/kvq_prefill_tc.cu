@@ -48,7 +48,8 @@ namespace {
 constexpr int kRows = 128;          // query rows per tile (MMA M)
 constexpr int kBlk = 128;           // cached tokens per block (MMA N of S, K of P V)
 constexpr int kD = 128;
-constexpr int kPfThreads = 448;     // warps 0-7 softmax, 8 producer, 9 MMA, 10-13 converters
+constexpr int kPfThreads = 576;     // warps 0-7 softmax, 8 producer, 9 MMA, 10-13 K converters,
+                                    // 14-17 V converters
 constexpr int kSoftWarps = 8, kProdWarp = 8, kMmaWarp = 9, kConvWarp0 = 10;
 constexpr int kNB = 2;              // K / V tile buffers
 constexpr int kTile = 32768;        // 128 x 128 16-bit elements
@@ -209,6 +210,13 @@ __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+__device__ __forceinline__ void st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7])
+               : "memory");
+}
+
 // Dequantized value of one low-bit code: (code - zero) * scale, or code * scale + minimum
 // (float zero point); exact in float32 for the integer zero point (<= 15 significant bits).
 __device__ __forceinline__ float lb_value(int code, float s, float z, bool fz) {
@@ -337,7 +345,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::RG; ++s) {
       mbar_init(&sh.raw_full[s], 1);
-      mbar_init(&sh.raw_empty[s], 4);                    // the four converter warps
+      mbar_init(&sh.raw_empty[s], 8);                    // the eight converter warps
     }
     for (int k = 0; k < NB; ++k) {
       mbar_init(&sh.k_full[k], 4);
@@ -402,34 +410,32 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     }
   } else if (warp >= kConvWarp0) {
     // ------------------------------------------------------------ converters
-    // thread (c, rr): 16-byte output chunk c (elements 8c..8c+7 of a row) of rows rr + 8i.
-    // Per block two parts, K then V, through one copy of the code: part 0 waits for the
-    // block's pages and for the softmax of block j - NB (done with this buffer's K
-    // multipliers, and S of j - NB with its K), part 1 for P V of block j - NB (done with
-    // its V); after part 1 the block's ring group is released.
-    const int ct = threadIdx.x - kConvWarp0 * 32;        // 0..127
+    // warps 10-13 convert K, warps 14-17 V; thread (c, rr): 16-byte output chunk c (elements
+    // 8c..8c+7 of a row) of rows rr + 8i.  K of block j waits for the block's pages and for
+    // the softmax of block j - NB (done with this buffer's K multipliers, and S of j - NB with
+    // its K); V of block j for the pages and for P V of block j - NB (done with its V).  The
+    // block's ring group is released once all eight warps have read it.
+    const int part = warp >= kConvWarp0 + 4 ? 1 : 0;
+    const int cw = (warp - kConvWarp0) & 3;
+    const int ct = cw * 32 + lane;                        // 0..127
     const int c = ct & 15, rr = ct >> 4;
-    const int cw = warp - kConvWarp0;
     if (!pf_wait(sh.q_ready, 0, sh.abort)) pf_fail(p, sh.abort);
     const float qsc = *sh.qscale;
     const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
     const int G = c >> 3;                                 // 64-channel group of the chunk
-    bool fail = false;
-    for (int j = 0; j < J && !fail && !*sh.abort; ++j) {
+    for (int j = 0; j < J && !*sh.abort; ++j) {
       const int kb = j % NB;
       const bool paged = j * L::PPB < npg;               // the block has pages in the ring
-#pragma unroll 1
-      for (int part = 0; part < 2; ++part) {
+      {
         bool ok = true;
         if (part == 0) {
           if (j >= NB && !pf_wait(&sh.p_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) ok = false;
-          if (ok && paged && !pf_wait(&sh.raw_full[j % L::RG], (j / L::RG) & 1, sh.abort)) ok = false;
         } else if (j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
           ok = false;
         }
+        if (ok && paged && !pf_wait(&sh.raw_full[j % L::RG], (j / L::RG) & 1, sh.abort)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) pf_fail(p, sh.abort);
-          fail = true;
           break;
         }
         // K: bad-token count; V: largest V scale
@@ -556,7 +562,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(part == 0 ? &sh.k_full[kb] : &sh.v_full[kb]);
-          if (part == 1 && paged) mbar_arrive(&sh.raw_empty[j % L::RG]);   // K and V read
+          if (paged) mbar_arrive(&sh.raw_empty[j % L::RG]);
         }
       }
     }
@@ -585,7 +591,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               // tokens 16 kk .. 16 kk + 15: chunk kk / 2 of P, its hi (pa 0) or lo (pa 1) half
-              tc::mma_ts(tbase + kTmO, tbase + 128 * sb + 32 * (kk >> 1) + 16 * pa + 8 * (kk & 1),
+              tc::mma_ts(tbase + kTmO, tbase + 128 * sb + 16 * kk + 8 * pa,
                          tc::desc_mnmajor(vt, kk), idPV, first ? 0u : 1u);
               first = false;
             }
@@ -677,26 +683,30 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         down = ldexpf(1.f, -eq);
         qscale = ldexpf(qscale, eq);
       }
-      uint32_t hi[32], lo[32];
+      // 32 columns (16 TMEM columns of 16-bit pairs) at a time
+#pragma unroll 1
+      for (int hq = 0; hq < 2; ++hq) {
+        uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 u = row_ok ? qp[i] : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 4; ++i) {
+          const uint4 u = row_ok ? qp[4 * hq + i] : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int d = 8 * i + e;
-          float a = elem(u, e), c2 = elem(u, e + 1);
-          if (kch != nullptr) {
-            a *= kch[d];
-            c2 *= kch[d + 1];
+          for (int e = 0; e < 8; e += 2) {
+            const int d = 32 * hq + 8 * i + e;
+            float a = elem(u, e), c2 = elem(u, e + 1);
+            if (kch != nullptr) {
+              a *= kch[d];
+              c2 *= kch[d + 1];
+            }
+            a *= down;
+            c2 *= down;
+            if constexpr (QP == 2) split2<kBf>(a, c2, hi[4 * i + e / 2], lo[4 * i + e / 2]);
+            else hi[4 * i + e / 2] = kBf ? pack_bf16x2(a, c2) : pack_f16x2(a, c2);
           }
-          a *= down;
-          c2 *= down;
-          if constexpr (QP == 2) split2<kBf>(a, c2, hi[4 * i + e / 2], lo[4 * i + e / 2]);
-          else hi[4 * i + e / 2] = kBf ? pack_bf16x2(a, c2) : pack_f16x2(a, c2);
         }
+        st16(lanebase + kTmQ + 32 * hf + 16 * hq, hi);
+        if constexpr (QP == 2) st16(lanebase + kTmQ + 64 + 32 * hf + 16 * hq, lo);
       }
-      tc::st32(lanebase + kTmQ + 32 * hf, hi);
-      if constexpr (QP == 2) tc::st32(lanebase + kTmQ + 64 + 32 * hf, lo);
       if (threadIdx.x == 0) *sh.qscale = qscale;
       tc::st_wait();
       tc::fence_before_sync();
@@ -804,19 +814,19 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       const float off = (m == -INFINITY ? 0.f : m) + (ev == INT_MIN ? 0.f : static_cast<float>(ev));
       const float* vsp = sh.vs + kb * kBlk + col0;
       // pass 2: e = 2^(x - off), the row sum, and e times the token's V scale as hi + lo
-      // 16-bit halves over the 32 score columns just read (each chunk: hi halves in its
-      // first 16 columns, lo halves in the next 16)
+      // 16-bit halves, 16 score columns at a time: P of those 16 keys overwrites their scores
+      // (hi halves in the first 8 TMEM columns, lo halves in the next 8)
       float2 lsum = make_float2(0.f, 0.f);
       const float2 noff = make_float2(-off, -off);
       auto pass2 = [&](auto masked) {
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t sr[32];
-          tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
-          uint32_t ph[16], pl[16];
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sr[16];
+          tc::ld16(lanebase + 128 * sb + col0 + 16 * cc, sr);
+          uint32_t ph[8], pl[8];
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const int t = 32 * cc + 2 * i;
+          for (int i = 0; i < 8; i += 2) {
+            const int t = 16 * cc + 2 * i;
             const float4 f = *reinterpret_cast<const float4*>(kq + t);
             const float4 vv = *reinterpret_cast<const float4*>(vsp + t);
             float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
@@ -834,8 +844,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
             split2<kBf>(__fmul2_rn(ea, make_float2(vv.x, vv.y)), ph[i], pl[i]);
             split2<kBf>(__fmul2_rn(eb, make_float2(vv.z, vv.w)), ph[i + 1], pl[i + 1]);
           }
-          st16(lanebase + 128 * sb + col0 + 32 * cc, ph);
-          st16(lanebase + 128 * sb + col0 + 32 * cc + 16, pl);
+          st8(lanebase + 128 * sb + col0 + 16 * cc, ph);
+          st8(lanebase + 128 * sb + col0 + 16 * cc + 8, pl);
         }
       };
       if (fast) pass2(std::false_type{});
@@ -866,24 +876,24 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         const float* vch = (p.mode == KVQ_SCALE_PER_CHANNEL) ? p.v_static + kvh * kD + col0 : nullptr;
         const long orow = (static_cast<long>(p.q_start[b]) + qi) * p.Hq + static_cast<long>(kvh) * g + h;
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t o[32];
-          tc::ld32(lanebase + kTmO + col0 + 32 * cc, o);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[16];
+          tc::ld16(lanebase + kTmO + col0 + 16 * cc, o);
           if (row_ok) {
-            float v[32];
+            float v[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              v[i] = __uint_as_float(o[i]) * inv * (vch != nullptr ? vch[32 * cc + i] : 1.f);
-            const long e0 = orow * kD + col0 + 32 * cc;          // a multiple of 32 elements
+            for (int i = 0; i < 16; ++i)
+              v[i] = __uint_as_float(o[i]) * inv * (vch != nullptr ? vch[16 * cc + i] : 1.f);
+            const long e0 = orow * kD + col0 + 16 * cc;          // a multiple of 16 elements
             if (p.out_dtype == KVQ_DTYPE_FP32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + e0);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             } else {
               const bool bf = p.out_dtype == KVQ_DTYPE_BF16;
               uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + e0);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
+              for (int i = 0; i < 2; ++i) {
                 uint32_t q4[4];
 #pragma unroll
                 for (int k2 = 0; k2 < 4; ++k2) {
