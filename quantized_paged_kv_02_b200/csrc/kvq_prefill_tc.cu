@@ -52,6 +52,7 @@ constexpr int kPfThreads = 576;     // warps 0-7 softmax, 8 producer, 9 MMA, 10-
                                     // 14-17 V converters
 constexpr int kSoftWarps = 8, kProdWarp = 8, kMmaWarp = 9, kConvWarp0 = 10;
 constexpr int kNB = 2;              // K / V tile buffers
+constexpr int kNQ = 4;              // slots of the per-token K multipliers (block j: slot j % 4)
 constexpr int kTile = 32768;        // 128 x 128 16-bit elements
 constexpr float kRescalePf = 8.f;   // log2 headroom before the running max is re-based
 // TMEM columns: scores / P of block j in [128 (j % 2), +128), O in [256, 384), Q from 384
@@ -91,17 +92,17 @@ struct PfLayout {
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = NB * KP * kTile;
   static constexpr int RAW_OFF = V_OFF + NB * VP * kTile;
-  static constexpr int KQ_OFF = RAW_OFF + RS * REC;        // float [NB][128]: K multiplier
-  static constexpr int VS_OFF = KQ_OFF + NB * kBlk * 4;    // float [NB][128]: V scale
+  static constexpr int KQ_OFF = RAW_OFF + RS * REC;        // float [kNQ][128]: K multiplier
+  static constexpr int VS_OFF = KQ_OFF + kNQ * kBlk * 4;   // float [NB][128]: V scale
   static constexpr int XM_OFF = VS_OFF + NB * kBlk * 4;    // float [3][2][128]: row maxima of
                                                            // the two halves (by block parity),
                                                            // then the row sums
   static constexpr int MISC_OFF = XM_OFF + 3 * 2 * kRows * 4;  // per (buffer, converter warp)
                                                                // vmax and bad-token counts; flags
-  static constexpr int BAR_OFF = MISC_OFF + 128;
+  static constexpr int BAR_OFF = MISC_OFF + 160;
   // raw_full, raw_empty [RG]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
-  // q_ready; fin; xch [4]
-  static constexpr int NBARS = 2 * RG + 3 * NB + 6 + 2 + 4;
+  // q_ready; fin; xch [4]; kq_full, kqfree [kNQ]
+  static constexpr int NBARS = 2 * RG + 3 * NB + 6 + 2 + 4 + 2 * kNQ;
   static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + RS * 4 + 64;
   static_assert(BYTES <= 227 * 1024, "fits the shared memory of one CTA");
   static_assert(BYTES > 114 * 1024, "one CTA per SM, so TMEM allocation never waits on a peer");
@@ -123,6 +124,8 @@ struct PfShared {
   uint64_t* q_ready;
   uint64_t* fin;                    // the MMA issuer's final commit
   uint64_t* xch;                    // [4]: the two softmax warps of a TMEM lane quarter
+  uint64_t* kq_full;                // [kNQ]: a slot of K multipliers (and bad-token counts) written
+  uint64_t* kqfree;                 // [kNQ]: the softmax is done with a slot of K multipliers
   float* xmax;
   int* page_ok;
   float* kq;                        // [NB][128] K multiplier of each token (NaN: bad page)
@@ -279,7 +282,7 @@ __device__ __forceinline__ float dense_part(uint8_t* smem, const PfShared& sh, i
     if constexpr (PT) ks = sc[row];
     // positions past the tile's last query are never visible: their multiplier is unused
     const bool badtok = have && !pk && pos <= pmax;
-    sh.kq[kb * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+    sh.kq[(j % kNQ) * kBlk + t] = valid ? qsc * ks : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
     return badtok ? 1.f : 0.f;
   }
   float vv = 1.f;
@@ -331,16 +334,18 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   sh.q_ready = sh.pv_done + 2;
   sh.fin = sh.q_ready + 1;
   sh.xch = sh.fin + 1;
+  sh.kq_full = sh.xch + 4;
+  sh.kqfree = sh.kq_full + kNQ;
   sh.xmax = reinterpret_cast<float*>(smem + L::XM_OFF);
   sh.page_ok = reinterpret_cast<int*>(bars + L::NBARS);
   sh.kq = reinterpret_cast<float*>(smem + L::KQ_OFF);
   sh.vs = reinterpret_cast<float*>(smem + L::VS_OFF);
-  sh.vmax = reinterpret_cast<float*>(smem + L::MISC_OFF);            // [NB][4]
-  sh.nbad = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);         // [NB][4]
-  sh.qscale = reinterpret_cast<float*>(smem + L::MISC_OFF + 64);
-  sh.tmem = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF + 68);
-  sh.abort = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 72);
-  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 80);   // [8] softmax amax
+  sh.vmax = reinterpret_cast<float*>(smem + L::MISC_OFF);            // [kNB][4]
+  sh.nbad = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);         // [kNQ][4]
+  sh.qscale = reinterpret_cast<float*>(smem + L::MISC_OFF + 96);
+  sh.tmem = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF + 100);
+  sh.abort = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 104);
+  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 112);  // [8] softmax amax
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::RG; ++s) {
@@ -360,6 +365,10 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     mbar_init(sh.q_ready, kSoftWarps);
     mbar_init(sh.fin, 1);
     for (int k = 0; k < 4; ++k) mbar_init(&sh.xch[k], 2);
+    for (int k = 0; k < kNQ; ++k) {
+      mbar_init(&sh.kq_full[k], 4);
+      mbar_init(&sh.kqfree[k], kSoftWarps);
+    }
     *sh.abort = 0;
     fence_mbar_init();
   }
@@ -379,6 +388,11 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     int jb = 0;
     for (; jb < nblk && ok_run; ++jb) {
       const int grp = jb % L::RG, round = jb / L::RG;
+      const int k = jb * L::PPB + lane, s = k % L::RS;
+      // the table entries are read before the wait for the ring group, so that their
+      // latency overlaps it
+      const bool mine = lane < L::PPB && k < npg;
+      const int blk = mine ? p.tables[static_cast<long>(b) * p.max_blocks + k] : -1;
       bool ok_lane = true;
       if (lane == 0 && round > 0 && !pf_wait(&sh.raw_empty[grp], (round - 1) & 1, sh.abort)) ok_lane = false;
       ok_run = __all_sync(0xffffffffu, ok_lane);
@@ -386,11 +400,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         if (lane == 0) pf_fail(p, sh.abort);
         break;
       }
-      const int k = jb * L::PPB + lane, s = k % L::RS;
       bool valid = false;
-      int blk = -1;
-      if (lane < L::PPB && k < npg) {
-        blk = p.tables[static_cast<long>(b) * p.max_blocks + k];
+      if (mine) {
         valid = blk >= 0 && blk < p.NB;
         sh.page_ok[s] = valid;
         if (!valid) record_fault(p.fault, KVQ_FAULT_BLOCK);
@@ -411,10 +422,10 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   } else if (warp >= kConvWarp0) {
     // ------------------------------------------------------------ converters
     // warps 10-13 convert K, warps 14-17 V; thread (c, rr): 16-byte output chunk c (elements
-    // 8c..8c+7 of a row) of rows rr + 8i.  K of block j waits for the block's pages and for
-    // the softmax of block j - NB (done with this buffer's K multipliers, and S of j - NB with
-    // its K); V of block j for the pages and for P V of block j - NB (done with its V).  The
-    // block's ring group is released once all eight warps have read it.
+    // 8c..8c+7 of a row) of rows rr + 8i.  K of block j waits for the block's pages, for S of
+    // block j - NB (done with this K tile buffer) and for the softmax of block j - kNQ (done
+    // with this slot of K multipliers); V of block j for the pages and for P V of block j - NB
+    // (done with its V).  The block's ring group is released once all eight warps have read it.
     const int part = warp >= kConvWarp0 + 4 ? 1 : 0;
     const int cw = (warp - kConvWarp0) & 3;
     const int ct = cw * 32 + lane;                        // 0..127
@@ -429,7 +440,10 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       {
         bool ok = true;
         if (part == 0) {
-          if (j >= NB && !pf_wait(&sh.p_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) ok = false;
+          // the K tile buffer: S of block j - NB has read it; the multiplier slot: the
+          // softmax of block j - kNQ is done with it
+          if (j >= NB && !pf_wait(&sh.s_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) ok = false;
+          if (ok && j >= kNQ && !pf_wait(&sh.kqfree[j % kNQ], ((j / kNQ) - 1) & 1, sh.abort)) ok = false;
         } else if (j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
           ok = false;
         }
@@ -499,7 +513,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
                 *reinterpret_cast<uint4*>(smem + L::K_OFF + (kb * 2 + 1) * kTile + tile_off(t, c)) = lo;
                 if (c == 0) {
                   const bool badtok = !ring && have && !pok && pos <= pmax;
-                  sh.kq[kb * kBlk + t] = valid ? qsc : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+                  sh.kq[(j % kNQ) * kBlk + t] = valid ? qsc : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
                   bad += badtok;
                 }
               }
@@ -552,7 +566,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         }
         if (part == 0) {
           const unsigned nbad = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(val));
-          if (lane == 0) sh.nbad[kb * 4 + cw] = static_cast<int>(nbad);
+          if (lane == 0) sh.nbad[(j % kNQ) * 4 + cw] = static_cast<int>(nbad);
         } else {
           // V scales are >= 0: their bit patterns order as the values do
           const unsigned vmb = __reduce_max_sync(0xffffffffu, __float_as_uint(val));
@@ -561,7 +575,12 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         tc::fence_async_shared();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(part == 0 ? &sh.k_full[kb] : &sh.v_full[kb]);
+          if (part == 0) {
+            mbar_arrive(&sh.k_full[kb]);
+            mbar_arrive(&sh.kq_full[j % kNQ]);
+          } else {
+            mbar_arrive(&sh.v_full[kb]);
+          }
           if (paged) mbar_arrive(&sh.raw_empty[j % L::RG]);
         }
       }
@@ -722,53 +741,69 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     bool ok = true;
     float* xm = sh.xmax;                                   // [2][2][128]: block parity, half, row
     for (int j = 0; j < J; ++j) {
-      const int sb = j & 1, kb = j % NB;
-      if (!pf_wait(&sh.k_full[kb], (j / NB) & 1, sh.abort) ||
+      const int sb = j & 1, kb = j % NB, qs = j % kNQ;
+      // the block's K multipliers through their own slot barrier: K of block j + NB may
+      // complete k_full once more before this wait (the next phase of kq_full[qs] needs
+      // this softmax's release of the slot)
+      if (!pf_wait(&sh.kq_full[qs], (j / kNQ) & 1, sh.abort) ||
           !pf_wait(&sh.s_full[sb], (j >> 1) & 1, sh.abort)) {
         ok = false;
       }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::fence_after_sync();
-      const float* kq = sh.kq + kb * kBlk + col0;
-      const bool fast = sh.nbad[kb * 4] + sh.nbad[kb * 4 + 1] + sh.nbad[kb * 4 + 2] + sh.nbad[kb * 4 + 3] == 0 &&
+      const float* kq = sh.kq + qs * kBlk + col0;
+      const bool fast = sh.nbad[qs * 4] + sh.nbad[qs * 4 + 1] + sh.nbad[qs * 4 + 2] + sh.nbad[qs * 4 + 3] == 0 &&
                         j * kBlk + kBlk - 1 <= pmin;   // uniform
       // causal boundary (position <= this row's) and tokens of bad pages (multiplier NaN)
       const int lim = row_ok ? pos_r - j * kBlk - col0 : -1;
-      // pass 1: the largest scaled score of this row's 64 columns, 32 at a time (read from
-      // TMEM again in pass 2; the loops are not unrolled, to keep the hot code small).  Blocks
-      // wholly visible to every row of the tile take a path with no per-score tests.
+      // pass 1: the largest scaled score of this row's 64 columns, 16 at a time (read from
+      // TMEM again in pass 2).  Blocks wholly visible to every row of the tile take a path
+      // with no per-score tests, in which the load of the next 16 columns is in flight while
+      // the current ones are reduced.
+      const uint32_t sbase = lanebase + 128 * sb + col0;
       float m0 = -INFINITY, m1 = -INFINITY;
-      if (fast) {
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t sr[32];
-          tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
+      uint32_t ra[16], rb[16];
+      auto max16 = [&](const uint32_t* r, int c0) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 f = *reinterpret_cast<const float4*>(kq + 32 * cc + i);
-            const float2 a = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
-                                        make_float2(f.x, f.y));
-            const float2 c = __fmul2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
-                                        make_float2(f.z, f.w));
-            m0 = max3(m0, a.x, a.y);
-            m1 = max3(m1, c.x, c.y);
-          }
+        for (int i = 0; i < 16; i += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(kq + c0 + i);
+          const float2 a = __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                      make_float2(f.x, f.y));
+          const float2 c = __fmul2_rn(make_float2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3])),
+                                      make_float2(f.z, f.w));
+          m0 = max3(m0, a.x, a.y);
+          m1 = max3(m1, c.x, c.y);
         }
+      };
+      if (fast) {
+        tc::ld16_issue(sbase, ra);
+        tc::ld_wait16(ra);
+        tc::ld16_issue(sbase + 16, rb);
+        max16(ra, 0);
+        tc::ld_wait16(rb);
+        tc::ld16_issue(sbase + 32, ra);
+        max16(rb, 16);
+        tc::ld_wait16(ra);
+        tc::ld16_issue(sbase + 48, rb);
+        max16(ra, 32);
+        tc::ld_wait16(rb);
+        max16(rb, 48);
       } else {
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t sr[32];
-          tc::ld32(lanebase + 128 * sb + col0 + 32 * cc, sr);
+        for (int cc = 0; cc < 4; ++cc) {
+          tc::ld16(sbase + 16 * cc, ra);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const int t = 32 * cc + i;
+          for (int i = 0; i < 16; i += 2) {
+            const int t = 16 * cc + i;
             const float2 f = *reinterpret_cast<const float2*>(kq + t);
-            const float2 a = __fmul2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), f);
+            const float2 a = __fmul2_rn(make_float2(__uint_as_float(ra[i]), __uint_as_float(ra[i + 1])), f);
             m0 = fmaxf(m0, (t <= lim && f.x == f.x) ? a.x : -INFINITY);
             m1 = fmaxf(m1, (t + 1 <= lim && f.y == f.y) ? a.y : -INFINITY);
           }
         }
       }
+      // the first 16 columns of pass 2 are read while the row maxima are exchanged
+      tc::ld16_issue(sbase, ra);
       float mx = fmaxf(m0, m1);
       // the row's max over both halves: exchange with the partner warp of this quarter
       xm[(sb * 2 + hf) * kRows + r] = mx;
@@ -818,43 +853,59 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       // (hi halves in the first 8 TMEM columns, lo halves in the next 8)
       float2 lsum = make_float2(0.f, 0.f);
       const float2 noff = make_float2(-off, -off);
-      auto pass2 = [&](auto masked) {
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t sr[16];
-          tc::ld16(lanebase + 128 * sb + col0 + 16 * cc, sr);
-          uint32_t ph[8], pl[8];
+      auto p16 = [&](const uint32_t* r, int c0, auto masked) {
+        uint32_t ph[8], pl[8];
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
-            const int t = 16 * cc + 2 * i;
-            const float4 f = *reinterpret_cast<const float4*>(kq + t);
-            const float4 vv = *reinterpret_cast<const float4*>(vsp + t);
-            float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                                   make_float2(f.x, f.y), noff);
-            float2 xb = __ffma2_rn(make_float2(__uint_as_float(sr[2 * i + 2]), __uint_as_float(sr[2 * i + 3])),
-                                   make_float2(f.z, f.w), noff);
-            if constexpr (decltype(masked)::value) {
-              if (!(t <= lim && f.x == f.x)) xa.x = -INFINITY;
-              if (!(t + 1 <= lim && f.y == f.y)) xa.y = -INFINITY;
-              if (!(t + 2 <= lim && f.z == f.z)) xb.x = -INFINITY;
-              if (!(t + 3 <= lim && f.w == f.w)) xb.y = -INFINITY;
-            }
-            const float2 ea = make_float2(ex2(xa.x), ex2(xa.y)), eb = make_float2(ex2(xb.x), ex2(xb.y));
-            lsum = __fadd2_rn(lsum, __fadd2_rn(ea, eb));
-            split2<kBf>(__fmul2_rn(ea, make_float2(vv.x, vv.y)), ph[i], pl[i]);
-            split2<kBf>(__fmul2_rn(eb, make_float2(vv.z, vv.w)), ph[i + 1], pl[i + 1]);
+        for (int i = 0; i < 8; i += 2) {
+          const int t = c0 + 2 * i;
+          const float4 f = *reinterpret_cast<const float4*>(kq + t);
+          const float4 vv = *reinterpret_cast<const float4*>(vsp + t);
+          float2 xa = __ffma2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                 make_float2(f.x, f.y), noff);
+          float2 xb = __ffma2_rn(make_float2(__uint_as_float(r[2 * i + 2]), __uint_as_float(r[2 * i + 3])),
+                                 make_float2(f.z, f.w), noff);
+          if constexpr (decltype(masked)::value) {
+            if (!(t <= lim && f.x == f.x)) xa.x = -INFINITY;
+            if (!(t + 1 <= lim && f.y == f.y)) xa.y = -INFINITY;
+            if (!(t + 2 <= lim && f.z == f.z)) xb.x = -INFINITY;
+            if (!(t + 3 <= lim && f.w == f.w)) xb.y = -INFINITY;
           }
-          st8(lanebase + 128 * sb + col0 + 16 * cc, ph);
-          st8(lanebase + 128 * sb + col0 + 16 * cc + 8, pl);
+          const float2 ea = make_float2(ex2(xa.x), ex2(xa.y)), eb = make_float2(ex2(xb.x), ex2(xb.y));
+          lsum = __fadd2_rn(lsum, __fadd2_rn(ea, eb));
+          split2<kBf>(__fmul2_rn(ea, make_float2(vv.x, vv.y)), ph[i], pl[i]);
+          split2<kBf>(__fmul2_rn(eb, make_float2(vv.z, vv.w)), ph[i + 1], pl[i + 1]);
         }
+        st8(sbase + c0, ph);
+        st8(sbase + c0 + 8, pl);
       };
-      if (fast) pass2(std::false_type{});
-      else pass2(std::true_type{});
+      tc::ld_wait16(ra);
+      if (fast) {
+        tc::ld16_issue(sbase + 16, rb);
+        p16(ra, 0, std::false_type{});
+        tc::ld_wait16(rb);
+        tc::ld16_issue(sbase + 32, ra);
+        p16(rb, 16, std::false_type{});
+        tc::ld_wait16(ra);
+        tc::ld16_issue(sbase + 48, rb);
+        p16(ra, 32, std::false_type{});
+        tc::ld_wait16(rb);
+        p16(rb, 48, std::false_type{});
+      } else {
+        p16(ra, 0, std::true_type{});
+#pragma unroll 1
+        for (int cc = 1; cc < 4; ++cc) {
+          tc::ld16(sbase + 16 * cc, rb);
+          p16(rb, 16 * cc, std::true_type{});
+        }
+      }
       l += lsum.x + lsum.y;
       tc::st_wait();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.p_full[sb]);
+      if (lane == 0) {
+        mbar_arrive(&sh.p_full[sb]);
+        mbar_arrive(&sh.kqfree[qs]);
+      }
     }
     if (!ok) {
       if (lane == 0) pf_fail(p, sh.abort);

@@ -132,6 +132,30 @@ __device__ __forceinline__ void ld16(uint32_t taddr, uint32_t* r) {
       : "memory");
 }
 
+// 16 consecutive columns of the calling warp's 32 lanes, NOT waited for: the registers may be
+// read only after ld_wait16 on the same array, which takes them as in-out operands so that
+// no use can be scheduled before the wait.
+__device__ __forceinline__ void ld16_issue(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Wait for every TMEM load of this thread in flight; r: the 16 registers of one of them.
+__device__ __forceinline__ void ld_wait16(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+
 // 64 consecutive columns of the calling warp's 32 lanes: two 32-column loads in flight,
 // one wait.
 __device__ __forceinline__ void ld64(uint32_t taddr, uint32_t* r) {

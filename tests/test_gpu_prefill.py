@@ -230,7 +230,7 @@ def test_prefill_bad_block_is_masked_and_counted():
                      int(w.context_lens.max())).cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
     cnt, bits = gc.read_fault()
-    assert cnt > 0 and (bits & 2)
+    assert cnt > 0 and bits == 2                      # the bad entry alone: no wait ran out
     assert np.isfinite(out).all()
     # sequence 0 without positions 32..47: the oracle over the remaining positions
     K, V = oc.gather(w.block_tables.numpy()[0], int(w.context_lens[0]))
