@@ -262,17 +262,25 @@ __device__ __forceinline__ float dense_part(uint8_t* smem, const PfShared& sh, i
   // row t of the tile: t & 7 == rr & 7 for all of this thread's rows, so the swizzled chunk is
   // the same for all; only the row offset changes
   uint8_t* tile = smem + (isv ? L::V_OFF : L::K_OFF) + kb * kTile + tile_off(rr, c) - rr * 128;
+  auto cvt = [&](const RawT& r) -> uint4 {
+    if constexpr (L::BITS == 8) return CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(r) : e4m3x8_to_f16(r);
+    else return r;
+  };
+  if (whole) {
 #pragma unroll
-  for (int pp = 0; pp < PPB; ++pp)
+    for (int pp = 0; pp < PPB; ++pp)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int t = pp * BS + rr + 8 * h;
-      uint4 out;
-      if constexpr (L::BITS == 8) out = CD == KVQ_DTYPE_INT8 ? i8x8_to_f16(w[pp][h]) : e4m3x8_to_f16(w[pp][h]);
-      else out = w[pp][h];
-      if (!whole && !(((pok >> pp) & 1u) && j * kBlk + t <= pmax)) out = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(tile + t * 128) = out;
-    }
+      for (int h = 0; h < 2; ++h) *reinterpret_cast<uint4*>(tile + (pp * BS + rr + 8 * h) * 128) = cvt(w[pp][h]);
+  } else {
+#pragma unroll
+    for (int pp = 0; pp < PPB; ++pp)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = pp * BS + rr + 8 * h;
+        const bool keep = ((pok >> pp) & 1u) && j * kBlk + t <= pmax;
+        *reinterpret_cast<uint4*>(tile + t * 128) = keep ? cvt(w[pp][h]) : make_uint4(0, 0, 0, 0);
+      }
+  }
   const int t = ct, pp = t >> 4, row = t & 15, k = j * PPB + pp, pos = j * kBlk + t;
   const bool have = k < npg, pk = (pok >> pp) & 1u;
   const bool valid = pk && pos <= pmax;
