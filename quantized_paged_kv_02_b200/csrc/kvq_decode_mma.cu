@@ -222,10 +222,10 @@ decode_mma_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         else static_s = sp[p.mode == KVQ_SCALE_PER_HEAD ? kvh : 0];
       }
       if (p.act_fp16)
-        quantize_row_part<__half, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
+        quantize_row_part<__half, CD, kD>(&u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
                                           static_s, chan_s);
       else
-        quantize_row_part<__nv_bfloat16, CD, kD>(u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
+        quantize_row_part<__nv_bfloat16, CD, kD>(&u, l, true, kv, pos % BS, BS, rec, L::OFF_V, L::OFF_S, PT,
                                                  static_s, chan_s);
       fence_proxy_async_global();
       __syncwarp();

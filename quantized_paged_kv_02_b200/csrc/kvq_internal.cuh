@@ -6,6 +6,8 @@
 //   [P-mem]  "大模型KV Cache显存优化与量化技术实践" (intelliparadigm.com)
 #pragma once
 
+#include <type_traits>
+
 #include <utility>
 
 #include <cuda_bf16.h>
@@ -38,12 +40,22 @@ template <> struct Act<__half> {
   static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 };
 
-// Eight 16-bit activation values packed in a uint4 -> float.
+// Eight 16-bit activation values packed in a uint4 -> float (bf16: the bits placed in the
+// upper half of a binary32, exact; fp16: the paired conversion).
 template <typename T>
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
-  const T* h = reinterpret_cast<const T*>(&u);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = Act<T>::to_f(h[i]);
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    } else {
+      const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      f[2 * i] = p.x;
+      f[2 * i + 1] = p.y;
+    }
+  }
 }
 
 __device__ __forceinline__ float e4m3_to_float(uint8_t c) {
@@ -74,54 +86,146 @@ __device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(div_rn(x, s), __NV_SATFINITE, __NV_E4M3));
 }
 
+// Codes of 8 values against one scale s > 0, equal to those of quant_int8 / quant_fp8 (the
+// quotient x / s rounded to float32 first).  Fast path: y = x * r with r = 1/s rounded
+// once (__frcp_rn); y is within 3.01 * 2^-24 |y| of the float32 quotient.  INT8 rounds y to an
+// integer by adding 1.5 * 2^23 (round to nearest even); if y lies within 2^-12 of a half
+// integer the two roundings could differ.  E4M3 rounds y (1 - 2^-20) and y (1 + 2^-20),
+// which bracket the quotient; rounding is monotonic, so if they agree the quotient rounds
+// the same.  A lane with any value near a midpoint, out of range (|y| >= 129 before
+// clamping when `bounded` is false) or not finite divides instead.  `bounded`: |x| is at
+// most 127 s, as for per-token scales taken from the row's own maximum.
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
+template <int CD>
+__device__ __forceinline__ uint2 quant8_same_scale(const float* x, float s, float r, bool bounded) {
+  bool ok = r <= 3.0e38f;
+  uint32_t w0, w1;
+  if constexpr (CD == KVQ_DTYPE_INT8) {
+    constexpr float kShift = 12582912.f;                  // 1.5 * 2^23
+    constexpr float kGap = 0.5f - 0.000244140625f;         // 1/2 - 2^-12
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float2 y = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(r, r));
+      if (!bounded) {
+        ok = ok && y.x == y.x && y.y == y.y;                // NaN: divide
+        y = make_float2(fminf(fmaxf(y.x, -129.f), 129.f), fminf(fmaxf(y.y, -129.f), 129.f));
+      }
+      const float2 t = __fadd2_rn(y, make_float2(kShift, kShift));
+      const float2 rn = __fadd2_rn(t, make_float2(-kShift, -kShift));
+      const float2 d = __ffma2_rn(rn, make_float2(-1.f, -1.f), y);   // y - round(y), exact
+      ok = ok && fabsf(d.x) < kGap && fabsf(d.y) < kGap;
+      int qa = __float_as_int(t.x) - 0x4B400000, qb = __float_as_int(t.y) - 0x4B400000;
+      if (!bounded) {
+        qa = max(-128, min(127, qa));
+        qb = max(-128, min(127, qb));
+      }
+      b[i] = static_cast<uint32_t>(qa);
+      b[i + 1] = static_cast<uint32_t>(qb);
+    }
+    w0 = pack4_low_bytes(b[0], b[1], b[2], b[3]);
+    w1 = pack4_low_bytes(b[4], b[5], b[6], b[7]);
+  } else {
+    constexpr float kDn = 1.f - 0x1p-20f, kUp = 1.f + 0x1p-20f;
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const float2 y = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(r, r));
+      const float2 lo = __fmul2_rn(y, make_float2(kDn, kDn)), hi = __fmul2_rn(y, make_float2(kUp, kUp));
+      uint32_t ca, cb;
+      asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
+          : "=r"(ca) : "f"(lo.y), "f"(lo.x));
+      asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
+          : "=r"(cb) : "f"(hi.y), "f"(hi.x));
+      ok = ok && ca == cb;
+      h[i / 2] = ca;
+    }
+    w0 = h[0] | (h[1] << 16);
+    w1 = h[2] | (h[3] << 16);
+  }
+  if (!ok) {
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
+    w0 = pack4_low_bytes(c[0], c[1], c[2], c[3]);
+    w1 = pack4_low_bytes(c[4], c[5], c[6], c[7]);
+  }
+  return make_uint2(w0, w1);
+}
+
 // One lane's share of quantizing one row (one token, one kv head, K or V) into its page
-// record.  A row is handled by D*2/16 consecutive lanes (a power of two dividing 32);
-// lane l holds activation elements [8l, 8l+8) in `u`.  `write` false: the lane joins the
-// shuffles but stores nothing.  Per-token modes reduce max|x| over the row's lanes and
-// store the float32 scale; static modes use `static_s`, or per channel the row's [D]
-// scales `chan_s`.  INT8: [P-mem] §3.1 对称量化算法 (scale = max|x|/127,
+// record.  A row is handled by D / (8 NV) consecutive lanes (a power of two dividing 32);
+// lane l holds activation elements [8 NV l, 8 NV l + 8 NV) in u[0..NV).  `write` false: the
+// lane joins the shuffles but stores nothing.  Per-token modes reduce max|x| over the
+// row's lanes and store the float32 scale; static modes use `static_s`, or per channel the
+// row's [D] scales `chan_s`.  INT8: [P-mem] §3.1 对称量化算法 (scale = max|x|/127,
 // q = clamp(round(x/scale), -128, 127)); FP8: [P-vLLM] "KV Cache量化策略" (E4M3 storage
 // with a scale).
-template <typename TA, int CD, int D>
-__device__ __forceinline__ void quantize_row_part(const uint4& u, int l, bool write, int kv, int off,
+template <typename TA, int CD, int D, int NV = 1>
+__device__ __forceinline__ void quantize_row_part(const uint4* u, int l, bool write, int kv, int off,
                                                   int bs, uint8_t* rec, int off_v, int off_s,
                                                   bool per_token, float static_s,
                                                   const float* chan_s = nullptr) {
-  constexpr int LPR = D * 2 / 16;
+  constexpr int E = 8 * NV;                 // elements per lane
+  constexpr int LPR = D / E;
   constexpr int ROWB = (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) ? 2 * D : D;
   uint8_t* dst_row = rec + (kv ? off_v : 0) + off * ROWB;
   if constexpr (CD == KVQ_DTYPE_BF16 || CD == KVQ_DTYPE_FP16) {
-    if (write) *reinterpret_cast<uint4*>(dst_row + l * 16) = u;
+    if (write) {
+#pragma unroll
+      for (int v = 0; v < NV; ++v) reinterpret_cast<uint4*>(dst_row + l * 16 * NV)[v] = u[v];
+    }
   } else {
-    float x[8];
-    unpack8<TA>(u, x);
+    float x[E];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) unpack8<TA>(u[v], x + 8 * v);
     float s = static_s;
     if (per_token) {
       float m = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+      for (int i = 0; i < E; ++i) m = fmaxf(m, fabsf(x[i]));
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       s = div_rn(m, QMax<CD>::v);
       if (write && l == 0) reinterpret_cast<float*>(rec + off_s)[(kv ? bs : 0) + off] = s;
     }
-    // PER_CHANNEL: chan_s is the row's [D] scales; this lane's are [8l, 8l+8)
-    float cs[8];
+    uint32_t w[2 * NV];
+    if (chan_s == nullptr && s != 0.f) {
+      const float r = __frcp_rn(s);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) cs[i] = s;
-    if (chan_s != nullptr) {
-      const float4 a = reinterpret_cast<const float4*>(chan_s)[2 * l];
-      const float4 b = reinterpret_cast<const float4*>(chan_s)[2 * l + 1];
-      cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
-      cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
-    }
-    uint32_t w0 = 0, w1 = 0;
+      for (int v = 0; v < NV; ++v) {
+        const uint2 c = quant8_same_scale<CD>(x + 8 * v, s, r, per_token);
+        w[2 * v] = c.x;
+        w[2 * v + 1] = c.y;
+      }
+    } else {
+      // PER_CHANNEL: chan_s is the row's [D] scales; this lane's are [E l, E l + E)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t c = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], cs[i]) : quant_fp8(x[i], cs[i]);
-      if (i < 4) w0 |= c << (8 * i); else w1 |= c << (8 * (i - 4));
+      for (int v = 0; v < NV; ++v) {
+        float cs[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cs[i] = s;
+        if (chan_s != nullptr) {
+          const float4 a = reinterpret_cast<const float4*>(chan_s)[(E * l + 8 * v) / 4];
+          const float4 b = reinterpret_cast<const float4*>(chan_s)[(E * l + 8 * v) / 4 + 1];
+          cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+          cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+        }
+        uint32_t c[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          c[i] = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[8 * v + i], cs[i]) : quant_fp8(x[8 * v + i], cs[i]);
+        w[2 * v] = pack4_low_bytes(c[0], c[1], c[2], c[3]);
+        w[2 * v + 1] = pack4_low_bytes(c[4], c[5], c[6], c[7]);
+      }
     }
-    if (write) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w0, w1);
+    if (write) {
+      if constexpr (NV == 1) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w[0], w[1]);
+      else *reinterpret_cast<uint4*>(dst_row + l * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 

@@ -33,39 +33,54 @@ struct WriteParams {
   int32_t* fault;
 };
 
+// grid (T, ceil(2 H LPR / blockDim)): token t = blockIdx.x; its 2H rows (K rows of heads
+// 0..H-1, then V rows) are spread over blockIdx.y and the CTA's threads (2 H LPR rounded up
+// to whole warps, at most 256), LPR = D / 16 lanes
+// per row with 16 activations (two 16-byte loads) each, so no index needs a division and
+// each lane's index and scale work covers 16 values.  bs_shift >= 0: the block size is
+// 2^bs_shift.
 template <typename TA, int CD, int D>
-__global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p) {
+__global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p, int bs_shift) {
   griddep_launch_dependents();   // a decode launched after this one may start its set-up
-  constexpr int LPR = D * 2 / 16;   // lanes per row
-  constexpr int RPW = 32 / LPR;     // rows per warp
-  const int lane = threadIdx.x & 31;
-  const long warp = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int l = lane % LPR;
-  const long task = warp * RPW + lane / LPR;   // (K or V, token, head), head fastest
-  const long TH = static_cast<long>(p.T) * p.H;
-  const bool valid = task < 2 * TH;
-  const int kv = valid ? static_cast<int>(task / TH) : 0;
-  const long th = valid ? task % TH : 0;
-  const int t = static_cast<int>(th / p.H);
-  const int h = static_cast<int>(th % p.H);
-  const int slot = valid ? p.slots[t] : -1;
+  constexpr int NV = 2;             // 16-byte chunks per lane
+  constexpr int LPR = D / (8 * NV); // lanes per row
+  const int RPB = blockDim.x / LPR;  // rows per CTA
+  const int l = threadIdx.x % LPR;
+  const int t = blockIdx.x;
+  const int r = blockIdx.y * RPB + threadIdx.x / LPR;   // row of the token: (kv, head)
+  const bool valid = r < 2 * p.H;
+  // rows past the token's 2H (the tail of the last CTA along y) stand in for head 0: they
+  // take part in the shuffles of their lane group but read and write nothing
+  const int kv = (valid && r >= p.H) ? 1 : 0;
+  const int h = valid ? r - kv * p.H : 0;
+  const int slot = p.slots[t];
   const long nslots = static_cast<long>(p.NB) * p.bs;
   const bool write = valid && slot >= 0 && slot < nslots;
-  if (valid && l == 0 && kv == 0 && h == 0 && (slot < -1 || slot >= nslots)) record_fault(p.fault, KVQ_FAULT_SLOT);
+  if (blockIdx.y == 0 && threadIdx.x == 0 && (slot < -1 || slot >= nslots)) record_fault(p.fault, KVQ_FAULT_SLOT);
 
-  uint4 u = make_uint4(0, 0, 0, 0);
-  const TA* src = static_cast<const TA*>(kv ? p.v : p.k) + th * D + l * 8;
-  if (write) u = *reinterpret_cast<const uint4*>(src);
-  const int blk = write ? slot / p.bs : 0;
-  const int off = write ? slot % p.bs : 0;
+  uint4 u[NV];
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const TA*>(kv ? p.v : p.k) +
+                                                    (static_cast<long>(t) * p.H + h) * D + l * 8 * NV);
+#pragma unroll
+  for (int v = 0; v < NV; ++v) u[v] = write ? src[v] : make_uint4(0, 0, 0, 0);
+  int blk = 0, off = 0;
+  if (write) {
+    if (bs_shift >= 0) {
+      blk = slot >> bs_shift;
+      off = slot & ((1 << bs_shift) - 1);
+    } else {
+      blk = slot / p.bs;
+      off = slot - blk * p.bs;
+    }
+  }
   // record of (block, head); this row's codes and (per-token) scale inside it
   uint8_t* rec = p.pages + (static_cast<long>(blk) * p.H + h) * p.record;
   const float* sp = kv ? p.v_static : p.k_static;
   const bool is_static = p.scale_mode == KVQ_SCALE_PER_HEAD || p.scale_mode == KVQ_SCALE_PER_TENSOR;
-  const float static_s = is_static ? sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0] : 0.f;
+  const float static_s = (valid && is_static) ? sp[p.scale_mode == KVQ_SCALE_PER_HEAD ? h : 0] : 0.f;
   const float* chan_s = p.scale_mode == KVQ_SCALE_PER_CHANNEL ? sp + static_cast<long>(h) * D : nullptr;
-  quantize_row_part<TA, CD, D>(u, l, write, kv, off, p.bs, rec, p.off_v, p.off_s,
-                               p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD, static_s, chan_s);
+  quantize_row_part<TA, CD, D, NV>(u, l, write, kv, off, p.bs, rec, p.off_v, p.off_s,
+                                   p.scale_mode == KVQ_SCALE_PER_TOKEN_HEAD, static_s, chan_s);
 }
 
 // ------------------------------------------------------------------ INT4 (KIVI)
@@ -256,12 +271,16 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
 
 template <typename TA, int CD, int D>
 cudaError_t dense_launch(const WriteParams& p, cudaStream_t s) {
-  constexpr int LPR = D * 2 / 16;
-  const long rows = 2L * p.T * p.H;
-  const long threads = (rows * LPR + 31) / 32 * 32;
-  const long blocks = (threads + 255) / 256;
-  if (blocks == 0) return cudaSuccess;
-  write_dense_kernel<TA, CD, D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  constexpr int LPR = D / 16;
+  if (p.T <= 0) return cudaSuccess;
+  const int need = 2 * p.H * LPR;                       // threads of one token
+  const int threads = need >= 256 ? 256 : (need + 31) / 32 * 32;
+  const int ys = (need + threads - 1) / threads;
+  if (ys > 65535) return cudaErrorInvalidValue;
+  int bs_shift = -1;
+  for (int k = 0; k < 31; ++k)
+    if ((1 << k) == p.bs) bs_shift = k;
+  write_dense_kernel<TA, CD, D><<<dim3(static_cast<unsigned>(p.T), static_cast<unsigned>(ys)), threads, 0, s>>>(p, bs_shift);
   return cudaGetLastError();
 }
 

@@ -125,6 +125,46 @@ def test_write_edge_cases():
     helpers.assert_same_cache(gc, oc)
 
 
+def test_write_rounding_midpoints():
+    """Quotients x / s exactly on a rounding midpoint (ties to even) and right beside one: an
+    INT8 per-token row whose maximum is 127 * 2^-3 (scale 2^-3, quotients n + 1/2), a static
+    INT8 scale of 1/2 with the same kind of row plus saturating values, and E4M3 midpoints
+    (1 + (2k + 1) / 16) * 2^e against a static FP8 scale of 1."""
+    from oracle import cache as ocache
+    from quantized_paged_kv_02_b200 import kvq
+    H, D, bs, NB = 2, 128, 16, 2
+    n = torch.arange(D, dtype=torch.float64)
+    half = ((n - 64) + 0.5) * 0.125                   # quotients -63.5 .. 63.5 at scale 2^-3
+    half[0] = 127 * 0.125                             # the row maximum: scale exactly 2^-3
+    mids = torch.tensor([(1 + (2 * (i % 8) + 1) / 16.0) * 2.0 ** ((i // 8) % 12 - 6) for i in range(D)],
+                        dtype=torch.float64)
+    mids = torch.where(n % 2 == 0, mids, -mids)
+    g = torch.Generator().manual_seed(11)
+    rows = torch.randn(6, H, D, generator=g, dtype=torch.float64)
+    rows[0, 0] = half
+    rows[1, 1] = half * 8                             # scale 1, quotients n + 1/2 up to 127
+    rows[2, 0] = mids
+    rows[3, 1] = mids * 4
+    rows[4, 0, :8] = torch.tensor([300.0, -300.0, 63.75, -63.75, 63.25, 0.25, -0.25, 0.75])
+    k = rows.to(torch.bfloat16)
+    v = (rows * 0.5).to(torch.bfloat16)
+    assert torch.equal(k[0, 0].double(), half) and torch.equal(k[2, 0].double(), mids)
+    slots = torch.tensor([0, 3, 16, 17, 30, 31], dtype=torch.int32)
+    cases = (("int8", "per_token_head", None), ("int8", "per_head", (0.5, 0.5)),
+             ("fp8", "per_head", (1.0, 0.25)))
+    for cd, mode, st in cases:
+        sk = None if st is None else torch.tensor([st[0], st[1]], dtype=torch.float32)
+        kw = {} if st is None else {"static_scales": (sk.numpy(), sk.numpy())}
+        oc = ocache.PagedCache(cd, "bf16", mode, NB, bs, H, D, **kw)
+        oc.write(helpers.np64(k), helpers.np64(v), slots.numpy())
+        gkw = {} if st is None else {"static_k_scale": sk.cuda(), "static_v_scale": sk.cuda()}
+        gc = kvq.PagedKVCache(cd, "bf16", mode, NB, bs, H, D, **gkw)
+        gc.write(k.cuda(), v.cuda(), slots.cuda())
+        torch.cuda.synchronize()
+        helpers.assert_same_cache(gc, oc)
+        assert gc.read_fault() == (0, 0)
+
+
 def test_int4_bad_run_is_skipped_and_counted():
     from quantized_paged_kv_02_b200 import kvq
     H, D = 1, 128
