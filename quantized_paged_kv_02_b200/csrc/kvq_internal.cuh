@@ -87,66 +87,57 @@ __device__ __forceinline__ uint8_t quant_fp8(float x, float s) {
 }
 
 // Codes of 8 values against one scale s > 0, equal to those of quant_int8 / quant_fp8 (the
-// quotient x / s rounded to float32 first).  Fast path: y = x * r with r = 1/s rounded
-// once (__frcp_rn); y is within 3.01 * 2^-24 |y| of the float32 quotient.  INT8 rounds y to an
-// integer by adding 1.5 * 2^23 (round to nearest even); if y lies within 2^-12 of a half
-// integer the two roundings could differ.  E4M3 rounds y (1 - 2^-20) and y (1 + 2^-20),
-// which bracket the quotient; rounding is monotonic, so if they agree the quotient rounds
-// the same.  A lane with any value near a midpoint, out of range (|y| >= 129 before
-// clamping when `bounded` is false) or not finite divides instead.  `bounded`: |x| is at
-// most 127 s, as for per-token scales taken from the row's own maximum.
+// quotient x / s rounded to float32 first).  The quotient is formed without a division by
+// Markstein's correction step (P. Markstein, IBM J. Res. Dev. 34(1), 1990): if r = RN(1/s)
+// and q is within one ulp of x / s, the remainder x - q s is exact as one FMA and
+// RN(q + (x - q s) r) is the correctly rounded quotient, as long as nothing overflows or
+// underflows.  q0 = RN(x r) can be up to 1.5 ulp away, so one first step
+// q1 = RN(q0 + RN(x - q0 s) r) (error far below one ulp) precedes the exact one.  Quotients
+// below 2^-126 in magnitude round to a zero code of the right sign either way.  INT8 then rounds to an integer by adding
+// 1.5 * 2^23 (round to nearest even); E4M3 converts with satfinite.  A lane with a quotient
+// or reciprocal that is not finite, or a scale below 2^-100, divides instead.  `bounded`:
+// |x| is at most 127 s, as for per-token scales taken from the row's own maximum; otherwise
+// the quotient is clamped to [-129, 129] before rounding and the code to [-128, 127] after.
 __device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
 }
 
 template <int CD>
 __device__ __forceinline__ uint2 quant8_same_scale(const float* x, float s, float r, bool bounded) {
-  bool ok = r <= 3.0e38f;
+  bool hard = !(r <= 3.0e38f) || !(s >= 7.9e-31f);
   uint32_t w0, w1;
-  if constexpr (CD == KVQ_DTYPE_INT8) {
-    constexpr float kShift = 12582912.f;                  // 1.5 * 2^23
-    constexpr float kGap = 0.5f - 0.000244140625f;         // 1/2 - 2^-12
-    uint32_t b[8];
+  uint32_t b[8];
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      float2 y = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(r, r));
-      if (!bounded) {
-        ok = ok && y.x == y.x && y.y == y.y;                // NaN: divide
-        y = make_float2(fminf(fmaxf(y.x, -129.f), 129.f), fminf(fmaxf(y.y, -129.f), 129.f));
-      }
-      const float2 t = __fadd2_rn(y, make_float2(kShift, kShift));
-      const float2 rn = __fadd2_rn(t, make_float2(-kShift, -kShift));
-      const float2 d = __ffma2_rn(rn, make_float2(-1.f, -1.f), y);   // y - round(y), exact
-      ok = ok && fabsf(d.x) < kGap && fabsf(d.y) < kGap;
-      int qa = __float_as_int(t.x) - 0x4B400000, qb = __float_as_int(t.y) - 0x4B400000;
-      if (!bounded) {
-        qa = max(-128, min(127, qa));
-        qb = max(-128, min(127, qb));
-      }
-      b[i] = static_cast<uint32_t>(qa);
-      b[i + 1] = static_cast<uint32_t>(qb);
-    }
-    w0 = pack4_low_bytes(b[0], b[1], b[2], b[3]);
-    w1 = pack4_low_bytes(b[4], b[5], b[6], b[7]);
-  } else {
-    constexpr float kDn = 1.f - 0x1p-20f, kUp = 1.f + 0x1p-20f;
-    uint32_t h[4];
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      const float2 y = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(r, r));
-      const float2 lo = __fmul2_rn(y, make_float2(kDn, kDn)), hi = __fmul2_rn(y, make_float2(kUp, kUp));
-      uint32_t ca, cb;
+  for (int i = 0; i < 8; i += 2) {
+    const float2 xv = make_float2(x[i], x[i + 1]);
+    const float2 q0 = __fmul2_rn(xv, make_float2(r, r));
+    const float2 q1 = __ffma2_rn(__ffma2_rn(q0, make_float2(-s, -s), xv), make_float2(r, r), q0);
+    const float2 e = __ffma2_rn(q1, make_float2(-s, -s), xv);          // exact remainder
+    float2 q = __ffma2_rn(e, make_float2(r, r), q1);                    // fl(x / s)
+    hard = hard || !(fabsf(q.x) <= 3.0e38f) || !(fabsf(q.y) <= 3.0e38f);
+    if constexpr (CD == KVQ_DTYPE_INT8) {
+      constexpr float kShift = 12582912.f;                               // 1.5 * 2^23
+      if (!bounded) q = make_float2(fminf(fmaxf(q.x, -129.f), 129.f), fminf(fmaxf(q.y, -129.f), 129.f));
+      const float2 t = __fadd2_rn(q, make_float2(kShift, kShift));
+      b[i] = __float_as_uint(t.x) - 0x4B400000u;
+      b[i + 1] = __float_as_uint(t.y) - 0x4B400000u;
+    } else {
+      uint32_t c;
       asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
-          : "=r"(ca) : "f"(lo.y), "f"(lo.x));
-      asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
-          : "=r"(cb) : "f"(hi.y), "f"(hi.x));
-      ok = ok && ca == cb;
-      h[i / 2] = ca;
+          : "=r"(c) : "f"(q.y), "f"(q.x));
+      b[i] = c & 0xFFu;
+      b[i + 1] = c >> 8;
     }
-    w0 = h[0] | (h[1] << 16);
-    w1 = h[2] | (h[3] << 16);
   }
-  if (!ok) {
+  if constexpr (CD == KVQ_DTYPE_INT8) {
+    if (!bounded) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) b[i] = static_cast<uint32_t>(max(-128, min(127, static_cast<int>(b[i]))));
+    }
+  }
+  w0 = pack4_low_bytes(b[0], b[1], b[2], b[3]);
+  w1 = pack4_low_bytes(b[4], b[5], b[6], b[7]);
+  if (hard) {
     uint32_t c[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) c[i] = (CD == KVQ_DTYPE_INT8) ? quant_int8(x[i], s) : quant_fp8(x[i], s);
@@ -223,8 +214,14 @@ __device__ __forceinline__ void quantize_row_part(const uint4* u, int l, bool wr
       }
     }
     if (write) {
-      if constexpr (NV == 1) *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w[0], w[1]);
-      else *reinterpret_cast<uint4*>(dst_row + l * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      if constexpr (NV == 1) {
+        *reinterpret_cast<uint2*>(dst_row + l * 8) = make_uint2(w[0], w[1]);
+      } else {
+        static_assert(NV % 2 == 0, "whole 16-byte code stores");
+#pragma unroll
+        for (int v = 0; v < NV / 2; ++v)
+          reinterpret_cast<uint4*>(dst_row + l * 8 * NV)[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
     }
   }
 }

@@ -35,14 +35,14 @@ struct WriteParams {
 
 // grid (T, ceil(2 H LPR / blockDim)): token t = blockIdx.x; its 2H rows (K rows of heads
 // 0..H-1, then V rows) are spread over blockIdx.y and the CTA's threads (2 H LPR rounded up
-// to whole warps, at most 256), LPR = D / 16 lanes
-// per row with 16 activations (two 16-byte loads) each, so no index needs a division and
-// each lane's index and scale work covers 16 values.  bs_shift >= 0: the block size is
+// to whole warps, at most 256), LPR = D / 32 lanes
+// per row with 32 activations (four 16-byte loads) each, so no index needs a division and
+// each lane's index and scale work covers 32 values.  bs_shift >= 0: the block size is
 // 2^bs_shift.
 template <typename TA, int CD, int D>
 __global__ void __launch_bounds__(256) write_dense_kernel(WriteParams p, int bs_shift) {
   griddep_launch_dependents();   // a decode launched after this one may start its set-up
-  constexpr int NV = 2;             // 16-byte chunks per lane
+  constexpr int NV = 4;             // 16-byte chunks per lane
   constexpr int LPR = D / (8 * NV); // lanes per row
   const int RPB = blockDim.x / LPR;  // rows per CTA
   const int l = threadIdx.x % LPR;
@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(128) write_int4_kernel(Int4WriteParams p) {
 
 template <typename TA, int CD, int D>
 cudaError_t dense_launch(const WriteParams& p, cudaStream_t s) {
-  constexpr int LPR = D / 16;
+  constexpr int LPR = D / 32;
   if (p.T <= 0) return cudaSuccess;
   const int need = 2 * p.H * LPR;                       // threads of one token
   const int threads = need >= 256 ? 256 : (need + 31) / 32 * 32;

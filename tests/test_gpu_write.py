@@ -165,6 +165,37 @@ def test_write_rounding_midpoints():
         assert gc.read_fault() == (0, 0)
 
 
+@pytest.mark.parametrize("cd,mode", [("int8", "per_token_head"), ("int8", "per_head"),
+                                     ("fp8", "per_head"), ("fp8", "per_token_head")])
+def test_write_many_rows_bit_exact(cd, mode):
+    """8192 tokens x 4 heads of values spread over 40 binades (row magnitudes 2^-20 .. 2^20,
+    some rows with a single large outlier), written with per-token or static scales: every
+    code and scale byte-identical to the oracle's binary32 division and rounding."""
+    from oracle import cache as ocache
+    from quantized_paged_kv_02_b200 import kvq
+    T, H, D, bs = 8192, 4, 128, 16
+    NB = T // bs
+    g = torch.Generator().manual_seed(21)
+    mag = torch.pow(2.0, torch.randint(-20, 21, (T, H, 1), generator=g).double())
+    k = (torch.randn(T, H, D, generator=g, dtype=torch.float64) * mag)
+    v = (torch.rand(T, H, D, generator=g, dtype=torch.float64) - 0.5) * mag
+    k[::7, :, 3] *= 50.0
+    k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    slots = torch.randperm(NB * bs, generator=g)[:T].to(torch.int32)
+    kw, gkw = {}, {}
+    if mode == "per_head":
+        sk = torch.tensor([0.003, 0.5, 7.0, 1e-5], dtype=torch.float32)
+        kw = {"static_scales": (sk.numpy(), (sk * 3).numpy())}
+        gkw = {"static_k_scale": sk.cuda(), "static_v_scale": (sk * 3).cuda()}
+    oc = ocache.PagedCache(cd, "bf16", mode, NB, bs, H, D, **kw)
+    oc.write(helpers.np64(k), helpers.np64(v), slots.numpy())
+    gc = kvq.PagedKVCache(cd, "bf16", mode, NB, bs, H, D, **gkw)
+    gc.write(k.cuda(), v.cuda(), slots.cuda())
+    torch.cuda.synchronize()
+    helpers.assert_same_cache(gc, oc)
+    assert gc.read_fault() == (0, 0)
+
+
 def test_int4_bad_run_is_skipped_and_counted():
     from quantized_paged_kv_02_b200 import kvq
     H, D = 1, 128
