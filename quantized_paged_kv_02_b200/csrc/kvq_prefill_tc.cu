@@ -6,21 +6,28 @@
 // A CTA owns one tile of 128 query rows of one (sequence, kv head): 128 / g query tokens x
 // the g query heads that share the kv head (row r = token r / g, head r % g), and walks the
 // causal window of its last query in blocks of 128 cached tokens (8 pages).  Each page is
-// dequantized ONCE into shared memory for all 128 rows, instead of once per query token:
+// dequantized ONCE into shared memory for all 128 rows, instead of once per query token.
+// Eighteen warps, each role waiting only on what it consumes (mbarriers, every wait
+// bounded):
 //
-//   warp 4      producer: one bulk copy per page record (K codes, V codes, per-token scales)
-//               into a ring of raw stages;
-//   warps 6-9   converters: codes -> 16-bit tiles in the tensor cores' 128-byte-swizzled
-//               layout (INT8 through the exact 1024-magic, E4M3 by the hardware conversion,
-//               16-bit caches copied), K as the K-major B operand of S = Q K^T and V as the
-//               MN-major B operand of O = P V, plus the per-token scales of the block;
-//   warp 5      MMA issuer: S_j = Q K_j^T (M 128, N 128 tokens, K 128) into one of two TMEM
+//   warp 8      producer: the table entries of a block's pages, then one bulk copy per page
+//               record (K codes, V codes, per-token scales) into a ring of raw stages that
+//               turns over a block at a time (one full and one empty barrier per block);
+//   warps 10-13 K converters and warps 14-17 V converters: codes -> 16-bit tiles in the
+//               tensor cores' 128-byte-swizzled layout (INT8 through the exact 1024-magic,
+//               E4M3 by the hardware conversion, 16-bit caches copied), K as the K-major B
+//               operand of S = Q K^T and V as the MN-major B operand of O = P V, plus the
+//               per-token multipliers (in four slots of their own) and V scales;
+//   warp 9      MMA issuer: S_j = Q K_j^T (M 128, N 128 tokens, K 128) into one of two TMEM
 //               score buffers, then O += P_{j-1} V_{j-1} (N 128 channels, K 128 tokens);
-//   warps 0-3   softmax: thread r owns query row r, reads its 128 scores from TMEM, scales
-//               them (per-token K scale, softmax scale, log2 e), masks the causal boundary,
-//               keeps the running max (re-based only when a score exceeds it by 2^8) and sum,
-//               folds the per-token V scale into P, and writes P back over its scores as
-//               fp16 (bf16 for bf16 caches) hi + lo halves, the A operand of the P V MMA.
+//   warps 0-7   softmax: the two warps of a TMEM lane quarter share its 32 query rows,
+//               64 score columns each; they read the scores from TMEM (the next 16 columns'
+//               load in flight while the current ones are used), scale them (per-token K
+//               scale, softmax scale, log2 e), mask the causal boundary, agree on the row
+//               maximum through a per-quarter barrier (re-based only when a score exceeds the
+//               running maximum by 2^8), keep the row sum, fold the per-token V scale into P
+//               and write P back over its scores as fp16 (bf16 for bf16 caches) hi + lo
+//               halves, the A operand of the P V MMA.
 //
 // Q lives in TMEM too (written once by the softmax warps), so shared memory holds only the
 // K / V tiles and the raw ring.  The contraction is exact in the codes: for INT8 / FP8 the
@@ -29,7 +36,8 @@
 // pair), and P's hi + lo halves keep 22 bits.  For INT4 / 2-bit caches the dequantized
 // value (code - zero) * scale (at most 15 significant bits) is split exactly into bf16 hi +
 // lo tiles; S takes both (and both halves of q when activations are fp16), P V takes
-// P hi V hi + P hi V lo + P lo V hi.  Scores, softmax and O accumulate in fp32.  Chunked prefill is one of the techniques [P-prod] "为什么长上下文更需要 KV Cache
+// P hi V hi + P hi V lo + P lo V hi.  Scores, softmax and O accumulate in fp32.
+// Chunked prefill is one of the techniques [P-prod] "为什么长上下文更需要 KV Cache
 // Quantization" lists beside cache quantization; dequantization inside attention is the
 // design of [P-vLLM] "PagedAttention与KV Cache量化协同工作原理".
 #include <cudaTypedefs.h>
