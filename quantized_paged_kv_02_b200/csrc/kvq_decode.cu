@@ -77,11 +77,13 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
 // sixteen at a time so their loads overlap.
 __global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
   const int C = p.ctas;
-  griddep_wait();                      // the partials of the decode kernel
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);   // b * Hq + hq
   const int lane = threadIdx.x & 31;
-  if (row >= p.rows) return;
-  const int b = row / p.Hq, hq = row - b * p.Hq;
+  // the partition and the candidate range depend only on the call's inputs (context lengths,
+  // block tables), which the decode kernel does not write: they are worked out before the
+  // wait for its partials, overlapping its tail
+  const bool active = row < p.rows;
+  const int b = active ? row / p.Hq : 0, hq = active ? row - b * p.Hq : 0;
   const int kvh = hq / p.g, h = hq - kvh * p.g;
   long long tot = 0, before = 0;
   int npb = 0;
@@ -108,6 +110,8 @@ __global__ void __launch_bounds__(256) segment_reduce_kernel(DecodeParams p) {
     c_last = static_cast<int>((U1 * C + P - 1) / P) - 1;
   }
   const int K = (c_last - c_first + 1) * kSegWarps;
+  griddep_wait();                      // the partials of the decode kernel
+  if (!active) return;
   const long long u = static_cast<long long>(b) * p.H + kvh;
   const float* ml = p.ws_ml;
   const float* o = p.ws_o + 4 * lane;
