@@ -249,7 +249,7 @@ __device__ __forceinline__ void split8(const float* v, uint4& hi, uint4& lo) {
 // of K (a visible position on a page that failed its table check), token ct's V scale for V.
 template <int CD, bool PT>
 __device__ __forceinline__ float dense_part(uint8_t* smem, const PfShared& sh, int j, int kb, bool isv,
-                                            int ct, int npg, int pmax, float qsc) {
+                                            int ct, int npg, int pmax, float& qsc, bool& have_q) {
   using L = PfLayout<CD, PT>;
   constexpr int PPB = L::PPB, BS = L::BS;
   using RawT = typename std::conditional<L::BITS == 8, uint2, uint4>::type;
@@ -294,6 +294,13 @@ __device__ __forceinline__ float dense_part(uint8_t* smem, const PfShared& sh, i
   const bool valid = pk && pos <= pmax;
   const float* sc = reinterpret_cast<const float*>(smem + L::RAW_OFF + (k % L::RS) * L::REC + L::OFF_S);
   if (!isv) {
+    if (!have_q) {
+      // the first block: q's scale (the tile above is converted meanwhile); a wait that
+      // runs out leaves the multipliers at 0 and the abort flag stops every role
+      if (pf_wait(sh.q_ready, 0, sh.abort)) qsc = *sh.qscale;
+      else *sh.abort = 1;
+      have_q = true;
+    }
     float ks = 1.f;
     if constexpr (PT) ks = sc[row];
     // positions past the tile's last query are never visible: their multiplier is unused
@@ -446,8 +453,10 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     const int cw = (warp - kConvWarp0) & 3;
     const int ct = cw * 32 + lane;                        // 0..127
     const int c = ct & 15, rr = ct >> 4;
-    if (!pf_wait(sh.q_ready, 0, sh.abort)) pf_fail(p, sh.abort);
-    const float qsc = *sh.qscale;
+    // q's power-of-two scale enters only the K multipliers: the K warps wait for it after
+    // converting their first block's tile, the V warps never
+    float qsc = 0.f;
+    bool have_q = part == 1;
     const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
     const int G = c >> 3;                                 // 64-channel group of the chunk
     for (int j = 0; j < J && !*sh.abort; ++j) {
@@ -471,8 +480,13 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         // K: bad-token count; V: largest V scale
         float val = 0.f;
         if constexpr (!L::LB) {
-          val = dense_part<CD, PT>(smem, sh, j, kb, part == 1, ct, npg, pmax, qsc);
+          val = dense_part<CD, PT>(smem, sh, j, kb, part == 1, ct, npg, pmax, qsc, have_q);
         } else if (part == 0) {
+          if (!have_q) {
+            if (!pf_wait(sh.q_ready, 0, sh.abort)) pf_fail(p, sh.abort);
+            qsc = *sh.qscale;
+            have_q = true;
+          }
           int bad = 0;
           // K: rows rr + 8i of every page of the block, chunk c (low-bit caches)
           for (int pp = 0; pp < L::PPB; ++pp) {
@@ -693,18 +707,20 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       float qscale = p.scale_log2;
       if (p.mode == KVQ_SCALE_PER_HEAD) qscale *= p.k_static[kvh];
       if (p.mode == KVQ_SCALE_PER_TENSOR) qscale *= p.k_static[0];
+      // the row's 64 values in one round of loads, kept in registers for both passes
+      uint4 qr[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qr[i] = row_ok ? qp[i] : make_uint4(0, 0, 0, 0);
       float down = 1.f;
       if constexpr (!kBf) {
         // the tile's largest |q| (times the channel scale) sets a power-of-two scale that
         // keeps q inside fp16
         float amax = 0.f;
-        if (row_ok) {
-#pragma unroll 4
-          for (int i = 0; i < 8; ++i) {
-            const uint4 u = qp[i];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(kch != nullptr ? elem(u, e) * kch[8 * i + e] : elem(u, e)));
-          }
+        for (int i = 0; i < 8; ++i) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            amax = fmaxf(amax, fabsf(kch != nullptr ? elem(qr[i], e) * kch[8 * i + e] : elem(qr[i], e)));
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -719,12 +735,12 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
         qscale = ldexpf(qscale, eq);
       }
       // 32 columns (16 TMEM columns of 16-bit pairs) at a time
-#pragma unroll 1
+#pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint4 u = row_ok ? qp[4 * hq + i] : make_uint4(0, 0, 0, 0);
+          const uint4 u = qr[4 * hq + i];
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             const int d = 32 * hq + 8 * i + e;
