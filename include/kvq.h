@@ -323,8 +323,13 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* cache, const void* q, int 
  *                 p < context_lens[b], the new one included.
  *   Other arguments as kvq_decode_attention (the workspace size is the same; there is no
  *   seq_ids argument).
- *   Dense caches (INT8, FP8 E4M3, BF16, FP16) with block_size 16 and head_dim 128 only;
- *   other caches return KVQ_ERR_UNSUPPORTED (use kvq_write + kvq_decode_attention).
+ *   Dense caches (INT8, FP8 E4M3, BF16, FP16) with block_size 16 and head_dim 128; and
+ *   INT4 / INT2 caches on the tensor-core path (head_dim 128, 3..8 query heads per kv head)
+ *   whose ring keeps at least one token (residual_len >= 1): there the new row of sequence b
+ *   goes to the residual ring of ring sequence b at position context_lens[b] - 1, as
+ *   kvq_write stores a row that completes no block (a 64-token group that has left the ring
+ *   window still needs kvq_flush_ring before the step).  Other caches return
+ *   KVQ_ERR_UNSUPPORTED (use kvq_write + kvq_decode_attention).
  *   The pages quantize on write and dequantize inside attention ([P-vLLM]
  *   "PagedAttention与KV Cache量化协同工作原理"); doing both in one launch saves a kernel and
  *   its launch per step.  Results equal kvq_write followed by kvq_decode_attention, bit

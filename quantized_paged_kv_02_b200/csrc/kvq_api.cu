@@ -125,8 +125,9 @@ kvq_status decode_entry(const kvq_cache_desc* c, const void* k_new, const void* 
   a.geo = g;
   st = plan_decode(g, batch, num_q_heads, max_context, &a.plan);
   if (st != KVQ_OK) return st;
-  // the append step lives in the tensor-core kernel's producer
-  if (append && a.plan.kernel != 1) return KVQ_ERR_UNSUPPORTED;
+  // the append step lives in the dense tensor-core kernel's producer, or for INT4 / INT2
+  // pages in the ring split (the new position is in the ring when the ring keeps >= 1 token)
+  if (append && a.plan.kernel != 1 && !(a.plan.kernel == 2 && g.residual_len >= 1)) return KVQ_ERR_UNSUPPORTED;
   if (a.plan.ws_bytes > 0) {
     if (workspace == nullptr || workspace_bytes < a.plan.ws_bytes || !aligned16(workspace))
       return KVQ_ERR_INVALID_ARG;

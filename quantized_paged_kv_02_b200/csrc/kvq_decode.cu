@@ -324,6 +324,7 @@ static DecodeParams make_params(const DecodeArgs& a) {
   p.k_new = a.k_new;
   p.v_new = a.v_new;
   p.pages_w = a.k_new != nullptr ? static_cast<uint8_t*>(a.c->pages) : nullptr;
+  p.residual_w = a.k_new != nullptr ? a.c->residual : nullptr;
   p.q_start = a.q_start;
   p.max_q_len = a.max_q_len;
   return p;

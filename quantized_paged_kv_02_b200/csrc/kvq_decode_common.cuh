@@ -37,6 +37,7 @@ struct DecodeParams {
   const void* k_new;
   const void* v_new;
   uint8_t* pages_w;          // the pool, writable (append step only)
+  void* residual_w;          // the INT4 / INT2 ring, writable (append step only)
   // prefill (kvq_prefill_attention): q is [Tq][Hq][D]; the queries of sequence b are rows
   // q_start[b] .. q_start[b+1]-1, the newest tokens of the sequence
   const int32_t* q_start;

@@ -93,6 +93,23 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
   const SeqInfo si = seq_info(p, b, kInt4, blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0);
   const int t0 = ring_only ? si.qb : split * p.chunk;
   const int t1 = ring_only ? si.n : min(si.n, t0 + p.chunk);
+  // append step (INT4 / INT2 with the ring split): this step's row of sequence b is position
+  // n - 1, always in the ring (the ring keeps at least one token); the first head tile of
+  // the (sequence, kv head) stores it there as kvq_write would, and every tile reads it from
+  // k_new / v_new, so no tile depends on another's store
+  const bool app = kInt4 && ring_only && p.k_new != nullptr && si.n > 0;
+  if (app && blockIdx.y % tiles == 0 && warp == 0) {
+    const long slot = (si.n - 1) % p.cap;
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const TA*>(kv ? p.v_new : p.k_new) +
+                                                        (static_cast<long>(b) * p.H + kvh) * D);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<TA*>(p.residual_w) +
+                                            ((static_cast<long>(si.sid) * 2 + kv) * p.H * p.cap +
+                                             static_cast<long>(kvh) * p.cap + slot) * D);
+      for (int i = lane; i < D / 8; i += 32) dst[i] = src[i];
+    }
+  }
 
   // query chunk (pre-multiplied by softmax_scale * log2 e)
   float qf[GT][EPL];
@@ -141,6 +158,10 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
         const long vrow = ((static_cast<long>(si.sid) * 2 + 1) * p.H + kvh) * p.cap + pos % p.cap;
         const TA* kr = static_cast<const TA*>(p.residual) + rrow * D + c * EPL;
         const TA* vr = static_cast<const TA*>(p.residual) + vrow * D + c * EPL;
+        if (app && pos == si.n - 1) {                  // this step's row, from the call
+          kr = static_cast<const TA*>(p.k_new) + (static_cast<long>(b) * p.H + kvh) * D + c * EPL;
+          vr = static_cast<const TA*>(p.v_new) + (static_cast<long>(b) * p.H + kvh) * D + c * EPL;
+        }
 #pragma unroll
         for (int i = 0; i < EPL; i += 8) {
           unpack8<TA>(*reinterpret_cast<const uint4*>(kr + i), &kf[j][i]);

@@ -89,10 +89,55 @@ def test_append_decode_full_size_c5():
     _check(w)
 
 
-def test_append_decode_rejects_unsupported_caches():
-    w = inputs.make("c4", small=True)                  # INT4 KIVI
-    c = helpers.gpu_cache(w)
+@pytest.mark.parametrize("name", ["c4", "c4-tok", "c4-fzp", "c4-int2", "c4-int2-tok"])
+def test_append_decode_low_bit_equals_write_then_decode(name):
+    """INT4 / 2-bit: each sequence's newest row goes to the residual ring in the same call as
+    decode; pages, ring and output equal kvq_write of every row followed by decode, bit for
+    bit (and so the oracle)."""
+    w = inputs.make(name, small=True)
     s = w.spec
+    ref = helpers.gpu_cache(w)
+    fused = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
+                             s.num_kv_heads, s.head_dim, device="cuda",
+                             residual_len=inputs.RESIDUAL_LEN, residual_cap=inputs.RESIDUAL_CAP,
+                             max_seqs=max(s.batch, 1), fill=0x5A)
+    idx, slots, sid, pos = inputs.int4_group_rows(w)
+    starts = w.seq_start.tolist()
+    last = {starts[b + 1] - 1 for b in range(s.batch) if starts[b + 1] > starts[b]}
+    keep = torch.tensor([int(i) not in last for i in idx.tolist()])
+    k, v = w.k.cuda(), w.v.cuda()
+    ki = idx[keep].cuda()
+    fused.write(k[ki].contiguous(), v[ki].contiguous(), slots[keep].cuda(), sid[keep].cuda(),
+                pos[keep].cuda())
+    k_new = torch.zeros((s.batch, s.num_kv_heads, s.head_dim), dtype=w.k.dtype)
+    v_new = torch.zeros_like(k_new)
+    for b in range(s.batch):
+        if starts[b + 1] > starts[b]:
+            k_new[b] = w.k[starts[b + 1] - 1].cpu()
+            v_new[b] = w.v[starts[b + 1] - 1].cpu()
+    q, tab, lens = w.q.cuda(), w.block_tables.cuda(), w.context_lens.cuda()
+    mc = max(w.max_context, 1)
+    want = ref.decode(q, tab, lens, mc)
+    got = fused.append_decode(k_new.cuda(), v_new.cuda(), q, tab, lens, mc)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(helpers.pool_bytes(fused.pages, fused.sizes[1]),
+                                  helpers.pool_bytes(ref.pages, ref.sizes[1]))
+    np.testing.assert_array_equal(helpers.pool_bytes(fused.residual, fused.sizes[3]),
+                                  helpers.pool_bytes(ref.residual, ref.sizes[3]))
+    assert torch.equal(got, want)
+    assert fused.read_fault() == (0, 0)
+    oc = helpers.oracle_cache(w)
+    exact = attention.decode_attention(oc, helpers.np64(w.q), w.block_tables.numpy(),
+                                       w.context_lens.numpy())
+    assert np.abs(got.cpu().numpy().astype(np.float64) - exact).max() <= TOL
+
+
+def test_append_decode_rejects_unsupported_caches():
+    w = inputs.make("c4", small=True)                  # INT4 KIVI with no ring: refused
+    s = w.spec
+    c = kvq.PagedKVCache(s.cache_dtype, s.act_dtype, s.scale_mode, w.num_blocks, s.block_size,
+                         s.num_kv_heads, s.head_dim, device="cuda", residual_len=0,
+                         residual_cap=inputs.RESIDUAL_CAP, max_seqs=max(s.batch, 1))
     k_new = torch.zeros((s.batch, s.num_kv_heads, s.head_dim), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(kvq.KVQError):
         c.append_decode(k_new, k_new, w.q.cuda(), w.block_tables.cuda(), w.context_lens.cuda(),
