@@ -101,13 +101,37 @@ __device__ __forceinline__ int2 sz_offsets(int base, int mt, int r) {
 }
 
 // (code s, code s + 16/BITS) of w -- the codes at the same place in its two 16-bit halves
-// -- as the fp16 bit patterns of code * 2^-24: a 4- or 2-bit code placed in the mantissa of
-// a zero exponent is an exact fp16 subnormal, so the tensor cores see c * 2^-24 with no
-// conversion instruction
+// -- as fp16 bit patterns: a 4- or 2-bit code anywhere in the low ten bits of a half with a
+// zero exponent is an exact fp16 subnormal, c * 2^(BITS pos - 24), so the tensor cores take
+// it with one mask and no conversion.  Codes are masked in place at pos = s % PER and only
+// every PER-th position needs a shifted copy of the word (ws[k] = w >> k SH): 4-bit codes
+// sit at nibble 0 or 1 of a source word (w, w >> 8), 2-bit codes at crumb 0, 1 or 2 (w,
+// w >> 6, w >> 12).  The factor 2^(BITS pos) (1 or 16; 1, 4 or 16) is taken out of the
+// other operand (keys: q'; values: the output rows).
 template <int BITS>
-__device__ __forceinline__ uint32_t code_pair(uint32_t w, int s) {
-  return (w >> (BITS * s)) & Rec<BITS>::kMask;
+struct CodeSel {
+  static constexpr int PER = BITS == 4 ? 2 : 3;       // positions per source word
+  static constexpr int SH = BITS * PER;               // shift between source words
+  static constexpr int NSRC = 16 / BITS / PER + (16 / BITS % PER ? 1 : 0);   // 2 or 3
+  static constexpr int pos(int s) { return s % PER; }
+  // log2 of the factor a code at position s carries
+  static constexpr int lg(int s) { return BITS * (s % PER); }
+};
+
+template <int BITS>
+__device__ __forceinline__ void code_sources(uint32_t w, uint32_t (&ws)[CodeSel<BITS>::NSRC]) {
+#pragma unroll
+  for (int k = 0; k < CodeSel<BITS>::NSRC; ++k) ws[k] = w >> (k * CodeSel<BITS>::SH);
 }
+
+template <int BITS>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&ws)[CodeSel<BITS>::NSRC], int s) {
+  using C = CodeSel<BITS>;
+  return ws[s / C::PER] & (Rec<BITS>::kMask << C::lg(s));
+}
+
+// 2^-e for a small compile-time e
+__host__ __device__ constexpr float inv_pow2(int e) { return e == 0 ? 1.f : 0.5f * inv_pow2(e - 1); }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -126,6 +150,7 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   constexpr int kRowB = R::kRowB, kOffV = R::kOffV, kOffKs = R::kOffKs, kOffKz = R::kOffKz;
   constexpr int kOffVsz = R::kOffVsz, kRec = R::kRec, kRecRows = R::kRecRows;
   constexpr int kStage = R::kStage, kTiles = R::kTiles, PW = R::PW;
+  using CS = CodeSel<BITS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* tiles = smem;
@@ -241,8 +266,10 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     // keep |q * scale| well inside fp16 for channel scales up to ~1000
     const int eq = amax > 0.f ? exponent_of(amax) - 5 : 0;
     const float qdown = pow2i(-eq);
+    // channel e of this lane is code position e % PW of its word, whose in-place code
+    // carries 2^lg: q (and with it q') of that channel is taken down by the same factor
 #pragma unroll
-    for (int e = 0; e < 32; ++e) qv[e] *= qdown;
+    for (int e = 0; e < 32; ++e) qv[e] *= qdown * inv_pow2(CS::lg(e % PW));
     const float qscale = p.scale_log2 * pow2i(eq);
     // keys per token: q's fp16 fragments and per-group sums, the same for every block;
     // k-step kc < 4 covers group 0, kc >= 4 group 1
@@ -257,7 +284,9 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         qt[kc][1] = pack_f16x2(qv[e0 + 1], qv[e0 + PW + 1]);
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qt[kc][0]));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qt[kc][1]));
-        part[kc >> 2] += (f0.x + f0.y) + (f1.x + f1.y);     // what the MMAs multiply
+        // what the MMAs multiply, the in-place factors restored (exact powers of two)
+        part[kc >> 2] += (f0.x + f0.y) * static_cast<float>(1 << CS::lg(e0 % PW)) +
+                         (f1.x + f1.y) * static_cast<float>(1 << CS::lg((e0 + 1) % PW));
       }
 #pragma unroll
       for (int G = 0; G < 2; ++G) {
@@ -341,16 +370,26 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           ql[kc][0] = pack_f16x2(a0 - f0.x, a1 - f0.y);
           ql[kc][1] = pack_f16x2(c0 - f1.x, c1 - f1.y);
         }
-        // integer zero points: ck = sum q' zk (subtracted); float: ck = -sum q mk
-        float corr = 0.f;
+        // integer zero points: ck = sum q' zk (subtracted); float: ck = -sum q mk; q and q'
+        // carry the in-place factors, so the sums are kept per factor and combined after
+        float cp[CS::PER];
+#pragma unroll
+        for (int k = 0; k < CS::PER; ++k) cp[k] = 0.f;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 z = __half22float2(*reinterpret_cast<const __half2*>(&zw[e]));
-          if constexpr (kFz)
-            corr = fmaf(-qv[2 * e], z.x, fmaf(-qv[2 * e + 1], z.y, corr));
-          else
-            corr = fmaf(qs[2 * e], z.x, fmaf(qs[2 * e + 1], z.y, corr));
+          const int k0 = CS::pos((2 * e) % PW), k1 = CS::pos((2 * e + 1) % PW);
+          if constexpr (kFz) {
+            cp[k0] = fmaf(-qv[2 * e], z.x, cp[k0]);
+            cp[k1] = fmaf(-qv[2 * e + 1], z.y, cp[k1]);
+          } else {
+            cp[k0] = fmaf(qs[2 * e], z.x, cp[k0]);
+            cp[k1] = fmaf(qs[2 * e + 1], z.y, cp[k1]);
+          }
         }
+        float corr = cp[0];
+#pragma unroll
+        for (int k = 1; k < CS::PER; ++k) corr = fmaf(cp[k], static_cast<float>(1 << (BITS * k)), corr);
         corr += __shfl_xor_sync(0xffffffffu, corr, 1);
         corr += __shfl_xor_sync(0xffffffffu, corr, 2);
         ck0 = __shfl_sync(0xffffffffu, corr, 8 * j);
@@ -381,11 +420,17 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             w1[1] = *reinterpret_cast<const uint32_t*>(sm + (ko[3] ^ flip));
           }
           float sg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          uint32_t x0[BITS][CS::NSRC], x1[BITS][CS::NSRC];
+#pragma unroll
+          for (int w = 0; w < BITS; ++w) {
+            code_sources<BITS>(w0[w], x0[w]);
+            code_sources<BITS>(w1[w], x1[w]);
+          }
 #pragma unroll
           for (int kc = 0; kc < 8; ++kc) {
             const int w = kc / (PW / 2), sp = 2 * (kc % (PW / 2));
-            const uint32_t a[4] = {code_pair<BITS>(w0[w], sp), code_pair<BITS>(w1[w], sp),
-                                   code_pair<BITS>(w0[w], sp + 1), code_pair<BITS>(w1[w], sp + 1)};
+            const uint32_t a[4] = {code_at<BITS>(x0[w], sp), code_at<BITS>(x1[w], sp),
+                                   code_at<BITS>(x0[w], sp + 1), code_at<BITS>(x1[w], sp + 1)};
             mma_f16(sg[kc >> 2], a, qt[kc]);
           }
           // (scale, zero) of tokens tr0 / tr1, groups 0 and 1: fp16 at kOffKs + 8t + 4G
@@ -419,11 +464,17 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             w1[0] = k1.x; w1[1] = k1.y;
           }
           float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t x0[BITS][CS::NSRC], x1[BITS][CS::NSRC];
+#pragma unroll
+          for (int w = 0; w < BITS; ++w) {
+            code_sources<BITS>(w0[w], x0[w]);
+            code_sources<BITS>(w1[w], x1[w]);
+          }
 #pragma unroll
           for (int kc = 0; kc < 8; ++kc) {
             const int w = kc / (PW / 2), sp = 2 * (kc % (PW / 2));
-            const uint32_t a[4] = {code_pair<BITS>(w0[w], sp), code_pair<BITS>(w1[w], sp),
-                                   code_pair<BITS>(w0[w], sp + 1), code_pair<BITS>(w1[w], sp + 1)};
+            const uint32_t a[4] = {code_at<BITS>(x0[w], sp), code_at<BITS>(x1[w], sp),
+                                   code_at<BITS>(x0[w], sp + 1), code_at<BITS>(x1[w], sp + 1)};
             mma_f16(sa, a, qh[kc]);
             mma_f16(sb, a, ql[kc]);
           }
@@ -550,9 +601,11 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             Z = prmt(vwd[2][G] | (vwd[3][G] << 16), 0u, sel);
             sh = 4 * (md & 1);
           }
+          // codes masked in place: rows r carry 2^sh, rows r + 8 2^(sh + BITS) (undone at
+          // the end; the products and sums are exact power-of-two multiples of the shifted ones)
           constexpr uint32_t m4 = R::kMask;
-          const uint32_t a[4] = {(Y >> sh) & m4, (Y >> (sh + BITS)) & m4, (Z >> sh) & m4,
-                                 (Z >> (sh + BITS)) & m4};
+          const uint32_t a[4] = {Y & (m4 << sh), Y & (m4 << (sh + BITS)), Z & (m4 << sh),
+                                 Z & (m4 << (sh + BITS))};
           mma_f16(o[md], a, pbh[G]);
           mma_f16(o[md], a, pbl[G]);
         }
@@ -573,10 +626,13 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll
     for (int md = 0; md < 8; ++md) {
       const int G = md >> 2;
-      o[md][0] = fmaf(o[md][0], 16777216.f, -cz[G][0]);
-      o[md][1] = fmaf(o[md][1], 16777216.f, -cz[G][1]);
-      o[md][2] = fmaf(o[md][2], 16777216.f, -cz[G][0]);
-      o[md][3] = fmaf(o[md][3], 16777216.f, -cz[G][1]);
+      // 2^24 (the subnormal codes) over the in-place factor of the tile's rows
+      const int sh = BITS == 4 ? 0 : 4 * (md & 1);
+      const float fr = 16777216.f * inv_pow2(sh), fr8 = 16777216.f * inv_pow2(sh + BITS);
+      o[md][0] = fmaf(o[md][0], fr, -cz[G][0]);
+      o[md][1] = fmaf(o[md][1], fr, -cz[G][1]);
+      o[md][2] = fmaf(o[md][2], fr8, -cz[G][0]);
+      o[md][3] = fmaf(o[md][3], fr8, -cz[G][1]);
     }
   }
   __syncthreads();
