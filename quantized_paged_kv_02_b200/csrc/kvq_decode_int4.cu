@@ -395,12 +395,17 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         ck0 = __shfl_sync(0xffffffffu, corr, 8 * j);
         ck1 = __shfl_sync(0xffffffffu, corr, 8 * j + 4);
       }
-#pragma unroll 1
+      // The block's four 16-token tiles in three phases, so that the warp has independent
+      // work in flight: the scores of every tile, one softmax update and one V-scale check
+      // for the block, then P and P V tile by tile.
+      // ------------------------------------------------ S^T = (C - Zk) Q'^T, all tiles
+      // sv[mt][0..3]: tokens 16mt + r (heads 2j, 2j+1) and 16mt + r + 8 (heads 2j, 2j+1)
+      float sv[kBS / 16][4];
+#pragma unroll
       for (int mt = 0; mt < kBS / 16; ++mt) {
         // rows r / r + 8 of the tile: tokens tr0 = 16mt + r and tr1 = tr0 + 8
         const uint8_t* sm = st + R::kTile * mt;
         const int flip = BITS == 2 ? 64 * (mt & 1) : 0;      // 2-bit: odd half-periods
-        // ------------------------------------------------ S^T = (C - Zk) Q'^T
         float s00, s01, s10, s11;
         if constexpr (kTok) {
           // codes of channels [16j, 16j+16) and [64+16j, 64+16j+16): the first BITS/2 words
@@ -483,17 +488,26 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           s10 = fmaf(sa[2] + sb[2], 16777216.f, -ck0) * qscale;
           s11 = fmaf(sa[3] + sb[3], 16777216.f, -ck1) * qscale;
         }
-        // ------------------------------------------------ softmax (log2 domain)
-        const bool grow = s00 > m[0] + kRescale4 || s10 > m[0] + kRescale4 ||
-                          s01 > m[1] + kRescale4 || s11 > m[1] + kRescale4;
-        if (__any_sync(0xffffffffu, grow)) {
-          float tm0 = fmaxf(s00, s10), tm1 = fmaxf(s01, s11);
+        sv[mt][0] = s00;
+        sv[mt][1] = s01;
+        sv[mt][2] = s10;
+        sv[mt][3] = s11;
+      }
+      // ------------------------------------------------ softmax (log2 domain), per block
+      {
+        float mx0 = fmaxf(sv[0][0], sv[0][2]), mx1 = fmaxf(sv[0][1], sv[0][3]);
+#pragma unroll
+        for (int mt = 1; mt < kBS / 16; ++mt) {
+          mx0 = fmaxf(mx0, fmaxf(sv[mt][0], sv[mt][2]));
+          mx1 = fmaxf(mx1, fmaxf(sv[mt][1], sv[mt][3]));
+        }
+        if (__any_sync(0xffffffffu, mx0 > m[0] + kRescale4 || mx1 > m[1] + kRescale4)) {
 #pragma unroll
           for (int off = 4; off < 32; off <<= 1) {
-            tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, off));
-            tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, off));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
           }
-          const float mn0 = fmaxf(m[0], tm0), mn1 = fmaxf(m[1], tm1);
+          const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
           const float c0 = m[0] == -INFINITY ? 0.f : ex2(m[0] - mn0);
           const float c1 = m[1] == -INFINITY ? 0.f : ex2(m[1] - mn1);
           m[0] = mn0;
@@ -509,21 +523,22 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             o[md][3] *= c1;
           }
         }
-        const float base0 = m[0] == -INFINITY ? 0.f : m[0], base1 = m[1] == -INFINITY ? 0.f : m[1];
-        const float p00 = ex2(s00 - base0), p10 = ex2(s10 - base0);
-        const float p01 = ex2(s01 - base1), p11 = ex2(s11 - base1);
-        l[0] += p00 + p10;
-        l[1] += p01 + p11;
-        // ------------------------------------------------ value scales folded into P
-        // vsz for token t, group G: (scale, zero) fp16 at kOffVsz + 8t + 4G
-        const int2 vo2 = sz_offsets(kOffVsz, mt, r);
-        const uint2 vz0 = *reinterpret_cast<const uint2*>(st + vo2.x);
-        const uint2 vz1 = *reinterpret_cast<const uint2*>(st + vo2.y);
-        const uint32_t sz00 = vz0.x, sz01 = vz0.y, sz10 = vz1.x, sz11 = vz1.y;
-        float vs[2][2] = {{__half2float(__ushort_as_half(sz00 & 0xFFFF)), __half2float(__ushort_as_half(sz01 & 0xFFFF))},
-                          {__half2float(__ushort_as_half(sz10 & 0xFFFF)), __half2float(__ushort_as_half(sz11 & 0xFFFF))}};
-        if (__any_sync(0xffffffffu, vs[0][0] >= vlim || vs[0][1] >= vlim || vs[1][0] >= vlim || vs[1][1] >= vlim)) {
-          float vm = fmaxf(fmaxf(vs[0][0], vs[0][1]), fmaxf(vs[1][0], vs[1][1]));
+      }
+      // ------------------------------------------------ value scales of the block
+      // vsz for token t, group G: (scale, zero) fp16 at kOffVsz + 8t + 4G (read again for
+      // each tile below)
+      {
+        float vm = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < kBS / 16; ++mt) {
+          const int2 vo2 = sz_offsets(kOffVsz, mt, r);
+          const uint2 vz0 = *reinterpret_cast<const uint2*>(st + vo2.x);
+          const uint2 vz1 = *reinterpret_cast<const uint2*>(st + vo2.y);
+          const uint32_t w4[4] = {vz0.x, vz0.y, vz1.x, vz1.y};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) vm = fmaxf(vm, __half2float(__ushort_as_half(w4[k] & 0xFFFF)));
+        }
+        if (__any_sync(0xffffffffu, vm >= vlim)) {
 #pragma unroll
           for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
           if (vm > 0.f) {
@@ -543,6 +558,22 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             }
           }
         }
+      }
+      const float base0 = m[0] == -INFINITY ? 0.f : m[0], base1 = m[1] == -INFINITY ? 0.f : m[1];
+#pragma unroll
+      for (int mt = 0; mt < kBS / 16; ++mt) {
+        const uint8_t* sm = st + R::kTile * mt;
+        const int flip = BITS == 2 ? 64 * (mt & 1) : 0;
+        const float p00 = ex2(sv[mt][0] - base0), p10 = ex2(sv[mt][2] - base0);
+        const float p01 = ex2(sv[mt][1] - base1), p11 = ex2(sv[mt][3] - base1);
+        l[0] += p00 + p10;
+        l[1] += p01 + p11;
+        const int2 vo2 = sz_offsets(kOffVsz, mt, r);
+        const uint2 vz0 = *reinterpret_cast<const uint2*>(st + vo2.x);
+        const uint2 vz1 = *reinterpret_cast<const uint2*>(st + vo2.y);
+        const uint32_t sz00 = vz0.x, sz01 = vz0.y, sz10 = vz1.x, sz11 = vz1.y;
+        float vs[2][2] = {{__half2float(__ushort_as_half(sz00 & 0xFFFF)), __half2float(__ushort_as_half(sz01 & 0xFFFF))},
+                          {__half2float(__ushort_as_half(sz10 & 0xFFFF)), __half2float(__ushort_as_half(sz11 & 0xFFFF))}};
         uint32_t pbh[2][2], pbl[2][2];
 #pragma unroll
         for (int G = 0; G < 2; ++G) {
