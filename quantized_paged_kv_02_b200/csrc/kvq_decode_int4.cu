@@ -355,8 +355,9 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&sw[e]));
-          qs[2 * e] = qv[2 * e] * f.x;
-          qs[2 * e + 1] = qv[2 * e + 1] * f.y;
+          const float2 q2 = __fmul2_rn(make_float2(qv[2 * e], qv[2 * e + 1]), f);
+          qs[2 * e] = q2.x;
+          qs[2 * e + 1] = q2.y;
         }
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
@@ -367,8 +368,10 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
           qh[kc][0] = h0;
           qh[kc][1] = h1;
-          ql[kc][0] = pack_f16x2(a0 - f0.x, a1 - f0.y);
-          ql[kc][1] = pack_f16x2(c0 - f1.x, c1 - f1.y);
+          const float2 r0 = __fadd2_rn(make_float2(a0, a1), make_float2(-f0.x, -f0.y));
+          const float2 r1 = __fadd2_rn(make_float2(c0, c1), make_float2(-f1.x, -f1.y));
+          ql[kc][0] = pack_f16x2(r0.x, r0.y);
+          ql[kc][1] = pack_f16x2(r1.x, r1.y);
         }
         // integer zero points: ck = sum q' zk (subtracted); float: ck = -sum q mk; q and q'
         // carry the in-place factors, so the sums are kept per factor and combined after
@@ -483,10 +486,16 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             mma_f16(sa, a, qh[kc]);
             mma_f16(sb, a, ql[kc]);
           }
-          s00 = fmaf(sa[0] + sb[0], 16777216.f, -ck0) * qscale;
-          s01 = fmaf(sa[1] + sb[1], 16777216.f, -ck1) * qscale;
-          s10 = fmaf(sa[2] + sb[2], 16777216.f, -ck0) * qscale;
-          s11 = fmaf(sa[3] + sb[3], 16777216.f, -ck1) * qscale;
+          const float2 two24 = make_float2(16777216.f, 16777216.f), nck = make_float2(-ck0, -ck1);
+          const float2 qsc2 = make_float2(qscale, qscale);
+          const float2 t0 = __fmul2_rn(__ffma2_rn(__fadd2_rn(make_float2(sa[0], sa[1]), make_float2(sb[0], sb[1])),
+                                                  two24, nck), qsc2);
+          const float2 t1 = __fmul2_rn(__ffma2_rn(__fadd2_rn(make_float2(sa[2], sa[3]), make_float2(sb[2], sb[3])),
+                                                  two24, nck), qsc2);
+          s00 = t0.x;
+          s01 = t0.y;
+          s10 = t1.x;
+          s11 = t1.y;
         }
         sv[mt][0] = s00;
         sv[mt][1] = s01;
@@ -528,7 +537,8 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       // vsz for token t, group G: (scale, zero) fp16 at kOffVsz + 8t + 4G (read again for
       // each tile below)
       {
-        float vm = 0.f;
+        // the largest scale by packed half maxima (the high halves, zero points, unused)
+        __half2 vm2 = __halves2half2(__ushort_as_half(0), __ushort_as_half(0));
 #pragma unroll
         for (int mt = 0; mt < kBS / 16; ++mt) {
           const int2 vo2 = sz_offsets(kOffVsz, mt, r);
@@ -536,8 +546,9 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           const uint2 vz1 = *reinterpret_cast<const uint2*>(st + vo2.y);
           const uint32_t w4[4] = {vz0.x, vz0.y, vz1.x, vz1.y};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) vm = fmaxf(vm, __half2float(__ushort_as_half(w4[k] & 0xFFFF)));
+          for (int k = 0; k < 4; ++k) vm2 = __hmax2(vm2, *reinterpret_cast<const __half2*>(&w4[k]));
         }
+        float vm = __low2float(vm2);
         if (__any_sync(0xffffffffu, vm >= vlim)) {
 #pragma unroll
           for (int off = 4; off < 32; off <<= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
@@ -564,10 +575,16 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       for (int mt = 0; mt < kBS / 16; ++mt) {
         const uint8_t* sm = st + R::kTile * mt;
         const int flip = BITS == 2 ? 64 * (mt & 1) : 0;
-        const float p00 = ex2(sv[mt][0] - base0), p10 = ex2(sv[mt][2] - base0);
-        const float p01 = ex2(sv[mt][1] - base1), p11 = ex2(sv[mt][3] - base1);
-        l[0] += p00 + p10;
-        l[1] += p01 + p11;
+        const float2 nb = make_float2(-base0, -base1);
+        const float2 x0 = __fadd2_rn(make_float2(sv[mt][0], sv[mt][1]), nb);
+        const float2 x1 = __fadd2_rn(make_float2(sv[mt][2], sv[mt][3]), nb);
+        const float p00 = ex2(x0.x), p01 = ex2(x0.y), p10 = ex2(x1.x), p11 = ex2(x1.y);
+        {
+          const float2 l2 = __fadd2_rn(make_float2(l[0], l[1]),
+                                       __fadd2_rn(make_float2(p00, p01), make_float2(p10, p11)));
+          l[0] = l2.x;
+          l[1] = l2.y;
+        }
         const int2 vo2 = sz_offsets(kOffVsz, mt, r);
         const uint2 vz0 = *reinterpret_cast<const uint2*>(st + vo2.x);
         const uint2 vz1 = *reinterpret_cast<const uint2*>(st + vo2.y);
@@ -578,21 +595,28 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll
         for (int G = 0; G < 2; ++G) {
           const float w0g = vs[0][G] * vinv, w1g = vs[1][G] * vinv;
-          const float q00 = p00 * w0g, q01 = p01 * w0g, q10 = p10 * w1g, q11 = p11 * w1g;
+          // (q00, q01): token tr0, heads 2j / 2j+1; (q10, q11): token tr1
+          const float2 qa = __fmul2_rn(make_float2(p00, p01), make_float2(w0g, w0g));
+          const float2 qb = __fmul2_rn(make_float2(p10, p11), make_float2(w1g, w1g));
           const float z0 = __half2float(__ushort_as_half((G ? sz01 : sz00) >> 16));
           const float z1 = __half2float(__ushort_as_half((G ? sz11 : sz10) >> 16));
+          float2 c2 = make_float2(cz[G][0], cz[G][1]);
           if constexpr (kFz) {
             // the minima enter unscaled: cz = -vinv * sum_t p mv
-            cz[G][0] = fmaf(-p00 * vinv, z0, fmaf(-p10 * vinv, z1, cz[G][0]));
-            cz[G][1] = fmaf(-p01 * vinv, z0, fmaf(-p11 * vinv, z1, cz[G][1]));
+            const float nz0 = -vinv * z0, nz1 = -vinv * z1;
+            c2 = __ffma2_rn(make_float2(p00, p01), make_float2(nz0, nz0),
+                            __ffma2_rn(make_float2(p10, p11), make_float2(nz1, nz1), c2));
           } else {
-            cz[G][0] = fmaf(q00, z0, fmaf(q10, z1, cz[G][0]));
-            cz[G][1] = fmaf(q01, z0, fmaf(q11, z1, cz[G][1]));
+            c2 = __ffma2_rn(qa, make_float2(z0, z0), __ffma2_rn(qb, make_float2(z1, z1), c2));
           }
-          const uint32_t h0 = pack_f16x2(q00, q01), h1 = pack_f16x2(q10, q11);
+          cz[G][0] = c2.x;
+          cz[G][1] = c2.y;
+          const uint32_t h0 = pack_f16x2(qa.x, qa.y), h1 = pack_f16x2(qb.x, qb.y);
           const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
           const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-          const uint32_t e0 = pack_f16x2(q00 - f0.x, q01 - f0.y), e1 = pack_f16x2(q10 - f1.x, q11 - f1.y);
+          const float2 d0 = __fadd2_rn(qa, make_float2(-f0.x, -f0.y));
+          const float2 d1 = __fadd2_rn(qb, make_float2(-f1.x, -f1.y));
+          const uint32_t e0 = pack_f16x2(d0.x, d0.y), e1 = pack_f16x2(d1.x, d1.y);
           pbh[G][0] = movmatrix_trans(h0);
           pbh[G][1] = movmatrix_trans(h1);
           pbl[G][0] = movmatrix_trans(e0);
