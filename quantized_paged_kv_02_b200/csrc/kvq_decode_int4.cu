@@ -78,7 +78,10 @@ struct Rec {
   static constexpr int kStage = kRec;                  // a multiple of 1024
   static constexpr int kTile = 16 * kRowB;             // 16 tokens of codes: 1024 or 512 bytes
   static constexpr int kTiles = kStages * kStage;
-  static constexpr int kBytes = 1024 + kTiles + kStages * 16 + kStages * 4;
+  // each consumer lane's 32 q values (KIVI forms: read once per block for the key-scale
+  // fold, so they need not stay in registers)
+  static constexpr int kQv = kC * 32 * 32 * 4;
+  static constexpr int kBytes = 1024 + kTiles + kQv + kStages * 16 + kStages * 4;
   static constexpr int PW = 16 / BITS;                 // codes in each 16-bit half of a word
   static constexpr uint32_t kMask = BITS == 4 ? 0x000F000Fu : 0x00030003u;
   static_assert(kStage % 1024 == 0, "stages start on the swizzle period");
@@ -154,7 +157,8 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTiles);
+  float4* qvs = reinterpret_cast<float4*>(smem + kTiles);   // [warp][8][lane]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTiles + R::kQv);
   uint64_t* empty = full + kStages;
   int* valid = reinterpret_cast<int*>(empty + kStages);
 
@@ -270,6 +274,12 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     // carries 2^lg: q (and with it q') of that channel is taken down by the same factor
 #pragma unroll
     for (int e = 0; e < 32; ++e) qv[e] *= qdown * inv_pow2(CS::lg(e % PW));
+    if constexpr (!kTok) {
+      // kept in shared memory for the per-block fold (conflict-free: lane-consecutive)
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        qvs[(warp * 8 + c) * 32 + lane] = make_float4(qv[4 * c], qv[4 * c + 1], qv[4 * c + 2], qv[4 * c + 3]);
+    }
     const float qscale = p.scale_log2 * pow2i(eq);
     // keys per token: q's fp16 fragments and per-group sums, the same for every block;
     // k-step kc < 4 covers group 0, kc >= 4 group 1
@@ -351,11 +361,20 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           sw[4 * c] = a.x; sw[4 * c + 1] = a.y; sw[4 * c + 2] = a.z; sw[4 * c + 3] = a.w;
           zw[4 * c] = z.x; zw[4 * c + 1] = z.y; zw[4 * c + 2] = z.z; zw[4 * c + 3] = z.w;
         }
+        float qq[32];                   // this lane's q, as stored above
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 v4 = qvs[(warp * 8 + c) * 32 + lane];
+          qq[4 * c] = v4.x;
+          qq[4 * c + 1] = v4.y;
+          qq[4 * c + 2] = v4.z;
+          qq[4 * c + 3] = v4.w;
+        }
         float qs[32];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&sw[e]));
-          const float2 q2 = __fmul2_rn(make_float2(qv[2 * e], qv[2 * e + 1]), f);
+          const float2 q2 = __fmul2_rn(make_float2(qq[2 * e], qq[2 * e + 1]), f);
           qs[2 * e] = q2.x;
           qs[2 * e + 1] = q2.y;
         }
@@ -383,8 +402,8 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           const float2 z = __half22float2(*reinterpret_cast<const __half2*>(&zw[e]));
           const int k0 = CS::pos((2 * e) % PW), k1 = CS::pos((2 * e + 1) % PW);
           if constexpr (kFz) {
-            cp[k0] = fmaf(-qv[2 * e], z.x, cp[k0]);
-            cp[k1] = fmaf(-qv[2 * e + 1], z.y, cp[k1]);
+            cp[k0] = fmaf(-qq[2 * e], z.x, cp[k0]);
+            cp[k1] = fmaf(-qq[2 * e + 1], z.y, cp[k1]);
           } else {
             cp[k0] = fmaf(qs[2 * e], z.x, cp[k0]);
             cp[k1] = fmaf(qs[2 * e + 1], z.y, cp[k1]);
