@@ -26,6 +26,9 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
   const int S = (p.ring_split >= 0 ? si.qb + p.chunk - 1 : si.n + p.chunk - 1) / p.chunk;
   const bool ring = p.ring_split >= 0 && si.n > si.qb;
   const int K = S + (ring ? 1 : 0);
+  // the split count depends only on the call's inputs; the partials are read after the
+  // decode kernels are done (the last of them waits for the one before it)
+  griddep_wait();
   const float* ml = p.ws_ml + static_cast<long>(row) * p.splits * 2;
   const float* o = p.ws_o + static_cast<long>(row) * p.splits * p.D;
   auto slot = [&](int k) { return k < S ? k : p.ring_split; };
@@ -336,8 +339,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.batch == 0) return cudaSuccess;
   cudaError_t e;
   if (a.plan.kernel == 2) {
-    e = launch_decode_int4(a, p, s);                 // block splits
-    if (e == cudaSuccess) e = launch_decode_simt(a, p, s);   // ring split
+    // the ring split first: its kernel is small and releases its dependents as it starts,
+    // so the block splits (launched as its dependent, reading nothing it writes) overlap it
+    e = launch_decode_simt(a, p, s);                 // ring split
+    if (e == cudaSuccess) e = launch_decode_int4(a, p, s);   // block splits
   } else {
     e = a.plan.kernel == 1 ? launch_decode_mma(a, p, s) : launch_decode_simt(a, p, s);
   }
@@ -345,8 +350,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.plan.kernel == 1) {
     e = launch_dependent(segment_reduce_kernel, dim3((a.batch * a.Hq + 7) / 8), dim3(256), 0, s, p);
   } else if (p.splits > 1) {
-    split_reduce_kernel<<<(a.batch * a.Hq + 7) / 8, 256, 0, s>>>(p, low_bit(g.cache_dtype));
-    e = cudaGetLastError();
+    e = launch_dependent(split_reduce_kernel, dim3((a.batch * a.Hq + 7) / 8), dim3(256), 0, s, p,
+                         low_bit(g.cache_dtype));
   }
   return e;
 }

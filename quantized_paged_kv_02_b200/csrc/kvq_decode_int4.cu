@@ -710,6 +710,7 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
   }
   __syncthreads();
+  griddep_launch_dependents();   // the split reduce may be scheduled (it waits for this grid)
 
   float* red_o = reinterpret_cast<float*>(tiles);           // [warp][head][D]
   float* red_ml = red_o + kC * 8 * kD;                      // [warp][head][2]
@@ -746,6 +747,9 @@ decode_int4_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
     store_partial_or_output(p, b, kvh * p.g + h, split, d, M, Lsum, O);
   }
+  // launched as the ring kernel's dependent: this grid completes only after that one, so the
+  // split reduce (this grid's dependent, waiting for it) sees both kernels' partials
+  griddep_wait();
 }
 
 }  // namespace
@@ -783,12 +787,14 @@ cudaError_t launch_bits(const DecodeArgs& a, const DecodeParams& p, cudaStream_t
   // page splits only; the ring split is launched separately
   const dim3 grid(p.ring_split, a.geo.H, a.batch);
   switch (a.geo.scale_mode) {
-    case KVQ_SCALE_KIVI: decode_int4_kernel<kKivi, BITS><<<grid, kT, R::kBytes, s>>>(p, tm); break;
-    case KVQ_SCALE_KIVI_FLOAT_ZERO: decode_int4_kernel<kKiviMin, BITS><<<grid, kT, R::kBytes, s>>>(p, tm); break;
-    case KVQ_SCALE_INT4_PER_TOKEN: decode_int4_kernel<kPerToken, BITS><<<grid, kT, R::kBytes, s>>>(p, tm); break;
+    // launched as the ring kernel's dependent (see the kernel's last lines)
+    case KVQ_SCALE_KIVI: return launch_dependent(decode_int4_kernel<kKivi, BITS>, grid, dim3(kT), R::kBytes, s, p, tm);
+    case KVQ_SCALE_KIVI_FLOAT_ZERO:
+      return launch_dependent(decode_int4_kernel<kKiviMin, BITS>, grid, dim3(kT), R::kBytes, s, p, tm);
+    case KVQ_SCALE_INT4_PER_TOKEN:
+      return launch_dependent(decode_int4_kernel<kPerToken, BITS>, grid, dim3(kT), R::kBytes, s, p, tm);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace

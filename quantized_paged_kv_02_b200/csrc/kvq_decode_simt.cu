@@ -19,6 +19,7 @@
 // HBM bandwidth when the ALUs keep up (small GQA groups).
 #include "kvq_internal.cuh"
 #include "kvq_decode_common.cuh"
+#include "kvq_ptx.cuh"
 
 namespace kvq {
 namespace {
@@ -80,6 +81,9 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(DecodeParams p) {
   constexpr bool kInt4 = CD == KVQ_DTYPE_INT4 || CD == KVQ_DTYPE_INT2;   // group codes + ring
   constexpr int ROWB = D * CB / EPL;    // bytes per cache row
 
+  // a kernel launched after this one as its dependent may start at once (the INT4 / INT2
+  // block kernel, which reads nothing this one writes, or the split reduce, which waits)
+  griddep_launch_dependents();
   // ring-only launch (INT4 blocks on tensor cores): this grid covers [qb, n) from the ring
   const bool ring_only = p.ring_split >= 0;
   const int split = ring_only ? p.ring_split : blockIdx.x;
