@@ -32,6 +32,17 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
   const float* ml = p.ws_ml + static_cast<long>(row) * p.splits * 2;
   const float* o = p.ws_o + static_cast<long>(row) * p.splits * p.D;
   auto slot = [&](int k) { return k < S ? k : p.ring_split; };
+  const bool has_d = 4 * lane < p.D;
+  auto row_of = [&](int k) {          // this lane's 4 channels of partial k (0 past the list)
+    return (has_d && k < K) ? *reinterpret_cast<const float4*>(o + static_cast<long>(slot(k)) * p.D + 4 * lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  // every listed split holds work and every partial row is read, so the first sixteen rows
+  // are loaded together with the (max, sum) pairs rather than after the weights
+  constexpr int kB = 16;
+  float4 v[kB];
+#pragma unroll
+  for (int t = 0; t < kB; ++t) v[t] = row_of(t);
   // max over the splits
   float M = -INFINITY;
   for (int k = lane; k < K; k += 32) M = fmaxf(M, ml[2 * slot(k)]);
@@ -39,7 +50,6 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const bool has_d = 4 * lane < p.D;
   for (int k0 = 0; k0 < K; k0 += 32) {
     const int k = k0 + lane;
     float w = 0.f;
@@ -49,14 +59,18 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(DecodeParams p, bool 
       L = fmaf(ml[2 * slot(k) + 1], w, L);
     }
     const int n = min(32, K - k0);
-    for (int i = 0; i < n; ++i) {
-      const float wi = __shfl_sync(0xffffffffu, w, i);
-      if (has_d) {
-        const float4 v = *reinterpret_cast<const float4*>(o + static_cast<long>(slot(k0 + i)) * p.D + 4 * lane);
-        acc.x = fmaf(v.x, wi, acc.x);
-        acc.y = fmaf(v.y, wi, acc.y);
-        acc.z = fmaf(v.z, wi, acc.z);
-        acc.w = fmaf(v.w, wi, acc.w);
+    for (int i0 = 0; i0 < n; i0 += kB) {
+      if (k0 + i0 > 0) {
+#pragma unroll
+        for (int t = 0; t < kB; ++t) v[t] = row_of(k0 + i0 + t);
+      }
+#pragma unroll
+      for (int t = 0; t < kB; ++t) {
+        const float wi = __shfl_sync(0xffffffffu, w, i0 + t);   // 0 past the list
+        acc.x = fmaf(v[t].x, wi, acc.x);
+        acc.y = fmaf(v[t].y, wi, acc.y);
+        acc.z = fmaf(v[t].z, wi, acc.z);
+        acc.w = fmaf(v[t].w, wi, acc.w);
       }
     }
   }
