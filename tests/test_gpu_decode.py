@@ -228,3 +228,42 @@ def test_int4_tensor_core_path_partial_groups(cd, mode, hq):
     got = _decode(gc, w).cpu().numpy().astype(np.float64)
     assert np.abs(got - _oracle(oc, w)).max() <= TOL
     assert gc.read_fault() == (0, 0)
+
+
+@pytest.mark.parametrize("name", ["c4", "c4-int2", "c4-tok", "c5", "c3"])
+def test_back_to_back_calls_share_a_workspace(name):
+    """Calls enqueued back to back on one workspace, with no host synchronization between
+    them, give exactly what each gives alone.  Within a call the kernels overlap (the
+    low-bit block kernel runs beside the ring-split kernel, the merges start early and
+    wait); a call's first kernel starts only after the previous call's last one, so no
+    call reads partials another call is writing.  The second call decodes a subset of the
+    batch with other queries, so its partial rows land on the first call's slots."""
+    w = _workload(name)
+    static = helpers.oracle_static_scales(w)
+    gc = helpers.gpu_cache(w, static=static)
+    B = w.spec.batch
+    half = max(1, B // 2)
+    q1 = w.q.cuda()
+    g = torch.Generator().manual_seed(1234)
+    q2 = torch.randn(w.q[:half].shape, generator=g).to(w.q.dtype).cuda()
+    tab, lens = w.block_tables.cuda(), w.context_lens.cuda()
+    mc = int(w.context_lens.max())
+    n = max(gc.workspace_size(B, q1.shape[1], mc), gc.workspace_size(half, q1.shape[1], mc), 16)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    # each call alone, synchronized
+    a1 = gc.decode(q1, tab, lens, mc, workspace=ws)
+    torch.cuda.synchronize()
+    a1 = a1.clone()
+    a2 = gc.decode(q2, tab[:half], lens[:half], mc, workspace=ws)
+    torch.cuda.synchronize()
+    a2 = a2.clone()
+    # the same calls enqueued back to back, three rounds
+    outs = []
+    for _ in range(3):
+        outs.append(gc.decode(q1, tab, lens, mc, workspace=ws))
+        outs.append(gc.decode(q2, tab[:half], lens[:half], mc, workspace=ws))
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        want = a1 if i % 2 == 0 else a2
+        assert torch.equal(o, want), (name, i)
+    assert gc.read_fault() == (0, 0)
