@@ -154,5 +154,8 @@ bool int4_mma_supported(const Geometry& g, int group);
 cudaError_t launch_decode_int4(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s);
 // Tensor map over the pages pool viewed as rows of 128 bytes; one box = one record.
 bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows);
+// Tensor map over `rows` rows of `row_bytes` bytes; one box is 128 bytes of `box_rows`
+// consecutive rows, copied with 128-byte swizzle (the tensor cores' tile layout).
+bool make_rows_map(CUtensorMap* map, const void* base, long rows, int row_bytes, int box_rows);
 
 }  // namespace kvq

@@ -875,6 +875,19 @@ bool make_pages_map(CUtensorMap* map, const void* base, long rows, int rec_rows)
   return res == CUDA_SUCCESS;
 }
 
+bool make_rows_map(CUtensorMap* map, const void* base, long rows, int row_bytes, int box_rows) {
+  auto enc = encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                           box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
+}
+
 bool mma_supported(const Geometry& g, int groups) {
   // any group of 1..8 query heads fills (part of) the N = 8 side of the tiles; the kernel
   // is bound by moving pages, so a partly empty tile costs little

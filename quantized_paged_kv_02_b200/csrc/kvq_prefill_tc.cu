@@ -59,7 +59,8 @@ constexpr int kD = 128;
 constexpr int kPfThreads = 576;     // warps 0-7 softmax, 8 producer, 9 MMA, 10-13 K converters,
                                     // 14-17 V converters
 constexpr int kSoftWarps = 8, kProdWarp = 8, kMmaWarp = 9, kConvWarp0 = 10;
-constexpr int kNB = 2;              // K / V tile buffers
+constexpr int kNB = 2;              // K / V tile buffers (raw ring caches)
+constexpr int kNBMax = 3;           // ... at most (16-bit caches, no raw ring: three)
 constexpr int kNQ = 4;              // slots of the per-token K multipliers (block j: slot j % 4)
 constexpr int kTile = 32768;        // 128 x 128 16-bit elements
 constexpr float kRescalePf = 8.f;   // log2 headroom before the running max is re-based
@@ -91,33 +92,39 @@ struct PfLayout {
   static constexpr int REC = (OFF_S + SCALES + 127) / 128 * 128;
   static constexpr int KP = LB ? 2 : 1;                    // K tiles whose sum is K (hi, lo)
   static constexpr int VP = LB ? 2 : 1;
-  static constexpr int NB = LB ? 1 : kNB;                  // K / V tile buffers
+  static constexpr int NB = LB ? 1 : (BITS == 16 ? 3 : kNB);   // K / V tile buffers
   static constexpr int RS = LB ? 4 : (BITS == 8 ? 16 : 8); // raw ring stages (pages)
   // the ring turns over in groups of one block's pages, each group with one full and one
   // empty barrier: the producer issues a block's pages together and the converters wait
   // once per block
   static constexpr int RG = RS / PPB;
+  // 16-bit caches: the rows are the tiles' values, so the producer copies them with TMA
+  // straight into the tile buffers (128-byte swizzle) and no raw ring is needed
+  static constexpr bool DIRECT = BITS == 16;
+  static constexpr int RAWB = DIRECT ? 0 : RS * REC;       // bytes of the raw ring
+  static constexpr int NPOK = DIRECT ? NB * PPB : RS;      // page-valid flags: by ring slot,
+                                                           // or by (tile buffer, page)
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = NB * KP * kTile;
   static constexpr int RAW_OFF = V_OFF + NB * VP * kTile;
-  static constexpr int KQ_OFF = RAW_OFF + RS * REC;        // float [kNQ][128]: K multiplier
+  static constexpr int KQ_OFF = RAW_OFF + RAWB;            // float [kNQ][128]: K multiplier
   static constexpr int VS_OFF = KQ_OFF + kNQ * kBlk * 4;   // float [NB][128]: V scale
   static constexpr int XM_OFF = VS_OFF + NB * kBlk * 4;    // float [3][2][128]: row maxima of
                                                            // the two halves (by block parity),
                                                            // then the row sums
   static constexpr int MISC_OFF = XM_OFF + 3 * 2 * kRows * 4;  // per (buffer, converter warp)
                                                                // vmax and bad-token counts; flags
-  static constexpr int BAR_OFF = MISC_OFF + 160;
+  static constexpr int BAR_OFF = MISC_OFF + 192;
   // raw_full, raw_empty [RG]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
-  // q_ready; fin; xch [4]; kq_full, kqfree [kNQ]
-  static constexpr int NBARS = 2 * RG + 3 * NB + 6 + 2 + 4 + 2 * kNQ;
-  static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + RS * 4 + 64;
+  // q_ready; fin; xch [4]; kq_full, kqfree [kNQ]; tile_full [NB] (16-bit caches)
+  static constexpr int NBARS = 2 * RG + 3 * NB + 6 + 2 + 4 + 2 * kNQ + NB;
+  static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + NPOK * 4 + 64;
   static_assert(BYTES <= 227 * 1024, "fits the shared memory of one CTA");
   static_assert(BYTES > 114 * 1024, "one CTA per SM, so TMEM allocation never waits on a peer");
   static_assert(RS % PPB == 0 && RG >= 1, "the raw ring holds whole blocks");
   static_assert(PPB <= 32, "one producer lane per page of a block");
   static_assert(REC % 16 == 0, "bulk copies move multiples of 16 bytes");
-  static_assert(NB <= kNB, "scale arrays");
+  static_assert(NB <= kNBMax, "scale arrays");
 };
 
 struct PfShared {
@@ -134,6 +141,7 @@ struct PfShared {
   uint64_t* xch;                    // [4]: the two softmax warps of a TMEM lane quarter
   uint64_t* kq_full;                // [kNQ]: a slot of K multipliers (and bad-token counts) written
   uint64_t* kqfree;                 // [kNQ]: the softmax is done with a slot of K multipliers
+  uint64_t* tile_full;              // [NB]: 16-bit caches: a block's K and V rows have landed
   float* xmax;
   int* page_ok;
   float* kq;                        // [NB][128] K multiplier of each token (NaN: bad page)
@@ -315,9 +323,42 @@ __device__ __forceinline__ float dense_part(uint8_t* smem, const PfShared& sh, i
   return vv;
 }
 
+// 16-bit caches, thread ct = token ct of block j, whose rows the producer copied into tile
+// buffer kb: K: the token's multiplier (softmax scale, NaN for a bad page, 0 past the
+// window); V: its scale (1 or 0) and, for a token outside the window or on a page that was
+// not copied, zeros over its row of the V tile (whatever the buffer held must not reach
+// P V; a masked score never does).  Returns as dense_part.
+template <int CD, bool PT>
+__device__ __forceinline__ float direct_part(uint8_t* smem, const PfShared& sh, int j, int kb, bool isv,
+                                             int ct, int npg, int pmax, float& qsc, bool& have_q) {
+  using L = PfLayout<CD, PT>;
+  constexpr int BS = L::BS;
+  const int t = ct, pp = t / BS, k = j * L::PPB + pp, pos = j * kBlk + t;
+  const bool have = k < npg, pk = have && sh.page_ok[kb * L::PPB + pp];
+  const bool valid = pk && pos <= pmax;
+  if (!isv) {
+    if (!have_q) {
+      if (pf_wait(sh.q_ready, 0, sh.abort)) qsc = *sh.qscale;
+      else *sh.abort = 1;
+      have_q = true;
+    }
+    const bool badtok = have && !pk && pos <= pmax;
+    sh.kq[(j % kNQ) * kBlk + t] = valid ? qsc : (badtok ? __uint_as_float(0x7fffffffu) : 0.f);
+    return badtok ? 1.f : 0.f;
+  }
+  if (!valid) {
+    uint8_t* tile = smem + L::V_OFF + kb * kTile;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) *reinterpret_cast<uint4*>(tile + tile_off(t, c)) = make_uint4(0, 0, 0, 0);
+  }
+  const float vv = valid ? 1.f : 0.f;
+  sh.vs[kb * kBlk + t] = vv;
+  return vv;
+}
+
 template <int CD, bool PT, int QP>
 __global__ void __launch_bounds__(kPfThreads, 1)
-prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
+prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap rows) {
   using L = PfLayout<CD, PT>;
   constexpr bool kBf = PfCode<CD>::kBf16;
   constexpr int BS = L::BS, NB = L::NB;
@@ -359,16 +400,17 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
   sh.xch = sh.fin + 1;
   sh.kq_full = sh.xch + 4;
   sh.kqfree = sh.kq_full + kNQ;
+  sh.tile_full = sh.kqfree + kNQ;
   sh.xmax = reinterpret_cast<float*>(smem + L::XM_OFF);
   sh.page_ok = reinterpret_cast<int*>(bars + L::NBARS);
   sh.kq = reinterpret_cast<float*>(smem + L::KQ_OFF);
   sh.vs = reinterpret_cast<float*>(smem + L::VS_OFF);
-  sh.vmax = reinterpret_cast<float*>(smem + L::MISC_OFF);            // [kNB][4]
-  sh.nbad = reinterpret_cast<int*>(smem + L::MISC_OFF + 32);         // [kNQ][4]
-  sh.qscale = reinterpret_cast<float*>(smem + L::MISC_OFF + 96);
-  sh.tmem = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF + 100);
-  sh.abort = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 104);
-  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 112);  // [8] softmax amax
+  sh.vmax = reinterpret_cast<float*>(smem + L::MISC_OFF);            // [kNBMax][4]
+  sh.nbad = reinterpret_cast<int*>(smem + L::MISC_OFF + 48);         // [kNQ][4]
+  sh.qscale = reinterpret_cast<float*>(smem + L::MISC_OFF + 112);
+  sh.tmem = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF + 116);
+  sh.abort = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 120);
+  float* red = reinterpret_cast<float*>(smem + L::MISC_OFF + 128);  // [8] softmax amax
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::RG; ++s) {
@@ -392,6 +434,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       mbar_init(&sh.kq_full[k], 4);
       mbar_init(&sh.kqfree[k], kSoftWarps);
     }
+    for (int k = 0; k < NB; ++k) mbar_init(&sh.tile_full[k], 1);
     *sh.abort = 0;
     fence_mbar_init();
   }
@@ -409,7 +452,53 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
     const int nblk = (npg + L::PPB - 1) / L::PPB;          // blocks with pages to copy
     bool ok_run = true;
     int jb = 0;
-    for (; jb < nblk && ok_run; ++jb) {
+    if constexpr (L::DIRECT) {
+      // 16-bit rows go straight into tile buffer kb = jb % NB: K rows (16 of a page) as the
+      // two 128-byte halves of the K tile's rows, V rows likewise; a buffer is refilled once
+      // S of block jb - NB (K) and P V of block jb - NB (V) have read it
+      for (; jb < nblk && ok_run; ++jb) {
+        const int kb = jb % NB;
+        const int k = jb * L::PPB + lane;
+        const bool mine = lane < L::PPB && k < npg;
+        const int blk = mine ? p.tables[static_cast<long>(b) * p.max_blocks + k] : -1;
+        bool ok_lane = true;
+        if (lane == 0 && jb >= NB) {
+          if (!pf_wait(&sh.s_full[(jb - NB) & 1], ((jb - NB) >> 1) & 1, sh.abort) ||
+              !pf_wait(&sh.vfree[kb], ((jb / NB) - 1) & 1, sh.abort))
+            ok_lane = false;
+        }
+        ok_run = __all_sync(0xffffffffu, ok_lane);
+        if (!ok_run) {
+          if (lane == 0) pf_fail(p, sh.abort);
+          break;
+        }
+        bool valid = false;
+        if (mine) {
+          valid = blk >= 0 && blk < p.NB;
+          sh.page_ok[kb * L::PPB + lane] = valid;
+          if (!valid) record_fault(p.fault, KVQ_FAULT_BLOCK);
+        }
+        const unsigned nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+        if (lane == 0) mbar_arrive_expect_tx(&sh.tile_full[kb], nvalid * L::REC);
+        __syncwarp();
+        if (valid) {
+          // the record's 32 rows of 256 bytes: K rows 0..15, V rows 16..31
+          const int y = (blk * p.H + kvh) * (2 * BS);
+          const int r0 = lane * BS * 128;                  // page lane's rows in a tile half
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            tma_load_2d(smem + L::K_OFF + kb * kTile + hh * 16384 + r0, &rows, &sh.tile_full[kb], 128 * hh, y);
+            tma_load_2d(smem + L::V_OFF + kb * kTile + hh * 16384 + r0, &rows, &sh.tile_full[kb], 128 * hh, y + BS);
+          }
+        }
+      }
+      // every copy issued must land before the CTA may exit
+      if (lane == 0) {
+        for (int j2 = max(0, jb - NB); j2 < jb; ++j2)
+          if (!mbar_drain(&sh.tile_full[j2 % NB], (j2 / NB) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
+      }
+    }
+    for (; !L::DIRECT && jb < nblk && ok_run; ++jb) {
       const int grp = jb % L::RG, round = jb / L::RG;
       const int k = jb * L::PPB + lane, s = k % L::RS;
       // the table entries are read before the wait for the ring group, so that their
@@ -438,7 +527,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       }
     }
     // every copy issued must land before the CTA may exit
-    if (lane == 0) {
+    if (!L::DIRECT && lane == 0) {
       for (int j2 = max(0, jb - L::RG); j2 < jb; ++j2)
         if (!mbar_drain(&sh.raw_full[j2 % L::RG], (j2 / L::RG) & 1)) record_fault(p.fault, KVQ_FAULT_TIMEOUT);
     }
@@ -465,21 +554,31 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
       {
         bool ok = true;
         if (part == 0) {
-          // the K tile buffer: S of block j - NB has read it; the multiplier slot: the
-          // softmax of block j - kNQ is done with it
-          if (j >= NB && !pf_wait(&sh.s_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort)) ok = false;
+          // the K tile buffer: S of block j - NB has read it (16-bit caches: the producer
+          // waited for that before refilling it); the multiplier slot: the softmax of block
+          // j - kNQ is done with it
+          if (!L::DIRECT && j >= NB && !pf_wait(&sh.s_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort))
+            ok = false;
           if (ok && j >= kNQ && !pf_wait(&sh.kqfree[j % kNQ], ((j / kNQ) - 1) & 1, sh.abort)) ok = false;
-        } else if (j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
+        } else if (!L::DIRECT && j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
           ok = false;
         }
-        if (ok && paged && !pf_wait(&sh.raw_full[j % L::RG], (j / L::RG) & 1, sh.abort)) ok = false;
+        if constexpr (L::DIRECT) {
+          // the block's rows in tile buffer kb (its refill waited for P V of block j - NB,
+          // so the V scales of buffer kb are free too)
+          if (ok && paged && !pf_wait(&sh.tile_full[kb], (j / NB) & 1, sh.abort)) ok = false;
+        } else {
+          if (ok && paged && !pf_wait(&sh.raw_full[j % L::RG], (j / L::RG) & 1, sh.abort)) ok = false;
+        }
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) pf_fail(p, sh.abort);
           break;
         }
         // K: bad-token count; V: largest V scale
         float val = 0.f;
-        if constexpr (!L::LB) {
+        if constexpr (L::DIRECT) {
+          val = direct_part<CD, PT>(smem, sh, j, kb, part == 1, ct, npg, pmax, qsc, have_q);
+        } else if constexpr (!L::LB) {
           val = dense_part<CD, PT>(smem, sh, j, kb, part == 1, ct, npg, pmax, qsc, have_q);
         } else if (part == 0) {
           if (!have_q) {
@@ -611,7 +710,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p) {
           } else {
             mbar_arrive(&sh.v_full[kb]);
           }
-          if (paged) mbar_arrive(&sh.raw_empty[j % L::RG]);
+          if (!L::DIRECT && paged) mbar_arrive(&sh.raw_empty[j % L::RG]);
         }
       }
     }
@@ -1016,7 +1115,12 @@ cudaError_t launch_pf(const DecodeArgs& a, const DecodeParams& p, cudaStream_t s
   if (attr_err != cudaSuccess) return attr_err;
   const int TQ = kRows / a.plan.g;
   const dim3 grid((a.max_q_len + TQ - 1) / TQ, a.geo.H, a.batch);
-  prefill_tc_kernel<CD, PT, QP><<<grid, kPfThreads, L::BYTES, s>>>(p);
+  CUtensorMap rows = {};                  // 16-bit caches: the pool as rows of 256 bytes
+  if constexpr (L::DIRECT) {
+    const long nrows = static_cast<long>(a.geo.NB) * a.geo.H * 2 * L::BS;
+    if (!make_rows_map(&rows, a.c->pages, nrows, L::ROWB, L::BS)) return cudaErrorInvalidValue;
+  }
+  prefill_tc_kernel<CD, PT, QP><<<grid, kPfThreads, L::BYTES, s>>>(p, rows);
   return cudaGetLastError();
 }
 
