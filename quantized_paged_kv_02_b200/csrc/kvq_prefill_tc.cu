@@ -59,8 +59,7 @@ constexpr int kD = 128;
 constexpr int kPfThreads = 576;     // warps 0-7 softmax, 8 producer, 9 MMA, 10-13 K converters,
                                     // 14-17 V converters
 constexpr int kSoftWarps = 8, kProdWarp = 8, kMmaWarp = 9, kConvWarp0 = 10;
-constexpr int kNB = 2;              // K / V tile buffers (raw ring caches)
-constexpr int kNBMax = 3;           // ... at most (16-bit caches, no raw ring: three)
+constexpr int kNBMax = 3;           // K / V tile buffers at most
 constexpr int kNQ = 4;              // slots of the per-token K multipliers (block j: slot j % 4)
 constexpr int kTile = 32768;        // 128 x 128 16-bit elements
 constexpr float kRescalePf = 8.f;   // log2 headroom before the running max is re-based
@@ -92,7 +91,14 @@ struct PfLayout {
   static constexpr int REC = (OFF_S + SCALES + 127) / 128 * 128;
   static constexpr int KP = LB ? 2 : 1;                    // K tiles whose sum is K (hi, lo)
   static constexpr int VP = LB ? 2 : 1;
-  static constexpr int NB = LB ? 1 : (BITS == 16 ? 3 : kNB);   // K / V tile buffers
+  // K / V tile buffers: a K tile is free once S has read it, a V tile only after P V.  16-bit
+  // caches (no raw ring) keep three of each; INT8 one K and three V tiles beside the
+  // two-block raw ring (measured 1% faster than two and two), E4M3 two and two (0.4%
+  // faster than one and three)
+  static constexpr bool I8 = CD == KVQ_DTYPE_INT8;
+  static constexpr int NBK = LB ? 1 : (BITS == 16 ? 3 : (I8 ? 1 : 2));
+  static constexpr int NBV = LB ? 1 : (BITS == 16 || I8 ? 3 : 2);
+  static constexpr int NB = NBV;                           // 16-bit caches: NBK == NBV
   static constexpr int RS = LB ? 4 : (BITS == 8 ? 16 : 8); // raw ring stages (pages)
   // the ring turns over in groups of one block's pages, each group with one full and one
   // empty barrier: the producer issues a block's pages together and the converters wait
@@ -105,26 +111,27 @@ struct PfLayout {
   static constexpr int NPOK = DIRECT ? NB * PPB : RS;      // page-valid flags: by ring slot,
                                                            // or by (tile buffer, page)
   static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = NB * KP * kTile;
-  static constexpr int RAW_OFF = V_OFF + NB * VP * kTile;
+  static constexpr int V_OFF = NBK * KP * kTile;
+  static constexpr int RAW_OFF = V_OFF + NBV * VP * kTile;
   static constexpr int KQ_OFF = RAW_OFF + RAWB;            // float [kNQ][128]: K multiplier
-  static constexpr int VS_OFF = KQ_OFF + kNQ * kBlk * 4;   // float [NB][128]: V scale
-  static constexpr int XM_OFF = VS_OFF + NB * kBlk * 4;    // float [3][2][128]: row maxima of
+  static constexpr int VS_OFF = KQ_OFF + kNQ * kBlk * 4;   // float [NBV][128]: V scale
+  static constexpr int XM_OFF = VS_OFF + NBV * kBlk * 4;    // float [3][2][128]: row maxima of
                                                            // the two halves (by block parity),
                                                            // then the row sums
   static constexpr int MISC_OFF = XM_OFF + 3 * 2 * kRows * 4;  // per (buffer, converter warp)
                                                                // vmax and bad-token counts; flags
   static constexpr int BAR_OFF = MISC_OFF + 192;
-  // raw_full, raw_empty [RG]; k_full, v_full, vfree [NB]; s_full, p_full, pv_done [2];
+  // raw_full, raw_empty [RG]; k_full [NBK]; v_full, vfree [NBV]; s_full, p_full, pv_done [2];
   // q_ready; fin; xch [4]; kq_full, kqfree [kNQ]; tile_full [NB] (16-bit caches)
-  static constexpr int NBARS = 2 * RG + 3 * NB + 6 + 2 + 4 + 2 * kNQ + NB;
+  static constexpr int NBARS = 2 * RG + NBK + 2 * NBV + 6 + 2 + 4 + 2 * kNQ + NB;
   static constexpr int BYTES = 1024 + BAR_OFF + NBARS * 8 + NPOK * 4 + 64;
   static_assert(BYTES <= 227 * 1024, "fits the shared memory of one CTA");
   static_assert(BYTES > 114 * 1024, "one CTA per SM, so TMEM allocation never waits on a peer");
   static_assert(RS % PPB == 0 && RG >= 1, "the raw ring holds whole blocks");
   static_assert(PPB <= 32, "one producer lane per page of a block");
   static_assert(REC % 16 == 0, "bulk copies move multiples of 16 bytes");
-  static_assert(NB <= kNBMax, "scale arrays");
+  static_assert(NBV <= kNBMax && NBK <= kNQ, "scale arrays, multiplier slots");
+  static_assert(!DIRECT || NBK == NBV, "16-bit caches fill K and V of a buffer together");
 };
 
 struct PfShared {
@@ -361,7 +368,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap rows) {
   using L = PfLayout<CD, PT>;
   constexpr bool kBf = PfCode<CD>::kBf16;
-  constexpr int BS = L::BS, NB = L::NB;
+  constexpr int BS = L::BS, NB = L::NB, NBK = L::NBK, NBV = L::NBV;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, kvh = blockIdx.y;
   const int g = p.g, TQ = kRows / g;
@@ -390,9 +397,9 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
   sh.raw_full = bars;
   sh.raw_empty = bars + L::RG;
   sh.k_full = bars + 2 * L::RG;
-  sh.v_full = sh.k_full + NB;
-  sh.vfree = sh.v_full + NB;
-  sh.s_full = sh.vfree + NB;
+  sh.v_full = sh.k_full + NBK;
+  sh.vfree = sh.v_full + NBV;
+  sh.s_full = sh.vfree + NBV;
   sh.p_full = sh.s_full + 2;
   sh.pv_done = sh.p_full + 2;
   sh.q_ready = sh.pv_done + 2;
@@ -417,8 +424,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       mbar_init(&sh.raw_full[s], 1);
       mbar_init(&sh.raw_empty[s], 8);                    // the eight converter warps
     }
-    for (int k = 0; k < NB; ++k) {
-      mbar_init(&sh.k_full[k], 4);
+    for (int k = 0; k < NBK; ++k) mbar_init(&sh.k_full[k], 4);
+    for (int k = 0; k < NBV; ++k) {
       mbar_init(&sh.v_full[k], 4);
       mbar_init(&sh.vfree[k], 1);
     }
@@ -549,7 +556,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     const bool fz = p.mode == KVQ_SCALE_KIVI_FLOAT_ZERO, ktok = p.mode == KVQ_SCALE_INT4_PER_TOKEN;
     const int G = c >> 3;                                 // 64-channel group of the chunk
     for (int j = 0; j < J && !*sh.abort; ++j) {
-      const int kb = j % NB;
+      // tile buffer of this part: K tiles by j % NBK, V tiles (and V scales) by j % NBV
+      const int kb = part == 0 ? j % NBK : j % NBV;
       const bool paged = j * L::PPB < npg;               // the block has pages in the ring
       {
         bool ok = true;
@@ -557,10 +565,10 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
           // the K tile buffer: S of block j - NB has read it (16-bit caches: the producer
           // waited for that before refilling it); the multiplier slot: the softmax of block
           // j - kNQ is done with it
-          if (!L::DIRECT && j >= NB && !pf_wait(&sh.s_full[(j - NB) & 1], ((j - NB) >> 1) & 1, sh.abort))
+          if (!L::DIRECT && j >= NBK && !pf_wait(&sh.s_full[(j - NBK) & 1], ((j - NBK) >> 1) & 1, sh.abort))
             ok = false;
           if (ok && j >= kNQ && !pf_wait(&sh.kqfree[j % kNQ], ((j / kNQ) - 1) & 1, sh.abort)) ok = false;
-        } else if (!L::DIRECT && j >= NB && !pf_wait(&sh.vfree[kb], ((j / NB) - 1) & 1, sh.abort)) {
+        } else if (!L::DIRECT && j >= NBV && !pf_wait(&sh.vfree[kb], ((j / NBV) - 1) & 1, sh.abort)) {
           ok = false;
         }
         if constexpr (L::DIRECT) {
@@ -723,8 +731,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       bool ok = pf_wait(sh.q_ready, 0, sh.abort);
       tc::fence_after_sync();
       auto pv = [&](int jj) -> bool {
-        const int sb = jj & 1, kb = jj % NB;
-        if (!pf_wait(&sh.v_full[kb], (jj / NB) & 1, sh.abort)) return false;
+        const int sb = jj & 1, kb = jj % NBV;
+        if (!pf_wait(&sh.v_full[kb], (jj / NBV) & 1, sh.abort)) return false;
         if (!pf_wait(&sh.p_full[sb], (jj >> 1) & 1, sh.abort)) return false;
         tc::fence_after_sync();
         // P hi V hi (+ P hi V lo + P lo V hi for split V) + P lo V hi ... : pairs (pa, vp),
@@ -749,8 +757,8 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         return true;
       };
       for (int j = 0; j < J && ok; ++j) {
-        const int sb = j & 1, kb = j % NB;
-        if (!pf_wait(&sh.k_full[kb], (j / NB) & 1, sh.abort)) { ok = false; break; }
+        const int sb = j & 1, kb = j % NBK;
+        if (!pf_wait(&sh.k_full[kb], (j / NBK) & 1, sh.abort)) { ok = false; break; }
         tc::fence_after_sync();
         bool first = true;
 #pragma unroll
@@ -872,7 +880,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
     bool ok = true;
     float* xm = sh.xmax;                                   // [2][2][128]: block parity, half, row
     for (int j = 0; j < J; ++j) {
-      const int sb = j & 1, kb = j % NB, qs = j % kNQ;
+      const int sb = j & 1, kb = j % NBV, qs = j % kNQ;     // kb: the V buffer
       // the block's K multipliers through their own slot barrier: K of block j + NB may
       // complete k_full once more before this wait (the next phase of kq_full[qs] needs
       // this softmax's release of the slot)
@@ -941,7 +949,7 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.xch[quarter]);
       if (!pf_wait(&sh.xch[quarter], j & 1, sh.abort)) ok = false;
-      if (!pf_wait(&sh.v_full[kb], (j / NB) & 1, sh.abort)) ok = false;
+      if (!pf_wait(&sh.v_full[kb], (j / NBV) & 1, sh.abort)) ok = false;
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       mx = fmaxf(mx, xm[(sb * 2 + (hf ^ 1)) * kRows + r]);
       // rescale factor of l and O: the max re-based (beyond 2^8) and / or the V normaliser
