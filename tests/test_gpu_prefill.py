@@ -216,10 +216,13 @@ def test_prefill_groups_and_types(key):
     assert gc.read_fault() == (0, 0)
 
 
-def test_prefill_bad_block_is_masked_and_counted():
+@pytest.mark.parametrize("name", ["c5", "c5-bf16"])
+def test_prefill_bad_block_is_masked_and_counted(name):
     """A block-table entry outside the pool: its tokens are left out of every query's window
-    (as if masked), the fault record counts it, and nothing else changes."""
-    w = inputs.make("c5", small=True)
+    (as if masked), the fault record counts it, and nothing else changes.  (bf16 caches take
+    the path whose pages are copied straight into the tiles: the bad page's rows are never
+    written there, so its V rows are zeroed and its scores masked.)"""
+    w = inputs.make(name, small=True)
     oc = helpers.oracle_cache(w)
     gc = helpers.gpu_cache(w)
     L = [50, 20, 5]
