@@ -13,11 +13,15 @@
 //   warp 8      producer: the table entries of a block's pages, then one bulk copy per page
 //               record (K codes, V codes, per-token scales) into a ring of raw stages that
 //               turns over a block at a time (one full and one empty barrier per block);
+//               for 16-bit caches, whose rows are the tiles' values, four TMA tensor copies
+//               per page straight into a K / V tile buffer (128-byte swizzle), no raw ring;
 //   warps 10-13 K converters and warps 14-17 V converters: codes -> 16-bit tiles in the
 //               tensor cores' 128-byte-swizzled layout (INT8 through the exact 1024-magic,
-//               E4M3 by the hardware conversion, 16-bit caches copied), K as the K-major B
-//               operand of S = Q K^T and V as the MN-major B operand of O = P V, plus the
-//               per-token multipliers (in four slots of their own) and V scales;
+//               E4M3 by the hardware conversion), K as the K-major B operand of S = Q K^T
+//               and V as the MN-major B operand of O = P V, plus the per-token multipliers
+//               (in four slots of their own) and V scales (for 16-bit caches only these,
+//               and zeros over the V rows outside the window); K and V tiles have their own
+//               buffer counts (a K tile is free once S has read it, a V tile after P V);
 //   warp 9      MMA issuer: S_j = Q K_j^T (M 128, N 128 tokens, K 128) into one of two TMEM
 //               score buffers, then O += P_{j-1} V_{j-1} (N 128 channels, K 128 tokens);
 //   warps 0-7   softmax: the two warps of a TMEM lane quarter share its 32 query rows,
