@@ -493,13 +493,14 @@ prefill_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant_
         if (lane == 0) mbar_arrive_expect_tx(&sh.tile_full[kb], nvalid * L::REC);
         __syncwarp();
         if (valid) {
-          // the record's 32 rows of 256 bytes: K rows 0..15, V rows 16..31
+          // the record's 32 rows of 256 bytes: K rows 0..15, V rows from OFF_V (16..31)
           const int y = (blk * p.H + kvh) * (2 * BS);
           const int r0 = lane * BS * 128;                  // page lane's rows in a tile half
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             tma_load_2d(smem + L::K_OFF + kb * kTile + hh * 16384 + r0, &rows, &sh.tile_full[kb], 128 * hh, y);
-            tma_load_2d(smem + L::V_OFF + kb * kTile + hh * 16384 + r0, &rows, &sh.tile_full[kb], 128 * hh, y + BS);
+            tma_load_2d(smem + L::V_OFF + kb * kTile + hh * 16384 + r0, &rows, &sh.tile_full[kb], 128 * hh,
+                        y + L::OFF_V / L::ROWB);
           }
         }
       }
