@@ -67,3 +67,25 @@ def decode_step_bytes(cache_dtype, scale_mode, batch, num_q_heads, num_kv_heads,
     total += batch * num_q_heads * D * act_bytes                        # q
     total += batch * num_q_heads * D * out_bytes                        # out
     return total
+
+
+def write_step_bytes(cache_dtype, scale_mode, rows, num_kv_heads, head_dim, act_bytes=2,
+                     to_ring=False):
+    """Bytes one write of `rows` new tokens must move: the K and V rows read (activation
+    values) and one int32 slot id per token, then what the cache stores for them -- codes at
+    the bytes per value of the size formula, plus one float32 scale per (token, kv head) for
+    K and V when scales are per token ([P-mem] §3.2 动态量化策略: a scale per token).  A
+    16-bit cache, and a low-bit cache whose new rows go to the residual ring, store the rows
+    as they are (act_bytes per value).  Static scales are read from the call's arguments,
+    not from the pool, and are not counted.
+    """
+    H, D = num_kv_heads, head_dim
+    total = Fraction(2 * rows * H * D * act_bytes)                      # K and V rows read
+    total += 4 * rows                                                   # slot ids
+    if to_ring or cache_dtype in ("bf16", "fp16"):
+        total += 2 * rows * H * D * act_bytes
+        return total
+    total += 2 * rows * H * D * BYTES_PER_VALUE[cache_dtype]            # K and V codes
+    if scale_mode == "per_token_head":
+        total += 2 * rows * H * 4                                       # K and V scales
+    return total

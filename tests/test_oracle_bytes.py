@@ -128,3 +128,42 @@ def test_bench_byte_counts_equal_the_oracle_model():
             got = roofline.decode_bytes(s.cache_dtype, s.scale_mode, s.num_q_heads,
                                         s.num_kv_heads, s.head_dim, s.block_size, lens)
             assert want.denominator == 1 and got == int(want), (name, lens)
+
+
+def test_write_step_bytes_components():
+    """The prefill write of the c5 layer (4 x 8192 new tokens, 8 kv heads, D 128, bf16 rows),
+    decomposed by hand: rows read 2 x 32768 x 8 x 128 x 2 = 134,217,728 B plus 4 B of slot id
+    per token; INT8 per token writes 1 byte per value plus a float32 scale per (token, kv head)
+    for K and V (67,108,864 + 2,097,152 = 69,206,016 B); FP8 with a static per-head scale
+    writes the codes only."""
+    rows_read, slots = 2 * 32768 * 8 * 128 * 2, 4 * 32768
+    assert rows_read == 134217728
+    i8 = bytes_model.write_step_bytes("int8", "per_token_head", 32768, 8, 128)
+    assert i8 == rows_read + slots + 67108864 + 2097152
+    f8 = bytes_model.write_step_bytes("fp8", "per_head", 32768, 8, 128)
+    assert f8 == rows_read + slots + 67108864
+    # the decode step's append: one row per sequence (24), INT8 per token
+    a8 = bytes_model.write_step_bytes("int8", "per_token_head", 24, 8, 128)
+    assert a8 == 2 * 24 * 8 * 128 * 2 + 4 * 24 + 2 * 24 * 8 * 128 + 2 * 24 * 8 * 4
+    # bf16 caches and rows that go to the INT4 residual ring store the rows as they are
+    assert bytes_model.write_step_bytes("bf16", "none", 24, 8, 128) == 2 * (2 * 24 * 8 * 128 * 2) + 4 * 24
+    assert bytes_model.write_step_bytes("int4", "kivi", 16, 8, 128, to_ring=True) == \
+        2 * (2 * 16 * 8 * 128 * 2) + 4 * 16
+
+
+def test_bench_write_bytes_equal_the_oracle():
+    """The write bytes bench.py adds to every step (and reports for the prefill write) are
+    the oracle's count, for every bench workload's append and both prefill-write caches."""
+    import bench
+    from quantized_paged_kv_02_b200 import inputs, roofline
+    for name in sorted(bench.WORKLOADS):
+        s = inputs._spec(name, False)
+        ring = inputs.low_bit(s.cache_dtype)
+        got = roofline.write_bytes(s.cache_dtype, s.scale_mode, s.batch, s.num_kv_heads, s.head_dim,
+                                   to_ring=ring)
+        want = bytes_model.write_step_bytes(s.cache_dtype, s.scale_mode, s.batch, s.num_kv_heads,
+                                            s.head_dim, to_ring=ring)
+        assert got == want, name
+    for cd, mode in (("int8", "per_token_head"), ("fp8", "per_head")):
+        assert roofline.write_bytes(cd, mode, 32768, 8, 128) == \
+            bytes_model.write_step_bytes(cd, mode, 32768, 8, 128)
