@@ -134,6 +134,14 @@ def tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def prefill_flops(batch, n, L, num_q_heads, head_dim):
+    """Algorithmic flops of a causal prefill chunk: the newest L of a sequence's n cached
+    tokens are its queries, query i (position n - L + i) sees positions 0 .. n - L + i; per
+    query head and visible position q.k and p.v take 2 D flops each."""
+    visible = batch * sum(n - L + i + 1 for i in range(L))
+    return 4.0 * head_dim * num_q_heads * visible
+
+
 def measure_prefill(device, l2, workload="c5", steps=20, batch=4, n=4096, chunk=512):
     """Chunked prefill on a layer of the named workload's cache type and heads (c5: INT8
     per-token-head, 64/8 heads, D 128, block 16): `batch` sequences of n cached tokens whose
@@ -163,8 +171,7 @@ def measure_prefill(device, l2, workload="c5", steps=20, batch=4, n=4096, chunk=
         b.record()
     torch.cuda.synchronize()
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    visible = s.batch * sum(n - L + i + 1 for i in range(L))
-    flops = 4.0 * s.head_dim * s.num_q_heads * visible
+    flops = prefill_flops(s.batch, n, L, s.num_q_heads, s.head_dim)
     peak, kind = tensor_peak()
     tf = flops / (ms * 1e-3) / 1e12
     res = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),

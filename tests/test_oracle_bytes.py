@@ -167,3 +167,18 @@ def test_bench_write_bytes_equal_the_oracle():
     for cd, mode in (("int8", "per_token_head"), ("fp8", "per_head")):
         assert roofline.write_bytes(cd, mode, 32768, 8, 128) == \
             bytes_model.write_step_bytes(cd, mode, 32768, 8, 128)
+
+
+def test_prefill_flops_count_visible_pairs():
+    """The prefill roofline's numerator: 4 D flops per (query head, visible position), the
+    visible positions those the causal window of each query reaches.  Counted here by
+    enumerating the mask (query i of an L-query chunk at the end of n cached tokens sees
+    position p iff p <= n - L + i), and the c5 prefill figure (4 x 4096 tokens, 512-query
+    chunks, 64 query heads, D 128) written out."""
+    import bench
+    for batch, n, L, hq, d in ((1, 5, 5, 1, 1), (2, 37, 9, 3, 16), (3, 200, 64, 2, 8)):
+        pairs = batch * sum(1 for i in range(L) for p in range(n) if p <= n - L + i)
+        assert bench.prefill_flops(batch, n, L, hq, d) == 4 * d * hq * pairs
+    per_seq = 512 * (4096 - 512) + 512 * 513 // 2            # sum over the chunk of n - L + i + 1
+    assert per_seq == 1966336
+    assert bench.prefill_flops(4, 4096, 512, 64, 128) == 4 * 128 * 64 * 4 * per_seq == 257731592192
