@@ -267,3 +267,22 @@ def test_back_to_back_calls_share_a_workspace(name):
         want = a1 if i % 2 == 0 else a2
         assert torch.equal(o, want), (name, i)
     assert gc.read_fault() == (0, 0)
+
+
+@pytest.mark.parametrize("cd,mode", [("int4", "kivi"), ("int2", "int4_per_token"), ("int4", "kivi_float_zero")])
+def test_low_bit_edge_lengths(cd, mode):
+    """Low-bit caches with an empty sequence, one token, sequences held wholly in the
+    residual ring (no whole 64-token group yet: 100, 191) and one just past a group (192):
+    block-kernel CTAs with no blocks, ring-only splits and every split count the reduce can
+    see, on the tensor-core path.  The empty sequence's output is zero."""
+    spec = inputs.Spec("c4-edge", cd, "bf16", mode, 6, 16, 2, 128, 64, lens=[0, 1, 100, 191, 192, 300],
+                       outliers="k", slack_blocks=2, seed=5)
+    w = inputs.from_spec(spec)
+    oc = helpers.oracle_cache(w)
+    gc = helpers.gpu_cache(w)
+    assert gc.decode_plan(spec.batch, spec.num_q_heads, w.max_context)[0] == 2   # tensor cores
+    got = _decode(gc, w).cpu().numpy().astype(np.float64)
+    want = _oracle(oc, w)
+    assert np.all(got[0] == 0)
+    assert np.abs(got - want).max() <= TOL
+    assert gc.read_fault() == (0, 0)
