@@ -197,6 +197,9 @@ SPECS = {
                                lens=[400, 130], slack_blocks=2, seed=32), [200, 130]),
     "fp8-mha-fp16act": (inputs.Spec("pf-mha", "fp8", "fp16", "per_token_head", 2, 2, 2, 128, 16,
                                     lens=[333, 47], slack_blocks=2, seed=33), [160, 47]),
+    # MHA over a bf16 cache: the rows copied straight into the tiles, 128-token query tiles
+    "bf16-mha": (inputs.Spec("pf-bf16-mha", "bf16", "bf16", "none", 3, 4, 4, 128, 16,
+                             lens=[333, 129, 260], slack_blocks=3, seed=34), [300, 129, 5]),
 }
 
 
